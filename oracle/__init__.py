@@ -1,0 +1,190 @@
+"""fp64 CPU oracle for the Kimi Delta Attention (KDA) operator -- TEST INFRASTRUCTURE.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may import
+this package.  The CUDA library never imports, links or executes anything here, and this package
+imports nothing from the CUDA library.
+
+The arithmetic lives in ``kda_oracle.c`` (plain C, fp64); this module only marshals numpy
+arrays into it.  Every function follows a passage of the pages:
+
+* ``seq``         -- the recurrence ``S_t = (I - b_t k_t k_t^T) Diag(a_t) S_{t-1} + b_t k_t v_t^T``
+                     with readout ``o_t = S_t^T q_t``; "Kimi Linear" explainer (xugj520.cn),
+                     section "Kimi Delta Attention的技术内核"; attention review (lanjinlin.com.cn),
+                     entry "KLA 25.10 kimi".
+* ``bruteforce``  -- the same recurrence with the dense transition matrix
+                     ``M_t = (I - b k k^T) Diag(a)`` materialised (textbook matrix products).
+* ``chunked``     -- the chunk-parallel / WY / UT form listed in the explainer's section
+                     "硬件效率的深度优化" (chunk size C, any C >= 1).
+* ``decode_step`` -- one token per sequence, in the loop order (decay, delta, update, output) of
+                     the review's GDN pseudo-code.
+
+Pins (checked in ``tests/test_oracle_pins.py``): the beta=0 closed form, exact write/retrieve
+with orthonormal keys at alpha=1 and beta=1, an exact rational worked example, the per-step
+delta invariant, brute force vs sequential, chunked vs sequential for several C, linearity in
+(V, S0), state passing, varlen vs separate runs, decode vs prefill, and a norm bound.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import sys
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kda_oracle.c")
+_LIB = os.path.join(_HERE, "libkda_oracle.so")
+_lib = None
+_lib_path = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``kda_oracle.c`` into ``libkda_oracle.so`` next to it (gcc, -O2, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-fPIC", "-shared", "-std=c11", "-Wall", "-Wextra", "-fno-fast-math",
+               "-ffp-contract=off", "-o", _LIB, _SRC, "-lm", "-lpthread"]
+        subprocess.run(cmd, check=True)
+    return _LIB
+
+
+def use_library(path: str) -> None:
+    """Point this wrapper at another build of the oracle (used by the mutant tests, which compile
+    deliberately broken copies of ``kda_oracle.c`` and check that the pins reject them)."""
+    global _lib, _lib_path
+    _lib, _lib_path = None, path
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        if _lib_path is None:
+            build()
+        lib = ctypes.CDLL(_lib_path or _LIB)
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        for name in ("kda_oracle_seq", "kda_oracle_bruteforce"):
+            f = getattr(lib, name)
+            f.argtypes = [P, P, P, P, P, P, P, I, I, I, I, P, P, P, I]
+            f.restype = I
+        lib.kda_oracle_chunked.argtypes = [P, P, P, P, P, P, P, I, I, I, I, P, P, P, I, I]
+        lib.kda_oracle_chunked.restype = I
+        lib.kda_oracle_decode_step.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
+        lib.kda_oracle_decode_step.restype = I
+        _lib = lib
+    return _lib
+
+
+def _f32(x):
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data
+
+
+def default_threads() -> int:
+    return max(1, len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count() or 1)
+
+
+def _prep(q, k, v, log_alpha, beta, S0, cu_seqlens):
+    q, k, v, la, b = _f32(q), _f32(k), _f32(v), _f32(log_alpha), _f32(beta)
+    if q.ndim == 4:  # [B, T, H, d] regular batch -> packed with cu_seqlens
+        B, T, H, dk = q.shape
+        dv = v.shape[-1]
+        if cu_seqlens is not None:
+            raise ValueError("cu_seqlens is only meaningful for packed [Ttot, H, d] inputs")
+        cu = np.arange(B + 1, dtype=np.int64) * T
+        q, k, la = (x.reshape(B * T, H, dk) for x in (q, k, la))
+        v = v.reshape(B * T, H, dv)
+        b = b.reshape(B * T, H)
+    else:
+        Ttot, H, dk = q.shape
+        dv = v.shape[-1]
+        cu = (np.array([0, Ttot], dtype=np.int64) if cu_seqlens is None
+              else np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64)))
+    N = len(cu) - 1
+    if k.shape != q.shape or la.shape != q.shape or v.shape[:2] != q.shape[:2] or b.shape != q.shape[:2]:
+        raise ValueError("inconsistent shapes")
+    s0 = None if S0 is None else np.ascontiguousarray(np.asarray(S0, dtype=np.float64).reshape(N, H, dk, dv))
+    return q, k, v, la, b, s0, cu, N, H, dk, dv
+
+
+def _call(fname, q, k, v, log_alpha, beta, S0, cu_seqlens, pairs, threads, extra=()):
+    shape4 = np.asarray(q).ndim == 4
+    q, k, v, la, b, s0, cu, N, H, dk, dv = _prep(q, k, v, log_alpha, beta, S0, cu_seqlens)
+    Ttot = q.shape[0]
+    out = np.zeros((Ttot, H, dv), dtype=np.float64)
+    sf = np.zeros((N, H, dk, dv), dtype=np.float64)
+    mask = None
+    if pairs is not None:
+        mask = np.zeros(N * H, dtype=np.int32)
+        for n, h in pairs:
+            mask[n * H + h] = 1
+    lib = _load()
+    fn = getattr(lib, fname)
+    rc = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(b), _ptr(s0), _ptr(cu), N, H, dk, dv,
+            _ptr(out), _ptr(sf), _ptr(mask), *extra, threads or default_threads())
+    if rc != 0:
+        raise RuntimeError(f"{fname} failed with status {rc}")
+    if shape4:
+        B = N
+        out = out.reshape(B, Ttot // B, H, dv)
+    return out, sf
+
+
+def seq(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, pairs=None, threads=None):
+    """The definition.  Inputs ``[B,T,H,d]`` or packed ``[Ttot,H,d]`` (+ ``cu_seqlens``).
+
+    Returns ``(out, S_final)`` in float64: out has the layout of ``v``, S_final is
+    ``[N, H, dk, dv]``.  ``pairs`` restricts the work to a list of ``(seq, head)`` pairs
+    (the other outputs stay zero)."""
+    return _call("kda_oracle_seq", q, k, v, log_alpha, beta, S0, cu_seqlens, pairs, threads)
+
+
+def bruteforce(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, pairs=None, threads=None):
+    """Dense transition-matrix form (short sequences)."""
+    return _call("kda_oracle_bruteforce", q, k, v, log_alpha, beta, S0, cu_seqlens, pairs, threads)
+
+
+def chunked(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, C=64, pairs=None, threads=None):
+    """Chunked WY/UT form with chunk size ``C``."""
+    # the C entry point takes C before the thread count
+    shape4 = np.asarray(q).ndim == 4
+    q_, k_, v_, la, b, s0, cu, N, H, dk, dv = _prep(q, k, v, log_alpha, beta, S0, cu_seqlens)
+    Ttot = q_.shape[0]
+    out = np.zeros((Ttot, H, dv), dtype=np.float64)
+    sf = np.zeros((N, H, dk, dv), dtype=np.float64)
+    mask = None
+    if pairs is not None:
+        mask = np.zeros(N * H, dtype=np.int32)
+        for n, h in pairs:
+            mask[n * H + h] = 1
+    rc = _load().kda_oracle_chunked(_ptr(q_), _ptr(k_), _ptr(v_), _ptr(la), _ptr(b), _ptr(s0), _ptr(cu), N, H,
+                                    dk, dv, _ptr(out), _ptr(sf), _ptr(mask), int(C),
+                                    threads or default_threads())
+    if rc != 0:
+        raise RuntimeError(f"kda_oracle_chunked failed with status {rc}")
+    if shape4:
+        out = out.reshape(N, Ttot // N, H, dv)
+    return out, sf
+
+
+def decode_step(q, k, v, log_alpha, beta, S):
+    """One token for each of N sequences.  ``q,k,log_alpha [N,H,dk]``, ``v [N,H,dv]``,
+    ``beta [N,H]``, ``S [N,H,dk,dv]`` (float64, returned updated as a new array).
+    Returns ``(out [N,H,dv] float64, S_new)``."""
+    q, k, v, la, b = _f32(q), _f32(k), _f32(v), _f32(log_alpha), _f32(beta)
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    S = np.array(S, dtype=np.float64, copy=True, order="C").reshape(N, H, dk, dv)
+    out = np.zeros((N, H, dv), dtype=np.float64)
+    rc = _load().kda_oracle_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(b), _ptr(S), N, H, dk, dv,
+                                        _ptr(out))
+    if rc != 0:
+        raise RuntimeError(f"kda_oracle_decode_step failed with status {rc}")
+    return out, S
+
+
+if __name__ == "__main__":  # pragma: no cover
+    print(build(force="--force" in sys.argv))

@@ -1,0 +1,383 @@
+/*
+ * kda_oracle.c -- plain, slow, fp64 CPU oracle for the Kimi Delta Attention (KDA) operator.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may call, link or load this file;
+ * only tests/, the smoke check and the bench's CPU-baseline leg use it.  It shares no code,
+ * header, table or helper with the CUDA library.
+ *
+ * What it computes (per sequence n, per head h, state S of shape d_k x d_v, row = key channel):
+ *
+ *   S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,   o_t = S_t^T q_t
+ *
+ *   - recurrence: "Kimi Linear: redefining long-context inference efficiency" (xugj520.cn),
+ *     section "Kimi Delta Attention的技术内核", the recurrent-form state update; the same formula
+ *     with the per-channel Diag(alpha_t) appears in the 2025 attention/MoE review (lanjinlin.com.cn),
+ *     entry "KLA 25.10 kimi", and its readout o_t = S_t^T q_t is the linear-attention formula
+ *     stated there.
+ *   - alpha_t = exp(log_alpha_t) per key channel, beta_t a per-head scalar per token.
+ *   - the decode step follows the per-token loop of the review's GDN pseudo-code (state decay,
+ *     value modification by S'^T k, rank-1 state update with beta, output from the UPDATED state).
+ *   - the chunked form follows the explainer's "硬件效率的深度优化" list: chunk-parallel compute
+ *     inside a chunk, recurrent state passing between chunks, a WY representation of the
+ *     chunk's rank-1 updates and a UT transform (the triangular inverse (I+A)^{-1}).
+ *
+ * Inputs are float32 arrays (the exact values the GPU receives; bf16 values are exactly
+ * representable in float32) and are widened to fp64.  All arithmetic is fp64.
+ *
+ * Layout: token-major.  q, k, log_alpha: [Ttot][H][dk]; v: [Ttot][H][dv]; beta: [Ttot][H];
+ * out: [Ttot][H][dv]; S0 / S_final: [N][H][dk][dv].  Sequence n owns tokens
+ * cu_seqlens[n] .. cu_seqlens[n+1]-1.  A regular batch of B sequences of length T is
+ * cu_seqlens = {0, T, 2T, ..., BT}.
+ *
+ * Three independent formulations:
+ *   kda_oracle_seq        the recurrence as written, step by step            (the definition)
+ *   kda_oracle_bruteforce the dense transition matrix M_t = (I - b k k^T) Diag(a), S = M S + b k v^T
+ *   kda_oracle_chunked    the chunk/WY/UT re-association, chunk size C        (exact up to rounding)
+ * and kda_oracle_decode_step, one token per sequence, in the review's loop order.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define IDX3(t, h, c, H, D) (((size_t)(t) * (size_t)(H) + (size_t)(h)) * (size_t)(D) + (size_t)(c))
+
+typedef struct {
+    const float *q, *k, *v, *log_alpha, *beta;
+    const double* S0;
+    const int64_t* cu_seqlens;
+    const int32_t* pair_mask;
+    int N, H, dk, dv, C;
+    double *out, *S_final;
+    int mode; /* 0 = sequential, 1 = chunked, 2 = brute force */
+    int next_pair;
+    pthread_mutex_t lock;
+    int status;
+} job_t;
+
+/* ------------------------------------------------------------------------------------------
+ * The definition, one (sequence, head) pair.
+ *   S' = Diag(alpha_t) S            (row c scaled by alpha_c = exp(log_alpha_c))
+ *   S  = S' - beta k (k^T S') + beta k v^T      ((I - beta k k^T) S' + beta k v^T, expanded)
+ *   o  = S^T q
+ * ------------------------------------------------------------------------------------------ */
+static void pair_seq(const job_t* J, int n, int h, double* S, double* w)
+{
+    const int H = J->H, dk = J->dk, dv = J->dv;
+    const int64_t t0 = J->cu_seqlens[n], t1 = J->cu_seqlens[n + 1];
+    for (int64_t t = t0; t < t1; ++t) {
+        const float* kt = J->k + IDX3(t, h, 0, H, dk);
+        const float* qt = J->q + IDX3(t, h, 0, H, dk);
+        const float* vt = J->v + IDX3(t, h, 0, H, dv);
+        const float* la = J->log_alpha + IDX3(t, h, 0, H, dk);
+        const double b = (double)J->beta[(size_t)t * H + h];
+        /* S' = Diag(alpha) S */
+        for (int c = 0; c < dk; ++c) {
+            const double a = exp((double)la[c]);
+            for (int j = 0; j < dv; ++j) S[(size_t)c * dv + j] *= a;
+        }
+        /* w = k^T S'  (a d_v row vector) */
+        for (int j = 0; j < dv; ++j) w[j] = 0.0;
+        for (int c = 0; c < dk; ++c) {
+            const double kc = (double)kt[c];
+            for (int j = 0; j < dv; ++j) w[j] += kc * S[(size_t)c * dv + j];
+        }
+        /* S = S' - b k w + b k v^T */
+        for (int c = 0; c < dk; ++c) {
+            const double kc = (double)kt[c];
+            for (int j = 0; j < dv; ++j)
+                S[(size_t)c * dv + j] += -b * kc * w[j] + b * kc * (double)vt[j];
+        }
+        /* o = S^T q */
+        if (J->out) {
+            double* o = J->out + IDX3(t, h, 0, H, dv);
+            for (int j = 0; j < dv; ++j) o[j] = 0.0;
+            for (int c = 0; c < dk; ++c) {
+                const double qc = (double)qt[c];
+                for (int j = 0; j < dv; ++j) o[j] += qc * S[(size_t)c * dv + j];
+            }
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------------------------
+ * Brute force: materialise the dense d_k x d_k transition M_t = (I - b k k^T) Diag(alpha) and
+ * apply S = M_t S + b k v^T with a textbook matrix product.  Meant for short sequences.
+ * ------------------------------------------------------------------------------------------ */
+static void pair_bruteforce(const job_t* J, int n, int h, double* S, double* M, double* S2)
+{
+    const int H = J->H, dk = J->dk, dv = J->dv;
+    const int64_t t0 = J->cu_seqlens[n], t1 = J->cu_seqlens[n + 1];
+    for (int64_t t = t0; t < t1; ++t) {
+        const float* kt = J->k + IDX3(t, h, 0, H, dk);
+        const float* qt = J->q + IDX3(t, h, 0, H, dk);
+        const float* vt = J->v + IDX3(t, h, 0, H, dv);
+        const float* la = J->log_alpha + IDX3(t, h, 0, H, dk);
+        const double b = (double)J->beta[(size_t)t * H + h];
+        for (int r = 0; r < dk; ++r)
+            for (int c = 0; c < dk; ++c) {
+                const double id = (r == c) ? 1.0 : 0.0;
+                M[(size_t)r * dk + c] = (id - b * (double)kt[r] * (double)kt[c]) * exp((double)la[c]);
+            }
+        for (int r = 0; r < dk; ++r)
+            for (int j = 0; j < dv; ++j) {
+                double acc = 0.0;
+                for (int c = 0; c < dk; ++c) acc += M[(size_t)r * dk + c] * S[(size_t)c * dv + j];
+                S2[(size_t)r * dv + j] = acc + b * (double)kt[r] * (double)vt[j];
+            }
+        memcpy(S, S2, sizeof(double) * (size_t)dk * dv);
+        if (J->out) {
+            double* o = J->out + IDX3(t, h, 0, H, dv);
+            for (int j = 0; j < dv; ++j) {
+                double acc = 0.0;
+                for (int c = 0; c < dk; ++c) acc += S[(size_t)c * dv + j] * (double)qt[c];
+                o[j] = acc;
+            }
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------------------------
+ * Chunked form (chunk-parallel inside, recurrent between chunks; WY representation; UT transform).
+ * Inside a chunk with start state S0 and local index r = 0..L-1:
+ *   g_r      = sum_{i<=r} log_alpha_i                     (per key channel; restarts every chunk)
+ *   A[r][i]  = beta_r sum_c k_rc k_ic exp(g_rc - g_ic),  i < r       (strictly lower)
+ *   T        = (I + A)^{-1} Diag(beta)                    (UT transform, forward substitution)
+ *   Kt[r][c] = k_rc exp(g_rc),  W = T Kt,  Uv = T V       (WY factors)
+ *   U        = Uv - W S0                                   (the chunk's corrected values u_r)
+ *   o_r      = sum_c q_rc exp(g_rc) S0[c][:] + sum_{i<=r} P[r][i] U[i],
+ *              P[r][i] = sum_c q_rc k_ic exp(g_rc - g_ic)
+ *   S_end    = Diag(exp(g_last)) S0 + sum_i (k_i * exp(g_last - g_i)) U_i^T
+ * Derivation: unrolling the recurrence inside the chunk gives
+ *   S_r = Diag(gamma_r) S0 + sum_{i<=r} Diag(gamma_r/gamma_i) k_i u_i^T,  gamma_r = exp(g_r),
+ *   u_r = beta_r (v_r - S'_r^T k_r), which is the unit-lower-triangular system
+ *   (I + A) U = Diag(beta)(V - Kt S0).
+ * ------------------------------------------------------------------------------------------ */
+static void pair_chunked(const job_t* J, int n, int h, double* S, double* scratch)
+{
+    const int H = J->H, dk = J->dk, dv = J->dv, C = J->C;
+    const int64_t t0 = J->cu_seqlens[n], t1 = J->cu_seqlens[n + 1];
+    double* g = scratch;                          /* C * dk */
+    double* A = g + (size_t)C * dk;               /* C * C */
+    double* Tm = A + (size_t)C * C;               /* C * C */
+    double* W = Tm + (size_t)C * C;               /* C * dk */
+    double* Uv = W + (size_t)C * dk;              /* C * dv */
+    double* U = Uv + (size_t)C * dv;              /* C * dv */
+    double* Snew = U + (size_t)C * dv;            /* dk * dv */
+    for (int64_t cs = t0; cs < t1; cs += C) {
+        const int L = (int)((t1 - cs) < C ? (t1 - cs) : C);
+        /* cumulative log gate */
+        for (int c = 0; c < dk; ++c) {
+            double acc = 0.0;
+            for (int r = 0; r < L; ++r) {
+                acc += (double)J->log_alpha[IDX3(cs + r, h, c, H, dk)];
+                g[(size_t)r * dk + c] = acc;
+            }
+        }
+        /* A (strictly lower) */
+        for (int r = 0; r < L; ++r) {
+            const double br = (double)J->beta[(size_t)(cs + r) * H + h];
+            for (int i = 0; i < L; ++i) {
+                double acc = 0.0;
+                if (i < r)
+                    for (int c = 0; c < dk; ++c)
+                        acc += (double)J->k[IDX3(cs + r, h, c, H, dk)] * (double)J->k[IDX3(cs + i, h, c, H, dk)] *
+                               exp(g[(size_t)r * dk + c] - g[(size_t)i * dk + c]);
+                A[(size_t)r * C + i] = br * acc;
+            }
+        }
+        /* T = (I + A)^{-1} Diag(beta): row r of (I+A) T = Diag(beta) gives
+           T[r][j] = beta_r [r==j] - sum_{i<r} A[r][i] T[i][j] */
+        for (int r = 0; r < L; ++r)
+            for (int j = 0; j < L; ++j) {
+                double acc = (r == j) ? (double)J->beta[(size_t)(cs + r) * H + h] : 0.0;
+                for (int i = 0; i < r; ++i) acc -= A[(size_t)r * C + i] * Tm[(size_t)i * C + j];
+                Tm[(size_t)r * C + j] = acc;
+            }
+        /* W = T Kt, Uv = T V */
+        for (int r = 0; r < L; ++r) {
+            for (int c = 0; c < dk; ++c) {
+                double acc = 0.0;
+                for (int i = 0; i < L; ++i)
+                    acc += Tm[(size_t)r * C + i] * (double)J->k[IDX3(cs + i, h, c, H, dk)] * exp(g[(size_t)i * dk + c]);
+                W[(size_t)r * dk + c] = acc;
+            }
+            for (int j = 0; j < dv; ++j) {
+                double acc = 0.0;
+                for (int i = 0; i < L; ++i) acc += Tm[(size_t)r * C + i] * (double)J->v[IDX3(cs + i, h, j, H, dv)];
+                Uv[(size_t)r * dv + j] = acc;
+            }
+        }
+        /* U = Uv - W S0 */
+        for (int r = 0; r < L; ++r)
+            for (int j = 0; j < dv; ++j) {
+                double acc = Uv[(size_t)r * dv + j];
+                for (int c = 0; c < dk; ++c) acc -= W[(size_t)r * dk + c] * S[(size_t)c * dv + j];
+                U[(size_t)r * dv + j] = acc;
+            }
+        /* outputs */
+        if (J->out) {
+            for (int r = 0; r < L; ++r) {
+                double* o = J->out + IDX3(cs + r, h, 0, H, dv);
+                for (int j = 0; j < dv; ++j) {
+                    double acc = 0.0;
+                    for (int c = 0; c < dk; ++c)
+                        acc += (double)J->q[IDX3(cs + r, h, c, H, dk)] * exp(g[(size_t)r * dk + c]) * S[(size_t)c * dv + j];
+                    o[j] = acc;
+                }
+                for (int i = 0; i <= r; ++i) {
+                    double p = 0.0;
+                    for (int c = 0; c < dk; ++c)
+                        p += (double)J->q[IDX3(cs + r, h, c, H, dk)] * (double)J->k[IDX3(cs + i, h, c, H, dk)] *
+                             exp(g[(size_t)r * dk + c] - g[(size_t)i * dk + c]);
+                    for (int j = 0; j < dv; ++j) o[j] += p * U[(size_t)i * dv + j];
+                }
+            }
+        }
+        /* state at the chunk end */
+        const double* glast = g + (size_t)(L - 1) * dk;
+        for (int c = 0; c < dk; ++c)
+            for (int j = 0; j < dv; ++j) {
+                double acc = exp(glast[c]) * S[(size_t)c * dv + j];
+                for (int i = 0; i < L; ++i)
+                    acc += (double)J->k[IDX3(cs + i, h, c, H, dk)] * exp(glast[c] - g[(size_t)i * dk + c]) *
+                           U[(size_t)i * dv + j];
+                Snew[(size_t)c * dv + j] = acc;
+            }
+        memcpy(S, Snew, sizeof(double) * (size_t)dk * dv);
+    }
+}
+
+static void* worker(void* arg)
+{
+    job_t* J = (job_t*)arg;
+    const int dk = J->dk, dv = J->dv, C = J->C > 0 ? J->C : 1;
+    const size_t sz = (size_t)dk * dv;
+    size_t extra;
+    if (J->mode == 0) extra = (size_t)dv;
+    else if (J->mode == 2) extra = (size_t)dk * dk + sz;
+    else extra = (size_t)C * dk * 2 + (size_t)C * C * 2 + (size_t)C * dv * 2 + sz;
+    double* S = (double*)malloc(sizeof(double) * (sz + extra));
+    if (!S) {
+        pthread_mutex_lock(&J->lock);
+        J->status = -2;
+        pthread_mutex_unlock(&J->lock);
+        return NULL;
+    }
+    double* work = S + sz;
+    for (;;) {
+        pthread_mutex_lock(&J->lock);
+        const int p = J->next_pair++;
+        pthread_mutex_unlock(&J->lock);
+        if (p >= J->N * J->H) break;
+        if (J->pair_mask && !J->pair_mask[p]) continue;
+        const int n = p / J->H, h = p % J->H;
+        if (J->S0) memcpy(S, J->S0 + (size_t)p * sz, sizeof(double) * sz);
+        else memset(S, 0, sizeof(double) * sz);
+        if (J->mode == 0) pair_seq(J, n, h, S, work);
+        else if (J->mode == 2) pair_bruteforce(J, n, h, S, work, work + (size_t)dk * dk);
+        else pair_chunked(J, n, h, S, work);
+        if (J->S_final) memcpy(J->S_final + (size_t)p * sz, S, sizeof(double) * sz);
+    }
+    free(S);
+    return NULL;
+}
+
+static int run(job_t* J, int num_threads)
+{
+    if (!J->q || !J->k || !J->v || !J->log_alpha || !J->beta || !J->cu_seqlens) return -1;
+    if (J->N < 0 || J->H <= 0 || J->dk <= 0 || J->dv <= 0) return -1;
+    for (int n = 0; n < J->N; ++n)
+        if (J->cu_seqlens[n + 1] < J->cu_seqlens[n]) return -1;
+    if (num_threads < 1) num_threads = 1;
+    J->next_pair = 0;
+    J->status = 0;
+    pthread_mutex_init(&J->lock, NULL);
+    pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)num_threads);
+    int started = 0;
+    for (int i = 0; i < num_threads; ++i)
+        if (pthread_create(&th[i], NULL, worker, J) == 0) ++started;
+    if (started == 0) worker(J);
+    for (int i = 0; i < started; ++i) pthread_join(th[i], NULL);
+    free(th);
+    pthread_mutex_destroy(&J->lock);
+    return J->status;
+}
+
+#define FILL_JOB(J, mode_, C_)                                                                    \
+    job_t J;                                                                                      \
+    memset(&J, 0, sizeof(J));                                                                     \
+    J.q = q; J.k = k; J.v = v; J.log_alpha = log_alpha; J.beta = beta; J.S0 = S0;                \
+    J.cu_seqlens = cu_seqlens; J.pair_mask = pair_mask; J.N = N; J.H = H; J.dk = dk; J.dv = dv;   \
+    J.C = (C_); J.out = out; J.S_final = S_final; J.mode = (mode_);
+
+/* The definition (sequential recurrence).  pair_mask: [N*H] (index n*H+h), nonzero = compute
+ * that pair, NULL = all pairs.  Returns 0 on success, -1 on bad arguments, -2 out of memory. */
+int kda_oracle_seq(const float* q, const float* k, const float* v, const float* log_alpha, const float* beta,
+                   const double* S0, const int64_t* cu_seqlens, int N, int H, int dk, int dv, double* out,
+                   double* S_final, const int32_t* pair_mask, int num_threads)
+{
+    FILL_JOB(J, 0, 1);
+    return run(&J, num_threads);
+}
+
+/* Dense transition-matrix form; for short sequences only. */
+int kda_oracle_bruteforce(const float* q, const float* k, const float* v, const float* log_alpha,
+                          const float* beta, const double* S0, const int64_t* cu_seqlens, int N, int H, int dk,
+                          int dv, double* out, double* S_final, const int32_t* pair_mask, int num_threads)
+{
+    FILL_JOB(J, 2, 1);
+    return run(&J, num_threads);
+}
+
+/* Chunked WY/UT form with chunk size C >= 1. */
+int kda_oracle_chunked(const float* q, const float* k, const float* v, const float* log_alpha, const float* beta,
+                       const double* S0, const int64_t* cu_seqlens, int N, int H, int dk, int dv, double* out,
+                       double* S_final, const int32_t* pair_mask, int C, int num_threads)
+{
+    if (C < 1) return -1;
+    FILL_JOB(J, 1, C);
+    return run(&J, num_threads);
+}
+
+/* One decode step for N independent sequences, in the loop order of the review's pseudo-code:
+ *   (a) decay       S' = S * exp(log_alpha)    (row c scaled)
+ *   (b) delta       d  = S'^T k,   v_mod = v - d
+ *   (c) update      S  = S' + k (beta v_mod)^T
+ *   (d) output      o  = S^T q                  (from the updated state)
+ * q, k, log_alpha: [N][H][dk]; v: [N][H][dv]; beta: [N][H]; S: [N][H][dk][dv] in/out; out: [N][H][dv]. */
+int kda_oracle_decode_step(const float* q, const float* k, const float* v, const float* log_alpha,
+                           const float* beta, double* S, int N, int H, int dk, int dv, double* out)
+{
+    if (!q || !k || !v || !log_alpha || !beta || !S || N < 0 || H <= 0 || dk <= 0 || dv <= 0) return -1;
+    double* d = (double*)malloc(sizeof(double) * (size_t)dv);
+    if (!d) return -2;
+    for (int p = 0; p < N * H; ++p) {
+        double* Sp = S + (size_t)p * dk * dv;
+        const float* kp = k + (size_t)p * dk;
+        const float* qp = q + (size_t)p * dk;
+        const float* vp = v + (size_t)p * dv;
+        const float* lp = log_alpha + (size_t)p * dk;
+        const double b = (double)beta[p];
+        for (int c = 0; c < dk; ++c) {
+            const double a = exp((double)lp[c]);
+            for (int j = 0; j < dv; ++j) Sp[(size_t)c * dv + j] *= a;
+        }
+        for (int j = 0; j < dv; ++j) {
+            double acc = 0.0;
+            for (int c = 0; c < dk; ++c) acc += Sp[(size_t)c * dv + j] * (double)kp[c];
+            d[j] = (double)vp[j] - acc; /* v_mod */
+        }
+        for (int c = 0; c < dk; ++c)
+            for (int j = 0; j < dv; ++j) Sp[(size_t)c * dv + j] += (double)kp[c] * (b * d[j]);
+        if (out)
+            for (int j = 0; j < dv; ++j) {
+                double acc = 0.0;
+                for (int c = 0; c < dk; ++c) acc += (double)qp[c] * Sp[(size_t)c * dv + j];
+                out[(size_t)p * dv + j] = acc;
+            }
+    }
+    free(d);
+    return 0;
+}

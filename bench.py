@@ -1,0 +1,415 @@
+#!/usr/bin/env python
+"""Benchmark of the KDA operator on B200: prints ONE JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Default workload: chunked prefill, B=1, H=32, T=32768, dk=dv=128, bf16 q/k/v, fp32 gates and
+state, S0 ~ N(0, 0.02^2).  A "step" is one kda_chunk_fwd call over that batch (all phases of the
+chunked prefill).  `value` is tokens/s over all ranks, device-timed with CUDA events on the
+launching stream with inputs resident in HBM; `e2e` is the same metric through the public API
+with the inputs copied from pinned host memory and out/S_final copied back inside the timed
+region.  A decode measurement (256 sequences x 32 heads, 512 successive single-token steps) is
+reported under "decode".  With N > 1 (torchrun) every rank runs an independent replica of the
+workload on its own GPU (no collective on the data path): weak scaling.
+
+--impl reference times the fp64 CPU oracle (the test oracle, as it stands) on a bounded sample of
+the same workload on this host's cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="prefill_32k")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target duration of the oracle sample")
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ------------------------------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ------------------------------------------------------------------------------------------------
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------------------
+# distributed plumbing (replicas only)
+# ------------------------------------------------------------------------------------------------
+def init_dist(torch):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(torch, world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(torch, world, x):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------------------------------------
+# CPU baseline: the fp64 oracle on a bounded sample of the workload
+# ------------------------------------------------------------------------------------------------
+def cpu_oracle_prefill(w, target_s, seed_offset=0):
+    """Time oracle.seq on all H heads of a prefix of the workload, sized to ~target_s seconds."""
+    import torch
+    import oracle
+    from gated_delta_rule_83_b200 import synth
+    threads = oracle.default_threads()
+
+    def run(T):
+        inp = synth.prefill_inputs(w, device="cpu", T=T, lengths=[T] if w.varlen else None,
+                                   seed=w.seed + seed_offset)
+        args = [synth.to_oracle(inp[x]) for x in ("q", "k", "v", "log_alpha", "beta")]
+        S0 = None if inp["S0"] is None else inp["S0"].double().numpy()
+        t0 = time.perf_counter()
+        oracle.seq(*args, S0=S0, threads=threads)
+        return time.perf_counter() - t0
+
+    probe_T = 128
+    dt = run(probe_T)
+    T = int(max(probe_T, min(w.T if not w.varlen else w.varlen[1], probe_T * target_s / max(dt, 1e-6))))
+    T = max(64, (T // 64) * 64)
+    dt = run(T)
+    return {"value": T / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{T} tokens x {w.H} heads (prefix of one sequence of the workload), fp64 sequential "
+                      f"recurrence, {threads} threads over heads, {dt:.1f} s"}
+
+
+def cpu_oracle_decode(w, target_s):
+    import oracle
+    from gated_delta_rule_83_b200 import synth
+    threads = 1
+    N = 8
+    S = np.asarray(synth.decode_state(w, N=N).double().numpy())
+    t0 = time.perf_counter()
+    steps = 0
+    while time.perf_counter() - t0 < target_s / 2 and steps < w.T:
+        inp = synth.decode_inputs(w, steps, N=N)
+        _, S = oracle.decode_step(*(synth.to_oracle(inp[x]) for x in ("q", "k", "v", "log_alpha", "beta")), S)
+        steps += 1
+    dt = time.perf_counter() - t0
+    return {"value": N * steps / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{N} sequences x {w.H} heads x {steps} decode steps, fp64, single thread, {dt:.1f} s"}
+
+
+# ------------------------------------------------------------------------------------------------
+# our arm
+# ------------------------------------------------------------------------------------------------
+def run_ours(args):
+    import torch
+    import gated_delta_rule_83_b200 as kda
+    from gated_delta_rule_83_b200 import synth
+
+    world, rank, local = init_dist(torch)
+    dev = torch.device("cuda", local)
+    hbm, tf, tf_sus, peak_kind = peaks()
+    w = synth.WORKLOADS[args.workload]
+    if w.kind != "prefill":
+        raise SystemExit("the headline workload is a prefill workload; decode is reported under 'decode'")
+
+    inp = synth.prefill_inputs(w, device=dev, seed=w.seed + 1000 * rank)
+    q, k, v, la, beta, S0, cu = (inp[x] for x in ("q", "k", "v", "log_alpha", "beta", "S0", "cu_seqlens"))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    tokens = B * T
+    out = torch.empty_like(v)
+    N = B if cu is None else cu.numel() - 1
+    S_fin = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    in_bytes = sum(x.numel() * x.element_size() for x in (q, k, v, la, beta) if x is not None)
+
+    def step():
+        kda.chunk_fwd(q, k, v, la, beta, S0=S0, cu_seqlens=cu, out=out, S_final=S_fin)
+
+    for _ in range(args.warmup):
+        step()
+    kda.check()
+    barrier(torch, world)
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    kda.profile_begin()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    prof = kda.profile_end()
+    barrier(torch, world)
+    clk = clocks.stop()
+    kda.check()
+    ms_local = e0.elapsed_time(e1)
+    ms = max_over_ranks(torch, world, ms_local)
+    ms_per_step = ms / args.steps
+    value = world * tokens * args.steps / (ms / 1e3)
+
+    # dominant kernel and roofline (algorithmic bytes of the whole prefill: q,k,v + log_alpha + beta in,
+    # out written; the state S0/S_final adds 2 x 64 KiB per (sequence, head))
+    launches = sum(n for n, _ in prof.values())
+    dom_name, (dom_n, dom_ms) = max(prof.items(), key=lambda kv: kv[1][1])
+    tok_heads = tokens * H
+    esz = q.element_size()
+    alg_bytes = tok_heads * (2 * dk * esz + dv * esz + 4 * dk + 4 + dv * esz) + \
+        (2 if S0 is not None else 1) * N * H * dk * dv * 4
+    step_dev_ms = sum(t for _, t in prof.values()) / args.steps
+    achieved = alg_bytes / (step_dev_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "kernel": "prefill step (all launches: " + ", ".join(sorted(prof)) + ")",
+                "dominant_kernel": dom_name, "dominant_share": dom_ms / max(sum(t for _, t in prof.values()), 1e-9),
+                "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                "peak_source": f"{peak_kind} hbm_gbs", "traffic": None,
+                "alg_bytes_per_step": alg_bytes, "device_ms_per_step": step_dev_ms}
+
+    # e2e: host buffers through the public API
+    e2e = None
+    try:
+        hq, hk, hv, hla, hb = (x.cpu().pin_memory() for x in (q, k, v, la, beta))
+        hS0 = S0.cpu().pin_memory() if S0 is not None else None
+        hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        hS = torch.empty(S_fin.shape, dtype=torch.float32).pin_memory()
+        dq, dk_, dv_, dla, db = (torch.empty_like(x) for x in (q, k, v, la, beta))
+        dS0 = torch.empty_like(S0) if S0 is not None else None
+        h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hla, hb)) + \
+            (hS0.numel() * 4 if hS0 is not None else 0)
+        d2h = hout.numel() * hout.element_size() + hS.numel() * 4
+
+        def e2e_step():
+            for d_, h_ in ((dq, hq), (dk_, hk), (dv_, hv), (dla, hla), (db, hb)):
+                d_.copy_(h_, non_blocking=True)
+            if dS0 is not None:
+                dS0.copy_(hS0, non_blocking=True)
+            kda.chunk_fwd(dq, dk_, dv_, dla, db, S0=dS0, cu_seqlens=cu, out=out, S_final=S_fin)
+            hout.copy_(out, non_blocking=True)
+            hS.copy_(S_fin, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier(torch, world)
+        n_e2e = max(2, min(args.steps, 5))
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_e2e = max_over_ranks(torch, world, e0.elapsed_time(e1))
+        e2e = {"value": world * tokens * n_e2e / (ms_e2e / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e / n_e2e,
+               "steps": n_e2e}
+        del hq, hk, hv, hla, hb, dq, dk_, dv_, dla, db
+    except Exception as ex:  # pragma: no cover
+        e2e = {"value": None, "unit": "tokens/s", "error": str(ex)[:200]}
+
+    del q, k, v, la, beta, out
+    torch.cuda.empty_cache()
+
+    decode = None
+    if not args.no_decode:
+        decode = bench_decode(torch, kda, synth, dev, stream, world, rank, hbm, peak_kind)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_oracle_prefill(w, args.cpu_seconds)
+
+    line = {"metric": "KDA prefill tokens/s (decode tokens/s under 'decode')", "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if esz == 2 else "f32",
+            "data": "synthetic (seeded; q,k ~N(0,1) L2-normalised, v ~N(0,1), log_alpha = log sigmoid(N(3,1)), "
+                    "beta = sigmoid(N(0,1)))",
+            "config": {"workload": w.name, "desc": w.desc, "B": B, "T": T, "H": H, "dk": dk, "dv": dv,
+                       "chunk": 64, "parallelism": f"replicas x{world} (independent problems, no collective)",
+                       "l2": f"inputs {in_bytes / 1e9:.2f} GB per step > L2 {L2_BYTES / 1e6:.0f} MB (no flush)"},
+            "roofline": roofline, "kernels": {k_: {"launches": n, "ms": t} for k_, (n, t) in prof.items()},
+            "gpu_launches": launches, "clocks": clk, "e2e": e2e, "decode": decode, "cpu_baseline": cpu}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def bench_decode(torch, kda, synth, dev, stream, world, rank, hbm, peak_kind, steps=None):
+    w = synth.WORKLOADS["decode_256x512"]
+    steps = steps or w.T
+    S = synth.decode_state(w, device=dev, seed=w.seed + 1000 * rank)
+    # per-step inputs, drawn fresh per step, pre-generated in HBM (one tensor per field with a step axis)
+    inp = synth.decode_inputs(w, 0, device=dev, steps=steps, seed=w.seed + 1000 * rank)
+    out = torch.empty((w.B, w.H, w.dv), dtype=torch.bfloat16, device=dev)
+    fields = [inp[x] for x in ("q", "k", "v", "log_alpha", "beta")]
+
+    def run(n):
+        for t in range(n):
+            kda.decode_step(fields[0][t], fields[1][t], fields[2][t], fields[3][t], fields[4][t], S, out=out)
+
+    run(8)
+    torch.cuda.synchronize(dev)
+    barrier(torch, world)
+    kda.profile_begin()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    run(steps)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    prof = kda.profile_end()
+    kda.check()
+    ms = max_over_ranks(torch, world, e0.elapsed_time(e1))
+    n, kms = prof["decode_step"]
+    pairs = w.B * w.H
+    alg = pairs * (2 * w.dk * w.dv * 4 + 2 * w.dk * 2 + w.dv * 2 + 4 * w.dk + 4 + w.dv * 2)
+    ach = alg / (kms / n / 1e3) / 1e9
+    return {"metric": "KDA decode tokens/s", "workload": w.name, "desc": w.desc,
+            "value": world * w.B * steps / (ms / 1e3), "unit": "tokens/s", "steps": steps,
+            "us_per_step": ms * 1e3 / steps,
+            "roofline": {"bound": "hbm", "kernel": "decode_step", "achieved": ach, "peak": hbm, "unit": "GB/s",
+                         "frac": ach / hbm, "peak_source": f"{peak_kind} hbm_gbs", "traffic": None,
+                         "alg_bytes_per_launch": alg, "device_us_per_launch": kms / n * 1e3},
+            "gpu_launches": n}
+
+
+# ------------------------------------------------------------------------------------------------
+# reference arm: the oracle on the host cores
+# ------------------------------------------------------------------------------------------------
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from gated_delta_rule_83_b200 import synth
+    w = synth.WORKLOADS[args.workload]
+    per_step = max(1.0, 60.0 / max(args.steps + args.warmup, 1))
+    for _ in range(args.warmup):
+        cpu_oracle_prefill(w, min(per_step, 2.0))
+    vals, samples = [], []
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        r = cpu_oracle_prefill(w, per_step)
+        vals.append(r["value"])
+        samples.append(r)
+    wall = time.perf_counter() - t0
+    v = statistics.median(vals)
+    cb = dict(samples[0])
+    cb["value"] = v
+    line = {"impl": "reference", "metric": "KDA prefill tokens/s (decode tokens/s under 'decode')", "value": v,
+            "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * wall / max(args.steps, 1), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, same generator as our arm)",
+            "config": {"workload": w.name, "desc": w.desc, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk, "dv": w.dv,
+                       "chunk": 64, "parallelism": "host cores (oracle)"},
+            "cpu_baseline": cb, "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                                        "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

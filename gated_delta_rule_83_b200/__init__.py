@@ -1,0 +1,12 @@
+"""B200-native Kimi Delta Attention (KDA) operator: chunked prefill and decode (libkda.so, sm_100a).
+
+Public API (a thin binding of the C ABI in include/kda.h):
+
+    out, S_final = chunk_fwd(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None)
+    out = decode_step(q, k, v, log_alpha, beta, S)        # S updated in place
+    check()                                               # raise on a device-side error
+"""
+from .kda import (KdaError, check, chunk_fwd, decode_step, load_library, profile_begin,  # noqa: F401
+                  profile_end, version, workspace_size)
+
+__all__ = ["chunk_fwd", "decode_step", "check", "workspace_size", "load_library", "version", "KdaError"]

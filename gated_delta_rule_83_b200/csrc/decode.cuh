@@ -1,0 +1,130 @@
+// decode.cuh -- fused single-token KDA decode step (state read once, written once).
+//
+// Per (sequence, head) the step is, in the order of the per-token loop in the attention review's
+// GDN/KDA pseudo-code (lanjinlin.com.cn, entry on Qwen3-Next GDN, the block that loads the
+// per-sequence state): decay S' = Diag(alpha) S; r = S'^T k; u = beta (v - r); S = S' + k u^T;
+// o = S^T q = S'^T q + u (q . k).  Both column reductions (r and S'^T q) come out of the single
+// read of S, and the rank-1 update is applied to the values still held in registers, so the
+// 64 KiB fp32 state of a 128x128 head crosses HBM exactly twice (one read, one write).
+//
+// Work decomposition: one CTA of 256 threads owns a 64-column slice of one head's state
+// (columns of S evolve independently).  A warp reads two 256-byte row segments per 128-bit load
+// instruction (lanes 0-15 row a, lanes 16-31 row a+1; each lane 4 consecutive columns), so every
+// state access is a fully coalesced, 16-byte-vectorised streaming load/store (ld.global.cs /
+// st.global.cs: the state is touched once per step and is far larger than L2).
+#pragma once
+
+#include "common.cuh"
+#include "profile.cuh"
+
+namespace kda {
+
+constexpr int kDecodeThreads = 256;
+constexpr int kDecodeSlice = 64;  // columns of S per CTA
+
+template <typename TIn, int DK>
+__global__ void __launch_bounds__(kDecodeThreads)
+decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
+                   const float* __restrict__ log_alpha, const float* __restrict__ beta, float* __restrict__ S,
+                   TIn* __restrict__ out, int dv)
+{
+    constexpr int RPT = DK / 16;  // state rows held per thread
+    const int nslices = dv / kDecodeSlice;
+    const int p = blockIdx.x / nslices;            // (sequence, head) pair, = n*H + h
+    const int j0 = (blockIdx.x % nslices) * kDecodeSlice;
+    const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
+    const int cg = l & 15;                         // columns j0 + 4cg .. j0 + 4cg + 3
+    const int rb = 2 * w + (l >> 4);               // rows rb + 16 i
+
+    __shared__ float s_a[DK], s_k[DK], s_q[DK];
+    __shared__ __align__(16) float s_red[8][16][8];
+
+    float* Sp = S + (size_t)p * DK * dv + j0;
+    float4 st[RPT];
+#pragma unroll
+    for (int i = 0; i < RPT; ++i)
+        st[i] = __ldcs(reinterpret_cast<const float4*>(Sp + (size_t)(rb + 16 * i) * dv) + cg);
+
+    for (int c = tid; c < DK; c += kDecodeThreads) {
+        s_a[c] = expf(log_alpha[(size_t)p * DK + c]);
+        s_k[c] = to_f32(k[(size_t)p * DK + c]);
+        s_q[c] = to_f32(q[(size_t)p * DK + c]);
+    }
+    __syncthreads();
+
+    float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f, q0 = 0.f, q1 = 0.f, q2 = 0.f, q3 = 0.f;
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) {
+        const int c = rb + 16 * i;
+        const float a = s_a[c], kc = s_k[c], qc = s_q[c];
+        st[i].x *= a; st[i].y *= a; st[i].z *= a; st[i].w *= a;
+        r0 = fmaf(st[i].x, kc, r0); r1 = fmaf(st[i].y, kc, r1); r2 = fmaf(st[i].z, kc, r2); r3 = fmaf(st[i].w, kc, r3);
+        q0 = fmaf(st[i].x, qc, q0); q1 = fmaf(st[i].y, qc, q1); q2 = fmaf(st[i].z, qc, q2); q3 = fmaf(st[i].w, qc, q3);
+    }
+    r0 += __shfl_xor_sync(0xffffffffu, r0, 16); r1 += __shfl_xor_sync(0xffffffffu, r1, 16);
+    r2 += __shfl_xor_sync(0xffffffffu, r2, 16); r3 += __shfl_xor_sync(0xffffffffu, r3, 16);
+    q0 += __shfl_xor_sync(0xffffffffu, q0, 16); q1 += __shfl_xor_sync(0xffffffffu, q1, 16);
+    q2 += __shfl_xor_sync(0xffffffffu, q2, 16); q3 += __shfl_xor_sync(0xffffffffu, q3, 16);
+    if (l < 16) {
+        float4* dst = reinterpret_cast<float4*>(&s_red[w][cg][0]);
+        dst[0] = make_float4(r0, r1, r2, r3);
+        dst[1] = make_float4(q0, q1, q2, q3);
+    }
+    __syncthreads();
+
+    float4 rr = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int ww = 0; ww < 8; ++ww) {
+        const float4 x = reinterpret_cast<const float4*>(&s_red[ww][cg][0])[0];
+        rr.x += x.x; rr.y += x.y; rr.z += x.z; rr.w += x.w;
+    }
+    const float b = beta[p];
+    const TIn* vp = v + (size_t)p * dv + j0 + 4 * cg;
+    const float u0 = b * (to_f32(vp[0]) - rr.x), u1 = b * (to_f32(vp[1]) - rr.y);
+    const float u2 = b * (to_f32(vp[2]) - rr.z), u3 = b * (to_f32(vp[3]) - rr.w);
+
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) {
+        const int c = rb + 16 * i;
+        const float kc = s_k[c];
+        float4 x = st[i];
+        x.x = fmaf(kc, u0, x.x); x.y = fmaf(kc, u1, x.y); x.z = fmaf(kc, u2, x.z); x.w = fmaf(kc, u3, x.w);
+        __stcs(reinterpret_cast<float4*>(Sp + (size_t)c * dv) + cg, x);
+    }
+
+    if (w == 0 && l < 16) {
+        float qk = 0.f;
+        for (int c = 0; c < DK; ++c) qk = fmaf(s_q[c], s_k[c], qk);
+        float4 ss = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int ww = 0; ww < 8; ++ww) {
+            const float4 x = reinterpret_cast<const float4*>(&s_red[ww][cg][4])[0];
+            ss.x += x.x; ss.y += x.y; ss.z += x.z; ss.w += x.w;
+        }
+        TIn* op = out + (size_t)p * dv + j0 + 4 * cg;
+        op[0] = from_f32<TIn>(fmaf(u0, qk, ss.x));
+        op[1] = from_f32<TIn>(fmaf(u1, qk, ss.y));
+        op[2] = from_f32<TIn>(fmaf(u2, qk, ss.z));
+        op[3] = from_f32<TIn>(fmaf(u3, qk, ss.w));
+    }
+}
+
+template <typename TIn>
+cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* la, const float* beta, float* S,
+                          void* out, int N, int H, int dk, int dv, cudaStream_t stream)
+{
+    const long long pairs = (long long)N * H;
+    const long long blocks = pairs * (dv / kDecodeSlice);
+    if (blocks == 0) return cudaSuccess;
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+    LaunchScope ls("decode_step", stream);
+    if (dk == 128)
+        decode_step_kernel<TIn, 128><<<(unsigned)blocks, kDecodeThreads, 0, stream>>>(
+            (const TIn*)q, (const TIn*)k, (const TIn*)v, la, beta, S, (TIn*)out, dv);
+    else
+        decode_step_kernel<TIn, 64><<<(unsigned)blocks, kDecodeThreads, 0, stream>>>(
+            (const TIn*)q, (const TIn*)k, (const TIn*)v, la, beta, S, (TIn*)out, dv);
+    return cudaGetLastError();
+}
+
+}  // namespace kda

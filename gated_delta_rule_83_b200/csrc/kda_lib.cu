@@ -1,0 +1,213 @@
+// kda_lib.cu -- the C ABI of libkda.so (declared in include/kda.h): argument validation,
+// workspace carving and kernel dispatch.  Every step of the operator runs in the kernels
+// included below; this file only checks arguments and launches.
+#include <cstdio>
+#include <cstring>
+
+#include "kda.h"
+#include "common.cuh"
+#include "chunks.cuh"
+#include "decode.cuh"
+#include "prefill_simt.cuh"
+#include "prefill_tc.cuh"
+#include "profile.cuh"
+
+using namespace kda;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+bool dims_supported(int dk, int dv) { return (dk == 64 || dk == 128) && (dv == 64 || dv == 128); }
+
+// The tensor-core path covers bf16 with dk = dv = 128; everything else runs the fp32 CUDA-core path.
+bool use_tc_path(kda_dtype dt, int dk, int dv) { return kTcPathReady && dt == KDA_BF16 && dk == 128 && dv == 128; }
+
+struct Plan {
+    int N;            // number of sequences
+    int Tseq;         // tokens per sequence (regular batches); 0 for varlen
+    long long Ttot;   // total tokens
+    int max_chunks;   // upper bound on the number of chunks
+    bool tc;
+    size_t off_bytes, slot_bytes, total_bytes;
+};
+
+kda_status make_plan(int B, int T, int H, int dk, int dv, bool varlen, int num_seqs, kda_dtype dt, Plan& p)
+{
+    if (dt != KDA_BF16 && dt != KDA_F32) return KDA_ERR_INVALID_ARG;
+    if (H <= 0 || T < 0 || B <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+    if (!dims_supported(dk, dv)) return KDA_ERR_UNSUPPORTED;
+    if (H > 65535) return KDA_ERR_UNSUPPORTED;
+    if (varlen) {
+        if (B != 1 || num_seqs <= 0) return KDA_ERR_INVALID_ARG;
+        p.N = num_seqs;
+        p.Tseq = 0;
+        p.Ttot = T;
+        p.max_chunks = T / kChunk + num_seqs;
+    } else {
+        p.N = B;
+        p.Tseq = T;
+        p.Ttot = (long long)B * T;
+        const long long mc = (long long)B * ((T + kChunk - 1) / kChunk);
+        if (mc > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+        p.max_chunks = (int)mc;
+    }
+    if (p.Ttot > 0x7fffffffLL || p.N > 65535 * 64) return KDA_ERR_UNSUPPORTED;
+    p.tc = use_tc_path(dt, dk, dv);
+    p.off_bytes = round_up(sizeof(int) * ((size_t)p.N + 1), kAlign);
+    p.slot_bytes = p.tc ? tc_slot_bytes() : round_up(sizeof(float) * simt_slot_floats(dk, dv), kAlign);
+    p.total_bytes = sizeof(WsHeader) + p.off_bytes + (size_t)p.max_chunks * (size_t)H * p.slot_bytes;
+    return KDA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* kda_status_string(kda_status s)
+{
+    switch (s) {
+        case KDA_OK: return "KDA_OK";
+        case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG";
+        case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED";
+        case KDA_ERR_CUDA: return "KDA_ERR_CUDA";
+        case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT";
+        case KDA_ERR_WORKSPACE: return "KDA_ERR_WORKSPACE";
+        case KDA_ERR_BAD_SEQLENS: return "KDA_ERR_BAD_SEQLENS";
+    }
+    return "KDA_ERR_UNKNOWN";
+}
+
+const char* kda_version(void) { return "kda-b200 0.1 sm_100a"; }
+
+kda_status kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int varlen, int num_seqs,
+                                        kda_dtype dt, size_t* bytes)
+{
+    if (!bytes) return KDA_ERR_INVALID_ARG;
+    Plan p;
+    const kda_status st = make_plan(B, T, H, dk, dv, varlen != 0, num_seqs, dt, p);
+    if (st != KDA_OK) return st;
+    *bytes = p.total_bytes;
+    return KDA_OK;
+}
+
+kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const float* log_alpha, const float* beta,
+                         const float* S0, const int32_t* cu_seqlens, int num_seqs, void* out, float* S_final,
+                         int B, int T, int H, int dk, int dv, kda_dtype dt, void* workspace,
+                         size_t workspace_bytes, kda_stream_t stream_)
+{
+    cudaStream_t stream = (cudaStream_t)stream_;
+    Plan p;
+    const kda_status st = make_plan(B, T, H, dk, dv, cu_seqlens != nullptr, num_seqs, dt, p);
+    if (st != KDA_OK) return st;
+    if (p.Ttot > 0 && (!q || !k || !v || !log_alpha || !beta || !out)) return KDA_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, log_alpha, beta, S0, out, S_final};
+    for (const void* x : ptrs)
+        if (x && !aligned16(x)) return KDA_ERR_INVALID_ARG;
+    if (cu_seqlens && ((uintptr_t)cu_seqlens & 3u)) return KDA_ERR_INVALID_ARG;
+    if (!workspace || ((uintptr_t)workspace % kAlign) || workspace_bytes < p.total_bytes) return KDA_ERR_WORKSPACE;
+
+    char* ws = (char*)workspace;
+    WsHeader* hdr = (WsHeader*)ws;
+    int* off = (int*)(ws + sizeof(WsHeader));
+    char* slots = ws + sizeof(WsHeader) + p.off_bytes;
+
+    {
+        LaunchScope ls("chunk_table", stream);
+        chunk_table_kernel<<<1, kTableThreads, 0, stream>>>(cu_seqlens, p.N, p.Tseq, p.Ttot, hdr, off);
+        if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
+    }
+
+    cudaError_t e;
+    if (p.tc) {
+        e = launch_tc_prefill(q, k, v, log_alpha, beta, S0, S_final, out, hdr, off, cu_seqlens, p.Tseq, p.N, H,
+                              p.max_chunks, slots, stream);
+    } else if (dt == KDA_BF16) {
+        e = launch_simt_prefill<__nv_bfloat16>(q, k, v, log_alpha, beta, S0, S_final, out, hdr, off, cu_seqlens,
+                                               p.Tseq, p.N, H, dk, dv, p.max_chunks, (float*)slots, stream);
+    } else {
+        e = launch_simt_prefill<float>(q, k, v, log_alpha, beta, S0, S_final, out, hdr, off, cu_seqlens, p.Tseq,
+                                       p.N, H, dk, dv, p.max_chunks, (float*)slots, stream);
+    }
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_decode_step(const void* q, const void* k, const void* v, const float* log_alpha, const float* beta,
+                           float* S_inout, void* out, int N, int H, int dk, int dv, kda_dtype dt,
+                           kda_stream_t stream_)
+{
+    cudaStream_t stream = (cudaStream_t)stream_;
+    if (dt != KDA_BF16 && dt != KDA_F32) return KDA_ERR_INVALID_ARG;
+    if (N < 0 || H <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+    if (!dims_supported(dk, dv)) return KDA_ERR_UNSUPPORTED;
+    if (N == 0) return KDA_OK;
+    if (!q || !k || !v || !log_alpha || !beta || !S_inout || !out) return KDA_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, log_alpha, beta, S_inout, out};
+    for (const void* x : ptrs)
+        if (!aligned16(x)) return KDA_ERR_INVALID_ARG;
+    const cudaError_t e = (dt == KDA_BF16)
+        ? launch_decode<__nv_bfloat16>(q, k, v, log_alpha, beta, S_inout, out, N, H, dk, dv, stream)
+        : launch_decode<float>(q, k, v, log_alpha, beta, S_inout, out, N, H, dk, dv, stream);
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_profile_begin(void)
+{
+    Profiler& p = profiler();
+    std::lock_guard<std::mutex> g(p.mu);
+    p.recs.clear();
+    p.used = 0;
+    p.on = true;
+    return KDA_OK;
+}
+
+kda_status kda_profile_end(void)
+{
+    Profiler& p = profiler();
+    std::lock_guard<std::mutex> g(p.mu);
+    p.on = false;
+    return KDA_OK;
+}
+
+int kda_profile_kernels(int max_kernels, const char** names, int* launches, double* total_ms)
+{
+    Profiler& p = profiler();
+    std::lock_guard<std::mutex> g(p.mu);
+    int n = 0;
+    for (const ProfRecord& r : p.recs) {
+        float ms = 0.f;
+        if (cudaEventSynchronize(r.stop) != cudaSuccess || cudaEventElapsedTime(&ms, r.start, r.stop) != cudaSuccess)
+            return -1;
+        int i = 0;
+        while (i < n && std::strcmp(names[i], r.name) != 0) ++i;
+        if (i == n) {
+            if (n == max_kernels) return -1;
+            names[n] = r.name;
+            launches[n] = 0;
+            total_ms[n] = 0.0;
+            ++n;
+        }
+        launches[i] += 1;
+        total_ms[i] += ms;
+    }
+    return n;
+}
+
+kda_status kda_check(kda_stream_t stream_)
+{
+    cudaStream_t stream = (cudaStream_t)stream_;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return KDA_ERR_CUDA;
+    int word = 0;
+    if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(int)) != cudaSuccess) return KDA_ERR_CUDA;
+    if (word != 0) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(int)) != cudaSuccess) return KDA_ERR_CUDA;
+        return (kda_status)word;
+    }
+    return KDA_OK;
+}
+
+}  // extern "C"

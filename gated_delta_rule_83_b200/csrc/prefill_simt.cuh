@@ -1,0 +1,297 @@
+// prefill_simt.cuh -- chunked KDA prefill on CUDA cores in fp32 (any dt, dk/dv in {64, 128}).
+//
+// This is the full-precision path: it serves the fp32 dtype (where a tensor-core path would round
+// operands to tf32 or bf16) and shapes the tensor-core path does not cover.  It follows the chunk
+// form of the recurrence (chunk-parallel inside a chunk, recurrent between chunks, WY
+// representation, UT transform -- "Kimi Linear" explainer, section "硬件效率的深度优化"):
+//
+//   phase A (one CTA per (chunk, head), all chunks in parallel):
+//     g_r   = sum_{i<=r} log_alpha_i                       (restarted every chunk)
+//     A     = strict_lower( beta_r sum_c k_rc k_ic e^{g_rc - g_ic} )
+//     P     = lower_incl(  sum_c q_rc k_ic e^{g_rc - g_ic} )
+//     T     = (I + A)^{-1} diag(beta)                      (forward substitution)
+//     W     = T (k * e^{g}),  Uv = T v,  Qg = q * e^{g},  Kd = k * e^{g_last - g},  gam = e^{g_last}
+//   phase B (one CTA per (sequence, head, 32-column slice of S), chunks in order):
+//     U = Uv - W S;   O = Qg S + P U;   S <- Diag(gam) S + Kd^T U
+//
+// The intra-chunk products factor e^{g_r - g_i} = e^{g_r - ref} e^{ref - g_i} around the centre of
+// each channel's in-chunk gate range, which keeps every factor within e^{+-80}; a chunk in which
+// some channel decays by more than e^-160 uses the exact per-element factor instead (never larger
+// than 1), so no gate value can overflow.  Padding rows of a partial chunk are identity steps
+// (k = q = v = 0, log_alpha = 0, beta = 0).
+#pragma once
+
+#include "common.cuh"
+#include "profile.cuh"
+
+namespace kda {
+
+constexpr int kSimtThreads = 256;
+constexpr int kSimtNV = 32;  // state columns per phase-B CTA
+
+// fp32 workspace slot of one (chunk, head): W | Qg | Kd [64 x dk] | P [64 x 64] | Uv [64 x dv] | gam [dk]
+__host__ __device__ inline size_t simt_slot_floats(int dk, int dv)
+{
+    return (size_t)kChunk * (3 * dk + kChunk + dv) + dk;
+}
+
+// Largest spread of the in-chunk cumulative gate (per channel) for which the factorised products
+// below stay finite in fp32: each factor is e^{+-x} with |x| <= kFactorSpread / 2 <= 80.
+constexpr float kFactorSpread = 160.f;
+
+template <typename TIn>
+__global__ void __launch_bounds__(kSimtThreads)
+simt_intra_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
+                  const float* __restrict__ log_alpha, const float* __restrict__ beta, const WsHeader* __restrict__ hdr,
+                  const int* __restrict__ off, const int32_t* __restrict__ cu, int Tseq, int N, int H, int dk, int dv,
+                  float* __restrict__ slots)
+{
+    extern __shared__ __align__(16) float smem[];
+    const int j = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+    if (hdr->bad || j >= hdr->total_chunks) return;
+    int n, L;
+    long long t0;
+    locate_chunk(j, off, cu, Tseq, N, n, t0, L);
+
+    float* sk = smem;                       // [64][dk]  k, later k e^{g - ref}
+    float* sq = sk + kChunk * dk;           // [64][dk]  q, later q e^{g - ref}
+    float* sg = sq + kChunk * dk;           // [64][dk]  g, later k e^{ref - g}
+    float* sv = sg + kChunk * dk;           // [64][dv]
+    float* sKt = sv + kChunk * dv;          // [64][dk]  k e^{g}
+    float* sA = sKt + kChunk * dk;          // [64][64]
+    float* sP = sA + kChunk * kChunk;       // [64][64]
+    float* sT = sP + kChunk * kChunk;       // [64][64]
+    float* sb = sT + kChunk * kChunk;       // [64]
+    float* sref = sb + kChunk;              // [dk]
+    __shared__ int s_wide;
+
+    if (tid == 0) s_wide = 0;
+    for (int e = tid; e < kChunk * dk; e += kSimtThreads) {
+        const int r = e / dk, c = e % dk;
+        float kv = 0.f, qv = 0.f, lv = 0.f;
+        if (r < L) {
+            const size_t gi = ((size_t)(t0 + r) * H + h) * dk + c;
+            kv = to_f32(k[gi]); qv = to_f32(q[gi]); lv = log_alpha[gi];
+        }
+        sk[e] = kv; sq[e] = qv; sg[e] = lv;
+    }
+    for (int e = tid; e < kChunk * dv; e += kSimtThreads) {
+        const int r = e / dv, c = e % dv;
+        sv[e] = (r < L) ? to_f32(v[((size_t)(t0 + r) * H + h) * dv + c]) : 0.f;
+    }
+    for (int r = tid; r < kChunk; r += kSimtThreads) sb[r] = (r < L) ? beta[(size_t)(t0 + r) * H + h] : 0.f;
+    __syncthreads();
+
+    // cumulative gate per channel; reference point = centre of the channel's range
+    for (int c = tid; c < dk; c += kSimtThreads) {
+        float acc = 0.f, lo = 0.f, hi = 0.f;
+        for (int r = 0; r < kChunk; ++r) {
+            acc += sg[r * dk + c];
+            sg[r * dk + c] = acc;
+            lo = fminf(lo, acc);
+            hi = fmaxf(hi, acc);
+        }
+        sref[c] = 0.5f * (lo + hi);
+        if (!(hi - lo <= kFactorSpread)) atomicOr(&s_wide, 1);
+    }
+    __syncthreads();
+
+    const size_t slot_f = simt_slot_floats(dk, dv);
+    float* slot = slots + ((size_t)j * H + h) * slot_f;
+    float* gW = slot;
+    float* gQ = gW + (size_t)kChunk * dk;
+    float* gKd = gQ + (size_t)kChunk * dk;
+    float* gP = gKd + (size_t)kChunk * dk;
+    float* gUv = gP + (size_t)kChunk * kChunk;
+    float* gGam = gUv + (size_t)kChunk * dv;
+
+    // gated operands that never overflow (every exponent <= 0)
+    for (int e = tid; e < kChunk * dk; e += kSimtThreads) {
+        const int r = e / dk, c = e % dk;
+        const float gl = sg[(kChunk - 1) * dk + c];
+        const float eg = expf(sg[e]);
+        gQ[e] = sq[e] * eg;
+        gKd[e] = sk[e] * expf(gl - sg[e]);
+        sKt[e] = sk[e] * eg;
+        if (r == 0) gGam[c] = expf(gl);
+    }
+    __syncthreads();
+
+    const bool wide = s_wide != 0;
+    if (!wide) {
+        // factorised form: e^{g_r - g_i} = e^{g_r - ref} e^{ref - g_i}, both factors within e^{+-80}
+        for (int e = tid; e < kChunk * dk; e += kSimtThreads) {
+            const int c = e % dk;
+            const float x = sg[e] - sref[c];
+            const float kv = sk[e];
+            sk[e] = kv * expf(x);
+            sq[e] = sq[e] * expf(x);
+            sg[e] = kv * expf(-x);
+        }
+        __syncthreads();
+        for (int e = tid; e < kChunk * kChunk; e += kSimtThreads) {
+            const int r = e / kChunk, i = e % kChunk;
+            float a = 0.f, p = 0.f;
+            if (i <= r) {
+                for (int c = 0; c < dk; ++c) {
+                    const float kb = sg[i * dk + c];
+                    a = fmaf(sk[r * dk + c], kb, a);
+                    p = fmaf(sq[r * dk + c], kb, p);
+                }
+            }
+            sA[e] = (i < r) ? sb[r] * a : 0.f;
+            sP[e] = p;
+        }
+    } else {
+        // some channel decays by more than e^-160 inside the chunk: exact per-element factors
+        for (int e = tid; e < kChunk * kChunk; e += kSimtThreads) {
+            const int r = e / kChunk, i = e % kChunk;
+            float a = 0.f, p = 0.f;
+            if (i <= r) {
+                for (int c = 0; c < dk; ++c) {
+                    const float kk = sk[i * dk + c] * expf(sg[r * dk + c] - sg[i * dk + c]);
+                    a = fmaf(sk[r * dk + c], kk, a);
+                    p = fmaf(sq[r * dk + c], kk, p);
+                }
+            }
+            sA[e] = (i < r) ? sb[r] * a : 0.f;
+            sP[e] = p;
+        }
+    }
+    __syncthreads();
+
+    // T = (I + A)^{-1} diag(beta): thread jj owns column jj; rows in order.
+    if (tid < kChunk) {
+        const int jj = tid;
+        for (int r = 0; r < kChunk; ++r) {
+            float t = (r == jj) ? sb[r] : 0.f;
+            for (int i = jj; i < r; ++i) t = fmaf(-sA[r * kChunk + i], sT[i * kChunk + jj], t);
+            sT[r * kChunk + jj] = (jj <= r) ? t : 0.f;
+        }
+    }
+    for (int e = tid; e < kChunk * kChunk; e += kSimtThreads) gP[e] = sP[e];
+    __syncthreads();
+
+    for (int e = tid; e < kChunk * dk; e += kSimtThreads) {
+        const int r = e / dk, c = e % dk;
+        float acc = 0.f;
+        for (int i = 0; i <= r; ++i) acc = fmaf(sT[r * kChunk + i], sKt[i * dk + c], acc);
+        gW[e] = acc;
+    }
+    for (int e = tid; e < kChunk * dv; e += kSimtThreads) {
+        const int r = e / dv, c = e % dv;
+        float acc = 0.f;
+        for (int i = 0; i <= r; ++i) acc = fmaf(sT[r * kChunk + i], sv[i * dv + c], acc);
+        gUv[e] = acc;
+    }
+}
+
+template <typename TOut>
+__global__ void __launch_bounds__(kSimtThreads)
+simt_inter_kernel(const float* S0, float* S_final, TOut* __restrict__ out, const WsHeader* __restrict__ hdr,
+                  const int* __restrict__ off, const int32_t* __restrict__ cu, int Tseq, int N, int H, int dk, int dv,
+                  const float* __restrict__ slots)
+{
+    extern __shared__ __align__(16) float smem[];
+    const int n = blockIdx.x, h = blockIdx.y, v0 = blockIdx.z * kSimtNV, tid = threadIdx.x;
+    if (hdr->bad) return;
+    constexpr int NV = kSimtNV;
+    float* sS = smem;                       // [dk][NV]
+    float* sW = sS + dk * NV;               // [64][dk]
+    float* sQ = sW + kChunk * dk;           // [64][dk]
+    float* sKd = sQ + kChunk * dk;          // [64][dk]
+    float* sP = sKd + kChunk * dk;          // [64][64]
+    float* sUv = sP + kChunk * kChunk;      // [64][NV]
+    float* sU = sUv + kChunk * NV;          // [64][NV]
+    float* sG = sU + kChunk * NV;           // [dk]
+
+    const size_t sidx = ((size_t)n * H + h) * dk * dv;
+    for (int e = tid; e < dk * NV; e += kSimtThreads) {
+        const int c = e / NV, jj = e % NV;
+        sS[e] = S0 ? S0[sidx + (size_t)c * dv + v0 + jj] : 0.f;
+    }
+    long long s0, s1;
+    seq_bounds(n, cu, Tseq, s0, s1);
+    const size_t slot_f = simt_slot_floats(dk, dv);
+    for (int j = off[n]; j < off[n + 1]; ++j) {
+        const long long t0 = s0 + (long long)(j - off[n]) * kChunk;
+        const int L = (s1 - t0) < kChunk ? (int)(s1 - t0) : kChunk;
+        const float* slot = slots + ((size_t)j * H + h) * slot_f;
+        const float* gW = slot;
+        const float* gQ = gW + (size_t)kChunk * dk;
+        const float* gKd = gQ + (size_t)kChunk * dk;
+        const float* gP = gKd + (size_t)kChunk * dk;
+        const float* gUv = gP + (size_t)kChunk * kChunk;
+        const float* gGam = gUv + (size_t)kChunk * dv;
+        __syncthreads();  // previous chunk finished with the staged operands
+        for (int e = tid; e < kChunk * dk; e += kSimtThreads) { sW[e] = gW[e]; sQ[e] = gQ[e]; sKd[e] = gKd[e]; }
+        for (int e = tid; e < kChunk * kChunk; e += kSimtThreads) sP[e] = gP[e];
+        for (int e = tid; e < kChunk * NV; e += kSimtThreads) sUv[e] = gUv[(e / NV) * dv + v0 + (e % NV)];
+        for (int e = tid; e < dk; e += kSimtThreads) sG[e] = gGam[e];
+        __syncthreads();
+        for (int e = tid; e < kChunk * NV; e += kSimtThreads) {
+            const int r = e / NV, jj = e % NV;
+            float x = 0.f;
+            for (int c = 0; c < dk; ++c) x = fmaf(sW[r * dk + c], sS[c * NV + jj], x);
+            sU[e] = sUv[e] - x;
+        }
+        __syncthreads();
+        for (int e = tid; e < kChunk * NV; e += kSimtThreads) {
+            const int r = e / NV, jj = e % NV;
+            if (r >= L) continue;
+            float o = 0.f;
+            for (int c = 0; c < dk; ++c) o = fmaf(sQ[r * dk + c], sS[c * NV + jj], o);
+            for (int i = 0; i <= r; ++i) o = fmaf(sP[r * kChunk + i], sU[i * NV + jj], o);
+            out[((size_t)(t0 + r) * H + h) * dv + v0 + jj] = from_f32<TOut>(o);
+        }
+        __syncthreads();
+        for (int e = tid; e < dk * NV; e += kSimtThreads) {
+            const int c = e / NV, jj = e % NV;
+            float s = sG[c] * sS[e];
+            for (int i = 0; i < kChunk; ++i) s = fmaf(sKd[i * dk + c], sU[i * NV + jj], s);
+            sS[e] = s;
+        }
+    }
+    __syncthreads();
+    if (S_final)
+        for (int e = tid; e < dk * NV; e += kSimtThreads) {
+            const int c = e / NV, jj = e % NV;
+            S_final[sidx + (size_t)c * dv + v0 + jj] = sS[e];
+        }
+}
+
+inline size_t simt_intra_smem(int dk, int dv)
+{
+    return sizeof(float) * ((size_t)kChunk * (4 * dk + dv) + 3 * kChunk * kChunk + kChunk + dk);
+}
+inline size_t simt_inter_smem(int dk, int dv)
+{
+    (void)dv;
+    return sizeof(float) * ((size_t)dk * kSimtNV + 3 * kChunk * dk + kChunk * kChunk + 2 * kChunk * kSimtNV + dk);
+}
+
+template <typename TIn>
+cudaError_t launch_simt_prefill(const void* q, const void* k, const void* v, const float* la, const float* beta,
+                                const float* S0, float* S_final, void* out, const WsHeader* hdr, const int* off,
+                                const int32_t* cu, int Tseq, int N, int H, int dk, int dv, int max_chunks, float* slots,
+                                cudaStream_t stream)
+{
+    const size_t smA = simt_intra_smem(dk, dv), smB = simt_inter_smem(dk, dv);
+    cudaError_t e = cudaFuncSetAttribute(simt_intra_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smA);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(simt_inter_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smB);
+    if (e != cudaSuccess) return e;
+    if (max_chunks > 0) {
+        LaunchScope ls("simt_intra", stream);
+        simt_intra_kernel<TIn><<<dim3(max_chunks, H), kSimtThreads, smA, stream>>>(
+            (const TIn*)q, (const TIn*)k, (const TIn*)v, la, beta, hdr, off, cu, Tseq, N, H, dk, dv, slots);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    LaunchScope ls("simt_inter", stream);
+    simt_inter_kernel<TIn><<<dim3(N, H, dv / kSimtNV), kSimtThreads, smB, stream>>>(
+        S0, S_final, (TIn*)out, hdr, off, cu, Tseq, N, H, dk, dv, slots);
+    return cudaGetLastError();
+}
+
+}  // namespace kda

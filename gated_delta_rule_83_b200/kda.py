@@ -1,0 +1,231 @@
+"""Thin Python binding of libkda.so (the C ABI declared in include/kda.h).
+
+Argument marshalling only: tensors are checked for device/dtype/layout, their device pointers and
+the current CUDA stream are handed to the C entry points, and status codes become exceptions.
+Every step of the operator runs in the library's CUDA kernels; there is no fallback of any kind,
+and importing a missing or unbuilt library raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libkda.so")
+
+KDA_BF16, KDA_F32 = 0, 1
+STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED", 3: "KDA_ERR_CUDA",
+          4: "KDA_ERR_TIMEOUT", 5: "KDA_ERR_WORKSPACE", 6: "KDA_ERR_BAD_SEQLENS"}
+
+# The C ABI, as declared in include/kda.h (name -> (restype, argtypes)).
+_P, _I, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+ABI = {
+    "kda_status_string": (ctypes.c_char_p, [_I]),
+    "kda_version": (ctypes.c_char_p, []),
+    "kda_chunk_fwd_workspace_size": (_I, [_I, _I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_SZ)]),
+    "kda_chunk_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _I, _P, _SZ, _P]),
+    "kda_decode_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "kda_check": (_I, [_P]),
+    "kda_profile_begin": (_I, []),
+    "kda_profile_end": (_I, []),
+    "kda_profile_kernels": (_I, [_I, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(_I),
+                                 ctypes.POINTER(ctypes.c_double)]),
+}
+
+_lib = None
+
+
+class KdaError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} returned {STATUS.get(code, code)}")
+        self.code = code
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libkda.so (build it first with ``python -m gated_delta_rule_83_b200.build``)."""
+    global _lib
+    if _lib is None or path != LIB_PATH:
+        if not os.path.exists(path):
+            raise ImportError(f"{path} is missing: build it with `python -m gated_delta_rule_83_b200.build`")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in ABI.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        if path != LIB_PATH:
+            return lib
+        _lib = lib
+    return _lib
+
+
+def _check(fn: str, code: int):
+    if code != 0:
+        raise KdaError(fn, code)
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return KDA_BF16
+    if t.dtype == torch.float32:
+        return KDA_F32
+    raise TypeError(f"q/k/v must be bfloat16 or float32, got {t.dtype}")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _req(t: torch.Tensor, name: str, dtype=None, device=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def _stream_handle(stream: Optional[torch.cuda.Stream], device) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return s.cuda_stream
+
+
+_workspaces = {}
+
+
+def workspace_size(B: int, T: int, H: int, dk: int, dv: int, varlen: bool = False, num_seqs: int = 0,
+                   dtype: torch.dtype = torch.bfloat16) -> int:
+    lib = load_library()
+    n = ctypes.c_size_t(0)
+    dt = KDA_BF16 if dtype == torch.bfloat16 else KDA_F32
+    _check("kda_chunk_fwd_workspace_size",
+           lib.kda_chunk_fwd_workspace_size(B, T, H, dk, dv, int(bool(varlen)), num_seqs, dt, ctypes.byref(n)))
+    return n.value
+
+
+def _get_workspace(nbytes: int, device, stream_handle: int) -> torch.Tensor:
+    key = (device, stream_handle)
+    ws = _workspaces.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+        _workspaces[key] = ws
+    return ws
+
+
+def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor, beta: torch.Tensor,
+              S0: Optional[torch.Tensor] = None, cu_seqlens: Optional[torch.Tensor] = None,
+              out: Optional[torch.Tensor] = None, S_final: Optional[torch.Tensor] = None,
+              output_final_state: bool = True, workspace: Optional[torch.Tensor] = None,
+              stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Chunked KDA prefill (``kda_chunk_fwd``).
+
+    q, k, log_alpha: [B, T, H, dk]; v: [B, T, H, dv]; beta: [B, T, H]; q/k/v bf16 or fp32, gates fp32.
+    S0 / S_final: [N, H, dk, dv] fp32 (N = B, or len(cu_seqlens) - 1 for packed varlen input with B = 1).
+    Returns (out [B, T, H, dv] in q's dtype, S_final or None).  S_final may be S0 (in place)."""
+    lib = load_library()
+    _req(q, "q")
+    dev = q.device
+    dtq = q.dtype
+    if q.dim() != 4:
+        raise ValueError("q must be [B, T, H, dk]")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    _req(k, "k", dtq, dev)
+    _req(v, "v", dtq, dev)
+    _req(log_alpha, "log_alpha", torch.float32, dev)
+    _req(beta, "beta", torch.float32, dev)
+    if k.shape != q.shape or log_alpha.shape != q.shape or tuple(v.shape) != (B, T, H, dv) or \
+            tuple(beta.shape) != (B, T, H):
+        raise ValueError("inconsistent shapes")
+    N = B
+    if cu_seqlens is not None:
+        _req(cu_seqlens, "cu_seqlens", torch.int32, dev)
+        N = cu_seqlens.numel() - 1
+        if B != 1:
+            raise ValueError("packed varlen input needs B == 1")
+    if S0 is not None:
+        _req(S0, "S0", torch.float32, dev)
+        if tuple(S0.shape) != (N, H, dk, dv):
+            raise ValueError(f"S0 must be [{N}, {H}, {dk}, {dv}]")
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=dtq, device=dev)
+    else:
+        _req(out, "out", dtq, dev)
+    if S_final is None and output_final_state:
+        S_final = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
+    elif S_final is not None:
+        _req(S_final, "S_final", torch.float32, dev)
+    sh = _stream_handle(stream, dev)
+    ws_bytes = workspace_size(B, T, H, dk, dv, cu_seqlens is not None, N, dtq)
+    if workspace is None:
+        workspace = _get_workspace(ws_bytes, dev, sh)
+    else:
+        _req(workspace, "workspace", torch.uint8, dev)
+    rc = lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0), _ptr(cu_seqlens), N,
+                           _ptr(out), _ptr(S_final), B, T, H, dk, dv, _dt(q), _ptr(workspace), workspace.numel(), sh)
+    _check("kda_chunk_fwd", rc)
+    return out, S_final
+
+
+def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor, beta: torch.Tensor,
+                S: torch.Tensor, out: Optional[torch.Tensor] = None,
+                stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """One KDA decode step (``kda_decode_step``); ``S`` [N, H, dk, dv] fp32 is updated in place.
+    q, k, log_alpha: [N, H, dk]; v: [N, H, dv]; beta: [N, H].  Returns out [N, H, dv]."""
+    lib = load_library()
+    _req(q, "q")
+    dev, dtq = q.device, q.dtype
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    _req(k, "k", dtq, dev)
+    _req(v, "v", dtq, dev)
+    _req(log_alpha, "log_alpha", torch.float32, dev)
+    _req(beta, "beta", torch.float32, dev)
+    _req(S, "S", torch.float32, dev)
+    if k.shape != q.shape or log_alpha.shape != q.shape or tuple(v.shape) != (N, H, dv) or \
+            tuple(beta.shape) != (N, H) or tuple(S.shape) != (N, H, dk, dv):
+        raise ValueError("inconsistent shapes")
+    if out is None:
+        out = torch.empty((N, H, dv), dtype=dtq, device=dev)
+    else:
+        _req(out, "out", dtq, dev)
+    rc = lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S), _ptr(out), N, H, dk,
+                             dv, _dt(q), _stream_handle(stream, dev))
+    _check("kda_decode_step", rc)
+    return out
+
+
+def check(stream: Optional[torch.cuda.Stream] = None):
+    """Synchronise and raise if a kernel recorded a device-side error (``kda_check``)."""
+    lib = load_library()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    _check("kda_check", lib.kda_check(_stream_handle(stream, dev)))
+
+
+def profile_begin():
+    """Start recording per-launch device times of the library's kernels (``kda_profile_begin``)."""
+    _check("kda_profile_begin", load_library().kda_profile_begin())
+
+
+def profile_end() -> dict:
+    """Stop recording and return ``{kernel name: (launches, total device ms)}``."""
+    lib = load_library()
+    _check("kda_profile_end", lib.kda_profile_end())
+    cap = 64
+    names = (ctypes.c_char_p * cap)()
+    launches = (ctypes.c_int * cap)()
+    ms = (ctypes.c_double * cap)()
+    n = lib.kda_profile_kernels(cap, names, launches, ms)
+    if n < 0:
+        raise KdaError("kda_profile_kernels", 3)
+    return {names[i].decode(): (launches[i], ms[i]) for i in range(n)}
+
+
+def version() -> str:
+    return load_library().kda_version().decode()

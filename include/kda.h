@@ -1,0 +1,149 @@
+/*
+ * kda.h -- C ABI of libkda.so: the Kimi Delta Attention (KDA) operator on NVIDIA B200 (sm_100a).
+ *
+ * The operator (forward only).  Per sequence n and head h a state S of shape d_k x d_v
+ * (row = key channel, fp32) evolves over the tokens t of the sequence as
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,     o_t = S_t^T q_t
+ *
+ * with alpha_t = exp(log_alpha_t) a per-key-channel forget gate and beta_t a per-head scalar.
+ * Source: "Kimi Linear: redefining long-context inference efficiency" (xugj520.cn), section
+ * "Kimi Delta Attention的技术内核" (the recurrent-form update) and the 2025 attention/MoE review
+ * (lanjinlin.com.cn), entry "KLA 25.10 kimi" (the per-channel Diag(alpha_t) form and the
+ * readout o_t = S_t^T q_t).  No scaling of q is applied (callers pre-scale q if they want one).
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers, 16-byte aligned, contiguous, row-major.
+ *   - q, k, v, out use the element type `dt` (KDA_BF16 or KDA_F32); log_alpha, beta and every
+ *     state are fp32.  Accumulation is fp32.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream) and
+ *     never synchronise.  The caller owns every buffer.  The library allocates no device memory.
+ *   - Host-checkable argument errors return KDA_ERR_INVALID_ARG / KDA_ERR_UNSUPPORTED before
+ *     anything is launched.  A launch failure returns KDA_ERR_CUDA.  Errors found on the device
+ *     (a malformed cu_seqlens array, a bounded wait that gave up) are recorded in a device error
+ *     word and reported by kda_check().
+ *   - Thread safety: calls on different streams are independent; each call only touches the
+ *     buffers it is given (and the workspace it is given).
+ */
+#ifndef KDA_H
+#define KDA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;                         /* = cudaStream_t */
+typedef struct CUstream_st* kda_stream_t;
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size, inconsistent arguments    */
+    KDA_ERR_UNSUPPORTED = 2,   /* valid but not implemented here (e.g. d_k not in {64, 128})    */
+    KDA_ERR_CUDA = 3,          /* a CUDA runtime call or kernel launch failed                  */
+    KDA_ERR_TIMEOUT = 4,       /* a bounded device-side wait gave up (reported by kda_check)   */
+    KDA_ERR_WORKSPACE = 5,     /* workspace pointer NULL/misaligned or smaller than required  */
+    KDA_ERR_BAD_SEQLENS = 6    /* cu_seqlens not 0 = c0 <= c1 <= ... <= cN = T (device check)  */
+} kda_status;
+
+typedef enum {
+    KDA_BF16 = 0,              /* q, k, v, out are bf16 */
+    KDA_F32 = 1                /* q, k, v, out are fp32 */
+} kda_dtype;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* kda_status_string(kda_status s);
+
+/* Library version string, e.g. "kda-b200 0.1 sm_100a". */
+const char* kda_version(void);
+
+/*
+ * kda_chunk_fwd_workspace_size -- bytes of device workspace kda_chunk_fwd needs.
+ *
+ * Same shape arguments as kda_chunk_fwd (`num_seqs` is used only when `varlen` is nonzero).
+ * The bound holds for every cu_seqlens with the given total T and num_seqs.  Writes the size to
+ * *bytes.  Returns KDA_ERR_INVALID_ARG / KDA_ERR_UNSUPPORTED for arguments kda_chunk_fwd would
+ * reject.
+ */
+kda_status kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int varlen, int num_seqs,
+                                        kda_dtype dt, size_t* bytes);
+
+/*
+ * kda_chunk_fwd -- chunked-parallel prefill (chunk size 64).
+ *
+ * The algorithm is the chunk form of the recurrence: inside each 64-token chunk the cumulative
+ * log-gate g_r = sum_{i<=r} log_alpha_i is restarted, the chunk's rank-1 updates are packed into
+ * a WY representation through the UT transform T = (I + strict_lower(diag(beta) (k*e^g)(k*e^-g)^T))^-1
+ * diag(beta), the intra-chunk products are dense tensor-core GEMMs, and the state is carried
+ * from chunk to chunk ("Kimi Linear" explainer, section "硬件效率的深度优化": chunked parallel
+ * computation, WY representation, UT transform; chunk size 64 as in the coreui.cn article,
+ * section 2.2 "硬件感知的块状计算").  The result equals the token-by-token recurrence up to
+ * rounding.
+ *
+ * Layout (token-major):
+ *   q, k       [B, T, H, dk]  dt
+ *   v          [B, T, H, dv]  dt
+ *   log_alpha  [B, T, H, dk]  fp32   (log of the forget gate, <= 0 expected; any finite value works)
+ *   beta       [B, T, H]      fp32
+ *   S0         [N, H, dk, dv] fp32 or NULL (= zero state)                  N = B, or num_seqs
+ *   out        [B, T, H, dv]  dt     (written)
+ *   S_final    [N, H, dk, dv] fp32 or NULL (not written); may alias S0 (in-place state passing)
+ * Varlen: if cu_seqlens (DEVICE int32 [num_seqs+1]) is non-NULL, B must be 1, the T tokens are
+ *   num_seqs packed sequences, sequence n = tokens cu_seqlens[n] .. cu_seqlens[n+1]-1, with its
+ *   own S0[n] / S_final[n].  Chunks restart at every sequence boundary.  A malformed array is
+ *   detected on the device: nothing is computed, out/S_final are left untouched, and
+ *   kda_check() returns KDA_ERR_BAD_SEQLENS.
+ * Supported: dk, dv in {64, 128}; dt in {KDA_BF16, KDA_F32}; T >= 0 (T = 0 copies S0 to S_final).
+ * Workspace: device memory of at least kda_chunk_fwd_workspace_size() bytes, 256-byte aligned,
+ *   owned by the caller, contents irrelevant on entry; it must not be used by another call that
+ *   runs concurrently.
+ */
+kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const float* log_alpha, const float* beta,
+                         const float* S0, const int32_t* cu_seqlens, int num_seqs, void* out, float* S_final,
+                         int B, int T, int H, int dk, int dv, kda_dtype dt, void* workspace,
+                         size_t workspace_bytes, kda_stream_t stream);
+
+/*
+ * kda_decode_step -- one token for each of N independent sequences, state updated in place.
+ *
+ * Follows the per-token loop of the attention review's GDN/KDA pseudo-code (lanjinlin.com.cn,
+ * the block that starts from the loaded per-sequence state): (a) decay S' = Diag(alpha) S,
+ * (b) value modification u = beta (v - S'^T k), (c) rank-1 update S = S' + k u^T, (d) output from
+ * the UPDATED state o = S^T q.  One read and one write of the state per call.
+ *
+ * Layout:
+ *   q, k, log_alpha [N, H, dk] (q, k: dt; log_alpha: fp32);  v [N, H, dv] dt;  beta [N, H] fp32;
+ *   S_inout [N, H, dk, dv] fp32 (read, then overwritten with the new state);  out [N, H, dv] dt.
+ * Supported: dk, dv in {64, 128}; N >= 0 (N = 0 is a no-op).
+ */
+kda_status kda_decode_step(const void* q, const void* k, const void* v, const float* log_alpha, const float* beta,
+                           float* S_inout, void* out, int N, int H, int dk, int dv, kda_dtype dt,
+                           kda_stream_t stream);
+
+/*
+ * kda_check -- synchronise `stream`, then read and clear the device error word of the current
+ * device.  Returns KDA_OK, KDA_ERR_CUDA (a sticky CUDA error), KDA_ERR_BAD_SEQLENS or
+ * KDA_ERR_TIMEOUT.
+ */
+kda_status kda_check(kda_stream_t stream);
+
+/*
+ * Per-launch timing, for benchmarks and profiles (not part of the operator).  Between
+ * kda_profile_begin() and kda_profile_end() every kernel the library launches is bracketed by two
+ * CUDA events recorded on the launch's own stream.  kda_profile_kernels() waits for the recorded
+ * events and fills, for up to `max_kernels` distinct kernels, a static name (valid for the life of
+ * the library), the number of launches and their summed device time in milliseconds; it returns
+ * the number of distinct kernels, or -1 if a buffer is too small or an event query failed.
+ * Recording is off by default and costs two event records per launch when on.
+ */
+kda_status kda_profile_begin(void);
+kda_status kda_profile_end(void);
+int kda_profile_kernels(int max_kernels, const char** names, int* launches, double* total_ms);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H */

@@ -1,0 +1,123 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every function that
+include/kda.h declares, and rejects bad arguments before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from gated_delta_rule_83_b200 import build, kda
+    build.build()
+    return kda.load_library()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "kda.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\**\s+\**(kda_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    for required in ("kda_chunk_fwd", "kda_decode_step", "kda_chunk_fwd_workspace_size", "kda_check",
+                     "kda_status_string", "kda_version"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"libkda.so does not export {name}"
+
+
+def test_binding_covers_the_abi():
+    from gated_delta_rule_83_b200 import kda
+    assert set(declared_functions()) <= set(kda.ABI)
+
+
+def test_status_strings(lib):
+    for code, name in [(0, b"KDA_OK"), (1, b"KDA_ERR_INVALID_ARG"), (2, b"KDA_ERR_UNSUPPORTED"),
+                       (5, b"KDA_ERR_WORKSPACE"), (6, b"KDA_ERR_BAD_SEQLENS")]:
+        assert lib.kda_status_string(code) == name
+    assert lib.kda_status_string(99) == b"KDA_ERR_UNKNOWN"
+    assert b"sm_100a" in lib.kda_version()
+
+
+def _ws(lib, *args):
+    n = ctypes.c_size_t(0)
+    rc = lib.kda_chunk_fwd_workspace_size(*args, ctypes.byref(n))
+    return rc, n.value
+
+
+def test_workspace_size_rules(lib):
+    rc, n = _ws(lib, 1, 32768, 32, 128, 128, 0, 0, 0)
+    assert rc == 0 and n > 0
+    rc2, n2 = _ws(lib, 1, 65536, 32, 128, 128, 1, 8, 0)   # varlen: bound grows with num_seqs
+    assert rc2 == 0 and n2 >= 2 * n - 4096
+    assert _ws(lib, 1, 256, 2, 96, 64, 0, 0, 0)[0] == 2    # dk unsupported
+    assert _ws(lib, 2, 256, 2, 64, 64, 1, 2, 0)[0] == 1    # varlen needs B == 1
+    assert _ws(lib, 1, -1, 2, 64, 64, 0, 0, 0)[0] == 1
+    assert _ws(lib, 1, 256, 2, 64, 64, 0, 0, 7)[0] == 1    # bad dtype
+    assert _ws(lib, 1, 0, 2, 64, 64, 0, 0, 1)[0] == 0      # T = 0 is valid
+
+
+def test_chunk_fwd_rejects_before_launch(lib):
+    fake = 0x100000  # never dereferenced: every call below fails validation first
+    # null inputs
+    rc = lib.kda_chunk_fwd(None, None, None, None, None, None, None, 0, None, None, 1, 64, 2, 64, 64, 1,
+                           fake, 1 << 30, None)
+    assert rc == 1
+    # misaligned pointer
+    rc = lib.kda_chunk_fwd(fake + 2, fake, fake, fake, fake, None, None, 0, fake, None, 1, 64, 2, 64, 64, 1,
+                           fake, 1 << 30, None)
+    assert rc == 1
+    # workspace missing / too small / misaligned
+    args = (fake, fake, fake, fake, fake, None, None, 0, fake, None, 1, 64, 2, 64, 64, 1)
+    assert lib.kda_chunk_fwd(*args, None, 1 << 30, None) == 5
+    assert lib.kda_chunk_fwd(*args, fake, 16, None) == 5
+    assert lib.kda_chunk_fwd(*args, fake + 16, 1 << 30, None) == 5
+    # unsupported head dims
+    assert lib.kda_chunk_fwd(fake, fake, fake, fake, fake, None, None, 0, fake, None, 1, 64, 2, 32, 64, 1,
+                             fake, 1 << 30, None) == 2
+
+
+def test_decode_rejects_before_launch(lib):
+    fake = 0x100000
+    assert lib.kda_decode_step(None, fake, fake, fake, fake, fake, fake, 4, 2, 64, 64, 0, None) == 1
+    assert lib.kda_decode_step(fake, fake, fake, fake, fake, fake, fake, 4, 2, 48, 64, 0, None) == 2
+    assert lib.kda_decode_step(fake, fake, fake, fake, fake, fake + 4, fake, 4, 2, 64, 64, 0, None) == 1
+    assert lib.kda_decode_step(fake, fake, fake, fake, fake, fake, fake, 4, 2, 64, 64, 3, None) == 1
+    # N = 0 is a no-op that touches nothing
+    assert lib.kda_decode_step(None, None, None, None, None, None, None, 0, 2, 64, 64, 0, None) == 0
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    from gated_delta_rule_83_b200 import kda
+    with pytest.raises(ImportError):
+        kda.load_library(str(tmp_path / "libkda.so"))
+
+
+def test_synth_distributions():
+    """The seeded generator matches the documented distributions (host-side, small sizes)."""
+    import numpy as np
+    import torch
+    from gated_delta_rule_83_b200 import synth
+    w = synth.WORKLOADS["prefill_32k"]
+    inp = synth.prefill_inputs(w, T=512, H=4)
+    k = inp["k"].float()
+    assert torch.allclose(k.norm(dim=-1), torch.ones(()), atol=1e-2)
+    la = inp["log_alpha"].double()
+    assert float(la.max()) < 0 and abs(float(la.mean()) - (-0.07)) < 0.03
+    b = inp["beta"]
+    assert 0 < float(b.min()) and float(b.max()) < 1 and abs(float(b.mean()) - 0.5) < 0.05
+    assert abs(float(inp["S0"].std()) - 0.02) < 0.002
+    lens = synth.varlen_lengths(2)
+    assert len(lens) == 8 and sum(lens) == 65536 and all(1024 <= x <= 16384 for x in lens)
+    assert lens == synth.varlen_lengths(2)
+    # same seed -> same bits
+    inp2 = synth.prefill_inputs(w, T=512, H=4)
+    assert torch.equal(inp["q"], inp2["q"]) and torch.equal(inp["log_alpha"], inp2["log_alpha"])

@@ -44,6 +44,9 @@ def parse():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target duration of the oracle sample")
+    ap.add_argument("--only", choices=["prefill", "decode"], default=None,
+                    help="run one part only (for profiling): no JSON contract line, prints that part's numbers")
+    ap.add_argument("--decode-steps", type=int, default=None, help="decode steps to time (default 512)")
     return ap.parse_args()
 
 
@@ -206,6 +209,12 @@ def run_ours(args):
     w = synth.WORKLOADS[args.workload]
     if w.kind != "prefill":
         raise SystemExit("the headline workload is a prefill workload; decode is reported under 'decode'")
+    if args.only == "decode":
+        stream = torch.cuda.current_stream(dev)
+        d = bench_decode(torch, kda, synth, dev, stream, world, rank, hbm, peak_kind, steps=args.decode_steps)
+        if rank == 0:
+            print(json.dumps(d), flush=True)
+        return
 
     inp = synth.prefill_inputs(w, device=dev, seed=w.seed + 1000 * rank)
     q, k, v, la, beta, S0, cu = (inp[x] for x in ("q", "k", "v", "log_alpha", "beta", "S0", "cu_seqlens"))
@@ -265,6 +274,8 @@ def run_ours(args):
     # e2e: host buffers through the public API
     e2e = None
     try:
+        if args.only is not None:
+            raise RuntimeError("skipped (--only)")
         hq, hk, hv, hla, hb = (x.cpu().pin_memory() for x in (q, k, v, la, beta))
         hS0 = S0.cpu().pin_memory() if S0 is not None else None
         hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
@@ -306,11 +317,11 @@ def run_ours(args):
     torch.cuda.empty_cache()
 
     decode = None
-    if not args.no_decode:
-        decode = bench_decode(torch, kda, synth, dev, stream, world, rank, hbm, peak_kind)
+    if not args.no_decode and args.only is None:
+        decode = bench_decode(torch, kda, synth, dev, stream, world, rank, hbm, peak_kind, steps=args.decode_steps)
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.only is None:
         cpu = cpu_oracle_prefill(w, args.cpu_seconds)
 
     line = {"metric": "KDA prefill tokens/s (decode tokens/s under 'decode')", "value": value, "unit": "tokens/s",

@@ -211,3 +211,56 @@ kda_status kda_check(kda_stream_t stream_)
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------------------------
+// Allocation-free variant of kda_chunk_fwd (declared in include/kda.h).
+//
+// For hosts that cannot allocate device memory at call time (engines that reserve all memory in
+// their own pool up front, plugin hooks that forbid cudaMalloc, fixed memory budgets), the
+// workspace comes from a static device array compiled into this file instead of from the caller.
+// The array exists once per GPU that loads the library and lives until the process exits.  In
+// host code its name is only a host-side stand-in, so its device address is looked up (once per
+// device, with that device current) with cudaGetSymbolAddress and passed to the kernels like any
+// other workspace pointer.  All calls on a device share the array; calls that overlap on the GPU
+// race.  Every scratch byte a kernel reads is written earlier in the same call, so nothing needs
+// clearing between calls.
+// ------------------------------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_noalloc_scratch[KDA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kNoallocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kNoallocMaxDevices] = {};
+
+kda_status noalloc_scratch_address(void** ptr)
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoallocMaxDevices) return KDA_ERR_CUDA;
+    std::lock_guard<std::mutex> g(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return KDA_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *ptr = g_noalloc_ptr[dev];
+    return KDA_OK;
+}
+
+}  // namespace
+
+extern "C" kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const float* log_alpha,
+                                            const float* beta, const float* S0, const int32_t* cu_seqlens,
+                                            int num_seqs, void* out, float* S_final, int B, int T, int H, int dk,
+                                            int dv, kda_dtype dt, kda_stream_t stream)
+{
+    Plan p;
+    const kda_status st = make_plan(B, T, H, dk, dv, cu_seqlens != nullptr, num_seqs, dt, p);
+    if (st != KDA_OK) return st;
+    if (p.total_bytes > (size_t)KDA_NOALLOC_SCRATCH_BYTES) return KDA_ERR_WORKSPACE;
+    void* scratch = nullptr;
+    const kda_status sa = noalloc_scratch_address(&scratch);
+    if (sa != KDA_OK) return sa;
+    return kda_chunk_fwd(q, k, v, log_alpha, beta, S0, cu_seqlens, num_seqs, out, S_final, B, T, H, dk, dv, dt,
+                         scratch, (size_t)KDA_NOALLOC_SCRATCH_BYTES, stream);
+}

@@ -28,6 +28,7 @@ ABI = {
     "kda_chunk_fwd_workspace_size": (_I, [_I, _I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_SZ)]),
     "kda_chunk_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _I, _P, _SZ, _P]),
     "kda_decode_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "kda_chunk_fwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
     "kda_check": (_I, [_P]),
     "kda_profile_begin": (_I, []),
     "kda_profile_end": (_I, []),
@@ -171,6 +172,29 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torc
                            _ptr(out), _ptr(S_final), B, T, H, dk, dv, _dt(q), _ptr(workspace), workspace.numel(), sh)
     _check("kda_chunk_fwd", rc)
     return out, S_final
+
+
+NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024  # KDA_NOALLOC_SCRATCH_BYTES in include/kda.h
+
+
+def chunk_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor,
+                      beta: torch.Tensor, S0: torch.Tensor, out: torch.Tensor, S_final: Optional[torch.Tensor],
+                      cu_seqlens: Optional[torch.Tensor] = None,
+                      stream: Optional[torch.cuda.Stream] = None) -> None:
+    """``kda_chunk_fwd_noalloc``: the chunked prefill for callers that cannot allocate device memory
+    (the library's built-in scratch replaces the workspace).  Every buffer, ``out`` and ``S_final``
+    included, is the caller's; nothing is allocated here either.  Problems whose workspace would
+    exceed ``NOALLOC_SCRATCH_BYTES`` raise ``KdaError`` (KDA_ERR_WORKSPACE)."""
+    lib = load_library()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    N = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    for t, name in ((q, "q"), (k, "k"), (v, "v"), (log_alpha, "log_alpha"), (beta, "beta"), (out, "out")):
+        _req(t, name)
+    rc = lib.kda_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0),
+                                   _ptr(cu_seqlens), N, _ptr(out), _ptr(S_final), B, T, H, dk, dv, _dt(q),
+                                   _stream_handle(stream, q.device))
+    _check("kda_chunk_fwd_noalloc", rc)
 
 
 def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor, beta: torch.Tensor,

@@ -130,6 +130,34 @@ kda_status kda_decode_step(const void* q, const void* k, const void* v, const fl
 kda_status kda_check(kda_stream_t stream);
 
 /*
+ * kda_chunk_fwd_noalloc -- kda_chunk_fwd for callers that cannot allocate device memory.
+ *
+ * The pages describe no counterpart: this is a deployment convenience of this library.  Some
+ * hosts of this operator cannot hand it a workspace: an engine whose device memory is fully
+ * reserved up front by its own pool, a plugin whose enqueue hook may not call cudaMalloc, or a
+ * runtime with a fixed, audited memory budget.  This entry point takes the same arguments as
+ * kda_chunk_fwd minus the workspace and uses instead a scratch array compiled into the library:
+ * KDA_NOALLOC_SCRATCH_BYTES bytes of static device memory on every GPU that loads the library,
+ * held until the process exits.  It calls no cudaMalloc, cudaFree or allocating library routine.
+ *   - Limit: a problem whose kda_chunk_fwd_workspace_size() exceeds KDA_NOALLOC_SCRATCH_BYTES is
+ *     rejected with KDA_ERR_WORKSPACE before anything is launched.  With bf16, dk = dv = 128 and
+ *     H = 32 that is a few thousand tokens per call; longer inputs can be fed in pieces, passing
+ *     S_final of one call as S0 of the next.
+ *   - The first call on a device looks up the array's device address on that device (make that
+ *     device current first); make this first call before any stream capture.
+ *   - All calls on a device share the one array: calls that overlap on the GPU (e.g. on two
+ *     streams at once) race and corrupt each other's results.  Serialise them.  The kernels
+ *     rewrite every scratch byte they read within the same call, so nothing has to start zeroed
+ *     and stale contents from an earlier call are harmless.
+ * Returns the same codes as kda_chunk_fwd.
+ */
+#define KDA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const float* log_alpha,
+                                 const float* beta, const float* S0, const int32_t* cu_seqlens, int num_seqs,
+                                 void* out, float* S_final, int B, int T, int H, int dk, int dv, kda_dtype dt,
+                                 kda_stream_t stream);
+
+/*
  * Per-launch timing, for benchmarks and profiles (not part of the operator).  Between
  * kda_profile_begin() and kda_profile_end() every kernel the library launches is bracketed by two
  * CUDA events recorded on the launch's own stream.  kda_profile_kernels() waits for the recorded

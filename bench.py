@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--only", choices=["prefill", "decode"], default=None,
                     help="run one part only (for profiling): no JSON contract line, prints that part's numbers")
     ap.add_argument("--decode-steps", type=int, default=None, help="decode steps to time (default 512)")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override the prefill sequence length (profiling of a smaller case only)")
     return ap.parse_args()
 
 
@@ -216,7 +218,7 @@ def run_ours(args):
             print(json.dumps(d), flush=True)
         return
 
-    inp = synth.prefill_inputs(w, device=dev, seed=w.seed + 1000 * rank)
+    inp = synth.prefill_inputs(w, device=dev, seed=w.seed + 1000 * rank, T=args.tokens)
     q, k, v, la, beta, S0, cu = (inp[x] for x in ("q", "k", "v", "log_alpha", "beta", "S0", "cu_seqlens"))
     B, T, H, dk = q.shape
     dv = v.shape[-1]

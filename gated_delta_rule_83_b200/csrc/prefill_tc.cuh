@@ -2,28 +2,30 @@
 //
 // The chunk form of the recurrence ("Kimi Linear" explainer, section "硬件效率的深度优化":
 // chunk-parallel work inside a chunk, recurrent state passing between chunks, WY representation,
-// UT transform; chunk size 64), split into two kernels:
+// UT transform; chunk size 64), split into two kernels.
 //
-// Phase A, one CTA per (chunk, head), every chunk in parallel (128 threads, thread c = channel c):
+// Phase A, one CTA per (chunk, head), all chunks in parallel (256 threads):
 //   g_r = sum_{i<=r} log_alpha_i (fp32, restarted every chunk); ref_c = centre of channel c's range
 //   Kf = k e^{g-ref}, Qf = q e^{g-ref}, Kb = k e^{ref-g}   (bf16 operands; every factor <= e^80)
-//   A' = Kf Kb^T, P' = Qf Kb^T                       tcgen05, M=64 N=64 K=128, fp32 in TMEM
-//   A = strict_lower(diag(beta) A'), P = lower_incl(P')     (= the exact e^{g_r - g_i} products)
-//   T = (I + A)^{-1} diag(beta)                      fp32 blocked triangular inverse (UT transform)
-//   W = T (k e^g), Uv = T v                          tcgen05, M=64 N=128 K=64 (B operands MN-major)
-//   writes bf16 operand images of W, Qg = q e^g, Kd^T = (k e^{g_last-g})^T, P, Uv and fp32 e^{g_last}
-//   to the workspace, already in the swizzled shared-memory layout phase B consumes.
+//   A' = Kf Kb^T, P' = Qf Kb^T                          tcgen05 M=64 N=64 K=128, fp32 in TMEM
+//   A = strict_lower(diag(beta) A'), P = lower_incl(P')        (= the exact e^{g_r - g_i} products)
+//   T = (I + A)^{-1} diag(beta)                         fp32 recursive-doubling triangular inverse
+//   [W' | Uv] = T [Kf | v], W = W' diag(e^ref)         tcgen05 M=64 N=256 K=64 (B operand MN-major)
+//   [P W | P Uv] = P [W | Uv]                           tcgen05 M=64 N=256 K=64
+//   Q' = q e^g - P W,  O0 = P Uv                        (the intra-chunk part of the output, folded in)
+//   writes bf16 operand images -- [W; Q'] stacked (128 rows), Kd = k e^{g_last-g}, Uv, O0 -- and fp32
+//   e^{g_last} to the workspace, already in the swizzled shared-memory layout phase B consumes.
 //   A chunk in which some channel's gate spreads over more than e^160 (far outside any trained
 //   gate) computes A and P with exact per-element factors on CUDA cores instead.
 //
-// Phase B, one CTA per (sequence, head, 32-column slice of S), chunks in order (128 threads):
-//   a 3-stage bulk-copy (cp.async.bulk) pipeline streams each chunk's operand images into shared
-//   memory; per chunk
-//     X = W S, O = Qg S                 tcgen05 M=64 N=32 K=128
-//     U = Uv - X  (-> bf16 U^T tile)
-//     O += P U, Y = Kd^T U              tcgen05 M=64/128 N=32 K=64
+// Phase B, one CTA per (sequence, head, 32-column slice of S), chunks in order.  Warp roles: four
+// compute warps, one MMA-issue warp, one bulk-copy warp.  A 3-stage cp.async.bulk pipeline streams
+// each chunk's images into shared memory; per chunk
+//     [X; O'] = [W; Q'] S               tcgen05 M=128 N=32 K=128   (one 8-instruction batch)
+//     U = Uv - X  (-> bf16 U tile)      out = O' + O0  (off the critical path)
+//     Y = Kd^T U                        tcgen05 M=128 N=32 K=64
 //     S <- Diag(e^{g_last}) S + Y       fp32 in registers (thread c owns row c of the slice)
-//   out = O (bf16), S_final = S (fp32).
+// which equals O = Qg S + P U with U = Uv - W S, the chunk form of o_t = S_t^T q_t.
 #pragma once
 
 #include "common.cuh"
@@ -35,88 +37,143 @@ namespace kda {
 constexpr bool kTcPathReady = true;
 
 // ---- workspace slot of one (chunk, head), bytes ------------------------------------------------
-constexpr uint32_t kSlotW = 0;          // W    [64 x 128] bf16, SW128 tile (2 atom columns)
-constexpr uint32_t kSlotQ = 16384;      // Qg   [64 x 128] bf16, SW128 tile
-constexpr uint32_t kSlotKd = 32768;     // Kd^T [128 x 64] bf16, SW128 tile
-constexpr uint32_t kSlotP = 49152;      // P    [64 x 64]  bf16, SW128 tile
-constexpr uint32_t kSlotUv = 57344;     // Uv   [4 slices][64][32] bf16, plain row-major
-constexpr uint32_t kSlotGam = 73728;    // e^{g_last} [128] fp32
-constexpr uint32_t kSlotBytes = 74240;
+constexpr uint32_t kSlotWQ = 0;         // [W; Q'] [128 x 128] bf16, SW128 tile (2 atom columns of 16 KB)
+constexpr uint32_t kSlotKd = 32768;     // Kd      [64 x 128]  bf16, SW128 tile (MN-major A operand of Kd^T U)
+constexpr uint32_t kSlotUv = 49152;     // Uv      [4 slices][64][32] bf16, slice layout (slice_chunk_off)
+constexpr uint32_t kSlotO0 = 65536;     // O0      [4 slices][64][32] bf16, slice layout (slice_chunk_off)
+constexpr uint32_t kSlotGam = 81920;    // e^{g_last} [128] fp32
+constexpr uint32_t kSlotBytes = 82432;
 inline size_t tc_slot_bytes() { return kSlotBytes; }
 
 constexpr int kTcNV = 32;               // state columns per phase-B CTA
 
+// Slice images ([64 rows][32 columns] bf16, 64-byte rows): 16-byte chunk m of row r is stored at
+// chunk position m ^ ((r >> 1) & 3), so eight consecutive rows read chunk by chunk hit distinct banks.
+__host__ __device__ __forceinline__ uint32_t slice_chunk_off(int r, int m) { return (uint32_t)(r * 64 + ((m ^ ((r >> 1) & 3)) << 4)); }
 constexpr float kTcFactorSpread = 160.f;
 
 // ------------------------------------------------------------------------------------------------
 // small device helpers
 // ------------------------------------------------------------------------------------------------
 __device__ __forceinline__ float lds_bf16(const uint8_t* p) { return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(p)); }
-__device__ __forceinline__ void sts_bf16(uint8_t* p, float x) { *reinterpret_cast<__nv_bfloat16*>(p) = __float2bfloat16_rn(x); }
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes)
 {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, uint32_t src_bytes)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
 __device__ __forceinline__ void cp_async_wait_all()
 {
     asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
-
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p)
 {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
+__device__ __forceinline__ void unpack8(const uint4& raw, float* f)
+{
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const float2 t = __bfloat1622float2(h[m]);
+        f[2 * m] = t.x;
+        f[2 * m + 1] = t.y;
+    }
+}
+__device__ __forceinline__ uint4 pack8(const float* f)
+{
+    return make_uint4(tc::pack_bf16(f[0], f[1]), tc::pack_bf16(f[2], f[3]), tc::pack_bf16(f[4], f[5]),
+                      tc::pack_bf16(f[6], f[7]));
+}
+__device__ __forceinline__ void named_sync(int id, int threads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+__device__ __forceinline__ void named_arrive(int id, int threads)
+{
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
 
 // ------------------------------------------------------------------------------------------------
-// UT transform: X = (I + A)^{-1} for a strictly lower 64 x 64 A (fp32, row stride 65), by 16 x 16
-// blocks: the diagonal blocks by forward substitution, then block row by block row
-// X_ij = -X_ii sum_{k=j}^{i-1} A_ik X_kj.  128 threads.  Y is 3 x 16 x 17 floats of scratch.
+// UT transform: X = (I + A)^{-1} for a strictly lower 64 x 64 A (fp32, row stride 68) by recursive
+// doubling: the four 16 x 16 diagonal blocks by forward substitution; then, inside each 32 x 32 half,
+// X_10 = -X_11 A_10 X_00; then the 32 x 32 off-diagonal block X_10 = -X_11 A_10 X_00 of the whole.
+// 256 threads.  X: row stride 64.  Y: scratch of 32 x 33 floats.
 // ------------------------------------------------------------------------------------------------
-constexpr int kTS = 65;  // row stride of A and X
+constexpr int kAS = 68;  // row stride of A
+constexpr int kXS = 64;  // row stride of X
 
 __device__ __forceinline__ void ut_inverse_64(const float* __restrict__ sA, float* __restrict__ sX, float* __restrict__ sY)
 {
     const int tid = threadIdx.x;
-    // zero X (upper blocks stay zero)
-    for (int e = tid; e < 64 * kTS; e += 128) sX[e] = 0.f;
+    // upper triangle blocks of X are zero
+    for (int e = tid; e < 64 * 64 / 4; e += 256) reinterpret_cast<float4*>(sX)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
     __syncthreads();
-    // diagonal blocks: warp kb inverts block kb, lane jj < 16 owns column jj
-    {
-        const int kb = tid >> 5, jj = tid & 31;
-        if (jj < 16) {
-            const int b = 16 * kb;
-            float x[16];
+    if (tid < 64) {  // diagonal 16 x 16 blocks: thread -> (block, column jj)
+        const int b = 16 * (tid >> 4), jj = tid & 15;
+        float x[16];
 #pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                float s = 0.f;
+        for (int r = 0; r < 16; ++r) {
+            float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-                for (int i = 0; i < r; ++i) s = fmaf(sA[(b + r) * kTS + b + i], x[i], s);
-                x[r] = (r == jj) ? 1.f : ((r < jj) ? 0.f : -s);
+            for (int i = 0; i + 1 < r; i += 2) {
+                s0 = fmaf(sA[(b + r) * kAS + b + i], x[i], s0);
+                s1 = fmaf(sA[(b + r) * kAS + b + i + 1], x[i + 1], s1);
             }
-#pragma unroll
-            for (int r = 0; r < 16; ++r) sX[(b + r) * kTS + b + jj] = x[r];
+            if (r & 1) s0 = fmaf(sA[(b + r) * kAS + b + r - 1], x[r - 1], s0);
+            x[r] = (r == jj) ? 1.f : ((r < jj) ? 0.f : -(s0 + s1));
         }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) sX[(b + r) * kXS + b + jj] = x[r];
     }
     __syncthreads();
-    // block rows 1..3
-    for (int bi = 1; bi < 4; ++bi) {
-        // Y_j = sum_{k=j}^{bi-1} A_{bi,k} X_{k,j}, for j = 0..bi-1 (bi blocks of 16 x 16)
-        for (int e = tid; e < bi * 256; e += 128) {
-            const int bj = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
-            float s = 0.f;
-            for (int kk = 16 * bj; kk < 16 * bi; ++kk) s = fmaf(sA[(16 * bi + rr) * kTS + kk], sX[kk * kTS + 16 * bj + cc], s);
-            sY[(bj * 16 + rr) * 17 + cc] = s;
-        }
-        __syncthreads();
-        // X_{bi,j} = -X_{bi,bi} Y_j
-        for (int e = tid; e < bi * 256; e += 128) {
-            const int bj = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
-            float s = 0.f;
+    {   // level 1: blocks (1,0) and (3,2); thread -> (pair p, row rr, columns cc, cc+1)
+        const int p = tid >> 7, rr = (tid >> 3) & 15, cc = (tid & 7) * 2;
+        const int bi = 16 * (2 * p + 1), bj = 16 * (2 * p);
+        float y0 = 0.f, y1 = 0.f;
 #pragma unroll
-            for (int kk = 0; kk < 16; ++kk) s = fmaf(sX[(16 * bi + rr) * kTS + 16 * bi + kk], sY[(bj * 16 + kk) * 17 + cc], s);
-            sX[(16 * bi + rr) * kTS + 16 * bj + cc] = -s;
+        for (int k = 0; k < 16; ++k) {
+            const float a = sA[(bi + rr) * kAS + bj + k];
+            y0 = fmaf(a, sX[(bj + k) * kXS + bj + cc], y0);
+            y1 = fmaf(a, sX[(bj + k) * kXS + bj + cc + 1], y1);
         }
+        sY[(p * 16 + rr) * 33 + cc] = y0;
+        sY[(p * 16 + rr) * 33 + cc + 1] = y1;
+        __syncthreads();
+        float x0 = 0.f, x1 = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const float xi = sX[(bi + rr) * kXS + bi + k];
+            x0 = fmaf(xi, sY[(p * 16 + k) * 33 + cc], x0);
+            x1 = fmaf(xi, sY[(p * 16 + k) * 33 + cc + 1], x1);
+        }
+        sX[(bi + rr) * kXS + bj + cc] = -x0;
+        sX[(bi + rr) * kXS + bj + cc + 1] = -x1;
+        __syncthreads();
+    }
+    {   // level 2: rows 32..63, columns 0..31; thread -> (row rr, columns cc..cc+3)
+        const int rr = tid >> 3, cc = (tid & 7) * 4;
+        float y[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+            const float a = sA[(32 + rr) * kAS + k];
+            const float4 xv = *reinterpret_cast<const float4*>(sX + k * kXS + cc);
+            y[0] = fmaf(a, xv.x, y[0]); y[1] = fmaf(a, xv.y, y[1]); y[2] = fmaf(a, xv.z, y[2]); y[3] = fmaf(a, xv.w, y[3]);
+        }
+#pragma unroll
+        for (int m = 0; m < 4; ++m) sY[rr * 33 + cc + m] = y[m];
+        __syncthreads();
+        float x[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+            const float xi = sX[(32 + rr) * kXS + 32 + k];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) x[m] = fmaf(xi, sY[k * 33 + cc + m], x[m]);
+        }
+        *reinterpret_cast<float4*>(sX + (32 + rr) * kXS + cc) = make_float4(-x[0], -x[1], -x[2], -x[3]);
         __syncthreads();
     }
 }
@@ -124,17 +181,17 @@ __device__ __forceinline__ void ut_inverse_64(const float* __restrict__ sA, floa
 // ------------------------------------------------------------------------------------------------
 // Phase A
 // ------------------------------------------------------------------------------------------------
-constexpr int kAThreads = 128;
-constexpr uint32_t kA_K = 0;        // Kf (raw k on load)                       16 KB
-constexpr uint32_t kA_Q = 16384;    // Qf (raw q on load)                       16 KB
-constexpr uint32_t kA_Kb = 32768;   // Kb; later T (bf16, 8 KB); wide case: g rows 0..31
-constexpr uint32_t kA_Kt = 49152;   // k e^g (B operand of W); wide case: g rows 32..63
-constexpr uint32_t kA_V = 65536;    // v                                        16 KB
-constexpr uint32_t kA_A = 81920;    // A fp32 [64][65]                          16640 B
-constexpr uint32_t kA_Y = 98560;    // solve scratch 3 x 16 x 17 fp32           3264 B
-constexpr uint32_t kA_Misc = 101888;// beta[64] ref[128] E[128] D[128] + tmem addr, flag, mbarrier
-constexpr uint32_t kA_Smem = kA_Misc + 2048 + 1024;  // + 1024 for aligning the dynamic base
-// X = (I+A)^{-1}, fp32 [64][65], overlays Kf/Qf (dead by then)
+constexpr int kAThreads = 256;
+constexpr uint32_t kA_K = 0;         // k -> Kf (wide: k e^g) -> W bf16 tile           16 KB  } B operand of
+constexpr uint32_t kA_V = 16384;     // v                  -> Uv bf16 tile             16 KB  } P [W | Uv]
+constexpr uint32_t kA_Q = 32768;     // q -> Qf (wide: q e^g)                          16 KB
+constexpr uint32_t kA_Kb = 49152;    // Kb -> X fp32 [64][64] -> T bf16 [64][64]       16 KB
+constexpr uint32_t kA_G = 65536;     // log_alpha -> g fp32 [64][132] -> A fp32 [64][68] + scratch + P tile
+constexpr uint32_t kA_Ysc = kA_G + 17408;   // solve scratch 32 x 33 fp32
+constexpr uint32_t kA_P = kA_G + 22528;     // P bf16 [64][64] tile (1024-aligned)
+constexpr uint32_t kA_Misc = kA_G + 33792;  // small arrays, TMEM address, flag, mbarrier (4 KB)
+constexpr uint32_t kA_Smem = kA_Misc + 4096 + 1024;  // + 1024 for aligning the dynamic base
+constexpr int kGS = 132;             // row stride of the g tile (floats)
 
 __global__ void __launch_bounds__(kAThreads, 2)
 tc_intra_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
@@ -152,14 +209,20 @@ tc_intra_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
 
     uint8_t* sm = align1024(smem_raw);
     const uint32_t sb = smem_u32(sm);
-    float* s_beta = reinterpret_cast<float*>(sm + kA_Misc);            // [64]
-    float* s_E = reinterpret_cast<float*>(sm + kA_Misc + 256);         // [128] e^{ref}
-    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + kA_Misc + 768);
-    int* s_wide = reinterpret_cast<int*>(sm + kA_Misc + 772);
-    const uint32_t mbar = smem_u32(sm + kA_Misc + 1024);
-    float* sA = reinterpret_cast<float*>(sm + kA_A);
-    float* sX = reinterpret_cast<float*>(sm + kA_K);
-    float* sY = reinterpret_cast<float*>(sm + kA_Y);
+    float* s_beta = reinterpret_cast<float*>(sm + kA_Misc);          // [64]
+    float* s_ref = reinterpret_cast<float*>(sm + kA_Misc + 256);     // [128]
+    float* s_E = reinterpret_cast<float*>(sm + kA_Misc + 768);       // [128] e^{ref} (1 in the wide case)
+    float* s_D = reinterpret_cast<float*>(sm + kA_Misc + 1280);      // [128] e^{g_last - ref}
+    float* s_carry = reinterpret_cast<float*>(sm + kA_Misc + 1792);  // [128] rows 0..31 total
+    float* s_lo = reinterpret_cast<float*>(sm + kA_Misc + 2304);     // [128] rows 32..63 min
+    float* s_hi = reinterpret_cast<float*>(sm + kA_Misc + 2816);     // [128] rows 32..63 max
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + kA_Misc + 3328);
+    int* s_wide = reinterpret_cast<int*>(sm + kA_Misc + 3332);
+    const uint32_t mbar = smem_u32(sm + kA_Misc + 3344);
+    float* sG = reinterpret_cast<float*>(sm + kA_G);
+    float* sA = reinterpret_cast<float*>(sm + kA_G);                 // after the gating pass
+    float* sY = reinterpret_cast<float*>(sm + kA_Ysc);
+    float* sX = reinterpret_cast<float*>(sm + kA_Kb);
     uint8_t* slot = slots + ((size_t)j * H + h) * kSlotBytes;
 
     if (tid == 0) {
@@ -171,7 +234,7 @@ tc_intra_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
         tmem_alloc(smem_u32(s_tmem), 256);
         tmem_relinquish();
     }
-    // raw k, q, v -> SW128 tiles (rows >= L zero-filled)
+    // raw k, q, v -> SW128 tiles; log_alpha -> g tile (rows >= L zero-filled: identity steps)
     for (int e = tid; e < 64 * 16; e += kAThreads) {
         const int r = e >> 4, ch = e & 15;
         const uint32_t o = sw128_chunk_off(r, ch, 64);
@@ -182,64 +245,105 @@ tc_intra_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
         cp_async16(sb + kA_Q + o, q + gi, nb);
         cp_async16(sb + kA_V + o, v + gi, nb);
     }
-    if (tid < 64) s_beta[tid] = tid < L ? beta[(size_t)(t0 + tid) * H + h] : 0.f;
-    __syncthreads();  // s_wide / mbarrier init / TMEM address visible
+    for (int e = tid; e < 64 * 32; e += kAThreads) {
+        const int r = e >> 5, ch = e & 31;
+        const int rr = r < L ? r : 0;
+        cp_async16(sb + kA_G + r * (kGS * 4) + ch * 16, log_alpha + ((size_t)(t0 + rr) * H + h) * 128 + ch * 4,
+                   r < L ? 16u : 0u);
+    }
+    if (tid < 64) cp_async4(sb + kA_Misc + 4 * tid, beta + (size_t)(t0 + (tid < L ? tid : 0)) * H + h, tid < L ? 4u : 0u);
+    cp_async_wait_all();
+    __syncthreads();
 
-    // cumulative gate of channel c = tid
-    const int c = tid;
-    float g[64];
-    float lo = 0.f, hi = 0.f;
+    // cumulative gate: thread (c, hf) scans rows 32*hf .. 32*hf+31 of channel c
+    const int c = tid & 127, hf = tid >> 7;
+    float gl[32];
     {
         float acc = 0.f;
 #pragma unroll
-        for (int r = 0; r < 64; ++r) {
-            const int rr = r < L ? r : L - 1;
-            float x = log_alpha[((size_t)(t0 + rr) * H + h) * 128 + c];
-            if (r >= L) x = 0.f;
-            acc += x;
-            g[r] = acc;
-            lo = fminf(lo, acc);
-            hi = fmaxf(hi, acc);
+        for (int u = 0; u < 32; ++u) {
+            acc += sG[(32 * hf + u) * kGS + c];
+            gl[u] = acc;
         }
     }
-    const float ref = 0.5f * (lo + hi);
-    const float glast = g[63];
-    if (!(hi - lo <= kTcFactorSpread)) atomicOr(s_wide, 1);
-    const float Ec = expf(ref);
-    const float Dc = expf(glast - ref);
-    s_E[c] = Ec;
-    *reinterpret_cast<float*>(slot + kSlotGam + 4 * c) = expf(glast);
-    cp_async_wait_all();
+    if (hf == 0) s_carry[c] = gl[31];
+    __syncthreads();
+    float lo, hi;
+    if (hf == 1) {
+        const float cr = s_carry[c];
+        lo = hi = cr;
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+            gl[u] += cr;
+            lo = fminf(lo, gl[u]);
+            hi = fmaxf(hi, gl[u]);
+        }
+        s_lo[c] = lo;
+        s_hi[c] = hi;
+        s_D[c] = gl[31];  // g_last, turned into e^{g_last - ref} below
+    } else {
+        lo = hi = 0.f;  // the chunk start (g = 0) is part of the range
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+            lo = fminf(lo, gl[u]);
+            hi = fmaxf(hi, gl[u]);
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < 32; ++u) sG[(32 * hf + u) * kGS + c] = gl[u];
+    __syncthreads();
+    if (hf == 0) {
+        lo = fminf(lo, s_lo[c]);
+        hi = fmaxf(hi, s_hi[c]);
+        const float ref = 0.5f * (lo + hi);
+        const float glast = s_D[c];
+        s_ref[c] = ref;
+        s_E[c] = exp_fast(ref);
+        s_D[c] = exp_fast(glast - ref);
+        *reinterpret_cast<float*>(slot + kSlotGam + 4 * c) = exp_fast(glast);
+        if (!(hi - lo <= kTcFactorSpread)) atomicOr(s_wide, 1);
+    }
     __syncthreads();
     const bool wide = *s_wide != 0;
     const uint32_t tmem = *s_tmem;
     uint32_t phase = 0;
     bool ok = true;
+    const int ch = tid & 15, rb = tid >> 4;  // element-wise passes: chunk ch of rows rb + 16 jj
+    const int wq = warp & 3;
+    const int rowq = 16 * wq + (lane & 15);  // M = 64 accumulator row held by this lane (lane < 16)
+    const uint32_t trow = tmem + ((uint32_t)(32 * wq) << 16);
 
     if (!wide) {
-        // gated operands in place + Kd^T image (row c of the [128 x 64] tile, 16-byte stores)
+        float ref8[8], D8[8];
 #pragma unroll
-        for (int rb = 0; rb < 64; rb += 8) {
-            uint32_t pk[4];
+        for (int m = 0; m < 8; ++m) {
+            ref8[m] = s_ref[8 * ch + m];
+            D8[m] = s_D[8 * ch + m];
+        }
 #pragma unroll
-            for (int m = 0; m < 8; m += 2) {
-                float kd[2];
+        for (int jj = 0; jj < 4; ++jj) {
+            const int r = rb + 16 * jj;
+            const uint32_t o = sw128_chunk_off(r, ch, 64);
+            float kv[8], qv[8];
+            unpack8(*reinterpret_cast<const uint4*>(sm + kA_K + o), kv);
+            unpack8(*reinterpret_cast<const uint4*>(sm + kA_Q + o), qv);
+            const float4 ga = *reinterpret_cast<const float4*>(sG + r * kGS + 8 * ch);
+            const float4 gb = *reinterpret_cast<const float4*>(sG + r * kGS + 8 * ch + 4);
+            const float g8[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+            float kf[8], qf[8], kb[8], kd[8];
 #pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int r = rb + m + u;
-                    const uint32_t o = sw128_off(r, c, 64);
-                    const float kv = lds_bf16(sm + kA_K + o), qv = lds_bf16(sm + kA_Q + o);
-                    const float x = g[r] - ref;
-                    const float ef = exp_fast(x), eb = exp_fast(-x);
-                    sts_bf16(sm + kA_K + o, kv * ef);
-                    sts_bf16(sm + kA_Q + o, qv * ef);
-                    sts_bf16(sm + kA_Kb + o, kv * eb);
-                    sts_bf16(sm + kA_Kt + o, kv * ef * Ec);
-                    kd[u] = kv * eb * Dc;
-                }
-                pk[m >> 1] = pack_bf16(kd[0], kd[1]);
+            for (int m = 0; m < 8; ++m) {
+                const float x = g8[m] - ref8[m];
+                const float ef = exp_fast(x), eb = exp_fast(-x);
+                kf[m] = kv[m] * ef;
+                qf[m] = qv[m] * ef;
+                kb[m] = kv[m] * eb;
+                kd[m] = kb[m] * D8[m];  // k e^{g_last - g}
             }
-            *reinterpret_cast<uint4*>(slot + kSlotKd + sw128_chunk_off(c, rb >> 3, 128)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            *reinterpret_cast<uint4*>(sm + kA_K + o) = pack8(kf);
+            *reinterpret_cast<uint4*>(sm + kA_Q + o) = pack8(qf);
+            *reinterpret_cast<uint4*>(sm + kA_Kb + o) = pack8(kb);
+            *reinterpret_cast<uint4*>(slot + kSlotKd + o) = pack8(kd);
         }
         fence_proxy_async();
         __syncthreads();
@@ -253,121 +357,182 @@ tc_intra_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
             }
             mma_commit(mbar);
         }
-        // Qg image = Qf * e^{ref} (same swizzled layout), while the MMAs run
-        for (int e = tid; e < 64 * 16; e += kAThreads) {
-            const int r = e >> 4, ch = e & 15;
-            const uint32_t o = sw128_chunk_off(r, ch, 64);
-            const uint4 raw = *reinterpret_cast<const uint4*>(sm + kA_Q + o);
-            const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(&raw);
-            uint32_t pk[4];
-#pragma unroll
-            for (int m = 0; m < 8; m += 2)
-                pk[m >> 1] = pack_bf16(__bfloat162float(hv[m]) * s_E[ch * 8 + m],
-                                       __bfloat162float(hv[m + 1]) * s_E[ch * 8 + m + 1]);
-            *reinterpret_cast<uint4*>(slot + kSlotQ + o) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        }
         ok = mbar_wait(mbar, phase);
         phase ^= 1;
         fence_after_sync();
-        // A' and P' rows (M = 64 layout: row 16*warp + lane at TMEM lane 32*warp + lane, lane < 16)
-        const int r = 16 * warp + (lane & 15);
-        const uint32_t trow = tmem + ((uint32_t)(32 * warp) << 16);
-        const float br = s_beta[r];
+        if (warp < 4) {  // A' rows -> A (fp32, diag(beta), strictly lower)
+            const float br = s_beta[rowq];
 #pragma unroll
-        for (int blk = 0; blk < 4; ++blk) {
-            float a[16];
-            tmem_ld16(trow + blk * 16, a);
-            tmem_wait_ld();
-            if (lane < 16) {
+            for (int blk = 0; blk < 4; ++blk) {
+                float a[16];
+                tmem_ld16(trow + blk * 16, a);
+                tmem_wait_ld();
+                if (lane < 16) {
 #pragma unroll
-                for (int m = 0; m < 16; ++m) {
-                    const int i = blk * 16 + m;
-                    sA[r * kTS + i] = (i < r) ? br * a[m] : 0.f;
+                    for (int m = 0; m < 16; m += 4) {
+                        const int i = blk * 16 + m;
+                        *reinterpret_cast<float4*>(sA + rowq * kAS + i) =
+                            make_float4(i < rowq ? br * a[m] : 0.f, i + 1 < rowq ? br * a[m + 1] : 0.f,
+                                        i + 2 < rowq ? br * a[m + 2] : 0.f, i + 3 < rowq ? br * a[m + 3] : 0.f);
+                    }
                 }
             }
-        }
+        } else {  // P' rows -> P (bf16 K-major tile, lower triangle incl. diagonal)
 #pragma unroll
-        for (int blk = 0; blk < 4; ++blk) {
-            float a[16];
-            tmem_ld16(trow + 64 + blk * 16, a);
-            tmem_wait_ld();
-            if (lane < 16) {
-                uint32_t pk[8];
+            for (int blk = 0; blk < 4; ++blk) {
+                float a[16];
+                tmem_ld16(trow + 64 + blk * 16, a);
+                tmem_wait_ld();
+                if (lane < 16) {
 #pragma unroll
-                for (int m = 0; m < 16; m += 2) {
-                    const int i = blk * 16 + m;
-                    pk[m >> 1] = pack_bf16(i <= r ? a[m] : 0.f, i + 1 <= r ? a[m + 1] : 0.f);
+                    for (int m = 0; m < 16; ++m) a[m] = (blk * 16 + m <= rowq) ? a[m] : 0.f;
+                    *reinterpret_cast<uint4*>(sm + kA_P + sw128_chunk_off(rowq, 2 * blk, 64)) = pack8(a);
+                    *reinterpret_cast<uint4*>(sm + kA_P + sw128_chunk_off(rowq, 2 * blk + 1, 64)) = pack8(a + 8);
                 }
-                *reinterpret_cast<uint4*>(slot + kSlotP + sw128_chunk_off(r, 2 * blk, 64)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                *reinterpret_cast<uint4*>(slot + kSlotP + sw128_chunk_off(r, 2 * blk + 1, 64)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
             }
         }
         fence_before_sync();
     } else {
-        // exact per-element factors on CUDA cores; g goes to shared memory (Kb and Kt areas)
-        float* sg = reinterpret_cast<float*>(sm + kA_Kb);
-#pragma unroll
-        for (int r = 0; r < 64; ++r) sg[r * 128 + c] = g[r];
-        __syncthreads();
-        for (int e = tid; e < 64 * 64; e += kAThreads) {
+        // some channel's gate spreads beyond e^160: exact per-element factors on CUDA cores
+        float av[16], pv[16];
+#pragma unroll 1
+        for (int m = 0; m < 16; ++m) {
+            const int e = tid + kAThreads * m;
             const int r = e >> 6, i = e & 63;
             float a = 0.f, p = 0.f;
             if (i <= r) {
                 for (int cc = 0; cc < 128; ++cc) {
-                    const float kk = lds_bf16(sm + kA_K + sw128_off(i, cc, 64)) * expf(sg[r * 128 + cc] - sg[i * 128 + cc]);
+                    const float kk = lds_bf16(sm + kA_K + sw128_off(i, cc, 64)) * expf(sG[r * kGS + cc] - sG[i * kGS + cc]);
                     a = fmaf(lds_bf16(sm + kA_K + sw128_off(r, cc, 64)), kk, a);
                     p = fmaf(lds_bf16(sm + kA_Q + sw128_off(r, cc, 64)), kk, p);
                 }
             }
-            sA[r * kTS + i] = (i < r) ? s_beta[r] * a : 0.f;
-            *reinterpret_cast<__nv_bfloat16*>(slot + kSlotP + sw128_off(r, i, 64)) = __float2bfloat16_rn(p);
+            av[m] = (i < r) ? s_beta[r] * a : 0.f;
+            pv[m] = p;
         }
-        __syncthreads();  // g in shared memory no longer needed
+        __syncthreads();  // every thread is done reading raw k and q across rows
+        // in place: k -> k e^g (B operand of W), q -> q e^g; Kd = k e^{g_last - g} to the image
+#pragma unroll 1
+        for (int jj = 0; jj < 4; ++jj) {
+            const int r = rb + 16 * jj;
+            const uint32_t o = sw128_chunk_off(r, ch, 64);
+            float kv[8], qv[8], kt[8], kd[8], qg[8];
+            unpack8(*reinterpret_cast<const uint4*>(sm + kA_K + o), kv);
+            unpack8(*reinterpret_cast<const uint4*>(sm + kA_Q + o), qv);
 #pragma unroll
-        for (int rb = 0; rb < 64; rb += 8) {
-            uint32_t pk[4];
-#pragma unroll
-            for (int m = 0; m < 8; m += 2) {
-                float kd[2];
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int r = rb + m + u;
-                    const uint32_t o = sw128_off(r, c, 64);
-                    const float kv = lds_bf16(sm + kA_K + o), qv = lds_bf16(sm + kA_Q + o);
-                    const float eg = expf(g[r]);
-                    sts_bf16(sm + kA_Kt + o, kv * eg);
-                    *reinterpret_cast<__nv_bfloat16*>(slot + kSlotQ + o) = __float2bfloat16_rn(qv * eg);
-                    kd[u] = kv * expf(glast - g[r]);
-                }
-                pk[m >> 1] = pack_bf16(kd[0], kd[1]);
+            for (int m = 0; m < 8; ++m) {
+                const float gv = sG[r * kGS + 8 * ch + m], gz = sG[63 * kGS + 8 * ch + m];
+                const float eg = expf(gv);
+                kt[m] = kv[m] * eg;
+                qg[m] = qv[m] * eg;
+                kd[m] = kv[m] * expf(gz - gv);
             }
-            *reinterpret_cast<uint4*>(slot + kSlotKd + sw128_chunk_off(c, rb >> 3, 128)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            *reinterpret_cast<uint4*>(sm + kA_K + o) = pack8(kt);
+            *reinterpret_cast<uint4*>(sm + kA_Q + o) = pack8(qg);
+            *reinterpret_cast<uint4*>(slot + kSlotKd + o) = pack8(kd);
+        }
+        __syncthreads();  // g no longer read: A and the P tile take its place
+        for (int cc = tid; cc < 128; cc += kAThreads) s_E[cc] = 1.f;
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+            const int e = tid + kAThreads * m;
+            const int r = e >> 6, i = e & 63;
+            sA[r * kAS + i] = av[m];
+            *reinterpret_cast<__nv_bfloat16*>(sm + kA_P + sw128_off(r, i, 64)) = __float2bfloat16_rn(pv[m]);
         }
     }
     ok = __syncthreads_and(ok);
 
-    // UT transform, then T = X diag(beta) as a bf16 K-major tile (over Kb)
+    // UT transform (X over Kb), then T = X diag(beta) as a bf16 K-major tile (also over Kb)
     if (ok) ut_inverse_64(sA, sX, sY);
-    for (int e = tid; e < 64 * 8 && ok; e += kAThreads) {
-        const int r = e >> 3, ch = e & 7;
-        uint32_t pk[4];
+    uint4 tch[2];
 #pragma unroll
-        for (int m = 0; m < 8; m += 2) {
-            const int i = ch * 8 + m;
-            pk[m >> 1] = pack_bf16(sX[r * kTS + i] * s_beta[i], sX[r * kTS + i + 1] * s_beta[i + 1]);
-        }
-        *reinterpret_cast<uint4*>(sm + kA_Kb + sw128_chunk_off(r, ch, 64)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    for (int u = 0; u < 2; ++u) {
+        const int e = tid + kAThreads * u;
+        const int r = e >> 3, c8 = e & 7;
+        float t8[8];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) t8[m] = sX[r * kXS + 8 * c8 + m] * s_beta[8 * c8 + m];
+        tch[u] = pack8(t8);
+    }
+    __syncthreads();  // X fully read
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const int e = tid + kAThreads * u;
+        *reinterpret_cast<uint4*>(sm + kA_Kb + sw128_chunk_off(e >> 3, e & 7, 64)) = tch[u];
     }
     fence_proxy_async();
     __syncthreads();
-    if (ok && tid == 0) {
+    if (ok && tid == 0) {  // [W' | Uv] = T [Kf | v]  (B operand: four atom columns over the K and V tiles)
         fence_after_sync();
-        const uint32_t id = idesc_bf16(64, 128, false, true);
+        const uint32_t id = idesc_bf16(64, 256, false, true);
 #pragma unroll
-        for (int kk = 0; kk < 64; kk += 16) {
-            mma_bf16(tmem + 0, desc_kmajor(sb + kA_Kb, 64, kk), desc_mnmajor(sb + kA_Kt, 64, kk), id, kk > 0);
-            mma_bf16(tmem + 128, desc_kmajor(sb + kA_Kb, 64, kk), desc_mnmajor(sb + kA_V, 64, kk), id, kk > 0);
+        for (int kk = 0; kk < 64; kk += 16)
+            mma_bf16(tmem + 0, desc_kmajor(sb + kA_Kb, 64, kk), desc_mnmajor(sb + kA_K, 64, kk), id, kk > 0);
+        mma_commit(mbar);
+    }
+    if (ok) {
+        ok = mbar_wait(mbar, phase);
+        phase ^= 1;
+        fence_after_sync();
+    }
+    ok = __syncthreads_and(ok);
+    if (ok) {
+        if (warp < 4) {  // W = W' diag(e^ref): image rows 0..63 of [W; Q'] and the W tile (over Kf)
+#pragma unroll
+            for (int b2 = 0; b2 < 8; b2 += 2) {
+                float a2[32];
+                tmem_ld16(trow + b2 * 16, a2);
+                tmem_ld16(trow + b2 * 16 + 16, a2 + 16);
+                tmem_wait_ld();
+#pragma unroll
+                for (int hb = 0; hb < 2; ++hb) {
+                    const int blk = b2 + hb;
+                    float* a = a2 + 16 * hb;
+                    if (lane < 16) {
+#pragma unroll
+                        for (int m = 0; m < 16; ++m) a[m] *= s_E[blk * 16 + m];
+                        const uint4 p0 = pack8(a), p1 = pack8(a + 8);
+                        *reinterpret_cast<uint4*>(slot + kSlotWQ + sw128_chunk_off(rowq, 2 * blk, 128)) = p0;
+                        *reinterpret_cast<uint4*>(slot + kSlotWQ + sw128_chunk_off(rowq, 2 * blk + 1, 128)) = p1;
+                        *reinterpret_cast<uint4*>(sm + kA_K + sw128_chunk_off(rowq, 2 * blk, 64)) = p0;
+                        *reinterpret_cast<uint4*>(sm + kA_K + sw128_chunk_off(rowq, 2 * blk + 1, 64)) = p1;
+                    }
+                }
+            }
+        } else {  // Uv -> image [slice][64][32] and the Uv tile (over v)
+#pragma unroll
+            for (int b2 = 0; b2 < 8; b2 += 2) {
+                float a2[32];
+                tmem_ld16(trow + 128 + b2 * 16, a2);
+                tmem_ld16(trow + 128 + b2 * 16 + 16, a2 + 16);
+                tmem_wait_ld();
+#pragma unroll
+                for (int hb = 0; hb < 2; ++hb) {
+                    const int blk = b2 + hb;
+                    float* a = a2 + 16 * hb;
+                    if (lane < 16) {
+                        const uint4 p0 = pack8(a), p1 = pack8(a + 8);
+                        const int col = blk * 16, sl = col >> 5, m0 = (col & 31) >> 3;
+                        uint8_t* dst = slot + kSlotUv + (size_t)sl * 4096;
+                        *reinterpret_cast<uint4*>(dst + slice_chunk_off(rowq, m0)) = p0;
+                        *reinterpret_cast<uint4*>(dst + slice_chunk_off(rowq, m0 + 1)) = p1;
+                        *reinterpret_cast<uint4*>(sm + kA_V + sw128_chunk_off(rowq, 2 * blk, 64)) = p0;
+                        *reinterpret_cast<uint4*>(sm + kA_V + sw128_chunk_off(rowq, 2 * blk + 1, 64)) = p1;
+                    }
+                }
+            }
         }
+    }
+    fence_proxy_async();
+    fence_before_sync();
+    ok = __syncthreads_and(ok);
+    if (ok && tid == 0) {  // [P W | P Uv] = P [W | Uv]  (B operand: four atom columns over the W and Uv tiles)
+        fence_after_sync();
+        const uint32_t id = idesc_bf16(64, 256, false, true);
+#pragma unroll
+        for (int kk = 0; kk < 64; kk += 16)
+            mma_bf16(tmem + 0, desc_kmajor(sb + kA_P, 64, kk), desc_mnmajor(sb + kA_K, 64, kk), id, kk > 0);
         mma_commit(mbar);
     }
     if (ok) {
@@ -376,34 +541,46 @@ tc_intra_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
     }
     ok = __syncthreads_and(ok);
     if (ok) {
-        const int r = 16 * warp + (lane & 15);
-        const uint32_t trow = tmem + ((uint32_t)(32 * warp) << 16);
+        if (warp < 4) {  // Q' = q e^g - P W -> image rows 64..127
 #pragma unroll
-        for (int blk = 0; blk < 8; ++blk) {  // W row r -> image
-            float a[16];
-            tmem_ld16(trow + blk * 16, a);
-            tmem_wait_ld();
-            if (lane < 16) {
-                uint32_t pk[8];
+            for (int b2 = 0; b2 < 8; b2 += 2) {
+                float a2[32];
+                tmem_ld16(trow + b2 * 16, a2);
+                tmem_ld16(trow + b2 * 16 + 16, a2 + 16);
+                tmem_wait_ld();
 #pragma unroll
-                for (int m = 0; m < 16; m += 2) pk[m >> 1] = pack_bf16(a[m], a[m + 1]);
-                *reinterpret_cast<uint4*>(slot + kSlotW + sw128_chunk_off(r, 2 * blk, 64)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                *reinterpret_cast<uint4*>(slot + kSlotW + sw128_chunk_off(r, 2 * blk + 1, 64)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                for (int hb = 0; hb < 2; ++hb) {
+                    const int blk = b2 + hb;
+                    float* a = a2 + 16 * hb;
+                    if (lane < 16) {
+                        float qf[16];
+                        unpack8(*reinterpret_cast<const uint4*>(sm + kA_Q + sw128_chunk_off(rowq, 2 * blk, 64)), qf);
+                        unpack8(*reinterpret_cast<const uint4*>(sm + kA_Q + sw128_chunk_off(rowq, 2 * blk + 1, 64)), qf + 8);
+#pragma unroll
+                        for (int m = 0; m < 16; ++m) a[m] = qf[m] * s_E[blk * 16 + m] - a[m];
+                        *reinterpret_cast<uint4*>(slot + kSlotWQ + sw128_chunk_off(64 + rowq, 2 * blk, 128)) = pack8(a);
+                        *reinterpret_cast<uint4*>(slot + kSlotWQ + sw128_chunk_off(64 + rowq, 2 * blk + 1, 128)) = pack8(a + 8);
+                    }
+                }
             }
-        }
+        } else {  // O0 = P Uv -> image [slice][64][32]
 #pragma unroll
-        for (int blk = 0; blk < 8; ++blk) {  // Uv row r -> [slice][64][32]
-            float a[16];
-            tmem_ld16(trow + 128 + blk * 16, a);
-            tmem_wait_ld();
-            if (lane < 16) {
-                uint32_t pk[8];
+            for (int b2 = 0; b2 < 8; b2 += 2) {
+                float a2[32];
+                tmem_ld16(trow + 128 + b2 * 16, a2);
+                tmem_ld16(trow + 128 + b2 * 16 + 16, a2 + 16);
+                tmem_wait_ld();
 #pragma unroll
-                for (int m = 0; m < 16; m += 2) pk[m >> 1] = pack_bf16(a[m], a[m + 1]);
-                const int col = blk * 16, sl = col >> 5;
-                uint8_t* dst = slot + kSlotUv + (size_t)(sl * 64 + r) * 64 + (col & 31) * 2;
-                *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                *reinterpret_cast<uint4*>(dst + 16) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                for (int hb = 0; hb < 2; ++hb) {
+                    const int blk = b2 + hb;
+                    float* a = a2 + 16 * hb;
+                    if (lane < 16) {
+                        const int col = blk * 16, sl = col >> 5, m0 = (col & 31) >> 3;
+                        uint8_t* dst = slot + kSlotO0 + (size_t)sl * 4096;
+                        *reinterpret_cast<uint4*>(dst + slice_chunk_off(rowq, m0)) = pack8(a);
+                        *reinterpret_cast<uint4*>(dst + slice_chunk_off(rowq, m0 + 1)) = pack8(a + 8);
+                    }
+                }
             }
         }
     }
@@ -415,21 +592,25 @@ tc_intra_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
 // ------------------------------------------------------------------------------------------------
 // Phase B
 // ------------------------------------------------------------------------------------------------
-constexpr int kBThreads = 128;
+constexpr int kBCompute = 128;              // 4 compute warps: thread c owns row c of the state slice
+constexpr int kBThreads = kBCompute + 64;   // + MMA-issue warp (4) + bulk-copy warp (5)
 constexpr int kBStages = 3;
-constexpr uint32_t kStageBytes = 62464;     // W | Qg | Kd^T | P (57344 B) + Uv slice (4096 B) + e^{g_last} (512 B)
-constexpr uint32_t kStUv = 57344, kStGam = 61440, kStTx = 61952;
-constexpr uint32_t kB_S = kBStages * kStageBytes;  // S^T tile [32 x 128] bf16 (8 KB)
-constexpr uint32_t kB_U = kB_S + 8192;             // U^T tile [32 x 64]  bf16 (4 KB)
-constexpr uint32_t kB_Misc = kB_U + 4096;          // mbarriers + TMEM address
+constexpr uint32_t kStWQ = 0, kStKd = 32768, kStUv = 49152, kStO0 = 53248, kStGam = 57344;
+constexpr uint32_t kStTx = 57856;           // bytes landing per stage
+constexpr uint32_t kStageBytes = 58368;     // 57 KB, 1024-aligned
+constexpr uint32_t kB_S = kBStages * kStageBytes;  // S slice: bf16 [128 rows][64] SW128 (32 columns used)
+constexpr uint32_t kB_U = kB_S + 16384;            // U:       bf16 [64 rows][64]  SW128 (32 columns used)
+constexpr uint32_t kB_Misc = kB_U + 8192;          // mbarriers + TMEM address
 constexpr uint32_t kB_Smem = kB_Misc + 256 + 1024;
+constexpr uint32_t kTmD1 = 0, kTmY = 32;           // TMEM columns: [X; O'] and Y
 
 __device__ __forceinline__ void tc_issue_stage(uint32_t stage_addr, uint32_t full_bar, const uint8_t* slot, int vt)
 {
     using namespace tc;
     mbar_arrive_expect_tx(full_bar, kStTx);
-    bulk_g2s(stage_addr, slot, kSlotUv, full_bar);
+    bulk_g2s(stage_addr + kStWQ, slot + kSlotWQ, kSlotUv, full_bar);  // [W; Q'] and Kd, contiguous
     bulk_g2s(stage_addr + kStUv, slot + kSlotUv + vt * 4096, 4096, full_bar);
+    bulk_g2s(stage_addr + kStO0, slot + kSlotO0 + vt * 4096, 4096, full_bar);
     bulk_g2s(stage_addr + kStGam, slot + kSlotGam, 512, full_bar);
 }
 
@@ -445,8 +626,9 @@ tc_inter_kernel(const float* S0, float* S_final, __nv_bfloat16* __restrict__ out
     if (hdr->bad) return;
     uint8_t* sm = align1024(smem_raw);
     const uint32_t sb = smem_u32(sm);
-    const uint32_t bar_full = smem_u32(sm + kB_Misc);       // kBStages barriers
-    const uint32_t bar_mma = bar_full + 8 * kBStages;
+    const uint32_t bar_full = smem_u32(sm + kB_Misc);   // kBStages barriers
+    const uint32_t bar_d1 = bar_full + 8 * kBStages;    // [X; O'] ready
+    const uint32_t bar_y = bar_d1 + 8;                  // Y ready
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + kB_Misc + 64);
 
     const int jb = off[n], je = off[n + 1], nch = je - jb;
@@ -455,39 +637,40 @@ tc_inter_kernel(const float* S0, float* S_final, __nv_bfloat16* __restrict__ out
 
     if (tid == 0) {
         for (int s = 0; s < kBStages; ++s) mbar_init(bar_full + 8 * s, 1);
-        mbar_init(bar_mma, 1);
+        mbar_init(bar_d1, 1);
+        mbar_init(bar_y, 1);
         mbar_fence_init();
     }
     if (warp == 0) {
-        tmem_alloc(smem_u32(s_tmem), 128);
+        tmem_alloc(smem_u32(s_tmem), 64);
         tmem_relinquish();
     }
-    // state slice: thread c owns row c, columns v0 .. v0+31
-    const int c = tid;
+    const int c = tid;  // compute threads: state row
     float S[kTcNV];
-    const size_t srow = (((size_t)n * H + h) * 128 + c) * 128 + v0;
-    if (S0) {
+    const size_t srow = (((size_t)n * H + h) * 128 + (c & 127)) * 128 + v0;
+    if (warp < 4) {
+        if (S0) {
 #pragma unroll
-        for (int m = 0; m < kTcNV; m += 4) {
-            const float4 x = *reinterpret_cast<const float4*>(S0 + srow + m);
-            S[m] = x.x; S[m + 1] = x.y; S[m + 2] = x.z; S[m + 3] = x.w;
+            for (int m = 0; m < kTcNV; m += 4) {
+                const float4 x = *reinterpret_cast<const float4*>(S0 + srow + m);
+                S[m] = x.x; S[m + 1] = x.y; S[m + 2] = x.z; S[m + 3] = x.w;
+            }
+        } else {
+#pragma unroll
+            for (int m = 0; m < kTcNV; ++m) S[m] = 0.f;
         }
-    } else {
 #pragma unroll
-        for (int m = 0; m < kTcNV; ++m) S[m] = 0.f;
+        for (int m = 0; m < 4; ++m) *reinterpret_cast<uint4*>(sm + kB_S + sw128_chunk_off(c, m, 128)) = pack8(S + 8 * m);
     }
-#pragma unroll
-    for (int m = 0; m < kTcNV; ++m) sts_bf16(sm + kB_S + sw128_off(m, c, 32), S[m]);
-    __syncthreads();  // barriers initialised, TMEM address visible
-    if (tid == 0)
+    fence_proxy_async();
+    __syncthreads();  // barriers initialised, TMEM address visible, S tile written
+    if (warp == 5 && lane == 0)
         for (int s = 0; s < kBStages && s < nch; ++s)
             tc_issue_stage(sb + s * kStageBytes, bar_full + 8 * s, slots + ((size_t)(jb + s) * H + h) * kSlotBytes, vt);
-    fence_proxy_async();
-    __syncthreads();
     const uint32_t tmem = *s_tmem;
-    const uint32_t tw = tmem + ((uint32_t)(32 * warp) << 16);
-    const int r = 16 * warp + (lane & 15);
-    uint32_t mphase = 0;
+    const uint32_t tw = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+    const uint32_t id_d1 = idesc_bf16(128, kTcNV, false, true);  // [W; Q'] S   (S MN-major)
+    const uint32_t id_y = idesc_bf16(128, kTcNV, true, true);    // Kd^T U      (Kd, U MN-major)
     bool ok = true;
 
     for (int it = 0; it < nch && ok; ++it) {
@@ -496,93 +679,86 @@ tc_inter_kernel(const float* S0, float* S_final, __nv_bfloat16* __restrict__ out
         const uint8_t* stp = sm + s * kStageBytes;
         const long long t0 = s0 + (long long)it * 64;
         const int L = (s1 - t0) < 64 ? (int)(s1 - t0) : 64;
-        ok = mbar_wait(bar_full + 8 * s, (uint32_t)(it / kBStages) & 1u);
-        if (ok && tid == 0) {
-            fence_after_sync();
-            const uint32_t id = idesc_bf16(64, kTcNV, false, false);
+        const uint32_t par = (uint32_t)it & 1u;
+        if (warp == 4) {
+            if (lane == 0) {
+                ok = mbar_wait(bar_full + 8 * s, (uint32_t)(it / kBStages) & 1u);
+                fence_after_sync();
+                if (ok) {
 #pragma unroll
-            for (int kk = 0; kk < 128; kk += 16) {
-                mma_bf16(tmem + 0, desc_kmajor(st + kSlotW, 64, kk), desc_kmajor(sb + kB_S, 32, kk), id, kk > 0);
-                mma_bf16(tmem + 32, desc_kmajor(st + kSlotQ, 64, kk), desc_kmajor(sb + kB_S, 32, kk), id, kk > 0);
-            }
-            mma_commit(bar_mma);
-        }
-        ok = ok && mbar_wait(bar_mma, mphase);
-        mphase ^= 1;
-        fence_after_sync();
-        {   // U = Uv - X  ->  U^T tile
-            float x[32];
-            tmem_ld16(tw + 0, x);
-            tmem_ld16(tw + 16, x + 16);
-            tmem_wait_ld();
-            if (lane < 16) {
-                const uint8_t* uv = stp + kStUv + r * 64;
-#pragma unroll
-                for (int m = 0; m < 32; m += 8) {
-                    const uint4 raw = *reinterpret_cast<const uint4*>(uv + 2 * m);
-                    const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(&raw);
-#pragma unroll
-                    for (int u = 0; u < 8; ++u)
-                        sts_bf16(sm + kB_U + sw128_off(m + u, r, 32), __bfloat162float(hv[u]) - x[m + u]);
+                    for (int kk = 0; kk < 128; kk += 16)
+                        mma_bf16(tmem + kTmD1, desc_kmajor(st + kStWQ, 128, kk), desc_mnmajor(sb + kB_S, 128, kk), id_d1,
+                                 kk > 0);
+                    mma_commit(bar_d1);
                 }
             }
-        }
-        fence_proxy_async();
-        fence_before_sync();
-        ok = __syncthreads_and(ok);
-        if (ok && tid == 0) {
-            fence_after_sync();
-            const uint32_t id64 = idesc_bf16(64, kTcNV, false, false);
-            const uint32_t id128 = idesc_bf16(128, kTcNV, false, false);
+            named_sync(1, 96);  // U tile written by warps 0 and 1
+            if (lane == 0 && ok) {
+                fence_after_sync();
 #pragma unroll
-            for (int kk = 0; kk < 64; kk += 16) {
-                mma_bf16(tmem + 32, desc_kmajor(st + kSlotP, 64, kk), desc_kmajor(sb + kB_U, 32, kk), id64, 1u);
-                mma_bf16(tmem + 64, desc_kmajor(st + kSlotKd, 128, kk), desc_kmajor(sb + kB_U, 32, kk), id128, kk > 0);
+                for (int kk = 0; kk < 64; kk += 16)
+                    mma_bf16(tmem + kTmY, desc_mnmajor(st + kStKd, 64, kk), desc_mnmajor(sb + kB_U, 64, kk), id_y, kk > 0);
+                mma_commit(bar_y);
             }
-            mma_commit(bar_mma);
-        }
-        ok = ok && mbar_wait(bar_mma, mphase);
-        mphase ^= 1;
-        fence_after_sync();
-        {   // S <- e^{g_last} S + Y
+        } else if (warp < 4) {
+            ok = mbar_wait(bar_full + 8 * s, (uint32_t)(it / kBStages) & 1u);
+            ok = ok && mbar_wait(bar_d1, par);
+            fence_after_sync();
+            float x[32];
+            tmem_ld16(tw + kTmD1, x);
+            tmem_ld16(tw + kTmD1 + 16, x + 16);
+            tmem_wait_ld();
+            if (warp < 2) {  // U = Uv - X, row r = c
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    float u[8];
+                    unpack8(*reinterpret_cast<const uint4*>(stp + kStUv + slice_chunk_off(c, m)), u);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) u[e] -= x[8 * m + e];
+                    *reinterpret_cast<uint4*>(sm + kB_U + sw128_chunk_off(c, m, 64)) = pack8(u);
+                }
+                fence_proxy_async();
+                named_arrive(1, 96);
+            } else {  // out = O' + O0, row r = c - 64
+                const int r = c - 64;
+                if (r < L && ok) {
+                    uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)(t0 + r) * H + h) * 128 + v0);
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        float u[8];
+                        unpack8(*reinterpret_cast<const uint4*>(stp + kStO0 + slice_chunk_off(r, m)), u);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) u[e] += x[8 * m + e];
+                        dst[m] = pack8(u);
+                    }
+                }
+            }
+            ok = ok && mbar_wait(bar_y, par);
+            fence_after_sync();
             float y[32];
-            tmem_ld16(tw + 64, y);
-            tmem_ld16(tw + 80, y + 16);
+            tmem_ld16(tw + kTmY, y);
+            tmem_ld16(tw + kTmY + 16, y + 16);
             tmem_wait_ld();
             const float gam = *reinterpret_cast<const float*>(stp + kStGam + 4 * c);
 #pragma unroll
-            for (int m = 0; m < kTcNV; ++m) {
-                S[m] = fmaf(gam, S[m], y[m]);
-                sts_bf16(sm + kB_S + sw128_off(m, c, 32), S[m]);
-            }
-        }
-        {   // O -> out
-            float o[32];
-            tmem_ld16(tw + 32, o);
-            tmem_ld16(tw + 48, o + 16);
-            tmem_wait_ld();
-            if (lane < 16 && r < L && ok) {
-                __nv_bfloat16* dst = out + ((size_t)(t0 + r) * H + h) * 128 + v0;
+            for (int m = 0; m < kTcNV; ++m) S[m] = fmaf(gam, S[m], y[m]);
 #pragma unroll
-                for (int m = 0; m < 32; m += 8)
-                    *reinterpret_cast<uint4*>(dst + m) = make_uint4(pack_bf16(o[m], o[m + 1]), pack_bf16(o[m + 2], o[m + 3]),
-                                                                    pack_bf16(o[m + 4], o[m + 5]), pack_bf16(o[m + 6], o[m + 7]));
-            }
+            for (int m = 0; m < 4; ++m) *reinterpret_cast<uint4*>(sm + kB_S + sw128_chunk_off(c, m, 128)) = pack8(S + 8 * m);
+            fence_proxy_async();
         }
-        fence_proxy_async();
         fence_before_sync();
         ok = __syncthreads_and(ok);
-        if (ok && tid == 0 && it + kBStages < nch)
+        if (warp == 5 && lane == 0 && ok && it + kBStages < nch)
             tc_issue_stage(st, bar_full + 8 * s, slots + ((size_t)(jb + it + kBStages) * H + h) * kSlotBytes, vt);
     }
-    if (S_final && ok) {
+    if (warp < 4 && S_final && ok) {
 #pragma unroll
         for (int m = 0; m < kTcNV; m += 4)
             *reinterpret_cast<float4*>(S_final + srow + m) = make_float4(S[m], S[m + 1], S[m + 2], S[m + 3]);
     }
     fence_before_sync();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, 128);
+    if (warp == 0) tmem_dealloc(tmem, 64);
 }
 
 inline cudaError_t launch_tc_prefill(const void* q, const void* k, const void* v, const float* la, const float* beta,

@@ -1,6 +1,8 @@
 """White-box check of the tensor-core prefill's phase A: the bf16 operand images it leaves in the
 workspace (swizzled shared-memory layout) are decoded here and compared with an fp64 numpy
-evaluation of their definitions.  Pinpoints a wrong descriptor or layout to one product."""
+evaluation of their definitions -- W = T (k e^g), Uv = T v, Q' = q e^g - P W, O0 = P Uv,
+Kd = k e^{g_last - g} and e^{g_last}, with T = (I + A)^{-1} diag(beta).  Pinpoints a wrong
+descriptor or layout to one product."""
 import numpy as np
 import pytest
 import torch
@@ -10,7 +12,7 @@ from gated_delta_rule_83_b200 import synth
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
-SLOT = dict(W=0, Q=16384, Kd=32768, P=49152, Uv=57344, gam=73728, bytes=74240)
+SLOT = dict(WQ=0, Kd=32768, Uv=49152, O0=65536, gam=81920, bytes=82432)
 
 
 def sw128_off(r, c, R):
@@ -25,6 +27,18 @@ def decode_tile(buf, base, R, C):
             o = sw128_off(r, c, R)
             b = int(raw[o]) | (int(raw[o + 1]) << 8)
             out[r, c] = np.frombuffer(np.uint32(b << 16).tobytes(), np.float32)[0]
+    return out
+
+
+def decode_slices(buf, base):
+    """[4 slices][64 rows][32 cols] bf16; chunk m of row r stored at chunk position m ^ ((r >> 1) & 3)."""
+    out = np.zeros((64, 128), np.float32)
+    for sl in range(4):
+        raw = buf[base + sl * 4096:base + (sl + 1) * 4096]
+        for r in range(64):
+            for m in range(4):
+                o = r * 64 + ((m ^ ((r >> 1) & 3)) << 4)
+                out[r, sl * 32 + m * 8:sl * 32 + m * 8 + 8] = bf16_to_f32(raw[o:o + 16].copy())
     return out
 
 
@@ -49,7 +63,7 @@ def expected_chunk(inp, t0, L, h):
     Uv = T @ v
     Qg = q * np.exp(g)
     Kd = k * np.exp(g[-1] - g)
-    return dict(W=W, Uv=Uv, Qg=Qg, Kd=Kd, P=P, gam=np.exp(g[-1]))
+    return dict(W=W, Uv=Uv, Qp=Qg - P @ W, O0=P @ Uv, Kd=Kd, gam=np.exp(g[-1]))
 
 
 def rel(a, b):
@@ -73,14 +87,13 @@ def test_phase_a_images():
         for h in range(H):
             base = slots0 + (j * H + h) * SLOT["bytes"]
             ex = expected_chunk(inp, t0, L, h)
-            Wg = decode_tile(buf, base + SLOT["W"], 64, 128)[:L]
-            Qg = decode_tile(buf, base + SLOT["Q"], 64, 128)[:L]
-            Kd = decode_tile(buf, base + SLOT["Kd"], 128, 64)[:, :L].T
-            P = decode_tile(buf, base + SLOT["P"], 64, 64)[:L, :L]
-            uv = bf16_to_f32(buf[base + SLOT["Uv"]:base + SLOT["Uv"] + 16384].copy()).reshape(4, 64, 32)
-            Uv = np.concatenate(list(uv), axis=1)[:L]
+            WQ = decode_tile(buf, base + SLOT["WQ"], 128, 128)
+            Wg, Qp = WQ[:L], WQ[64:64 + L]
+            Kd = decode_tile(buf, base + SLOT["Kd"], 64, 128)[:L]
+            Uv = decode_slices(buf, base + SLOT["Uv"])[:L]
+            O0 = decode_slices(buf, base + SLOT["O0"])[:L]
             gam = buf[base + SLOT["gam"]:base + SLOT["gam"] + 512].copy().view(np.float32)
-            errs = dict(Qg=rel(Qg, ex["Qg"]), Kd=rel(Kd, ex["Kd"]), P=rel(P, ex["P"]), W=rel(Wg, ex["W"]),
-                        Uv=rel(Uv, ex["Uv"]), gam=rel(gam, ex["gam"]))
+            errs = dict(Qp=rel(Qp, ex["Qp"]), Kd=rel(Kd, ex["Kd"]), W=rel(Wg, ex["W"]), Uv=rel(Uv, ex["Uv"]),
+                        O0=rel(O0, ex["O0"]), gam=rel(gam, ex["gam"]))
             for name, e in errs.items():
                 assert e < 2e-2, f"chunk {j} head {h}: {name} error {e:.3e} (all: {errs})"

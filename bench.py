@@ -61,6 +61,27 @@ def peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+def kernel_traffic(name, units):
+    """DRAM bytes per launch of one of our kernels, from the committed ncu summary under profiles/
+    (dram__bytes_read.sum + dram__bytes_write.sum per unit, scaled by the units one launch processes).
+    Returns (bytes or None, source note); None once the kernel's sources changed since the capture."""
+    import glob
+    import hashlib
+    import re
+    pat = re.compile(r"<!-- bench-traffic kernel=(\S+) per_unit_bytes=(\d+) unit=(\S+) sha1=(\w+) sources=(\S+) -->")
+    for f in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        for m in pat.finditer(open(f).read()):
+            if m.group(1) != name:
+                continue
+            h = hashlib.sha1()
+            for src in m.group(5).split(","):
+                h.update(open(os.path.join(ROOT, src), "rb").read())
+            if h.hexdigest()[:16] != m.group(4):
+                return None, f"{os.path.basename(f)}: stale, the kernel changed since the capture"
+            return int(m.group(2)) * units, f"{os.path.basename(f)} ({m.group(2)} B per {m.group(3)} x {units})"
+    return None, "no capture"
+
+
 # ------------------------------------------------------------------------------------------------
 # clocks sampled during the timed region
 # ------------------------------------------------------------------------------------------------
@@ -257,21 +278,29 @@ def run_ours(args):
     ms_per_step = ms / args.steps
     value = world * tokens * args.steps / (ms / 1e3)
 
-    # dominant kernel and roofline (algorithmic bytes of the whole prefill: q,k,v + log_alpha + beta in,
-    # out written; the state S0/S_final adds 2 x 64 KiB per (sequence, head))
+    # dominant kernel and roofline.  Algorithmic bytes of the prefill per token x head: q, k (bf16),
+    # log_alpha (fp32), v (bf16), beta (fp32) read and out (bf16) written -- 1540 B at dk = dv = 128 --
+    # plus the state S0 (if given) and S_final, 64 KiB each per (sequence, head).
     launches = sum(n for n, _ in prof.values())
     dom_name, (dom_n, dom_ms) = max(prof.items(), key=lambda kv: kv[1][1])
     tok_heads = tokens * H
     esz = q.element_size()
     alg_bytes = tok_heads * (2 * dk * esz + dv * esz + 4 * dk + 4 + dv * esz) + \
         (2 if S0 is not None else 1) * N * H * dk * dv * 4
+    dom_launch_ms = dom_ms / dom_n
+    achieved = alg_bytes / (dom_launch_ms / 1e3) / 1e9
     step_dev_ms = sum(t for _, t in prof.values()) / args.steps
-    achieved = alg_bytes / (step_dev_ms / 1e3) / 1e9
-    roofline = {"bound": "hbm", "kernel": "prefill step (all launches: " + ", ".join(sorted(prof)) + ")",
-                "dominant_kernel": dom_name, "dominant_share": dom_ms / max(sum(t for _, t in prof.values()), 1e-9),
-                "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                "peak_source": f"{peak_kind} hbm_gbs", "traffic": None,
-                "alg_bytes_per_step": alg_bytes, "device_ms_per_step": step_dev_ms}
+    lens = inp["lengths"] if inp["lengths"] is not None else [T] * B
+    units = sum((x + 63) // 64 for x in lens) * H  # chunk x head pairs per launch
+    traffic, traffic_src = kernel_traffic(dom_name, units)
+    roofline = {"bound": "hbm", "kernel": dom_name, "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                "frac": achieved / hbm, "traffic": traffic, "traffic_source": traffic_src,
+                "peak_source": f"{peak_kind} hbm_gbs (of {peak_kind})",
+                "alg_bytes_per_launch": alg_bytes, "alg_bytes_per_token_head": alg_bytes / tok_heads,
+                "launch_ms": dom_launch_ms, "share_of_step": dom_ms / max(sum(t for _, t in prof.values()), 1e-12),
+                "path": {"kernels": sorted(prof), "device_ms_per_step": step_dev_ms,
+                         "achieved": alg_bytes / (step_dev_ms / 1e3) / 1e9,
+                         "frac": alg_bytes / (step_dev_ms / 1e3) / 1e9 / hbm}}
 
     # e2e: host buffers through the public API
     e2e = None
@@ -373,11 +402,13 @@ def bench_decode(torch, kda, synth, dev, stream, world, rank, hbm, peak_kind, st
     pairs = w.B * w.H
     alg = pairs * (2 * w.dk * w.dv * 4 + 2 * w.dk * 2 + w.dv * 2 + 4 * w.dk + 4 + w.dv * 2)
     ach = alg / (kms / n / 1e3) / 1e9
+    traffic, traffic_src = kernel_traffic("decode_step", pairs)
     return {"metric": "KDA decode tokens/s", "workload": w.name, "desc": w.desc,
             "value": world * w.B * steps / (ms / 1e3), "unit": "tokens/s", "steps": steps,
             "us_per_step": ms * 1e3 / steps,
             "roofline": {"bound": "hbm", "kernel": "decode_step", "achieved": ach, "peak": hbm, "unit": "GB/s",
-                         "frac": ach / hbm, "peak_source": f"{peak_kind} hbm_gbs", "traffic": None,
+                         "frac": ach / hbm, "peak_source": f"{peak_kind} hbm_gbs (of {peak_kind})", "traffic": traffic,
+                         "traffic_source": traffic_src,
                          "alg_bytes_per_launch": alg, "device_us_per_launch": kms / n * 1e3},
             "gpu_launches": n}
 

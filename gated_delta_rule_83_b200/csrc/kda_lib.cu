@@ -14,6 +14,23 @@
 
 using namespace kda;
 
+namespace kda {
+// Waits on an mbarrier that nothing ever completes, through the same bounded wait the
+// tensor-core kernels use: the wait gives up, records KDA_ERR_TIMEOUT and the kernel returns.
+__global__ void selftest_timeout_kernel()
+{
+    __shared__ __align__(8) uint64_t bar;
+    const uint32_t a = tc::smem_u32(&bar);
+    if (threadIdx.x == 0) {
+        tc::mbar_init(a, 1);
+        tc::mbar_fence_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) (void)tc::mbar_wait(a, 0);
+    __syncthreads();
+}
+}  // namespace kda
+
 namespace {
 
 constexpr size_t kAlign = 256;
@@ -194,6 +211,13 @@ int kda_profile_kernels(int max_kernels, const char** names, int* launches, doub
         total_ms[i] += ms;
     }
     return n;
+}
+
+kda_status kda_selftest_timeout(kda_stream_t stream_)
+{
+    LaunchScope ls("selftest_timeout", (cudaStream_t)stream_);
+    selftest_timeout_kernel<<<1, 32, 0, (cudaStream_t)stream_>>>();
+    return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
 kda_status kda_check(kda_stream_t stream_)

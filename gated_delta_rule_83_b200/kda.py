@@ -30,6 +30,7 @@ ABI = {
     "kda_decode_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "kda_chunk_fwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
     "kda_check": (_I, [_P]),
+    "kda_selftest_timeout": (_I, [_P]),
     "kda_profile_begin": (_I, []),
     "kda_profile_end": (_I, []),
     "kda_profile_kernels": (_I, [_I, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(_I),

@@ -130,6 +130,15 @@ kda_status kda_decode_step(const void* q, const void* k, const void* v, const fl
 kda_status kda_check(kda_stream_t stream);
 
 /*
+ * kda_selftest_timeout -- exercises the failure path of the library's bounded device waits (no
+ * operator work): launches one small kernel that waits, with the same bounded wait the tensor-core
+ * kernels use, on a barrier nothing ever completes.  The wait gives up after ~0.2 s, records
+ * KDA_ERR_TIMEOUT in the device error word and the kernel exits normally; the next kda_check()
+ * returns KDA_ERR_TIMEOUT and clears the word.  The context stays usable.
+ */
+kda_status kda_selftest_timeout(kda_stream_t stream);
+
+/*
  * kda_chunk_fwd_noalloc -- kda_chunk_fwd for callers that cannot allocate device memory.
  *
  * The pages describe no counterpart: this is a deployment convenience of this library.  Some

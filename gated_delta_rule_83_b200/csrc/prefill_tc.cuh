@@ -629,7 +629,9 @@ tc_inter_kernel(const float* S0, float* S_final, __nv_bfloat16* __restrict__ out
     const uint32_t bar_full = smem_u32(sm + kB_Misc);   // kBStages barriers
     const uint32_t bar_d1 = bar_full + 8 * kBStages;    // [X; O'] ready
     const uint32_t bar_y = bar_d1 + 8;                  // Y ready
-    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + kB_Misc + 64);
+    const uint32_t bar_empty = bar_y + 8;               // kBStages barriers: stage consumed (128 arrivals)
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + kB_Misc + 128);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(sm + kB_Misc + 132);
 
     const int jb = off[n], je = off[n + 1], nch = je - jb;
     long long s0, s1;
@@ -639,7 +641,9 @@ tc_inter_kernel(const float* S0, float* S_final, __nv_bfloat16* __restrict__ out
         for (int s = 0; s < kBStages; ++s) mbar_init(bar_full + 8 * s, 1);
         mbar_init(bar_d1, 1);
         mbar_init(bar_y, 1);
+        for (int s = 0; s < kBStages; ++s) mbar_init(bar_empty + 8 * s, kBCompute);
         mbar_fence_init();
+        *s_abort = 0;
     }
     if (warp == 0) {
         tmem_alloc(smem_u32(s_tmem), 64);
@@ -671,86 +675,120 @@ tc_inter_kernel(const float* S0, float* S_final, __nv_bfloat16* __restrict__ out
     const uint32_t tw = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
     const uint32_t id_d1 = idesc_bf16(128, kTcNV, false, true);  // [W; Q'] S   (S MN-major)
     const uint32_t id_y = idesc_bf16(128, kTcNV, true, true);    // Kd^T U      (Kd, U MN-major)
+    // descriptor bases; per K step only the 14-bit start address field advances (never carries)
+    const uint64_t dS = desc_sw128(sb + kB_S, 128 * 128, 1024u), dU = desc_sw128(sb + kB_U, 64 * 128, 1024u);
     bool ok = true;
 
-    for (int it = 0; it < nch && ok; ++it) {
+    // Roles per chunk (no CTA-wide barrier inside the loop):
+    //   warp 4 (MMA)     : [X; O'] = [W; Q'] S once the S tile is ready (barrier 2), Y = Kd^T U once
+    //                      the U tile is ready (barrier 1)
+    //   warps 0-1        : U = Uv - X -> U tile, arrive on barrier 1
+    //   warps 2-3        : out = O' + O0
+    //   warps 0-3        : S <- e^{g_last} S + Y -> S tile; arrive on the stage's "empty" mbarrier
+    //                      (stage read) and on barrier 2 (S ready)
+    //   warp 5 (copies)  : refills the stage of chunk it with chunk it+3 once it is empty
+    // A bounded wait that gives up raises the CTA's abort flag; every later wait then fails at once,
+    // so the loop still runs its barriers to the end without hanging and exits quickly.
+    for (int it = 0; it < nch; ++it) {
         const int s = it % kBStages;
         const uint32_t st = sb + s * kStageBytes;
         const uint8_t* stp = sm + s * kStageBytes;
         const long long t0 = s0 + (long long)it * 64;
         const int L = (s1 - t0) < 64 ? (int)(s1 - t0) : 64;
         const uint32_t par = (uint32_t)it & 1u;
+        const bool refill = it + kBStages < nch;
         if (warp == 4) {
+            if (it > 0) named_sync(2, 160);  // S tile of this chunk written
             if (lane == 0) {
-                ok = mbar_wait(bar_full + 8 * s, (uint32_t)(it / kBStages) & 1u);
+                ok = ok && mbar_wait_ab(bar_full + 8 * s, (uint32_t)(it / kBStages) & 1u, s_abort);
                 fence_after_sync();
                 if (ok) {
+                    const uint64_t dA = desc_sw128(st + kStWQ, 16u, 1024u);
 #pragma unroll
                     for (int kk = 0; kk < 128; kk += 16)
-                        mma_bf16(tmem + kTmD1, desc_kmajor(st + kStWQ, 128, kk), desc_mnmajor(sb + kB_S, 128, kk), id_d1,
-                                 kk > 0);
+                        mma_bf16(tmem + kTmD1, dA + (uint64_t)((((kk >> 6) * 16384) + ((kk & 63) << 1)) >> 4),
+                                 dS + (uint64_t)((kk * 128) >> 4), id_d1, kk > 0);
                     mma_commit(bar_d1);
                 }
             }
             named_sync(1, 96);  // U tile written by warps 0 and 1
             if (lane == 0 && ok) {
                 fence_after_sync();
+                const uint64_t dK = desc_sw128(st + kStKd, 64 * 128, 1024u);
 #pragma unroll
                 for (int kk = 0; kk < 64; kk += 16)
-                    mma_bf16(tmem + kTmY, desc_mnmajor(st + kStKd, 64, kk), desc_mnmajor(sb + kB_U, 64, kk), id_y, kk > 0);
+                    mma_bf16(tmem + kTmY, dK + (uint64_t)((kk * 128) >> 4), dU + (uint64_t)((kk * 128) >> 4), id_y, kk > 0);
                 mma_commit(bar_y);
             }
-        } else if (warp < 4) {
-            ok = mbar_wait(bar_full + 8 * s, (uint32_t)(it / kBStages) & 1u);
-            ok = ok && mbar_wait(bar_d1, par);
+        } else if (warp == 5) {
+            if (refill && lane == 0) {  // stage s fully consumed (128 compute-thread arrivals) -> refill
+                ok = ok && mbar_wait_ab(bar_empty + 8 * s, (uint32_t)(it / kBStages) & 1u, s_abort);
+                if (ok)
+                    tc_issue_stage(st, bar_full + 8 * s, slots + ((size_t)(jb + it + kBStages) * H + h) * kSlotBytes, vt);
+            }
+        } else {
+            ok = ok && mbar_wait_ab(bar_full + 8 * s, (uint32_t)(it / kBStages) & 1u, s_abort);
+            ok = ok && mbar_wait_ab(bar_d1, par, s_abort);
             fence_after_sync();
             float x[32];
             tmem_ld16(tw + kTmD1, x);
             tmem_ld16(tw + kTmD1 + 16, x + 16);
             tmem_wait_ld();
             if (warp < 2) {  // U = Uv - X, row r = c
+                uint4 raw[4];
+#pragma unroll
+                for (int m = 0; m < 4; ++m) raw[m] = *reinterpret_cast<const uint4*>(stp + kStUv + slice_chunk_off(c, m));
+                uint4 pk[4];
 #pragma unroll
                 for (int m = 0; m < 4; ++m) {
                     float u[8];
-                    unpack8(*reinterpret_cast<const uint4*>(stp + kStUv + slice_chunk_off(c, m)), u);
+                    unpack8(raw[m], u);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) u[e] -= x[8 * m + e];
-                    *reinterpret_cast<uint4*>(sm + kB_U + sw128_chunk_off(c, m, 64)) = pack8(u);
+                    pk[m] = pack8(u);
                 }
+#pragma unroll
+                for (int m = 0; m < 4; ++m) *reinterpret_cast<uint4*>(sm + kB_U + sw128_chunk_off(c, m, 64)) = pk[m];
                 fence_proxy_async();
                 named_arrive(1, 96);
             } else {  // out = O' + O0, row r = c - 64
                 const int r = c - 64;
+                uint4 raw[4];
+#pragma unroll
+                for (int m = 0; m < 4; ++m) raw[m] = *reinterpret_cast<const uint4*>(stp + kStO0 + slice_chunk_off(r & 63, m));
                 if (r < L && ok) {
                     uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)(t0 + r) * H + h) * 128 + v0);
 #pragma unroll
                     for (int m = 0; m < 4; ++m) {
                         float u[8];
-                        unpack8(*reinterpret_cast<const uint4*>(stp + kStO0 + slice_chunk_off(r, m)), u);
+                        unpack8(raw[m], u);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) u[e] += x[8 * m + e];
                         dst[m] = pack8(u);
                     }
                 }
             }
-            ok = ok && mbar_wait(bar_y, par);
+            const float gam = *reinterpret_cast<const float*>(stp + kStGam + 4 * c);
+            ok = ok && mbar_wait_ab(bar_y, par, s_abort);
             fence_after_sync();
+            if (refill) mbar_arrive(bar_empty + 8 * s);  // last read of stage s done (MMAs on it complete)
             float y[32];
             tmem_ld16(tw + kTmY, y);
             tmem_ld16(tw + kTmY + 16, y + 16);
             tmem_wait_ld();
-            const float gam = *reinterpret_cast<const float*>(stp + kStGam + 4 * c);
 #pragma unroll
             for (int m = 0; m < kTcNV; ++m) S[m] = fmaf(gam, S[m], y[m]);
+            uint4 pk[4];
 #pragma unroll
-            for (int m = 0; m < 4; ++m) *reinterpret_cast<uint4*>(sm + kB_S + sw128_chunk_off(c, m, 128)) = pack8(S + 8 * m);
+            for (int m = 0; m < 4; ++m) pk[m] = pack8(S + 8 * m);
+#pragma unroll
+            for (int m = 0; m < 4; ++m) *reinterpret_cast<uint4*>(sm + kB_S + sw128_chunk_off(c, m, 128)) = pk[m];
             fence_proxy_async();
+            fence_before_sync();
+            if (it + 1 < nch) named_arrive(2, 160);  // S tile ready for the next chunk
         }
-        fence_before_sync();
-        ok = __syncthreads_and(ok);
-        if (warp == 5 && lane == 0 && ok && it + kBStages < nch)
-            tc_issue_stage(st, bar_full + 8 * s, slots + ((size_t)(jb + it + kBStages) * H + h) * kSlotBytes, vt);
     }
+    ok = __syncthreads_and(ok && !*s_abort);
     if (warp < 4 && S_final && ok) {
 #pragma unroll
         for (int m = 0; m < kTcNV; m += 4)

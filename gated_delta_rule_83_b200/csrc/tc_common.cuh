@@ -119,6 +119,10 @@ __device__ __forceinline__ void mbar_init(uint32_t addr, uint32_t count)
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(addr), "r"(count) : "memory");
 }
 __device__ __forceinline__ void mbar_fence_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+__device__ __forceinline__ void mbar_arrive(uint32_t addr)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(addr) : "memory");
+}
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t addr, uint32_t bytes)
 {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(addr), "r"(bytes) : "memory");
@@ -144,6 +148,21 @@ __device__ __forceinline__ bool mbar_wait(uint32_t addr, uint32_t parity)
     while (clock64() - start < 400000000LL)
         if (mbar_try_wait(addr, parity)) return true;
     set_error(KDA_ERR_TIMEOUT);
+    return false;
+}
+
+// As mbar_wait, but also gives up at once when *abort is set, and sets it when it gives up itself:
+// after one wait in a CTA times out, every later wait in that CTA returns false immediately.
+__device__ __forceinline__ bool mbar_wait_ab(uint32_t addr, uint32_t parity, volatile int* abort)
+{
+    if (mbar_try_wait(addr, parity)) return true;
+    const long long start = clock64();
+    while (clock64() - start < 400000000LL) {
+        if (mbar_try_wait(addr, parity)) return true;
+        if (*abort) return false;
+    }
+    set_error(KDA_ERR_TIMEOUT);
+    *abort = 1;
     return false;
 }
 

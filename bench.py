@@ -47,6 +47,7 @@ def parse():
     ap.add_argument("--only", choices=["prefill", "decode"], default=None,
                     help="run one part only (for profiling): no JSON contract line, prints that part's numbers")
     ap.add_argument("--decode-steps", type=int, default=None, help="decode steps to time (default 512)")
+    ap.add_argument("--no-extra", action="store_true", help="skip the varlen and 1M-token workloads")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override the prefill sequence length (profiling of a smaller case only)")
     return ap.parse_args()
@@ -163,13 +164,24 @@ def barrier(torch, world):
         dist.barrier()
 
 
-def max_over_ranks(torch, world, x):
+def max_over_ranks(torch, world, x, device="cuda"):
+    """Max of a per-rank scalar over all ranks (the slowest rank's time defines the job's time)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(world, units_per_rank_step, steps, max_ms):
+    """Whole-job throughput: every rank processes its own replica of the workload (weak scaling)."""
+    return world * units_per_rank_step * steps / (max_ms / 1e3)
+
+
+def replica_seed(seed, rank):
+    """Each rank draws an independent problem of the same shape."""
+    return seed + 1000 * rank
 
 
 # ------------------------------------------------------------------------------------------------
@@ -239,7 +251,7 @@ def run_ours(args):
             print(json.dumps(d), flush=True)
         return
 
-    inp = synth.prefill_inputs(w, device=dev, seed=w.seed + 1000 * rank, T=args.tokens)
+    inp = synth.prefill_inputs(w, device=dev, seed=replica_seed(w.seed, rank), T=args.tokens)
     q, k, v, la, beta, S0, cu = (inp[x] for x in ("q", "k", "v", "log_alpha", "beta", "S0", "cu_seqlens"))
     B, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -276,7 +288,7 @@ def run_ours(args):
     ms_local = e0.elapsed_time(e1)
     ms = max_over_ranks(torch, world, ms_local)
     ms_per_step = ms / args.steps
-    value = world * tokens * args.steps / (ms / 1e3)
+    value = job_throughput(world, tokens, args.steps, ms)
 
     # dominant kernel and roofline.  Algorithmic bytes of the prefill per token x head: q, k (bf16),
     # log_alpha (fp32), v (bf16), beta (fp32) read and out (bf16) written -- 1540 B at dk = dv = 128 --
@@ -344,8 +356,15 @@ def run_ours(args):
     except Exception as ex:  # pragma: no cover
         e2e = {"value": None, "unit": "tokens/s", "error": str(ex)[:200]}
 
-    del q, k, v, la, beta, out
+    del q, k, v, la, beta, out, inp
     torch.cuda.empty_cache()
+
+    extra = None
+    if not args.no_extra and args.only is None:
+        extra = {}
+        for name in ("varlen_64k", "long_1m"):
+            torch.cuda.empty_cache()
+            extra[name] = bench_prefill_workload(torch, kda, synth, dev, stream, world, rank, name, steps=3, warmup=2)
 
     decode = None
     if not args.no_decode and args.only is None:
@@ -364,6 +383,7 @@ def run_ours(args):
                        "chunk": 64, "parallelism": f"replicas x{world} (independent problems, no collective)",
                        "l2": f"inputs {in_bytes / 1e9:.2f} GB per step > L2 {L2_BYTES / 1e6:.0f} MB (no flush)"},
             "roofline": roofline, "kernels": {k_: {"launches": n, "ms": t} for k_, (n, t) in prof.items()},
+            "other_workloads": extra,
             "gpu_launches": launches, "clocks": clk, "e2e": e2e, "decode": decode, "cpu_baseline": cpu}
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -372,12 +392,48 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def bench_prefill_workload(torch, kda, synth, dev, stream, world, rank, name, steps, warmup):
+    """Device-timed throughput of another prefill workload (same method as the headline)."""
+    w = synth.WORKLOADS[name]
+    inp = synth.prefill_inputs(w, device=dev, seed=replica_seed(w.seed, rank))
+    q, k, v, la, beta, S0, cu = (inp[x] for x in ("q", "k", "v", "log_alpha", "beta", "S0", "cu_seqlens"))
+    out = torch.empty_like(v)
+    N = q.shape[0] if cu is None else cu.numel() - 1
+    S_fin = torch.empty((N, w.H, w.dk, w.dv), dtype=torch.float32, device=dev)
+    tokens = q.shape[0] * q.shape[1]
+
+    def step():
+        kda.chunk_fwd(q, k, v, la, beta, S0=S0, cu_seqlens=cu, out=out, S_final=S_fin)
+
+    for _ in range(warmup):
+        step()
+    kda.check()
+    barrier(torch, world)
+    torch.cuda.synchronize(dev)
+    kda.profile_begin()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    prof = kda.profile_end()
+    kda.check()
+    ms = max_over_ranks(torch, world, e0.elapsed_time(e1))
+    res = {"desc": w.desc, "tokens": tokens, "steps": steps, "ms_per_step": ms / steps,
+           "value": job_throughput(world, tokens, steps, ms), "unit": "tokens/s",
+           "kernels": {k_: {"launches": n, "ms": t} for k_, (n, t) in prof.items()}}
+    del inp, q, k, v, la, beta, S0, out, S_fin
+    return res
+
+
 def bench_decode(torch, kda, synth, dev, stream, world, rank, hbm, peak_kind, steps=None):
     w = synth.WORKLOADS["decode_256x512"]
     steps = steps or w.T
-    S = synth.decode_state(w, device=dev, seed=w.seed + 1000 * rank)
+    S = synth.decode_state(w, device=dev, seed=replica_seed(w.seed, rank))
     # per-step inputs, drawn fresh per step, pre-generated in HBM (one tensor per field with a step axis)
-    inp = synth.decode_inputs(w, 0, device=dev, steps=steps, seed=w.seed + 1000 * rank)
+    inp = synth.decode_inputs(w, 0, device=dev, steps=steps, seed=replica_seed(w.seed, rank))
     out = torch.empty((w.B, w.H, w.dv), dtype=torch.bfloat16, device=dev)
     fields = [inp[x] for x in ("q", "k", "v", "log_alpha", "beta")]
 
@@ -404,7 +460,7 @@ def bench_decode(torch, kda, synth, dev, stream, world, rank, hbm, peak_kind, st
     ach = alg / (kms / n / 1e3) / 1e9
     traffic, traffic_src = kernel_traffic("decode_step", pairs)
     return {"metric": "KDA decode tokens/s", "workload": w.name, "desc": w.desc,
-            "value": world * w.B * steps / (ms / 1e3), "unit": "tokens/s", "steps": steps,
+            "value": job_throughput(world, w.B, steps, ms), "unit": "tokens/s", "steps": steps,
             "us_per_step": ms * 1e3 / steps,
             "roofline": {"bound": "hbm", "kernel": "decode_step", "achieved": ach, "peak": hbm, "unit": "GB/s",
                          "frac": ach / hbm, "peak_source": f"{peak_kind} hbm_gbs (of {peak_kind})", "traffic": traffic,

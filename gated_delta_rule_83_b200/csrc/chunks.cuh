@@ -1,5 +1,10 @@
 // chunks.cuh -- per-sequence chunk table for the chunked prefill (regular batches and varlen).
 //
+// Besides the chunk offsets the kernel writes order[N]: the sequences sorted by length, longest
+// first (stable; identity for regular batches and for more than kOrderMax sequences).  The
+// sequential phase launches its CTAs in this order, so the longest chains start first and short
+// ones fill in behind them.
+//
 // Chunks never straddle a sequence boundary: sequence n of length len_n owns ceil(len_n / 64)
 // chunks, the last one possibly partial.  The table is off[n] = sum_{m<n} ceil(len_m / 64)
 // (off[N] = total) plus a header with the total and a "bad input" flag.  One CTA computes it
@@ -13,10 +18,13 @@
 namespace kda {
 
 constexpr int kTableThreads = 1024;
+constexpr int kOrderMax = 1024;
 
 __global__ void __launch_bounds__(kTableThreads)
-chunk_table_kernel(const int32_t* __restrict__ cu, int N, int Tseq, long long Ttot, WsHeader* hdr, int* off)
+chunk_table_kernel(const int32_t* __restrict__ cu, int N, int Tseq, long long Ttot, WsHeader* hdr, int* off,
+                   int* order)
 {
+    __shared__ int s_len[kOrderMax];
     __shared__ int s_warp[32];
     __shared__ int s_carry;
     __shared__ int s_bad;
@@ -61,6 +69,22 @@ chunk_table_kernel(const int32_t* __restrict__ cu, int N, int Tseq, long long Tt
         __syncthreads();
         if (tid == kTableThreads - 1) s_carry = excl + cnt;
         __syncthreads();
+    }
+    // longest-first order of the sequences
+    if (cu && !bad && N <= kOrderMax) {
+        for (int n = tid; n < N; n += kTableThreads) s_len[n] = cu[n + 1] - cu[n];
+        __syncthreads();
+        for (int i = tid; i < N; i += kTableThreads) {
+            const int li = s_len[i];
+            int rank = 0;
+            for (int jj = 0; jj < N; ++jj) {
+                const int lj = s_len[jj];
+                rank += (lj > li) || (lj == li && jj < i);
+            }
+            order[rank] = i;
+        }
+    } else {
+        for (int n = tid; n < N; n += kTableThreads) order[n] = n;
     }
     if (tid == 0) {
         off[N] = s_carry;

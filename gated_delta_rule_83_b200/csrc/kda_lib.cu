@@ -74,7 +74,7 @@ kda_status make_plan(int B, int T, int H, int dk, int dv, bool varlen, int num_s
     }
     if (p.Ttot > 0x7fffffffLL || p.N > 65535 * 64) return KDA_ERR_UNSUPPORTED;
     p.tc = use_tc_path(dt, dk, dv);
-    p.off_bytes = round_up(sizeof(int) * ((size_t)p.N + 1), kAlign);
+    p.off_bytes = round_up(sizeof(int) * (2 * (size_t)p.N + 1), kAlign);  // off[N+1] + order[N]
     p.slot_bytes = p.tc ? tc_slot_bytes() : round_up(sizeof(float) * simt_slot_floats(dk, dv), kAlign);
     p.total_bytes = sizeof(WsHeader) + p.off_bytes + (size_t)p.max_chunks * (size_t)H * p.slot_bytes;
     return KDA_OK;
@@ -134,7 +134,8 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const floa
 
     {
         LaunchScope ls("chunk_table", stream);
-        chunk_table_kernel<<<1, kTableThreads, 0, stream>>>(cu_seqlens, p.N, p.Tseq, p.Ttot, hdr, off);
+        chunk_table_kernel<<<1, kTableThreads, 0, stream>>>(cu_seqlens, p.N, p.Tseq, p.Ttot, hdr, off,
+                                                             off + p.N + 1);
         if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
     }
 

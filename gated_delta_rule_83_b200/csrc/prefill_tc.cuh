@@ -18,7 +18,8 @@
 //   A chunk in which some channel's gate spreads over more than e^160 (far outside any trained
 //   gate) computes A and P with exact per-element factors on CUDA cores instead.
 //
-// Phase B, one CTA per (sequence, head, 32-column slice of S), chunks in order.  Warp roles: four
+// Phase B, one CTA per (sequence, head, 32-column slice of S), chunks in order, longest sequences
+// launched first.  Warp roles: four
 // compute warps, one MMA-issue warp, one bulk-copy warp.  A 3-stage cp.async.bulk pipeline streams
 // each chunk's images into shared memory; per chunk
 //     [X; O'] = [W; Q'] S               tcgen05 M=128 N=32 K=128   (one 8-instruction batch)
@@ -621,7 +622,10 @@ tc_inter_kernel(const float* S0, float* S_final, __nv_bfloat16* __restrict__ out
 {
     using namespace tc;
     extern __shared__ uint8_t smem_raw[];
-    const int n = blockIdx.x, h = blockIdx.y, vt = blockIdx.z, v0 = vt * kTcNV;
+    // 1-D grid, longest sequences first: CTA L -> (sequence order[L / (4H)], head, 32-column slice)
+    const int L_cta = blockIdx.x, per_seq = 4 * H;
+    const int rank = L_cta / per_seq, rem = L_cta - rank * per_seq;
+    const int n = off[N + 1 + rank], h = rem >> 2, vt = rem & 3, v0 = vt * kTcNV;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (hdr->bad) return;
     uint8_t* sm = align1024(smem_raw);
@@ -817,7 +821,9 @@ inline cudaError_t launch_tc_prefill(const void* q, const void* k, const void* v
         if (e != cudaSuccess) return e;
     }
     LaunchScope ls("tc_inter", stream);
-    tc_inter_kernel<<<dim3(N, H, 128 / kTcNV), kBThreads, kB_Smem, stream>>>(
+    const long long nb = (long long)N * H * (128 / kTcNV);
+    if (nb > 0x7fffffffLL) return cudaErrorInvalidValue;
+    tc_inter_kernel<<<(unsigned)nb, kBThreads, kB_Smem, stream>>>(
         S0, S_final, (__nv_bfloat16*)out, hdr, off, cu, Tseq, N, H, (const uint8_t*)slots);
     return cudaGetLastError();
 }

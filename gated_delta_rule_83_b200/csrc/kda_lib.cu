@@ -142,7 +142,7 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const floa
     cudaError_t e;
     if (p.tc) {
         e = launch_tc_prefill(q, k, v, log_alpha, beta, S0, S_final, out, hdr, off, cu_seqlens, p.Tseq, p.N, H,
-                              p.max_chunks, slots, stream);
+                              p.max_chunks, p.Ttot, slots, stream);
     } else if (dt == KDA_BF16) {
         e = launch_simt_prefill<__nv_bfloat16>(q, k, v, log_alpha, beta, S0, S_final, out, hdr, off, cu_seqlens,
                                                p.Tseq, p.N, H, dk, dv, p.max_chunks, (float*)slots, stream);

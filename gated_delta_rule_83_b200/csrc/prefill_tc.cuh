@@ -29,6 +29,8 @@
 // which equals O = Qg S + P U with U = Uv - W S, the chunk form of o_t = S_t^T q_t.
 #pragma once
 
+#include <cuda.h>  // CUtensorMap and its enums (the encoder is fetched through the runtime)
+
 #include "common.cuh"
 #include "profile.cuh"
 #include "tc_common.cuh"
@@ -38,19 +40,19 @@ namespace kda {
 constexpr bool kTcPathReady = true;
 
 // ---- workspace slot of one (chunk, head), bytes ------------------------------------------------
-constexpr uint32_t kSlotWQ = 0;         // [W; Q'] [128 x 128] bf16, SW128 tile (2 atom columns of 16 KB)
-constexpr uint32_t kSlotKd = 32768;     // Kd      [64 x 128]  bf16, SW128 tile (MN-major A operand of Kd^T U)
-constexpr uint32_t kSlotUv = 49152;     // Uv      [4 slices][64][32] bf16, slice layout (slice_chunk_off)
-constexpr uint32_t kSlotO0 = 65536;     // O0      [4 slices][64][32] bf16, slice layout (slice_chunk_off)
+// Every image is a 64-row SW128 tile, bf16 [64 x 128] (two 8 KB atom columns), exactly as phase A
+// holds it in shared memory, so phase A writes each with bulk copies.
+constexpr uint32_t kSlotW = 0;          // W
+constexpr uint32_t kSlotQ = 16384;      // Q'
+constexpr uint32_t kSlotKd = 32768;     // Kd  (MN-major A operand of Kd^T U)
+constexpr uint32_t kSlotUv = 49152;     // Uv
+constexpr uint32_t kSlotO0 = 65536;     // O0
 constexpr uint32_t kSlotGam = 81920;    // e^{g_last} [128] fp32
 constexpr uint32_t kSlotBytes = 82432;
 inline size_t tc_slot_bytes() { return kSlotBytes; }
 
 constexpr int kTcNV = 32;               // state columns per phase-B CTA
 
-// Slice images ([64 rows][32 columns] bf16, 64-byte rows): 16-byte chunk m of row r is stored at
-// chunk position m ^ ((r >> 1) & 3), so eight consecutive rows read chunk by chunk hit distinct banks.
-__host__ __device__ __forceinline__ uint32_t slice_chunk_off(int r, int m) { return (uint32_t)(r * 64 + ((m ^ ((r >> 1) & 3)) << 4)); }
 constexpr float kTcFactorSpread = 160.f;
 
 // ------------------------------------------------------------------------------------------------
@@ -183,20 +185,30 @@ __device__ __forceinline__ void ut_inverse_64(const float* __restrict__ sA, floa
 // Phase A
 // ------------------------------------------------------------------------------------------------
 constexpr int kAThreads = 256;
-constexpr uint32_t kA_K = 0;         // k -> Kf (wide: k e^g) -> W bf16 tile           16 KB  } B operand of
-constexpr uint32_t kA_V = 16384;     // v                  -> Uv bf16 tile             16 KB  } P [W | Uv]
-constexpr uint32_t kA_Q = 32768;     // q -> Qf (wide: q e^g)                          16 KB
-constexpr uint32_t kA_Kb = 49152;    // Kb -> X fp32 [64][64] -> T bf16 [64][64]       16 KB
-constexpr uint32_t kA_G = 65536;     // log_alpha -> g fp32 [64][132] -> A fp32 [64][68] + scratch + P tile
+constexpr uint32_t kA_KQ = 0;        // [k; q] -> [Kf; Qf] stacked (128 rows, atom columns at 0 / 16384): 32 KB
+                                     //   later W in the k rows, Q' in the q rows
+constexpr uint32_t kA_V = 32768;     // v -> Uv -> O0 (64 rows, 16 KB)
+constexpr uint32_t kA_Kb = 49152;    // Kb -> Kd (scaled in place) -> X fp32 [64][64] -> T bf16 (16 KB)
+constexpr uint32_t kA_G = 65536;     // log_alpha -> g fp32 [64][128] -> A fp32 [64][68] + scratch + P tile (32 KB)
 constexpr uint32_t kA_Ysc = kA_G + 17408;   // solve scratch 32 x 33 fp32
 constexpr uint32_t kA_P = kA_G + 22528;     // P bf16 [64][64] tile (1024-aligned)
-constexpr uint32_t kA_Misc = kA_G + 33792;  // small arrays, TMEM address, flag, mbarrier (4 KB)
+constexpr uint32_t kA_Misc = kA_G + 32768;  // small arrays, TMEM address, flag, mbarrier (4 KB)
 constexpr uint32_t kA_Smem = kA_Misc + 4096 + 1024;  // + 1024 for aligning the dynamic base
-constexpr int kGS = 132;             // row stride of the g tile (floats)
+constexpr int kGS = 128;             // row stride of the g tile (floats)
+constexpr uint32_t kKQ_LBO = 16384;  // distance between the atom columns of the stacked [k; q] tile
+
+__device__ __forceinline__ void bulk_s2g(void* dst, uint32_t src_smem, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src_smem), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 __global__ void __launch_bounds__(kAThreads, 2)
-tc_intra_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-                const __nv_bfloat16* __restrict__ v, const float* __restrict__ log_alpha,
+tc_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_la,
                 const float* __restrict__ beta, const WsHeader* __restrict__ hdr, const int* __restrict__ off,
                 const int32_t* __restrict__ cu, int Tseq, int N, int H, uint8_t* __restrict__ slots)
 {
@@ -220,6 +232,7 @@ tc_intra_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + kA_Misc + 3328);
     int* s_wide = reinterpret_cast<int*>(sm + kA_Misc + 3332);
     const uint32_t mbar = smem_u32(sm + kA_Misc + 3344);
+    const uint32_t mbar_ld = smem_u32(sm + kA_Misc + 3352);
     float* sG = reinterpret_cast<float*>(sm + kA_G);
     float* sA = reinterpret_cast<float*>(sm + kA_G);                 // after the gating pass
     float* sY = reinterpret_cast<float*>(sm + kA_Ysc);
@@ -229,31 +242,38 @@ tc_intra_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
     if (tid == 0) {
         *s_wide = 0;
         mbar_init(mbar, 1);
+        mbar_init(mbar_ld, 1);
         mbar_fence_init();
+        // the chunk's k, q (into the stacked tile: atom column a = k rows then q rows), v and
+        // log_alpha: seven TMA boxes of 64 tokens; tokens past the tensor's end arrive as zeros
+        mbar_arrive_expect_tx(mbar_ld, 6 * 8192 + 32768);
+        const int tt = (int)t0;
+        tma_load_3d(sb + kA_KQ, &tm_k, 0, h, tt, mbar_ld);
+        tma_load_3d(sb + kA_KQ + 8192, &tm_q, 0, h, tt, mbar_ld);
+        tma_load_3d(sb + kA_KQ + kKQ_LBO, &tm_k, 64, h, tt, mbar_ld);
+        tma_load_3d(sb + kA_KQ + kKQ_LBO + 8192, &tm_q, 64, h, tt, mbar_ld);
+        tma_load_3d(sb + kA_V, &tm_v, 0, h, tt, mbar_ld);
+        tma_load_3d(sb + kA_V + 8192, &tm_v, 64, h, tt, mbar_ld);
+        tma_load_3d(sb + kA_G, &tm_la, 0, h, tt, mbar_ld);
     }
     if (warp == 0) {
         tmem_alloc(smem_u32(s_tmem), 256);
         tmem_relinquish();
     }
-    // raw k, q, v -> SW128 tiles; log_alpha -> g tile (rows >= L zero-filled: identity steps)
-    for (int e = tid; e < 64 * 16; e += kAThreads) {
-        const int r = e >> 4, ch = e & 15;
-        const uint32_t o = sw128_chunk_off(r, ch, 64);
-        const int rr = r < L ? r : 0;
-        const size_t gi = ((size_t)(t0 + rr) * H + h) * 128 + ch * 8;
-        const uint32_t nb = r < L ? 16u : 0u;
-        cp_async16(sb + kA_K + o, k + gi, nb);
-        cp_async16(sb + kA_Q + o, q + gi, nb);
-        cp_async16(sb + kA_V + o, v + gi, nb);
-    }
-    for (int e = tid; e < 64 * 32; e += kAThreads) {
-        const int r = e >> 5, ch = e & 31;
-        const int rr = r < L ? r : 0;
-        cp_async16(sb + kA_G + r * (kGS * 4) + ch * 16, log_alpha + ((size_t)(t0 + rr) * H + h) * 128 + ch * 4,
-                   r < L ? 16u : 0u);
-    }
     if (tid < 64) cp_async4(sb + kA_Misc + 4 * tid, beta + (size_t)(t0 + (tid < L ? tid : 0)) * H + h, tid < L ? 4u : 0u);
     cp_async_wait_all();
+    __syncthreads();  // mbarrier initialised
+    bool ok = mbar_wait(mbar_ld, 0);
+    if (L < 64) {  // rows past the sequence (another sequence's tokens, or zeros): identity steps
+        for (int e = tid; e < (64 - L) * 16; e += kAThreads) {
+            const int r = L + (e >> 4), chh = e & 15;
+            *reinterpret_cast<uint4*>(sm + kA_KQ + sw128_chunk_off(r, chh, 128)) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(sm + kA_KQ + sw128_chunk_off(64 + r, chh, 128)) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(sm + kA_V + sw128_chunk_off(r, chh, 64)) = make_uint4(0, 0, 0, 0);
+        }
+        for (int e = tid; e < (64 - L) * 32; e += kAThreads)
+            *reinterpret_cast<float4*>(sG + (L + (e >> 5)) * kGS + 4 * (e & 31)) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     __syncthreads();
 
     // cumulative gate: thread (c, hf) scans rows 32*hf .. 32*hf+31 of channel c
@@ -308,30 +328,26 @@ tc_intra_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
     const bool wide = *s_wide != 0;
     const uint32_t tmem = *s_tmem;
     uint32_t phase = 0;
-    bool ok = true;
     const int ch = tid & 15, rb = tid >> 4;  // element-wise passes: chunk ch of rows rb + 16 jj
     const int wq = warp & 3;
     const int rowq = 16 * wq + (lane & 15);  // M = 64 accumulator row held by this lane (lane < 16)
     const uint32_t trow = tmem + ((uint32_t)(32 * wq) << 16);
 
     if (!wide) {
-        float ref8[8], D8[8];
+        float ref8[8];
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            ref8[m] = s_ref[8 * ch + m];
-            D8[m] = s_D[8 * ch + m];
-        }
+        for (int m = 0; m < 8; ++m) ref8[m] = s_ref[8 * ch + m];
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
             const int r = rb + 16 * jj;
-            const uint32_t o = sw128_chunk_off(r, ch, 64);
+            const uint32_t ok_ = sw128_chunk_off(r, ch, 128), oq = sw128_chunk_off(64 + r, ch, 128);
             float kv[8], qv[8];
-            unpack8(*reinterpret_cast<const uint4*>(sm + kA_K + o), kv);
-            unpack8(*reinterpret_cast<const uint4*>(sm + kA_Q + o), qv);
+            unpack8(*reinterpret_cast<const uint4*>(sm + kA_KQ + ok_), kv);
+            unpack8(*reinterpret_cast<const uint4*>(sm + kA_KQ + oq), qv);
             const float4 ga = *reinterpret_cast<const float4*>(sG + r * kGS + 8 * ch);
             const float4 gb = *reinterpret_cast<const float4*>(sG + r * kGS + 8 * ch + 4);
             const float g8[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
-            float kf[8], qf[8], kb[8], kd[8];
+            float kf[8], qf[8], kb[8];
 #pragma unroll
             for (int m = 0; m < 8; ++m) {
                 const float x = g8[m] - ref8[m];
@@ -339,58 +355,59 @@ tc_intra_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
                 kf[m] = kv[m] * ef;
                 qf[m] = qv[m] * ef;
                 kb[m] = kv[m] * eb;
-                kd[m] = kb[m] * D8[m];  // k e^{g_last - g}
             }
-            *reinterpret_cast<uint4*>(sm + kA_K + o) = pack8(kf);
-            *reinterpret_cast<uint4*>(sm + kA_Q + o) = pack8(qf);
-            *reinterpret_cast<uint4*>(sm + kA_Kb + o) = pack8(kb);
-            *reinterpret_cast<uint4*>(slot + kSlotKd + o) = pack8(kd);
+            *reinterpret_cast<uint4*>(sm + kA_KQ + ok_) = pack8(kf);
+            *reinterpret_cast<uint4*>(sm + kA_KQ + oq) = pack8(qf);
+            *reinterpret_cast<uint4*>(sm + kA_Kb + sw128_chunk_off(r, ch, 64)) = pack8(kb);
         }
         fence_proxy_async();
         __syncthreads();
-        if (tid == 0) {
+        if (tid == 0) {  // [A'; P'] = [Kf; Qf] Kb^T: one M = 128 batch
             fence_after_sync();
-            const uint32_t id = idesc_bf16(64, 64, false, false);
+            const uint32_t id = idesc_bf16(128, 64, false, false);
 #pragma unroll
-            for (int kk = 0; kk < 128; kk += 16) {
-                mma_bf16(tmem + 0, desc_kmajor(sb + kA_K, 64, kk), desc_kmajor(sb + kA_Kb, 64, kk), id, kk > 0);
-                mma_bf16(tmem + 64, desc_kmajor(sb + kA_Q, 64, kk), desc_kmajor(sb + kA_Kb, 64, kk), id, kk > 0);
-            }
+            for (int kk = 0; kk < 128; kk += 16)
+                mma_bf16(tmem + 0, desc_kmajor(sb + kA_KQ, 128, kk), desc_kmajor(sb + kA_Kb, 64, kk), id, kk > 0);
             mma_commit(mbar);
         }
         ok = mbar_wait(mbar, phase);
         phase ^= 1;
         fence_after_sync();
-        if (warp < 4) {  // A' rows -> A (fp32, diag(beta), strictly lower)
-            const float br = s_beta[rowq];
+        {   // warps 0,1 (and 4,5): A' rows 0..63; warps 2,3 (and 6,7): P' rows; warps < 4 columns 0..31, >= 4 32..63
+            const int col0 = (warp >> 2) * 32;
+            float a[32];
+            tmem_ld16(tmem + ((uint32_t)(32 * wq) << 16) + col0, a);
+            tmem_ld16(tmem + ((uint32_t)(32 * wq) << 16) + col0 + 16, a + 16);
+            tmem_wait_ld();
+            if (wq < 2) {
+                const int r = 32 * wq + lane;
+                const float br = s_beta[r];
 #pragma unroll
-            for (int blk = 0; blk < 4; ++blk) {
-                float a[16];
-                tmem_ld16(trow + blk * 16, a);
-                tmem_wait_ld();
-                if (lane < 16) {
-#pragma unroll
-                    for (int m = 0; m < 16; m += 4) {
-                        const int i = blk * 16 + m;
-                        *reinterpret_cast<float4*>(sA + rowq * kAS + i) =
-                            make_float4(i < rowq ? br * a[m] : 0.f, i + 1 < rowq ? br * a[m + 1] : 0.f,
-                                        i + 2 < rowq ? br * a[m + 2] : 0.f, i + 3 < rowq ? br * a[m + 3] : 0.f);
-                    }
+                for (int m = 0; m < 32; m += 4) {
+                    const int i = col0 + m;
+                    *reinterpret_cast<float4*>(sA + r * kAS + i) =
+                        make_float4(i < r ? br * a[m] : 0.f, i + 1 < r ? br * a[m + 1] : 0.f,
+                                    i + 2 < r ? br * a[m + 2] : 0.f, i + 3 < r ? br * a[m + 3] : 0.f);
                 }
-            }
-        } else {  // P' rows -> P (bf16 K-major tile, lower triangle incl. diagonal)
+            } else {
+                const int r = 32 * (wq - 2) + lane;
 #pragma unroll
-            for (int blk = 0; blk < 4; ++blk) {
-                float a[16];
-                tmem_ld16(trow + 64 + blk * 16, a);
-                tmem_wait_ld();
-                if (lane < 16) {
+                for (int m = 0; m < 32; ++m) a[m] = (col0 + m <= r) ? a[m] : 0.f;
 #pragma unroll
-                    for (int m = 0; m < 16; ++m) a[m] = (blk * 16 + m <= rowq) ? a[m] : 0.f;
-                    *reinterpret_cast<uint4*>(sm + kA_P + sw128_chunk_off(rowq, 2 * blk, 64)) = pack8(a);
-                    *reinterpret_cast<uint4*>(sm + kA_P + sw128_chunk_off(rowq, 2 * blk + 1, 64)) = pack8(a + 8);
-                }
+                for (int m = 0; m < 4; ++m)
+                    *reinterpret_cast<uint4*>(sm + kA_P + sw128_chunk_off(r, (col0 >> 3) + m, 64)) = pack8(a + 8 * m);
             }
+        }
+        // Kd = Kb diag(e^{g_last - ref}) in place (Kb was consumed by the MMA above)
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            const int r = rb + 16 * jj;
+            uint4* p = reinterpret_cast<uint4*>(sm + kA_Kb + sw128_chunk_off(r, ch, 64));
+            float kb[8];
+            unpack8(*p, kb);
+#pragma unroll
+            for (int m = 0; m < 8; ++m) kb[m] *= s_D[8 * ch + m];
+            *p = pack8(kb);
         }
         fence_before_sync();
     } else {
@@ -403,23 +420,23 @@ tc_intra_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
             float a = 0.f, p = 0.f;
             if (i <= r) {
                 for (int cc = 0; cc < 128; ++cc) {
-                    const float kk = lds_bf16(sm + kA_K + sw128_off(i, cc, 64)) * expf(sG[r * kGS + cc] - sG[i * kGS + cc]);
-                    a = fmaf(lds_bf16(sm + kA_K + sw128_off(r, cc, 64)), kk, a);
-                    p = fmaf(lds_bf16(sm + kA_Q + sw128_off(r, cc, 64)), kk, p);
+                    const float kk = lds_bf16(sm + kA_KQ + sw128_off(i, cc, 128)) * expf(sG[r * kGS + cc] - sG[i * kGS + cc]);
+                    a = fmaf(lds_bf16(sm + kA_KQ + sw128_off(r, cc, 128)), kk, a);
+                    p = fmaf(lds_bf16(sm + kA_KQ + sw128_off(64 + r, cc, 128)), kk, p);
                 }
             }
             av[m] = (i < r) ? s_beta[r] * a : 0.f;
             pv[m] = p;
         }
         __syncthreads();  // every thread is done reading raw k and q across rows
-        // in place: k -> k e^g (B operand of W), q -> q e^g; Kd = k e^{g_last - g} to the image
+        // in place: k -> k e^g (B operand of W), q -> q e^g; Kd = k e^{g_last - g} into the Kb area
 #pragma unroll 1
         for (int jj = 0; jj < 4; ++jj) {
             const int r = rb + 16 * jj;
-            const uint32_t o = sw128_chunk_off(r, ch, 64);
+            const uint32_t ok_ = sw128_chunk_off(r, ch, 128), oq = sw128_chunk_off(64 + r, ch, 128);
             float kv[8], qv[8], kt[8], kd[8], qg[8];
-            unpack8(*reinterpret_cast<const uint4*>(sm + kA_K + o), kv);
-            unpack8(*reinterpret_cast<const uint4*>(sm + kA_Q + o), qv);
+            unpack8(*reinterpret_cast<const uint4*>(sm + kA_KQ + ok_), kv);
+            unpack8(*reinterpret_cast<const uint4*>(sm + kA_KQ + oq), qv);
 #pragma unroll
             for (int m = 0; m < 8; ++m) {
                 const float gv = sG[r * kGS + 8 * ch + m], gz = sG[63 * kGS + 8 * ch + m];
@@ -428,9 +445,9 @@ tc_intra_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
                 qg[m] = qv[m] * eg;
                 kd[m] = kv[m] * expf(gz - gv);
             }
-            *reinterpret_cast<uint4*>(sm + kA_K + o) = pack8(kt);
-            *reinterpret_cast<uint4*>(sm + kA_Q + o) = pack8(qg);
-            *reinterpret_cast<uint4*>(slot + kSlotKd + o) = pack8(kd);
+            *reinterpret_cast<uint4*>(sm + kA_KQ + ok_) = pack8(kt);
+            *reinterpret_cast<uint4*>(sm + kA_KQ + oq) = pack8(qg);
+            *reinterpret_cast<uint4*>(sm + kA_Kb + sw128_chunk_off(r, ch, 64)) = pack8(kd);
         }
         __syncthreads();  // g no longer read: A and the P tile take its place
         for (int cc = tid; cc < 128; cc += kAThreads) s_E[cc] = 1.f;
@@ -442,9 +459,16 @@ tc_intra_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
             *reinterpret_cast<__nv_bfloat16*>(sm + kA_P + sw128_off(r, i, 64)) = __float2bfloat16_rn(pv[m]);
         }
     }
+    fence_proxy_async();
     ok = __syncthreads_and(ok);
+    if (tid == 0) {  // Kd image out; the Kb area is free once the copy has read it
+        bulk_s2g(slot + kSlotKd, sb + kA_Kb, 16384);
+        bulk_commit();
+        bulk_wait_read();
+    }
+    __syncthreads();
 
-    // UT transform (X over Kb), then T = X diag(beta) as a bf16 K-major tile (also over Kb)
+    // UT transform (X over Kd), then T = X diag(beta) as a bf16 K-major tile (also over Kd)
     if (ok) ut_inverse_64(sA, sX, sY);
     uint4 tch[2];
 #pragma unroll
@@ -464,12 +488,14 @@ tc_intra_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
     }
     fence_proxy_async();
     __syncthreads();
-    if (ok && tid == 0) {  // [W' | Uv] = T [Kf | v]  (B operand: four atom columns over the K and V tiles)
+    if (ok && tid == 0) {  // W' = T Kf (B: k rows of the stacked tile), Uv = T v
         fence_after_sync();
-        const uint32_t id = idesc_bf16(64, 256, false, true);
+        const uint32_t id = idesc_bf16(64, 128, false, true);
 #pragma unroll
-        for (int kk = 0; kk < 64; kk += 16)
-            mma_bf16(tmem + 0, desc_kmajor(sb + kA_Kb, 64, kk), desc_mnmajor(sb + kA_K, 64, kk), id, kk > 0);
+        for (int kk = 0; kk < 64; kk += 16) {
+            mma_bf16(tmem + 0, desc_kmajor(sb + kA_Kb, 64, kk), desc_sw128(sb + kA_KQ + kk * 128, kKQ_LBO, 1024u), id, kk > 0);
+            mma_bf16(tmem + 128, desc_kmajor(sb + kA_Kb, 64, kk), desc_mnmajor(sb + kA_V, 64, kk), id, kk > 0);
+        }
         mma_commit(mbar);
     }
     if (ok) {
@@ -479,48 +505,32 @@ tc_intra_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
     }
     ok = __syncthreads_and(ok);
     if (ok) {
-        if (warp < 4) {  // W = W' diag(e^ref): image rows 0..63 of [W; Q'] and the W tile (over Kf)
+        if (warp < 4) {  // W = W' diag(e^ref) -> the k rows of the stacked tile (Kf consumed)
 #pragma unroll
             for (int b2 = 0; b2 < 8; b2 += 2) {
                 float a2[32];
                 tmem_ld16(trow + b2 * 16, a2);
                 tmem_ld16(trow + b2 * 16 + 16, a2 + 16);
                 tmem_wait_ld();
+                if (lane < 16) {
 #pragma unroll
-                for (int hb = 0; hb < 2; ++hb) {
-                    const int blk = b2 + hb;
-                    float* a = a2 + 16 * hb;
-                    if (lane < 16) {
+                    for (int m = 0; m < 32; ++m) a2[m] *= s_E[b2 * 16 + m];
 #pragma unroll
-                        for (int m = 0; m < 16; ++m) a[m] *= s_E[blk * 16 + m];
-                        const uint4 p0 = pack8(a), p1 = pack8(a + 8);
-                        *reinterpret_cast<uint4*>(slot + kSlotWQ + sw128_chunk_off(rowq, 2 * blk, 128)) = p0;
-                        *reinterpret_cast<uint4*>(slot + kSlotWQ + sw128_chunk_off(rowq, 2 * blk + 1, 128)) = p1;
-                        *reinterpret_cast<uint4*>(sm + kA_K + sw128_chunk_off(rowq, 2 * blk, 64)) = p0;
-                        *reinterpret_cast<uint4*>(sm + kA_K + sw128_chunk_off(rowq, 2 * blk + 1, 64)) = p1;
-                    }
+                    for (int m = 0; m < 4; ++m)
+                        *reinterpret_cast<uint4*>(sm + kA_KQ + sw128_chunk_off(rowq, 2 * b2 + m, 128)) = pack8(a2 + 8 * m);
                 }
             }
-        } else {  // Uv -> image [slice][64][32] and the Uv tile (over v)
+        } else {  // Uv -> the v tile (v consumed)
 #pragma unroll
             for (int b2 = 0; b2 < 8; b2 += 2) {
                 float a2[32];
                 tmem_ld16(trow + 128 + b2 * 16, a2);
                 tmem_ld16(trow + 128 + b2 * 16 + 16, a2 + 16);
                 tmem_wait_ld();
+                if (lane < 16) {
 #pragma unroll
-                for (int hb = 0; hb < 2; ++hb) {
-                    const int blk = b2 + hb;
-                    float* a = a2 + 16 * hb;
-                    if (lane < 16) {
-                        const uint4 p0 = pack8(a), p1 = pack8(a + 8);
-                        const int col = blk * 16, sl = col >> 5, m0 = (col & 31) >> 3;
-                        uint8_t* dst = slot + kSlotUv + (size_t)sl * 4096;
-                        *reinterpret_cast<uint4*>(dst + slice_chunk_off(rowq, m0)) = p0;
-                        *reinterpret_cast<uint4*>(dst + slice_chunk_off(rowq, m0 + 1)) = p1;
-                        *reinterpret_cast<uint4*>(sm + kA_V + sw128_chunk_off(rowq, 2 * blk, 64)) = p0;
-                        *reinterpret_cast<uint4*>(sm + kA_V + sw128_chunk_off(rowq, 2 * blk + 1, 64)) = p1;
-                    }
+                    for (int m = 0; m < 4; ++m)
+                        *reinterpret_cast<uint4*>(sm + kA_V + sw128_chunk_off(rowq, 2 * b2 + m, 64)) = pack8(a2 + 8 * m);
                 }
             }
         }
@@ -528,13 +538,21 @@ tc_intra_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
     fence_proxy_async();
     fence_before_sync();
     ok = __syncthreads_and(ok);
-    if (ok && tid == 0) {  // [P W | P Uv] = P [W | Uv]  (B operand: four atom columns over the W and Uv tiles)
+    if (ok && tid == 0) {
+        // W and Uv images out (bulk), then [P W | P Uv] = P [W | Uv]
+        bulk_s2g(slot + kSlotW, sb + kA_KQ, 8192);
+        bulk_s2g(slot + kSlotW + 8192, sb + kA_KQ + kKQ_LBO, 8192);
+        bulk_s2g(slot + kSlotUv, sb + kA_V, 16384);
+        bulk_commit();
         fence_after_sync();
-        const uint32_t id = idesc_bf16(64, 256, false, true);
+        const uint32_t id = idesc_bf16(64, 128, false, true);
 #pragma unroll
-        for (int kk = 0; kk < 64; kk += 16)
-            mma_bf16(tmem + 0, desc_kmajor(sb + kA_P, 64, kk), desc_mnmajor(sb + kA_K, 64, kk), id, kk > 0);
+        for (int kk = 0; kk < 64; kk += 16) {
+            mma_bf16(tmem + 0, desc_kmajor(sb + kA_P, 64, kk), desc_sw128(sb + kA_KQ + kk * 128, kKQ_LBO, 1024u), id, kk > 0);
+            mma_bf16(tmem + 128, desc_kmajor(sb + kA_P, 64, kk), desc_mnmajor(sb + kA_V, 64, kk), id, kk > 0);
+        }
         mma_commit(mbar);
+        bulk_wait_read();  // the Uv tile is overwritten by O0 below
     }
     if (ok) {
         ok = mbar_wait(mbar, phase);
@@ -542,51 +560,52 @@ tc_intra_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
     }
     ok = __syncthreads_and(ok);
     if (ok) {
-        if (warp < 4) {  // Q' = q e^g - P W -> image rows 64..127
+        if (warp < 4) {  // Q' = Qf e^ref - P W -> the q rows of the stacked tile, in place
 #pragma unroll
             for (int b2 = 0; b2 < 8; b2 += 2) {
                 float a2[32];
                 tmem_ld16(trow + b2 * 16, a2);
                 tmem_ld16(trow + b2 * 16 + 16, a2 + 16);
                 tmem_wait_ld();
+                if (lane < 16) {
 #pragma unroll
-                for (int hb = 0; hb < 2; ++hb) {
-                    const int blk = b2 + hb;
-                    float* a = a2 + 16 * hb;
-                    if (lane < 16) {
-                        float qf[16];
-                        unpack8(*reinterpret_cast<const uint4*>(sm + kA_Q + sw128_chunk_off(rowq, 2 * blk, 64)), qf);
-                        unpack8(*reinterpret_cast<const uint4*>(sm + kA_Q + sw128_chunk_off(rowq, 2 * blk + 1, 64)), qf + 8);
+                    for (int m = 0; m < 4; ++m) {
+                        uint4* p = reinterpret_cast<uint4*>(sm + kA_KQ + sw128_chunk_off(64 + rowq, 2 * b2 + m, 128));
+                        float qf[8];
+                        unpack8(*p, qf);
 #pragma unroll
-                        for (int m = 0; m < 16; ++m) a[m] = qf[m] * s_E[blk * 16 + m] - a[m];
-                        *reinterpret_cast<uint4*>(slot + kSlotWQ + sw128_chunk_off(64 + rowq, 2 * blk, 128)) = pack8(a);
-                        *reinterpret_cast<uint4*>(slot + kSlotWQ + sw128_chunk_off(64 + rowq, 2 * blk + 1, 128)) = pack8(a + 8);
+                        for (int e = 0; e < 8; ++e) qf[e] = qf[e] * s_E[b2 * 16 + 8 * m + e] - a2[8 * m + e];
+                        *p = pack8(qf);
                     }
                 }
             }
-        } else {  // O0 = P Uv -> image [slice][64][32]
+        } else {  // O0 = P Uv -> the v tile
 #pragma unroll
             for (int b2 = 0; b2 < 8; b2 += 2) {
                 float a2[32];
                 tmem_ld16(trow + 128 + b2 * 16, a2);
                 tmem_ld16(trow + 128 + b2 * 16 + 16, a2 + 16);
                 tmem_wait_ld();
+                if (lane < 16) {
 #pragma unroll
-                for (int hb = 0; hb < 2; ++hb) {
-                    const int blk = b2 + hb;
-                    float* a = a2 + 16 * hb;
-                    if (lane < 16) {
-                        const int col = blk * 16, sl = col >> 5, m0 = (col & 31) >> 3;
-                        uint8_t* dst = slot + kSlotO0 + (size_t)sl * 4096;
-                        *reinterpret_cast<uint4*>(dst + slice_chunk_off(rowq, m0)) = pack8(a);
-                        *reinterpret_cast<uint4*>(dst + slice_chunk_off(rowq, m0 + 1)) = pack8(a + 8);
-                    }
+                    for (int m = 0; m < 4; ++m)
+                        *reinterpret_cast<uint4*>(sm + kA_V + sw128_chunk_off(rowq, 2 * b2 + m, 64)) = pack8(a2 + 8 * m);
                 }
             }
         }
     }
+    fence_proxy_async();
     fence_before_sync();
     __syncthreads();
+    if (tid == 0) {  // Q' and O0 images out
+        if (ok) {
+            bulk_s2g(slot + kSlotQ, sb + kA_KQ + 8192, 8192);
+            bulk_s2g(slot + kSlotQ + 8192, sb + kA_KQ + kKQ_LBO + 8192, 8192);
+            bulk_s2g(slot + kSlotO0, sb + kA_V, 16384);
+            bulk_commit();
+        }
+        bulk_wait_all();
+    }
     if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
@@ -596,9 +615,11 @@ tc_intra_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
 constexpr int kBCompute = 128;              // 4 compute warps: thread c owns row c of the state slice
 constexpr int kBThreads = kBCompute + 64;   // + MMA-issue warp (4) + bulk-copy warp (5)
 constexpr int kBStages = 3;
-constexpr uint32_t kStWQ = 0, kStKd = 32768, kStUv = 49152, kStO0 = 53248, kStGam = 57344;
-constexpr uint32_t kStTx = 57856;           // bytes landing per stage
-constexpr uint32_t kStageBytes = 58368;     // 57 KB, 1024-aligned
+// stage: [W; Q'] stacked 128-row tile (32 KB) | Kd (16 KB) | the Uv and O0 atom columns holding this
+// CTA's 32-column slice (8 KB each) | e^{g_last} (512 B)
+constexpr uint32_t kStWQ = 0, kStKd = 32768, kStUv = 49152, kStO0 = 57344, kStGam = 65536;
+constexpr uint32_t kStTx = 66048;           // bytes landing per stage
+constexpr uint32_t kStageBytes = 66560;     // 65 KB, 1024-aligned
 constexpr uint32_t kB_S = kBStages * kStageBytes;  // S slice: bf16 [128 rows][64] SW128 (32 columns used)
 constexpr uint32_t kB_U = kB_S + 16384;            // U:       bf16 [64 rows][64]  SW128 (32 columns used)
 constexpr uint32_t kB_Misc = kB_U + 8192;          // mbarriers + TMEM address
@@ -609,9 +630,14 @@ __device__ __forceinline__ void tc_issue_stage(uint32_t stage_addr, uint32_t ful
 {
     using namespace tc;
     mbar_arrive_expect_tx(full_bar, kStTx);
-    bulk_g2s(stage_addr + kStWQ, slot + kSlotWQ, kSlotUv, full_bar);  // [W; Q'] and Kd, contiguous
-    bulk_g2s(stage_addr + kStUv, slot + kSlotUv + vt * 4096, 4096, full_bar);
-    bulk_g2s(stage_addr + kStO0, slot + kSlotO0 + vt * 4096, 4096, full_bar);
+    // [W; Q'] as one 128-row tile: atom column a holds W rows then Q' rows
+    bulk_g2s(stage_addr + kStWQ, slot + kSlotW, 8192, full_bar);
+    bulk_g2s(stage_addr + kStWQ + 8192, slot + kSlotQ, 8192, full_bar);
+    bulk_g2s(stage_addr + kStWQ + 16384, slot + kSlotW + 8192, 8192, full_bar);
+    bulk_g2s(stage_addr + kStWQ + 24576, slot + kSlotQ + 8192, 8192, full_bar);
+    bulk_g2s(stage_addr + kStKd, slot + kSlotKd, 16384, full_bar);
+    bulk_g2s(stage_addr + kStUv, slot + kSlotUv + (vt >> 1) * 8192, 8192, full_bar);
+    bulk_g2s(stage_addr + kStO0, slot + kSlotO0 + (vt >> 1) * 8192, 8192, full_bar);
     bulk_g2s(stage_addr + kStGam, slot + kSlotGam, 512, full_bar);
 }
 
@@ -626,6 +652,7 @@ tc_inter_kernel(const float* S0, float* S_final, __nv_bfloat16* __restrict__ out
     const int L_cta = blockIdx.x, per_seq = 4 * H;
     const int rank = L_cta / per_seq, rem = L_cta - rank * per_seq;
     const int n = off[N + 1 + rank], h = rem >> 2, vt = rem & 3, v0 = vt * kTcNV;
+    const int cq = 4 * (vt & 1);  // first 16-byte chunk of this slice inside its Uv / O0 atom column
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (hdr->bad) return;
     uint8_t* sm = align1024(smem_raw);
@@ -741,7 +768,7 @@ tc_inter_kernel(const float* S0, float* S_final, __nv_bfloat16* __restrict__ out
             if (warp < 2) {  // U = Uv - X, row r = c
                 uint4 raw[4];
 #pragma unroll
-                for (int m = 0; m < 4; ++m) raw[m] = *reinterpret_cast<const uint4*>(stp + kStUv + slice_chunk_off(c, m));
+                for (int m = 0; m < 4; ++m) raw[m] = *reinterpret_cast<const uint4*>(stp + kStUv + sw128_chunk_off(c, cq + m, 64));
                 uint4 pk[4];
 #pragma unroll
                 for (int m = 0; m < 4; ++m) {
@@ -759,7 +786,7 @@ tc_inter_kernel(const float* S0, float* S_final, __nv_bfloat16* __restrict__ out
                 const int r = c - 64;
                 uint4 raw[4];
 #pragma unroll
-                for (int m = 0; m < 4; ++m) raw[m] = *reinterpret_cast<const uint4*>(stp + kStO0 + slice_chunk_off(r & 63, m));
+                for (int m = 0; m < 4; ++m) raw[m] = *reinterpret_cast<const uint4*>(stp + kStO0 + sw128_chunk_off(r & 63, cq + m, 64));
                 if (r < L && ok) {
                     uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)(t0 + r) * H + h) * 128 + v0);
 #pragma unroll
@@ -803,20 +830,59 @@ tc_inter_kernel(const float* S0, float* S_final, __nv_bfloat16* __restrict__ out
     if (warp == 0) tmem_dealloc(tmem, 64);
 }
 
+// cuTensorMapEncodeTiled, fetched from the driver through the runtime (no link against libcuda)
+typedef CUresult (*TensorMapEncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                      const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                      CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline TensorMapEncodeFn tensor_map_encoder()
+{
+    static TensorMapEncodeFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        cudaDriverEntryPointQueryResult res;
+        void* p = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &res) == cudaSuccess &&
+            res == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<TensorMapEncodeFn>(p);
+    }
+    return fn;
+}
+
+// [tokens][H][128] row-major tensor as a 3-D map (d, head, token), box = 64 tokens x 1 head x box_d
+inline bool make_token_map(CUtensorMap* m, const void* base, bool bf16, int H, long long ntok, int box_d)
+{
+    TensorMapEncodeFn enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t esz = bf16 ? 2 : 4;
+    const cuuint64_t dims[3] = {128, (cuuint64_t)H, (cuuint64_t)ntok};
+    const cuuint64_t strides[2] = {128 * esz, 128 * esz * (cuuint64_t)H};
+    const cuuint32_t box[3] = {(cuuint32_t)box_d, 1, 64};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base),
+               dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               bf16 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 inline cudaError_t launch_tc_prefill(const void* q, const void* k, const void* v, const float* la, const float* beta,
                                      const float* S0, float* S_final, void* out, const WsHeader* hdr, const int* off,
-                                     const int32_t* cu, int Tseq, int N, int H, int max_chunks, char* slots,
-                                     cudaStream_t stream)
+                                     const int32_t* cu, int Tseq, int N, int H, int max_chunks, long long Ttot,
+                                     char* slots, cudaStream_t stream)
 {
     cudaError_t e = cudaFuncSetAttribute(tc_intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kA_Smem);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(tc_inter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kB_Smem);
     if (e != cudaSuccess) return e;
-    if (max_chunks > 0) {
+    if (max_chunks > 0 && Ttot > 0) {
+        alignas(64) CUtensorMap tq, tk, tv, tla;
+        if (!make_token_map(&tq, q, true, H, Ttot, 64) || !make_token_map(&tk, k, true, H, Ttot, 64) ||
+            !make_token_map(&tv, v, true, H, Ttot, 64) || !make_token_map(&tla, la, false, H, Ttot, 128))
+            return cudaErrorInvalidValue;
         LaunchScope ls("tc_intra", stream);
-        tc_intra_kernel<<<dim3(max_chunks, H), kAThreads, kA_Smem, stream>>>(
-            (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, la, beta, hdr, off, cu, Tseq, N,
-            H, (uint8_t*)slots);
+        tc_intra_kernel<<<dim3(max_chunks, H), kAThreads, kA_Smem, stream>>>(tq, tk, tv, tla, beta, hdr, off, cu, Tseq,
+                                                                               N, H, (uint8_t*)slots);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

@@ -175,6 +175,17 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst_smem, const void* src, uin
                  : "memory");
 }
 
+// ---- TMA tiled load (3-D tensor map), completion counted on an mbarrier -----------------------
+// The innermost coordinate c0 times the element size is always a multiple of 16 bytes here.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst_smem, const void* tmap, int c0, int c1, int c2, uint32_t mbar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::
+            "r"(dst_smem),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(mbar)
+        : "memory");
+}
+
 // ---- small helpers ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b)
 {

@@ -12,7 +12,7 @@ from gated_delta_rule_83_b200 import synth
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
-SLOT = dict(WQ=0, Kd=32768, Uv=49152, O0=65536, gam=81920, bytes=82432)
+SLOT = dict(W=0, Q=16384, Kd=32768, Uv=49152, O0=65536, gam=81920, bytes=82432)
 
 
 def sw128_off(r, c, R):
@@ -27,18 +27,6 @@ def decode_tile(buf, base, R, C):
             o = sw128_off(r, c, R)
             b = int(raw[o]) | (int(raw[o + 1]) << 8)
             out[r, c] = np.frombuffer(np.uint32(b << 16).tobytes(), np.float32)[0]
-    return out
-
-
-def decode_slices(buf, base):
-    """[4 slices][64 rows][32 cols] bf16; chunk m of row r stored at chunk position m ^ ((r >> 1) & 3)."""
-    out = np.zeros((64, 128), np.float32)
-    for sl in range(4):
-        raw = buf[base + sl * 4096:base + (sl + 1) * 4096]
-        for r in range(64):
-            for m in range(4):
-                o = r * 64 + ((m ^ ((r >> 1) & 3)) << 4)
-                out[r, sl * 32 + m * 8:sl * 32 + m * 8 + 8] = bf16_to_f32(raw[o:o + 16].copy())
     return out
 
 
@@ -81,17 +69,17 @@ def test_phase_a_images():
     kda.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], S0=d["S0"], workspace=ws)
     kda.check()
     buf = ws.cpu().numpy()
-    slots0 = 256 + 256   # header + chunk table (N+1 ints rounded to 256 B)
+    slots0 = 256 + 256   # header + chunk table and sequence order (2N+1 ints rounded to 256 B)
     H = 2
     for j, (t0, L) in enumerate([(0, 64), (64, 36)]):
         for h in range(H):
             base = slots0 + (j * H + h) * SLOT["bytes"]
             ex = expected_chunk(inp, t0, L, h)
-            WQ = decode_tile(buf, base + SLOT["WQ"], 128, 128)
-            Wg, Qp = WQ[:L], WQ[64:64 + L]
+            Wg = decode_tile(buf, base + SLOT["W"], 64, 128)[:L]
+            Qp = decode_tile(buf, base + SLOT["Q"], 64, 128)[:L]
             Kd = decode_tile(buf, base + SLOT["Kd"], 64, 128)[:L]
-            Uv = decode_slices(buf, base + SLOT["Uv"])[:L]
-            O0 = decode_slices(buf, base + SLOT["O0"])[:L]
+            Uv = decode_tile(buf, base + SLOT["Uv"], 64, 128)[:L]
+            O0 = decode_tile(buf, base + SLOT["O0"], 64, 128)[:L]
             gam = buf[base + SLOT["gam"]:base + SLOT["gam"] + 512].copy().view(np.float32)
             errs = dict(Qp=rel(Qp, ex["Qp"]), Kd=rel(Kd, ex["Kd"]), W=rel(Wg, ex["W"]), Uv=rel(Uv, ex["Uv"]),
                         O0=rel(O0, ex["O0"]), gam=rel(gam, ex["gam"]))

@@ -188,7 +188,7 @@ constexpr int kAThreads = 256;
 constexpr uint32_t kA_KQ = 0;        // [k; q] -> [Kf; Qf] stacked (128 rows, atom columns at 0 / 16384): 32 KB
                                      //   later W in the k rows, Q' in the q rows
 constexpr uint32_t kA_V = 32768;     // v -> Uv -> O0 (64 rows, 16 KB)
-constexpr uint32_t kA_Kb = 49152;    // Kb -> Kd (scaled in place) -> X fp32 [64][64] -> T bf16 (16 KB)
+constexpr uint32_t kA_Kb = 49152;    // Kb -> X fp32 [64][64] -> T bf16 (16 KB)
 constexpr uint32_t kA_G = 65536;     // log_alpha -> g fp32 [64][128] -> A fp32 [64][68] + scratch + P tile (32 KB)
 constexpr uint32_t kA_Ysc = kA_G + 17408;   // solve scratch 32 x 33 fp32
 constexpr uint32_t kA_P = kA_G + 22528;     // P bf16 [64][64] tile (1024-aligned)
@@ -215,10 +215,19 @@ tc_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     using namespace tc;
     extern __shared__ uint8_t smem_raw[];
     const int j = blockIdx.x, h = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    if (hdr->bad || j >= hdr->total_chunks) return;
     int n, L;
     long long t0;
-    locate_chunk(j, off, cu, Tseq, N, n, t0, L);
+    if (cu == nullptr) {  // regular batches of Tseq tokens: the chunk follows from j alone
+        const int cpb = (Tseq + kChunk - 1) / kChunk;
+        n = j / cpb;
+        const int c = j - n * cpb;
+        if (n >= N) return;
+        t0 = (long long)n * Tseq + (long long)c * kChunk;
+        L = min(kChunk, Tseq - c * kChunk);
+    } else {
+        if (hdr->bad || j >= hdr->total_chunks) return;
+        locate_chunk(j, off, cu, Tseq, N, n, t0, L);
+    }
 
     uint8_t* sm = align1024(smem_raw);
     const uint32_t sb = smem_u32(sm);
@@ -261,9 +270,9 @@ tc_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tmem_relinquish();
     }
     if (tid < 64) cp_async4(sb + kA_Misc + 4 * tid, beta + (size_t)(t0 + (tid < L ? tid : 0)) * H + h, tid < L ? 4u : 0u);
-    cp_async_wait_all();
     __syncthreads();  // mbarrier initialised
     bool ok = mbar_wait(mbar_ld, 0);
+    cp_async_wait_all();
     if (L < 64) {  // rows past the sequence (another sequence's tokens, or zeros): identity steps
         for (int e = tid; e < (64 - L) * 16; e += kAThreads) {
             const int r = L + (e >> 4), chh = e & 15;
@@ -330,13 +339,17 @@ tc_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     uint32_t phase = 0;
     const int ch = tid & 15, rb = tid >> 4;  // element-wise passes: chunk ch of rows rb + 16 jj
     const int wq = warp & 3;
-    const int rowq = 16 * wq + (lane & 15);  // M = 64 accumulator row held by this lane (lane < 16)
+    const int rowq = 16 * wq + (lane & 15);  // M = 64 accumulator row held by this thread
+    const int hc = (lane >> 4) * 64;         // ... and its half of the 128 columns
     const uint32_t trow = tmem + ((uint32_t)(32 * wq) << 16);
 
     if (!wide) {
-        float ref8[8];
+        float ref8[8], d8[8];
 #pragma unroll
-        for (int m = 0; m < 8; ++m) ref8[m] = s_ref[8 * ch + m];
+        for (int m = 0; m < 8; ++m) {
+            ref8[m] = s_ref[8 * ch + m];
+            d8[m] = s_D[8 * ch + m];
+        }
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
             const int r = rb + 16 * jj;
@@ -347,7 +360,7 @@ tc_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const float4 ga = *reinterpret_cast<const float4*>(sG + r * kGS + 8 * ch);
             const float4 gb = *reinterpret_cast<const float4*>(sG + r * kGS + 8 * ch + 4);
             const float g8[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
-            float kf[8], qf[8], kb[8];
+            float kf[8], qf[8], kb[8], kd[8];
 #pragma unroll
             for (int m = 0; m < 8; ++m) {
                 const float x = g8[m] - ref8[m];
@@ -355,10 +368,13 @@ tc_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 kf[m] = kv[m] * ef;
                 qf[m] = qv[m] * ef;
                 kb[m] = kv[m] * eb;
+                kd[m] = kb[m] * d8[m];
             }
+            const uint32_t okd = sw128_chunk_off(r, ch, 64);
             *reinterpret_cast<uint4*>(sm + kA_KQ + ok_) = pack8(kf);
             *reinterpret_cast<uint4*>(sm + kA_KQ + oq) = pack8(qf);
-            *reinterpret_cast<uint4*>(sm + kA_Kb + sw128_chunk_off(r, ch, 64)) = pack8(kb);
+            *reinterpret_cast<uint4*>(sm + kA_Kb + okd) = pack8(kb);
+            *reinterpret_cast<uint4*>(slot + kSlotKd + okd) = pack8(kd);  // Kd = Kb diag(e^{g_last - ref})
         }
         fence_proxy_async();
         __syncthreads();
@@ -398,17 +414,6 @@ tc_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     *reinterpret_cast<uint4*>(sm + kA_P + sw128_chunk_off(r, (col0 >> 3) + m, 64)) = pack8(a + 8 * m);
             }
         }
-        // Kd = Kb diag(e^{g_last - ref}) in place (Kb was consumed by the MMA above)
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-            const int r = rb + 16 * jj;
-            uint4* p = reinterpret_cast<uint4*>(sm + kA_Kb + sw128_chunk_off(r, ch, 64));
-            float kb[8];
-            unpack8(*p, kb);
-#pragma unroll
-            for (int m = 0; m < 8; ++m) kb[m] *= s_D[8 * ch + m];
-            *p = pack8(kb);
-        }
         fence_before_sync();
     } else {
         // some channel's gate spreads beyond e^160: exact per-element factors on CUDA cores
@@ -429,7 +434,7 @@ tc_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             pv[m] = p;
         }
         __syncthreads();  // every thread is done reading raw k and q across rows
-        // in place: k -> k e^g (B operand of W), q -> q e^g; Kd = k e^{g_last - g} into the Kb area
+        // in place: k -> k e^g (B operand of W), q -> q e^g; Kd = k e^{g_last - g} straight to the slot
 #pragma unroll 1
         for (int jj = 0; jj < 4; ++jj) {
             const int r = rb + 16 * jj;
@@ -447,7 +452,7 @@ tc_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             *reinterpret_cast<uint4*>(sm + kA_KQ + ok_) = pack8(kt);
             *reinterpret_cast<uint4*>(sm + kA_KQ + oq) = pack8(qg);
-            *reinterpret_cast<uint4*>(sm + kA_Kb + sw128_chunk_off(r, ch, 64)) = pack8(kd);
+            *reinterpret_cast<uint4*>(slot + kSlotKd + sw128_chunk_off(r, ch, 64)) = pack8(kd);
         }
         __syncthreads();  // g no longer read: A and the P tile take its place
         for (int cc = tid; cc < 128; cc += kAThreads) s_E[cc] = 1.f;
@@ -459,16 +464,9 @@ tc_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             *reinterpret_cast<__nv_bfloat16*>(sm + kA_P + sw128_off(r, i, 64)) = __float2bfloat16_rn(pv[m]);
         }
     }
-    fence_proxy_async();
-    ok = __syncthreads_and(ok);
-    if (tid == 0) {  // Kd image out; the Kb area is free once the copy has read it
-        bulk_s2g(slot + kSlotKd, sb + kA_Kb, 16384);
-        bulk_commit();
-        bulk_wait_read();
-    }
-    __syncthreads();
+    ok = __syncthreads_and(ok);  // A complete; Kb consumed
 
-    // UT transform (X over Kd), then T = X diag(beta) as a bf16 K-major tile (also over Kd)
+    // UT transform (X over Kb), then T = X diag(beta) as a bf16 K-major tile (also over Kb)
     if (ok) ut_inverse_64(sA, sX, sY);
     uint4 tch[2];
 #pragma unroll
@@ -507,31 +505,27 @@ tc_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (ok) {
         if (warp < 4) {  // W = W' diag(e^ref) -> the k rows of the stacked tile (Kf consumed)
 #pragma unroll
-            for (int b2 = 0; b2 < 8; b2 += 2) {
+            for (int b2 = 0; b2 < 64; b2 += 32) {
                 float a2[32];
-                tmem_ld16(trow + b2 * 16, a2);
-                tmem_ld16(trow + b2 * 16 + 16, a2 + 16);
+                tmem_ld16_pair<64>(trow + b2, a2);
+                tmem_ld16_pair<64>(trow + b2 + 16, a2 + 16);
                 tmem_wait_ld();
-                if (lane < 16) {
 #pragma unroll
-                    for (int m = 0; m < 32; ++m) a2[m] *= s_E[b2 * 16 + m];
+                for (int m = 0; m < 32; ++m) a2[m] *= s_E[hc + b2 + m];
 #pragma unroll
-                    for (int m = 0; m < 4; ++m)
-                        *reinterpret_cast<uint4*>(sm + kA_KQ + sw128_chunk_off(rowq, 2 * b2 + m, 128)) = pack8(a2 + 8 * m);
-                }
+                for (int m = 0; m < 4; ++m)
+                    *reinterpret_cast<uint4*>(sm + kA_KQ + sw128_chunk_off(rowq, (hc + b2) / 8 + m, 128)) = pack8(a2 + 8 * m);
             }
         } else {  // Uv -> the v tile (v consumed)
 #pragma unroll
-            for (int b2 = 0; b2 < 8; b2 += 2) {
+            for (int b2 = 0; b2 < 64; b2 += 32) {
                 float a2[32];
-                tmem_ld16(trow + 128 + b2 * 16, a2);
-                tmem_ld16(trow + 128 + b2 * 16 + 16, a2 + 16);
+                tmem_ld16_pair<64>(trow + 128 + b2, a2);
+                tmem_ld16_pair<64>(trow + 128 + b2 + 16, a2 + 16);
                 tmem_wait_ld();
-                if (lane < 16) {
 #pragma unroll
-                    for (int m = 0; m < 4; ++m)
-                        *reinterpret_cast<uint4*>(sm + kA_V + sw128_chunk_off(rowq, 2 * b2 + m, 64)) = pack8(a2 + 8 * m);
-                }
+                for (int m = 0; m < 4; ++m)
+                    *reinterpret_cast<uint4*>(sm + kA_V + sw128_chunk_off(rowq, (hc + b2) / 8 + m, 64)) = pack8(a2 + 8 * m);
             }
         }
     }
@@ -562,35 +556,31 @@ tc_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (ok) {
         if (warp < 4) {  // Q' = Qf e^ref - P W -> the q rows of the stacked tile, in place
 #pragma unroll
-            for (int b2 = 0; b2 < 8; b2 += 2) {
+            for (int b2 = 0; b2 < 64; b2 += 32) {
                 float a2[32];
-                tmem_ld16(trow + b2 * 16, a2);
-                tmem_ld16(trow + b2 * 16 + 16, a2 + 16);
+                tmem_ld16_pair<64>(trow + b2, a2);
+                tmem_ld16_pair<64>(trow + b2 + 16, a2 + 16);
                 tmem_wait_ld();
-                if (lane < 16) {
 #pragma unroll
-                    for (int m = 0; m < 4; ++m) {
-                        uint4* p = reinterpret_cast<uint4*>(sm + kA_KQ + sw128_chunk_off(64 + rowq, 2 * b2 + m, 128));
-                        float qf[8];
-                        unpack8(*p, qf);
+                for (int m = 0; m < 4; ++m) {
+                    uint4* p = reinterpret_cast<uint4*>(sm + kA_KQ + sw128_chunk_off(64 + rowq, (hc + b2) / 8 + m, 128));
+                    float qf[8];
+                    unpack8(*p, qf);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) qf[e] = qf[e] * s_E[b2 * 16 + 8 * m + e] - a2[8 * m + e];
-                        *p = pack8(qf);
-                    }
+                    for (int e = 0; e < 8; ++e) qf[e] = qf[e] * s_E[hc + b2 + 8 * m + e] - a2[8 * m + e];
+                    *p = pack8(qf);
                 }
             }
         } else {  // O0 = P Uv -> the v tile
 #pragma unroll
-            for (int b2 = 0; b2 < 8; b2 += 2) {
+            for (int b2 = 0; b2 < 64; b2 += 32) {
                 float a2[32];
-                tmem_ld16(trow + 128 + b2 * 16, a2);
-                tmem_ld16(trow + 128 + b2 * 16 + 16, a2 + 16);
+                tmem_ld16_pair<64>(trow + 128 + b2, a2);
+                tmem_ld16_pair<64>(trow + 128 + b2 + 16, a2 + 16);
                 tmem_wait_ld();
-                if (lane < 16) {
 #pragma unroll
-                    for (int m = 0; m < 4; ++m)
-                        *reinterpret_cast<uint4*>(sm + kA_V + sw128_chunk_off(rowq, 2 * b2 + m, 64)) = pack8(a2 + 8 * m);
-                }
+                for (int m = 0; m < 4; ++m)
+                    *reinterpret_cast<uint4*>(sm + kA_V + sw128_chunk_off(rowq, (hc + b2) / 8 + m, 64)) = pack8(a2 + 8 * m);
             }
         }
     }

@@ -108,6 +108,22 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v)
 #pragma unroll
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
+// M = 64 accumulators keep row r in lane (r % 16) + 32 (r / 16): the 16x32bx2 shape reads lanes
+// base .. base+15 twice, threads 0-15 at columns [taddr, +16) and threads 16-31 at columns
+// [taddr + OFF, +16), so every thread of the warp receives a row.
+template <int OFF>
+__device__ __forceinline__ void tmem_ld16_pair(uint32_t taddr, float* v)
+{
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16], %17;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+          "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr), "n"(OFF)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // generic-proxy shared-memory writes -> visible to the async proxy (tensor core, bulk copy)

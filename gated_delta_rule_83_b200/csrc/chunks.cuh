@@ -90,6 +90,7 @@ chunk_table_kernel(const int32_t* __restrict__ cu, int N, int Tseq, long long Tt
         off[N] = s_carry;
         hdr->total_chunks = s_carry;
         hdr->bad = bad;
+        hdr->next_unit = 0;
         if (bad) set_error(KDA_ERR_BAD_SEQLENS);
     }
 }

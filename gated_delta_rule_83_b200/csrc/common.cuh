@@ -30,7 +30,8 @@ constexpr int kChunk = 64;
 struct WsHeader {
     int total_chunks;   // sum over sequences of ceil(len / 64)
     int bad;            // nonzero: cu_seqlens malformed, nothing is computed
-    int pad[62];
+    int next_unit;      // work counter of the persistent intra-chunk kernel (zeroed with the table)
+    int pad[61];
 };
 
 // Map a global chunk index j (0 <= j < total) to (sequence n, first token t0, length L), with

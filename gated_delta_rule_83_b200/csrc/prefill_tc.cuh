@@ -4,12 +4,13 @@
 // chunk-parallel work inside a chunk, recurrent state passing between chunks, WY representation,
 // UT transform; chunk size 64), split into two kernels.
 //
-// Phase A, one CTA per (chunk, head), all chunks in parallel (256 threads):
-//   g_r = sum_{i<=r} log_alpha_i (fp32, restarted every chunk); ref_c = centre of channel c's range
+// Phase A, persistent (two 256-thread CTAs per SM), one (chunk, head) unit at a time per CTA, units
+// claimed from a work counter one ahead so that the next unit's inputs load during this one:
+//   g_r = sum_{i<=r} log_alpha_i (fp32, log2 units, restarted every chunk); ref_c = centre of channel c's range
 //   Kf = k e^{g-ref}, Qf = q e^{g-ref}, Kb = k e^{ref-g}   (bf16 operands; every factor <= e^80)
 //   A' = Kf Kb^T, P' = Qf Kb^T                          tcgen05 M=64 N=64 K=128, fp32 in TMEM
 //   A = strict_lower(diag(beta) A'), P = lower_incl(P')        (= the exact e^{g_r - g_i} products)
-//   T = (I + A)^{-1} diag(beta)                         fp32 recursive-doubling triangular inverse
+//   T = (I + A)^{-1} diag(beta)                         fp32 recursive-doubling triangular inverse (in place)
 //   [W' | Uv] = T [Kf | v], W = W' diag(e^ref)         tcgen05 M=64 N=256 K=64 (B operand MN-major)
 //   [P W | P Uv] = P [W | Uv]                           tcgen05 M=64 N=256 K=64
 //   Q' = q e^g - P W,  O0 = P Uv                        (the intra-chunk part of the output, folded in)
@@ -53,7 +54,7 @@ inline size_t tc_slot_bytes() { return kSlotBytes; }
 
 constexpr int kTcNV = 32;               // state columns per phase-B CTA
 
-constexpr float kTcFactorSpread = 160.f;
+constexpr float kTcFactorSpread = 230.f;  // log2 units (about e^159): every factor 2^(+-(g2 - ref2)) <= 2^115
 
 // ------------------------------------------------------------------------------------------------
 // small device helpers
@@ -101,38 +102,38 @@ __device__ __forceinline__ void named_arrive(int id, int threads)
 }
 
 // ------------------------------------------------------------------------------------------------
-// UT transform: X = (I + A)^{-1} for a strictly lower 64 x 64 A (fp32, row stride 68) by recursive
-// doubling: the four 16 x 16 diagonal blocks by forward substitution; then, inside each 32 x 32 half,
-// X_10 = -X_11 A_10 X_00; then the 32 x 32 off-diagonal block X_10 = -X_11 A_10 X_00 of the whole.
-// 256 threads.  X: row stride 64.  Y: scratch of 32 x 33 floats.
+// UT transform, in place: a strictly lower 64 x 64 A (fp32, row stride 68, zero on and above the
+// diagonal) is overwritten by X = (I + A)^{-1}, by recursive doubling: the four 16 x 16 diagonal
+// blocks by forward substitution; then, inside each 32 x 32 half, X_10 = -X_11 A_10 X_00; then the
+// 32 x 32 off-diagonal block X_10 = -X_11 A_10 X_00 of the whole.  256 threads.  Y: scratch of
+// 32 x 36 floats (16-byte aligned rows).
 // ------------------------------------------------------------------------------------------------
-constexpr int kAS = 68;  // row stride of A
-constexpr int kXS = 64;  // row stride of X
+constexpr int kAS = 68;  // row stride of A / X
 
-__device__ __forceinline__ void ut_inverse_64(const float* __restrict__ sA, float* __restrict__ sX, float* __restrict__ sY)
+__device__ __forceinline__ void ut_inverse_64_inplace(float* __restrict__ sA, float* __restrict__ sY)
 {
     const int tid = threadIdx.x;
-    // upper triangle blocks of X are zero
-    for (int e = tid; e < 64 * 64 / 4; e += 256) reinterpret_cast<float4*>(sX)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-    __syncthreads();
-    if (tid < 64) {  // diagonal 16 x 16 blocks: thread -> (block, column jj)
+    {   // diagonal 16 x 16 blocks: thread -> (block, column jj); written back once every block is read
         const int b = 16 * (tid >> 4), jj = tid & 15;
         float x[16];
+        if (tid < 64) {  // right-looking: once x_i is known, fold it into the partial sums of rows > i
+            float s[16];
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            float s0 = 0.f, s1 = 0.f;
+            for (int r = 0; r < 16; ++r) s[r] = 0.f;
 #pragma unroll
-            for (int i = 0; i + 1 < r; i += 2) {
-                s0 = fmaf(sA[(b + r) * kAS + b + i], x[i], s0);
-                s1 = fmaf(sA[(b + r) * kAS + b + i + 1], x[i + 1], s1);
+            for (int i = 0; i < 16; ++i) {
+                x[i] = (i == jj) ? 1.f : ((i < jj) ? 0.f : -s[i]);
+#pragma unroll
+                for (int r = i + 1; r < 16; ++r) s[r] = fmaf(sA[(b + r) * kAS + b + i], x[i], s[r]);
             }
-            if (r & 1) s0 = fmaf(sA[(b + r) * kAS + b + r - 1], x[r - 1], s0);
-            x[r] = (r == jj) ? 1.f : ((r < jj) ? 0.f : -(s0 + s1));
         }
+        __syncthreads();
+        if (tid < 64) {
 #pragma unroll
-        for (int r = 0; r < 16; ++r) sX[(b + r) * kXS + b + jj] = x[r];
+            for (int r = 0; r < 16; ++r) sA[(b + r) * kAS + b + jj] = x[r];
+        }
+        __syncthreads();
     }
-    __syncthreads();
     {   // level 1: blocks (1,0) and (3,2); thread -> (pair p, row rr, columns cc, cc+1)
         const int p = tid >> 7, rr = (tid >> 3) & 15, cc = (tid & 7) * 2;
         const int bi = 16 * (2 * p + 1), bj = 16 * (2 * p);
@@ -140,21 +141,21 @@ __device__ __forceinline__ void ut_inverse_64(const float* __restrict__ sA, floa
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
             const float a = sA[(bi + rr) * kAS + bj + k];
-            y0 = fmaf(a, sX[(bj + k) * kXS + bj + cc], y0);
-            y1 = fmaf(a, sX[(bj + k) * kXS + bj + cc + 1], y1);
+            const float2 xv = *reinterpret_cast<const float2*>(sA + (bj + k) * kAS + bj + cc);
+            y0 = fmaf(a, xv.x, y0);
+            y1 = fmaf(a, xv.y, y1);
         }
-        sY[(p * 16 + rr) * 33 + cc] = y0;
-        sY[(p * 16 + rr) * 33 + cc + 1] = y1;
-        __syncthreads();
+        *reinterpret_cast<float2*>(sY + (p * 16 + rr) * 34 + cc) = make_float2(y0, y1);
+        __syncthreads();  // A_10 read: X_10 takes its place
         float x0 = 0.f, x1 = 0.f;
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
-            const float xi = sX[(bi + rr) * kXS + bi + k];
-            x0 = fmaf(xi, sY[(p * 16 + k) * 33 + cc], x0);
-            x1 = fmaf(xi, sY[(p * 16 + k) * 33 + cc + 1], x1);
+            const float xi = sA[(bi + rr) * kAS + bi + k];
+            const float2 yv = *reinterpret_cast<const float2*>(sY + (p * 16 + k) * 34 + cc);
+            x0 = fmaf(xi, yv.x, x0);
+            x1 = fmaf(xi, yv.y, x1);
         }
-        sX[(bi + rr) * kXS + bj + cc] = -x0;
-        sX[(bi + rr) * kXS + bj + cc + 1] = -x1;
+        *reinterpret_cast<float2*>(sA + (bi + rr) * kAS + bj + cc) = make_float2(-x0, -x1);
         __syncthreads();
     }
     {   // level 2: rows 32..63, columns 0..31; thread -> (row rr, columns cc..cc+3)
@@ -163,20 +164,19 @@ __device__ __forceinline__ void ut_inverse_64(const float* __restrict__ sA, floa
 #pragma unroll
         for (int k = 0; k < 32; ++k) {
             const float a = sA[(32 + rr) * kAS + k];
-            const float4 xv = *reinterpret_cast<const float4*>(sX + k * kXS + cc);
+            const float4 xv = *reinterpret_cast<const float4*>(sA + k * kAS + cc);
             y[0] = fmaf(a, xv.x, y[0]); y[1] = fmaf(a, xv.y, y[1]); y[2] = fmaf(a, xv.z, y[2]); y[3] = fmaf(a, xv.w, y[3]);
         }
-#pragma unroll
-        for (int m = 0; m < 4; ++m) sY[rr * 33 + cc + m] = y[m];
+        *reinterpret_cast<float4*>(sY + rr * 36 + cc) = make_float4(y[0], y[1], y[2], y[3]);
         __syncthreads();
         float x[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int k = 0; k < 32; ++k) {
-            const float xi = sX[(32 + rr) * kXS + 32 + k];
-#pragma unroll
-            for (int m = 0; m < 4; ++m) x[m] = fmaf(xi, sY[k * 33 + cc + m], x[m]);
+            const float xi = sA[(32 + rr) * kAS + 32 + k];
+            const float4 yv = *reinterpret_cast<const float4*>(sY + k * 36 + cc);
+            x[0] = fmaf(xi, yv.x, x[0]); x[1] = fmaf(xi, yv.y, x[1]); x[2] = fmaf(xi, yv.z, x[2]); x[3] = fmaf(xi, yv.w, x[3]);
         }
-        *reinterpret_cast<float4*>(sX + (32 + rr) * kXS + cc) = make_float4(-x[0], -x[1], -x[2], -x[3]);
+        *reinterpret_cast<float4*>(sA + (32 + rr) * kAS + cc) = make_float4(-x[0], -x[1], -x[2], -x[3]);
         __syncthreads();
     }
 }
@@ -184,15 +184,20 @@ __device__ __forceinline__ void ut_inverse_64(const float* __restrict__ sA, floa
 // ------------------------------------------------------------------------------------------------
 // Phase A
 // ------------------------------------------------------------------------------------------------
+// Persistent: CTA b starts with (chunk, head) unit b (unit u = chunk * H + head) and claims each
+// further unit from a work counter one unit ahead, so that its inputs can be prefetched.
+// Each input buffer is refilled with the next unit's data as soon as the current unit is done with
+// it: v once MMA2 has read it, log_alpha once MMA3 has read P (the last tenant of its region), k and
+// q once the last images have left for the workspace.
 constexpr int kAThreads = 256;
-constexpr uint32_t kA_KQ = 0;        // [k; q] -> [Kf; Qf] stacked (128 rows, atom columns at 0 / 16384): 32 KB
-                                     //   later W in the k rows, Q' in the q rows
-constexpr uint32_t kA_V = 32768;     // v -> Uv -> O0 (64 rows, 16 KB)
-constexpr uint32_t kA_Kb = 49152;    // Kb -> X fp32 [64][64] -> T bf16 (16 KB)
-constexpr uint32_t kA_G = 65536;     // log_alpha -> g fp32 [64][128] -> A fp32 [64][68] + scratch + P tile (32 KB)
-constexpr uint32_t kA_Ysc = kA_G + 17408;   // solve scratch 32 x 33 fp32
+constexpr uint32_t kA_KQ = 0;        // 32 KB: [k; q] -> [Kf; Qf] stacked (128 rows, atom columns at 0 / 16384)
+                                     //   -> W in the k rows, Q' in the q rows
+constexpr uint32_t kA_V = 32768;     // 16 KB: v
+constexpr uint32_t kA_B = 49152;     // 16 KB: Kb -> T -> Uv -> O0
+constexpr uint32_t kA_G = 65536;     // 32 KB: log_alpha -> g fp32 [64][128] -> A / X fp32 [64][68] + scratch + P tile
+constexpr uint32_t kA_Ysc = kA_G + 17408;   // solve scratch 32 x 36 fp32
 constexpr uint32_t kA_P = kA_G + 22528;     // P bf16 [64][64] tile (1024-aligned)
-constexpr uint32_t kA_Misc = kA_G + 32768;  // small arrays, TMEM address, flag, mbarrier (4 KB)
+constexpr uint32_t kA_Misc = kA_G + 32768;  // small arrays, TMEM address, flags, mbarriers (4 KB)
 constexpr uint32_t kA_Smem = kA_Misc + 4096 + 1024;  // + 1024 for aligning the dynamic base
 constexpr int kGS = 128;             // row stride of the g tile (floats)
 constexpr uint32_t kKQ_LBO = 16384;  // distance between the atom columns of the stacked [k; q] tile
@@ -206,33 +211,45 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// (chunk, head) unit u = chunk * H + head -> head, sequence, first token, length
+__device__ __forceinline__ void tc_unit(long long u, int H, const int* __restrict__ off, const int32_t* __restrict__ cu,
+                                        int Tseq, int N, int& h, int& n, long long& t0, int& L)
+{
+    const long long j = u / H;
+    h = (int)(u - j * H);
+    if (cu == nullptr) {  // regular batches of Tseq tokens: the chunk follows from j alone
+        const int cpb = (Tseq + kChunk - 1) / kChunk;
+        n = (int)(j / cpb);
+        const int c = (int)(j - (long long)n * cpb);
+        t0 = (long long)n * Tseq + (long long)c * kChunk;
+        L = min(kChunk, Tseq - c * kChunk);
+    } else {
+        locate_chunk((int)j, off, cu, Tseq, N, n, t0, L);
+    }
+}
+
 __global__ void __launch_bounds__(kAThreads, 2)
 tc_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_la,
-                const float* __restrict__ beta, const WsHeader* __restrict__ hdr, const int* __restrict__ off,
+                const float* __restrict__ beta, WsHeader* __restrict__ hdr, const int* __restrict__ off,
                 const int32_t* __restrict__ cu, int Tseq, int N, int H, uint8_t* __restrict__ slots)
 {
     using namespace tc;
     extern __shared__ uint8_t smem_raw[];
-    const int j = blockIdx.x, h = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    int n, L;
-    long long t0;
-    if (cu == nullptr) {  // regular batches of Tseq tokens: the chunk follows from j alone
-        const int cpb = (Tseq + kChunk - 1) / kChunk;
-        n = j / cpb;
-        const int c = j - n * cpb;
-        if (n >= N) return;
-        t0 = (long long)n * Tseq + (long long)c * kChunk;
-        L = min(kChunk, Tseq - c * kChunk);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    long long nunits;
+    if (cu == nullptr) {
+        nunits = (long long)N * ((Tseq + kChunk - 1) / kChunk) * H;
     } else {
-        if (hdr->bad || j >= hdr->total_chunks) return;
-        locate_chunk(j, off, cu, Tseq, N, n, t0, L);
+        if (hdr->bad) return;
+        nunits = (long long)hdr->total_chunks * H;
     }
+    if ((long long)blockIdx.x >= nunits) return;
 
     uint8_t* sm = align1024(smem_raw);
     const uint32_t sb = smem_u32(sm);
     float* s_beta = reinterpret_cast<float*>(sm + kA_Misc);          // [64]
-    float* s_ref = reinterpret_cast<float*>(sm + kA_Misc + 256);     // [128]
+    float* s_ref = reinterpret_cast<float*>(sm + kA_Misc + 256);     // [128] (log2 units)
     float* s_E = reinterpret_cast<float*>(sm + kA_Misc + 768);       // [128] e^{ref} (1 in the wide case)
     float* s_D = reinterpret_cast<float*>(sm + kA_Misc + 1280);      // [128] e^{g_last - ref}
     float* s_carry = reinterpret_cast<float*>(sm + kA_Misc + 1792);  // [128] rows 0..31 total
@@ -240,362 +257,435 @@ tc_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     float* s_hi = reinterpret_cast<float*>(sm + kA_Misc + 2816);     // [128] rows 32..63 max
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + kA_Misc + 3328);
     int* s_wide = reinterpret_cast<int*>(sm + kA_Misc + 3332);
-    const uint32_t mbar = smem_u32(sm + kA_Misc + 3344);
-    const uint32_t mbar_ld = smem_u32(sm + kA_Misc + 3352);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(sm + kA_Misc + 3336);
+    const uint32_t mbar = smem_u32(sm + kA_Misc + 3344);     // MMA completions
+    const uint32_t mbar_la = smem_u32(sm + kA_Misc + 3352);  // log_alpha landed
+    const uint32_t mbar_kq = mbar_la + 8, mbar_v = mbar_la + 16;
+    // the unit after this one, claimed and decoded by thread 0: {u, t0} and {head, length}
+    long long* s_next = reinterpret_cast<long long*>(sm + kA_Misc + 3376);
+    int* s_next_hl = reinterpret_cast<int*>(sm + kA_Misc + 3392);
     float* sG = reinterpret_cast<float*>(sm + kA_G);
     float* sA = reinterpret_cast<float*>(sm + kA_G);                 // after the gating pass
     float* sY = reinterpret_cast<float*>(sm + kA_Ysc);
-    float* sX = reinterpret_cast<float*>(sm + kA_Kb);
-    uint8_t* slot = slots + ((size_t)j * H + h) * kSlotBytes;
 
+    // TMA boxes of 64 tokens of one head; tokens past the tensor's end arrive as zeros
+    auto issue_la = [&](int hh, long long tt) {
+        mbar_arrive_expect_tx(mbar_la, 32768);
+        tma_load_3d(sb + kA_G, &tm_la, 0, hh, (int)tt, mbar_la);
+    };
+    auto issue_kq = [&](int hh, long long tt) {  // stacked tile: atom column a = k rows then q rows
+        mbar_arrive_expect_tx(mbar_kq, 4 * 8192);
+        tma_load_3d(sb + kA_KQ, &tm_k, 0, hh, (int)tt, mbar_kq);
+        tma_load_3d(sb + kA_KQ + 8192, &tm_q, 0, hh, (int)tt, mbar_kq);
+        tma_load_3d(sb + kA_KQ + kKQ_LBO, &tm_k, 64, hh, (int)tt, mbar_kq);
+        tma_load_3d(sb + kA_KQ + kKQ_LBO + 8192, &tm_q, 64, hh, (int)tt, mbar_kq);
+    };
+    auto issue_v = [&](int hh, long long tt) {
+        mbar_arrive_expect_tx(mbar_v, 2 * 8192);
+        tma_load_3d(sb + kA_V, &tm_v, 0, hh, (int)tt, mbar_v);
+        tma_load_3d(sb + kA_V + 8192, &tm_v, 64, hh, (int)tt, mbar_v);
+    };
+    auto issue_beta = [&](int hh, long long tt, int LL) {  // threads 0..63; rows past the end read as 0
+        cp_async4(sb + kA_Misc + 4 * tid, beta + (size_t)(tt + (tid < LL ? tid : 0)) * H + hh, tid < LL ? 4u : 0u);
+    };
+
+    int h, n, L;
+    long long t0;
+    tc_unit(blockIdx.x, H, off, cu, Tseq, N, h, n, t0, L);
     if (tid == 0) {
-        *s_wide = 0;
+        *s_abort = 0;
         mbar_init(mbar, 1);
-        mbar_init(mbar_ld, 1);
+        mbar_init(mbar_la, 1);
+        mbar_init(mbar_kq, 1);
+        mbar_init(mbar_v, 1);
         mbar_fence_init();
-        // the chunk's k, q (into the stacked tile: atom column a = k rows then q rows), v and
-        // log_alpha: seven TMA boxes of 64 tokens; tokens past the tensor's end arrive as zeros
-        mbar_arrive_expect_tx(mbar_ld, 6 * 8192 + 32768);
-        const int tt = (int)t0;
-        tma_load_3d(sb + kA_KQ, &tm_k, 0, h, tt, mbar_ld);
-        tma_load_3d(sb + kA_KQ + 8192, &tm_q, 0, h, tt, mbar_ld);
-        tma_load_3d(sb + kA_KQ + kKQ_LBO, &tm_k, 64, h, tt, mbar_ld);
-        tma_load_3d(sb + kA_KQ + kKQ_LBO + 8192, &tm_q, 64, h, tt, mbar_ld);
-        tma_load_3d(sb + kA_V, &tm_v, 0, h, tt, mbar_ld);
-        tma_load_3d(sb + kA_V + 8192, &tm_v, 64, h, tt, mbar_ld);
-        tma_load_3d(sb + kA_G, &tm_la, 0, h, tt, mbar_ld);
+        issue_la(h, t0);
+        issue_kq(h, t0);
+        issue_v(h, t0);
     }
+    if (tid < 64) issue_beta(h, t0, L);
     if (warp == 0) {
         tmem_alloc(smem_u32(s_tmem), 256);
         tmem_relinquish();
     }
-    if (tid < 64) cp_async4(sb + kA_Misc + 4 * tid, beta + (size_t)(t0 + (tid < L ? tid : 0)) * H + h, tid < L ? 4u : 0u);
-    __syncthreads();  // mbarrier initialised
-    bool ok = mbar_wait(mbar_ld, 0);
-    cp_async_wait_all();
-    if (L < 64) {  // rows past the sequence (another sequence's tokens, or zeros): identity steps
-        for (int e = tid; e < (64 - L) * 16; e += kAThreads) {
-            const int r = L + (e >> 4), chh = e & 15;
-            *reinterpret_cast<uint4*>(sm + kA_KQ + sw128_chunk_off(r, chh, 128)) = make_uint4(0, 0, 0, 0);
-            *reinterpret_cast<uint4*>(sm + kA_KQ + sw128_chunk_off(64 + r, chh, 128)) = make_uint4(0, 0, 0, 0);
-            *reinterpret_cast<uint4*>(sm + kA_V + sw128_chunk_off(r, chh, 64)) = make_uint4(0, 0, 0, 0);
-        }
-        for (int e = tid; e < (64 - L) * 32; e += kAThreads)
-            *reinterpret_cast<float4*>(sG + (L + (e >> 5)) * kGS + 4 * (e & 31)) = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    __syncthreads();
-
-    // cumulative gate: thread (c, hf) scans rows 32*hf .. 32*hf+31 of channel c
-    const int c = tid & 127, hf = tid >> 7;
-    float gl[32];
-    {
-        float acc = 0.f;
-#pragma unroll
-        for (int u = 0; u < 32; ++u) {
-            acc += sG[(32 * hf + u) * kGS + c];
-            gl[u] = acc;
-        }
-    }
-    if (hf == 0) s_carry[c] = gl[31];
-    __syncthreads();
-    float lo, hi;
-    if (hf == 1) {
-        const float cr = s_carry[c];
-        lo = hi = cr;
-#pragma unroll
-        for (int u = 0; u < 32; ++u) {
-            gl[u] += cr;
-            lo = fminf(lo, gl[u]);
-            hi = fmaxf(hi, gl[u]);
-        }
-        s_lo[c] = lo;
-        s_hi[c] = hi;
-        s_D[c] = gl[31];  // g_last, turned into e^{g_last - ref} below
-    } else {
-        lo = hi = 0.f;  // the chunk start (g = 0) is part of the range
-#pragma unroll
-        for (int u = 0; u < 32; ++u) {
-            lo = fminf(lo, gl[u]);
-            hi = fmaxf(hi, gl[u]);
-        }
-    }
-#pragma unroll
-    for (int u = 0; u < 32; ++u) sG[(32 * hf + u) * kGS + c] = gl[u];
-    __syncthreads();
-    if (hf == 0) {
-        lo = fminf(lo, s_lo[c]);
-        hi = fmaxf(hi, s_hi[c]);
-        const float ref = 0.5f * (lo + hi);
-        const float glast = s_D[c];
-        s_ref[c] = ref;
-        s_E[c] = exp_fast(ref);
-        s_D[c] = exp_fast(glast - ref);
-        *reinterpret_cast<float*>(slot + kSlotGam + 4 * c) = exp_fast(glast);
-        if (!(hi - lo <= kTcFactorSpread)) atomicOr(s_wide, 1);
-    }
-    __syncthreads();
-    const bool wide = *s_wide != 0;
+    fence_before_sync();
+    __syncthreads();  // mbarriers initialised, TMEM address visible
+    fence_after_sync();
     const uint32_t tmem = *s_tmem;
-    uint32_t phase = 0;
     const int ch = tid & 15, rb = tid >> 4;  // element-wise passes: chunk ch of rows rb + 16 jj
     const int wq = warp & 3;
     const int rowq = 16 * wq + (lane & 15);  // M = 64 accumulator row held by this thread
     const int hc = (lane >> 4) * 64;         // ... and its half of the 128 columns
     const uint32_t trow = tmem + ((uint32_t)(32 * wq) << 16);
+    const int c = tid & 127, hf = tid >> 7;  // gate scan: channel c, rows 32 hf .. 32 hf + 31
+    uint32_t mphase = 0;
+    bool ok = true, has_next = false;
+    int it = 0;
 
-    if (!wide) {
-        float ref8[8], d8[8];
-#pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            ref8[m] = s_ref[8 * ch + m];
-            d8[m] = s_D[8 * ch + m];
-        }
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-            const int r = rb + 16 * jj;
-            const uint32_t ok_ = sw128_chunk_off(r, ch, 128), oq = sw128_chunk_off(64 + r, ch, 128);
-            float kv[8], qv[8];
-            unpack8(*reinterpret_cast<const uint4*>(sm + kA_KQ + ok_), kv);
-            unpack8(*reinterpret_cast<const uint4*>(sm + kA_KQ + oq), qv);
-            const float4 ga = *reinterpret_cast<const float4*>(sG + r * kGS + 8 * ch);
-            const float4 gb = *reinterpret_cast<const float4*>(sG + r * kGS + 8 * ch + 4);
-            const float g8[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
-            float kf[8], qf[8], kb[8], kd[8];
-#pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                const float x = g8[m] - ref8[m];
-                const float ef = exp_fast(x), eb = exp_fast(-x);
-                kf[m] = kv[m] * ef;
-                qf[m] = qv[m] * ef;
-                kb[m] = kv[m] * eb;
-                kd[m] = kb[m] * d8[m];
+    for (long long u = blockIdx.x; u < nunits; ++it) {
+        int claim = 0;  // thread 0: the next unit (gridDim.x + claim), from the work counter
+        if (tid == 0) claim = atomicAdd(&hdr->next_unit, 1);
+        const uint32_t par = (uint32_t)it & 1u;
+        uint8_t* slot = slots + (size_t)u * kSlotBytes;
+
+        if (tid == 0) *s_wide = 0;
+        ok = mbar_wait_ab(mbar_la, par, s_abort) && ok;
+        if (L < 64) {  // rows past the sequence (another sequence's tokens, or zeros): identity steps
+            ok = mbar_wait_ab(mbar_kq, par, s_abort) && ok;
+            ok = mbar_wait_ab(mbar_v, par, s_abort) && ok;
+            for (int e = tid; e < (64 - L) * 16; e += kAThreads) {
+                const int r = L + (e >> 4), chh = e & 15;
+                *reinterpret_cast<uint4*>(sm + kA_KQ + sw128_chunk_off(r, chh, 128)) = make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4*>(sm + kA_KQ + sw128_chunk_off(64 + r, chh, 128)) = make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4*>(sm + kA_V + sw128_chunk_off(r, chh, 64)) = make_uint4(0, 0, 0, 0);
             }
-            const uint32_t okd = sw128_chunk_off(r, ch, 64);
-            *reinterpret_cast<uint4*>(sm + kA_KQ + ok_) = pack8(kf);
-            *reinterpret_cast<uint4*>(sm + kA_KQ + oq) = pack8(qf);
-            *reinterpret_cast<uint4*>(sm + kA_Kb + okd) = pack8(kb);
-            *reinterpret_cast<uint4*>(slot + kSlotKd + okd) = pack8(kd);  // Kd = Kb diag(e^{g_last - ref})
+            for (int e = tid; e < (64 - L) * 32; e += kAThreads)
+                *reinterpret_cast<float4*>(sG + (L + (e >> 5)) * kGS + 4 * (e & 31)) = make_float4(0.f, 0.f, 0.f, 0.f);
+            __syncthreads();
         }
-        fence_proxy_async();
+
+        // cumulative gate in log2 units (g2 = log2(e) g): thread (c, hf) scans rows 32 hf .. 32 hf + 31
+        float gl[32];
+        {
+            float acc = 0.f;
+#pragma unroll
+            for (int u2 = 0; u2 < 32; ++u2) {
+                acc = fmaf(sG[(32 * hf + u2) * kGS + c], kLog2e, acc);
+                gl[u2] = acc;
+            }
+        }
+        if (hf == 0) s_carry[c] = gl[31];
         __syncthreads();
-        if (tid == 0) {  // [A'; P'] = [Kf; Qf] Kb^T: one M = 128 batch
-            fence_after_sync();
-            const uint32_t id = idesc_bf16(128, 64, false, false);
+        float lo, hi;
+        if (hf == 1) {
+            const float cr = s_carry[c];
+            lo = hi = cr;
 #pragma unroll
-            for (int kk = 0; kk < 128; kk += 16)
-                mma_bf16(tmem + 0, desc_kmajor(sb + kA_KQ, 128, kk), desc_kmajor(sb + kA_Kb, 64, kk), id, kk > 0);
-            mma_commit(mbar);
+            for (int u2 = 0; u2 < 32; ++u2) {
+                gl[u2] += cr;
+                lo = fminf(lo, gl[u2]);
+                hi = fmaxf(hi, gl[u2]);
+            }
+            s_lo[c] = lo;
+            s_hi[c] = hi;
+            s_D[c] = gl[31];  // g_last, turned into e^{g_last - ref} below
+        } else {
+            lo = hi = 0.f;  // the chunk start (g = 0) is part of the range
+#pragma unroll
+            for (int u2 = 0; u2 < 32; ++u2) {
+                lo = fminf(lo, gl[u2]);
+                hi = fmaxf(hi, gl[u2]);
+            }
         }
-        ok = mbar_wait(mbar, phase);
-        phase ^= 1;
-        fence_after_sync();
-        {   // warps 0,1 (and 4,5): A' rows 0..63; warps 2,3 (and 6,7): P' rows; warps < 4 columns 0..31, >= 4 32..63
-            const int col0 = (warp >> 2) * 32;
-            float a[32];
-            tmem_ld16(tmem + ((uint32_t)(32 * wq) << 16) + col0, a);
-            tmem_ld16(tmem + ((uint32_t)(32 * wq) << 16) + col0 + 16, a + 16);
-            tmem_wait_ld();
-            if (wq < 2) {
-                const int r = 32 * wq + lane;
-                const float br = s_beta[r];
 #pragma unroll
-                for (int m = 0; m < 32; m += 4) {
-                    const int i = col0 + m;
-                    *reinterpret_cast<float4*>(sA + r * kAS + i) =
-                        make_float4(i < r ? br * a[m] : 0.f, i + 1 < r ? br * a[m + 1] : 0.f,
-                                    i + 2 < r ? br * a[m + 2] : 0.f, i + 3 < r ? br * a[m + 3] : 0.f);
+        for (int u2 = 0; u2 < 32; ++u2) sG[(32 * hf + u2) * kGS + c] = gl[u2];
+        __syncthreads();
+        if (hf == 0) {
+            lo = fminf(lo, s_lo[c]);
+            hi = fmaxf(hi, s_hi[c]);
+            const float ref = 0.5f * (lo + hi);
+            const float glast = s_D[c];
+            s_ref[c] = ref;
+            s_E[c] = ex2_approx(ref);
+            s_D[c] = ex2_approx(glast - ref);
+            *reinterpret_cast<float*>(slot + kSlotGam + 4 * c) = ex2_approx(glast);
+            if (!(hi - lo <= kTcFactorSpread)) atomicOr(s_wide, 1);
+        }
+        if (tid == 0) {  // decode the claimed next unit for the prefetches below
+            int hh = 0, nn = 0, LL = 0;
+            long long tt = 0;
+            const long long un = (long long)gridDim.x + claim;
+            if (un < nunits) tc_unit(un, H, off, cu, Tseq, N, hh, nn, tt, LL);
+            s_next[0] = un;
+            s_next[1] = tt;
+            s_next_hl[0] = hh;
+            s_next_hl[1] = LL;
+        }
+        ok = mbar_wait_ab(mbar_kq, par, s_abort) && ok;  // k and q in place
+        cp_async_wait_all();                             // beta in place
+        __syncthreads();
+        has_next = s_next[0] < nunits;
+        const bool wide = *s_wide != 0;
+
+        if (!wide) {
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const int r = rb + 16 * jj;
+                const float4 ra = *reinterpret_cast<const float4*>(s_ref + 8 * ch);
+                const float4 rbv = *reinterpret_cast<const float4*>(s_ref + 8 * ch + 4);
+                const float4 da = *reinterpret_cast<const float4*>(s_D + 8 * ch);
+                const float4 db = *reinterpret_cast<const float4*>(s_D + 8 * ch + 4);
+                const float ref8[8] = {ra.x, ra.y, ra.z, ra.w, rbv.x, rbv.y, rbv.z, rbv.w};
+                const float d8[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
+                const uint32_t ok_ = sw128_chunk_off(r, ch, 128), oq = sw128_chunk_off(64 + r, ch, 128);
+                float kv[8], qv[8];
+                unpack8(*reinterpret_cast<const uint4*>(sm + kA_KQ + ok_), kv);
+                unpack8(*reinterpret_cast<const uint4*>(sm + kA_KQ + oq), qv);
+                const float4 ga = *reinterpret_cast<const float4*>(sG + r * kGS + 8 * ch);
+                const float4 gb = *reinterpret_cast<const float4*>(sG + r * kGS + 8 * ch + 4);
+                const float g8[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+                float kf[8], qf[8], kb[8], kd[8];
+#pragma unroll
+                for (int m = 0; m < 8; ++m) {
+                    const float x = g8[m] - ref8[m];
+                    const float ef = ex2_approx(x), eb = ex2_approx(-x);
+                    kf[m] = kv[m] * ef;
+                    qf[m] = qv[m] * ef;
+                    kb[m] = kv[m] * eb;
+                    kd[m] = kb[m] * d8[m];
                 }
-            } else {
-                const int r = 32 * (wq - 2) + lane;
+                const uint32_t okd = sw128_chunk_off(r, ch, 64);
+                *reinterpret_cast<uint4*>(sm + kA_KQ + ok_) = pack8(kf);
+                *reinterpret_cast<uint4*>(sm + kA_KQ + oq) = pack8(qf);
+                *reinterpret_cast<uint4*>(sm + kA_B + okd) = pack8(kb);
+                *reinterpret_cast<uint4*>(slot + kSlotKd + okd) = pack8(kd);  // Kd = Kb diag(e^{g_last - ref})
+            }
+            fence_proxy_async();
+            __syncthreads();
+            if (tid == 0 && ok) {  // [A'; P'] = [Kf; Qf] Kb^T: one M = 128 batch
+                fence_after_sync();
+                const uint32_t id = idesc_bf16(128, 64, false, false);
 #pragma unroll
-                for (int m = 0; m < 32; ++m) a[m] = (col0 + m <= r) ? a[m] : 0.f;
+                for (int kk = 0; kk < 128; kk += 16)
+                    mma_bf16(tmem + 0, desc_kmajor(sb + kA_KQ, 128, kk), desc_kmajor(sb + kA_B, 64, kk), id, kk > 0);
+                mma_commit(mbar);
+            }
+            ok = mbar_wait_ab(mbar, mphase, s_abort) && ok;
+            mphase ^= 1;
+            fence_after_sync();
+            {   // warps 0,1 (and 4,5): A' rows 0..63; warps 2,3 (and 6,7): P' rows; warps < 4 columns 0..31, >= 4 32..63
+                const int col0 = (warp >> 2) * 32;
+                float a[32];
+                tmem_ld16(tmem + ((uint32_t)(32 * wq) << 16) + col0, a);
+                tmem_ld16(tmem + ((uint32_t)(32 * wq) << 16) + col0 + 16, a + 16);
+                tmem_wait_ld();
+                if (wq < 2) {
+                    const int r = 32 * wq + lane;
+                    const float br = s_beta[r];
 #pragma unroll
-                for (int m = 0; m < 4; ++m)
-                    *reinterpret_cast<uint4*>(sm + kA_P + sw128_chunk_off(r, (col0 >> 3) + m, 64)) = pack8(a + 8 * m);
+                    for (int m = 0; m < 32; m += 4) {
+                        const int i = col0 + m;
+                        *reinterpret_cast<float4*>(sA + r * kAS + i) =
+                            make_float4(i < r ? br * a[m] : 0.f, i + 1 < r ? br * a[m + 1] : 0.f,
+                                        i + 2 < r ? br * a[m + 2] : 0.f, i + 3 < r ? br * a[m + 3] : 0.f);
+                    }
+                } else {
+                    const int r = 32 * (wq - 2) + lane;
+#pragma unroll
+                    for (int m = 0; m < 32; ++m) a[m] = (col0 + m <= r) ? a[m] : 0.f;
+#pragma unroll
+                    for (int m = 0; m < 4; ++m)
+                        *reinterpret_cast<uint4*>(sm + kA_P + sw128_chunk_off(r, (col0 >> 3) + m, 64)) = pack8(a + 8 * m);
+                }
+            }
+        } else {
+            // some channel's gate spreads beyond e^159: exact per-element factors on CUDA cores
+            float av[16], pv[16];
+#pragma unroll 1
+            for (int m = 0; m < 16; ++m) {
+                const int e = tid + kAThreads * m;
+                const int r = e >> 6, i = e & 63;
+                float a = 0.f, p = 0.f;
+                if (i <= r) {
+                    for (int cc = 0; cc < 128; ++cc) {
+                        const float kk = lds_bf16(sm + kA_KQ + sw128_off(i, cc, 128)) * ex2_approx(sG[r * kGS + cc] - sG[i * kGS + cc]);
+                        a = fmaf(lds_bf16(sm + kA_KQ + sw128_off(r, cc, 128)), kk, a);
+                        p = fmaf(lds_bf16(sm + kA_KQ + sw128_off(64 + r, cc, 128)), kk, p);
+                    }
+                }
+                av[m] = (i < r) ? s_beta[r] * a : 0.f;
+                pv[m] = p;
+            }
+            __syncthreads();  // every thread is done reading raw k and q across rows
+            // in place: k -> k e^g (B operand of W), q -> q e^g; Kd = k e^{g_last - g} straight to the slot
+#pragma unroll 1
+            for (int jj = 0; jj < 4; ++jj) {
+                const int r = rb + 16 * jj;
+                const uint32_t ok_ = sw128_chunk_off(r, ch, 128), oq = sw128_chunk_off(64 + r, ch, 128);
+                float kv[8], qv[8], kt[8], kd[8], qg[8];
+                unpack8(*reinterpret_cast<const uint4*>(sm + kA_KQ + ok_), kv);
+                unpack8(*reinterpret_cast<const uint4*>(sm + kA_KQ + oq), qv);
+#pragma unroll
+                for (int m = 0; m < 8; ++m) {
+                    const float gv = sG[r * kGS + 8 * ch + m], gz = sG[63 * kGS + 8 * ch + m];
+                    const float eg = ex2_approx(gv);
+                    kt[m] = kv[m] * eg;
+                    qg[m] = qv[m] * eg;
+                    kd[m] = kv[m] * ex2_approx(gz - gv);
+                }
+                *reinterpret_cast<uint4*>(sm + kA_KQ + ok_) = pack8(kt);
+                *reinterpret_cast<uint4*>(sm + kA_KQ + oq) = pack8(qg);
+                *reinterpret_cast<uint4*>(slot + kSlotKd + sw128_chunk_off(r, ch, 64)) = pack8(kd);
+            }
+            __syncthreads();  // g no longer read: A and the P tile take its place
+            for (int cc = tid; cc < 128; cc += kAThreads) s_E[cc] = 1.f;
+#pragma unroll
+            for (int m = 0; m < 16; ++m) {
+                const int e = tid + kAThreads * m;
+                const int r = e >> 6, i = e & 63;
+                sA[r * kAS + i] = av[m];
+                *reinterpret_cast<__nv_bfloat16*>(sm + kA_P + sw128_off(r, i, 64)) = __float2bfloat16_rn(pv[m]);
             }
         }
         fence_before_sync();
-    } else {
-        // some channel's gate spreads beyond e^160: exact per-element factors on CUDA cores
-        float av[16], pv[16];
-#pragma unroll 1
-        for (int m = 0; m < 16; ++m) {
-            const int e = tid + kAThreads * m;
-            const int r = e >> 6, i = e & 63;
-            float a = 0.f, p = 0.f;
-            if (i <= r) {
-                for (int cc = 0; cc < 128; ++cc) {
-                    const float kk = lds_bf16(sm + kA_KQ + sw128_off(i, cc, 128)) * expf(sG[r * kGS + cc] - sG[i * kGS + cc]);
-                    a = fmaf(lds_bf16(sm + kA_KQ + sw128_off(r, cc, 128)), kk, a);
-                    p = fmaf(lds_bf16(sm + kA_KQ + sw128_off(64 + r, cc, 128)), kk, p);
-                }
-            }
-            av[m] = (i < r) ? s_beta[r] * a : 0.f;
-            pv[m] = p;
-        }
-        __syncthreads();  // every thread is done reading raw k and q across rows
-        // in place: k -> k e^g (B operand of W), q -> q e^g; Kd = k e^{g_last - g} straight to the slot
-#pragma unroll 1
-        for (int jj = 0; jj < 4; ++jj) {
-            const int r = rb + 16 * jj;
-            const uint32_t ok_ = sw128_chunk_off(r, ch, 128), oq = sw128_chunk_off(64 + r, ch, 128);
-            float kv[8], qv[8], kt[8], kd[8], qg[8];
-            unpack8(*reinterpret_cast<const uint4*>(sm + kA_KQ + ok_), kv);
-            unpack8(*reinterpret_cast<const uint4*>(sm + kA_KQ + oq), qv);
-#pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                const float gv = sG[r * kGS + 8 * ch + m], gz = sG[63 * kGS + 8 * ch + m];
-                const float eg = expf(gv);
-                kt[m] = kv[m] * eg;
-                qg[m] = qv[m] * eg;
-                kd[m] = kv[m] * expf(gz - gv);
-            }
-            *reinterpret_cast<uint4*>(sm + kA_KQ + ok_) = pack8(kt);
-            *reinterpret_cast<uint4*>(sm + kA_KQ + oq) = pack8(qg);
-            *reinterpret_cast<uint4*>(slot + kSlotKd + sw128_chunk_off(r, ch, 64)) = pack8(kd);
-        }
-        __syncthreads();  // g no longer read: A and the P tile take its place
-        for (int cc = tid; cc < 128; cc += kAThreads) s_E[cc] = 1.f;
-#pragma unroll
-        for (int m = 0; m < 16; ++m) {
-            const int e = tid + kAThreads * m;
-            const int r = e >> 6, i = e & 63;
-            sA[r * kAS + i] = av[m];
-            *reinterpret_cast<__nv_bfloat16*>(sm + kA_P + sw128_off(r, i, 64)) = __float2bfloat16_rn(pv[m]);
-        }
-    }
-    ok = __syncthreads_and(ok);  // A complete; Kb consumed
+        ok = __syncthreads_and(ok);  // A and the P tile complete; the tensor core is done with Kb
 
-    // UT transform (X over Kb), then T = X diag(beta) as a bf16 K-major tile (also over Kb)
-    if (ok) ut_inverse_64(sA, sX, sY);
-    uint4 tch[2];
+        // UT transform (X in place of A), then T = X diag(beta) as a bf16 K-major tile over Kb
+        if (ok) ut_inverse_64_inplace(sA, sY);
+        uint4 tch[2];
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-        const int e = tid + kAThreads * u;
-        const int r = e >> 3, c8 = e & 7;
-        float t8[8];
+        for (int u2 = 0; u2 < 2; ++u2) {
+            const int e = tid + kAThreads * u2;
+            const int r = e >> 3, c8 = e & 7;
+            float t8[8];
 #pragma unroll
-        for (int m = 0; m < 8; ++m) t8[m] = sX[r * kXS + 8 * c8 + m] * s_beta[8 * c8 + m];
-        tch[u] = pack8(t8);
-    }
-    __syncthreads();  // X fully read
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-        const int e = tid + kAThreads * u;
-        *reinterpret_cast<uint4*>(sm + kA_Kb + sw128_chunk_off(e >> 3, e & 7, 64)) = tch[u];
-    }
-    fence_proxy_async();
-    __syncthreads();
-    if (ok && tid == 0) {  // W' = T Kf (B: k rows of the stacked tile), Uv = T v
-        fence_after_sync();
-        const uint32_t id = idesc_bf16(64, 128, false, true);
-#pragma unroll
-        for (int kk = 0; kk < 64; kk += 16) {
-            mma_bf16(tmem + 0, desc_kmajor(sb + kA_Kb, 64, kk), desc_sw128(sb + kA_KQ + kk * 128, kKQ_LBO, 1024u), id, kk > 0);
-            mma_bf16(tmem + 128, desc_kmajor(sb + kA_Kb, 64, kk), desc_mnmajor(sb + kA_V, 64, kk), id, kk > 0);
+            for (int m = 0; m < 8; ++m) t8[m] = sA[r * kAS + 8 * c8 + m] * s_beta[8 * c8 + m];
+            tch[u2] = pack8(t8);
         }
-        mma_commit(mbar);
-    }
-    if (ok) {
-        ok = mbar_wait(mbar, phase);
-        phase ^= 1;
-        fence_after_sync();
-    }
-    ok = __syncthreads_and(ok);
-    if (ok) {
-        if (warp < 4) {  // W = W' diag(e^ref) -> the k rows of the stacked tile (Kf consumed)
+        __syncthreads();
 #pragma unroll
-            for (int b2 = 0; b2 < 64; b2 += 32) {
-                float a2[32];
-                tmem_ld16_pair<64>(trow + b2, a2);
-                tmem_ld16_pair<64>(trow + b2 + 16, a2 + 16);
-                tmem_wait_ld();
+        for (int u2 = 0; u2 < 2; ++u2) {
+            const int e = tid + kAThreads * u2;
+            *reinterpret_cast<uint4*>(sm + kA_B + sw128_chunk_off(e >> 3, e & 7, 64)) = tch[u2];
+        }
+        fence_proxy_async();
+        __syncthreads();
+        if (tid == 0) ok = mbar_wait_ab(mbar_v, par, s_abort) && ok;  // v in place
+        if (ok && tid == 0) {  // W' = T Kf (B: k rows of the stacked tile), Uv = T v
+            fence_after_sync();
+            const uint32_t id = idesc_bf16(64, 128, false, true);
 #pragma unroll
-                for (int m = 0; m < 32; ++m) a2[m] *= s_E[hc + b2 + m];
-#pragma unroll
-                for (int m = 0; m < 4; ++m)
-                    *reinterpret_cast<uint4*>(sm + kA_KQ + sw128_chunk_off(rowq, (hc + b2) / 8 + m, 128)) = pack8(a2 + 8 * m);
+            for (int kk = 0; kk < 64; kk += 16) {
+                mma_bf16(tmem + 0, desc_kmajor(sb + kA_B, 64, kk), desc_sw128(sb + kA_KQ + kk * 128, kKQ_LBO, 1024u), id, kk > 0);
+                mma_bf16(tmem + 128, desc_kmajor(sb + kA_B, 64, kk), desc_mnmajor(sb + kA_V, 64, kk), id, kk > 0);
             }
-        } else {  // Uv -> the v tile (v consumed)
-#pragma unroll
-            for (int b2 = 0; b2 < 64; b2 += 32) {
-                float a2[32];
-                tmem_ld16_pair<64>(trow + 128 + b2, a2);
-                tmem_ld16_pair<64>(trow + 128 + b2 + 16, a2 + 16);
-                tmem_wait_ld();
-#pragma unroll
-                for (int m = 0; m < 4; ++m)
-                    *reinterpret_cast<uint4*>(sm + kA_V + sw128_chunk_off(rowq, (hc + b2) / 8 + m, 64)) = pack8(a2 + 8 * m);
-            }
+            mma_commit(mbar);
         }
-    }
-    fence_proxy_async();
-    fence_before_sync();
-    ok = __syncthreads_and(ok);
-    if (ok && tid == 0) {
-        // W and Uv images out (bulk), then [P W | P Uv] = P [W | Uv]
-        bulk_s2g(slot + kSlotW, sb + kA_KQ, 8192);
-        bulk_s2g(slot + kSlotW + 8192, sb + kA_KQ + kKQ_LBO, 8192);
-        bulk_s2g(slot + kSlotUv, sb + kA_V, 16384);
-        bulk_commit();
+        ok = mbar_wait_ab(mbar, mphase, s_abort) && ok;
+        mphase ^= 1;
+        ok = mbar_wait_ab(mbar_v, par, s_abort) && ok;  // (long complete) orders this thread after the v copy
         fence_after_sync();
-        const uint32_t id = idesc_bf16(64, 128, false, true);
+        ok = __syncthreads_and(ok);
+        if (ok) {
+            if (warp < 4) {  // W = W' diag(e^ref) -> the k rows of the stacked tile (Kf consumed)
 #pragma unroll
-        for (int kk = 0; kk < 64; kk += 16) {
-            mma_bf16(tmem + 0, desc_kmajor(sb + kA_P, 64, kk), desc_sw128(sb + kA_KQ + kk * 128, kKQ_LBO, 1024u), id, kk > 0);
-            mma_bf16(tmem + 128, desc_kmajor(sb + kA_P, 64, kk), desc_mnmajor(sb + kA_V, 64, kk), id, kk > 0);
-        }
-        mma_commit(mbar);
-        bulk_wait_read();  // the Uv tile is overwritten by O0 below
-    }
-    if (ok) {
-        ok = mbar_wait(mbar, phase);
-        fence_after_sync();
-    }
-    ok = __syncthreads_and(ok);
-    if (ok) {
-        if (warp < 4) {  // Q' = Qf e^ref - P W -> the q rows of the stacked tile, in place
+                for (int b2 = 0; b2 < 64; b2 += 32) {
+                    float a2[32];
+                    tmem_ld16_pair<64>(trow + b2, a2);
+                    tmem_ld16_pair<64>(trow + b2 + 16, a2 + 16);
+                    tmem_wait_ld();
 #pragma unroll
-            for (int b2 = 0; b2 < 64; b2 += 32) {
-                float a2[32];
-                tmem_ld16_pair<64>(trow + b2, a2);
-                tmem_ld16_pair<64>(trow + b2 + 16, a2 + 16);
-                tmem_wait_ld();
+                    for (int m = 0; m < 32; ++m) a2[m] *= s_E[hc + b2 + m];
 #pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    uint4* p = reinterpret_cast<uint4*>(sm + kA_KQ + sw128_chunk_off(64 + rowq, (hc + b2) / 8 + m, 128));
-                    float qf[8];
-                    unpack8(*p, qf);
+                    for (int m = 0; m < 4; ++m)
+                        *reinterpret_cast<uint4*>(sm + kA_KQ + sw128_chunk_off(rowq, (hc + b2) / 8 + m, 128)) = pack8(a2 + 8 * m);
+                }
+            } else {  // Uv -> the T tile's place (T consumed)
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) qf[e] = qf[e] * s_E[hc + b2 + 8 * m + e] - a2[8 * m + e];
-                    *p = pack8(qf);
+                for (int b2 = 0; b2 < 64; b2 += 32) {
+                    float a2[32];
+                    tmem_ld16_pair<64>(trow + 128 + b2, a2);
+                    tmem_ld16_pair<64>(trow + 128 + b2 + 16, a2 + 16);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int m = 0; m < 4; ++m)
+                        *reinterpret_cast<uint4*>(sm + kA_B + sw128_chunk_off(rowq, (hc + b2) / 8 + m, 64)) = pack8(a2 + 8 * m);
                 }
             }
-        } else {  // O0 = P Uv -> the v tile
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        ok = __syncthreads_and(ok);
+        if (tid == 0) {
+            if (has_next) issue_v(s_next_hl[0], s_next[1]);  // the v tile is free: MMA2 has read it
+            if (ok) {
+                // W and Uv images out (bulk), then [P W | P Uv] = P [W | Uv]
+                bulk_s2g(slot + kSlotW, sb + kA_KQ, 8192);
+                bulk_s2g(slot + kSlotW + 8192, sb + kA_KQ + kKQ_LBO, 8192);
+                bulk_s2g(slot + kSlotUv, sb + kA_B, 16384);
+                bulk_commit();
+                fence_after_sync();
+                const uint32_t id = idesc_bf16(64, 128, false, true);
 #pragma unroll
-            for (int b2 = 0; b2 < 64; b2 += 32) {
-                float a2[32];
-                tmem_ld16_pair<64>(trow + 128 + b2, a2);
-                tmem_ld16_pair<64>(trow + 128 + b2 + 16, a2 + 16);
-                tmem_wait_ld();
+                for (int kk = 0; kk < 64; kk += 16) {
+                    mma_bf16(tmem + 0, desc_kmajor(sb + kA_P, 64, kk), desc_sw128(sb + kA_KQ + kk * 128, kKQ_LBO, 1024u), id, kk > 0);
+                    mma_bf16(tmem + 128, desc_kmajor(sb + kA_P, 64, kk), desc_mnmajor(sb + kA_B, 64, kk), id, kk > 0);
+                }
+                mma_commit(mbar);
+            }
+            bulk_wait_read();  // the Uv tile is overwritten by O0 below
+        }
+        ok = mbar_wait_ab(mbar, mphase, s_abort) && ok;
+        mphase ^= 1;
+        fence_after_sync();
+        ok = __syncthreads_and(ok);
+        if (has_next) {  // the log_alpha region is free (P consumed) and beta has been read
+            if (tid == 0) issue_la(s_next_hl[0], s_next[1]);
+            if (tid < 64) issue_beta(s_next_hl[0], s_next[1], s_next_hl[1]);
+        }
+        if (ok) {
+            if (warp < 4) {  // Q' = Qf e^ref - P W -> the q rows of the stacked tile, in place
 #pragma unroll
-                for (int m = 0; m < 4; ++m)
-                    *reinterpret_cast<uint4*>(sm + kA_V + sw128_chunk_off(rowq, (hc + b2) / 8 + m, 64)) = pack8(a2 + 8 * m);
+                for (int b2 = 0; b2 < 64; b2 += 32) {
+                    float a2[32];
+                    tmem_ld16_pair<64>(trow + b2, a2);
+                    tmem_ld16_pair<64>(trow + b2 + 16, a2 + 16);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        uint4* p = reinterpret_cast<uint4*>(sm + kA_KQ + sw128_chunk_off(64 + rowq, (hc + b2) / 8 + m, 128));
+                        float qf[8];
+                        unpack8(*p, qf);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) qf[e] = qf[e] * s_E[hc + b2 + 8 * m + e] - a2[8 * m + e];
+                        *p = pack8(qf);
+                    }
+                }
+            } else {  // O0 = P Uv -> the Uv tile's place
+#pragma unroll
+                for (int b2 = 0; b2 < 64; b2 += 32) {
+                    float a2[32];
+                    tmem_ld16_pair<64>(trow + 128 + b2, a2);
+                    tmem_ld16_pair<64>(trow + 128 + b2 + 16, a2 + 16);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int m = 0; m < 4; ++m)
+                        *reinterpret_cast<uint4*>(sm + kA_B + sw128_chunk_off(rowq, (hc + b2) / 8 + m, 64)) = pack8(a2 + 8 * m);
+                }
             }
         }
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+        if (tid == 0) {  // Q' and O0 images out; then the next chunk's k and q take the stacked tile
+            if (ok) {
+                bulk_s2g(slot + kSlotQ, sb + kA_KQ + 8192, 8192);
+                bulk_s2g(slot + kSlotQ + 8192, sb + kA_KQ + kKQ_LBO + 8192, 8192);
+                bulk_s2g(slot + kSlotO0, sb + kA_B, 16384);
+                bulk_commit();
+            }
+            bulk_wait_read();
+            if (has_next) issue_kq(s_next_hl[0], s_next[1]);
+        }
+        ok = __syncthreads_and(ok);  // the Kb tile of the next chunk may overwrite O0 from here on
+        if (!ok) break;
+        u = s_next[0];
+        t0 = s_next[1];
+        h = s_next_hl[0];
+        L = s_next_hl[1];
     }
-    fence_proxy_async();
-    fence_before_sync();
-    __syncthreads();
-    if (tid == 0) {  // Q' and O0 images out
-        if (ok) {
-            bulk_s2g(slot + kSlotQ, sb + kA_KQ + 8192, 8192);
-            bulk_s2g(slot + kSlotQ + 8192, sb + kA_KQ + kKQ_LBO + 8192, 8192);
-            bulk_s2g(slot + kSlotO0, sb + kA_V, 16384);
-            bulk_commit();
+    if (tid == 0) {
+        if (!ok && has_next) {  // loads for the next chunk may still be landing: bounded waits
+            const uint32_t pn = ((uint32_t)it + 1u) & 1u;
+            (void)mbar_wait(mbar_la, pn);
+            (void)mbar_wait(mbar_kq, pn);
+            (void)mbar_wait(mbar_v, pn);
         }
         bulk_wait_all();
     }
+    cp_async_wait_all();
+    fence_before_sync();
+    __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
@@ -870,9 +960,14 @@ inline cudaError_t launch_tc_prefill(const void* q, const void* k, const void* v
         if (!make_token_map(&tq, q, true, H, Ttot, 64) || !make_token_map(&tk, k, true, H, Ttot, 64) ||
             !make_token_map(&tv, v, true, H, Ttot, 64) || !make_token_map(&tla, la, false, H, Ttot, 128))
             return cudaErrorInvalidValue;
+        // persistent: two CTAs per SM (the register and shared-memory budget of one CTA is half an SM)
+        int dev = 0, sms = 148;
+        if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        const long long units = (long long)max_chunks * H;
+        const unsigned grid = (unsigned)(units < 2LL * sms ? units : 2LL * sms);
         LaunchScope ls("tc_intra", stream);
-        tc_intra_kernel<<<dim3(max_chunks, H), kAThreads, kA_Smem, stream>>>(tq, tk, tv, tla, beta, hdr, off, cu, Tseq,
-                                                                               N, H, (uint8_t*)slots);
+        tc_intra_kernel<<<grid, kAThreads, kA_Smem, stream>>>(tq, tk, tv, tla, beta, const_cast<WsHeader*>(hdr), off, cu, Tseq, N, H,
+                                                              (uint8_t*)slots);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

@@ -209,6 +209,15 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b)
     return *reinterpret_cast<uint32_t*>(&h);
 }
 __device__ __forceinline__ float exp_fast(float x) { return exp2f(x * 1.4426950408889634f); }
+// 2^x with the hardware's approximate base-2 exponential (relative error ~2^-22 over the normal
+// range; results below 2^-126 flush to zero).
+__device__ __forceinline__ float ex2_approx(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+constexpr float kLog2e = 1.4426950408889634f;
 
 }  // namespace tc
 }  // namespace kda

@@ -23,7 +23,7 @@ constexpr int kDecodeThreads = 256;
 constexpr int kDecodeSlice = 64;  // columns of S per CTA
 
 template <typename TIn, int DK>
-__global__ void __launch_bounds__(kDecodeThreads)
+__global__ void __launch_bounds__(kDecodeThreads, 3)
 decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
                    const float* __restrict__ log_alpha, const float* __restrict__ beta, float* __restrict__ S,
                    TIn* __restrict__ out, int dv)
@@ -38,6 +38,7 @@ decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const T
 
     __shared__ float s_a[DK], s_k[DK], s_q[DK];
     __shared__ __align__(16) float s_red[8][16][8];
+    __shared__ float s_qk[8];  // per-warp partial q . k
 
     float* Sp = S + (size_t)p * DK * dv + j0;
     float4 st[RPT];
@@ -45,6 +46,10 @@ decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const T
     for (int i = 0; i < RPT; ++i)
         st[i] = __ldcs(reinterpret_cast<const float4*>(Sp + (size_t)(rb + 16 * i) * dv) + cg);
 
+    // the step's small inputs, loaded alongside the state so that no load sits on the critical path
+    const float b = beta[p];
+    const TIn* vp = v + (size_t)p * dv + j0 + 4 * cg;
+    const float v0 = to_f32(vp[0]), v1 = to_f32(vp[1]), v2 = to_f32(vp[2]), v3 = to_f32(vp[3]);
     for (int c = tid; c < DK; c += kDecodeThreads) {
         s_a[c] = expf(log_alpha[(size_t)p * DK + c]);
         s_k[c] = to_f32(k[(size_t)p * DK + c]);
@@ -52,11 +57,12 @@ decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const T
     }
     __syncthreads();
 
-    float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f, q0 = 0.f, q1 = 0.f, q2 = 0.f, q3 = 0.f;
+    float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f, q0 = 0.f, q1 = 0.f, q2 = 0.f, q3 = 0.f, qk = 0.f;
 #pragma unroll
     for (int i = 0; i < RPT; ++i) {
         const int c = rb + 16 * i;
         const float a = s_a[c], kc = s_k[c], qc = s_q[c];
+        qk = fmaf(qc, kc, qk);  // rows rb + 16 i: the two half-warps together cover this warp's rows
         st[i].x *= a; st[i].y *= a; st[i].z *= a; st[i].w *= a;
         r0 = fmaf(st[i].x, kc, r0); r1 = fmaf(st[i].y, kc, r1); r2 = fmaf(st[i].z, kc, r2); r3 = fmaf(st[i].w, kc, r3);
         q0 = fmaf(st[i].x, qc, q0); q1 = fmaf(st[i].y, qc, q1); q2 = fmaf(st[i].z, qc, q2); q3 = fmaf(st[i].w, qc, q3);
@@ -70,6 +76,8 @@ decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const T
         dst[0] = make_float4(r0, r1, r2, r3);
         dst[1] = make_float4(q0, q1, q2, q3);
     }
+    qk += __shfl_xor_sync(0xffffffffu, qk, 16);  // lanes l and l ^ 16 hold the warp's two rows of each pair
+    if (l == 0) s_qk[w] = qk;
     __syncthreads();
 
     float4 rr = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -78,10 +86,8 @@ decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const T
         const float4 x = reinterpret_cast<const float4*>(&s_red[ww][cg][0])[0];
         rr.x += x.x; rr.y += x.y; rr.z += x.z; rr.w += x.w;
     }
-    const float b = beta[p];
-    const TIn* vp = v + (size_t)p * dv + j0 + 4 * cg;
-    const float u0 = b * (to_f32(vp[0]) - rr.x), u1 = b * (to_f32(vp[1]) - rr.y);
-    const float u2 = b * (to_f32(vp[2]) - rr.z), u3 = b * (to_f32(vp[3]) - rr.w);
+    const float u0 = b * (v0 - rr.x), u1 = b * (v1 - rr.y);
+    const float u2 = b * (v2 - rr.z), u3 = b * (v3 - rr.w);
 
 #pragma unroll
     for (int i = 0; i < RPT; ++i) {
@@ -93,8 +99,9 @@ decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const T
     }
 
     if (w == 0 && l < 16) {
-        float qk = 0.f;
-        for (int c = 0; c < DK; ++c) qk = fmaf(s_q[c], s_k[c], qk);
+        float qk_all = 0.f;
+#pragma unroll
+        for (int ww = 0; ww < 8; ++ww) qk_all += s_qk[ww];
         float4 ss = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int ww = 0; ww < 8; ++ww) {
@@ -102,10 +109,10 @@ decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const T
             ss.x += x.x; ss.y += x.y; ss.z += x.z; ss.w += x.w;
         }
         TIn* op = out + (size_t)p * dv + j0 + 4 * cg;
-        op[0] = from_f32<TIn>(fmaf(u0, qk, ss.x));
-        op[1] = from_f32<TIn>(fmaf(u1, qk, ss.y));
-        op[2] = from_f32<TIn>(fmaf(u2, qk, ss.z));
-        op[3] = from_f32<TIn>(fmaf(u3, qk, ss.w));
+        op[0] = from_f32<TIn>(fmaf(u0, qk_all, ss.x));
+        op[1] = from_f32<TIn>(fmaf(u1, qk_all, ss.y));
+        op[2] = from_f32<TIn>(fmaf(u2, qk_all, ss.z));
+        op[3] = from_f32<TIn>(fmaf(u3, qk_all, ss.w));
     }
 }
 

@@ -22,15 +22,16 @@ namespace kda {
 constexpr int kDecodeThreads = 256;
 constexpr int kDecodeSlice = 64;  // columns of S per CTA
 
-template <typename TIn, int DK>
+template <typename TIn, int DK, bool GROUPED>
 __global__ void __launch_bounds__(kDecodeThreads, 3)
 decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
                    const float* __restrict__ log_alpha, const float* __restrict__ beta, float* __restrict__ S,
-                   TIn* __restrict__ out, int dv)
+                   TIn* __restrict__ out, int dv, int H, int G)
 {
     constexpr int RPT = DK / 16;  // state rows held per thread
     const int nslices = dv / kDecodeSlice;
     const int p = blockIdx.x / nslices;            // (sequence, head) pair, = n*H + h
+    const int pq = GROUPED ? (p / H) * (H / G) + (p % H) / G : p;  // its q/k head: n*Hk + h/G (G = H/Hk)
     const int j0 = (blockIdx.x % nslices) * kDecodeSlice;
     const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
     const int cg = l & 15;                         // columns j0 + 4cg .. j0 + 4cg + 3
@@ -52,8 +53,8 @@ decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const T
     const float v0 = to_f32(vp[0]), v1 = to_f32(vp[1]), v2 = to_f32(vp[2]), v3 = to_f32(vp[3]);
     for (int c = tid; c < DK; c += kDecodeThreads) {
         s_a[c] = expf(log_alpha[(size_t)p * DK + c]);
-        s_k[c] = to_f32(k[(size_t)p * DK + c]);
-        s_q[c] = to_f32(q[(size_t)p * DK + c]);
+        s_k[c] = to_f32(k[(size_t)pq * DK + c]);
+        s_q[c] = to_f32(q[(size_t)pq * DK + c]);
     }
     __syncthreads();
 
@@ -118,19 +119,23 @@ decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const T
 
 template <typename TIn>
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* la, const float* beta, float* S,
-                          void* out, int N, int H, int dk, int dv, cudaStream_t stream)
+                          void* out, int N, int H, int Hk, int dk, int dv, cudaStream_t stream)
 {
     const long long pairs = (long long)N * H;
     const long long blocks = pairs * (dv / kDecodeSlice);
     if (blocks == 0) return cudaSuccess;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
     LaunchScope ls("decode_step", stream);
-    if (dk == 128)
-        decode_step_kernel<TIn, 128><<<(unsigned)blocks, kDecodeThreads, 0, stream>>>(
-            (const TIn*)q, (const TIn*)k, (const TIn*)v, la, beta, S, (TIn*)out, dv);
-    else
-        decode_step_kernel<TIn, 64><<<(unsigned)blocks, kDecodeThreads, 0, stream>>>(
-            (const TIn*)q, (const TIn*)k, (const TIn*)v, la, beta, S, (TIn*)out, dv);
+    const int G = H / Hk;
+    const dim3 grid((unsigned)blocks);
+    const TIn *qq = (const TIn*)q, *kk = (const TIn*)k, *vv = (const TIn*)v;
+    if (dk == 128) {
+        if (G == 1) decode_step_kernel<TIn, 128, false><<<grid, kDecodeThreads, 0, stream>>>(qq, kk, vv, la, beta, S, (TIn*)out, dv, H, G);
+        else decode_step_kernel<TIn, 128, true><<<grid, kDecodeThreads, 0, stream>>>(qq, kk, vv, la, beta, S, (TIn*)out, dv, H, G);
+    } else {
+        if (G == 1) decode_step_kernel<TIn, 64, false><<<grid, kDecodeThreads, 0, stream>>>(qq, kk, vv, la, beta, S, (TIn*)out, dv, H, G);
+        else decode_step_kernel<TIn, 64, true><<<grid, kDecodeThreads, 0, stream>>>(qq, kk, vv, la, beta, S, (TIn*)out, dv, H, G);
+    }
     return cudaGetLastError();
 }
 

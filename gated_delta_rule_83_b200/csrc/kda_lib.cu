@@ -80,6 +80,20 @@ kda_status make_plan(int B, int T, int H, int dk, int dv, bool varlen, int num_s
     return KDA_OK;
 }
 
+// Options of the extended entry points: Hk = q/k heads (0 -> H); reserved fields must be zero.
+kda_status parse_options(const kda_options* opt, int H, int& Hk)
+{
+    Hk = H;
+    if (!opt) return KDA_OK;
+    for (int r : opt->reserved)
+        if (r != 0) return KDA_ERR_INVALID_ARG;
+    if (opt->num_qk_heads != 0) {
+        if (opt->num_qk_heads < 0 || H % opt->num_qk_heads != 0) return KDA_ERR_INVALID_ARG;
+        Hk = opt->num_qk_heads;
+    }
+    return KDA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -111,12 +125,15 @@ kda_status kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int
     return KDA_OK;
 }
 
-kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const float* log_alpha, const float* beta,
-                         const float* S0, const int32_t* cu_seqlens, int num_seqs, void* out, float* S_final,
-                         int B, int T, int H, int dk, int dv, kda_dtype dt, void* workspace,
-                         size_t workspace_bytes, kda_stream_t stream_)
+kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v, const float* log_alpha, const float* beta,
+                            const float* S0, const int32_t* cu_seqlens, int num_seqs, void* out, float* S_final,
+                            int B, int T, int H, int dk, int dv, kda_dtype dt, const kda_options* opt,
+                            void* workspace, size_t workspace_bytes, kda_stream_t stream_)
 {
     cudaStream_t stream = (cudaStream_t)stream_;
+    int Hk = H;
+    const kda_status so = parse_options(opt, H, Hk);
+    if (so != KDA_OK) return so;
     Plan p;
     const kda_status st = make_plan(B, T, H, dk, dv, cu_seqlens != nullptr, num_seqs, dt, p);
     if (st != KDA_OK) return st;
@@ -141,25 +158,37 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const floa
 
     cudaError_t e;
     if (p.tc) {
-        e = launch_tc_prefill(q, k, v, log_alpha, beta, S0, S_final, out, hdr, off, cu_seqlens, p.Tseq, p.N, H,
+        e = launch_tc_prefill(q, k, v, log_alpha, beta, S0, S_final, out, hdr, off, cu_seqlens, p.Tseq, p.N, H, Hk,
                               p.max_chunks, p.Ttot, slots, stream);
     } else if (dt == KDA_BF16) {
         e = launch_simt_prefill<__nv_bfloat16>(q, k, v, log_alpha, beta, S0, S_final, out, hdr, off, cu_seqlens,
-                                               p.Tseq, p.N, H, dk, dv, p.max_chunks, (float*)slots, stream);
+                                               p.Tseq, p.N, H, Hk, dk, dv, p.max_chunks, (float*)slots, stream);
     } else {
         e = launch_simt_prefill<float>(q, k, v, log_alpha, beta, S0, S_final, out, hdr, off, cu_seqlens, p.Tseq,
-                                       p.N, H, dk, dv, p.max_chunks, (float*)slots, stream);
+                                       p.N, H, Hk, dk, dv, p.max_chunks, (float*)slots, stream);
     }
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
-kda_status kda_decode_step(const void* q, const void* k, const void* v, const float* log_alpha, const float* beta,
-                           float* S_inout, void* out, int N, int H, int dk, int dv, kda_dtype dt,
-                           kda_stream_t stream_)
+kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const float* log_alpha, const float* beta,
+                         const float* S0, const int32_t* cu_seqlens, int num_seqs, void* out, float* S_final,
+                         int B, int T, int H, int dk, int dv, kda_dtype dt, void* workspace,
+                         size_t workspace_bytes, kda_stream_t stream)
+{
+    return kda_chunk_fwd_ex(q, k, v, log_alpha, beta, S0, cu_seqlens, num_seqs, out, S_final, B, T, H, dk, dv, dt,
+                            nullptr, workspace, workspace_bytes, stream);
+}
+
+kda_status kda_decode_step_ex(const void* q, const void* k, const void* v, const float* log_alpha,
+                              const float* beta, float* S_inout, void* out, int N, int H, int dk, int dv,
+                              kda_dtype dt, const kda_options* opt, kda_stream_t stream_)
 {
     cudaStream_t stream = (cudaStream_t)stream_;
     if (dt != KDA_BF16 && dt != KDA_F32) return KDA_ERR_INVALID_ARG;
     if (N < 0 || H <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+    int Hk = H;
+    const kda_status so = parse_options(opt, H, Hk);
+    if (so != KDA_OK) return so;
     if (!dims_supported(dk, dv)) return KDA_ERR_UNSUPPORTED;
     if (N == 0) return KDA_OK;
     if (!q || !k || !v || !log_alpha || !beta || !S_inout || !out) return KDA_ERR_INVALID_ARG;
@@ -167,9 +196,16 @@ kda_status kda_decode_step(const void* q, const void* k, const void* v, const fl
     for (const void* x : ptrs)
         if (!aligned16(x)) return KDA_ERR_INVALID_ARG;
     const cudaError_t e = (dt == KDA_BF16)
-        ? launch_decode<__nv_bfloat16>(q, k, v, log_alpha, beta, S_inout, out, N, H, dk, dv, stream)
-        : launch_decode<float>(q, k, v, log_alpha, beta, S_inout, out, N, H, dk, dv, stream);
+        ? launch_decode<__nv_bfloat16>(q, k, v, log_alpha, beta, S_inout, out, N, H, Hk, dk, dv, stream)
+        : launch_decode<float>(q, k, v, log_alpha, beta, S_inout, out, N, H, Hk, dk, dv, stream);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_decode_step(const void* q, const void* k, const void* v, const float* log_alpha, const float* beta,
+                           float* S_inout, void* out, int N, int H, int dk, int dv, kda_dtype dt,
+                           kda_stream_t stream)
+{
+    return kda_decode_step_ex(q, k, v, log_alpha, beta, S_inout, out, N, H, dk, dv, dt, nullptr, stream);
 }
 
 kda_status kda_profile_begin(void)

@@ -43,8 +43,8 @@ template <typename TIn>
 __global__ void __launch_bounds__(kSimtThreads)
 simt_intra_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
                   const float* __restrict__ log_alpha, const float* __restrict__ beta, const WsHeader* __restrict__ hdr,
-                  const int* __restrict__ off, const int32_t* __restrict__ cu, int Tseq, int N, int H, int dk, int dv,
-                  float* __restrict__ slots)
+                  const int* __restrict__ off, const int32_t* __restrict__ cu, int Tseq, int N, int H, int Hk, int dk,
+                  int dv, float* __restrict__ slots)
 {
     extern __shared__ __align__(16) float smem[];
     const int j = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
@@ -71,7 +71,8 @@ simt_intra_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TI
         float kv = 0.f, qv = 0.f, lv = 0.f;
         if (r < L) {
             const size_t gi = ((size_t)(t0 + r) * H + h) * dk + c;
-            kv = to_f32(k[gi]); qv = to_f32(q[gi]); lv = log_alpha[gi];
+            const size_t qi = ((size_t)(t0 + r) * Hk + h / (H / Hk)) * dk + c;  // q/k head of value head h
+            kv = to_f32(k[qi]); qv = to_f32(q[qi]); lv = log_alpha[gi];
         }
         sk[e] = kv; sq[e] = qv; sg[e] = lv;
     }
@@ -273,8 +274,8 @@ inline size_t simt_inter_smem(int dk, int dv)
 template <typename TIn>
 cudaError_t launch_simt_prefill(const void* q, const void* k, const void* v, const float* la, const float* beta,
                                 const float* S0, float* S_final, void* out, const WsHeader* hdr, const int* off,
-                                const int32_t* cu, int Tseq, int N, int H, int dk, int dv, int max_chunks, float* slots,
-                                cudaStream_t stream)
+                                const int32_t* cu, int Tseq, int N, int H, int Hk, int dk, int dv, int max_chunks,
+                                float* slots, cudaStream_t stream)
 {
     const size_t smA = simt_intra_smem(dk, dv), smB = simt_inter_smem(dk, dv);
     cudaError_t e = cudaFuncSetAttribute(simt_intra_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smA);
@@ -284,7 +285,7 @@ cudaError_t launch_simt_prefill(const void* q, const void* k, const void* v, con
     if (max_chunks > 0) {
         LaunchScope ls("simt_intra", stream);
         simt_intra_kernel<TIn><<<dim3(max_chunks, H), kSimtThreads, smA, stream>>>(
-            (const TIn*)q, (const TIn*)k, (const TIn*)v, la, beta, hdr, off, cu, Tseq, N, H, dk, dv, slots);
+            (const TIn*)q, (const TIn*)k, (const TIn*)v, la, beta, hdr, off, cu, Tseq, N, H, Hk, dk, dv, slots);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

@@ -232,7 +232,7 @@ __global__ void __launch_bounds__(kAThreads, 2)
 tc_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_la,
                 const float* __restrict__ beta, WsHeader* __restrict__ hdr, const int* __restrict__ off,
-                const int32_t* __restrict__ cu, int Tseq, int N, int H, uint8_t* __restrict__ slots)
+                const int32_t* __restrict__ cu, int Tseq, int N, int H, int G, uint8_t* __restrict__ slots)
 {
     using namespace tc;
     extern __shared__ uint8_t smem_raw[];
@@ -274,11 +274,12 @@ tc_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tma_load_3d(sb + kA_G, &tm_la, 0, hh, (int)tt, mbar_la);
     };
     auto issue_kq = [&](int hh, long long tt) {  // stacked tile: atom column a = k rows then q rows
+        const int hq = hh / G;                         // the q/k head of value head hh (grouped heads)
         mbar_arrive_expect_tx(mbar_kq, 4 * 8192);
-        tma_load_3d(sb + kA_KQ, &tm_k, 0, hh, (int)tt, mbar_kq);
-        tma_load_3d(sb + kA_KQ + 8192, &tm_q, 0, hh, (int)tt, mbar_kq);
-        tma_load_3d(sb + kA_KQ + kKQ_LBO, &tm_k, 64, hh, (int)tt, mbar_kq);
-        tma_load_3d(sb + kA_KQ + kKQ_LBO + 8192, &tm_q, 64, hh, (int)tt, mbar_kq);
+        tma_load_3d(sb + kA_KQ, &tm_k, 0, hq, (int)tt, mbar_kq);
+        tma_load_3d(sb + kA_KQ + 8192, &tm_q, 0, hq, (int)tt, mbar_kq);
+        tma_load_3d(sb + kA_KQ + kKQ_LBO, &tm_k, 64, hq, (int)tt, mbar_kq);
+        tma_load_3d(sb + kA_KQ + kKQ_LBO + 8192, &tm_q, 64, hq, (int)tt, mbar_kq);
     };
     auto issue_v = [&](int hh, long long tt) {
         mbar_arrive_expect_tx(mbar_v, 2 * 8192);
@@ -948,7 +949,7 @@ inline bool make_token_map(CUtensorMap* m, const void* base, bool bf16, int H, l
 
 inline cudaError_t launch_tc_prefill(const void* q, const void* k, const void* v, const float* la, const float* beta,
                                      const float* S0, float* S_final, void* out, const WsHeader* hdr, const int* off,
-                                     const int32_t* cu, int Tseq, int N, int H, int max_chunks, long long Ttot,
+                                     const int32_t* cu, int Tseq, int N, int H, int Hk, int max_chunks, long long Ttot,
                                      char* slots, cudaStream_t stream)
 {
     cudaError_t e = cudaFuncSetAttribute(tc_intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kA_Smem);
@@ -957,7 +958,7 @@ inline cudaError_t launch_tc_prefill(const void* q, const void* k, const void* v
     if (e != cudaSuccess) return e;
     if (max_chunks > 0 && Ttot > 0) {
         alignas(64) CUtensorMap tq, tk, tv, tla;
-        if (!make_token_map(&tq, q, true, H, Ttot, 64) || !make_token_map(&tk, k, true, H, Ttot, 64) ||
+        if (!make_token_map(&tq, q, true, Hk, Ttot, 64) || !make_token_map(&tk, k, true, Hk, Ttot, 64) ||
             !make_token_map(&tv, v, true, H, Ttot, 64) || !make_token_map(&tla, la, false, H, Ttot, 128))
             return cudaErrorInvalidValue;
         // persistent: two CTAs per SM (the register and shared-memory budget of one CTA is half an SM)
@@ -966,7 +967,7 @@ inline cudaError_t launch_tc_prefill(const void* q, const void* k, const void* v
         const long long units = (long long)max_chunks * H;
         const unsigned grid = (unsigned)(units < 2LL * sms ? units : 2LL * sms);
         LaunchScope ls("tc_intra", stream);
-        tc_intra_kernel<<<grid, kAThreads, kA_Smem, stream>>>(tq, tk, tv, tla, beta, const_cast<WsHeader*>(hdr), off, cu, Tseq, N, H,
+        tc_intra_kernel<<<grid, kAThreads, kA_Smem, stream>>>(tq, tk, tv, tla, beta, const_cast<WsHeader*>(hdr), off, cu, Tseq, N, H, H / Hk,
                                                               (uint8_t*)slots);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;

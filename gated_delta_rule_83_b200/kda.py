@@ -22,12 +22,22 @@ STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED", 3: "K
 
 # The C ABI, as declared in include/kda.h (name -> (restype, argtypes)).
 _P, _I, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+
+
+class KdaOptions(ctypes.Structure):
+    """``kda_options`` of include/kda.h (zero = the plain entry points' behaviour)."""
+    _fields_ = [("num_qk_heads", ctypes.c_int), ("reserved", ctypes.c_int * 7)]
+
+
 ABI = {
     "kda_status_string": (ctypes.c_char_p, [_I]),
     "kda_version": (ctypes.c_char_p, []),
     "kda_chunk_fwd_workspace_size": (_I, [_I, _I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_SZ)]),
     "kda_chunk_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _I, _P, _SZ, _P]),
     "kda_decode_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "kda_chunk_fwd_ex": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _I,
+                              ctypes.POINTER(KdaOptions), _P, _SZ, _P]),
+    "kda_decode_step_ex": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, ctypes.POINTER(KdaOptions), _P]),
     "kda_chunk_fwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
     "kda_check": (_I, [_P]),
     "kda_selftest_timeout": (_I, [_P]),
@@ -127,23 +137,25 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torc
               stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Chunked KDA prefill (``kda_chunk_fwd``).
 
-    q, k, log_alpha: [B, T, H, dk]; v: [B, T, H, dv]; beta: [B, T, H]; q/k/v bf16 or fp32, gates fp32.
+    q, k: [B, T, Hk, dk]; log_alpha: [B, T, H, dk]; v: [B, T, H, dv]; beta: [B, T, H]; q/k/v bf16 or
+    fp32, gates fp32.  Hk = H, or a divisor of H (grouped heads, ``kda_chunk_fwd_ex``: value head h
+    reads q/k head h // (H // Hk)).
     S0 / S_final: [N, H, dk, dv] fp32 (N = B, or len(cu_seqlens) - 1 for packed varlen input with B = 1).
     Returns (out [B, T, H, dv] in q's dtype, S_final or None).  S_final may be S0 (in place)."""
     lib = load_library()
     _req(q, "q")
     dev = q.device
     dtq = q.dtype
-    if q.dim() != 4:
-        raise ValueError("q must be [B, T, H, dk]")
-    B, T, H, dk = q.shape
-    dv = v.shape[-1]
+    if q.dim() != 4 or v.dim() != 4:
+        raise ValueError("q must be [B, T, Hk, dk] and v [B, T, H, dv]")
+    B, T, Hk, dk = q.shape
+    H, dv = v.shape[2], v.shape[-1]
     _req(k, "k", dtq, dev)
     _req(v, "v", dtq, dev)
     _req(log_alpha, "log_alpha", torch.float32, dev)
     _req(beta, "beta", torch.float32, dev)
-    if k.shape != q.shape or log_alpha.shape != q.shape or tuple(v.shape) != (B, T, H, dv) or \
-            tuple(beta.shape) != (B, T, H):
+    if k.shape != q.shape or tuple(log_alpha.shape) != (B, T, H, dk) or tuple(v.shape) != (B, T, H, dv) or \
+            tuple(beta.shape) != (B, T, H) or H % Hk != 0:
         raise ValueError("inconsistent shapes")
     N = B
     if cu_seqlens is not None:
@@ -169,9 +181,17 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torc
         workspace = _get_workspace(ws_bytes, dev, sh)
     else:
         _req(workspace, "workspace", torch.uint8, dev)
-    rc = lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0), _ptr(cu_seqlens), N,
-                           _ptr(out), _ptr(S_final), B, T, H, dk, dv, _dt(q), _ptr(workspace), workspace.numel(), sh)
-    _check("kda_chunk_fwd", rc)
+    if Hk == H:
+        rc = lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0), _ptr(cu_seqlens),
+                               N, _ptr(out), _ptr(S_final), B, T, H, dk, dv, _dt(q), _ptr(workspace),
+                               workspace.numel(), sh)
+        _check("kda_chunk_fwd", rc)
+    else:
+        opt = KdaOptions(num_qk_heads=Hk)
+        rc = lib.kda_chunk_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0),
+                                  _ptr(cu_seqlens), N, _ptr(out), _ptr(S_final), B, T, H, dk, dv, _dt(q),
+                                  ctypes.byref(opt), _ptr(workspace), workspace.numel(), sh)
+        _check("kda_chunk_fwd_ex", rc)
     return out, S_final
 
 
@@ -202,27 +222,34 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: to
                 S: torch.Tensor, out: Optional[torch.Tensor] = None,
                 stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
     """One KDA decode step (``kda_decode_step``); ``S`` [N, H, dk, dv] fp32 is updated in place.
-    q, k, log_alpha: [N, H, dk]; v: [N, H, dv]; beta: [N, H].  Returns out [N, H, dv]."""
+    q, k: [N, Hk, dk]; log_alpha: [N, H, dk]; v: [N, H, dv]; beta: [N, H], with Hk = H or a divisor of
+    H (grouped heads, ``kda_decode_step_ex``).  Returns out [N, H, dv]."""
     lib = load_library()
     _req(q, "q")
     dev, dtq = q.device, q.dtype
-    N, H, dk = q.shape
-    dv = v.shape[-1]
+    N, Hk, dk = q.shape
+    H, dv = v.shape[1], v.shape[-1]
     _req(k, "k", dtq, dev)
     _req(v, "v", dtq, dev)
     _req(log_alpha, "log_alpha", torch.float32, dev)
     _req(beta, "beta", torch.float32, dev)
     _req(S, "S", torch.float32, dev)
-    if k.shape != q.shape or log_alpha.shape != q.shape or tuple(v.shape) != (N, H, dv) or \
-            tuple(beta.shape) != (N, H) or tuple(S.shape) != (N, H, dk, dv):
+    if k.shape != q.shape or tuple(log_alpha.shape) != (N, H, dk) or tuple(v.shape) != (N, H, dv) or \
+            tuple(beta.shape) != (N, H) or tuple(S.shape) != (N, H, dk, dv) or H % Hk != 0:
         raise ValueError("inconsistent shapes")
     if out is None:
         out = torch.empty((N, H, dv), dtype=dtq, device=dev)
     else:
         _req(out, "out", dtq, dev)
-    rc = lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S), _ptr(out), N, H, dk,
-                             dv, _dt(q), _stream_handle(stream, dev))
-    _check("kda_decode_step", rc)
+    if Hk == H:
+        rc = lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S), _ptr(out), N, H,
+                                 dk, dv, _dt(q), _stream_handle(stream, dev))
+        _check("kda_decode_step", rc)
+    else:
+        opt = KdaOptions(num_qk_heads=Hk)
+        rc = lib.kda_decode_step_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S), _ptr(out), N,
+                                    H, dk, dv, _dt(q), ctypes.byref(opt), _stream_handle(stream, dev))
+        _check("kda_decode_step_ex", rc)
     return out
 
 

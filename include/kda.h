@@ -123,6 +123,44 @@ kda_status kda_decode_step(const void* q, const void* k, const void* v, const fl
                            kda_stream_t stream);
 
 /*
+ * Options of the extended entry points kda_chunk_fwd_ex and kda_decode_step_ex.  Zero-initialise
+ * the struct, then set the fields that differ from the plain entry points:
+ *
+ *   num_qk_heads  Grouped q/k heads.  q and k hold Hk = num_qk_heads heads ([B, T, Hk, dk] for the
+ *                 prefill, [N, Hk, dk] for decode) and value head h reads q/k head h / (H / Hk).
+ *                 Every other tensor (v, log_alpha, beta, out, S0, S_final, S_inout) keeps its H
+ *                 heads: the gates and the state belong to the value head.  0 means H (one q/k
+ *                 head per value head, the plain entry points).  H must be a multiple of Hk,
+ *                 else KDA_ERR_INVALID_ARG.  The attention review's GDN pseudo-code
+ *                 (lanjinlin.com.cn, entry on Qwen3-Next GDN) comments its q/k and value head
+ *                 counts separately; this is that layout.
+ *   reserved      Must be zero (KDA_ERR_INVALID_ARG otherwise).
+ */
+typedef struct {
+    int num_qk_heads;
+    int reserved[7];
+} kda_options;
+
+/*
+ * kda_chunk_fwd_ex -- kda_chunk_fwd with options (`opt` may be NULL: the plain behaviour).
+ * Same arguments, layout, workspace (kda_chunk_fwd_workspace_size with the value-head count H),
+ * errors and asynchrony as kda_chunk_fwd; with opt->num_qk_heads = Hk, q and k are [B, T, Hk, dk].
+ */
+kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v, const float* log_alpha, const float* beta,
+                            const float* S0, const int32_t* cu_seqlens, int num_seqs, void* out, float* S_final,
+                            int B, int T, int H, int dk, int dv, kda_dtype dt, const kda_options* opt,
+                            void* workspace, size_t workspace_bytes, kda_stream_t stream);
+
+/*
+ * kda_decode_step_ex -- kda_decode_step with options (`opt` may be NULL: the plain behaviour).
+ * Same arguments, layout and errors as kda_decode_step; with opt->num_qk_heads = Hk, q and k are
+ * [N, Hk, dk].
+ */
+kda_status kda_decode_step_ex(const void* q, const void* k, const void* v, const float* log_alpha,
+                              const float* beta, float* S_inout, void* out, int N, int H, int dk, int dv,
+                              kda_dtype dt, const kda_options* opt, kda_stream_t stream);
+
+/*
  * kda_check -- synchronise `stream`, then read and clear the device error word of the current
  * device.  Returns KDA_OK, KDA_ERR_CUDA (a sticky CUDA error), KDA_ERR_BAD_SEQLENS or
  * KDA_ERR_TIMEOUT.

@@ -18,6 +18,10 @@ arrays into it.  Every function follows a passage of the pages:
 * ``decode_step`` -- one token per sequence, in the loop order (decay, delta, update, output) of
                      the review's GDN pseudo-code.
 
+``seq``, ``chunked`` and ``decode_step`` also take q and k with fewer heads than v (grouped heads:
+value head h reads q/k head h // (H // Hk)), as in the head-count comments of the review's GDN
+pseudo-code.
+
 Pins (checked in ``tests/test_oracle_pins.py``): the beta=0 closed form, exact write/retrieve
 with orthonormal keys at alpha=1 and beta=1, an exact rational worked example, the per-step
 delta invariant, brute force vs sequential, chunked vs sequential for several C, linearity in
@@ -71,6 +75,12 @@ def _load():
         lib.kda_oracle_chunked.restype = I
         lib.kda_oracle_decode_step.argtypes = [P, P, P, P, P, P, I, I, I, I, P]
         lib.kda_oracle_decode_step.restype = I
+        lib.kda_oracle_seq_grouped.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, P, P, P, I]
+        lib.kda_oracle_seq_grouped.restype = I
+        lib.kda_oracle_chunked_grouped.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, P, P, P, I, I]
+        lib.kda_oracle_chunked_grouped.restype = I
+        lib.kda_oracle_decode_step_grouped.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P]
+        lib.kda_oracle_decode_step_grouped.restype = I
         _lib = lib
     return _lib
 
@@ -88,31 +98,36 @@ def default_threads() -> int:
 
 
 def _prep(q, k, v, log_alpha, beta, S0, cu_seqlens):
+    """q, k may have fewer heads (Hk) than v, log_alpha and beta (H), with H a multiple of Hk:
+    value head h then reads q/k head h // (H // Hk) (grouped heads)."""
     q, k, v, la, b = _f32(q), _f32(k), _f32(v), _f32(log_alpha), _f32(beta)
     if q.ndim == 4:  # [B, T, H, d] regular batch -> packed with cu_seqlens
-        B, T, H, dk = q.shape
-        dv = v.shape[-1]
+        B, T, Hk, dk = q.shape
+        H, dv = v.shape[2], v.shape[-1]
         if cu_seqlens is not None:
             raise ValueError("cu_seqlens is only meaningful for packed [Ttot, H, d] inputs")
         cu = np.arange(B + 1, dtype=np.int64) * T
-        q, k, la = (x.reshape(B * T, H, dk) for x in (q, k, la))
+        q, k = (x.reshape(B * T, Hk, dk) for x in (q, k))
+        la = la.reshape(B * T, H, dk)
         v = v.reshape(B * T, H, dv)
         b = b.reshape(B * T, H)
     else:
-        Ttot, H, dk = q.shape
-        dv = v.shape[-1]
+        Ttot, Hk, dk = q.shape
+        H, dv = v.shape[1], v.shape[-1]
         cu = (np.array([0, Ttot], dtype=np.int64) if cu_seqlens is None
               else np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64)))
     N = len(cu) - 1
-    if k.shape != q.shape or la.shape != q.shape or v.shape[:2] != q.shape[:2] or b.shape != q.shape[:2]:
+    Ttot = q.shape[0]
+    if k.shape != q.shape or la.shape != (Ttot, H, dk) or v.shape[:2] != (Ttot, H) or b.shape != (Ttot, H) \
+            or H % Hk != 0:
         raise ValueError("inconsistent shapes")
     s0 = None if S0 is None else np.ascontiguousarray(np.asarray(S0, dtype=np.float64).reshape(N, H, dk, dv))
-    return q, k, v, la, b, s0, cu, N, H, dk, dv
+    return q, k, v, la, b, s0, cu, N, H, Hk, dk, dv
 
 
 def _call(fname, q, k, v, log_alpha, beta, S0, cu_seqlens, pairs, threads, extra=()):
     shape4 = np.asarray(q).ndim == 4
-    q, k, v, la, b, s0, cu, N, H, dk, dv = _prep(q, k, v, log_alpha, beta, S0, cu_seqlens)
+    q, k, v, la, b, s0, cu, N, H, Hk, dk, dv = _prep(q, k, v, log_alpha, beta, S0, cu_seqlens)
     Ttot = q.shape[0]
     out = np.zeros((Ttot, H, dv), dtype=np.float64)
     sf = np.zeros((N, H, dk, dv), dtype=np.float64)
@@ -122,9 +137,14 @@ def _call(fname, q, k, v, log_alpha, beta, S0, cu_seqlens, pairs, threads, extra
         for n, h in pairs:
             mask[n * H + h] = 1
     lib = _load()
-    fn = getattr(lib, fname)
-    rc = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(b), _ptr(s0), _ptr(cu), N, H, dk, dv,
-            _ptr(out), _ptr(sf), _ptr(mask), *extra, threads or default_threads())
+    if Hk != H:
+        if fname != "kda_oracle_seq":
+            raise ValueError(f"{fname} takes one q/k head per value head")
+        rc = lib.kda_oracle_seq_grouped(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(b), _ptr(s0), _ptr(cu), N, H,
+                                        Hk, dk, dv, _ptr(out), _ptr(sf), _ptr(mask), threads or default_threads())
+    else:
+        rc = getattr(lib, fname)(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(b), _ptr(s0), _ptr(cu), N, H, dk, dv,
+                                 _ptr(out), _ptr(sf), _ptr(mask), *extra, threads or default_threads())
     if rc != 0:
         raise RuntimeError(f"{fname} failed with status {rc}")
     if shape4:
@@ -151,7 +171,7 @@ def chunked(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, C=64, pairs=None
     """Chunked WY/UT form with chunk size ``C``."""
     # the C entry point takes C before the thread count
     shape4 = np.asarray(q).ndim == 4
-    q_, k_, v_, la, b, s0, cu, N, H, dk, dv = _prep(q, k, v, log_alpha, beta, S0, cu_seqlens)
+    q_, k_, v_, la, b, s0, cu, N, H, Hk, dk, dv = _prep(q, k, v, log_alpha, beta, S0, cu_seqlens)
     Ttot = q_.shape[0]
     out = np.zeros((Ttot, H, dv), dtype=np.float64)
     sf = np.zeros((N, H, dk, dv), dtype=np.float64)
@@ -160,9 +180,9 @@ def chunked(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, C=64, pairs=None
         mask = np.zeros(N * H, dtype=np.int32)
         for n, h in pairs:
             mask[n * H + h] = 1
-    rc = _load().kda_oracle_chunked(_ptr(q_), _ptr(k_), _ptr(v_), _ptr(la), _ptr(b), _ptr(s0), _ptr(cu), N, H,
-                                    dk, dv, _ptr(out), _ptr(sf), _ptr(mask), int(C),
-                                    threads or default_threads())
+    rc = _load().kda_oracle_chunked_grouped(_ptr(q_), _ptr(k_), _ptr(v_), _ptr(la), _ptr(b), _ptr(s0), _ptr(cu),
+                                            N, H, Hk, dk, dv, _ptr(out), _ptr(sf), _ptr(mask), int(C),
+                                            threads or default_threads())
     if rc != 0:
         raise RuntimeError(f"kda_oracle_chunked failed with status {rc}")
     if shape4:
@@ -171,16 +191,19 @@ def chunked(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, C=64, pairs=None
 
 
 def decode_step(q, k, v, log_alpha, beta, S):
-    """One token for each of N sequences.  ``q,k,log_alpha [N,H,dk]``, ``v [N,H,dv]``,
-    ``beta [N,H]``, ``S [N,H,dk,dv]`` (float64, returned updated as a new array).
+    """One token for each of N sequences.  ``q,k [N,Hk,dk]``, ``log_alpha [N,H,dk]``, ``v [N,H,dv]``,
+    ``beta [N,H]``, ``S [N,H,dk,dv]`` (float64, returned updated as a new array); Hk = H, or a
+    divisor of H (value head h reads q/k head h // (H // Hk)).
     Returns ``(out [N,H,dv] float64, S_new)``."""
     q, k, v, la, b = _f32(q), _f32(k), _f32(v), _f32(log_alpha), _f32(beta)
-    N, H, dk = q.shape
-    dv = v.shape[-1]
+    N, Hk, dk = q.shape
+    H, dv = v.shape[1], v.shape[-1]
+    if k.shape != q.shape or la.shape != (N, H, dk) or b.shape != (N, H) or H % Hk != 0:
+        raise ValueError("inconsistent shapes")
     S = np.array(S, dtype=np.float64, copy=True, order="C").reshape(N, H, dk, dv)
     out = np.zeros((N, H, dv), dtype=np.float64)
-    rc = _load().kda_oracle_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(b), _ptr(S), N, H, dk, dv,
-                                        _ptr(out))
+    rc = _load().kda_oracle_decode_step_grouped(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(b), _ptr(S), N, H, Hk,
+                                                dk, dv, _ptr(out))
     if rc != 0:
         raise RuntimeError(f"kda_oracle_decode_step failed with status {rc}")
     return out, S

@@ -42,6 +42,8 @@
 #include <string.h>
 
 #define IDX3(t, h, c, H, D) (((size_t)(t) * (size_t)(H) + (size_t)(h)) * (size_t)(D) + (size_t)(c))
+/* q and k of value head h: head h / (H / Hk) of the Hk q/k heads */
+#define QKIDX(J, t, h, c) IDX3(t, (h) / ((J)->H / (J)->Hk), c, (J)->Hk, (J)->dk)
 
 typedef struct {
     const float *q, *k, *v, *log_alpha, *beta;
@@ -49,6 +51,7 @@ typedef struct {
     const int64_t* cu_seqlens;
     const int32_t* pair_mask;
     int N, H, dk, dv, C;
+    int Hk; /* q/k heads; value head h reads q/k head h / (H / Hk) (grouped heads); Hk = H: one each */
     double *out, *S_final;
     int mode; /* 0 = sequential, 1 = chunked, 2 = brute force */
     int next_pair;
@@ -67,8 +70,8 @@ static void pair_seq(const job_t* J, int n, int h, double* S, double* w)
     const int H = J->H, dk = J->dk, dv = J->dv;
     const int64_t t0 = J->cu_seqlens[n], t1 = J->cu_seqlens[n + 1];
     for (int64_t t = t0; t < t1; ++t) {
-        const float* kt = J->k + IDX3(t, h, 0, H, dk);
-        const float* qt = J->q + IDX3(t, h, 0, H, dk);
+        const float* kt = J->k + QKIDX(J, t, h, 0);
+        const float* qt = J->q + QKIDX(J, t, h, 0);
         const float* vt = J->v + IDX3(t, h, 0, H, dv);
         const float* la = J->log_alpha + IDX3(t, h, 0, H, dk);
         const double b = (double)J->beta[(size_t)t * H + h];
@@ -110,8 +113,8 @@ static void pair_bruteforce(const job_t* J, int n, int h, double* S, double* M, 
     const int H = J->H, dk = J->dk, dv = J->dv;
     const int64_t t0 = J->cu_seqlens[n], t1 = J->cu_seqlens[n + 1];
     for (int64_t t = t0; t < t1; ++t) {
-        const float* kt = J->k + IDX3(t, h, 0, H, dk);
-        const float* qt = J->q + IDX3(t, h, 0, H, dk);
+        const float* kt = J->k + QKIDX(J, t, h, 0);
+        const float* qt = J->q + QKIDX(J, t, h, 0);
         const float* vt = J->v + IDX3(t, h, 0, H, dv);
         const float* la = J->log_alpha + IDX3(t, h, 0, H, dk);
         const double b = (double)J->beta[(size_t)t * H + h];
@@ -182,7 +185,7 @@ static void pair_chunked(const job_t* J, int n, int h, double* S, double* scratc
                 double acc = 0.0;
                 if (i < r)
                     for (int c = 0; c < dk; ++c)
-                        acc += (double)J->k[IDX3(cs + r, h, c, H, dk)] * (double)J->k[IDX3(cs + i, h, c, H, dk)] *
+                        acc += (double)J->k[QKIDX(J, cs + r, h, c)] * (double)J->k[QKIDX(J, cs + i, h, c)] *
                                exp(g[(size_t)r * dk + c] - g[(size_t)i * dk + c]);
                 A[(size_t)r * C + i] = br * acc;
             }
@@ -200,7 +203,7 @@ static void pair_chunked(const job_t* J, int n, int h, double* S, double* scratc
             for (int c = 0; c < dk; ++c) {
                 double acc = 0.0;
                 for (int i = 0; i < L; ++i)
-                    acc += Tm[(size_t)r * C + i] * (double)J->k[IDX3(cs + i, h, c, H, dk)] * exp(g[(size_t)i * dk + c]);
+                    acc += Tm[(size_t)r * C + i] * (double)J->k[QKIDX(J, cs + i, h, c)] * exp(g[(size_t)i * dk + c]);
                 W[(size_t)r * dk + c] = acc;
             }
             for (int j = 0; j < dv; ++j) {
@@ -223,13 +226,13 @@ static void pair_chunked(const job_t* J, int n, int h, double* S, double* scratc
                 for (int j = 0; j < dv; ++j) {
                     double acc = 0.0;
                     for (int c = 0; c < dk; ++c)
-                        acc += (double)J->q[IDX3(cs + r, h, c, H, dk)] * exp(g[(size_t)r * dk + c]) * S[(size_t)c * dv + j];
+                        acc += (double)J->q[QKIDX(J, cs + r, h, c)] * exp(g[(size_t)r * dk + c]) * S[(size_t)c * dv + j];
                     o[j] = acc;
                 }
                 for (int i = 0; i <= r; ++i) {
                     double p = 0.0;
                     for (int c = 0; c < dk; ++c)
-                        p += (double)J->q[IDX3(cs + r, h, c, H, dk)] * (double)J->k[IDX3(cs + i, h, c, H, dk)] *
+                        p += (double)J->q[QKIDX(J, cs + r, h, c)] * (double)J->k[QKIDX(J, cs + i, h, c)] *
                              exp(g[(size_t)r * dk + c] - g[(size_t)i * dk + c]);
                     for (int j = 0; j < dv; ++j) o[j] += p * U[(size_t)i * dv + j];
                 }
@@ -241,7 +244,7 @@ static void pair_chunked(const job_t* J, int n, int h, double* S, double* scratc
             for (int j = 0; j < dv; ++j) {
                 double acc = exp(glast[c]) * S[(size_t)c * dv + j];
                 for (int i = 0; i < L; ++i)
-                    acc += (double)J->k[IDX3(cs + i, h, c, H, dk)] * exp(glast[c] - g[(size_t)i * dk + c]) *
+                    acc += (double)J->k[QKIDX(J, cs + i, h, c)] * exp(glast[c] - g[(size_t)i * dk + c]) *
                            U[(size_t)i * dv + j];
                 Snew[(size_t)c * dv + j] = acc;
             }
@@ -288,6 +291,7 @@ static int run(job_t* J, int num_threads)
 {
     if (!J->q || !J->k || !J->v || !J->log_alpha || !J->beta || !J->cu_seqlens) return -1;
     if (J->N < 0 || J->H <= 0 || J->dk <= 0 || J->dv <= 0) return -1;
+    if (J->Hk <= 0 || J->H % J->Hk != 0) return -1;
     for (int n = 0; n < J->N; ++n)
         if (J->cu_seqlens[n + 1] < J->cu_seqlens[n]) return -1;
     if (num_threads < 1) num_threads = 1;
@@ -310,7 +314,7 @@ static int run(job_t* J, int num_threads)
     memset(&J, 0, sizeof(J));                                                                     \
     J.q = q; J.k = k; J.v = v; J.log_alpha = log_alpha; J.beta = beta; J.S0 = S0;                \
     J.cu_seqlens = cu_seqlens; J.pair_mask = pair_mask; J.N = N; J.H = H; J.dk = dk; J.dv = dv;   \
-    J.C = (C_); J.out = out; J.S_final = S_final; J.mode = (mode_);
+    J.C = (C_); J.out = out; J.S_final = S_final; J.mode = (mode_); J.Hk = H;
 
 /* The definition (sequential recurrence).  pair_mask: [N*H] (index n*H+h), nonzero = compute
  * that pair, NULL = all pairs.  Returns 0 on success, -1 on bad arguments, -2 out of memory. */
@@ -341,22 +345,48 @@ int kda_oracle_chunked(const float* q, const float* k, const float* v, const flo
     return run(&J, num_threads);
 }
 
+/* Grouped q/k heads: q and k are [Ttot][Hk][dk] and value head h reads q/k head h / (H / Hk);
+ * v, log_alpha, beta, out and the states keep their H heads.  Hk = H is kda_oracle_seq /
+ * kda_oracle_chunked. */
+int kda_oracle_seq_grouped(const float* q, const float* k, const float* v, const float* log_alpha,
+                           const float* beta, const double* S0, const int64_t* cu_seqlens, int N, int H, int Hk,
+                           int dk, int dv, double* out, double* S_final, const int32_t* pair_mask, int num_threads)
+{
+    FILL_JOB(J, 0, 1);
+    J.Hk = Hk;
+    return run(&J, num_threads);
+}
+
+int kda_oracle_chunked_grouped(const float* q, const float* k, const float* v, const float* log_alpha,
+                               const float* beta, const double* S0, const int64_t* cu_seqlens, int N, int H, int Hk,
+                               int dk, int dv, double* out, double* S_final, const int32_t* pair_mask, int C,
+                               int num_threads)
+{
+    if (C < 1) return -1;
+    FILL_JOB(J, 1, C);
+    J.Hk = Hk;
+    return run(&J, num_threads);
+}
+
 /* One decode step for N independent sequences, in the loop order of the review's pseudo-code:
  *   (a) decay       S' = S * exp(log_alpha)    (row c scaled)
  *   (b) delta       d  = S'^T k,   v_mod = v - d
  *   (c) update      S  = S' + k (beta v_mod)^T
  *   (d) output      o  = S^T q                  (from the updated state)
- * q, k, log_alpha: [N][H][dk]; v: [N][H][dv]; beta: [N][H]; S: [N][H][dk][dv] in/out; out: [N][H][dv]. */
-int kda_oracle_decode_step(const float* q, const float* k, const float* v, const float* log_alpha,
-                           const float* beta, double* S, int N, int H, int dk, int dv, double* out)
+ * q, k: [N][Hk][dk] (value head h reads q/k head h / (H / Hk)); log_alpha: [N][H][dk]; v: [N][H][dv];
+ * beta: [N][H]; S: [N][H][dk][dv] in/out; out: [N][H][dv]. */
+int kda_oracle_decode_step_grouped(const float* q, const float* k, const float* v, const float* log_alpha,
+                                   const float* beta, double* S, int N, int H, int Hk, int dk, int dv, double* out)
 {
     if (!q || !k || !v || !log_alpha || !beta || !S || N < 0 || H <= 0 || dk <= 0 || dv <= 0) return -1;
+    if (Hk <= 0 || H % Hk != 0) return -1;
     double* d = (double*)malloc(sizeof(double) * (size_t)dv);
     if (!d) return -2;
     for (int p = 0; p < N * H; ++p) {
         double* Sp = S + (size_t)p * dk * dv;
-        const float* kp = k + (size_t)p * dk;
-        const float* qp = q + (size_t)p * dk;
+        const size_t pk = (size_t)(p / H) * Hk + (size_t)((p % H) / (H / Hk));  /* q/k head of pair p */
+        const float* kp = k + pk * dk;
+        const float* qp = q + pk * dk;
         const float* vp = v + (size_t)p * dv;
         const float* lp = log_alpha + (size_t)p * dk;
         const double b = (double)beta[p];
@@ -380,4 +410,11 @@ int kda_oracle_decode_step(const float* q, const float* k, const float* v, const
     }
     free(d);
     return 0;
+}
+
+/* Hk = H: one q/k head per value head. */
+int kda_oracle_decode_step(const float* q, const float* k, const float* v, const float* log_alpha,
+                           const float* beta, double* S, int N, int H, int dk, int dv, double* out)
+{
+    return kda_oracle_decode_step_grouped(q, k, v, log_alpha, beta, S, N, H, H, dk, dv, out);
 }

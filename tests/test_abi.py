@@ -95,6 +95,30 @@ def test_decode_rejects_before_launch(lib):
     assert lib.kda_decode_step(None, None, None, None, None, None, None, 0, 2, 64, 64, 0, None) == 0
 
 
+def test_options_are_validated_before_launch(lib):
+    """kda_options: num_qk_heads must divide H and the reserved words must be zero; a NULL or
+    zeroed options struct behaves like the plain entry point (here: the same argument errors)."""
+    from gated_delta_rule_83_b200.kda import KdaOptions
+    fake = 0x100000  # never dereferenced
+    args = (fake, fake, fake, fake, fake, None, None, 0, fake, None, 1, 64, 6, 64, 64, 1)
+    bad_group = KdaOptions(num_qk_heads=4)          # 6 % 4 != 0
+    assert lib.kda_chunk_fwd_ex(*args, ctypes.byref(bad_group), fake, 1 << 30, None) == 1
+    neg = KdaOptions(num_qk_heads=-2)
+    assert lib.kda_chunk_fwd_ex(*args, ctypes.byref(neg), fake, 1 << 30, None) == 1
+    res = KdaOptions(num_qk_heads=3)
+    res.reserved[2] = 1
+    assert lib.kda_chunk_fwd_ex(*args, ctypes.byref(res), fake, 1 << 30, None) == 1
+    ok_group = KdaOptions(num_qk_heads=3)
+    # a valid group with a missing workspace fails only on the workspace, like kda_chunk_fwd
+    assert lib.kda_chunk_fwd_ex(*args, ctypes.byref(ok_group), None, 1 << 30, None) == 5
+    assert lib.kda_chunk_fwd_ex(*args, None, None, 1 << 30, None) == 5
+    dargs = (fake, fake, fake, fake, fake, fake, fake, 4, 6, 64, 64, 0)
+    assert lib.kda_decode_step_ex(*dargs, ctypes.byref(bad_group), None) == 1
+    assert lib.kda_decode_step_ex(*dargs[:6], fake + 4, *dargs[7:], ctypes.byref(ok_group), None) == 1  # misaligned out
+    assert lib.kda_decode_step_ex(None, None, None, None, None, None, None, 0, 6, 64, 64, 0,
+                                  ctypes.byref(ok_group), None) == 0  # N = 0: no-op
+
+
 def test_missing_library_fails_loudly(tmp_path):
     from gated_delta_rule_83_b200 import kda
     with pytest.raises(ImportError):

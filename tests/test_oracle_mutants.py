@@ -36,6 +36,9 @@ MUTANTS = [
     ("chunked: P excludes the diagonal",
      "for (int i = 0; i <= r; ++i) {\n                    double p = 0.0;",
      "for (int i = 0; i < r; ++i) {\n                    double p = 0.0;"),
+    ("grouped: value head h reads q/k head h % Hk",
+     "#define QKIDX(J, t, h, c) IDX3(t, (h) / ((J)->H / (J)->Hk), c, (J)->Hk, (J)->dk)",
+     "#define QKIDX(J, t, h, c) IDX3(t, (h) % (J)->Hk, c, (J)->Hk, (J)->dk)"),
     ("decode: output from the decayed (pre-update) state",
      "for (int c = 0; c < dk; ++c)\n            for (int j = 0; j < dv; ++j) Sp[(size_t)c * dv + j] += (double)kp[c] * (b * d[j]);\n        if (out)",
      "if (out)"),
@@ -53,6 +56,7 @@ def _pins():
         lambda o: pins.test_chunked_vs_seq(o, 16),
         lambda o: pins.test_decode_equals_prefill(o),
         lambda o: pins.test_per_step_invariant(o),
+        lambda o: pins.test_grouped_heads_equal_repeated_qk(o, "seq"),
     ]
 
 

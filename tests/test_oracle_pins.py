@@ -286,3 +286,39 @@ def test_identity_and_empty(oracle):
     o2, s2 = oracle.seq(q, k, v, la, b, S0=np.zeros((1, 1, 4, 4)))
     np.testing.assert_array_equal(o1, o2)
     np.testing.assert_array_equal(s1, s2)
+
+
+# ---------------------------------------------------------------------------------------------
+# 13. grouped q/k heads (the head-count comments of the review's GDN pseudo-code: fewer q/k heads
+#     than value heads, each q/k head shared by a group of value heads)
+# ---------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("form", ["seq", "chunked", "decode"])
+def test_grouped_heads_equal_repeated_qk(oracle, form):
+    """A grouped call must equal the one-head-per-value-head call on q and k repeated by numpy
+    (np.repeat along the head axis).  Catches: value head h reading q/k head h % Hk instead of
+    h // (H // Hk), or reading the value-head index into the smaller q/k array."""
+    H, Hk, dk, dv = 6, 2, 8, 8
+    G = H // Hk
+    if form == "decode":
+        rng = np.random.default_rng(21)
+        N = 3
+        q = rng.standard_normal((N, Hk, dk)).astype(np.float32)
+        k = rng.standard_normal((N, Hk, dk)).astype(np.float32)
+        v = rng.standard_normal((N, H, dv)).astype(np.float32)
+        la = np.log(1.0 / (1.0 + np.exp(-rng.normal(3.0, 1.0, (N, H, dk))))).astype(np.float32)
+        b = rng.uniform(0.0, 1.0, (N, H)).astype(np.float32)
+        S = rng.standard_normal((N, H, dk, dv))
+        o_g, s_g = oracle.decode_step(q, k, v, la, b, S)
+        o_r, s_r = oracle.decode_step(np.repeat(q, G, axis=1), np.repeat(k, G, axis=1), v, la, b, S)
+    else:
+        Ttot = 150
+        q, k, v, la, b, S0 = rand_case(22, Ttot, H, dk, dv)
+        q, k = q[:, :Hk], k[:, :Hk]
+        cu = np.array([0, 70, 150], dtype=np.int64)
+        S0 = np.random.default_rng(23).standard_normal((2, H, dk, dv))
+        fn = oracle.seq if form == "seq" else (lambda *a, **kw: oracle.chunked(*a, C=16, **kw))
+        o_g, s_g = fn(q, k, v, la, b, S0=S0, cu_seqlens=cu)
+        o_r, s_r = fn(np.repeat(q, G, axis=1), np.repeat(k, G, axis=1), v, la, b, S0=S0, cu_seqlens=cu)
+    assert np.array_equal(o_g, o_r) and np.array_equal(s_g, s_r)
+    # and the groups really share: value heads of one group differ only through v, gates and state
+    assert rel(o_g[..., 0, :], o_g[..., 1, :]) > 1e-3

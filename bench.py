@@ -365,6 +365,14 @@ def run_ours(args):
         for name in ("varlen_64k", "long_1m"):
             torch.cuda.empty_cache()
             extra[name] = bench_prefill_workload(torch, kda, synth, dev, stream, world, rank, name, steps=3, warmup=2)
+        torch.cuda.empty_cache()
+        # grouped q/k heads (kda_chunk_fwd_ex): the 32K workload with 16 q/k heads shared by 32 value heads
+        extra["prefill_32k_qk16"] = bench_prefill_workload(torch, kda, synth, dev, stream, world, rank,
+                                                           "prefill_32k", steps=5, warmup=2, qk_heads=16)
+        torch.cuda.empty_cache()
+        # input prologue (kda_options.prologue = all bits): raw q/k and gate/beta logits, transformed in-kernel
+        extra["prefill_32k_prologue"] = bench_prefill_workload(torch, kda, synth, dev, stream, world, rank,
+                                                               "prefill_32k", steps=5, warmup=2, prologue=7)
 
     decode = None
     if not args.no_decode and args.only is None:
@@ -392,18 +400,25 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def bench_prefill_workload(torch, kda, synth, dev, stream, world, rank, name, steps, warmup):
-    """Device-timed throughput of another prefill workload (same method as the headline)."""
+def bench_prefill_workload(torch, kda, synth, dev, stream, world, rank, name, steps, warmup, qk_heads=None,
+                           prologue=0):
+    """Device-timed throughput of another prefill workload (same method as the headline).  With
+    ``qk_heads``, q and k keep only that many heads, shared by groups of value heads.  With
+    ``prologue`` the call passes that kda_options.prologue value (the workload's inputs stand in
+    for raw projections: the in-kernel transforms cost the same whatever the values)."""
     w = synth.WORKLOADS[name]
     inp = synth.prefill_inputs(w, device=dev, seed=replica_seed(w.seed, rank))
     q, k, v, la, beta, S0, cu = (inp[x] for x in ("q", "k", "v", "log_alpha", "beta", "S0", "cu_seqlens"))
+    if qk_heads is not None:
+        q, k = q[:, :, :qk_heads].contiguous(), k[:, :, :qk_heads].contiguous()
+        inp["q"], inp["k"] = q, k
     out = torch.empty_like(v)
     N = q.shape[0] if cu is None else cu.numel() - 1
     S_fin = torch.empty((N, w.H, w.dk, w.dv), dtype=torch.float32, device=dev)
     tokens = q.shape[0] * q.shape[1]
 
     def step():
-        kda.chunk_fwd(q, k, v, la, beta, S0=S0, cu_seqlens=cu, out=out, S_final=S_fin)
+        kda.chunk_fwd(q, k, v, la, beta, S0=S0, cu_seqlens=cu, out=out, S_final=S_fin, prologue=prologue)
 
     for _ in range(warmup):
         step()
@@ -421,7 +436,10 @@ def bench_prefill_workload(torch, kda, synth, dev, stream, world, rank, name, st
     prof = kda.profile_end()
     kda.check()
     ms = max_over_ranks(torch, world, e0.elapsed_time(e1))
-    res = {"desc": w.desc, "tokens": tokens, "steps": steps, "ms_per_step": ms / steps,
+    desc = w.desc if qk_heads is None else f"{w.desc}; q/k with {qk_heads} heads shared by groups of value heads"
+    if prologue:
+        desc += f"; input prologue {prologue} (q/k L2 norm, log-sigmoid gate logits, sigmoid beta logits in-kernel)"
+    res = {"desc": desc, "tokens": tokens, "steps": steps, "ms_per_step": ms / steps,
            "value": job_throughput(world, tokens, steps, ms), "unit": "tokens/s",
            "kernels": {k_: {"launches": n, "ms": t} for k_, (n, t) in prof.items()}}
     del inp, q, k, v, la, beta, S0, out, S_fin

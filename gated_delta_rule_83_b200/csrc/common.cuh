@@ -26,6 +26,12 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 // Chunk length used by every prefill path.
 constexpr int kChunk = 64;
 
+// Input prologue (kda_options.prologue): activations of raw projections, in fp32.
+constexpr float kQkNormEps = 1e-6f;  // x / sqrt(sum x^2 + eps) for the q/k L2 normalisation
+__device__ __forceinline__ float sigmoid_f(float x) { return 1.f / (1.f + expf(-x)); }
+// log sigmoid(x) = min(x, 0) - log(1 + e^{-|x|}), written so that neither branch overflows
+__device__ __forceinline__ float log_sigmoid_f(float x) { return fminf(x, 0.f) - log1pf(expf(-fabsf(x))); }
+
 // Workspace header written by the chunk-table kernel (first 256 bytes of every workspace).
 struct WsHeader {
     int total_chunks;   // sum over sequences of ceil(len / 64)

@@ -22,11 +22,11 @@ namespace kda {
 constexpr int kDecodeThreads = 256;
 constexpr int kDecodeSlice = 64;  // columns of S per CTA
 
-template <typename TIn, int DK, bool GROUPED>
+template <typename TIn, int DK, bool GROUPED, bool PRO>
 __global__ void __launch_bounds__(kDecodeThreads, 3)
 decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
                    const float* __restrict__ log_alpha, const float* __restrict__ beta, float* __restrict__ S,
-                   TIn* __restrict__ out, int dv, int H, int G)
+                   TIn* __restrict__ out, int dv, int H, int G, unsigned pro)
 {
     constexpr int RPT = DK / 16;  // state rows held per thread
     const int nslices = dv / kDecodeSlice;
@@ -48,13 +48,42 @@ decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const T
         st[i] = __ldcs(reinterpret_cast<const float4*>(Sp + (size_t)(rb + 16 * i) * dv) + cg);
 
     // the step's small inputs, loaded alongside the state so that no load sits on the critical path
-    const float b = beta[p];
+    const float b = (PRO && (pro & KDA_PROLOGUE_BETA_LOGITS)) ? sigmoid_f(beta[p]) : beta[p];
     const TIn* vp = v + (size_t)p * dv + j0 + 4 * cg;
     const float v0 = to_f32(vp[0]), v1 = to_f32(vp[1]), v2 = to_f32(vp[2]), v3 = to_f32(vp[3]);
     for (int c = tid; c < DK; c += kDecodeThreads) {
-        s_a[c] = expf(log_alpha[(size_t)p * DK + c]);
+        const float la = log_alpha[(size_t)p * DK + c];
+        s_a[c] = (PRO && (pro & KDA_PROLOGUE_GATE_LOGITS)) ? sigmoid_f(la) : expf(la);  // alpha = sigmoid(logit)
         s_k[c] = to_f32(k[(size_t)pq * DK + c]);
         s_q[c] = to_f32(q[(size_t)pq * DK + c]);
+    }
+    if (PRO && (pro & KDA_PROLOGUE_L2NORM_QK)) {  // q and k normalised over d_k (threads 0..DK-1 hold them)
+        __shared__ float s_nrm[DK / 32][2];
+        float kk = 0.f, qq = 0.f;
+        if (tid < DK) {
+            kk = s_k[tid] * s_k[tid];
+            qq = s_q[tid] * s_q[tid];
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            kk += __shfl_xor_sync(0xffffffffu, kk, o);
+            qq += __shfl_xor_sync(0xffffffffu, qq, o);
+        }
+        if (tid < DK && l == 0) {
+            s_nrm[w][0] = kk;
+            s_nrm[w][1] = qq;
+        }
+        __syncthreads();
+        if (tid < DK) {
+            float sk = 0.f, sq = 0.f;
+#pragma unroll
+            for (int i = 0; i < DK / 32; ++i) {
+                sk += s_nrm[i][0];
+                sq += s_nrm[i][1];
+            }
+            s_k[tid] = to_f32(from_f32<TIn>(s_k[tid] * rsqrtf(sk + kQkNormEps)));
+            s_q[tid] = to_f32(from_f32<TIn>(s_q[tid] * rsqrtf(sq + kQkNormEps)));
+        }
     }
     __syncthreads();
 
@@ -119,7 +148,7 @@ decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const T
 
 template <typename TIn>
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* la, const float* beta, float* S,
-                          void* out, int N, int H, int Hk, int dk, int dv, cudaStream_t stream)
+                          void* out, int N, int H, int Hk, unsigned pro, int dk, int dv, cudaStream_t stream)
 {
     const long long pairs = (long long)N * H;
     const long long blocks = pairs * (dv / kDecodeSlice);
@@ -129,13 +158,23 @@ cudaError_t launch_decode(const void* q, const void* k, const void* v, const flo
     const int G = H / Hk;
     const dim3 grid((unsigned)blocks);
     const TIn *qq = (const TIn*)q, *kk = (const TIn*)k, *vv = (const TIn*)v;
+    TIn* oo = (TIn*)out;
+    // one instantiation per (d_k, grouped, prologue) so that the plain step carries none of the options
+#define KDA_DECODE_LAUNCH(DKV, GR, PR) \
+    decode_step_kernel<TIn, DKV, GR, PR><<<grid, kDecodeThreads, 0, stream>>>(qq, kk, vv, la, beta, S, oo, dv, H, G, pro)
+    const bool gr = G != 1, pr = pro != 0;
     if (dk == 128) {
-        if (G == 1) decode_step_kernel<TIn, 128, false><<<grid, kDecodeThreads, 0, stream>>>(qq, kk, vv, la, beta, S, (TIn*)out, dv, H, G);
-        else decode_step_kernel<TIn, 128, true><<<grid, kDecodeThreads, 0, stream>>>(qq, kk, vv, la, beta, S, (TIn*)out, dv, H, G);
+        if (!gr && !pr) KDA_DECODE_LAUNCH(128, false, false);
+        else if (gr && !pr) KDA_DECODE_LAUNCH(128, true, false);
+        else if (!gr) KDA_DECODE_LAUNCH(128, false, true);
+        else KDA_DECODE_LAUNCH(128, true, true);
     } else {
-        if (G == 1) decode_step_kernel<TIn, 64, false><<<grid, kDecodeThreads, 0, stream>>>(qq, kk, vv, la, beta, S, (TIn*)out, dv, H, G);
-        else decode_step_kernel<TIn, 64, true><<<grid, kDecodeThreads, 0, stream>>>(qq, kk, vv, la, beta, S, (TIn*)out, dv, H, G);
+        if (!gr && !pr) KDA_DECODE_LAUNCH(64, false, false);
+        else if (gr && !pr) KDA_DECODE_LAUNCH(64, true, false);
+        else if (!gr) KDA_DECODE_LAUNCH(64, false, true);
+        else KDA_DECODE_LAUNCH(64, true, true);
     }
+#undef KDA_DECODE_LAUNCH
     return cudaGetLastError();
 }
 

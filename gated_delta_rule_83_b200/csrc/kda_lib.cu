@@ -80,10 +80,12 @@ kda_status make_plan(int B, int T, int H, int dk, int dv, bool varlen, int num_s
     return KDA_OK;
 }
 
-// Options of the extended entry points: Hk = q/k heads (0 -> H); reserved fields must be zero.
-kda_status parse_options(const kda_options* opt, int H, int& Hk)
+// Options of the extended entry points: Hk = q/k heads (0 -> H), prologue bits; reserved fields
+// must be zero.
+kda_status parse_options(const kda_options* opt, int H, int& Hk, unsigned& pro)
 {
     Hk = H;
+    pro = 0;
     if (!opt) return KDA_OK;
     for (int r : opt->reserved)
         if (r != 0) return KDA_ERR_INVALID_ARG;
@@ -91,6 +93,9 @@ kda_status parse_options(const kda_options* opt, int H, int& Hk)
         if (opt->num_qk_heads < 0 || H % opt->num_qk_heads != 0) return KDA_ERR_INVALID_ARG;
         Hk = opt->num_qk_heads;
     }
+    const unsigned known = KDA_PROLOGUE_L2NORM_QK | KDA_PROLOGUE_GATE_LOGITS | KDA_PROLOGUE_BETA_LOGITS;
+    if (opt->prologue & ~known) return KDA_ERR_INVALID_ARG;
+    pro = opt->prologue;
     return KDA_OK;
 }
 
@@ -132,7 +137,8 @@ kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v, const f
 {
     cudaStream_t stream = (cudaStream_t)stream_;
     int Hk = H;
-    const kda_status so = parse_options(opt, H, Hk);
+    unsigned pro = 0;
+    const kda_status so = parse_options(opt, H, Hk, pro);
     if (so != KDA_OK) return so;
     Plan p;
     const kda_status st = make_plan(B, T, H, dk, dv, cu_seqlens != nullptr, num_seqs, dt, p);
@@ -158,14 +164,14 @@ kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v, const f
 
     cudaError_t e;
     if (p.tc) {
-        e = launch_tc_prefill(q, k, v, log_alpha, beta, S0, S_final, out, hdr, off, cu_seqlens, p.Tseq, p.N, H, Hk,
+        e = launch_tc_prefill(q, k, v, log_alpha, beta, S0, S_final, out, hdr, off, cu_seqlens, p.Tseq, p.N, H, Hk, pro,
                               p.max_chunks, p.Ttot, slots, stream);
     } else if (dt == KDA_BF16) {
         e = launch_simt_prefill<__nv_bfloat16>(q, k, v, log_alpha, beta, S0, S_final, out, hdr, off, cu_seqlens,
-                                               p.Tseq, p.N, H, Hk, dk, dv, p.max_chunks, (float*)slots, stream);
+                                               p.Tseq, p.N, H, Hk, pro, dk, dv, p.max_chunks, (float*)slots, stream);
     } else {
         e = launch_simt_prefill<float>(q, k, v, log_alpha, beta, S0, S_final, out, hdr, off, cu_seqlens, p.Tseq,
-                                       p.N, H, Hk, dk, dv, p.max_chunks, (float*)slots, stream);
+                                       p.N, H, Hk, pro, dk, dv, p.max_chunks, (float*)slots, stream);
     }
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
@@ -187,7 +193,8 @@ kda_status kda_decode_step_ex(const void* q, const void* k, const void* v, const
     if (dt != KDA_BF16 && dt != KDA_F32) return KDA_ERR_INVALID_ARG;
     if (N < 0 || H <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
     int Hk = H;
-    const kda_status so = parse_options(opt, H, Hk);
+    unsigned pro = 0;
+    const kda_status so = parse_options(opt, H, Hk, pro);
     if (so != KDA_OK) return so;
     if (!dims_supported(dk, dv)) return KDA_ERR_UNSUPPORTED;
     if (N == 0) return KDA_OK;
@@ -196,8 +203,8 @@ kda_status kda_decode_step_ex(const void* q, const void* k, const void* v, const
     for (const void* x : ptrs)
         if (!aligned16(x)) return KDA_ERR_INVALID_ARG;
     const cudaError_t e = (dt == KDA_BF16)
-        ? launch_decode<__nv_bfloat16>(q, k, v, log_alpha, beta, S_inout, out, N, H, Hk, dk, dv, stream)
-        : launch_decode<float>(q, k, v, log_alpha, beta, S_inout, out, N, H, Hk, dk, dv, stream);
+        ? launch_decode<__nv_bfloat16>(q, k, v, log_alpha, beta, S_inout, out, N, H, Hk, pro, dk, dv, stream)
+        : launch_decode<float>(q, k, v, log_alpha, beta, S_inout, out, N, H, Hk, pro, dk, dv, stream);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

@@ -43,8 +43,8 @@ template <typename TIn>
 __global__ void __launch_bounds__(kSimtThreads)
 simt_intra_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
                   const float* __restrict__ log_alpha, const float* __restrict__ beta, const WsHeader* __restrict__ hdr,
-                  const int* __restrict__ off, const int32_t* __restrict__ cu, int Tseq, int N, int H, int Hk, int dk,
-                  int dv, float* __restrict__ slots)
+                  const int* __restrict__ off, const int32_t* __restrict__ cu, int Tseq, int N, int H, int Hk,
+                  unsigned pro, int dk, int dv, float* __restrict__ slots)
 {
     extern __shared__ __align__(16) float smem[];
     const int j = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
@@ -73,6 +73,7 @@ simt_intra_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TI
             const size_t gi = ((size_t)(t0 + r) * H + h) * dk + c;
             const size_t qi = ((size_t)(t0 + r) * Hk + h / (H / Hk)) * dk + c;  // q/k head of value head h
             kv = to_f32(k[qi]); qv = to_f32(q[qi]); lv = log_alpha[gi];
+            if (pro & KDA_PROLOGUE_GATE_LOGITS) lv = log_sigmoid_f(lv);  // rows past the end stay 0 (identity)
         }
         sk[e] = kv; sq[e] = qv; sg[e] = lv;
     }
@@ -80,8 +81,31 @@ simt_intra_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TI
         const int r = e / dv, c = e % dv;
         sv[e] = (r < L) ? to_f32(v[((size_t)(t0 + r) * H + h) * dv + c]) : 0.f;
     }
-    for (int r = tid; r < kChunk; r += kSimtThreads) sb[r] = (r < L) ? beta[(size_t)(t0 + r) * H + h] : 0.f;
+    for (int r = tid; r < kChunk; r += kSimtThreads) {
+        float b = 0.f;
+        if (r < L) {
+            b = beta[(size_t)(t0 + r) * H + h];
+            if (pro & KDA_PROLOGUE_BETA_LOGITS) b = sigmoid_f(b);
+        }
+        sb[r] = b;
+    }
     __syncthreads();
+    if (pro & KDA_PROLOGUE_L2NORM_QK) {  // rows of k (i < 64) and q (i >= 64), normalised at the input precision
+        for (int i = tid; i < 2 * kChunk; i += kSimtThreads) {
+            float* row = (i < kChunk ? sk : sq) + (i & (kChunk - 1)) * dk;
+            float ss = 0.f;
+            for (int c0 = 0; c0 < dk; ++c0) {
+                const float x = row[(c0 + i) & (dk - 1)];  // rotated start: no bank conflicts
+                ss = fmaf(x, x, ss);
+            }
+            const float inv = rsqrtf(ss + kQkNormEps);
+            for (int c0 = 0; c0 < dk; ++c0) {
+                const int c = (c0 + i) & (dk - 1);
+                row[c] = to_f32(from_f32<TIn>(row[c] * inv));
+            }
+        }
+        __syncthreads();
+    }
 
     // cumulative gate per channel; reference point = centre of the channel's range
     for (int c = tid; c < dk; c += kSimtThreads) {
@@ -274,8 +298,8 @@ inline size_t simt_inter_smem(int dk, int dv)
 template <typename TIn>
 cudaError_t launch_simt_prefill(const void* q, const void* k, const void* v, const float* la, const float* beta,
                                 const float* S0, float* S_final, void* out, const WsHeader* hdr, const int* off,
-                                const int32_t* cu, int Tseq, int N, int H, int Hk, int dk, int dv, int max_chunks,
-                                float* slots, cudaStream_t stream)
+                                const int32_t* cu, int Tseq, int N, int H, int Hk, unsigned pro, int dk, int dv,
+                                int max_chunks, float* slots, cudaStream_t stream)
 {
     const size_t smA = simt_intra_smem(dk, dv), smB = simt_inter_smem(dk, dv);
     cudaError_t e = cudaFuncSetAttribute(simt_intra_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smA);
@@ -285,7 +309,7 @@ cudaError_t launch_simt_prefill(const void* q, const void* k, const void* v, con
     if (max_chunks > 0) {
         LaunchScope ls("simt_intra", stream);
         simt_intra_kernel<TIn><<<dim3(max_chunks, H), kSimtThreads, smA, stream>>>(
-            (const TIn*)q, (const TIn*)k, (const TIn*)v, la, beta, hdr, off, cu, Tseq, N, H, Hk, dk, dv, slots);
+            (const TIn*)q, (const TIn*)k, (const TIn*)v, la, beta, hdr, off, cu, Tseq, N, H, Hk, pro, dk, dv, slots);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

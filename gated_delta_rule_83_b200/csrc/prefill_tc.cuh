@@ -228,11 +228,13 @@ __device__ __forceinline__ void tc_unit(long long u, int H, const int* __restric
     }
 }
 
+template <bool PRO>  // PRO: some input-prologue bit is set (the plain instance carries none of that code)
 __global__ void __launch_bounds__(kAThreads, 2)
 tc_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_la,
                 const float* __restrict__ beta, WsHeader* __restrict__ hdr, const int* __restrict__ off,
-                const int32_t* __restrict__ cu, int Tseq, int N, int H, int G, uint8_t* __restrict__ slots)
+                const int32_t* __restrict__ cu, int Tseq, int N, int H, int G, unsigned pro,
+                uint8_t* __restrict__ slots)
 {
     using namespace tc;
     extern __shared__ uint8_t smem_raw[];
@@ -348,10 +350,14 @@ tc_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // cumulative gate in log2 units (g2 = log2(e) g): thread (c, hf) scans rows 32 hf .. 32 hf + 31
         float gl[32];
         {
+            // rows past the sequence contribute nothing (identity steps), whatever their input
+            const bool logits = PRO && (pro & KDA_PROLOGUE_GATE_LOGITS) != 0;
             float acc = 0.f;
 #pragma unroll
             for (int u2 = 0; u2 < 32; ++u2) {
-                acc = fmaf(sG[(32 * hf + u2) * kGS + c], kLog2e, acc);
+                const float x = sG[(32 * hf + u2) * kGS + c];
+                const float l2 = logits ? log2_sigmoid(x) : x * kLog2e;
+                acc += (32 * hf + u2 < L) ? l2 : 0.f;
                 gl[u2] = acc;
             }
         }
@@ -404,9 +410,43 @@ tc_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         ok = mbar_wait_ab(mbar_kq, par, s_abort) && ok;  // k and q in place
         cp_async_wait_all();                             // beta in place
+        if (PRO && (pro & KDA_PROLOGUE_BETA_LOGITS) && tid < 64) s_beta[tid] = tid < L ? sigmoid_f(s_beta[tid]) : 0.f;
         __syncthreads();
         has_next = s_next[0] < nunits;
         const bool wide = *s_wide != 0;
+        if (PRO && (pro & KDA_PROLOGUE_L2NORM_QK)) {
+            // k and q rows normalised in place (fp32 norms over the 128 channels held by the 16 threads
+            // of a half-warp, then rounded back to bf16) before anything reads them
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const int r = rb + 16 * jj;
+                uint4* pk = reinterpret_cast<uint4*>(sm + kA_KQ + sw128_chunk_off(r, ch, 128));
+                uint4* pq = reinterpret_cast<uint4*>(sm + kA_KQ + sw128_chunk_off(64 + r, ch, 128));
+                float kv[8], qv[8];
+                unpack8(*pk, kv);
+                unpack8(*pq, qv);
+                float sk = 0.f, sq = 0.f;
+#pragma unroll
+                for (int m = 0; m < 8; ++m) {
+                    sk = fmaf(kv[m], kv[m], sk);
+                    sq = fmaf(qv[m], qv[m], sq);
+                }
+#pragma unroll
+                for (int o = 1; o < 16; o <<= 1) {
+                    sk += __shfl_xor_sync(0xffffffffu, sk, o);
+                    sq += __shfl_xor_sync(0xffffffffu, sq, o);
+                }
+                const float ik = rsqrtf(sk + kQkNormEps), iq = rsqrtf(sq + kQkNormEps);
+#pragma unroll
+                for (int m = 0; m < 8; ++m) {
+                    kv[m] *= ik;
+                    qv[m] *= iq;
+                }
+                *pk = pack8(kv);
+                *pq = pack8(qv);
+            }
+            __syncthreads();
+        }
 
         if (!wide) {
 #pragma unroll
@@ -949,10 +989,13 @@ inline bool make_token_map(CUtensorMap* m, const void* base, bool bf16, int H, l
 
 inline cudaError_t launch_tc_prefill(const void* q, const void* k, const void* v, const float* la, const float* beta,
                                      const float* S0, float* S_final, void* out, const WsHeader* hdr, const int* off,
-                                     const int32_t* cu, int Tseq, int N, int H, int Hk, int max_chunks, long long Ttot,
+                                     const int32_t* cu, int Tseq, int N, int H, int Hk, unsigned pro, int max_chunks,
+                                     long long Ttot,
                                      char* slots, cudaStream_t stream)
 {
-    cudaError_t e = cudaFuncSetAttribute(tc_intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kA_Smem);
+    cudaError_t e = cudaFuncSetAttribute(tc_intra_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kA_Smem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(tc_intra_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kA_Smem);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(tc_inter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kB_Smem);
     if (e != cudaSuccess) return e;
@@ -967,8 +1010,9 @@ inline cudaError_t launch_tc_prefill(const void* q, const void* k, const void* v
         const long long units = (long long)max_chunks * H;
         const unsigned grid = (unsigned)(units < 2LL * sms ? units : 2LL * sms);
         LaunchScope ls("tc_intra", stream);
-        tc_intra_kernel<<<grid, kAThreads, kA_Smem, stream>>>(tq, tk, tv, tla, beta, const_cast<WsHeader*>(hdr), off, cu, Tseq, N, H, H / Hk,
-                                                              (uint8_t*)slots);
+        auto* kern = pro ? tc_intra_kernel<true> : tc_intra_kernel<false>;
+        kern<<<grid, kAThreads, kA_Smem, stream>>>(tq, tk, tv, tla, beta, const_cast<WsHeader*>(hdr), off, cu, Tseq,
+                                                  N, H, H / Hk, pro, (uint8_t*)slots);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

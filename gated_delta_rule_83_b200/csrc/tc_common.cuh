@@ -218,6 +218,19 @@ __device__ __forceinline__ float ex2_approx(float x)
     return y;
 }
 constexpr float kLog2e = 1.4426950408889634f;
+// log2(x) with the hardware's approximate base-2 logarithm (x > 0, normal range)
+__device__ __forceinline__ float lg2_approx(float x)
+{
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+// log2 sigmoid(a) = min(a, 0) log2(e) - log2(1 + 2^{-|a| log2(e)}): the gate logit's log-space
+// forget gate, in the log2 units the tensor-core path accumulates
+__device__ __forceinline__ float log2_sigmoid(float a)
+{
+    return fminf(a, 0.f) * kLog2e - lg2_approx(1.f + ex2_approx(-fabsf(a) * kLog2e));
+}
 
 }  // namespace tc
 }  // namespace kda

@@ -26,7 +26,13 @@ _P, _I, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
 
 class KdaOptions(ctypes.Structure):
     """``kda_options`` of include/kda.h (zero = the plain entry points' behaviour)."""
-    _fields_ = [("num_qk_heads", ctypes.c_int), ("reserved", ctypes.c_int * 7)]
+    _fields_ = [("num_qk_heads", ctypes.c_int), ("prologue", ctypes.c_uint), ("reserved", ctypes.c_int * 6)]
+
+
+# kda_options.prologue bits (KDA_PROLOGUE_* in include/kda.h)
+PROLOGUE_L2NORM_QK = 1     # q and k normalised per (token, q/k head) over d_k inside the kernels
+PROLOGUE_GATE_LOGITS = 2   # log_alpha holds raw gate logits a: log_alpha = log sigmoid(a)
+PROLOGUE_BETA_LOGITS = 4   # beta holds raw logits b: beta = sigmoid(b)
 
 
 ABI = {
@@ -134,13 +140,14 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torc
               S0: Optional[torch.Tensor] = None, cu_seqlens: Optional[torch.Tensor] = None,
               out: Optional[torch.Tensor] = None, S_final: Optional[torch.Tensor] = None,
               output_final_state: bool = True, workspace: Optional[torch.Tensor] = None,
-              stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+              stream: Optional[torch.cuda.Stream] = None, prologue: int = 0) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Chunked KDA prefill (``kda_chunk_fwd``).
 
     q, k: [B, T, Hk, dk]; log_alpha: [B, T, H, dk]; v: [B, T, H, dv]; beta: [B, T, H]; q/k/v bf16 or
     fp32, gates fp32.  Hk = H, or a divisor of H (grouped heads, ``kda_chunk_fwd_ex``: value head h
     reads q/k head h // (H // Hk)).
     S0 / S_final: [N, H, dk, dv] fp32 (N = B, or len(cu_seqlens) - 1 for packed varlen input with B = 1).
+    ``prologue``: PROLOGUE_* bits (raw q/k and gate logits transformed inside the kernels).
     Returns (out [B, T, H, dv] in q's dtype, S_final or None).  S_final may be S0 (in place)."""
     lib = load_library()
     _req(q, "q")
@@ -181,13 +188,13 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torc
         workspace = _get_workspace(ws_bytes, dev, sh)
     else:
         _req(workspace, "workspace", torch.uint8, dev)
-    if Hk == H:
+    if Hk == H and not prologue:
         rc = lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0), _ptr(cu_seqlens),
                                N, _ptr(out), _ptr(S_final), B, T, H, dk, dv, _dt(q), _ptr(workspace),
                                workspace.numel(), sh)
         _check("kda_chunk_fwd", rc)
     else:
-        opt = KdaOptions(num_qk_heads=Hk)
+        opt = KdaOptions(num_qk_heads=Hk, prologue=prologue)
         rc = lib.kda_chunk_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0),
                                   _ptr(cu_seqlens), N, _ptr(out), _ptr(S_final), B, T, H, dk, dv, _dt(q),
                                   ctypes.byref(opt), _ptr(workspace), workspace.numel(), sh)
@@ -220,10 +227,10 @@ def chunk_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alp
 
 def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor, beta: torch.Tensor,
                 S: torch.Tensor, out: Optional[torch.Tensor] = None,
-                stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+                stream: Optional[torch.cuda.Stream] = None, prologue: int = 0) -> torch.Tensor:
     """One KDA decode step (``kda_decode_step``); ``S`` [N, H, dk, dv] fp32 is updated in place.
     q, k: [N, Hk, dk]; log_alpha: [N, H, dk]; v: [N, H, dv]; beta: [N, H], with Hk = H or a divisor of
-    H (grouped heads, ``kda_decode_step_ex``).  Returns out [N, H, dv]."""
+    H (grouped heads, ``kda_decode_step_ex``).  ``prologue``: PROLOGUE_* bits.  Returns out [N, H, dv]."""
     lib = load_library()
     _req(q, "q")
     dev, dtq = q.device, q.dtype
@@ -241,12 +248,12 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: to
         out = torch.empty((N, H, dv), dtype=dtq, device=dev)
     else:
         _req(out, "out", dtq, dev)
-    if Hk == H:
+    if Hk == H and not prologue:
         rc = lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S), _ptr(out), N, H,
                                  dk, dv, _dt(q), _stream_handle(stream, dev))
         _check("kda_decode_step", rc)
     else:
-        opt = KdaOptions(num_qk_heads=Hk)
+        opt = KdaOptions(num_qk_heads=Hk, prologue=prologue)
         rc = lib.kda_decode_step_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S), _ptr(out), N,
                                     H, dk, dv, _dt(q), ctypes.byref(opt), _stream_handle(stream, dev))
         _check("kda_decode_step_ex", rc)

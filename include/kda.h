@@ -134,11 +134,25 @@ kda_status kda_decode_step(const void* q, const void* k, const void* v, const fl
  *                 else KDA_ERR_INVALID_ARG.  The attention review's GDN pseudo-code
  *                 (lanjinlin.com.cn, entry on Qwen3-Next GDN) comments its q/k and value head
  *                 counts separately; this is that layout.
+ *   prologue      Input transforms applied inside the kernels, so the caller can pass the raw
+ *                 projections (a set of KDA_PROLOGUE_* bits; 0 = inputs used as given):
+ *                   KDA_PROLOGUE_L2NORM_QK    q and k are normalised per (token, q/k head) over the
+ *                                             d_k axis in fp32, x / sqrt(sum x^2 + 1e-6), then used
+ *                                             at the input precision (bf16 inputs: rounded to bf16).
+ *                   KDA_PROLOGUE_GATE_LOGITS  the log_alpha argument holds raw gate logits a:
+ *                                             log_alpha = log sigmoid(a) (the log-space forget gate
+ *                                             of the coreui.cn article, section 4.2).
+ *                   KDA_PROLOGUE_BETA_LOGITS  the beta argument holds raw logits b: beta = sigmoid(b).
+ *                 Other bits: KDA_ERR_INVALID_ARG.
  *   reserved      Must be zero (KDA_ERR_INVALID_ARG otherwise).
  */
+#define KDA_PROLOGUE_L2NORM_QK 1u
+#define KDA_PROLOGUE_GATE_LOGITS 2u
+#define KDA_PROLOGUE_BETA_LOGITS 4u
 typedef struct {
     int num_qk_heads;
-    int reserved[7];
+    unsigned prologue;
+    int reserved[6];
 } kda_options;
 
 /*

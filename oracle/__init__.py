@@ -18,6 +18,9 @@ arrays into it.  Every function follows a passage of the pages:
 * ``decode_step`` -- one token per sequence, in the loop order (decay, delta, update, output) of
                      the review's GDN pseudo-code.
 
+``prologue`` is the input transform of the kernels' optional prologue (q/k L2 normalisation,
+log-sigmoid gate logits, sigmoid beta logits), applied in front of the other functions.
+
 ``seq``, ``chunked`` and ``decode_step`` also take q and k with fewer heads than v (grouped heads:
 value head h reads q/k head h // (H // Hk)), as in the head-count comments of the review's GDN
 pseudo-code.
@@ -207,6 +210,27 @@ def decode_step(q, k, v, log_alpha, beta, S):
     if rc != 0:
         raise RuntimeError(f"kda_oracle_decode_step failed with status {rc}")
     return out, S
+
+
+QK_NORM_EPS = 1e-6  # x / sqrt(sum x^2 + eps): the epsilon of the in-kernel q/k normalisation
+
+
+def prologue(q, k, log_alpha, beta, l2norm_qk=False, gate_logits=False, beta_logits=False):
+    """The input prologue in fp64, as a preprocessing step in front of ``seq`` / ``chunked`` /
+    ``decode_step``: q and k normalised over their last (d_k) axis, ``x / sqrt(sum x^2 + eps)``;
+    gate logits a turned into ``log_alpha = log sigmoid(a)`` (the log-space forget gate of the
+    coreui.cn article, section 4.2); beta logits b into ``beta = sigmoid(b)``.  Library routines
+    (numpy, scipy.special.log_expit / expit) carry every step.  Returns float64 arrays."""
+    import scipy.special as sp
+    q, k, la, b = (np.asarray(x, dtype=np.float64) for x in (q, k, log_alpha, beta))
+    if l2norm_qk:
+        q = q / np.sqrt(np.sum(q * q, axis=-1, keepdims=True) + QK_NORM_EPS)
+        k = k / np.sqrt(np.sum(k * k, axis=-1, keepdims=True) + QK_NORM_EPS)
+    if gate_logits:
+        la = sp.log_expit(la)
+    if beta_logits:
+        b = sp.expit(b)
+    return q, k, la, b
 
 
 if __name__ == "__main__":  # pragma: no cover

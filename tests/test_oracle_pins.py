@@ -322,3 +322,36 @@ def test_grouped_heads_equal_repeated_qk(oracle, form):
     assert np.array_equal(o_g, o_r) and np.array_equal(s_g, s_r)
     # and the groups really share: value heads of one group differ only through v, gates and state
     assert rel(o_g[..., 0, :], o_g[..., 1, :]) > 1e-3
+
+
+# ---------------------------------------------------------------------------------------------
+# 14. input prologue: q/k L2 normalisation, log-sigmoid gate logits, sigmoid beta logits
+# ---------------------------------------------------------------------------------------------
+def test_prologue_transforms(oracle):
+    """Pinned by facts of the functions themselves, not by their code.  Catches: a normalisation over
+    the wrong axis or without the square root, log sigmoid with a wrong sign or branch, sigmoid of
+    -b, and transforms applied when their flag is off."""
+    rng = np.random.default_rng(31)
+    q = rng.standard_normal((5, 3, 16)) * 3.0
+    k = rng.standard_normal((5, 3, 16)) * 0.1
+    a = np.array([-60.0, -5.0, -1.0, 0.0, 1.0, 3.0, 40.0])
+    b = np.array([-3.0, 0.0, 2.0])
+    qn, kn, la, bb = oracle.prologue(q, k, a, b, l2norm_qk=True, gate_logits=True, beta_logits=True)
+    # unit rows (up to the 1e-6 epsilon under the square root), same directions
+    nq, nk = np.linalg.norm(qn, axis=-1), np.linalg.norm(kn, axis=-1)
+    assert np.allclose(nq, np.sqrt(np.sum(q * q, -1) / (np.sum(q * q, -1) + 1e-6)), rtol=1e-14)
+    assert np.all(np.abs(nq - 1) < 1e-6) and np.all(np.abs(nk - 1) < 1e-3)
+    assert np.allclose(qn * np.linalg.norm(q, axis=-1, keepdims=True), q * nq[..., None], rtol=1e-12)
+    z, _, _, _ = oracle.prologue(np.zeros((1, 4)), np.zeros((1, 4)), 0.0, 0.0, l2norm_qk=True)
+    assert np.all(z == 0)                                        # a zero row stays zero
+    # log sigmoid: log(1/2) at 0; ~x for x << 0; ~-e^{-x} for x >> 0; log of sigma(x) elsewhere
+    assert la[3] == np.log(0.5)
+    assert abs(la[0] - (-60.0)) < 1e-20 and abs(la[6] + np.exp(-40.0)) < 1e-30
+    mid = a[1:6]
+    assert np.allclose(la[1:6], np.log(1.0 / (1.0 + np.exp(-mid))), rtol=1e-13)
+    assert np.all(la <= 0)
+    # sigmoid: 1/2 at 0, symmetric s(-x) = 1 - s(x)
+    assert bb[1] == 0.5 and abs(bb[0] - (1 - oracle.prologue(q, k, a, -b, beta_logits=True)[3][0])) < 1e-15
+    # flags off: inputs returned unchanged
+    q2, k2, la2, b2 = oracle.prologue(q, k, a, b)
+    assert np.array_equal(q2, q) and np.array_equal(k2, k) and np.array_equal(la2, a) and np.array_equal(b2, b)

@@ -374,6 +374,11 @@ def run_ours(args):
         extra["prefill_32k_prologue"] = bench_prefill_workload(torch, kda, synth, dev, stream, world, rank,
                                                                "prefill_32k", steps=5, warmup=2, prologue=7)
 
+    gnorm = None
+    if not args.no_extra and args.only is None:
+        torch.cuda.empty_cache()
+        gnorm = bench_gated_norm(torch, kda, dev, stream, world, hbm, peak_kind, rows=B * T * H, d=dv)
+
     decode = None
     if not args.no_decode and args.only is None:
         decode = bench_decode(torch, kda, synth, dev, stream, world, rank, hbm, peak_kind, steps=args.decode_steps)
@@ -391,7 +396,7 @@ def run_ours(args):
                        "chunk": 64, "parallelism": f"replicas x{world} (independent problems, no collective)",
                        "l2": f"inputs {in_bytes / 1e9:.2f} GB per step > L2 {L2_BYTES / 1e6:.0f} MB (no flush)"},
             "roofline": roofline, "kernels": {k_: {"launches": n, "ms": t} for k_, (n, t) in prof.items()},
-            "other_workloads": extra,
+            "other_workloads": extra, "gated_rmsnorm": gnorm,
             "gpu_launches": launches, "clocks": clk, "e2e": e2e, "decode": decode, "cpu_baseline": cpu}
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -443,6 +448,39 @@ def bench_prefill_workload(torch, kda, synth, dev, stream, world, rank, name, st
            "value": job_throughput(world, tokens, steps, ms), "unit": "tokens/s",
            "kernels": {k_: {"launches": n, "ms": t} for k_, (n, t) in prof.items()}}
     del inp, q, k, v, la, beta, S0, out, S_fin
+    return res
+
+
+def bench_gated_norm(torch, kda, dev, stream, world, hbm, peak_kind, rows, d, iters=20):
+    """kda_gated_rmsnorm on the prefill output's shape: bf16 o and z, fp32 weight, sigmoid gate,
+    full-width groups.  HBM-bound: o and z read once, y written once."""
+    g = torch.Generator(device=dev).manual_seed(123)
+    o = torch.randn(rows, d, device=dev, generator=g).to(torch.bfloat16)
+    z = torch.randn(rows, d, device=dev, generator=g).to(torch.bfloat16)
+    w = torch.rand(d, device=dev, generator=g) + 0.5
+    y = torch.empty_like(o)
+    for _ in range(3):
+        kda.gated_rmsnorm(o, z, weight=w, gate="sigmoid", out=y)
+    kda.check()
+    barrier(torch, world)
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(iters):
+        kda.gated_rmsnorm(o, z, weight=w, gate="sigmoid", out=y)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    kda.check()
+    us = max_over_ranks(torch, world, e0.elapsed_time(e1)) * 1e3 / iters
+    nbytes = 3 * rows * d * 2 + d * 4
+    ach = nbytes / (us * 1e-6) / 1e9
+    res = {"desc": f"{rows} rows x {d} bf16, sigmoid gate, weight, group = {d}", "us_per_launch": us,
+           "rows_per_s": world * rows / (us * 1e-6),
+           "roofline": {"bound": "hbm", "kernel": "gated_rmsnorm", "achieved": ach, "peak": hbm, "unit": "GB/s",
+                        "frac": ach / hbm, "peak_source": f"{peak_kind} hbm_gbs (of {peak_kind})",
+                        "alg_bytes_per_launch": nbytes}}
+    del o, z, y
     return res
 
 

@@ -7,7 +7,8 @@ Public API (a thin binding of the C ABI in include/kda.h):
     check()                                               # raise on a device-side error
 """
 from .kda import (PROLOGUE_BETA_LOGITS, PROLOGUE_GATE_LOGITS, PROLOGUE_L2NORM_QK, KdaError,  # noqa: F401
-                  check, chunk_fwd, decode_step, load_library, profile_begin, profile_end, version,
-                  workspace_size)
+                  check, chunk_fwd, decode_step, gated_rmsnorm, load_library, profile_begin, profile_end,
+                  version, workspace_size)
 
-__all__ = ["chunk_fwd", "decode_step", "check", "workspace_size", "load_library", "version", "KdaError"]
+__all__ = ["chunk_fwd", "decode_step", "gated_rmsnorm", "check", "workspace_size", "load_library", "version",
+           "KdaError"]

@@ -8,6 +8,7 @@
 #include "common.cuh"
 #include "chunks.cuh"
 #include "decode.cuh"
+#include "gated_norm.cuh"
 #include "prefill_simt.cuh"
 #include "prefill_tc.cuh"
 #include "profile.cuh"
@@ -213,6 +214,26 @@ kda_status kda_decode_step(const void* q, const void* k, const void* v, const fl
                            kda_stream_t stream)
 {
     return kda_decode_step_ex(q, k, v, log_alpha, beta, S_inout, out, N, H, dk, dv, dt, nullptr, stream);
+}
+
+kda_status kda_gated_rmsnorm(const void* o, const void* z, const float* weight, void* y, long long rows, int d,
+                             int group, float eps, kda_gate_act act, kda_dtype dt, kda_stream_t stream_)
+{
+    if (dt != KDA_BF16 && dt != KDA_F32) return KDA_ERR_INVALID_ARG;
+    if (rows < 0 || d <= 0) return KDA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return KDA_ERR_UNSUPPORTED;
+    const int g = group == 0 ? d : group;
+    if (g < 8 || g > d || (g & (g - 1)) != 0 || d % g != 0) return KDA_ERR_INVALID_ARG;
+    if (!(eps > 0.f) || (act != KDA_GATE_IDENTITY && act != KDA_GATE_SIGMOID)) return KDA_ERR_INVALID_ARG;
+    if (rows == 0) return KDA_OK;
+    if (!o || !z || !y || !aligned16(o) || !aligned16(z) || !aligned16(y) || (weight && !aligned16(weight)))
+        return KDA_ERR_INVALID_ARG;
+    cudaStream_t stream = (cudaStream_t)stream_;
+    const int sg = act == KDA_GATE_SIGMOID ? 1 : 0;
+    const cudaError_t e = dt == KDA_BF16
+        ? launch_gated_rmsnorm<__nv_bfloat16>(o, z, weight, y, rows, d, g, eps, sg, stream)
+        : launch_gated_rmsnorm<float>(o, z, weight, y, rows, d, g, eps, sg, stream);
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
 kda_status kda_profile_begin(void)

@@ -44,6 +44,7 @@ ABI = {
     "kda_chunk_fwd_ex": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _I,
                               ctypes.POINTER(KdaOptions), _P, _SZ, _P]),
     "kda_decode_step_ex": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, ctypes.POINTER(KdaOptions), _P]),
+    "kda_gated_rmsnorm": (_I, [_P, _P, _P, _P, ctypes.c_longlong, _I, _I, ctypes.c_float, _I, _I, _P]),
     "kda_chunk_fwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
     "kda_check": (_I, [_P]),
     "kda_selftest_timeout": (_I, [_P]),
@@ -257,6 +258,33 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: to
         rc = lib.kda_decode_step_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S), _ptr(out), N,
                                     H, dk, dv, _dt(q), ctypes.byref(opt), _stream_handle(stream, dev))
         _check("kda_decode_step_ex", rc)
+    return out
+
+
+def gated_rmsnorm(o: torch.Tensor, z: torch.Tensor, weight: Optional[torch.Tensor] = None, group: int = 0,
+                  eps: float = 1e-6, gate: str = "none", out: Optional[torch.Tensor] = None,
+                  stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Output gate ``y = o / sqrt(mean_group(o^2) + eps) * weight * act(z)`` (``kda_gated_rmsnorm``).
+    o, z: [..., d] (bf16 or fp32, same shape), d in {64, 128}; weight [d] fp32 or None; group 0 (= d)
+    or a power of two >= 8 dividing d; gate "none" or "sigmoid".  ``out`` may be ``o`` (in place)."""
+    lib = load_library()
+    _req(o, "o")
+    dev, dt = o.device, o.dtype
+    _req(z, "z", dt, dev)
+    if z.shape != o.shape:
+        raise ValueError("o and z must have the same shape")
+    if weight is not None:
+        _req(weight, "weight", torch.float32, dev)
+    if out is None:
+        out = torch.empty_like(o)
+    else:
+        _req(out, "out", dt, dev)
+    d = o.shape[-1]
+    rows = o.numel() // d if d else 0
+    act = {"none": 0, "sigmoid": 1}[gate]
+    rc = lib.kda_gated_rmsnorm(_ptr(o), _ptr(z), _ptr(weight), _ptr(out), rows, d, group, eps, act, _dt(o),
+                               _stream_handle(stream, dev))
+    _check("kda_gated_rmsnorm", rc)
     return out
 
 

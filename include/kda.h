@@ -175,6 +175,34 @@ kda_status kda_decode_step_ex(const void* q, const void* k, const void* v, const
                               kda_dtype dt, const kda_options* opt, kda_stream_t stream);
 
 /*
+ * kda_gated_rmsnorm -- the output gate of a KDA layer, one fused streaming pass:
+ *
+ *     y = o / sqrt(mean_g(o^2) + eps) * weight * act(z)
+ *
+ * The attention review's GDN/KDA pseudo-code (lanjinlin.com.cn, entry on Qwen3-Next GDN, step
+ * "门控归一化") normalises the attention output with an RMS norm and multiplies it by the output gate
+ * z; the review's Ring-linear notes take that norm over groups of channels, each group on its own
+ * (grouped RMS norm), and fuse the norm, the gate's sigmoid and the product into one kernel.
+ *
+ *   o, z, y   [rows, d] element type dt, contiguous (e.g. the [B, T, H, dv] output of
+ *             kda_chunk_fwd with rows = B*T*H, d = dv, and the gate in the same layout);
+ *             y may alias o (in place).
+ *   weight    [d] fp32 per-channel scale, or NULL (= ones).
+ *   group     channels per norm group: 0 (= d) or a power of two in [8, d] dividing d.
+ *   eps       > 0, added to the mean square.
+ *   act       KDA_GATE_IDENTITY (z used as given) or KDA_GATE_SIGMOID (sigmoid(z)).
+ * Supported: d in {64, 128}.  rows >= 0 (0 is a no-op).  Pointers 16-byte aligned.
+ * Errors: KDA_ERR_INVALID_ARG for null/misaligned pointers, a bad group, eps <= 0 or an unknown
+ * act; KDA_ERR_UNSUPPORTED for other d.
+ */
+typedef enum {
+    KDA_GATE_IDENTITY = 0,
+    KDA_GATE_SIGMOID = 1
+} kda_gate_act;
+kda_status kda_gated_rmsnorm(const void* o, const void* z, const float* weight, void* y, long long rows, int d,
+                             int group, float eps, kda_gate_act act, kda_dtype dt, kda_stream_t stream);
+
+/*
  * kda_check -- synchronise `stream`, then read and clear the device error word of the current
  * device.  Returns KDA_OK, KDA_ERR_CUDA (a sticky CUDA error), KDA_ERR_BAD_SEQLENS or
  * KDA_ERR_TIMEOUT.

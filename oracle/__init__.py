@@ -18,6 +18,8 @@ arrays into it.  Every function follows a passage of the pages:
 * ``decode_step`` -- one token per sequence, in the loop order (decay, delta, update, output) of
                      the review's GDN pseudo-code.
 
+``gated_rmsnorm`` is the output gate (grouped RMS norm times the gate z).
+
 ``prologue`` is the input transform of the kernels' optional prologue (q/k L2 normalisation,
 log-sigmoid gate logits, sigmoid beta logits), applied in front of the other functions.
 
@@ -231,6 +233,28 @@ def prologue(q, k, log_alpha, beta, l2norm_qk=False, gate_logits=False, beta_log
     if beta_logits:
         b = sp.expit(b)
     return q, k, la, b
+
+
+def gated_rmsnorm(o, z, weight=None, group=None, eps=1e-6, gate="none"):
+    """The output gate of the review's GDN pseudo-code (section "门控归一化": the normalised attention
+    output times the output gate z), with the grouped RMS norm of the Ring-linear notes (the norm
+    taken over groups of ``group`` channels of the last axis, each group on its own):
+
+        y = o / sqrt(mean_group(o^2) + eps) * weight * act(z),   act = identity or sigmoid.
+
+    fp64 numpy; ``weight`` [d] or None (ones); ``group`` None = the whole last axis."""
+    import scipy.special as sp
+    o = np.asarray(o, dtype=np.float64)
+    d = o.shape[-1]
+    g = d if group is None else int(group)
+    if d % g:
+        raise ValueError("group must divide the last axis")
+    og = o.reshape(o.shape[:-1] + (d // g, g))
+    y = (og / np.sqrt(np.mean(og * og, axis=-1, keepdims=True) + eps)).reshape(o.shape)
+    if weight is not None:
+        y = y * np.asarray(weight, dtype=np.float64)
+    zz = np.asarray(z, dtype=np.float64)
+    return y * (sp.expit(zz) if gate == "sigmoid" else zz)
 
 
 if __name__ == "__main__":  # pragma: no cover

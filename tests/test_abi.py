@@ -121,6 +121,18 @@ def test_options_are_validated_before_launch(lib):
                                   ctypes.byref(ok_group), None) == 0  # N = 0: no-op
 
 
+def test_gated_rmsnorm_rejects_before_launch(lib):
+    fake = 0x100000
+    c = ctypes.c_float
+    assert lib.kda_gated_rmsnorm(fake, fake, None, fake, 10, 96, 0, c(1e-6), 0, 0, None) == 2      # d
+    assert lib.kda_gated_rmsnorm(fake, fake, None, fake, 10, 128, 24, c(1e-6), 0, 0, None) == 1    # group
+    assert lib.kda_gated_rmsnorm(fake, fake, None, fake, 10, 64, 128, c(1e-6), 0, 0, None) == 1    # group > d
+    assert lib.kda_gated_rmsnorm(fake, fake, None, fake, 10, 128, 0, c(0.0), 0, 0, None) == 1      # eps
+    assert lib.kda_gated_rmsnorm(fake, fake, None, fake, 10, 128, 0, c(1e-6), 5, 0, None) == 1     # act
+    assert lib.kda_gated_rmsnorm(fake + 8, fake, None, fake, 10, 128, 0, c(1e-6), 0, 0, None) == 1  # aligned
+    assert lib.kda_gated_rmsnorm(None, None, None, None, 0, 128, 0, c(1e-6), 0, 0, None) == 0      # rows = 0
+
+
 def test_missing_library_fails_loudly(tmp_path):
     from gated_delta_rule_83_b200 import kda
     with pytest.raises(ImportError):

@@ -355,3 +355,31 @@ def test_prologue_transforms(oracle):
     # flags off: inputs returned unchanged
     q2, k2, la2, b2 = oracle.prologue(q, k, a, b)
     assert np.array_equal(q2, q) and np.array_equal(k2, k) and np.array_equal(la2, a) and np.array_equal(b2, b)
+
+
+# ---------------------------------------------------------------------------------------------
+# 15. output gate: grouped RMS norm times the gate z
+# ---------------------------------------------------------------------------------------------
+def test_gated_rmsnorm(oracle):
+    """Pinned by torch's own rms_norm (float64, a library routine) and by facts of the norm.  Catches:
+    the norm over the wrong axis or group, a missing square root or mean, the gate not applied or
+    applied before the norm, the weight dropped."""
+    import torch
+    rng = np.random.default_rng(41)
+    o = rng.standard_normal((3, 5, 64)) * 4.0
+    z = rng.standard_normal((3, 5, 64))
+    w = rng.uniform(0.5, 1.5, 64)
+    y = oracle.gated_rmsnorm(o, z, weight=w, eps=1e-6)
+    ref = torch.nn.functional.rms_norm(torch.from_numpy(o), (64,), torch.from_numpy(w), eps=1e-6).numpy() * z
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-14)
+    # grouped: each group of 16 normalised on its own = rms_norm over a reshaped last axis
+    yg = oracle.gated_rmsnorm(o, np.ones_like(o), group=16, eps=1e-6)
+    refg = torch.nn.functional.rms_norm(torch.from_numpy(o.reshape(3, 5, 4, 16)), (16,), eps=1e-6).numpy()
+    assert np.allclose(yg, refg.reshape(o.shape), rtol=1e-12)
+    # unit RMS per group (up to eps), invariant to a positive scale of o
+    ms = np.mean(yg.reshape(3, 5, 4, 16) ** 2, axis=-1)
+    assert np.all(np.abs(ms - 1) < 1e-6)
+    assert np.allclose(oracle.gated_rmsnorm(7.5 * o, z), oracle.gated_rmsnorm(o, z), rtol=1e-6)
+    # sigmoid gate: z = 0 halves the normalised output
+    y0 = oracle.gated_rmsnorm(o, np.zeros_like(o), gate="sigmoid")
+    assert np.allclose(y0, 0.5 * oracle.gated_rmsnorm(o, np.ones_like(o)), rtol=1e-14)

@@ -373,6 +373,10 @@ def run_ours(args):
         # input prologue (kda_options.prologue = all bits): raw q/k and gate/beta logits, transformed in-kernel
         extra["prefill_32k_prologue"] = bench_prefill_workload(torch, kda, synth, dev, stream, world, rank,
                                                                "prefill_32k", steps=5, warmup=2, prologue=7)
+        torch.cuda.empty_cache()
+        # bf16 gates (KDA_PROLOGUE_GATE_BF16): the largest input halved, 1284 instead of 1540 B per token-head
+        extra["prefill_32k_gate_bf16"] = bench_prefill_workload(torch, kda, synth, dev, stream, world, rank,
+                                                                "prefill_32k", steps=5, warmup=2, gate_bf16=True)
 
     gnorm = None
     if not args.no_extra and args.only is None:
@@ -406,17 +410,21 @@ def run_ours(args):
 
 
 def bench_prefill_workload(torch, kda, synth, dev, stream, world, rank, name, steps, warmup, qk_heads=None,
-                           prologue=0):
+                           prologue=0, gate_bf16=False):
     """Device-timed throughput of another prefill workload (same method as the headline).  With
     ``qk_heads``, q and k keep only that many heads, shared by groups of value heads.  With
     ``prologue`` the call passes that kda_options.prologue value (the workload's inputs stand in
-    for raw projections: the in-kernel transforms cost the same whatever the values)."""
+    for raw projections: the in-kernel transforms cost the same whatever the values).  With
+    ``gate_bf16`` log_alpha is passed as bf16 (half its bytes)."""
     w = synth.WORKLOADS[name]
     inp = synth.prefill_inputs(w, device=dev, seed=replica_seed(w.seed, rank))
     q, k, v, la, beta, S0, cu = (inp[x] for x in ("q", "k", "v", "log_alpha", "beta", "S0", "cu_seqlens"))
     if qk_heads is not None:
         q, k = q[:, :, :qk_heads].contiguous(), k[:, :, :qk_heads].contiguous()
         inp["q"], inp["k"] = q, k
+    if gate_bf16:
+        la = la.to(torch.bfloat16)
+        inp["log_alpha"] = la
     out = torch.empty_like(v)
     N = q.shape[0] if cu is None else cu.numel() - 1
     S_fin = torch.empty((N, w.H, w.dk, w.dv), dtype=torch.float32, device=dev)
@@ -444,6 +452,8 @@ def bench_prefill_workload(torch, kda, synth, dev, stream, world, rank, name, st
     desc = w.desc if qk_heads is None else f"{w.desc}; q/k with {qk_heads} heads shared by groups of value heads"
     if prologue:
         desc += f"; input prologue {prologue} (q/k L2 norm, log-sigmoid gate logits, sigmoid beta logits in-kernel)"
+    if gate_bf16:
+        desc += "; log_alpha in bf16"
     res = {"desc": desc, "tokens": tokens, "steps": steps, "ms_per_step": ms / steps,
            "value": job_throughput(world, tokens, steps, ms), "unit": "tokens/s",
            "kernels": {k_: {"launches": n, "ms": t} for k_, (n, t) in prof.items()}}

@@ -6,7 +6,8 @@ Public API (a thin binding of the C ABI in include/kda.h):
     out = decode_step(q, k, v, log_alpha, beta, S)        # S updated in place
     check()                                               # raise on a device-side error
 """
-from .kda import (PROLOGUE_BETA_LOGITS, PROLOGUE_GATE_LOGITS, PROLOGUE_L2NORM_QK, KdaError,  # noqa: F401
+from .kda import (PROLOGUE_BETA_LOGITS, PROLOGUE_GATE_BF16, PROLOGUE_GATE_LOGITS, PROLOGUE_L2NORM_QK,  # noqa: F401
+                  KdaError,
                   check, chunk_fwd, decode_step, gated_rmsnorm, load_library, profile_begin, profile_end,
                   version, workspace_size)
 

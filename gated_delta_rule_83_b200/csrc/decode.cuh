@@ -25,7 +25,7 @@ constexpr int kDecodeSlice = 64;  // columns of S per CTA
 template <typename TIn, int DK, bool GROUPED, bool PRO>
 __global__ void __launch_bounds__(kDecodeThreads, 3)
 decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
-                   const float* __restrict__ log_alpha, const float* __restrict__ beta, float* __restrict__ S,
+                   const void* __restrict__ log_alpha, const float* __restrict__ beta, float* __restrict__ S,
                    TIn* __restrict__ out, int dv, int H, int G, unsigned pro)
 {
     constexpr int RPT = DK / 16;  // state rows held per thread
@@ -52,7 +52,10 @@ decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const T
     const TIn* vp = v + (size_t)p * dv + j0 + 4 * cg;
     const float v0 = to_f32(vp[0]), v1 = to_f32(vp[1]), v2 = to_f32(vp[2]), v3 = to_f32(vp[3]);
     for (int c = tid; c < DK; c += kDecodeThreads) {
-        const float la = log_alpha[(size_t)p * DK + c];
+        const size_t ia = (size_t)p * DK + c;  // gates fp32, or bf16 with the bf16-gate bit
+        const float la = (PRO && (pro & KDA_PROLOGUE_GATE_BF16))
+                             ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(log_alpha)[ia])
+                             : reinterpret_cast<const float*>(log_alpha)[ia];
         s_a[c] = (PRO && (pro & KDA_PROLOGUE_GATE_LOGITS)) ? sigmoid_f(la) : expf(la);  // alpha = sigmoid(logit)
         s_k[c] = to_f32(k[(size_t)pq * DK + c]);
         s_q[c] = to_f32(q[(size_t)pq * DK + c]);
@@ -147,7 +150,7 @@ decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const T
 }
 
 template <typename TIn>
-cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* la, const float* beta, float* S,
+cudaError_t launch_decode(const void* q, const void* k, const void* v, const void* la, const float* beta, float* S,
                           void* out, int N, int H, int Hk, unsigned pro, int dk, int dv, cudaStream_t stream)
 {
     const long long pairs = (long long)N * H;

@@ -94,7 +94,8 @@ kda_status parse_options(const kda_options* opt, int H, int& Hk, unsigned& pro)
         if (opt->num_qk_heads < 0 || H % opt->num_qk_heads != 0) return KDA_ERR_INVALID_ARG;
         Hk = opt->num_qk_heads;
     }
-    const unsigned known = KDA_PROLOGUE_L2NORM_QK | KDA_PROLOGUE_GATE_LOGITS | KDA_PROLOGUE_BETA_LOGITS;
+    const unsigned known =
+        KDA_PROLOGUE_L2NORM_QK | KDA_PROLOGUE_GATE_LOGITS | KDA_PROLOGUE_BETA_LOGITS | KDA_PROLOGUE_GATE_BF16;
     if (opt->prologue & ~known) return KDA_ERR_INVALID_ARG;
     pro = opt->prologue;
     return KDA_OK;
@@ -131,7 +132,7 @@ kda_status kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int
     return KDA_OK;
 }
 
-kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v, const float* log_alpha, const float* beta,
+kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v, const void* log_alpha, const float* beta,
                             const float* S0, const int32_t* cu_seqlens, int num_seqs, void* out, float* S_final,
                             int B, int T, int H, int dk, int dv, kda_dtype dt, const kda_options* opt,
                             void* workspace, size_t workspace_bytes, kda_stream_t stream_)
@@ -186,7 +187,7 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const floa
                             nullptr, workspace, workspace_bytes, stream);
 }
 
-kda_status kda_decode_step_ex(const void* q, const void* k, const void* v, const float* log_alpha,
+kda_status kda_decode_step_ex(const void* q, const void* k, const void* v, const void* log_alpha,
                               const float* beta, float* S_inout, void* out, int N, int H, int dk, int dv,
                               kda_dtype dt, const kda_options* opt, kda_stream_t stream_)
 {

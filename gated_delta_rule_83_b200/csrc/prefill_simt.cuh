@@ -42,7 +42,7 @@ constexpr float kFactorSpread = 160.f;
 template <typename TIn>
 __global__ void __launch_bounds__(kSimtThreads)
 simt_intra_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
-                  const float* __restrict__ log_alpha, const float* __restrict__ beta, const WsHeader* __restrict__ hdr,
+                  const void* __restrict__ log_alpha, const float* __restrict__ beta, const WsHeader* __restrict__ hdr,
                   const int* __restrict__ off, const int32_t* __restrict__ cu, int Tseq, int N, int H, int Hk,
                   unsigned pro, int dk, int dv, float* __restrict__ slots)
 {
@@ -72,7 +72,9 @@ simt_intra_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TI
         if (r < L) {
             const size_t gi = ((size_t)(t0 + r) * H + h) * dk + c;
             const size_t qi = ((size_t)(t0 + r) * Hk + h / (H / Hk)) * dk + c;  // q/k head of value head h
-            kv = to_f32(k[qi]); qv = to_f32(q[qi]); lv = log_alpha[gi];
+            kv = to_f32(k[qi]); qv = to_f32(q[qi]);
+            lv = (pro & KDA_PROLOGUE_GATE_BF16) ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(log_alpha)[gi])
+                                                : reinterpret_cast<const float*>(log_alpha)[gi];
             if (pro & KDA_PROLOGUE_GATE_LOGITS) lv = log_sigmoid_f(lv);  // rows past the end stay 0 (identity)
         }
         sk[e] = kv; sq[e] = qv; sg[e] = lv;
@@ -296,7 +298,7 @@ inline size_t simt_inter_smem(int dk, int dv)
 }
 
 template <typename TIn>
-cudaError_t launch_simt_prefill(const void* q, const void* k, const void* v, const float* la, const float* beta,
+cudaError_t launch_simt_prefill(const void* q, const void* k, const void* v, const void* la, const float* beta,
                                 const float* S0, float* S_final, void* out, const WsHeader* hdr, const int* off,
                                 const int32_t* cu, int Tseq, int N, int H, int Hk, unsigned pro, int dk, int dv,
                                 int max_chunks, float* slots, cudaStream_t stream)

@@ -194,7 +194,8 @@ constexpr uint32_t kA_KQ = 0;        // 32 KB: [k; q] -> [Kf; Qf] stacked (128 r
                                      //   -> W in the k rows, Q' in the q rows
 constexpr uint32_t kA_V = 32768;     // 16 KB: v
 constexpr uint32_t kA_B = 49152;     // 16 KB: Kb -> T -> Uv -> O0
-constexpr uint32_t kA_G = 65536;     // 32 KB: log_alpha -> g fp32 [64][128] -> A / X fp32 [64][68] + scratch + P tile
+constexpr uint32_t kA_G = 65536;     // 32 KB: log_alpha (fp32, or bf16 in the upper 16 KB) -> g fp32 [64][128]
+                                     //   -> A / X fp32 [64][68] + scratch + P tile
 constexpr uint32_t kA_Ysc = kA_G + 17408;   // solve scratch 32 x 36 fp32
 constexpr uint32_t kA_P = kA_G + 22528;     // P bf16 [64][64] tile (1024-aligned)
 constexpr uint32_t kA_Misc = kA_G + 32768;  // small arrays, TMEM address, flags, mbarriers (4 KB)
@@ -228,7 +229,10 @@ __device__ __forceinline__ void tc_unit(long long u, int H, const int* __restric
     }
 }
 
-template <bool PRO>  // PRO: some input-prologue bit is set (the plain instance carries none of that code)
+// PRO: some q/k or beta/gate-activation prologue bit is set (the plain instance carries none of that code)
+// LA16: log_alpha arrives as bf16 (16 KB per unit, landed in the upper half of the gate region and
+// widened to the fp32 g tile by the gate scan)
+template <bool PRO, bool LA16>
 __global__ void __launch_bounds__(kAThreads, 2)
 tc_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_la,
@@ -272,8 +276,8 @@ tc_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     // TMA boxes of 64 tokens of one head; tokens past the tensor's end arrive as zeros
     auto issue_la = [&](int hh, long long tt) {
-        mbar_arrive_expect_tx(mbar_la, 32768);
-        tma_load_3d(sb + kA_G, &tm_la, 0, hh, (int)tt, mbar_la);
+        mbar_arrive_expect_tx(mbar_la, LA16 ? 16384 : 32768);
+        tma_load_3d(sb + kA_G + (LA16 ? 16384 : 0), &tm_la, 0, hh, (int)tt, mbar_la);
     };
     auto issue_kq = [&](int hh, long long tt) {  // stacked tile: atom column a = k rows then q rows
         const int hq = hh / G;                         // the q/k head of value head hh (grouped heads)
@@ -342,8 +346,9 @@ tc_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 *reinterpret_cast<uint4*>(sm + kA_KQ + sw128_chunk_off(64 + r, chh, 128)) = make_uint4(0, 0, 0, 0);
                 *reinterpret_cast<uint4*>(sm + kA_V + sw128_chunk_off(r, chh, 64)) = make_uint4(0, 0, 0, 0);
             }
-            for (int e = tid; e < (64 - L) * 32; e += kAThreads)
-                *reinterpret_cast<float4*>(sG + (L + (e >> 5)) * kGS + 4 * (e & 31)) = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (!LA16)
+                for (int e = tid; e < (64 - L) * 32; e += kAThreads)
+                    *reinterpret_cast<float4*>(sG + (L + (e >> 5)) * kGS + 4 * (e & 31)) = make_float4(0.f, 0.f, 0.f, 0.f);
             __syncthreads();
         }
 
@@ -352,10 +357,11 @@ tc_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         {
             // rows past the sequence contribute nothing (identity steps), whatever their input
             const bool logits = PRO && (pro & KDA_PROLOGUE_GATE_LOGITS) != 0;
+            const __nv_bfloat16* sG16 = reinterpret_cast<const __nv_bfloat16*>(sm + kA_G + 16384);
             float acc = 0.f;
 #pragma unroll
             for (int u2 = 0; u2 < 32; ++u2) {
-                const float x = sG[(32 * hf + u2) * kGS + c];
+                const float x = LA16 ? __bfloat162float(sG16[(32 * hf + u2) * 128 + c]) : sG[(32 * hf + u2) * kGS + c];
                 const float l2 = logits ? log2_sigmoid(x) : x * kLog2e;
                 acc += (32 * hf + u2 < L) ? l2 : 0.f;
                 gl[u2] = acc;
@@ -385,6 +391,7 @@ tc_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
         }
 #pragma unroll
+        // (LA16: the bf16 source under rows 32..63 has been read by every thread before the barrier above)
         for (int u2 = 0; u2 < 32; ++u2) sG[(32 * hf + u2) * kGS + c] = gl[u2];
         __syncthreads();
         if (hf == 0) {
@@ -971,38 +978,42 @@ inline TensorMapEncodeFn tensor_map_encoder()
     return fn;
 }
 
-// [tokens][H][128] row-major tensor as a 3-D map (d, head, token), box = 64 tokens x 1 head x box_d
+// [tokens][H][128] row-major tensor as a 3-D map (d, head, token), box = 64 tokens x 1 head x box_d;
+// bf16 tiles of 64 channels land 128B-swizzled (MMA operands), every other box unswizzled
 inline bool make_token_map(CUtensorMap* m, const void* base, bool bf16, int H, long long ntok, int box_d)
 {
     TensorMapEncodeFn enc = tensor_map_encoder();
     if (!enc) return false;
     const cuuint64_t esz = bf16 ? 2 : 4;
+    const bool swz = bf16 && box_d * esz == 128;
     const cuuint64_t dims[3] = {128, (cuuint64_t)H, (cuuint64_t)ntok};
     const cuuint64_t strides[2] = {128 * esz, 128 * esz * (cuuint64_t)H};
     const cuuint32_t box[3] = {(cuuint32_t)box_d, 1, 64};
     const cuuint32_t estr[3] = {1, 1, 1};
     return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base),
                dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-               bf16 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               swz ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-inline cudaError_t launch_tc_prefill(const void* q, const void* k, const void* v, const float* la, const float* beta,
+inline cudaError_t launch_tc_prefill(const void* q, const void* k, const void* v, const void* la, const float* beta,
                                      const float* S0, float* S_final, void* out, const WsHeader* hdr, const int* off,
                                      const int32_t* cu, int Tseq, int N, int H, int Hk, unsigned pro, int max_chunks,
                                      long long Ttot,
                                      char* slots, cudaStream_t stream)
 {
-    cudaError_t e = cudaFuncSetAttribute(tc_intra_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kA_Smem);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(tc_intra_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kA_Smem);
+    // instance: (any q/k, beta or gate-activation bit, bf16 gates)
+    const bool la16 = (pro & KDA_PROLOGUE_GATE_BF16) != 0, pr = (pro & ~KDA_PROLOGUE_GATE_BF16) != 0;
+    auto* kern = pr ? (la16 ? tc_intra_kernel<true, true> : tc_intra_kernel<true, false>)
+                    : (la16 ? tc_intra_kernel<false, true> : tc_intra_kernel<false, false>);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kA_Smem);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(tc_inter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kB_Smem);
     if (e != cudaSuccess) return e;
     if (max_chunks > 0 && Ttot > 0) {
         alignas(64) CUtensorMap tq, tk, tv, tla;
         if (!make_token_map(&tq, q, true, Hk, Ttot, 64) || !make_token_map(&tk, k, true, Hk, Ttot, 64) ||
-            !make_token_map(&tv, v, true, H, Ttot, 64) || !make_token_map(&tla, la, false, H, Ttot, 128))
+            !make_token_map(&tv, v, true, H, Ttot, 64) || !make_token_map(&tla, la, la16, H, Ttot, 128))
             return cudaErrorInvalidValue;
         // persistent: two CTAs per SM (the register and shared-memory budget of one CTA is half an SM)
         int dev = 0, sms = 148;
@@ -1010,7 +1021,6 @@ inline cudaError_t launch_tc_prefill(const void* q, const void* k, const void* v
         const long long units = (long long)max_chunks * H;
         const unsigned grid = (unsigned)(units < 2LL * sms ? units : 2LL * sms);
         LaunchScope ls("tc_intra", stream);
-        auto* kern = pro ? tc_intra_kernel<true> : tc_intra_kernel<false>;
         kern<<<grid, kAThreads, kA_Smem, stream>>>(tq, tk, tv, tla, beta, const_cast<WsHeader*>(hdr), off, cu, Tseq,
                                                   N, H, H / Hk, pro, (uint8_t*)slots);
         e = cudaGetLastError();

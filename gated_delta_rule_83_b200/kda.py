@@ -33,6 +33,7 @@ class KdaOptions(ctypes.Structure):
 PROLOGUE_L2NORM_QK = 1     # q and k normalised per (token, q/k head) over d_k inside the kernels
 PROLOGUE_GATE_LOGITS = 2   # log_alpha holds raw gate logits a: log_alpha = log sigmoid(a)
 PROLOGUE_BETA_LOGITS = 4   # beta holds raw logits b: beta = sigmoid(b)
+PROLOGUE_GATE_BF16 = 8     # log_alpha (or its logits) is bf16; set by the binding from log_alpha's dtype
 
 
 ABI = {
@@ -93,6 +94,17 @@ def _dt(t: torch.Tensor) -> int:
     raise TypeError(f"q/k/v must be bfloat16 or float32, got {t.dtype}")
 
 
+def _gate_bits(log_alpha: torch.Tensor, prologue: int) -> int:
+    """log_alpha may be fp32 or bf16; bf16 selects PROLOGUE_GATE_BF16 (exact widening in the kernels)."""
+    if log_alpha.dtype == torch.bfloat16:
+        return prologue | PROLOGUE_GATE_BF16
+    if log_alpha.dtype != torch.float32:
+        raise TypeError(f"log_alpha must be float32 or bfloat16, got {log_alpha.dtype}")
+    if prologue & PROLOGUE_GATE_BF16:
+        raise TypeError("PROLOGUE_GATE_BF16 set for a float32 log_alpha")
+    return prologue
+
+
 def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else t.data_ptr()
 
@@ -145,8 +157,8 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torc
     """Chunked KDA prefill (``kda_chunk_fwd``).
 
     q, k: [B, T, Hk, dk]; log_alpha: [B, T, H, dk]; v: [B, T, H, dv]; beta: [B, T, H]; q/k/v bf16 or
-    fp32, gates fp32.  Hk = H, or a divisor of H (grouped heads, ``kda_chunk_fwd_ex``: value head h
-    reads q/k head h // (H // Hk)).
+    fp32, beta fp32, log_alpha fp32 or bf16 (``kda_chunk_fwd_ex`` with PROLOGUE_GATE_BF16).  Hk = H, or
+    a divisor of H (grouped heads, ``kda_chunk_fwd_ex``: value head h reads q/k head h // (H // Hk)).
     S0 / S_final: [N, H, dk, dv] fp32 (N = B, or len(cu_seqlens) - 1 for packed varlen input with B = 1).
     ``prologue``: PROLOGUE_* bits (raw q/k and gate logits transformed inside the kernels).
     Returns (out [B, T, H, dv] in q's dtype, S_final or None).  S_final may be S0 (in place)."""
@@ -160,7 +172,8 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torc
     H, dv = v.shape[2], v.shape[-1]
     _req(k, "k", dtq, dev)
     _req(v, "v", dtq, dev)
-    _req(log_alpha, "log_alpha", torch.float32, dev)
+    _req(log_alpha, "log_alpha", None, dev)
+    prologue = _gate_bits(log_alpha, prologue)
     _req(beta, "beta", torch.float32, dev)
     if k.shape != q.shape or tuple(log_alpha.shape) != (B, T, H, dk) or tuple(v.shape) != (B, T, H, dv) or \
             tuple(beta.shape) != (B, T, H) or H % Hk != 0:
@@ -231,7 +244,8 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: to
                 stream: Optional[torch.cuda.Stream] = None, prologue: int = 0) -> torch.Tensor:
     """One KDA decode step (``kda_decode_step``); ``S`` [N, H, dk, dv] fp32 is updated in place.
     q, k: [N, Hk, dk]; log_alpha: [N, H, dk]; v: [N, H, dv]; beta: [N, H], with Hk = H or a divisor of
-    H (grouped heads, ``kda_decode_step_ex``).  ``prologue``: PROLOGUE_* bits.  Returns out [N, H, dv]."""
+    H (grouped heads, ``kda_decode_step_ex``); log_alpha fp32 or bf16.  ``prologue``: PROLOGUE_* bits.
+    Returns out [N, H, dv]."""
     lib = load_library()
     _req(q, "q")
     dev, dtq = q.device, q.dtype
@@ -239,7 +253,8 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: to
     H, dv = v.shape[1], v.shape[-1]
     _req(k, "k", dtq, dev)
     _req(v, "v", dtq, dev)
-    _req(log_alpha, "log_alpha", torch.float32, dev)
+    _req(log_alpha, "log_alpha", None, dev)
+    prologue = _gate_bits(log_alpha, prologue)
     _req(beta, "beta", torch.float32, dev)
     _req(S, "S", torch.float32, dev)
     if k.shape != q.shape or tuple(log_alpha.shape) != (N, H, dk) or tuple(v.shape) != (N, H, dv) or \

@@ -143,12 +143,19 @@ kda_status kda_decode_step(const void* q, const void* k, const void* v, const fl
  *                                             log_alpha = log sigmoid(a) (the log-space forget gate
  *                                             of the coreui.cn article, section 4.2).
  *                   KDA_PROLOGUE_BETA_LOGITS  the beta argument holds raw logits b: beta = sigmoid(b).
+ *                   KDA_PROLOGUE_GATE_BF16    the log_alpha argument (log alpha, or gate logits with
+ *                                             KDA_PROLOGUE_GATE_LOGITS) points at bf16 values in the
+ *                                             same [.., H, dk] layout instead of fp32.  Each value is
+ *                                             widened to fp32 exactly on load, so the result is
+ *                                             bit-identical to the fp32 call on the same values; the
+ *                                             largest input of the prefill is halved.  Any dt.
  *                 Other bits: KDA_ERR_INVALID_ARG.
  *   reserved      Must be zero (KDA_ERR_INVALID_ARG otherwise).
  */
 #define KDA_PROLOGUE_L2NORM_QK 1u
 #define KDA_PROLOGUE_GATE_LOGITS 2u
 #define KDA_PROLOGUE_BETA_LOGITS 4u
+#define KDA_PROLOGUE_GATE_BF16 8u
 typedef struct {
     int num_qk_heads;
     unsigned prologue;
@@ -159,8 +166,9 @@ typedef struct {
  * kda_chunk_fwd_ex -- kda_chunk_fwd with options (`opt` may be NULL: the plain behaviour).
  * Same arguments, layout, workspace (kda_chunk_fwd_workspace_size with the value-head count H),
  * errors and asynchrony as kda_chunk_fwd; with opt->num_qk_heads = Hk, q and k are [B, T, Hk, dk].
+ * log_alpha is fp32, or bf16 with KDA_PROLOGUE_GATE_BF16.
  */
-kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v, const float* log_alpha, const float* beta,
+kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v, const void* log_alpha, const float* beta,
                             const float* S0, const int32_t* cu_seqlens, int num_seqs, void* out, float* S_final,
                             int B, int T, int H, int dk, int dv, kda_dtype dt, const kda_options* opt,
                             void* workspace, size_t workspace_bytes, kda_stream_t stream);
@@ -168,9 +176,9 @@ kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v, const f
 /*
  * kda_decode_step_ex -- kda_decode_step with options (`opt` may be NULL: the plain behaviour).
  * Same arguments, layout and errors as kda_decode_step; with opt->num_qk_heads = Hk, q and k are
- * [N, Hk, dk].
+ * [N, Hk, dk].  log_alpha is fp32, or bf16 with KDA_PROLOGUE_GATE_BF16.
  */
-kda_status kda_decode_step_ex(const void* q, const void* k, const void* v, const float* log_alpha,
+kda_status kda_decode_step_ex(const void* q, const void* k, const void* v, const void* log_alpha,
                               const float* beta, float* S_inout, void* out, int N, int H, int dk, int dv,
                               kda_dtype dt, const kda_options* opt, kda_stream_t stream);
 

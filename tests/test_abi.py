@@ -108,9 +108,9 @@ def test_options_are_validated_before_launch(lib):
     res = KdaOptions(num_qk_heads=3)
     res.reserved[2] = 1
     assert lib.kda_chunk_fwd_ex(*args, ctypes.byref(res), fake, 1 << 30, None) == 1
-    unknown = KdaOptions(prologue=8)                # not a KDA_PROLOGUE_* bit
+    unknown = KdaOptions(prologue=16)               # not a KDA_PROLOGUE_* bit
     assert lib.kda_chunk_fwd_ex(*args, ctypes.byref(unknown), fake, 1 << 30, None) == 1
-    ok_group = KdaOptions(num_qk_heads=3, prologue=7)
+    ok_group = KdaOptions(num_qk_heads=3, prologue=15)
     # a valid group with a missing workspace fails only on the workspace, like kda_chunk_fwd
     assert lib.kda_chunk_fwd_ex(*args, ctypes.byref(ok_group), None, 1 << 30, None) == 5
     assert lib.kda_chunk_fwd_ex(*args, None, None, 1 << 30, None) == 5

@@ -18,6 +18,9 @@ arrays into it.  Every function follows a passage of the pages:
 * ``decode_step`` -- one token per sequence, in the loop order (decay, delta, update, output) of
                      the review's GDN pseudo-code.
 
+``bwd`` is the reverse-mode derivative of ``seq`` (the training backward pass): the recurrence's
+step differentiated as written, walking the tokens backwards.
+
 ``gated_rmsnorm`` is the output gate (grouped RMS norm times the gate z).
 
 ``prologue`` is the input transform of the kernels' optional prologue (q/k L2 normalisation,
@@ -86,6 +89,8 @@ def _load():
         lib.kda_oracle_chunked_grouped.restype = I
         lib.kda_oracle_decode_step_grouped.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P]
         lib.kda_oracle_decode_step_grouped.restype = I
+        lib.kda_oracle_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, P, P, P, P, P, P, P, I]
+        lib.kda_oracle_bwd.restype = I
         _lib = lib
     return _lib
 
@@ -212,6 +217,45 @@ def decode_step(q, k, v, log_alpha, beta, S):
     if rc != 0:
         raise RuntimeError(f"kda_oracle_decode_step failed with status {rc}")
     return out, S
+
+
+def bwd(q, k, v, log_alpha, beta, dout, S0=None, dS_final=None, cu_seqlens=None, pairs=None, threads=None):
+    """Reverse-mode derivative of ``seq`` for the loss ``sum(dout * out) + sum(dS_final * S_final)``.
+
+    Same inputs as ``seq`` plus the cotangents ``dout`` (layout of ``v``) and ``dS_final``
+    ``[N, H, dk, dv]`` (None = 0).  Grouped q/k heads: the per-value-head derivatives of q and k
+    are summed over each group (value head h reads q/k head h // (H // Hk)).
+    Returns a dict of float64 arrays ``dq, dk`` (layout of q), ``dv`` (of v), ``dlog_alpha``,
+    ``dbeta`` and ``dS0`` ``[N, H, dk, dv]``."""
+    shape4 = np.asarray(q).ndim == 4
+    q_, k_, v_, la, b, s0, cu, N, H, Hk, dk, dv = _prep(q, k, v, log_alpha, beta, S0, cu_seqlens)
+    Ttot = q_.shape[0]
+    G = H // Hk
+    if G != 1:  # one q/k copy per value head
+        q_, k_ = (np.ascontiguousarray(np.repeat(x, G, axis=1)) for x in (q_, k_))
+    do = np.ascontiguousarray(np.asarray(dout, dtype=np.float64).reshape(Ttot, H, dv))
+    dsf = None if dS_final is None else np.ascontiguousarray(
+        np.asarray(dS_final, dtype=np.float64).reshape(N, H, dk, dv))
+    dq = np.zeros((Ttot, H, dk)); dk_ = np.zeros((Ttot, H, dk)); dv_ = np.zeros((Ttot, H, dv))
+    dla = np.zeros((Ttot, H, dk)); db = np.zeros((Ttot, H)); ds0 = np.zeros((N, H, dk, dv))
+    mask = None
+    if pairs is not None:
+        mask = np.zeros(N * H, dtype=np.int32)
+        for n, h in pairs:
+            mask[n * H + h] = 1
+    rc = _load().kda_oracle_bwd(_ptr(q_), _ptr(k_), _ptr(v_), _ptr(la), _ptr(b), _ptr(s0), _ptr(do), _ptr(dsf),
+                                _ptr(cu), N, H, dk, dv, _ptr(dq), _ptr(dk_), _ptr(dv_), _ptr(dla), _ptr(db),
+                                _ptr(ds0), _ptr(mask), threads or default_threads())
+    if rc != 0:
+        raise RuntimeError(f"kda_oracle_bwd failed with status {rc}")
+    if G != 1:
+        dq, dk_ = (x.reshape(Ttot, Hk, G, dk).sum(axis=2) for x in (dq, dk_))
+    res = dict(dq=dq, dk=dk_, dv=dv_, dlog_alpha=dla, dbeta=db, dS0=ds0)
+    if shape4:
+        T = Ttot // N
+        for key in ("dq", "dk", "dv", "dlog_alpha", "dbeta"):
+            res[key] = res[key].reshape((N, T) + res[key].shape[1:])
+    return res
 
 
 QK_NORM_EPS = 1e-6  # x / sqrt(sum x^2 + eps): the epsilon of the in-kernel q/k normalisation

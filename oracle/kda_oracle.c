@@ -34,6 +34,9 @@
  *   kda_oracle_bruteforce the dense transition matrix M_t = (I - b k k^T) Diag(a), S = M S + b k v^T
  *   kda_oracle_chunked    the chunk/WY/UT re-association, chunk size C        (exact up to rounding)
  * and kda_oracle_decode_step, one token per sequence, in the review's loop order.
+ * kda_oracle_bwd is the reverse-mode derivative of kda_oracle_seq (the training backward pass):
+ * the same step differentiated as written, tokens walked backwards, states recomputed from
+ * checkpoints.
  */
 #include <math.h>
 #include <pthread.h>
@@ -417,4 +420,222 @@ int kda_oracle_decode_step(const float* q, const float* k, const float* v, const
                            const float* beta, double* S, int N, int H, int dk, int dv, double* out)
 {
     return kda_oracle_decode_step_grouped(q, k, v, log_alpha, beta, S, N, H, H, dk, dv, out);
+}
+
+/* ==========================================================================================
+ * Backward pass (reverse-mode derivative of the recurrence), for a scalar loss
+ *     f = sum_t <dout_t, o_t> + <dS_final, S_final>
+ * given the cotangents dout ([Ttot][H][dv]) and dS_final ([N][H][dk][dv], or NULL = 0).
+ * Returns df/dq, df/dk ([Ttot][H][dk], one entry per VALUE head), df/dv, df/dlog_alpha,
+ * df/dbeta and df/dS0.
+ *
+ * The forward step, written the way the derivative is taken (the same update as pair_seq):
+ *   M   = Diag(alpha_t) S_{t-1}                 (alpha = exp(log_alpha), row c scaled)
+ *   w   = M^T k_t,   u = beta_t (v_t - w)       (u: the corrected value written at step t)
+ *   S_t = M + k_t u^T                           (= (I - beta k k^T) M + beta k v^T)
+ *   o_t = S_t^T q_t
+ * Walking t backwards with G = df/dS_t (starting from dS_final):
+ *   G    += q_t dout_t^T,          dq_t = S_t dout_t
+ *   du    = G^T k_t,               dk_t = G u
+ *   dbeta = du . (v_t - w),        dv_t = beta du,        dw = -beta du
+ *   dk_t += M dw,                  dM   = G + k_t dw^T
+ *   dlog_alpha_c = alpha_c sum_j dM[c][j] S_{t-1}[c][j],  G <- Diag(alpha) dM   (= df/dS_{t-1})
+ * The states S_{t-1}, S_t are recomputed forward from checkpoints kept every kBwdSeg steps, so
+ * memory stays O(T/kBwdSeg + kBwdSeg) states per pair whatever the sequence length.
+ * ========================================================================================== */
+#define kBwdSeg 64
+
+typedef struct {
+    const float *q, *k, *v, *log_alpha, *beta;
+    const double *S0, *dout, *dS_final;
+    const int64_t* cu_seqlens;
+    const int32_t* pair_mask;
+    int N, H, dk, dv;
+    double *dq, *dk_, *dv_, *dla, *dbeta, *dS0;
+    int next_pair;
+    pthread_mutex_t lock;
+    int status;
+} bjob_t;
+
+/* one forward step S <- step(S) at token t of head h (the update of pair_seq, outputs omitted) */
+static void bwd_step_fwd(const bjob_t* J, int64_t t, int h, double* S, double* w)
+{
+    const int H = J->H, dk = J->dk, dv = J->dv;
+    const float* kt = J->k + IDX3(t, h, 0, H, dk);
+    const float* vt = J->v + IDX3(t, h, 0, H, dv);
+    const float* la = J->log_alpha + IDX3(t, h, 0, H, dk);
+    const double b = (double)J->beta[(size_t)t * H + h];
+    for (int c = 0; c < dk; ++c) {
+        const double a = exp((double)la[c]);
+        for (int j = 0; j < dv; ++j) S[(size_t)c * dv + j] *= a;
+    }
+    for (int j = 0; j < dv; ++j) w[j] = 0.0;
+    for (int c = 0; c < dk; ++c)
+        for (int j = 0; j < dv; ++j) w[j] += (double)kt[c] * S[(size_t)c * dv + j];
+    for (int c = 0; c < dk; ++c)
+        for (int j = 0; j < dv; ++j) S[(size_t)c * dv + j] += (double)kt[c] * b * ((double)vt[j] - w[j]);
+}
+
+static void pair_bwd(const bjob_t* J, int n, int h, double* ck, double* seg, double* G, double* M, double* w,
+                     double* du)
+{
+    const int H = J->H, dk = J->dk, dv = J->dv;
+    const size_t sz = (size_t)dk * dv;
+    const size_t p = (size_t)n * H + h;
+    const int64_t t0 = J->cu_seqlens[n], t1 = J->cu_seqlens[n + 1];
+    const int64_t nseg = (t1 - t0 + kBwdSeg - 1) / kBwdSeg;
+    /* checkpoints: ck[s] = state before token t0 + s * kBwdSeg */
+    double* S = seg;
+    if (J->S0) memcpy(S, J->S0 + p * sz, sizeof(double) * sz);
+    else memset(S, 0, sizeof(double) * sz);
+    for (int64_t s = 0; s < nseg; ++s) {
+        memcpy(ck + (size_t)s * sz, S, sizeof(double) * sz);
+        const int64_t e = (t0 + (s + 1) * kBwdSeg < t1) ? t0 + (s + 1) * kBwdSeg : t1;
+        for (int64_t t = t0 + s * kBwdSeg; t < e; ++t) bwd_step_fwd(J, t, h, S, w);
+    }
+    /* G = df/dS_final */
+    if (J->dS_final) memcpy(G, J->dS_final + p * sz, sizeof(double) * sz);
+    else memset(G, 0, sizeof(double) * sz);
+    for (int64_t s = nseg - 1; s >= 0; --s) {
+        const int64_t ts = t0 + s * kBwdSeg;
+        const int64_t e = (ts + kBwdSeg < t1) ? ts + kBwdSeg : t1;
+        /* seg[i] = state before token ts + i, i = 0 .. e - ts */
+        memcpy(seg, ck + (size_t)s * sz, sizeof(double) * sz);
+        for (int64_t t = ts; t < e; ++t) {
+            memcpy(seg + (size_t)(t - ts + 1) * sz, seg + (size_t)(t - ts) * sz, sizeof(double) * sz);
+            bwd_step_fwd(J, t, h, seg + (size_t)(t - ts + 1) * sz, w);
+        }
+        for (int64_t t = e - 1; t >= ts; --t) {
+            const double* Sp = seg + (size_t)(t - ts) * sz;     /* S_{t-1} */
+            const double* St = seg + (size_t)(t - ts + 1) * sz; /* S_t */
+            const float* qt = J->q + IDX3(t, h, 0, H, dk);
+            const float* kt = J->k + IDX3(t, h, 0, H, dk);
+            const float* vt = J->v + IDX3(t, h, 0, H, dv);
+            const float* la = J->log_alpha + IDX3(t, h, 0, H, dk);
+            const double* dot = J->dout + IDX3(t, h, 0, H, dv);
+            const double b = (double)J->beta[(size_t)t * H + h];
+            double* dqt = J->dq + IDX3(t, h, 0, H, dk);
+            double* dkt = J->dk_ + IDX3(t, h, 0, H, dk);
+            double* dvt = J->dv_ + IDX3(t, h, 0, H, dv);
+            double* dlat = J->dla + IDX3(t, h, 0, H, dk);
+            /* readout o_t = S_t^T q_t */
+            for (int c = 0; c < dk; ++c) {
+                double acc = 0.0;
+                for (int j = 0; j < dv; ++j) {
+                    G[(size_t)c * dv + j] += (double)qt[c] * dot[j];
+                    acc += St[(size_t)c * dv + j] * dot[j];
+                }
+                dqt[c] = acc;
+            }
+            /* M = Diag(alpha) S_{t-1},  w = M^T k,  u = beta (v - w) */
+            for (int c = 0; c < dk; ++c) {
+                const double a = exp((double)la[c]);
+                for (int j = 0; j < dv; ++j) M[(size_t)c * dv + j] = a * Sp[(size_t)c * dv + j];
+            }
+            for (int j = 0; j < dv; ++j) {
+                double acc = 0.0;
+                for (int c = 0; c < dk; ++c) acc += M[(size_t)c * dv + j] * (double)kt[c];
+                w[j] = acc;
+            }
+            /* S_t = M + k u^T */
+            double db = 0.0;
+            for (int j = 0; j < dv; ++j) {
+                double acc = 0.0;
+                for (int c = 0; c < dk; ++c) acc += G[(size_t)c * dv + j] * (double)kt[c];
+                du[j] = acc;                               /* du = G^T k */
+                db += acc * ((double)vt[j] - w[j]);        /* u = beta (v - w) */
+                dvt[j] = b * acc;
+            }
+            J->dbeta[(size_t)t * H + h] = db;
+            for (int c = 0; c < dk; ++c) {
+                double acc = 0.0, acc2 = 0.0;
+                for (int j = 0; j < dv; ++j) {
+                    acc += G[(size_t)c * dv + j] * b * ((double)vt[j] - w[j]);  /* G u */
+                    acc2 += M[(size_t)c * dv + j] * (-b * du[j]);               /* M dw */
+                }
+                dkt[c] = acc + acc2;
+            }
+            /* dM = G + k dw^T, then the decay */
+            for (int c = 0; c < dk; ++c) {
+                const double a = exp((double)la[c]);
+                double da = 0.0;
+                for (int j = 0; j < dv; ++j) {
+                    const double dm = G[(size_t)c * dv + j] + (double)kt[c] * (-b * du[j]);
+                    da += dm * Sp[(size_t)c * dv + j];
+                    G[(size_t)c * dv + j] = a * dm;
+                }
+                dlat[c] = a * da;
+            }
+        }
+    }
+    if (J->dS0) memcpy(J->dS0 + p * sz, G, sizeof(double) * sz);
+}
+
+static void* bwd_worker(void* arg)
+{
+    bjob_t* J = (bjob_t*)arg;
+    const int dk = J->dk, dv = J->dv;
+    const size_t sz = (size_t)dk * dv;
+    int64_t maxlen = 0;
+    for (int n = 0; n < J->N; ++n)
+        if (J->cu_seqlens[n + 1] - J->cu_seqlens[n] > maxlen) maxlen = J->cu_seqlens[n + 1] - J->cu_seqlens[n];
+    const size_t nck = (size_t)((maxlen + kBwdSeg - 1) / kBwdSeg) + 1;
+    double* buf = (double*)malloc(sizeof(double) * (sz * (nck + kBwdSeg + 1 + 2) + 2 * (size_t)dv));
+    if (!buf) {
+        pthread_mutex_lock(&J->lock);
+        J->status = -2;
+        pthread_mutex_unlock(&J->lock);
+        return NULL;
+    }
+    double* ck = buf;
+    double* seg = ck + sz * nck;
+    double* G = seg + sz * (kBwdSeg + 1);
+    double* M = G + sz;
+    double* w = M + sz;
+    double* du = w + dv;
+    for (;;) {
+        pthread_mutex_lock(&J->lock);
+        const int p = J->next_pair++;
+        pthread_mutex_unlock(&J->lock);
+        if (p >= J->N * J->H) break;
+        if (J->pair_mask && !J->pair_mask[p]) continue;
+        pair_bwd(J, p / J->H, p % J->H, ck, seg, G, M, w, du);
+    }
+    free(buf);
+    return NULL;
+}
+
+/* Backward of kda_oracle_seq (one q/k head per value head).  Inputs as kda_oracle_seq plus
+ * dout [Ttot][H][dv] and dS_final [N][H][dk][dv] (NULL = 0); outputs (all fp64, caller-owned):
+ * dq, dk [Ttot][H][dk], dv [Ttot][H][dv], dlog_alpha [Ttot][H][dk], dbeta [Ttot][H],
+ * dS0 [N][H][dk][dv] (NULL = not wanted).  Pairs outside pair_mask are left untouched.
+ * Returns 0, -1 on bad arguments, -2 out of memory. */
+int kda_oracle_bwd(const float* q, const float* k, const float* v, const float* log_alpha, const float* beta,
+                   const double* S0, const double* dout, const double* dS_final, const int64_t* cu_seqlens, int N,
+                   int H, int dk, int dv, double* dq, double* dk_out, double* dv_out, double* dlog_alpha,
+                   double* dbeta, double* dS0, const int32_t* pair_mask, int num_threads)
+{
+    if (!q || !k || !v || !log_alpha || !beta || !dout || !cu_seqlens) return -1;
+    if (!dq || !dk_out || !dv_out || !dlog_alpha || !dbeta) return -1;
+    if (N < 0 || H <= 0 || dk <= 0 || dv <= 0) return -1;
+    for (int n = 0; n < N; ++n)
+        if (cu_seqlens[n + 1] < cu_seqlens[n]) return -1;
+    bjob_t J;
+    memset(&J, 0, sizeof(J));
+    J.q = q; J.k = k; J.v = v; J.log_alpha = log_alpha; J.beta = beta;
+    J.S0 = S0; J.dout = dout; J.dS_final = dS_final; J.cu_seqlens = cu_seqlens; J.pair_mask = pair_mask;
+    J.N = N; J.H = H; J.dk = dk; J.dv = dv;
+    J.dq = dq; J.dk_ = dk_out; J.dv_ = dv_out; J.dla = dlog_alpha; J.dbeta = dbeta; J.dS0 = dS0;
+    if (num_threads < 1) num_threads = 1;
+    pthread_mutex_init(&J.lock, NULL);
+    pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)num_threads);
+    int started = 0;
+    if (th)
+        for (int i = 0; i < num_threads; ++i)
+            if (pthread_create(&th[i], NULL, bwd_worker, &J) == 0) ++started;
+    if (started == 0) bwd_worker(&J);
+    for (int i = 0; i < started; ++i) pthread_join(th[i], NULL);
+    free(th);
+    pthread_mutex_destroy(&J.lock);
+    return J.status;
 }

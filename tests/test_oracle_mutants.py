@@ -6,6 +6,7 @@ import subprocess
 import pytest
 
 import oracle as oracle_mod
+from tests import test_oracle_bwd as bwd_pins
 from tests import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle_mod.__file__), "kda_oracle.c")
@@ -39,6 +40,24 @@ MUTANTS = [
     ("grouped: value head h reads q/k head h % Hk",
      "#define QKIDX(J, t, h, c) IDX3(t, (h) / ((J)->H / (J)->Hk), c, (J)->Hk, (J)->dk)",
      "#define QKIDX(J, t, h, c) IDX3(t, (h) % (J)->Hk, c, (J)->Hk, (J)->dk)"),
+    ("bwd: dM loses the k dw^T term",
+     "const double dm = G[(size_t)c * dv + j] + (double)kt[c] * (-b * du[j]);",
+     "const double dm = G[(size_t)c * dv + j];"),
+    ("bwd: dv without beta",
+     "dvt[j] = b * acc;",
+     "dvt[j] = acc;"),
+    ("bwd: carried cotangent not decayed",
+     "G[(size_t)c * dv + j] = a * dm;",
+     "G[(size_t)c * dv + j] = dm;"),
+    ("bwd: dq from the state before the step",
+     "acc += St[(size_t)c * dv + j] * dot[j];",
+     "acc += Sp[(size_t)c * dv + j] * dot[j];"),
+    ("bwd: dk misses the M dw term",
+     "dkt[c] = acc + acc2;",
+     "dkt[c] = acc;"),
+    ("bwd: recomputed segment starts one step late",
+     "memcpy(seg, ck + (size_t)s * sz, sizeof(double) * sz);\n        for (int64_t t = ts; t < e; ++t) {",
+     "memcpy(seg, ck + (size_t)s * sz, sizeof(double) * sz);\n        for (int64_t t = ts + 1; t < e; ++t) {"),
     ("decode: output from the decayed (pre-update) state",
      "for (int c = 0; c < dk; ++c)\n            for (int j = 0; j < dv; ++j) Sp[(size_t)c * dv + j] += (double)kp[c] * (b * d[j]);\n        if (out)",
      "if (out)"),
@@ -57,6 +76,8 @@ def _pins():
         lambda o: pins.test_decode_equals_prefill(o),
         lambda o: pins.test_per_step_invariant(o),
         lambda o: pins.test_grouped_heads_equal_repeated_qk(o, "seq"),
+        lambda o: bwd_pins.test_bwd_matches_finite_differences(o),
+        lambda o: bwd_pins.test_bwd_single_step_closed_form(o),
     ]
 
 

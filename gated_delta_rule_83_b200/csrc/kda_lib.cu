@@ -5,6 +5,7 @@
 #include <cstring>
 
 #include "kda.h"
+#include "backward_simt.cuh"
 #include "common.cuh"
 #include "chunks.cuh"
 #include "decode.cuh"
@@ -78,6 +79,26 @@ kda_status make_plan(int B, int T, int H, int dk, int dv, bool varlen, int num_s
     p.off_bytes = round_up(sizeof(int) * (2 * (size_t)p.N + 1), kAlign);  // off[N+1] + order[N]
     p.slot_bytes = p.tc ? tc_slot_bytes() : round_up(sizeof(float) * simt_slot_floats(dk, dv), kAlign);
     p.total_bytes = sizeof(WsHeader) + p.off_bytes + (size_t)p.max_chunks * (size_t)H * p.slot_bytes;
+    return KDA_OK;
+}
+
+// Backward workspace: the forward's header and chunk table, then per (chunk, head) the CUDA-core
+// forward slot, the chunk's start state, its end cotangent and the state-side scratch.
+struct BwdPlan {
+    Plan f;
+    size_t slot_bytes, state_bytes, scr_bytes, total_bytes;
+};
+
+kda_status make_bwd_plan(int B, int T, int H, int dk, int dv, bool varlen, int num_seqs, kda_dtype dt, BwdPlan& p)
+{
+    const kda_status st = make_plan(B, T, H, dk, dv, varlen, num_seqs, dt, p.f);
+    if (st != KDA_OK) return st;
+    const size_t units = (size_t)p.f.max_chunks * (size_t)H;
+    // dense per-unit strides: the kernels index these regions as float arrays
+    p.slot_bytes = sizeof(float) * simt_slot_floats(dk, dv);
+    p.state_bytes = sizeof(float) * (size_t)dk * dv;
+    p.scr_bytes = sizeof(float) * bwd_scr_floats(dk, dv);
+    p.total_bytes = sizeof(WsHeader) + p.f.off_bytes + units * (p.slot_bytes + 2 * p.state_bytes + p.scr_bytes);
     return KDA_OK;
 }
 
@@ -215,6 +236,68 @@ kda_status kda_decode_step(const void* q, const void* k, const void* v, const fl
                            kda_stream_t stream)
 {
     return kda_decode_step_ex(q, k, v, log_alpha, beta, S_inout, out, N, H, dk, dv, dt, nullptr, stream);
+}
+
+kda_status kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int varlen, int num_seqs,
+                                        kda_dtype dt, size_t* bytes)
+{
+    if (!bytes) return KDA_ERR_INVALID_ARG;
+    BwdPlan p;
+    const kda_status st = make_bwd_plan(B, T, H, dk, dv, varlen != 0, num_seqs, dt, p);
+    if (st != KDA_OK) return st;
+    *bytes = p.total_bytes;
+    return KDA_OK;
+}
+
+kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, const void* log_alpha, const float* beta,
+                         const float* S0, const int32_t* cu_seqlens, int num_seqs, const void* dout,
+                         const float* dS_final, void* dq, void* dk_out, void* dv_out, float* dlog_alpha, float* dbeta,
+                         float* dS0, int B, int T, int H, int dk, int dv, kda_dtype dt, const kda_options* opt,
+                         void* workspace, size_t workspace_bytes, kda_stream_t stream_)
+{
+    cudaStream_t stream = (cudaStream_t)stream_;
+    int Hk = H;
+    unsigned pro = 0;
+    const kda_status so = parse_options(opt, H, Hk, pro);
+    if (so != KDA_OK) return so;
+    if (Hk != H || (pro & ~KDA_PROLOGUE_GATE_BF16)) return KDA_ERR_UNSUPPORTED;
+    BwdPlan p;
+    const kda_status st = make_bwd_plan(B, T, H, dk, dv, cu_seqlens != nullptr, num_seqs, dt, p);
+    if (st != KDA_OK) return st;
+    if (p.f.Ttot > 0 && (!q || !k || !v || !log_alpha || !beta || !dout || !dq || !dk_out || !dv_out ||
+                         !dlog_alpha || !dbeta))
+        return KDA_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, log_alpha, beta, S0, dout, dS_final, dq, dk_out, dv_out, dlog_alpha, dbeta, dS0};
+    for (const void* x : ptrs)
+        if (x && !aligned16(x)) return KDA_ERR_INVALID_ARG;
+    if (cu_seqlens && ((uintptr_t)cu_seqlens & 3u)) return KDA_ERR_INVALID_ARG;
+    if (!workspace || ((uintptr_t)workspace % kAlign) || workspace_bytes < p.total_bytes) return KDA_ERR_WORKSPACE;
+
+    char* ws = (char*)workspace;
+    WsHeader* hdr = (WsHeader*)ws;
+    int* off = (int*)(ws + sizeof(WsHeader));
+    const size_t units = (size_t)p.f.max_chunks * (size_t)H;
+    char* slots = ws + sizeof(WsHeader) + p.f.off_bytes;
+    char* states = slots + units * p.slot_bytes;
+    char* cot = states + units * p.state_bytes;
+    char* scr = cot + units * p.state_bytes;
+    {
+        LaunchScope ls("chunk_table", stream);
+        chunk_table_kernel<<<1, kTableThreads, 0, stream>>>(cu_seqlens, p.f.N, p.f.Tseq, p.f.Ttot, hdr, off,
+                                                             off + p.f.N + 1);
+        if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
+    }
+    // the per-unit regions are indexed by (chunk, head) with the dense strides of the kernels
+    const cudaError_t e = (dt == KDA_BF16)
+        ? launch_simt_backward<__nv_bfloat16>(q, k, v, log_alpha, beta, S0, dout, dS_final, dq, dk_out, dv_out,
+                                              dlog_alpha, dbeta, dS0, hdr, off, cu_seqlens, p.f.Tseq, p.f.N, H, pro,
+                                              dk, dv, p.f.max_chunks, (float*)slots, (float*)states, (float*)cot,
+                                              (float*)scr, stream)
+        : launch_simt_backward<float>(q, k, v, log_alpha, beta, S0, dout, dS_final, dq, dk_out, dv_out, dlog_alpha,
+                                      dbeta, dS0, hdr, off, cu_seqlens, p.f.Tseq, p.f.N, H, pro, dk, dv,
+                                      p.f.max_chunks, (float*)slots, (float*)states, (float*)cot, (float*)scr,
+                                      stream);
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
 kda_status kda_gated_rmsnorm(const void* o, const void* z, const float* weight, void* y, long long rows, int d,

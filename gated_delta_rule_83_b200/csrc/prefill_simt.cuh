@@ -217,7 +217,7 @@ template <typename TOut>
 __global__ void __launch_bounds__(kSimtThreads)
 simt_inter_kernel(const float* S0, float* S_final, TOut* __restrict__ out, const WsHeader* __restrict__ hdr,
                   const int* __restrict__ off, const int32_t* __restrict__ cu, int Tseq, int N, int H, int dk, int dv,
-                  const float* __restrict__ slots)
+                  const float* __restrict__ slots, float* __restrict__ S_chunks)
 {
     extern __shared__ __align__(16) float smem[];
     const int n = blockIdx.x, h = blockIdx.y, v0 = blockIdx.z * kSimtNV, tid = threadIdx.x;
@@ -251,6 +251,10 @@ simt_inter_kernel(const float* S0, float* S_final, TOut* __restrict__ out, const
         const float* gUv = gP + (size_t)kChunk * kChunk;
         const float* gGam = gUv + (size_t)kChunk * dv;
         __syncthreads();  // previous chunk finished with the staged operands
+        if (S_chunks) {  // the chunk's start state, kept for the backward pass
+            float* dst = S_chunks + ((size_t)j * H + h) * dk * dv + v0;
+            for (int e = tid; e < dk * NV; e += kSimtThreads) dst[(size_t)(e / NV) * dv + (e % NV)] = sS[e];
+        }
         for (int e = tid; e < kChunk * dk; e += kSimtThreads) { sW[e] = gW[e]; sQ[e] = gQ[e]; sKd[e] = gKd[e]; }
         for (int e = tid; e < kChunk * kChunk; e += kSimtThreads) sP[e] = gP[e];
         for (int e = tid; e < kChunk * NV; e += kSimtThreads) sUv[e] = gUv[(e / NV) * dv + v0 + (e % NV)];
@@ -265,7 +269,7 @@ simt_inter_kernel(const float* S0, float* S_final, TOut* __restrict__ out, const
         __syncthreads();
         for (int e = tid; e < kChunk * NV; e += kSimtThreads) {
             const int r = e / NV, jj = e % NV;
-            if (r >= L) continue;
+            if (r >= L || out == nullptr) continue;
             float o = 0.f;
             for (int c = 0; c < dk; ++c) o = fmaf(sQ[r * dk + c], sS[c * NV + jj], o);
             for (int i = 0; i <= r; ++i) o = fmaf(sP[r * kChunk + i], sU[i * NV + jj], o);
@@ -317,7 +321,7 @@ cudaError_t launch_simt_prefill(const void* q, const void* k, const void* v, con
     }
     LaunchScope ls("simt_inter", stream);
     simt_inter_kernel<TIn><<<dim3(N, H, dv / kSimtNV), kSimtThreads, smB, stream>>>(
-        S0, S_final, (TIn*)out, hdr, off, cu, Tseq, N, H, dk, dv, slots);
+        S0, S_final, (TIn*)out, hdr, off, cu, Tseq, N, H, dk, dv, slots, nullptr);
     return cudaGetLastError();
 }
 

@@ -47,6 +47,9 @@ ABI = {
     "kda_decode_step_ex": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, ctypes.POINTER(KdaOptions), _P]),
     "kda_gated_rmsnorm": (_I, [_P, _P, _P, _P, ctypes.c_longlong, _I, _I, ctypes.c_float, _I, _I, _P]),
     "kda_chunk_fwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
+    "kda_chunk_bwd_workspace_size": (_I, [_I, _I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_SZ)]),
+    "kda_chunk_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
+                           ctypes.POINTER(KdaOptions), _P, _SZ, _P]),
     "kda_check": (_I, [_P]),
     "kda_selftest_timeout": (_I, [_P]),
     "kda_profile_begin": (_I, []),
@@ -214,6 +217,80 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torc
                                   ctypes.byref(opt), _ptr(workspace), workspace.numel(), sh)
         _check("kda_chunk_fwd_ex", rc)
     return out, S_final
+
+
+def bwd_workspace_size(B: int, T: int, H: int, dk: int, dv: int, varlen: bool = False, num_seqs: int = 0,
+                       dtype: torch.dtype = torch.bfloat16) -> int:
+    lib = load_library()
+    n = ctypes.c_size_t(0)
+    dt = KDA_BF16 if dtype == torch.bfloat16 else KDA_F32
+    _check("kda_chunk_bwd_workspace_size",
+           lib.kda_chunk_bwd_workspace_size(B, T, H, dk, dv, int(bool(varlen)), num_seqs, dt, ctypes.byref(n)))
+    return n.value
+
+
+def chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor, beta: torch.Tensor,
+              dout: torch.Tensor, S0: Optional[torch.Tensor] = None, dS_final: Optional[torch.Tensor] = None,
+              cu_seqlens: Optional[torch.Tensor] = None, want_dS0: bool = True, grads: Optional[dict] = None,
+              workspace: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None) -> dict:
+    """Backward pass of ``chunk_fwd`` (``kda_chunk_bwd``): the derivatives of
+    ``L = sum(dout * out) + sum(dS_final * S_final)`` with respect to every input.
+
+    Inputs as ``chunk_fwd`` (one q/k head per value head; log_alpha fp32 or bf16) plus ``dout``
+    (layout and dtype of ``out``) and ``dS_final`` ([N, H, dk, dv] fp32 or None).  Returns a dict
+    ``dq, dk, dv`` (dtype of q), ``dlog_alpha`` (fp32), ``dbeta`` (fp32) and ``dS0`` (fp32, or None
+    when ``want_dS0`` is False).  ``grads`` may hold preallocated output tensors under those keys."""
+    lib = load_library()
+    _req(q, "q")
+    dev, dtq = q.device, q.dtype
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    for t, name in ((k, "k"), (v, "v"), (dout, "dout")):
+        _req(t, name, dtq, dev)
+    _req(log_alpha, "log_alpha", None, dev)
+    pro = _gate_bits(log_alpha, 0)
+    _req(beta, "beta", torch.float32, dev)
+    if k.shape != q.shape or tuple(log_alpha.shape) != (B, T, H, dk) or tuple(v.shape) != (B, T, H, dv) or \
+            tuple(beta.shape) != (B, T, H) or dout.shape != v.shape:
+        raise ValueError("inconsistent shapes")
+    N = B
+    if cu_seqlens is not None:
+        _req(cu_seqlens, "cu_seqlens", torch.int32, dev)
+        N = cu_seqlens.numel() - 1
+        if B != 1:
+            raise ValueError("packed varlen input needs B == 1")
+    for t, name in ((S0, "S0"), (dS_final, "dS_final")):
+        if t is not None:
+            _req(t, name, torch.float32, dev)
+            if tuple(t.shape) != (N, H, dk, dv):
+                raise ValueError(f"{name} must be [{N}, {H}, {dk}, {dv}]")
+    g = dict(grads or {})
+    want = {"dq": (q.shape, dtq), "dk": (q.shape, dtq), "dv": (v.shape, dtq),
+            "dlog_alpha": (log_alpha.shape, torch.float32), "dbeta": (beta.shape, torch.float32)}
+    if want_dS0:
+        want["dS0"] = ((N, H, dk, dv), torch.float32)
+    for key, (shape, dt) in want.items():
+        if g.get(key) is None:
+            g[key] = torch.empty(shape, dtype=dt, device=dev)
+        else:
+            _req(g[key], key, dt, dev)
+            if tuple(g[key].shape) != tuple(shape):
+                raise ValueError(f"{key} must be {tuple(shape)}")
+    if not want_dS0:
+        g["dS0"] = None
+    sh = _stream_handle(stream, dev)
+    ws_bytes = bwd_workspace_size(B, T, H, dk, dv, cu_seqlens is not None, N, dtq)
+    if workspace is None:
+        workspace = _get_workspace(ws_bytes, dev, sh)
+    else:
+        _req(workspace, "workspace", torch.uint8, dev)
+    opt = KdaOptions(num_qk_heads=0, prologue=pro)
+    rc = lib.kda_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0), _ptr(cu_seqlens), N,
+                           _ptr(dout), _ptr(dS_final), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]),
+                           _ptr(g["dlog_alpha"]), _ptr(g["dbeta"]), _ptr(g["dS0"]), B, T, H, dk, dv, _dt(q),
+                           ctypes.byref(opt), _ptr(workspace), workspace.numel(), sh)
+    _check("kda_chunk_bwd", rc)
+    return g
 
 
 NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024  # KDA_NOALLOC_SCRATCH_BYTES in include/kda.h

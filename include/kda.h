@@ -183,6 +183,42 @@ kda_status kda_decode_step_ex(const void* q, const void* k, const void* v, const
                               kda_dtype dt, const kda_options* opt, kda_stream_t stream);
 
 /*
+ * kda_chunk_bwd -- the backward pass of kda_chunk_fwd (training): the derivatives of a scalar loss
+ * L with respect to every input, given the cotangents of the outputs,
+ *
+ *     dq = dL/dq, dk = dL/dk, dv = dL/dv, dlog_alpha = dL/dlog_alpha, dbeta = dL/dbeta, dS0 = dL/dS0,
+ *
+ * for L = sum(dout * out) + sum(dS_final * S_final) with (out, S_final) = kda_chunk_fwd(...).  The
+ * pages mention a custom backward only in passing; the derivative is that of the recurrence of the
+ * "Kimi Linear" explainer (section "Kimi Delta Attention的技术内核"), taken through the chunk form
+ * its section "硬件效率的深度优化" lists: the forward is recomputed chunk-parallel keeping only each
+ * chunk's start state, the state cotangent runs backwards over the chunks, and the input
+ * derivatives are again chunk-parallel.  Arithmetic is fp32 on CUDA cores.
+ *
+ *   q, k, v, log_alpha, beta, S0, cu_seqlens, num_seqs, B, T, H, dk, dv, dt:  exactly as given to
+ *                kda_chunk_fwd (same layout, same meaning).
+ *   dout       [B, T, H, dv] (or packed [T, H, dv]) in dt: dL/dout.
+ *   dS_final   [N, H, dk, dv] fp32, or NULL: dL/dS_final = 0.
+ *   dq, dk     [B, T, H, dk] in dt;  dv [B, T, H, dv] in dt;  dlog_alpha [B, T, H, dk] fp32;
+ *   dbeta      [B, T, H] fp32;  dS0 [N, H, dk, dv] fp32 or NULL (not wanted).  All written whole.
+ *   opt        NULL, or num_qk_heads 0 / H and prologue 0 or KDA_PROLOGUE_GATE_BF16 (log_alpha in
+ *              bf16); anything else returns KDA_ERR_UNSUPPORTED.
+ *   workspace  >= kda_chunk_bwd_workspace_size(...) bytes, 256-byte aligned, owned by the caller
+ *              (about 4 * 64 * max(dk, dv) * 4 bytes per (64-token chunk, head) plus the state and
+ *              its cotangent for each chunk).
+ * Pointers 16-byte aligned (cu_seqlens 4), device memory, no overlap between outputs and inputs.
+ * Errors: as kda_chunk_fwd.  Asynchronous on `stream`; a malformed cu_seqlens sets the device
+ * error word (read by kda_check) and computes nothing.
+ */
+kda_status kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int varlen, int num_seqs,
+                                        kda_dtype dt, size_t* bytes);
+kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, const void* log_alpha, const float* beta,
+                         const float* S0, const int32_t* cu_seqlens, int num_seqs, const void* dout,
+                         const float* dS_final, void* dq, void* dk, void* dv, float* dlog_alpha, float* dbeta,
+                         float* dS0, int B, int T, int H, int dk_dim, int dv_dim, kda_dtype dt,
+                         const kda_options* opt, void* workspace, size_t workspace_bytes, kda_stream_t stream);
+
+/*
  * kda_gated_rmsnorm -- the output gate of a KDA layer, one fused streaming pass:
  *
  *     y = o / sqrt(mean_g(o^2) + eps) * weight * act(z)

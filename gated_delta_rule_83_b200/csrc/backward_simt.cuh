@@ -10,14 +10,13 @@
 //     U    = Uv - W S,   O = Qg S + P U,   S_next = Diag(gam) S + Kd^T U
 //
 //   1. forward recompute: the CUDA-core phase A, then its phase B storing every chunk's start
-//      state S_c (the only forward intermediate kept).
+//      state S_c and its corrected values U.
 //   2. reverse chain over chunks (one CTA per (sequence, head, 32 state columns), chunks last to
 //      first), carrying D = dL/dS_next:
 //          dU = P^T dO + Kd D
 //          D <- Diag(gam) D + Qg^T dO - W^T dU          (= dL/dS at the chunk start)
-//      storing every chunk's end cotangent D_c; D after the first chunk is dL/dS0.
-//   3. chunk-parallel, state side (one CTA per (chunk, head)): with S_c and D_c,
-//          U = Uv - W S_c,  dU = P^T dO + Kd D_c,
+//      storing every chunk's end cotangent D_c and dU; D after the first chunk is dL/dS0.
+//   3. chunk-parallel, state side (one CTA per (chunk, head)): with S_c, D_c, U and dU,
 //          dQg = dO S_c^T,  dW = -dU S_c^T,  dKd = U D_c^T,  dP = lower_incl(dO U^T),
 //          dgam_c = sum_j D_c[c][j] S_c[c][j]
 //   4. chunk-parallel, input side (one CTA per (chunk, head)): through the UT transform,
@@ -29,8 +28,9 @@
 //      e^{g_r - g_i}) and the gating itself to dq, dk and dg; dlog_alpha is the reverse cumulative
 //      sum of dg inside the chunk (g restarts every chunk).
 //
-// Steps 3 and 4 work on 32-channel tiles of the key dimension, so each CTA holds a few 64 x 64
-// matrices plus tiles.  The per-channel factors use the same centre-of-range reference as the
+// Steps 3 and 4 work on tiles of the key dimension, so each CTA holds a few 64 x 64 matrices plus
+// tiles; their products are register-tiled (each thread owns a 4 x 4, 4 x 2 or 8 x 2 block of
+// rows tr + 16 i and columns tc + 16 j, so the shared-memory reads of a warp hit distinct banks).  The per-channel factors use the same centre-of-range reference as the
 // forward; a tile whose in-chunk gate spread exceeds kFactorSpread takes the exact per-element
 // factor e^{g_r - g_i} (never above 1) instead.  Padding rows of a partial chunk are identity
 // steps with zero inputs and zero cotangents, so they contribute nothing.
@@ -46,87 +46,240 @@ constexpr int kBwdCT = 32;        // key channels per tile
 constexpr int kBwdLT = kBwdCT + 1; // padded tile row stride
 constexpr int kBwdL64 = kChunk + 1;
 
-// fp32 scratch of one (chunk, head) between steps 3 and 4:
-//   dU [64 x dv] | dQg [64 x dk] | dW [64 x dk] | dKd [64 x dk] | dP [64 x 64] | dgam [dk]
+// fp32 scratch of one (chunk, head), written by steps 1-3 and read by steps 3-4:
+//   U [64 x dv] | dU [64 x dv] | dQg [64 x dk] | dW [64 x dk] | dKd [64 x dk] | dP [64 x 64] | dgam [dk]
 __host__ __device__ inline size_t bwd_scr_floats(int dk, int dv)
 {
-    return (size_t)kChunk * dv + 3 * (size_t)kChunk * dk + (size_t)kChunk * kChunk + dk;
+    return 2 * (size_t)kChunk * dv + 3 * (size_t)kChunk * dk + (size_t)kChunk * kChunk + dk;
+}
+
+// 16-byte asynchronous global -> shared copies (zero-filled past src_bytes), in commit groups
+__device__ __forceinline__ void bwd_cp16(float* dst, const void* src, uint32_t src_bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+                 "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bwd_cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void bwd_cp_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// n floats (a multiple of 4), contiguous, by all threads
+__device__ __forceinline__ void bwd_cp_block(float* dst, const float* src, int n)
+{
+    for (int e = 4 * threadIdx.x; e < n; e += 4 * kSimtThreads) bwd_cp16(dst + e, src + e, 16);
+}
+
+// chunk j of sequence n (global chunk index) -> first token and length
+__device__ __forceinline__ void bwd_chunk_span(int j, int n, const int* __restrict__ off, long long s0, long long s1,
+                                               long long& t0, int& L)
+{
+    t0 = s0 + (long long)(j - off[n]) * kChunk;
+    L = (s1 - t0) < kChunk ? (int)(s1 - t0) : kChunk;
 }
 
 // ------------------------------------------------------------------------------------------------
-// Step 2: reverse chain of the state cotangent
+// Step 1b: forward chain keeping each chunk's start state and its U (one CTA per (sequence, head,
+// 32 state columns)).  Chunk c's W and Uv, and its Kd and gam, are copied in two cp.async groups
+// while the previous chunk's other half computes.
 // ------------------------------------------------------------------------------------------------
-template <typename TIn>
+template <int DK>
 __global__ void __launch_bounds__(kSimtThreads)
-bwd_dstate_kernel(const TIn* __restrict__ dout, const float* __restrict__ dS_final, float* __restrict__ dS0,
-                  const WsHeader* __restrict__ hdr, const int* __restrict__ off, const int32_t* __restrict__ cu,
-                  int Tseq, int N, int H, int dk, int dv, const float* __restrict__ slots,
-                  float* __restrict__ dSn_chunks)
+bwd_fwd_chain_kernel(const float* __restrict__ S0, const WsHeader* __restrict__ hdr, const int* __restrict__ off,
+                     const int32_t* __restrict__ cu, int Tseq, int N, int H, int dv, const float* __restrict__ slots,
+                     float* __restrict__ S_chunks, float* __restrict__ scr)
 {
     extern __shared__ __align__(16) float smem[];
     const int n = blockIdx.x, h = blockIdx.y, v0 = blockIdx.z * kSimtNV, tid = threadIdx.x;
     if (hdr->bad) return;
-    constexpr int NV = kSimtNV;
-    float* sD = smem;                       // [dk][NV]   D = dL/dS
-    float* sW = sD + dk * NV;               // [64][dk]
-    float* sQ = sW + kChunk * dk;           // [64][dk]
-    float* sKd = sQ + kChunk * dk;          // [64][dk]
-    float* sP = sKd + kChunk * dk;          // [64][64]
-    float* sO = sP + kChunk * kChunk;       // [64][NV]   dO
-    float* sU = sO + kChunk * NV;           // [64][NV]   dU
-    float* sG = sU + kChunk * NV;           // [dk]
-
-    const size_t sidx = ((size_t)n * H + h) * dk * dv;
-    for (int e = tid; e < dk * NV; e += kSimtThreads) {
-        const int c = e / NV, jj = e % NV;
-        sD[e] = dS_final ? dS_final[sidx + (size_t)c * dv + v0 + jj] : 0.f;
+    constexpr int NV = kSimtNV, TMD = DK / 16;
+    float* sS = smem;                 // [DK][NV]
+    float* sW = sS + DK * NV;         // [64][DK]
+    float* sKd = sW + kChunk * DK;    // [64][DK]
+    float* sUv = sKd + kChunk * DK;   // [64][NV]
+    float* sU = sUv + kChunk * NV;    // [64][NV]
+    float* sG = sU + kChunk * NV;     // [DK]
+    const int tr = tid >> 4, tc = tid & 15;
+    const size_t slot_f = simt_slot_floats(DK, dv), scr_f = bwd_scr_floats(DK, dv);
+    const size_t sidx = ((size_t)n * H + h) * DK * dv;
+    for (int e = tid; e < DK * NV; e += kSimtThreads)
+        sS[e] = S0 ? S0[sidx + (size_t)(e / NV) * dv + v0 + (e % NV)] : 0.f;
+    const int j0 = off[n], j1 = off[n + 1];
+    auto issue_w = [&](int j) {  // W and the Uv columns of chunk j
+        const float* slot = slots + ((size_t)j * H + h) * slot_f;
+        bwd_cp_block(sW, slot, kChunk * DK);
+        const float* gUv = slot + (size_t)kChunk * (3 * DK + kChunk);
+        for (int e = 4 * tid; e < kChunk * NV; e += 4 * kSimtThreads)
+            bwd_cp16(sUv + e, gUv + (size_t)(e / NV) * dv + v0 + (e % NV), 16);
+        bwd_cp_commit();
+    };
+    auto issue_k = [&](int j) {  // Kd and gam of chunk j
+        const float* slot = slots + ((size_t)j * H + h) * slot_f;
+        bwd_cp_block(sKd, slot + 2 * (size_t)kChunk * DK, kChunk * DK);
+        bwd_cp_block(sG, slot + (size_t)kChunk * (3 * DK + kChunk + dv), DK);
+        bwd_cp_commit();
+    };
+    if (j0 < j1) {
+        issue_w(j0);
+        issue_k(j0);
     }
+    for (int j = j0; j < j1; ++j) {
+        const size_t u = (size_t)j * H + h;
+        bwd_cp_wait<1>();  // W, Uv of chunk j landed (Kd may still be in flight)
+        __syncthreads();
+        float* dst = S_chunks + u * DK * dv + v0;
+        for (int e = tid; e < DK * NV; e += kSimtThreads) dst[(size_t)(e / NV) * dv + (e % NV)] = sS[e];
+        {  // U = Uv - W S
+            float x[4][2] = {};
+            mm_acc<4, 2>(x, sW, DK, 1, sS, NV, 1, DK, tr, tc);
+            float* gU = scr + u * scr_f + v0;
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int b = 0; b < 2; ++b) {
+                    const int r = tr + 16 * a, jj = tc + 16 * b;
+                    const float uu = sUv[r * NV + jj] - x[a][b];
+                    sU[r * NV + jj] = uu;
+                    gU[(size_t)r * dv + jj] = uu;
+                }
+        }
+        __syncthreads();
+        if (j + 1 < j1) issue_w(j + 1);
+        else bwd_cp_commit();  // keep one group per step
+        bwd_cp_wait<1>();      // Kd, gam of chunk j
+        __syncthreads();
+        {  // S <- Diag(gam) S + Kd^T U
+            float acc[TMD][2];
+#pragma unroll
+            for (int a = 0; a < TMD; ++a)
+#pragma unroll
+                for (int b = 0; b < 2; ++b) acc[a][b] = sG[tr + 16 * a] * sS[(tr + 16 * a) * NV + tc + 16 * b];
+            mm_acc<TMD, 2>(acc, sKd, 1, DK, sU, NV, 1, kChunk, tr, tc);
+            __syncthreads();  // every thread has read the old S
+#pragma unroll
+            for (int a = 0; a < TMD; ++a)
+#pragma unroll
+                for (int b = 0; b < 2; ++b) sS[(tr + 16 * a) * NV + tc + 16 * b] = acc[a][b];
+        }
+        __syncthreads();
+        if (j + 1 < j1) issue_k(j + 1);
+        else bwd_cp_commit();
+    }
+    bwd_cp_wait<0>();
+}
+
+// ------------------------------------------------------------------------------------------------
+// Step 2: reverse chain of the state cotangent (chunks last to first).  {P, Kd} and {Qg, W, gam}
+// of the next chunk are copied while the current chunk's other half computes; dO of the next chunk
+// is loaded into registers one half-step ahead.
+// ------------------------------------------------------------------------------------------------
+template <typename TIn, int DK>
+__global__ void __launch_bounds__(kSimtThreads)
+bwd_dstate_kernel(const TIn* __restrict__ dout, const float* __restrict__ dS_final, float* __restrict__ dS0,
+                  const WsHeader* __restrict__ hdr, const int* __restrict__ off, const int32_t* __restrict__ cu,
+                  int Tseq, int N, int H, int dv, const float* __restrict__ slots, float* __restrict__ dSn_chunks,
+                  float* __restrict__ scr)
+{
+    extern __shared__ __align__(16) float smem[];
+    const int n = blockIdx.x, h = blockIdx.y, v0 = blockIdx.z * kSimtNV, tid = threadIdx.x;
+    if (hdr->bad) return;
+    constexpr int NV = kSimtNV, TMD = DK / 16;
+    constexpr int OPT = kChunk * NV / kSimtThreads;  // dO elements per thread
+    float* sD = smem;                 // [DK][NV]   D = dL/dS
+    float* sW = sD + DK * NV;         // [64][DK]
+    float* sQ = sW + kChunk * DK;     // [64][DK]
+    float* sKd = sQ + kChunk * DK;    // [64][DK]
+    float* sP = sKd + kChunk * DK;    // [64][64]
+    float* sO = sP + kChunk * kChunk; // [64][NV]   dO
+    float* sU = sO + kChunk * NV;     // [64][NV]   dU
+    float* sG = sU + kChunk * NV;     // [DK]
+    const int tr = tid >> 4, tc = tid & 15;
+    const size_t slot_f = simt_slot_floats(DK, dv), scr_f = bwd_scr_floats(DK, dv);
+    const size_t sidx = ((size_t)n * H + h) * DK * dv;
+    for (int e = tid; e < DK * NV; e += kSimtThreads)
+        sD[e] = dS_final ? dS_final[sidx + (size_t)(e / NV) * dv + v0 + (e % NV)] : 0.f;
     long long s0, s1;
     seq_bounds(n, cu, Tseq, s0, s1);
-    const size_t slot_f = simt_slot_floats(dk, dv);
-    for (int j = off[n + 1] - 1; j >= off[n]; --j) {
-        const long long t0 = s0 + (long long)(j - off[n]) * kChunk;
-        const int L = (s1 - t0) < kChunk ? (int)(s1 - t0) : kChunk;
+    const int j0 = off[n], j1 = off[n + 1];
+    auto issue_pk = [&](int j) {
         const float* slot = slots + ((size_t)j * H + h) * slot_f;
-        const float* gW = slot;
-        const float* gQ = gW + (size_t)kChunk * dk;
-        const float* gKd = gQ + (size_t)kChunk * dk;
-        const float* gP = gKd + (size_t)kChunk * dk;
-        const float* gGam = gP + (size_t)kChunk * kChunk + (size_t)kChunk * dv;
-        __syncthreads();  // the previous chunk is done with the staged operands and D is final
-        float* dst = dSn_chunks + ((size_t)j * H + h) * dk * dv + v0;
-        for (int e = tid; e < dk * NV; e += kSimtThreads) dst[(size_t)(e / NV) * dv + (e % NV)] = sD[e];
-        for (int e = tid; e < kChunk * dk; e += kSimtThreads) { sW[e] = gW[e]; sQ[e] = gQ[e]; sKd[e] = gKd[e]; }
-        for (int e = tid; e < kChunk * kChunk; e += kSimtThreads) sP[e] = gP[e];
-        for (int e = tid; e < kChunk * NV; e += kSimtThreads) {
-            const int r = e / NV, jj = e % NV;
-            sO[e] = (r < L) ? to_f32(dout[((size_t)(t0 + r) * H + h) * dv + v0 + jj]) : 0.f;
+        bwd_cp_block(sKd, slot + 2 * (size_t)kChunk * DK, kChunk * DK);
+        bwd_cp_block(sP, slot + 3 * (size_t)kChunk * DK, kChunk * kChunk);
+        bwd_cp_commit();
+    };
+    auto issue_qw = [&](int j) {
+        const float* slot = slots + ((size_t)j * H + h) * slot_f;
+        bwd_cp_block(sW, slot, kChunk * DK);
+        bwd_cp_block(sQ, slot + (size_t)kChunk * DK, kChunk * DK);
+        bwd_cp_block(sG, slot + (size_t)kChunk * (3 * DK + kChunk + dv), DK);
+        bwd_cp_commit();
+    };
+    float od[OPT];  // dO of the chunk about to be processed, rows past its end zero
+    auto load_do = [&](int j) {
+        long long t0;
+        int L;
+        bwd_chunk_span(j, n, off, s0, s1, t0, L);
+#pragma unroll
+        for (int m = 0; m < OPT; ++m) {
+            const int e = tid + m * kSimtThreads, r = e / NV, jj = e % NV;
+            od[m] = (r < L) ? to_f32(dout[((size_t)(t0 + r) * H + h) * dv + v0 + jj]) : 0.f;
         }
-        for (int e = tid; e < dk; e += kSimtThreads) sG[e] = gGam[e];
-        __syncthreads();
-        // dU = P^T dO + Kd D
-        for (int e = tid; e < kChunk * NV; e += kSimtThreads) {
-            const int i = e / NV, jj = e % NV;
-            float x = 0.f;
-            for (int r = i; r < kChunk; ++r) x = fmaf(sP[r * kChunk + i], sO[r * NV + jj], x);
-            for (int c = 0; c < dk; ++c) x = fmaf(sKd[i * dk + c], sD[c * NV + jj], x);
-            sU[e] = x;
-        }
-        __syncthreads();
-        // D <- Diag(gam) D + Qg^T dO - W^T dU   (each thread rewrites only its own element)
-        for (int e = tid; e < dk * NV; e += kSimtThreads) {
-            const int c = e / NV, jj = e % NV;
-            float s = sG[c] * sD[e];
-            for (int r = 0; r < kChunk; ++r) {
-                s = fmaf(sQ[r * dk + c], sO[r * NV + jj], s);
-                s = fmaf(-sW[r * dk + c], sU[r * NV + jj], s);
-            }
-            sD[e] = s;
-        }
+    };
+    if (j0 < j1) {
+        issue_pk(j1 - 1);
+        issue_qw(j1 - 1);
+        load_do(j1 - 1);
     }
+    for (int j = j1 - 1; j >= j0; --j) {
+        const size_t u = (size_t)j * H + h;
+        bwd_cp_wait<1>();  // P, Kd of chunk j
+        __syncthreads();   // ... visible to all, and the previous step is done with D and dO
+#pragma unroll
+        for (int m = 0; m < OPT; ++m) sO[tid + m * kSimtThreads] = od[m];
+        float* dst = dSn_chunks + u * DK * dv + v0;
+        for (int e = tid; e < DK * NV; e += kSimtThreads) dst[(size_t)(e / NV) * dv + (e % NV)] = sD[e];
+        __syncthreads();
+        {  // dU = P^T dO + Kd D
+            float x[4][2] = {};
+            mm_acc<4, 2>(x, sP, 1, kChunk, sO, NV, 1, kChunk, tr, tc);
+            mm_acc<4, 2>(x, sKd, DK, 1, sD, NV, 1, DK, tr, tc);
+            float* gdU = scr + u * scr_f + (size_t)kChunk * dv + v0;
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int b = 0; b < 2; ++b) {
+                    const int i = tr + 16 * a, jj = tc + 16 * b;
+                    sU[i * NV + jj] = x[a][b];
+                    gdU[(size_t)i * dv + jj] = x[a][b];
+                }
+        }
+        __syncthreads();
+        if (j > j0) issue_pk(j - 1);
+        else bwd_cp_commit();
+        bwd_cp_wait<1>();  // Qg, W, gam of chunk j
+        __syncthreads();
+        {  // D <- Diag(gam) D + Qg^T dO - W^T dU
+            float acc[TMD][2], neg[TMD][2] = {};
+#pragma unroll
+            for (int a = 0; a < TMD; ++a)
+#pragma unroll
+                for (int b = 0; b < 2; ++b) acc[a][b] = sG[tr + 16 * a] * sD[(tr + 16 * a) * NV + tc + 16 * b];
+            mm_acc<TMD, 2>(acc, sQ, 1, DK, sO, NV, 1, kChunk, tr, tc);
+            mm_acc<TMD, 2>(neg, sW, 1, DK, sU, NV, 1, kChunk, tr, tc);
+            if (j > j0) load_do(j - 1);
+            __syncthreads();  // every thread has read the old D, Qg, W
+#pragma unroll
+            for (int a = 0; a < TMD; ++a)
+#pragma unroll
+                for (int b = 0; b < 2; ++b) sD[(tr + 16 * a) * NV + tc + 16 * b] = acc[a][b] - neg[a][b];
+        }
+        if (j > j0) issue_qw(j - 1);
+        else bwd_cp_commit();
+    }
+    bwd_cp_wait<0>();
     __syncthreads();
     if (dS0)
-        for (int e = tid; e < dk * NV; e += kSimtThreads)
+        for (int e = tid; e < DK * NV; e += kSimtThreads)
             dS0[sidx + (size_t)(e / NV) * dv + v0 + (e % NV)] = sD[e];
 }
 
@@ -137,8 +290,8 @@ template <typename TIn>
 __global__ void __launch_bounds__(kSimtThreads)
 bwd_state_side_kernel(const TIn* __restrict__ dout, const WsHeader* __restrict__ hdr, const int* __restrict__ off,
                       const int32_t* __restrict__ cu, int Tseq, int N, int H, int dk, int dv,
-                      const float* __restrict__ slots, const float* __restrict__ S_chunks,
-                      const float* __restrict__ dSn_chunks, float* __restrict__ scr)
+                      const float* __restrict__ S_chunks, const float* __restrict__ dSn_chunks,
+                      float* __restrict__ scr)
 {
     extern __shared__ __align__(16) float smem[];
     const int j = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
@@ -147,102 +300,83 @@ bwd_state_side_kernel(const TIn* __restrict__ dout, const WsHeader* __restrict__
     long long t0;
     locate_chunk(j, off, cu, Tseq, N, n, t0, L);
     const int LDV = dv + 1;
-    float* sU = smem;                       // [64][dv+1]  U
-    float* sdU = sU + kChunk * LDV;         // [64][dv+1]  dU
-    float* sO = sdU + kChunk * LDV;         // [64][dv+1]  dO
-    float* sP = sO + kChunk * LDV;          // [64][64]
-    float* sS = sP + kChunk * kChunk;       // [32][dv+1]  tile of S_c
-    float* sD = sS + kBwdCT * LDV;          // [32][dv+1]  tile of D_c
-    float* sWt = sD + kBwdCT * LDV;         // [64][33]    tile of W
-    float* sKt = sWt + kChunk * kBwdLT;     // [64][33]    tile of Kd
+    float* sO = smem;               // [64][dv+1]  dO
+    float* sU = sO + kChunk * LDV;  // [64][dv+1]  U
+    float* sdU = sU + kChunk * LDV; // [64][dv+1]  dU
+    float* sS = sdU + kChunk * LDV; // [64][dv+1]  64 channels (rows) of S_c
+    float* sD = sS + kChunk * LDV;  // [64][dv+1]  ... and of D_c
 
     const size_t u = (size_t)j * H + h;
-    const float* slot = slots + u * simt_slot_floats(dk, dv);
-    const float* gW = slot;
-    const float* gKd = gW + 2 * (size_t)kChunk * dk;
-    const float* gP = gKd + (size_t)kChunk * dk;
-    const float* gUv = gP + (size_t)kChunk * kChunk;
     const float* Sc = S_chunks + u * dk * dv;
     const float* Dc = dSn_chunks + u * dk * dv;
     float* o = scr + u * bwd_scr_floats(dk, dv);
-    float* oU = o;                                  // dU
-    float* oQg = oU + (size_t)kChunk * dv;          // dQg
-    float* oW = oQg + (size_t)kChunk * dk;          // dW
-    float* oKd = oW + (size_t)kChunk * dk;          // dKd
-    float* oP = oKd + (size_t)kChunk * dk;          // dP
-    float* oGam = oP + (size_t)kChunk * kChunk;     // dgam
+    const float* oU = o;
+    const float* odU = oU + (size_t)kChunk * dv;
+    float* oQg = o + 2 * (size_t)kChunk * dv;
+    float* oW = oQg + (size_t)kChunk * dk;
+    float* oKd = oW + (size_t)kChunk * dk;
+    float* oP = oKd + (size_t)kChunk * dk;
+    float* oGam = oP + (size_t)kChunk * kChunk;
 
     for (int e = tid; e < kChunk * dv; e += kSimtThreads) {
         const int r = e / dv, jj = e % dv;
-        sU[r * LDV + jj] = gUv[e];
         sO[r * LDV + jj] = (r < L) ? to_f32(dout[((size_t)(t0 + r) * H + h) * dv + jj]) : 0.f;
+        sU[r * LDV + jj] = oU[e];
+        sdU[r * LDV + jj] = odU[e];
     }
-    for (int e = tid; e < kChunk * kChunk; e += kSimtThreads) sP[e] = gP[e];
     __syncthreads();
-    for (int e = tid; e < kChunk * dv; e += kSimtThreads) {  // dU = P^T dO
-        const int i = e / dv, jj = e % dv;
-        float x = 0.f;
-        for (int r = i; r < kChunk; ++r) x = fmaf(sP[r * kChunk + i], sO[r * LDV + jj], x);
-        sdU[i * LDV + jj] = x;
+    const int tr = tid >> 4, tc = tid & 15;
+    {  // dP = lower_incl(dO U^T)
+        float acc[4][4] = {};
+        mm_acc<4, 4>(acc, sO, LDV, 1, sU, 1, LDV, dv, tr, tc);
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const int r = tr + 16 * a, i = tc + 16 * b;
+                oP[r * kChunk + i] = (i <= r) ? acc[a][b] : 0.f;
+            }
     }
-    // U -= W S_c and dU += Kd D_c, one 32-row tile of the state at a time
-    for (int c0 = 0; c0 < dk; c0 += kBwdCT) {
-        __syncthreads();
-        for (int e = tid; e < kBwdCT * dv; e += kSimtThreads) {
-            const int cc = e / dv, jj = e % dv;
-            sS[cc * LDV + jj] = Sc[(size_t)(c0 + cc) * dv + jj];
-            sD[cc * LDV + jj] = Dc[(size_t)(c0 + cc) * dv + jj];
-        }
-        for (int e = tid; e < kChunk * kBwdCT; e += kSimtThreads) {
-            const int r = e / kBwdCT, cc = e % kBwdCT;
-            sWt[r * kBwdLT + cc] = gW[(size_t)r * dk + c0 + cc];
-            sKt[r * kBwdLT + cc] = gKd[(size_t)r * dk + c0 + cc];
-        }
+    // dQg = dO S_c^T, dW = -dU S_c^T, dKd = U D_c^T, dgam = rowsum(D_c * S_c), 64 channels at a time
+    for (int c0 = 0; c0 < dk; c0 += kChunk) {
         __syncthreads();
         for (int e = tid; e < kChunk * dv; e += kSimtThreads) {
-            const int r = e / dv, jj = e % dv;
-            float x = sU[r * LDV + jj], y = sdU[r * LDV + jj];
-#pragma unroll 8
-            for (int cc = 0; cc < kBwdCT; ++cc) {
-                x = fmaf(-sWt[r * kBwdLT + cc], sS[cc * LDV + jj], x);
-                y = fmaf(sKt[r * kBwdLT + cc], sD[cc * LDV + jj], y);
-            }
-            sU[r * LDV + jj] = x;
-            sdU[r * LDV + jj] = y;
-        }
-    }
-    __syncthreads();
-    for (int e = tid; e < kChunk * kChunk; e += kSimtThreads) {  // dP = lower_incl(dO U^T)
-        const int r = e / kChunk, i = e % kChunk;
-        float x = 0.f;
-        if (i <= r)
-            for (int jj = 0; jj < dv; ++jj) x = fmaf(sO[r * LDV + jj], sU[i * LDV + jj], x);
-        oP[e] = x;
-    }
-    for (int e = tid; e < kChunk * dv; e += kSimtThreads) oU[e] = sdU[(e / dv) * LDV + (e % dv)];
-    // dQg = dO S_c^T, dW = -dU S_c^T, dKd = U D_c^T, dgam = rowsum(D_c * S_c), per tile of channels
-    for (int c0 = 0; c0 < dk; c0 += kBwdCT) {
-        __syncthreads();
-        for (int e = tid; e < kBwdCT * dv; e += kSimtThreads) {
             const int cc = e / dv, jj = e % dv;
             sS[cc * LDV + jj] = Sc[(size_t)(c0 + cc) * dv + jj];
             sD[cc * LDV + jj] = Dc[(size_t)(c0 + cc) * dv + jj];
         }
         __syncthreads();
-        for (int e = tid; e < kChunk * kBwdCT; e += kSimtThreads) {
-            const int r = e / kBwdCT, cc = e % kBwdCT;
-            float a = 0.f, b = 0.f, c = 0.f;
-            for (int jj = 0; jj < dv; ++jj) {
-                const float s = sS[cc * LDV + jj];
-                a = fmaf(sO[r * LDV + jj], s, a);
-                b = fmaf(sdU[r * LDV + jj], s, b);
-                c = fmaf(sU[r * LDV + jj], sD[cc * LDV + jj], c);
+        float aq[4][4] = {}, aw[4][4] = {}, ak[4][4] = {};
+#pragma unroll 2
+        for (int jj = 0; jj < dv; ++jj) {
+            float x0[4], x1[4], x2[4], bs[4], bd[4];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                x0[a] = sO[(tr + 16 * a) * LDV + jj];
+                x1[a] = sdU[(tr + 16 * a) * LDV + jj];
+                x2[a] = sU[(tr + 16 * a) * LDV + jj];
+                bs[a] = sS[(tc + 16 * a) * LDV + jj];
+                bd[a] = sD[(tc + 16 * a) * LDV + jj];
             }
-            oQg[(size_t)r * dk + c0 + cc] = a;
-            oW[(size_t)r * dk + c0 + cc] = -b;
-            oKd[(size_t)r * dk + c0 + cc] = c;
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    aq[a][b] = fmaf(x0[a], bs[b], aq[a][b]);
+                    aw[a][b] = fmaf(x1[a], bs[b], aw[a][b]);
+                    ak[a][b] = fmaf(x2[a], bd[b], ak[a][b]);
+                }
         }
-        if (tid < kBwdCT) {
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const size_t oi = (size_t)(tr + 16 * a) * dk + c0 + tc + 16 * b;
+                oQg[oi] = aq[a][b];
+                oW[oi] = -aw[a][b];
+                oKd[oi] = ak[a][b];
+            }
+        if (tid < kChunk) {
             float g = 0.f;
             for (int jj = 0; jj < dv; ++jj) g = fmaf(sD[tid * LDV + jj], sS[tid * LDV + jj], g);
             oGam[c0 + tid] = g;
@@ -255,18 +389,26 @@ bwd_state_side_kernel(const TIn* __restrict__ dout, const WsHeader* __restrict__
 // ------------------------------------------------------------------------------------------------
 // cumulative gate of one 32-channel tile (rows past the chunk's end add nothing), its reference
 // point and whether the factorised form is safe for it
+// (tg must hold no live data: it is filled with the gates, then scanned in place)
 __device__ __forceinline__ void bwd_gate_tile(const void* __restrict__ log_alpha, bool la16, long long t0, int L,
                                               int H, int h, int dk, int c0, float* tg, float* tref, int* s_wide)
 {
     const int tid = threadIdx.x;
+    for (int e = tid; e < kChunk * kBwdCT; e += kSimtThreads) {
+        const int r = e / kBwdCT, cc = e % kBwdCT;
+        float x = 0.f;
+        if (r < L) {
+            const size_t ia = ((size_t)(t0 + r) * H + h) * dk + c0 + cc;
+            x = la16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(log_alpha)[ia])
+                     : reinterpret_cast<const float*>(log_alpha)[ia];
+        }
+        tg[r * kBwdLT + cc] = x;
+    }
+    __syncthreads();
     if (tid < kBwdCT) {
         float acc = 0.f, lo = 0.f, hi = 0.f;
         for (int r = 0; r < kChunk; ++r) {
-            if (r < L) {
-                const size_t ia = ((size_t)(t0 + r) * H + h) * dk + c0 + tid;
-                acc += la16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(log_alpha)[ia])
-                            : reinterpret_cast<const float*>(log_alpha)[ia];
-            }
+            acc += tg[r * kBwdLT + tid];  // rows past the chunk's end hold 0
             tg[r * kBwdLT + tid] = acc;
             lo = fminf(lo, acc);
             hi = fmaxf(hi, acc);
@@ -283,6 +425,14 @@ __device__ __forceinline__ void bwd_load_tile(const TIn* __restrict__ x, long lo
     for (int e = threadIdx.x; e < kChunk * kBwdCT; e += kSimtThreads) {
         const int r = e / kBwdCT, cc = e % kBwdCT;
         t[r * kBwdLT + cc] = (r < L) ? to_f32(x[((size_t)(t0 + r) * H + h) * d + c0 + cc]) : 0.f;
+    }
+}
+
+__device__ __forceinline__ void bwd_load_scr_tile(const float* __restrict__ x, int ld, int c0, float* t)
+{
+    for (int e = threadIdx.x; e < kChunk * kBwdCT; e += kSimtThreads) {
+        const int r = e / kBwdCT, cc = e % kBwdCT;
+        t[r * kBwdLT + cc] = x[(size_t)r * ld + c0 + cc];
     }
 }
 
@@ -304,12 +454,13 @@ bwd_input_side_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, cons
     const bool la16 = (pro & KDA_PROLOGUE_GATE_BF16) != 0;
     constexpr int M64 = kChunk * kBwdL64;
     constexpr int MT = kChunk * kBwdLT;
+    constexpr int L64 = kBwdL64, LT = kBwdLT;
     float* sAt = smem;            // [64][65] At = strict_lower(Kf Kb^T) (without beta)
     float* sN = sAt + M64;        // [64][65] N = (I + Diag(beta) At)^{-1}
     float* sM = sN + M64;         // [64][65] dT -> dN -> dM -> dAt
     float* sY = sM + M64;         // [64][65] dN N^T
     float* sdP = sY + M64;        // [64][65] dP
-    float* tk = sdP + M64;        // tiles [64][33]: k, q, g and four temporaries
+    float* tk = sdP + M64;        // tiles [64][33]: k (or v), q, g and four temporaries
     float* tq = tk + MT;
     float* tg = tq + MT;
     float* tA = tg + MT;
@@ -323,77 +474,68 @@ bwd_input_side_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, cons
 
     const size_t u = (size_t)j * H + h;
     const float* o = scr + u * bwd_scr_floats(dk, dv);
-    const float* gdU = o;
+    const float* gdU = o + (size_t)kChunk * dv;
     const float* gdQg = gdU + (size_t)kChunk * dv;
     const float* gdW = gdQg + (size_t)kChunk * dk;
     const float* gdKd = gdW + (size_t)kChunk * dk;
     const float* gdP = gdKd + (size_t)kChunk * dk;
     const float* gdGam = gdP + (size_t)kChunk * kChunk;
+    const int tr = tid >> 4, tc = tid & 15;
 
-    for (int r = tid; r < kChunk; r += kSimtThreads) {
-        sb[r] = (r < L) ? beta[(size_t)(t0 + r) * H + h] : 0.f;
-        sdb[r] = 0.f;
-    }
-    for (int e = tid; e < kChunk * kChunk; e += kSimtThreads) {
-        const int r = e / kChunk, i = e % kChunk;
-        sAt[r * kBwdL64 + i] = 0.f;
-        sM[r * kBwdL64 + i] = 0.f;
-        sdP[r * kBwdL64 + i] = gdP[e];
-    }
+    for (int r = tid; r < kChunk; r += kSimtThreads) sb[r] = (r < L) ? beta[(size_t)(t0 + r) * H + h] : 0.f;
+    for (int e = tid; e < kChunk * kChunk; e += kSimtThreads) sdP[(e / kChunk) * L64 + (e % kChunk)] = gdP[e];
 
-    // ---- step 4a: At and dT = dW Kt^T, accumulated over channel tiles; dT += dU V^T over value tiles
+    // ---- step 4a: At and dT = dW Kt^T + dU V^T, accumulated in registers over tiles
+    float accA[4][4] = {}, accT[4][4] = {};
     for (int c0 = 0; c0 < dk; c0 += kBwdCT) {
         __syncthreads();
         if (tid == 0) s_wide = 0;
         __syncthreads();
         bwd_load_tile(k, t0, L, H, h, dk, c0, tk);
         bwd_gate_tile(log_alpha, la16, t0, L, H, h, dk, c0, tg, tref, &s_wide);
-        for (int e = tid; e < kChunk * kBwdCT; e += kSimtThreads) {
-            const int r = e / kBwdCT, cc = e % kBwdCT;
-            tD[r * kBwdLT + cc] = gdW[(size_t)r * dk + c0 + cc];
-        }
+        bwd_load_scr_tile(gdW, dk, c0, tD);
         __syncthreads();
         const bool wide = s_wide != 0;
         for (int e = tid; e < kChunk * kBwdCT; e += kSimtThreads) {
             const int r = e / kBwdCT, cc = e % kBwdCT;
-            const float g = tg[r * kBwdLT + cc], x = g - tref[cc], kv = tk[r * kBwdLT + cc];
-            tA[r * kBwdLT + cc] = kv * expf(x);   // Kf
-            tB[r * kBwdLT + cc] = kv * expf(-x);  // Kb
-            tC[r * kBwdLT + cc] = kv * expf(g);   // Kt
+            const float g = tg[r * LT + cc], x = g - tref[cc], kv = tk[r * LT + cc];
+            tA[r * LT + cc] = wide ? 0.f : kv * expf(x);   // Kf
+            tB[r * LT + cc] = wide ? 0.f : kv * expf(-x);  // Kb
+            tC[r * LT + cc] = kv * expf(g);                // Kt
         }
         __syncthreads();
-        for (int e = tid; e < kChunk * kChunk; e += kSimtThreads) {
-            const int r = e / kChunk, i = e % kChunk;
-            if (i > r) continue;
-            float a = 0.f, t = 0.f;
-            if (!wide) {
-                for (int cc = 0; cc < kBwdCT; ++cc) a = fmaf(tA[r * kBwdLT + cc], tB[i * kBwdLT + cc], a);
-            } else {
-                for (int cc = 0; cc < kBwdCT; ++cc)
-                    a = fmaf(tk[r * kBwdLT + cc] * tk[i * kBwdLT + cc],
-                             expf(tg[r * kBwdLT + cc] - tg[i * kBwdLT + cc]), a);
-            }
-            for (int cc = 0; cc < kBwdCT; ++cc) t = fmaf(tD[r * kBwdLT + cc], tC[i * kBwdLT + cc], t);
-            if (i < r) sAt[r * kBwdL64 + i] += a;
-            sM[r * kBwdL64 + i] += t;
+        if (!wide) {
+            mm_acc<4, 4>(accA, tA, LT, 1, tB, 1, LT, kBwdCT, tr, tc);
+        } else {
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    const int r = tr + 16 * a, i = tc + 16 * b;
+                    if (i >= r) continue;
+                    float x = 0.f;
+                    for (int cc = 0; cc < kBwdCT; ++cc)
+                        x = fmaf(tk[r * LT + cc] * tk[i * LT + cc], expf(tg[r * LT + cc] - tg[i * LT + cc]), x);
+                    accA[a][b] += x;
+                }
         }
+        mm_acc<4, 4>(accT, tD, LT, 1, tC, 1, LT, kBwdCT, tr, tc);
     }
     for (int c0 = 0; c0 < dv; c0 += kBwdCT) {
         __syncthreads();
         bwd_load_tile(v, t0, L, H, h, dv, c0, tk);
-        for (int e = tid; e < kChunk * kBwdCT; e += kSimtThreads) {
-            const int r = e / kBwdCT, cc = e % kBwdCT;
-            tD[r * kBwdLT + cc] = gdU[(size_t)r * dv + c0 + cc];
-        }
+        bwd_load_scr_tile(gdU, dv, c0, tD);
         __syncthreads();
-        for (int e = tid; e < kChunk * kChunk; e += kSimtThreads) {
-            const int r = e / kChunk, i = e % kChunk;
-            if (i > r) continue;
-            float t = 0.f;
-            for (int cc = 0; cc < kBwdCT; ++cc) t = fmaf(tD[r * kBwdLT + cc], tk[i * kBwdLT + cc], t);
-            sM[r * kBwdL64 + i] += t;
-        }
+        mm_acc<4, 4>(accT, tD, LT, 1, tk, 1, LT, kBwdCT, tr, tc);
     }
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            const int r = tr + 16 * a, i = tc + 16 * b;
+            sAt[r * L64 + i] = (i < r) ? accA[a][b] : 0.f;
+            sM[r * L64 + i] = (i <= r) ? accT[a][b] : 0.f;
+        }
     __syncthreads();
 
     // ---- step 4b: the UT transform backwards
@@ -401,44 +543,49 @@ bwd_input_side_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, cons
         const int jj = tid;
         for (int r = 0; r < kChunk; ++r) {
             float t = (r == jj) ? 1.f : 0.f;
-            for (int i = jj; i < r; ++i) t = fmaf(-sb[r] * sAt[r * kBwdL64 + i], sN[i * kBwdL64 + jj], t);
-            sN[r * kBwdL64 + jj] = (jj <= r) ? t : 0.f;
+            for (int i = jj; i < r; ++i) t = fmaf(-sb[r] * sAt[r * L64 + i], sN[i * L64 + jj], t);
+            sN[r * L64 + jj] = (jj <= r) ? t : 0.f;
         }
     }
     __syncthreads();
-    if (tid < kChunk) {  // dbeta_i += sum_r dT[r][i] N[r][i]   (T = N Diag(beta))
+    if (tid < kChunk) {  // dbeta_i = sum_r dT[r][i] N[r][i]   (T = N Diag(beta))
         float x = 0.f;
-        for (int r = tid; r < kChunk; ++r) x = fmaf(sM[r * kBwdL64 + tid], sN[r * kBwdL64 + tid], x);
+        for (int r = tid; r < kChunk; ++r) x = fmaf(sM[r * L64 + tid], sN[r * L64 + tid], x);
         sdb[tid] = x;
     }
     __syncthreads();
     for (int e = tid; e < kChunk * kChunk; e += kSimtThreads) {  // dN = dT Diag(beta)
         const int r = e / kChunk, i = e % kChunk;
-        sM[r * kBwdL64 + i] = (i <= r) ? sM[r * kBwdL64 + i] * sb[i] : 0.f;
+        sM[r * L64 + i] *= sb[i];
     }
     __syncthreads();
-    for (int e = tid; e < kChunk * kChunk; e += kSimtThreads) {  // Y = dN N^T
-        const int r = e / kChunk, b = e % kChunk;
-        const int amax = r < b ? r : b;
-        float x = 0.f;
-        for (int a = 0; a <= amax; ++a) x = fmaf(sM[r * kBwdL64 + a], sN[b * kBwdL64 + a], x);
-        sY[r * kBwdL64 + b] = x;
+    {  // Y = dN N^T
+        float acc[4][4] = {};
+        mm_acc<4, 4>(acc, sM, L64, 1, sN, 1, L64, kChunk, tr, tc);
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) sY[(tr + 16 * a) * L64 + tc + 16 * b] = acc[a][b];
     }
     __syncthreads();
-    for (int e = tid; e < kChunk * kChunk; e += kSimtThreads) {  // dM = -N^T Y, strictly lower
-        const int r = e / kChunk, i = e % kChunk;
-        float x = 0.f;
-        if (i < r)
-            for (int a = r; a < kChunk; ++a) x = fmaf(sN[a * kBwdL64 + r], sY[a * kBwdL64 + i], x);
-        sM[r * kBwdL64 + i] = -x;
+    {  // dM = -N^T Y, strictly lower (dN is no longer needed: overwritten in place)
+        float acc[4][4] = {};
+        mm_acc<4, 4>(acc, sN, 1, L64, sY, L64, 1, kChunk, tr, tc);
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const int r = tr + 16 * a, i = tc + 16 * b;
+                sM[r * L64 + i] = (i < r) ? -acc[a][b] : 0.f;
+            }
     }
     __syncthreads();
     if (tid < kChunk) {  // dbeta_r += sum_i dM[r][i] At[r][i];  dAt = Diag(beta) dM
         const int r = tid;
         float x = 0.f;
         for (int i = 0; i < r; ++i) {
-            x = fmaf(sM[r * kBwdL64 + i], sAt[r * kBwdL64 + i], x);
-            sM[r * kBwdL64 + i] *= sb[r];
+            x = fmaf(sM[r * L64 + i], sAt[r * L64 + i], x);
+            sM[r * L64 + i] *= sb[r];
         }
         sdb[r] += x;
     }
@@ -453,92 +600,93 @@ bwd_input_side_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, cons
         bwd_load_tile(k, t0, L, H, h, dk, c0, tk);
         bwd_load_tile(q, t0, L, H, h, dk, c0, tq);
         bwd_gate_tile(log_alpha, la16, t0, L, H, h, dk, c0, tg, tref, &s_wide);
-        for (int e = tid; e < kChunk * kBwdCT; e += kSimtThreads) {
-            const int r = e / kBwdCT, cc = e % kBwdCT;
-            tD[r * kBwdLT + cc] = gdW[(size_t)r * dk + c0 + cc];
-        }
+        bwd_load_scr_tile(gdW, dk, c0, tD);
         __syncthreads();
         const bool wide = s_wide != 0;
         if (!wide)
             for (int e = tid; e < kChunk * kBwdCT; e += kSimtThreads) {
                 const int r = e / kBwdCT, cc = e % kBwdCT;
-                const float x = tg[r * kBwdLT + cc] - tref[cc];
+                const float x = tg[r * LT + cc] - tref[cc];
                 const float ex = expf(x), emx = expf(-x);
-                tA[r * kBwdLT + cc] = tk[r * kBwdLT + cc] * ex;   // Kf
-                tB[r * kBwdLT + cc] = tk[r * kBwdLT + cc] * emx;  // Kb
-                tC[r * kBwdLT + cc] = tq[r * kBwdLT + cc] * ex;   // Qf
+                tA[r * LT + cc] = tk[r * LT + cc] * ex;   // Kf
+                tB[r * LT + cc] = tk[r * LT + cc] * emx;  // Kb
+                tC[r * LT + cc] = tq[r * LT + cc] * ex;   // Qf
             }
         __syncthreads();
-        // per (row, channel): RowP = sum_i dP[r][i] k_i E(r,i), RowA = sum_i dAt[r][i] k_i E(r,i),
-        // Col = sum_r (dP[r][i] q_r + dAt[r][i] k_r) E(r,i), dKt = sum_r T[r][i] dW[r]
-        constexpr int PT = (kChunk * kBwdCT) / kSimtThreads;  // elements per thread
-        float accq[PT], acck[PT], accg[PT], accl[PT];
+        // per (row r, channel): rowP = sum_i dP[r][i] k_i E(r,i), rowA = sum_i dAt[r][i] k_i E(r,i),
+        // col = sum_a (dP[a][r] q_a + dAt[a][r] k_a) E(a,r), dKt = beta_r sum_a N[a][r] dW[a]
+        float rowP[4][2] = {}, rowA[4][2] = {}, col[4][2] = {}, dkt[4][2] = {};
+        if (!wide) {
+            mm_acc<4, 2>(rowP, sdP, L64, 1, tB, LT, 1, kChunk, tr, tc);
+            mm_acc<4, 2>(rowA, sM, L64, 1, tB, LT, 1, kChunk, tr, tc);
+            mm_acc<4, 2>(col, sdP, 1, L64, tC, LT, 1, kChunk, tr, tc);
+            mm_acc<4, 2>(col, sM, 1, L64, tA, LT, 1, kChunk, tr, tc);
+        } else {
 #pragma unroll
-        for (int m = 0; m < PT; ++m) {
-            const int e = tid + m * kSimtThreads;
-            const int r = e / kBwdCT, cc = e % kBwdCT;
-            float rowP = 0.f, rowA = 0.f, col = 0.f, dkt = 0.f;
-            if (!wide) {
-                float sp = 0.f, sa = 0.f;
-                for (int i = 0; i <= r; ++i) {
-                    const float kb = tB[i * kBwdLT + cc];
-                    sp = fmaf(sdP[r * kBwdL64 + i], kb, sp);
-                    sa = fmaf(sM[r * kBwdL64 + i], kb, sa);  // dAt is zero on the diagonal
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int b = 0; b < 2; ++b) {
+                    const int r = tr + 16 * a, cc = tc + 16 * b;
+                    const float gr = tg[r * LT + cc];
+                    for (int i = 0; i <= r; ++i) {
+                        const float ke = tk[i * LT + cc] * expf(gr - tg[i * LT + cc]);
+                        rowP[a][b] = fmaf(sdP[r * L64 + i], ke, rowP[a][b]);
+                        rowA[a][b] = fmaf(sM[r * L64 + i], ke, rowA[a][b]);
+                    }
+                    for (int i = r; i < kChunk; ++i)
+                        col[a][b] = fmaf(fmaf(sdP[i * L64 + r], tq[i * LT + cc], sM[i * L64 + r] * tk[i * LT + cc]),
+                                         expf(tg[i * LT + cc] - gr), col[a][b]);
                 }
-                float sc = 0.f;
-                for (int a = r; a < kChunk; ++a)
-                    sc = fmaf(sdP[a * kBwdL64 + r], tC[a * kBwdLT + cc], fmaf(sM[a * kBwdL64 + r], tA[a * kBwdLT + cc], sc));
-                const float x = tg[r * kBwdLT + cc] - tref[cc];
-                rowP = sp * expf(x);
-                rowA = sa * expf(x);
-                col = sc * expf(-x);
-            } else {
-                const float gr = tg[r * kBwdLT + cc];
-                for (int i = 0; i <= r; ++i) {
-                    const float ke = tk[i * kBwdLT + cc] * expf(gr - tg[i * kBwdLT + cc]);
-                    rowP = fmaf(sdP[r * kBwdL64 + i], ke, rowP);
-                    rowA = fmaf(sM[r * kBwdL64 + i], ke, rowA);
+        }
+        mm_acc<4, 2>(dkt, sN, 1, L64, tD, LT, 1, kChunk, tr, tc);
+        float accg[4][2], accl[4][2];
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+                const int r = tr + 16 * a, cc = tc + 16 * b;
+                const float g = tg[r * LT + cc], gl = tg[(kChunk - 1) * LT + cc];
+                if (!wide) {
+                    const float x = g - tref[cc];
+                    const float ex = expf(x);
+                    rowP[a][b] *= ex;
+                    rowA[a][b] *= ex;
+                    col[a][b] *= expf(-x);
                 }
-                for (int a = r; a < kChunk; ++a) {
-                    const float ea = expf(tg[a * kBwdLT + cc] - gr);
-                    col = fmaf(fmaf(sdP[a * kBwdL64 + r], tq[a * kBwdLT + cc],
-                                    sM[a * kBwdL64 + r] * tk[a * kBwdLT + cc]), ea, col);
+                const float kt = dkt[a][b] * sb[r];
+                const float eg = expf(g), egl = expf(gl - g);
+                const float qv = tq[r * LT + cc], kv = tk[r * LT + cc];
+                const size_t gi = (size_t)r * dk + c0 + cc;
+                const float dQg = gdQg[gi], dKd = gdKd[gi];
+                const float vq = rowP[a][b] + dQg * eg;
+                const float vk = rowA[a][b] + col[a][b] + kt * eg + dKd * egl;
+                accg[a][b] = qv * rowP[a][b] + kv * rowA[a][b] - kv * col[a][b] + (dQg * qv + kt * kv) * eg -
+                             dKd * kv * egl;
+                accl[a][b] = dKd * kv * egl;  // chunk-end term of g_last, summed below
+                if (r < L) {
+                    const size_t oi = ((size_t)(t0 + r) * H + h) * dk + c0 + cc;
+                    dq[oi] = from_f32<TIn>(vq);
+                    dk_out[oi] = from_f32<TIn>(vk);
                 }
             }
-            for (int a = r; a < kChunk; ++a) dkt = fmaf(sN[a * kBwdL64 + r], tD[a * kBwdLT + cc], dkt);
-            dkt *= sb[r];
-            const float g = tg[r * kBwdLT + cc], gl = tg[(kChunk - 1) * kBwdLT + cc];
-            const float eg = expf(g), egl = expf(gl - g);
-            const float qv = tq[r * kBwdLT + cc], kv = tk[r * kBwdLT + cc];
-            const float dQg = gdQg[(size_t)r * dk + c0 + cc], dKd = gdKd[(size_t)r * dk + c0 + cc];
-            accq[m] = rowP + dQg * eg;
-            acck[m] = rowA + col + dkt * eg + dKd * egl;
-            accg[m] = qv * rowP + kv * rowA - kv * col + (dQg * qv + dkt * kv) * eg - dKd * kv * egl;
-            accl[m] = dKd * kv * egl;  // chunk-end term of g_last, summed below
-        }
         __syncthreads();  // every thread is done with Kf / Kb / Qf
 #pragma unroll
-        for (int m = 0; m < PT; ++m) {
-            const int e = tid + m * kSimtThreads;
-            const int r = e / kBwdCT, cc = e % kBwdCT;
-            tA[r * kBwdLT + cc] = accl[m];
-            tB[r * kBwdLT + cc] = accg[m];
-            if (r < L) {
-                const size_t oi = ((size_t)(t0 + r) * H + h) * dk + c0 + cc;
-                dq[oi] = from_f32<TIn>(accq[m]);
-                dk_out[oi] = from_f32<TIn>(acck[m]);
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+                const int r = tr + 16 * a, cc = tc + 16 * b;
+                tA[r * LT + cc] = accl[a][b];
+                tB[r * LT + cc] = accg[a][b];
             }
-        }
         __syncthreads();
         if (tid < kBwdCT) {  // g_last terms, then dlog_alpha = reverse cumulative sum of dg
             const int cc = tid;
             float s = 0.f;
-            for (int r = 0; r < kChunk; ++r) s += tA[r * kBwdLT + cc];
-            const float gl = tg[(kChunk - 1) * kBwdLT + cc];
-            s += gdGam[c0 + cc] * expf(gl);
+            for (int r = 0; r < kChunk; ++r) s += tA[r * LT + cc];
+            s += gdGam[c0 + cc] * expf(tg[(kChunk - 1) * LT + cc]);
             float acc = s;
             for (int r = kChunk - 1; r >= 0; --r) {
-                acc += tB[r * kBwdLT + cc];
+                acc += tB[r * LT + cc];
                 if (r < L) dla[((size_t)(t0 + r) * H + h) * dk + c0 + cc] = acc;
             }
         }
@@ -547,35 +695,65 @@ bwd_input_side_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, cons
     // ---- step 4d: dV = T^T dU = Diag(beta) N^T dU
     for (int c0 = 0; c0 < dv; c0 += kBwdCT) {
         __syncthreads();
-        for (int e = tid; e < kChunk * kBwdCT; e += kSimtThreads) {
-            const int r = e / kBwdCT, cc = e % kBwdCT;
-            tD[r * kBwdLT + cc] = gdU[(size_t)r * dv + c0 + cc];
-        }
+        bwd_load_scr_tile(gdU, dv, c0, tD);
         __syncthreads();
-        for (int e = tid; e < kChunk * kBwdCT; e += kSimtThreads) {
-            const int i = e / kBwdCT, cc = e % kBwdCT;
-            if (i >= L) continue;
-            float x = 0.f;
-            for (int a = i; a < kChunk; ++a) x = fmaf(sN[a * kBwdL64 + i], tD[a * kBwdLT + cc], x);
-            dv_out[((size_t)(t0 + i) * H + h) * dv + c0 + cc] = from_f32<TIn>(sb[i] * x);
-        }
+        float acc[4][2] = {};
+        mm_acc<4, 2>(acc, sN, 1, L64, tD, LT, 1, kChunk, tr, tc);
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+                const int i = tr + 16 * a, cc = tc + 16 * b;
+                if (i < L) dv_out[((size_t)(t0 + i) * H + h) * dv + c0 + cc] = from_f32<TIn>(sb[i] * acc[a][b]);
+            }
     }
 }
 
-inline size_t bwd_dstate_smem(int dk, int dv) { return simt_inter_smem(dk, dv); }
+inline size_t bwd_fwd_chain_smem(int dk, int dv)
+{
+    (void)dv;
+    return sizeof(float) * ((size_t)dk * kSimtNV + 2 * kChunk * dk + 2 * kChunk * kSimtNV + dk);
+}
+inline size_t bwd_dstate_smem(int dk, int dv)
+{
+    (void)dv;
+    return sizeof(float) * ((size_t)dk * kSimtNV + 3 * kChunk * dk + kChunk * kChunk + 2 * kChunk * kSimtNV + dk);
+}
 inline size_t bwd_state_side_smem(int dk, int dv)
 {
     (void)dk;
-    return sizeof(float) * ((size_t)3 * kChunk * (dv + 1) + kChunk * kChunk + 2 * kBwdCT * (dv + 1) +
-                            2 * kChunk * kBwdLT);
+    return sizeof(float) * (size_t)5 * kChunk * (dv + 1);
 }
 inline size_t bwd_input_side_smem()
 {
     return sizeof(float) * ((size_t)5 * kChunk * kBwdL64 + 7 * kChunk * kBwdLT + 2 * kChunk + kBwdCT);
 }
 
+template <typename TIn, int DK>
+cudaError_t launch_bwd_chains(const float* S0, const void* dout, const float* dS_final, float* dS0,
+                              const WsHeader* hdr, const int* off, const int32_t* cu, int Tseq, int N, int H, int dv,
+                              const float* slots, float* S_chunks, float* dSn_chunks, float* scr, cudaStream_t stream)
+{
+    const size_t smF = bwd_fwd_chain_smem(DK, dv), smD = bwd_dstate_smem(DK, dv);
+    cudaError_t e = cudaFuncSetAttribute(bwd_fwd_chain_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smF);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(bwd_dstate_kernel<TIn, DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smD);
+    if (e != cudaSuccess) return e;
+    const dim3 grid(N, H, dv / kSimtNV);
+    {
+        LaunchScope ls("bwd_fwd_states", stream);
+        bwd_fwd_chain_kernel<DK><<<grid, kSimtThreads, smF, stream>>>(S0, hdr, off, cu, Tseq, N, H, dv, slots,
+                                                                      S_chunks, scr);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    LaunchScope ls("bwd_dstate", stream);
+    bwd_dstate_kernel<TIn, DK><<<grid, kSimtThreads, smD, stream>>>((const TIn*)dout, dS_final, dS0, hdr, off, cu,
+                                                                   Tseq, N, H, dv, slots, dSn_chunks, scr);
+    return cudaGetLastError();
+}
+
 // Steps 1-4.  Workspace regions (all per (chunk, head) of the forward's chunk table): the
-// CUDA-core forward slots, chunk start states, chunk end cotangents and the step-3 scratch.
+// CUDA-core forward slots, chunk start states, chunk end cotangents and the per-chunk scratch.
 template <typename TIn>
 cudaError_t launch_simt_backward(const void* q, const void* k, const void* v, const void* la, const float* beta,
                                  const float* S0, const void* dout, const float* dS_final, void* dq, void* dk_out,
@@ -584,13 +762,8 @@ cudaError_t launch_simt_backward(const void* q, const void* k, const void* v, co
                                  int dv, int max_chunks, float* slots, float* S_chunks, float* dSn_chunks, float* scr,
                                  cudaStream_t stream)
 {
-    const size_t smA = simt_intra_smem(dk, dv), smB = simt_inter_smem(dk, dv), smD = bwd_dstate_smem(dk, dv),
-                 smS = bwd_state_side_smem(dk, dv), smI = bwd_input_side_smem();
+    const size_t smA = simt_intra_smem(dk, dv), smS = bwd_state_side_smem(dk, dv), smI = bwd_input_side_smem();
     cudaError_t e = cudaFuncSetAttribute(simt_intra_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smA);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(simt_inter_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smB);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(bwd_dstate_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smD);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(bwd_state_side_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smS);
     if (e == cudaSuccess)
@@ -603,23 +776,16 @@ cudaError_t launch_simt_backward(const void* q, const void* k, const void* v, co
             qq, kk, vv, la, beta, hdr, off, cu, Tseq, N, H, H, pro & KDA_PROLOGUE_GATE_BF16, dk, dv, slots);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    {
-        LaunchScope ls("bwd_fwd_states", stream);
-        simt_inter_kernel<TIn><<<dim3(N, H, dv / kSimtNV), kSimtThreads, smB, stream>>>(
-            S0, nullptr, (TIn*)nullptr, hdr, off, cu, Tseq, N, H, dk, dv, slots, S_chunks);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    }
-    {
-        LaunchScope ls("bwd_dstate", stream);
-        bwd_dstate_kernel<TIn><<<dim3(N, H, dv / kSimtNV), kSimtThreads, smD, stream>>>(
-            (const TIn*)dout, dS_final, dS0, hdr, off, cu, Tseq, N, H, dk, dv, slots, dSn_chunks);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    }
+    e = (dk == 128) ? launch_bwd_chains<TIn, 128>(S0, dout, dS_final, dS0, hdr, off, cu, Tseq, N, H, dv, slots,
+                                                  S_chunks, dSn_chunks, scr, stream)
+                    : launch_bwd_chains<TIn, 64>(S0, dout, dS_final, dS0, hdr, off, cu, Tseq, N, H, dv, slots,
+                                                 S_chunks, dSn_chunks, scr, stream);
+    if (e != cudaSuccess) return e;
     if (max_chunks > 0) {
         {
             LaunchScope ls("bwd_state_side", stream);
             bwd_state_side_kernel<TIn><<<dim3(max_chunks, H), kSimtThreads, smS, stream>>>(
-                (const TIn*)dout, hdr, off, cu, Tseq, N, H, dk, dv, slots, S_chunks, dSn_chunks, scr);
+                (const TIn*)dout, hdr, off, cu, Tseq, N, H, dk, dv, S_chunks, dSn_chunks, scr);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
         }
         LaunchScope ls("bwd_input_side", stream);

@@ -39,6 +39,41 @@ __host__ __device__ inline size_t simt_slot_floats(int dk, int dv)
 // below stay finite in fp32: each factor is e^{+-x} with |x| <= kFactorSpread / 2 <= 80.
 constexpr float kFactorSpread = 160.f;
 
+// acc[i][j] += sum_k A(tr + 16 i, k) B(k, tc + 16 j), with A(r, k) = A[r * ars + k * aks] and
+// B(k, c) = B[k * bks + c * bcs] in shared memory (thread tid: tr = tid / 16, tc = tid % 16).  Each
+// thread owns a TM x TN block of interleaved rows and columns, so the B reads of a warp fall on
+// distinct banks whenever bcs = 1 or bcs is odd, and its A reads on two addresses.
+template <int TM, int TN>
+__device__ __forceinline__ void mm_acc(float (&acc)[TM][TN], const float* A, int ars, int aks, const float* B,
+                                       int bks, int bcs, int K, int tr, int tc)
+{
+#pragma unroll 4
+    for (int k = 0; k < K; ++k) {
+        float a[TM], b[TN];
+#pragma unroll
+        for (int i = 0; i < TM; ++i) a[i] = A[(tr + 16 * i) * ars + k * aks];
+#pragma unroll
+        for (int j = 0; j < TN; ++j) b[j] = B[k * bks + (tc + 16 * j) * bcs];
+#pragma unroll
+        for (int i = 0; i < TM; ++i)
+#pragma unroll
+            for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+}
+
+// out[r][c] = sum_{i} T[r][i] X[i][c] for the 64 x D block (T in [64][65], X in [64][D+1]), written
+// to a dense global [64][D] array
+template <int D>
+__device__ __forceinline__ void simt_apply_t(const float* sT, const float* X, float* __restrict__ out, int tr, int tc)
+{
+    float acc[4][D / 16] = {};
+    mm_acc<4, D / 16>(acc, sT, kChunk + 1, 1, X, D + 1, 1, kChunk, tr, tc);
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < D / 16; ++b) out[(size_t)(tr + 16 * a) * D + tc + 16 * b] = acc[a][b];
+}
+
 template <typename TIn>
 __global__ void __launch_bounds__(kSimtThreads)
 simt_intra_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
@@ -53,17 +88,21 @@ simt_intra_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TI
     long long t0;
     locate_chunk(j, off, cu, Tseq, N, n, t0, L);
 
-    float* sk = smem;                       // [64][dk]  k, later k e^{g - ref}
-    float* sq = sk + kChunk * dk;           // [64][dk]  q, later q e^{g - ref}
-    float* sg = sq + kChunk * dk;           // [64][dk]  g, later k e^{ref - g}
-    float* sv = sg + kChunk * dk;           // [64][dv]
-    float* sKt = sv + kChunk * dv;          // [64][dk]  k e^{g}
-    float* sA = sKt + kChunk * dk;          // [64][64]
-    float* sP = sA + kChunk * kChunk;       // [64][64]
-    float* sT = sP + kChunk * kChunk;       // [64][64]
-    float* sb = sT + kChunk * kChunk;       // [64]
+    // row strides padded by one float, so column walks of a warp hit distinct banks
+    const int LK = dk + 1, LV = dv + 1;
+    constexpr int L64 = kChunk + 1;
+    float* sk = smem;                       // [64][dk+1]  k, later k e^{g - ref}
+    float* sq = sk + kChunk * LK;           // [64][dk+1]  q, later q e^{g - ref}
+    float* sg = sq + kChunk * LK;           // [64][dk+1]  g, later k e^{ref - g}
+    float* sv = sg + kChunk * LK;           // [64][dv+1]
+    float* sKt = sv + kChunk * LV;          // [64][dk+1]  k e^{g}
+    float* sA = sKt + kChunk * LK;          // [64][65]
+    float* sP = sA + kChunk * L64;          // [64][65]
+    float* sT = sP + kChunk * L64;          // [64][65]
+    float* sb = sT + kChunk * L64;          // [64]
     float* sref = sb + kChunk;              // [dk]
     __shared__ int s_wide;
+    const int tr = tid >> 4, tc = tid & 15;
 
     if (tid == 0) s_wide = 0;
     for (int e = tid; e < kChunk * dk; e += kSimtThreads) {
@@ -77,11 +116,11 @@ simt_intra_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TI
                                                 : reinterpret_cast<const float*>(log_alpha)[gi];
             if (pro & KDA_PROLOGUE_GATE_LOGITS) lv = log_sigmoid_f(lv);  // rows past the end stay 0 (identity)
         }
-        sk[e] = kv; sq[e] = qv; sg[e] = lv;
+        sk[r * LK + c] = kv; sq[r * LK + c] = qv; sg[r * LK + c] = lv;
     }
     for (int e = tid; e < kChunk * dv; e += kSimtThreads) {
         const int r = e / dv, c = e % dv;
-        sv[e] = (r < L) ? to_f32(v[((size_t)(t0 + r) * H + h) * dv + c]) : 0.f;
+        sv[r * LV + c] = (r < L) ? to_f32(v[((size_t)(t0 + r) * H + h) * dv + c]) : 0.f;
     }
     for (int r = tid; r < kChunk; r += kSimtThreads) {
         float b = 0.f;
@@ -94,10 +133,10 @@ simt_intra_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TI
     __syncthreads();
     if (pro & KDA_PROLOGUE_L2NORM_QK) {  // rows of k (i < 64) and q (i >= 64), normalised at the input precision
         for (int i = tid; i < 2 * kChunk; i += kSimtThreads) {
-            float* row = (i < kChunk ? sk : sq) + (i & (kChunk - 1)) * dk;
+            float* row = (i < kChunk ? sk : sq) + (i & (kChunk - 1)) * LK;
             float ss = 0.f;
             for (int c0 = 0; c0 < dk; ++c0) {
-                const float x = row[(c0 + i) & (dk - 1)];  // rotated start: no bank conflicts
+                const float x = row[(c0 + i) & (dk - 1)];  // rotated start: fewer bank conflicts
                 ss = fmaf(x, x, ss);
             }
             const float inv = rsqrtf(ss + kQkNormEps);
@@ -113,8 +152,8 @@ simt_intra_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TI
     for (int c = tid; c < dk; c += kSimtThreads) {
         float acc = 0.f, lo = 0.f, hi = 0.f;
         for (int r = 0; r < kChunk; ++r) {
-            acc += sg[r * dk + c];
-            sg[r * dk + c] = acc;
+            acc += sg[r * LK + c];
+            sg[r * LK + c] = acc;
             lo = fminf(lo, acc);
             hi = fmaxf(hi, acc);
         }
@@ -134,12 +173,12 @@ simt_intra_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TI
 
     // gated operands that never overflow (every exponent <= 0)
     for (int e = tid; e < kChunk * dk; e += kSimtThreads) {
-        const int r = e / dk, c = e % dk;
-        const float gl = sg[(kChunk - 1) * dk + c];
-        const float eg = expf(sg[e]);
-        gQ[e] = sq[e] * eg;
-        gKd[e] = sk[e] * expf(gl - sg[e]);
-        sKt[e] = sk[e] * eg;
+        const int r = e / dk, c = e % dk, x = r * LK + c;
+        const float gl = sg[(kChunk - 1) * LK + c];
+        const float eg = expf(sg[x]);
+        gQ[e] = sq[x] * eg;
+        gKd[e] = sk[x] * expf(gl - sg[x]);
+        sKt[x] = sk[x] * eg;
         if (r == 0) gGam[c] = expf(gl);
     }
     __syncthreads();
@@ -148,27 +187,41 @@ simt_intra_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TI
     if (!wide) {
         // factorised form: e^{g_r - g_i} = e^{g_r - ref} e^{ref - g_i}, both factors within e^{+-80}
         for (int e = tid; e < kChunk * dk; e += kSimtThreads) {
-            const int c = e % dk;
-            const float x = sg[e] - sref[c];
-            const float kv = sk[e];
-            sk[e] = kv * expf(x);
-            sq[e] = sq[e] * expf(x);
-            sg[e] = kv * expf(-x);
+            const int r = e / dk, c = e % dk, x0 = r * LK + c;
+            const float x = sg[x0] - sref[c];
+            const float kv = sk[x0];
+            sk[x0] = kv * expf(x);
+            sq[x0] = sq[x0] * expf(x);
+            sg[x0] = kv * expf(-x);
         }
         __syncthreads();
-        for (int e = tid; e < kChunk * kChunk; e += kSimtThreads) {
-            const int r = e / kChunk, i = e % kChunk;
-            float a = 0.f, p = 0.f;
-            if (i <= r) {
-                for (int c = 0; c < dk; ++c) {
-                    const float kb = sg[i * dk + c];
-                    a = fmaf(sk[r * dk + c], kb, a);
-                    p = fmaf(sq[r * dk + c], kb, p);
-                }
+        // A = Kf Kb^T and P = Qf Kb^T, register-tiled (4 x 4 per thread, shared Kb reads)
+        float a_[4][4] = {}, p_[4][4] = {};
+#pragma unroll 2
+        for (int c = 0; c < dk; ++c) {
+            float kf[4], qf[4], kb[4];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                kf[a] = sk[(tr + 16 * a) * LK + c];
+                qf[a] = sq[(tr + 16 * a) * LK + c];
+                kb[a] = sg[(tc + 16 * a) * LK + c];
             }
-            sA[e] = (i < r) ? sb[r] * a : 0.f;
-            sP[e] = p;
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    a_[a][b] = fmaf(kf[a], kb[b], a_[a][b]);
+                    p_[a][b] = fmaf(qf[a], kb[b], p_[a][b]);
+                }
         }
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const int r = tr + 16 * a, i = tc + 16 * b;
+                sA[r * L64 + i] = (i < r) ? sb[r] * a_[a][b] : 0.f;
+                sP[r * L64 + i] = (i <= r) ? p_[a][b] : 0.f;
+            }
     } else {
         // some channel decays by more than e^-160 inside the chunk: exact per-element factors
         for (int e = tid; e < kChunk * kChunk; e += kSimtThreads) {
@@ -176,13 +229,13 @@ simt_intra_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TI
             float a = 0.f, p = 0.f;
             if (i <= r) {
                 for (int c = 0; c < dk; ++c) {
-                    const float kk = sk[i * dk + c] * expf(sg[r * dk + c] - sg[i * dk + c]);
-                    a = fmaf(sk[r * dk + c], kk, a);
-                    p = fmaf(sq[r * dk + c], kk, p);
+                    const float kk = sk[i * LK + c] * expf(sg[r * LK + c] - sg[i * LK + c]);
+                    a = fmaf(sk[r * LK + c], kk, a);
+                    p = fmaf(sq[r * LK + c], kk, p);
                 }
             }
-            sA[e] = (i < r) ? sb[r] * a : 0.f;
-            sP[e] = p;
+            sA[r * L64 + i] = (i < r) ? sb[r] * a : 0.f;
+            sP[r * L64 + i] = p;
         }
     }
     __syncthreads();
@@ -192,32 +245,25 @@ simt_intra_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TI
         const int jj = tid;
         for (int r = 0; r < kChunk; ++r) {
             float t = (r == jj) ? sb[r] : 0.f;
-            for (int i = jj; i < r; ++i) t = fmaf(-sA[r * kChunk + i], sT[i * kChunk + jj], t);
-            sT[r * kChunk + jj] = (jj <= r) ? t : 0.f;
+            for (int i = jj; i < r; ++i) t = fmaf(-sA[r * L64 + i], sT[i * L64 + jj], t);
+            sT[r * L64 + jj] = (jj <= r) ? t : 0.f;
         }
     }
-    for (int e = tid; e < kChunk * kChunk; e += kSimtThreads) gP[e] = sP[e];
+    for (int e = tid; e < kChunk * kChunk; e += kSimtThreads) gP[e] = sP[(e / kChunk) * L64 + (e % kChunk)];
     __syncthreads();
 
-    for (int e = tid; e < kChunk * dk; e += kSimtThreads) {
-        const int r = e / dk, c = e % dk;
-        float acc = 0.f;
-        for (int i = 0; i <= r; ++i) acc = fmaf(sT[r * kChunk + i], sKt[i * dk + c], acc);
-        gW[e] = acc;
-    }
-    for (int e = tid; e < kChunk * dv; e += kSimtThreads) {
-        const int r = e / dv, c = e % dv;
-        float acc = 0.f;
-        for (int i = 0; i <= r; ++i) acc = fmaf(sT[r * kChunk + i], sv[i * dv + c], acc);
-        gUv[e] = acc;
-    }
+    // W = T Kt, Uv = T V (T is lower triangular with zeros above the diagonal)
+    if (dk == 128) simt_apply_t<128>(sT, sKt, gW, tr, tc);
+    else simt_apply_t<64>(sT, sKt, gW, tr, tc);
+    if (dv == 128) simt_apply_t<128>(sT, sv, gUv, tr, tc);
+    else simt_apply_t<64>(sT, sv, gUv, tr, tc);
 }
 
 template <typename TOut>
 __global__ void __launch_bounds__(kSimtThreads)
 simt_inter_kernel(const float* S0, float* S_final, TOut* __restrict__ out, const WsHeader* __restrict__ hdr,
                   const int* __restrict__ off, const int32_t* __restrict__ cu, int Tseq, int N, int H, int dk, int dv,
-                  const float* __restrict__ slots, float* __restrict__ S_chunks)
+                  const float* __restrict__ slots)
 {
     extern __shared__ __align__(16) float smem[];
     const int n = blockIdx.x, h = blockIdx.y, v0 = blockIdx.z * kSimtNV, tid = threadIdx.x;
@@ -251,10 +297,6 @@ simt_inter_kernel(const float* S0, float* S_final, TOut* __restrict__ out, const
         const float* gUv = gP + (size_t)kChunk * kChunk;
         const float* gGam = gUv + (size_t)kChunk * dv;
         __syncthreads();  // previous chunk finished with the staged operands
-        if (S_chunks) {  // the chunk's start state, kept for the backward pass
-            float* dst = S_chunks + ((size_t)j * H + h) * dk * dv + v0;
-            for (int e = tid; e < dk * NV; e += kSimtThreads) dst[(size_t)(e / NV) * dv + (e % NV)] = sS[e];
-        }
         for (int e = tid; e < kChunk * dk; e += kSimtThreads) { sW[e] = gW[e]; sQ[e] = gQ[e]; sKd[e] = gKd[e]; }
         for (int e = tid; e < kChunk * kChunk; e += kSimtThreads) sP[e] = gP[e];
         for (int e = tid; e < kChunk * NV; e += kSimtThreads) sUv[e] = gUv[(e / NV) * dv + v0 + (e % NV)];
@@ -269,7 +311,7 @@ simt_inter_kernel(const float* S0, float* S_final, TOut* __restrict__ out, const
         __syncthreads();
         for (int e = tid; e < kChunk * NV; e += kSimtThreads) {
             const int r = e / NV, jj = e % NV;
-            if (r >= L || out == nullptr) continue;
+            if (r >= L) continue;
             float o = 0.f;
             for (int c = 0; c < dk; ++c) o = fmaf(sQ[r * dk + c], sS[c * NV + jj], o);
             for (int i = 0; i <= r; ++i) o = fmaf(sP[r * kChunk + i], sU[i * NV + jj], o);
@@ -293,7 +335,7 @@ simt_inter_kernel(const float* S0, float* S_final, TOut* __restrict__ out, const
 
 inline size_t simt_intra_smem(int dk, int dv)
 {
-    return sizeof(float) * ((size_t)kChunk * (4 * dk + dv) + 3 * kChunk * kChunk + kChunk + dk);
+    return sizeof(float) * ((size_t)kChunk * (4 * (dk + 1) + dv + 1) + 3 * kChunk * (kChunk + 1) + kChunk + dk);
 }
 inline size_t simt_inter_smem(int dk, int dv)
 {
@@ -321,7 +363,7 @@ cudaError_t launch_simt_prefill(const void* q, const void* k, const void* v, con
     }
     LaunchScope ls("simt_inter", stream);
     simt_inter_kernel<TIn><<<dim3(N, H, dv / kSimtNV), kSimtThreads, smB, stream>>>(
-        S0, S_final, (TIn*)out, hdr, off, cu, Tseq, N, H, dk, dv, slots, nullptr);
+        S0, S_final, (TIn*)out, hdr, off, cu, Tseq, N, H, dk, dv, slots);
     return cudaGetLastError();
 }
 

@@ -44,7 +44,7 @@ def parse():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target duration of the oracle sample")
-    ap.add_argument("--only", choices=["prefill", "decode"], default=None,
+    ap.add_argument("--only", choices=["prefill", "decode", "backward", "gated_norm"], default=None,
                     help="run one part only (for profiling): no JSON contract line, prints that part's numbers")
     ap.add_argument("--decode-steps", type=int, default=None, help="decode steps to time (default 512)")
     ap.add_argument("--no-extra", action="store_true", help="skip the varlen and 1M-token workloads")
@@ -244,9 +244,16 @@ def run_ours(args):
     w = synth.WORKLOADS[args.workload]
     if w.kind != "prefill":
         raise SystemExit("the headline workload is a prefill workload; decode is reported under 'decode'")
-    if args.only == "decode":
+    if args.only in ("decode", "backward", "gated_norm"):
         stream = torch.cuda.current_stream(dev)
-        d = bench_decode(torch, kda, synth, dev, stream, world, rank, hbm, peak_kind, steps=args.decode_steps)
+        if args.only == "decode":
+            d = bench_decode(torch, kda, synth, dev, stream, world, rank, hbm, peak_kind, steps=args.decode_steps)
+        elif args.only == "backward":
+            d = bench_backward(torch, kda, synth, dev, stream, world, rank, hbm, peak_kind, steps=args.steps,
+                               warmup=args.warmup, tokens=args.tokens)
+        else:
+            rows = (args.tokens or w.T) * w.B * w.H
+            d = bench_gated_norm(torch, kda, dev, stream, world, hbm, peak_kind, rows=rows, d=w.dv, iters=args.steps)
         if rank == 0:
             print(json.dumps(d), flush=True)
         return
@@ -383,6 +390,12 @@ def run_ours(args):
         torch.cuda.empty_cache()
         gnorm = bench_gated_norm(torch, kda, dev, stream, world, hbm, peak_kind, rows=B * T * H, d=dv)
 
+    backward = None
+    if not args.no_extra and args.only is None:
+        torch.cuda.empty_cache()
+        backward = bench_backward(torch, kda, synth, dev, stream, world, rank, hbm, peak_kind)
+        torch.cuda.empty_cache()
+
     decode = None
     if not args.no_decode and args.only is None:
         decode = bench_decode(torch, kda, synth, dev, stream, world, rank, hbm, peak_kind, steps=args.decode_steps)
@@ -400,7 +413,7 @@ def run_ours(args):
                        "chunk": 64, "parallelism": f"replicas x{world} (independent problems, no collective)",
                        "l2": f"inputs {in_bytes / 1e9:.2f} GB per step > L2 {L2_BYTES / 1e6:.0f} MB (no flush)"},
             "roofline": roofline, "kernels": {k_: {"launches": n, "ms": t} for k_, (n, t) in prof.items()},
-            "other_workloads": extra, "gated_rmsnorm": gnorm,
+            "other_workloads": extra, "gated_rmsnorm": gnorm, "backward": backward,
             "gpu_launches": launches, "clocks": clk, "e2e": e2e, "decode": decode, "cpu_baseline": cpu}
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -491,6 +504,54 @@ def bench_gated_norm(torch, kda, dev, stream, world, hbm, peak_kind, rows, d, it
                         "frac": ach / hbm, "peak_source": f"{peak_kind} hbm_gbs (of {peak_kind})",
                         "alg_bytes_per_launch": nbytes}}
     del o, z, y
+    return res
+
+
+BWD_BYTES_PER_TOKEN_HEAD = 2824  # read q, k, v, dO (bf16), log_alpha, beta; write dq, dk, dv, dlog_alpha, dbeta
+
+
+def bench_backward(torch, kda, synth, dev, stream, world, rank, hbm, peak_kind, steps=3, warmup=2, tokens=None):
+    """kda_chunk_bwd on the 32K-token prefill workload (the training backward of the same call):
+    random bf16 cotangent of the output, none on the final state.  Device-timed like the headline;
+    the roofline is against the algorithmic bytes of the inputs, cotangent and gradients."""
+    w = synth.WORKLOADS["prefill_32k"]
+    inp = synth.prefill_inputs(w, device=dev, seed=replica_seed(w.seed, rank), T=tokens)
+    g = torch.Generator(device=dev).manual_seed(replica_seed(77, rank))
+    do = torch.randn(inp["v"].shape, generator=g, device=dev).to(inp["v"].dtype)
+    q, k, v, la, beta, S0 = (inp[x] for x in ("q", "k", "v", "log_alpha", "beta", "S0"))
+    grads = None
+
+    def step():
+        nonlocal grads
+        grads = kda.chunk_bwd(q, k, v, la, beta, do, S0=S0, grads=grads)
+
+    for _ in range(warmup):
+        step()
+    kda.check()
+    barrier(torch, world)
+    torch.cuda.synchronize(dev)
+    kda.profile_begin()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    prof = kda.profile_end()
+    kda.check()
+    ms = max_over_ranks(torch, world, e0.elapsed_time(e1))
+    tokens = q.shape[0] * q.shape[1]
+    nbytes = BWD_BYTES_PER_TOKEN_HEAD * tokens * w.H
+    ach = nbytes / (ms / steps * 1e-3) / 1e9
+    res = {"desc": f"{w.desc}; backward (kda_chunk_bwd), bf16 dO, fp32 CUDA-core kernels",
+           "tokens": tokens, "steps": steps, "ms_per_step": ms / steps,
+           "value": job_throughput(world, tokens, steps, ms), "unit": "tokens/s",
+           "kernels": {k_: {"launches": n, "ms": t} for k_, (n, t) in prof.items()},
+           "roofline": {"bound": "hbm", "kernel": "whole backward", "achieved": ach, "peak": hbm, "unit": "GB/s",
+                        "frac": ach / hbm, "peak_source": f"{peak_kind} hbm_gbs (of {peak_kind})",
+                        "alg_bytes_per_token_head": BWD_BYTES_PER_TOKEN_HEAD, "alg_bytes_per_step": nbytes}}
+    del inp, q, k, v, la, beta, S0, do, grads
     return res
 
 

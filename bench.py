@@ -330,20 +330,17 @@ def run_ours(args):
         hS0 = S0.cpu().pin_memory() if S0 is not None else None
         hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
         hS = torch.empty(S_fin.shape, dtype=torch.float32).pin_memory()
-        dq, dk_, dv_, dla, db = (torch.empty_like(x) for x in (q, k, v, la, beta))
-        dS0 = torch.empty_like(S0) if S0 is not None else None
         h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hla, hb)) + \
             (hS0.numel() * 4 if hS0 is not None else 0)
         d2h = hout.numel() * hout.element_size() + hS.numel() * 4
+        if cu is not None:
+            raise RuntimeError("the host-pipelined entry point takes regular batches")
 
         def e2e_step():
-            for d_, h_ in ((dq, hq), (dk_, hk), (dv_, hv), (dla, hla), (db, hb)):
-                d_.copy_(h_, non_blocking=True)
-            if dS0 is not None:
-                dS0.copy_(hS0, non_blocking=True)
-            kda.chunk_fwd(dq, dk_, dv_, dla, db, S0=dS0, cu_seqlens=cu, out=out, S_final=S_fin)
-            hout.copy_(out, non_blocking=True)
-            hS.copy_(S_fin, non_blocking=True)
+            # the public host entry point: segments copied in, computed and copied out on
+            # overlapping streams (kda_chunk_fwd_host), joined into `stream`
+            kda.chunk_fwd_host(hq, hk, hv, hla, hb, S0=hS0, out=hout, S_final=hS, segment_tokens=E2E_SEGMENT,
+                               stream=stream, synchronize=False)
 
         for _ in range(2):
             e2e_step()
@@ -358,8 +355,8 @@ def run_ours(args):
         ms_e2e = max_over_ranks(torch, world, e0.elapsed_time(e1))
         e2e = {"value": world * tokens * n_e2e / (ms_e2e / 1e3), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e / n_e2e,
-               "steps": n_e2e}
-        del hq, hk, hv, hla, hb, dq, dk_, dv_, dla, db
+               "steps": n_e2e, "api": f"kda_chunk_fwd_host, {E2E_SEGMENT}-token segments, pinned host buffers"}
+        del hq, hk, hv, hla, hb
     except Exception as ex:  # pragma: no cover
         e2e = {"value": None, "unit": "tokens/s", "error": str(ex)[:200]}
 
@@ -507,6 +504,7 @@ def bench_gated_norm(torch, kda, dev, stream, world, hbm, peak_kind, rows, d, it
     return res
 
 
+E2E_SEGMENT = 4096  # tokens per pipelined segment of the host entry point
 BWD_BYTES_PER_TOKEN_HEAD = 2824  # read q, k, v, dO (bf16), log_alpha, beta; write dq, dk, dv, dlog_alpha, dbeta
 
 

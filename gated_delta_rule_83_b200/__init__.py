@@ -3,14 +3,15 @@
 Public API (a thin binding of the C ABI in include/kda.h):
 
     out, S_final = chunk_fwd(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None)
+    out, S_final = chunk_fwd_host(q, k, v, log_alpha, beta)  # host tensors, pipelined copies
     grads = chunk_bwd(q, k, v, log_alpha, beta, dout, S0=None, dS_final=None)   # training backward
     out = decode_step(q, k, v, log_alpha, beta, S)        # S updated in place
     check()                                               # raise on a device-side error
 """
 from .kda import (PROLOGUE_BETA_LOGITS, PROLOGUE_GATE_BF16, PROLOGUE_GATE_LOGITS, PROLOGUE_L2NORM_QK,  # noqa: F401
                   KdaError,
-                  bwd_workspace_size, check, chunk_bwd, chunk_fwd, decode_step, gated_rmsnorm, load_library,
+                  bwd_workspace_size, check, chunk_bwd, chunk_fwd, chunk_fwd_host, decode_step, gated_rmsnorm, load_library,
                   profile_begin, profile_end, version, workspace_size)
 
-__all__ = ["chunk_fwd", "chunk_bwd", "decode_step", "gated_rmsnorm", "check", "workspace_size",
+__all__ = ["chunk_fwd", "chunk_fwd_host", "chunk_bwd", "decode_step", "gated_rmsnorm", "check", "workspace_size",
            "bwd_workspace_size", "load_library", "version", "KdaError"]

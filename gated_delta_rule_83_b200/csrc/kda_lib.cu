@@ -437,3 +437,156 @@ extern "C" kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const 
     return kda_chunk_fwd(q, k, v, log_alpha, beta, S0, cu_seqlens, num_seqs, out, S_final, B, T, H, dk, dv, dt,
                          scratch, (size_t)KDA_NOALLOC_SCRATCH_BYTES, stream);
 }
+
+// ------------------------------------------------------------------------------------------------
+// Host-resident inputs: segments of the token axis stream in on one copy stream, run on the
+// caller's stream and stream out on another, double-buffered, with the state carried on the device.
+// ------------------------------------------------------------------------------------------------
+namespace {
+
+struct HostPlan {
+    int nseg, seg;
+    size_t in_bytes[5];  // q, k, v, log_alpha, beta of a full segment
+    size_t slot_in, slot_out, state, fwd_ws, total;
+};
+
+kda_status make_host_plan(int B, int T, int H, int Hk, int dk, int dv, kda_dtype dt, unsigned pro, int seg,
+                          HostPlan& p)
+{
+    if (seg <= 0 || seg % kChunk != 0 || T <= 0) return KDA_ERR_INVALID_ARG;
+    Plan f;
+    const int s = seg < T ? seg : T;
+    const kda_status st = make_plan(B, s, H, dk, dv, false, 0, dt, f);
+    if (st != KDA_OK) return st;
+    const size_t esz = dt == KDA_BF16 ? 2 : 4, lsz = (pro & KDA_PROLOGUE_GATE_BF16) ? 2 : 4;
+    const size_t tok = (size_t)B * s;
+    p.seg = s;
+    p.nseg = (T + s - 1) / s;
+    p.in_bytes[0] = p.in_bytes[1] = tok * Hk * dk * esz;
+    p.in_bytes[2] = tok * H * dv * esz;
+    p.in_bytes[3] = tok * H * dk * lsz;
+    p.in_bytes[4] = tok * H * sizeof(float);
+    p.slot_in = 0;
+    for (size_t b : p.in_bytes) p.slot_in += round_up(b, kAlign);
+    p.slot_out = round_up(tok * H * dv * esz, kAlign);
+    p.state = round_up(sizeof(float) * (size_t)B * H * dk * dv, kAlign);
+    p.fwd_ws = round_up(f.total_bytes, kAlign);
+    p.total = 2 * (p.slot_in + p.slot_out) + p.state + p.fwd_ws;
+    return KDA_OK;
+}
+
+}  // namespace
+
+extern "C" kda_status kda_chunk_fwd_host_workspace_size(int B, int T, int H, int dk, int dv, kda_dtype dt,
+                                                        const kda_options* opt, int segment_tokens, size_t* bytes)
+{
+    if (!bytes) return KDA_ERR_INVALID_ARG;
+    int Hk = H;
+    unsigned pro = 0;
+    const kda_status so = parse_options(opt, H, Hk, pro);
+    if (so != KDA_OK) return so;
+    HostPlan p;
+    const kda_status st = make_host_plan(B, T, H, Hk, dk, dv, dt, pro, segment_tokens, p);
+    if (st != KDA_OK) return st;
+    *bytes = p.total;
+    return KDA_OK;
+}
+
+extern "C" kda_status kda_chunk_fwd_host(const void* q, const void* k, const void* v, const void* log_alpha,
+                                         const float* beta, const float* S0, void* out, float* S_final, int B,
+                                         int T, int H, int dk, int dv, kda_dtype dt, const kda_options* opt,
+                                         int segment_tokens, void* workspace, size_t workspace_bytes,
+                                         kda_stream_t stream_)
+{
+    cudaStream_t stream = (cudaStream_t)stream_;
+    int Hk = H;
+    unsigned pro = 0;
+    const kda_status so = parse_options(opt, H, Hk, pro);
+    if (so != KDA_OK) return so;
+    HostPlan p;
+    const kda_status st = make_host_plan(B, T, H, Hk, dk, dv, dt, pro, segment_tokens, p);
+    if (st != KDA_OK) return st;
+    if (!q || !k || !v || !log_alpha || !beta || !out) return KDA_ERR_INVALID_ARG;
+    if (!workspace || ((uintptr_t)workspace % kAlign) || workspace_bytes < p.total) return KDA_ERR_WORKSPACE;
+
+    char* ws = (char*)workspace;
+    char* slot_in[2] = {ws, ws + p.slot_in};
+    char* slot_out[2] = {ws + 2 * p.slot_in, ws + 2 * p.slot_in + p.slot_out};
+    float* state = (float*)(ws + 2 * (p.slot_in + p.slot_out));
+    char* fwd_ws = ws + 2 * (p.slot_in + p.slot_out) + p.state;
+    const size_t esz = dt == KDA_BF16 ? 2 : 4, lsz = (pro & KDA_PROLOGUE_GATE_BF16) ? 2 : 4;
+    // per token of one sequence: bytes of q, k, v, log_alpha, beta, out
+    const size_t per_tok[6] = {(size_t)Hk * dk * esz, (size_t)Hk * dk * esz, (size_t)H * dv * esz,
+                               (size_t)H * dk * lsz, (size_t)H * sizeof(float), (size_t)H * dv * esz};
+    const char* src[5] = {(const char*)q, (const char*)k, (const char*)v, (const char*)log_alpha,
+                          (const char*)beta};
+
+    cudaStream_t cin = nullptr, cout = nullptr;
+    cudaEvent_t ev_in[2] = {nullptr, nullptr}, ev_comp[2] = {nullptr, nullptr}, ev_out[2] = {nullptr, nullptr};
+    cudaEvent_t ev_start = nullptr;
+    kda_status rs = KDA_ERR_CUDA;
+    bool ok = cudaStreamCreateWithFlags(&cin, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&cout, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&ev_start, cudaEventDisableTiming) == cudaSuccess;
+    for (int i = 0; i < 2 && ok; ++i)
+        ok = cudaEventCreateWithFlags(&ev_in[i], cudaEventDisableTiming) == cudaSuccess &&
+             cudaEventCreateWithFlags(&ev_comp[i], cudaEventDisableTiming) == cudaSuccess &&
+             cudaEventCreateWithFlags(&ev_out[i], cudaEventDisableTiming) == cudaSuccess;
+    // the copy streams start after everything already queued on the caller's stream
+    ok = ok && cudaEventRecord(ev_start, stream) == cudaSuccess && cudaStreamWaitEvent(cin, ev_start, 0) == cudaSuccess &&
+         cudaStreamWaitEvent(cout, ev_start, 0) == cudaSuccess;
+    const size_t sbytes = sizeof(float) * (size_t)B * H * dk * dv;
+    if (ok) ok = (S0 ? cudaMemcpyAsync(state, S0, sbytes, cudaMemcpyHostToDevice, stream)
+                     : cudaMemsetAsync(state, 0, sbytes, stream)) == cudaSuccess;
+    kda_options o2 = opt ? *opt : kda_options{};
+    for (int i = 0; i < p.nseg && ok; ++i) {
+        const int b = i & 1;
+        const long long t0 = (long long)i * p.seg;
+        const int len = (int)((T - t0) < p.seg ? (T - t0) : p.seg);
+        // inputs of segment i into slot b, once segment i - 2 has finished reading it
+        if (i >= 2) ok = cudaStreamWaitEvent(cin, ev_comp[b], 0) == cudaSuccess;
+        char* dst = slot_in[b];
+        void* dptr[5];
+        for (int f = 0; f < 5 && ok; ++f) {
+            dptr[f] = dst;
+            const size_t w = per_tok[f] * (size_t)len;
+            ok = cudaMemcpy2DAsync(dst, w, src[f] + per_tok[f] * (size_t)t0, per_tok[f] * (size_t)T, w, B,
+                                   cudaMemcpyHostToDevice, cin) == cudaSuccess;
+            dst += round_up(p.in_bytes[f], kAlign);
+        }
+        ok = ok && cudaEventRecord(ev_in[b], cin) == cudaSuccess;
+        // compute on the caller's stream, once the inputs landed and slot b's previous output left
+        ok = ok && cudaStreamWaitEvent(stream, ev_in[b], 0) == cudaSuccess;
+        if (ok && i >= 2) ok = cudaStreamWaitEvent(stream, ev_out[b], 0) == cudaSuccess;
+        if (!ok) break;
+        const kda_status fs = kda_chunk_fwd_ex(dptr[0], dptr[1], dptr[2], dptr[3], (const float*)dptr[4], state,
+                                               nullptr, 0, slot_out[b], state, B, len, H, dk, dv, dt, &o2, fwd_ws,
+                                               p.fwd_ws, stream);
+        if (fs != KDA_OK) {
+            rs = fs;
+            ok = false;
+            break;
+        }
+        ok = cudaEventRecord(ev_comp[b], stream) == cudaSuccess;
+        // outputs of segment i back to the host
+        ok = ok && cudaStreamWaitEvent(cout, ev_comp[b], 0) == cudaSuccess;
+        ok = ok && cudaMemcpy2DAsync((char*)out + per_tok[5] * (size_t)t0, per_tok[5] * (size_t)T, slot_out[b],
+                                     per_tok[5] * (size_t)len, per_tok[5] * (size_t)len, B, cudaMemcpyDeviceToHost,
+                                     cout) == cudaSuccess;
+        ok = ok && cudaEventRecord(ev_out[b], cout) == cudaSuccess;
+    }
+    if (ok && S_final) ok = cudaMemcpyAsync(S_final, state, sbytes, cudaMemcpyDeviceToHost, stream) == cudaSuccess;
+    // the caller's stream completes only after every copy of this call
+    for (int b = 0; b < 2 && ok; ++b)
+        if (p.nseg > b) ok = cudaStreamWaitEvent(stream, ev_out[b], 0) == cudaSuccess;
+    if (ok) rs = KDA_OK;
+    for (int i = 0; i < 2; ++i) {
+        if (ev_in[i]) cudaEventDestroy(ev_in[i]);
+        if (ev_comp[i]) cudaEventDestroy(ev_comp[i]);
+        if (ev_out[i]) cudaEventDestroy(ev_out[i]);
+    }
+    if (ev_start) cudaEventDestroy(ev_start);
+    if (cin) cudaStreamDestroy(cin);
+    if (cout) cudaStreamDestroy(cout);
+    return rs;
+}

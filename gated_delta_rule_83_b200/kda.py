@@ -50,6 +50,10 @@ ABI = {
     "kda_chunk_bwd_workspace_size": (_I, [_I, _I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_SZ)]),
     "kda_chunk_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
                            ctypes.POINTER(KdaOptions), _P, _SZ, _P]),
+    "kda_chunk_fwd_host_workspace_size": (_I, [_I, _I, _I, _I, _I, _I, ctypes.POINTER(KdaOptions), _I,
+                                              ctypes.POINTER(_SZ)]),
+    "kda_chunk_fwd_host": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.POINTER(KdaOptions),
+                                _I, _P, _SZ, _P]),
     "kda_check": (_I, [_P]),
     "kda_selftest_timeout": (_I, [_P]),
     "kda_profile_begin": (_I, []),
@@ -216,6 +220,69 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torc
                                   _ptr(cu_seqlens), N, _ptr(out), _ptr(S_final), B, T, H, dk, dv, _dt(q),
                                   ctypes.byref(opt), _ptr(workspace), workspace.numel(), sh)
         _check("kda_chunk_fwd_ex", rc)
+    return out, S_final
+
+
+def _host(t: torch.Tensor, name: str, dtype=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host tensor (pinned for overlap)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def chunk_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor, beta: torch.Tensor,
+                   S0: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                   S_final: Optional[torch.Tensor] = None, output_final_state: bool = True, prologue: int = 0,
+                   segment_tokens: int = 4096, device=None, workspace: Optional[torch.Tensor] = None,
+                   stream: Optional[torch.cuda.Stream] = None, synchronize: bool = True):
+    """``kda_chunk_fwd_host``: the prefill on HOST tensors (pinned for overlap), pipelined in
+    segments of ``segment_tokens`` tokens: copies in, kernels and copies out overlap.  Same shapes
+    and options as ``chunk_fwd`` (regular batches).  Outputs are host tensors (pinned when
+    allocated here).  With ``synchronize`` the call waits for the stream before returning."""
+    lib = load_library()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    _host(q, "q")
+    dtq = q.dtype
+    B, T, Hk, dk = q.shape
+    H, dv = v.shape[2], v.shape[-1]
+    _host(k, "k", dtq)
+    _host(v, "v", dtq)
+    _host(log_alpha, "log_alpha")
+    prologue = _gate_bits(log_alpha, prologue)
+    _host(beta, "beta", torch.float32)
+    if k.shape != q.shape or tuple(log_alpha.shape) != (B, T, H, dk) or tuple(v.shape) != (B, T, H, dv) or \
+            tuple(beta.shape) != (B, T, H) or H % Hk != 0:
+        raise ValueError("inconsistent shapes")
+    if S0 is not None:
+        _host(S0, "S0", torch.float32)
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=dtq).pin_memory()
+    else:
+        _host(out, "out", dtq)
+    if S_final is None and output_final_state:
+        S_final = torch.empty((B, H, dk, dv), dtype=torch.float32).pin_memory()
+    elif S_final is not None:
+        _host(S_final, "S_final", torch.float32)
+    opt = KdaOptions(num_qk_heads=Hk, prologue=prologue)
+    n = ctypes.c_size_t(0)
+    _check("kda_chunk_fwd_host_workspace_size",
+           lib.kda_chunk_fwd_host_workspace_size(B, T, H, dk, dv, _dt(q), ctypes.byref(opt), segment_tokens,
+                                                 ctypes.byref(n)))
+    sh = _stream_handle(stream, dev)
+    if workspace is None:
+        workspace = _get_workspace(n.value, dev, sh)
+    else:
+        _req(workspace, "workspace", torch.uint8, dev)
+    rc = lib.kda_chunk_fwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0), _ptr(out),
+                                _ptr(S_final), B, T, H, dk, dv, _dt(q), ctypes.byref(opt), segment_tokens,
+                                _ptr(workspace), workspace.numel(), sh)
+    _check("kda_chunk_fwd_host", rc)
+    if synchronize:
+        (stream or torch.cuda.current_stream(dev)).synchronize()
     return out, S_final
 
 

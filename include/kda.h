@@ -183,6 +183,36 @@ kda_status kda_decode_step_ex(const void* q, const void* k, const void* v, const
                               kda_dtype dt, const kda_options* opt, kda_stream_t stream);
 
 /*
+ * kda_chunk_fwd_host -- kda_chunk_fwd on HOST-resident inputs and outputs, pipelined.
+ *
+ * A deployment path of this library (the pages describe none): when q, k, v, log_alpha, beta (and
+ * S0) live in host memory, the call splits the token axis into segments of `segment_tokens` and
+ * runs them through a double-buffered pipeline.  Segment i + 1 is copied in on a copy stream while
+ * segment i runs on `stream` and segment i - 1 is copied out on a second copy stream, so the host
+ * link's two directions and the kernels overlap.  The state is carried from segment to segment on
+ * the device; results are bit-identical to one kda_chunk_fwd_ex call on the whole input, because
+ * the segments start on chunk boundaries.
+ *   q, k, v, log_alpha, beta, S0, out, S_final: HOST pointers, layouts as kda_chunk_fwd /
+ *                kda_chunk_fwd_ex (regular batches of B sequences of T tokens; S0, S_final may be
+ *                NULL).  Use page-locked (pinned) memory: pageable memory works but does not overlap.
+ *   opt          as kda_chunk_fwd_ex (grouped heads, prologue bits incl. bf16 gates), or NULL.
+ *   segment_tokens  a positive multiple of 64 (4096 is a good value for 32 heads of 128).
+ *   workspace    DEVICE memory, >= kda_chunk_fwd_host_workspace_size(...) bytes, 256-byte aligned:
+ *                two input and two output segment buffers, the state and the chunk workspace.
+ * Asynchronous on `stream`: the host buffers must stay untouched, and out / S_final are complete,
+ * only once `stream` has been synchronised (the call's copy streams are joined into it).  Creates
+ * and destroys two streams and a few events per call.  Errors: as kda_chunk_fwd_ex, and
+ * KDA_ERR_INVALID_ARG for a segment length that is not a positive multiple of 64, T <= 0 or a NULL
+ * input; after KDA_ERR_CUDA the outputs are undefined.
+ */
+kda_status kda_chunk_fwd_host_workspace_size(int B, int T, int H, int dk, int dv, kda_dtype dt,
+                                             const kda_options* opt, int segment_tokens, size_t* bytes);
+kda_status kda_chunk_fwd_host(const void* q, const void* k, const void* v, const void* log_alpha,
+                              const float* beta, const float* S0, void* out, float* S_final, int B, int T,
+                              int H, int dk, int dv, kda_dtype dt, const kda_options* opt, int segment_tokens,
+                              void* workspace, size_t workspace_bytes, kda_stream_t stream);
+
+/*
  * kda_chunk_bwd -- the backward pass of kda_chunk_fwd (training): the derivatives of a scalar loss
  * L with respect to every input, given the cotangents of the outputs,
  *

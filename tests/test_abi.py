@@ -159,3 +159,18 @@ def test_synth_distributions():
     # same seed -> same bits
     inp2 = synth.prefill_inputs(w, T=512, H=4)
     assert torch.equal(inp["q"], inp2["q"]) and torch.equal(inp["log_alpha"], inp2["log_alpha"])
+
+
+def test_host_pipeline_rejects_before_launch(lib):
+    """kda_chunk_fwd_host validates the segment length and the workspace before any CUDA call."""
+    fake = 0x100000
+    n = ctypes.c_size_t(0)
+    assert lib.kda_chunk_fwd_host_workspace_size(1, 1000, 2, 128, 128, 0, None, 100, ctypes.byref(n)) == 1
+    assert lib.kda_chunk_fwd_host_workspace_size(1, 0, 2, 128, 128, 0, None, 128, ctypes.byref(n)) == 1
+    assert lib.kda_chunk_fwd_host_workspace_size(1, 1000, 2, 128, 128, 0, None, 128, ctypes.byref(n)) == 0
+    assert n.value > 0
+    args = (fake, fake, fake, fake, fake, None, fake, None, 1, 1000, 2, 128, 128, 0, None)
+    assert lib.kda_chunk_fwd_host(*args, 96, fake, 1 << 40, None) == 1         # segment not a multiple of 64
+    assert lib.kda_chunk_fwd_host(*args, 128, None, 1 << 40, None) == 5        # no workspace
+    assert lib.kda_chunk_fwd_host(*args, 128, fake, 16, None) == 5             # workspace too small
+

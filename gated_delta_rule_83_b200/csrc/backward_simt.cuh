@@ -436,14 +436,15 @@ __device__ __forceinline__ void bwd_load_scr_tile(const float* __restrict__ x, i
     }
 }
 
+// Step 4, first half (one CTA per (chunk, head)): At and dT over all channel and value tiles, the
+// UT transform backwards (N, dbeta, dM -> dAt) and dV.  N and dAt go to the unit's scratch (over U
+// and dU, both dead by then) for the second half.
 template <typename TIn>
-__global__ void __launch_bounds__(kSimtThreads)
-bwd_input_side_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
-                      const void* __restrict__ log_alpha, const float* __restrict__ beta,
-                      const WsHeader* __restrict__ hdr, const int* __restrict__ off, const int32_t* __restrict__ cu,
-                      int Tseq, int N, int H, unsigned pro, int dk, int dv, const float* __restrict__ scr,
-                      TIn* __restrict__ dq, TIn* __restrict__ dk_out, TIn* __restrict__ dv_out,
-                      float* __restrict__ dla, float* __restrict__ dbeta)
+__global__ void __launch_bounds__(kSimtThreads, 2)
+bwd_ut_kernel(const TIn* __restrict__ k, const TIn* __restrict__ v, const void* __restrict__ log_alpha,
+              const float* __restrict__ beta, const WsHeader* __restrict__ hdr, const int* __restrict__ off,
+              const int32_t* __restrict__ cu, int Tseq, int N, int H, unsigned pro, int dk, int dv,
+              float* __restrict__ scr, TIn* __restrict__ dv_out, float* __restrict__ dbeta)
 {
     extern __shared__ __align__(16) float smem[];
     const int j = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
@@ -458,32 +459,25 @@ bwd_input_side_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, cons
     float* sAt = smem;            // [64][65] At = strict_lower(Kf Kb^T) (without beta)
     float* sN = sAt + M64;        // [64][65] N = (I + Diag(beta) At)^{-1}
     float* sM = sN + M64;         // [64][65] dT -> dN -> dM -> dAt
-    float* sY = sM + M64;         // [64][65] dN N^T
-    float* sdP = sY + M64;        // [64][65] dP
-    float* tk = sdP + M64;        // tiles [64][33]: k (or v), q, g and four temporaries
-    float* tq = tk + MT;
-    float* tg = tq + MT;
+    float* tk = sM + M64;         // tiles [64][33]: k (or v), g and four temporaries
+    float* tg = tk + MT;
     float* tA = tg + MT;
     float* tB = tA + MT;
     float* tC = tB + MT;
     float* tD = tC + MT;
+    float* sY = tA;               // [64][65] dN N^T, over tA..tB (the tiles are idle in the UT step)
     float* sb = tD + MT;          // [64] beta
     float* sdb = sb + kChunk;     // [64] dbeta
     float* tref = sdb + kChunk;   // [32]
     __shared__ int s_wide;
 
     const size_t u = (size_t)j * H + h;
-    const float* o = scr + u * bwd_scr_floats(dk, dv);
+    float* o = scr + u * bwd_scr_floats(dk, dv);
     const float* gdU = o + (size_t)kChunk * dv;
-    const float* gdQg = gdU + (size_t)kChunk * dv;
-    const float* gdW = gdQg + (size_t)kChunk * dk;
-    const float* gdKd = gdW + (size_t)kChunk * dk;
-    const float* gdP = gdKd + (size_t)kChunk * dk;
-    const float* gdGam = gdP + (size_t)kChunk * kChunk;
+    const float* gdW = gdU + (size_t)kChunk * dv + (size_t)kChunk * dk;
     const int tr = tid >> 4, tc = tid & 15;
 
     for (int r = tid; r < kChunk; r += kSimtThreads) sb[r] = (r < L) ? beta[(size_t)(t0 + r) * H + h] : 0.f;
-    for (int e = tid; e < kChunk * kChunk; e += kSimtThreads) sdP[(e / kChunk) * L64 + (e % kChunk)] = gdP[e];
 
     // ---- step 4a: At and dT = dW Kt^T + dU V^T, accumulated in registers over tiles
     float accA[4][4] = {}, accT[4][4] = {};
@@ -592,106 +586,6 @@ bwd_input_side_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, cons
     __syncthreads();
     for (int r = tid; r < L; r += kSimtThreads) dbeta[(size_t)(t0 + r) * H + h] = sdb[r];
 
-    // ---- step 4c: dq, dk, dlog_alpha per channel tile
-    for (int c0 = 0; c0 < dk; c0 += kBwdCT) {
-        __syncthreads();
-        if (tid == 0) s_wide = 0;
-        __syncthreads();
-        bwd_load_tile(k, t0, L, H, h, dk, c0, tk);
-        bwd_load_tile(q, t0, L, H, h, dk, c0, tq);
-        bwd_gate_tile(log_alpha, la16, t0, L, H, h, dk, c0, tg, tref, &s_wide);
-        bwd_load_scr_tile(gdW, dk, c0, tD);
-        __syncthreads();
-        const bool wide = s_wide != 0;
-        if (!wide)
-            for (int e = tid; e < kChunk * kBwdCT; e += kSimtThreads) {
-                const int r = e / kBwdCT, cc = e % kBwdCT;
-                const float x = tg[r * LT + cc] - tref[cc];
-                const float ex = expf(x), emx = expf(-x);
-                tA[r * LT + cc] = tk[r * LT + cc] * ex;   // Kf
-                tB[r * LT + cc] = tk[r * LT + cc] * emx;  // Kb
-                tC[r * LT + cc] = tq[r * LT + cc] * ex;   // Qf
-            }
-        __syncthreads();
-        // per (row r, channel): rowP = sum_i dP[r][i] k_i E(r,i), rowA = sum_i dAt[r][i] k_i E(r,i),
-        // col = sum_a (dP[a][r] q_a + dAt[a][r] k_a) E(a,r), dKt = beta_r sum_a N[a][r] dW[a]
-        float rowP[4][2] = {}, rowA[4][2] = {}, col[4][2] = {}, dkt[4][2] = {};
-        if (!wide) {
-            mm_acc<4, 2>(rowP, sdP, L64, 1, tB, LT, 1, kChunk, tr, tc);
-            mm_acc<4, 2>(rowA, sM, L64, 1, tB, LT, 1, kChunk, tr, tc);
-            mm_acc<4, 2>(col, sdP, 1, L64, tC, LT, 1, kChunk, tr, tc);
-            mm_acc<4, 2>(col, sM, 1, L64, tA, LT, 1, kChunk, tr, tc);
-        } else {
-#pragma unroll
-            for (int a = 0; a < 4; ++a)
-#pragma unroll
-                for (int b = 0; b < 2; ++b) {
-                    const int r = tr + 16 * a, cc = tc + 16 * b;
-                    const float gr = tg[r * LT + cc];
-                    for (int i = 0; i <= r; ++i) {
-                        const float ke = tk[i * LT + cc] * expf(gr - tg[i * LT + cc]);
-                        rowP[a][b] = fmaf(sdP[r * L64 + i], ke, rowP[a][b]);
-                        rowA[a][b] = fmaf(sM[r * L64 + i], ke, rowA[a][b]);
-                    }
-                    for (int i = r; i < kChunk; ++i)
-                        col[a][b] = fmaf(fmaf(sdP[i * L64 + r], tq[i * LT + cc], sM[i * L64 + r] * tk[i * LT + cc]),
-                                         expf(tg[i * LT + cc] - gr), col[a][b]);
-                }
-        }
-        mm_acc<4, 2>(dkt, sN, 1, L64, tD, LT, 1, kChunk, tr, tc);
-        float accg[4][2], accl[4][2];
-#pragma unroll
-        for (int a = 0; a < 4; ++a)
-#pragma unroll
-            for (int b = 0; b < 2; ++b) {
-                const int r = tr + 16 * a, cc = tc + 16 * b;
-                const float g = tg[r * LT + cc], gl = tg[(kChunk - 1) * LT + cc];
-                if (!wide) {
-                    const float x = g - tref[cc];
-                    const float ex = expf(x);
-                    rowP[a][b] *= ex;
-                    rowA[a][b] *= ex;
-                    col[a][b] *= expf(-x);
-                }
-                const float kt = dkt[a][b] * sb[r];
-                const float eg = expf(g), egl = expf(gl - g);
-                const float qv = tq[r * LT + cc], kv = tk[r * LT + cc];
-                const size_t gi = (size_t)r * dk + c0 + cc;
-                const float dQg = gdQg[gi], dKd = gdKd[gi];
-                const float vq = rowP[a][b] + dQg * eg;
-                const float vk = rowA[a][b] + col[a][b] + kt * eg + dKd * egl;
-                accg[a][b] = qv * rowP[a][b] + kv * rowA[a][b] - kv * col[a][b] + (dQg * qv + kt * kv) * eg -
-                             dKd * kv * egl;
-                accl[a][b] = dKd * kv * egl;  // chunk-end term of g_last, summed below
-                if (r < L) {
-                    const size_t oi = ((size_t)(t0 + r) * H + h) * dk + c0 + cc;
-                    dq[oi] = from_f32<TIn>(vq);
-                    dk_out[oi] = from_f32<TIn>(vk);
-                }
-            }
-        __syncthreads();  // every thread is done with Kf / Kb / Qf
-#pragma unroll
-        for (int a = 0; a < 4; ++a)
-#pragma unroll
-            for (int b = 0; b < 2; ++b) {
-                const int r = tr + 16 * a, cc = tc + 16 * b;
-                tA[r * LT + cc] = accl[a][b];
-                tB[r * LT + cc] = accg[a][b];
-            }
-        __syncthreads();
-        if (tid < kBwdCT) {  // g_last terms, then dlog_alpha = reverse cumulative sum of dg
-            const int cc = tid;
-            float s = 0.f;
-            for (int r = 0; r < kChunk; ++r) s += tA[r * LT + cc];
-            s += gdGam[c0 + cc] * expf(tg[(kChunk - 1) * LT + cc]);
-            float acc = s;
-            for (int r = kChunk - 1; r >= 0; --r) {
-                acc += tB[r * LT + cc];
-                if (r < L) dla[((size_t)(t0 + r) * H + h) * dk + c0 + cc] = acc;
-            }
-        }
-    }
-
     // ---- step 4d: dV = T^T dU = Diag(beta) N^T dU
     for (int c0 = 0; c0 < dv; c0 += kBwdCT) {
         __syncthreads();
@@ -706,6 +600,164 @@ bwd_input_side_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, cons
                 const int i = tr + 16 * a, cc = tc + 16 * b;
                 if (i < L) dv_out[((size_t)(t0 + i) * H + h) * dv + c0 + cc] = from_f32<TIn>(sb[i] * acc[a][b]);
             }
+    }
+    // N and dAt out for the gate half (U and dU are no longer read)
+    __syncthreads();
+    float* gN = o;
+    float* gdAt = o + (size_t)kChunk * dv;
+    for (int e = tid; e < kChunk * kChunk; e += kSimtThreads) {
+        const int r = e / kChunk, i = e % kChunk;
+        gN[e] = sN[r * L64 + i];
+        gdAt[e] = sM[r * L64 + i];
+    }
+}
+
+// Step 4, second half (one CTA per (chunk, head, 32-channel tile)): dq, dk and dlog_alpha through
+// the gated products P = Qf Kb^T, At = Kf Kb^T and the gating itself.
+template <typename TIn>
+__global__ void __launch_bounds__(kSimtThreads, 2)
+bwd_gate_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const void* __restrict__ log_alpha,
+                const float* __restrict__ beta, const WsHeader* __restrict__ hdr, const int* __restrict__ off,
+                const int32_t* __restrict__ cu, int Tseq, int N, int H, unsigned pro, int dk, int dv,
+                const float* __restrict__ scr, TIn* __restrict__ dq, TIn* __restrict__ dk_out,
+                float* __restrict__ dla)
+{
+    extern __shared__ __align__(16) float smem[];
+    const int j = blockIdx.x, h = blockIdx.y, c0 = blockIdx.z * kBwdCT, tid = threadIdx.x;
+    if (hdr->bad || j >= hdr->total_chunks) return;
+    int n, L;
+    long long t0;
+    locate_chunk(j, off, cu, Tseq, N, n, t0, L);
+    const bool la16 = (pro & KDA_PROLOGUE_GATE_BF16) != 0;
+    constexpr int M64 = kChunk * kBwdL64;
+    constexpr int MT = kChunk * kBwdLT;
+    constexpr int L64 = kBwdL64, LT = kBwdLT;
+    float* sN = smem;             // [64][65] N
+    float* sM = sN + M64;         // [64][65] dAt
+    float* sdP = sM + M64;        // [64][65] dP
+    float* tk = sdP + M64;        // tiles [64][33]: k, q, g, dW and three temporaries
+    float* tq = tk + MT;
+    float* tg = tq + MT;
+    float* tA = tg + MT;
+    float* tB = tA + MT;
+    float* tC = tB + MT;
+    float* tD = tC + MT;
+    float* sb = tD + MT;          // [64] beta
+    float* tref = sb + kChunk;    // [32]
+    __shared__ int s_wide;
+
+    const size_t u = (size_t)j * H + h;
+    const float* o = scr + u * bwd_scr_floats(dk, dv);
+    const float* gN = o;
+    const float* gdAt = o + (size_t)kChunk * dv;
+    const float* gdQg = o + 2 * (size_t)kChunk * dv;
+    const float* gdW = gdQg + (size_t)kChunk * dk;
+    const float* gdKd = gdW + (size_t)kChunk * dk;
+    const float* gdP = gdKd + (size_t)kChunk * dk;
+    const float* gdGam = gdP + (size_t)kChunk * kChunk;
+    const int tr = tid >> 4, tc = tid & 15;
+
+    if (tid == 0) s_wide = 0;
+    for (int r = tid; r < kChunk; r += kSimtThreads) sb[r] = (r < L) ? beta[(size_t)(t0 + r) * H + h] : 0.f;
+    for (int e = tid; e < kChunk * kChunk; e += kSimtThreads) {
+        const int x = (e / kChunk) * L64 + (e % kChunk);
+        sN[x] = gN[e];
+        sM[x] = gdAt[e];
+        sdP[x] = gdP[e];
+    }
+    bwd_load_tile(k, t0, L, H, h, dk, c0, tk);
+    bwd_load_tile(q, t0, L, H, h, dk, c0, tq);
+    bwd_load_scr_tile(gdW, dk, c0, tD);
+    __syncthreads();  // s_wide zeroed before the gate tile flags it
+    bwd_gate_tile(log_alpha, la16, t0, L, H, h, dk, c0, tg, tref, &s_wide);
+    __syncthreads();
+    const bool wide = s_wide != 0;
+    if (!wide)
+        for (int e = tid; e < kChunk * kBwdCT; e += kSimtThreads) {
+            const int r = e / kBwdCT, cc = e % kBwdCT;
+            const float x = tg[r * LT + cc] - tref[cc];
+            const float ex = expf(x), emx = expf(-x);
+            tA[r * LT + cc] = tk[r * LT + cc] * ex;   // Kf
+            tB[r * LT + cc] = tk[r * LT + cc] * emx;  // Kb
+            tC[r * LT + cc] = tq[r * LT + cc] * ex;   // Qf
+        }
+    __syncthreads();
+    // per (row r, channel): rowP = sum_i dP[r][i] k_i E(r,i), rowA = sum_i dAt[r][i] k_i E(r,i),
+    // col = sum_a (dP[a][r] q_a + dAt[a][r] k_a) E(a,r), dKt = beta_r sum_a N[a][r] dW[a]
+    float rowP[4][2] = {}, rowA[4][2] = {}, col[4][2] = {}, dkt[4][2] = {};
+    if (!wide) {
+        mm_acc<4, 2>(rowP, sdP, L64, 1, tB, LT, 1, kChunk, tr, tc);
+        mm_acc<4, 2>(rowA, sM, L64, 1, tB, LT, 1, kChunk, tr, tc);
+        mm_acc<4, 2>(col, sdP, 1, L64, tC, LT, 1, kChunk, tr, tc);
+        mm_acc<4, 2>(col, sM, 1, L64, tA, LT, 1, kChunk, tr, tc);
+    } else {
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+                const int r = tr + 16 * a, cc = tc + 16 * b;
+                const float gr = tg[r * LT + cc];
+                for (int i = 0; i <= r; ++i) {
+                    const float ke = tk[i * LT + cc] * expf(gr - tg[i * LT + cc]);
+                    rowP[a][b] = fmaf(sdP[r * L64 + i], ke, rowP[a][b]);
+                    rowA[a][b] = fmaf(sM[r * L64 + i], ke, rowA[a][b]);
+                }
+                for (int i = r; i < kChunk; ++i)
+                    col[a][b] = fmaf(fmaf(sdP[i * L64 + r], tq[i * LT + cc], sM[i * L64 + r] * tk[i * LT + cc]),
+                                     expf(tg[i * LT + cc] - gr), col[a][b]);
+            }
+    }
+    mm_acc<4, 2>(dkt, sN, 1, L64, tD, LT, 1, kChunk, tr, tc);
+    float accg[4][2], accl[4][2];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+            const int r = tr + 16 * a, cc = tc + 16 * b;
+            const float g = tg[r * LT + cc], gl = tg[(kChunk - 1) * LT + cc];
+            if (!wide) {
+                const float x = g - tref[cc];
+                const float ex = expf(x);
+                rowP[a][b] *= ex;
+                rowA[a][b] *= ex;
+                col[a][b] *= expf(-x);
+            }
+            const float kt = dkt[a][b] * sb[r];
+            const float eg = expf(g), egl = expf(gl - g);
+            const float qv = tq[r * LT + cc], kv = tk[r * LT + cc];
+            const size_t gi = (size_t)r * dk + c0 + cc;
+            const float dQg = gdQg[gi], dKd = gdKd[gi];
+            const float vq = rowP[a][b] + dQg * eg;
+            const float vk = rowA[a][b] + col[a][b] + kt * eg + dKd * egl;
+            accg[a][b] = qv * rowP[a][b] + kv * rowA[a][b] - kv * col[a][b] + (dQg * qv + kt * kv) * eg -
+                         dKd * kv * egl;
+            accl[a][b] = dKd * kv * egl;  // chunk-end term of g_last, summed below
+            if (r < L) {
+                const size_t oi = ((size_t)(t0 + r) * H + h) * dk + c0 + cc;
+                dq[oi] = from_f32<TIn>(vq);
+                dk_out[oi] = from_f32<TIn>(vk);
+            }
+        }
+    __syncthreads();  // every thread is done with Kf / Kb / Qf
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+            const int r = tr + 16 * a, cc = tc + 16 * b;
+            tA[r * LT + cc] = accl[a][b];
+            tB[r * LT + cc] = accg[a][b];
+        }
+    __syncthreads();
+    if (tid < kBwdCT) {  // g_last terms, then dlog_alpha = reverse cumulative sum of dg
+        const int cc = tid;
+        float s = 0.f;
+        for (int r = 0; r < kChunk; ++r) s += tA[r * LT + cc];
+        s += gdGam[c0 + cc] * expf(tg[(kChunk - 1) * LT + cc]);
+        float acc = s;
+        for (int r = kChunk - 1; r >= 0; --r) {
+            acc += tB[r * LT + cc];
+            if (r < L) dla[((size_t)(t0 + r) * H + h) * dk + c0 + cc] = acc;
+        }
     }
 }
 
@@ -724,9 +776,13 @@ inline size_t bwd_state_side_smem(int dk, int dv)
     (void)dk;
     return sizeof(float) * (size_t)5 * kChunk * (dv + 1);
 }
-inline size_t bwd_input_side_smem()
+inline size_t bwd_ut_smem()
 {
-    return sizeof(float) * ((size_t)5 * kChunk * kBwdL64 + 7 * kChunk * kBwdLT + 2 * kChunk + kBwdCT);
+    return sizeof(float) * ((size_t)3 * kChunk * kBwdL64 + 6 * kChunk * kBwdLT + 2 * kChunk + kBwdCT);
+}
+inline size_t bwd_gate_smem()
+{
+    return sizeof(float) * ((size_t)3 * kChunk * kBwdL64 + 7 * kChunk * kBwdLT + kChunk + kBwdCT);
 }
 
 template <typename TIn, int DK>
@@ -762,12 +818,15 @@ cudaError_t launch_simt_backward(const void* q, const void* k, const void* v, co
                                  int dv, int max_chunks, float* slots, float* S_chunks, float* dSn_chunks, float* scr,
                                  cudaStream_t stream)
 {
-    const size_t smA = simt_intra_smem(dk, dv), smS = bwd_state_side_smem(dk, dv), smI = bwd_input_side_smem();
+    const size_t smA = simt_intra_smem(dk, dv), smS = bwd_state_side_smem(dk, dv), smU = bwd_ut_smem(),
+                 smG = bwd_gate_smem();
     cudaError_t e = cudaFuncSetAttribute(simt_intra_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smA);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(bwd_state_side_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smS);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(bwd_input_side_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smI);
+        e = cudaFuncSetAttribute(bwd_ut_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smU);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(bwd_gate_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smG);
     if (e != cudaSuccess) return e;
     const TIn *qq = (const TIn*)q, *kk = (const TIn*)k, *vv = (const TIn*)v;
     if (max_chunks > 0) {
@@ -788,10 +847,17 @@ cudaError_t launch_simt_backward(const void* q, const void* k, const void* v, co
                 (const TIn*)dout, hdr, off, cu, Tseq, N, H, dk, dv, S_chunks, dSn_chunks, scr);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
         }
-        LaunchScope ls("bwd_input_side", stream);
-        bwd_input_side_kernel<TIn><<<dim3(max_chunks, H), kSimtThreads, smI, stream>>>(
-            qq, kk, vv, la, beta, hdr, off, cu, Tseq, N, H, pro & KDA_PROLOGUE_GATE_BF16, dk, dv, scr, (TIn*)dq,
-            (TIn*)dk_out, (TIn*)dv_out, dla, dbeta);
+        {
+            LaunchScope ls("bwd_ut", stream);
+            bwd_ut_kernel<TIn><<<dim3(max_chunks, H), kSimtThreads, smU, stream>>>(
+                kk, vv, la, beta, hdr, off, cu, Tseq, N, H, pro & KDA_PROLOGUE_GATE_BF16, dk, dv, scr, (TIn*)dv_out,
+                dbeta);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
+        LaunchScope ls("bwd_gate", stream);
+        bwd_gate_kernel<TIn><<<dim3(max_chunks, H, dk / kBwdCT), kSimtThreads, smG, stream>>>(
+            qq, kk, la, beta, hdr, off, cu, Tseq, N, H, pro & KDA_PROLOGUE_GATE_BF16, dk, dv, scr, (TIn*)dq,
+            (TIn*)dk_out, dla);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     return cudaSuccess;

@@ -443,7 +443,7 @@ template <typename TIn>
 __global__ void __launch_bounds__(kSimtThreads, 2)
 bwd_ut_kernel(const TIn* __restrict__ k, const TIn* __restrict__ v, const void* __restrict__ log_alpha,
               const float* __restrict__ beta, const WsHeader* __restrict__ hdr, const int* __restrict__ off,
-              const int32_t* __restrict__ cu, int Tseq, int N, int H, unsigned pro, int dk, int dv,
+              const int32_t* __restrict__ cu, int Tseq, int N, int H, int Hk, unsigned pro, int dk, int dv,
               float* __restrict__ scr, TIn* __restrict__ dv_out, float* __restrict__ dbeta)
 {
     extern __shared__ __align__(16) float smem[];
@@ -485,7 +485,7 @@ bwd_ut_kernel(const TIn* __restrict__ k, const TIn* __restrict__ v, const void* 
         __syncthreads();
         if (tid == 0) s_wide = 0;
         __syncthreads();
-        bwd_load_tile(k, t0, L, H, h, dk, c0, tk);
+        bwd_load_tile(k, t0, L, Hk, h / (H / Hk), dk, c0, tk);  // the q/k head of value head h
         bwd_gate_tile(log_alpha, la16, t0, L, H, h, dk, c0, tg, tref, &s_wide);
         bwd_load_scr_tile(gdW, dk, c0, tD);
         __syncthreads();
@@ -618,9 +618,9 @@ template <typename TIn>
 __global__ void __launch_bounds__(kSimtThreads, 2)
 bwd_gate_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const void* __restrict__ log_alpha,
                 const float* __restrict__ beta, const WsHeader* __restrict__ hdr, const int* __restrict__ off,
-                const int32_t* __restrict__ cu, int Tseq, int N, int H, unsigned pro, int dk, int dv,
+                const int32_t* __restrict__ cu, int Tseq, int N, int H, int Hk, unsigned pro, int dk, int dv,
                 const float* __restrict__ scr, TIn* __restrict__ dq, TIn* __restrict__ dk_out,
-                float* __restrict__ dla)
+                float* __restrict__ dla, float* __restrict__ dq_acc, float* __restrict__ dk_acc)
 {
     extern __shared__ __align__(16) float smem[];
     const int j = blockIdx.x, h = blockIdx.y, c0 = blockIdx.z * kBwdCT, tid = threadIdx.x;
@@ -665,8 +665,8 @@ bwd_gate_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const void
         sM[x] = gdAt[e];
         sdP[x] = gdP[e];
     }
-    bwd_load_tile(k, t0, L, H, h, dk, c0, tk);
-    bwd_load_tile(q, t0, L, H, h, dk, c0, tq);
+    bwd_load_tile(k, t0, L, Hk, h / (H / Hk), dk, c0, tk);  // the q/k head of value head h
+    bwd_load_tile(q, t0, L, Hk, h / (H / Hk), dk, c0, tq);
     bwd_load_scr_tile(gdW, dk, c0, tD);
     __syncthreads();  // s_wide zeroed before the gate tile flags it
     bwd_gate_tile(log_alpha, la16, t0, L, H, h, dk, c0, tg, tref, &s_wide);
@@ -734,8 +734,13 @@ bwd_gate_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const void
             accl[a][b] = dKd * kv * egl;  // chunk-end term of g_last, summed below
             if (r < L) {
                 const size_t oi = ((size_t)(t0 + r) * H + h) * dk + c0 + cc;
-                dq[oi] = from_f32<TIn>(vq);
-                dk_out[oi] = from_f32<TIn>(vk);
+                if (dq_acc) {  // grouped heads: per value head, summed over each group afterwards
+                    dq_acc[oi] = vq;
+                    dk_acc[oi] = vk;
+                } else {
+                    dq[oi] = from_f32<TIn>(vq);
+                    dk_out[oi] = from_f32<TIn>(vk);
+                }
             }
         }
     __syncthreads();  // every thread is done with Kf / Kb / Qf
@@ -759,6 +764,22 @@ bwd_gate_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const void
             if (r < L) dla[((size_t)(t0 + r) * H + h) * dk + c0 + cc] = acc;
         }
     }
+}
+
+// grouped q/k heads: dq[t][hk][c] = sum over the G value heads hk*G .. hk*G+G-1 of the per-value-head
+// gradients (value head h reads q/k head h / G)
+template <typename TIn>
+__global__ void __launch_bounds__(256)
+bwd_group_sum_kernel(const float* __restrict__ acc, TIn* __restrict__ out, long long n_out, int G, int dk)
+{
+    const long long e = (long long)blockIdx.x * 256 + threadIdx.x;
+    if (e >= n_out) return;
+    const long long row = e / dk;  // (t, hk)
+    const int c = (int)(e - row * dk);
+    const float* src = acc + (size_t)row * G * dk + c;  // rows t*H + hk*G + g are consecutive
+    float s = 0.f;
+    for (int g = 0; g < G; ++g) s += src[(size_t)g * dk];
+    out[e] = from_f32<TIn>(s);
 }
 
 inline size_t bwd_fwd_chain_smem(int dk, int dv)
@@ -814,9 +835,9 @@ template <typename TIn>
 cudaError_t launch_simt_backward(const void* q, const void* k, const void* v, const void* la, const float* beta,
                                  const float* S0, const void* dout, const float* dS_final, void* dq, void* dk_out,
                                  void* dv_out, float* dla, float* dbeta, float* dS0, const WsHeader* hdr,
-                                 const int* off, const int32_t* cu, int Tseq, int N, int H, unsigned pro, int dk,
-                                 int dv, int max_chunks, float* slots, float* S_chunks, float* dSn_chunks, float* scr,
-                                 cudaStream_t stream)
+                                 const int* off, const int32_t* cu, int Tseq, int N, int H, int Hk, unsigned pro,
+                                 int dk, int dv, int max_chunks, long long Ttot, float* slots, float* S_chunks,
+                                 float* dSn_chunks, float* scr, float* dq_acc, float* dk_acc, cudaStream_t stream)
 {
     const size_t smA = simt_intra_smem(dk, dv), smS = bwd_state_side_smem(dk, dv), smU = bwd_ut_smem(),
                  smG = bwd_gate_smem();
@@ -832,7 +853,7 @@ cudaError_t launch_simt_backward(const void* q, const void* k, const void* v, co
     if (max_chunks > 0) {
         LaunchScope ls("bwd_fwd_intra", stream);
         simt_intra_kernel<TIn><<<dim3(max_chunks, H), kSimtThreads, smA, stream>>>(
-            qq, kk, vv, la, beta, hdr, off, cu, Tseq, N, H, H, pro & KDA_PROLOGUE_GATE_BF16, dk, dv, slots);
+            qq, kk, vv, la, beta, hdr, off, cu, Tseq, N, H, Hk, pro & KDA_PROLOGUE_GATE_BF16, dk, dv, slots);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     e = (dk == 128) ? launch_bwd_chains<TIn, 128>(S0, dout, dS_final, dS0, hdr, off, cu, Tseq, N, H, dv, slots,
@@ -850,15 +871,27 @@ cudaError_t launch_simt_backward(const void* q, const void* k, const void* v, co
         {
             LaunchScope ls("bwd_ut", stream);
             bwd_ut_kernel<TIn><<<dim3(max_chunks, H), kSimtThreads, smU, stream>>>(
-                kk, vv, la, beta, hdr, off, cu, Tseq, N, H, pro & KDA_PROLOGUE_GATE_BF16, dk, dv, scr, (TIn*)dv_out,
-                dbeta);
+                kk, vv, la, beta, hdr, off, cu, Tseq, N, H, Hk, pro & KDA_PROLOGUE_GATE_BF16, dk, dv, scr,
+                (TIn*)dv_out, dbeta);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
         }
-        LaunchScope ls("bwd_gate", stream);
-        bwd_gate_kernel<TIn><<<dim3(max_chunks, H, dk / kBwdCT), kSimtThreads, smG, stream>>>(
-            qq, kk, la, beta, hdr, off, cu, Tseq, N, H, pro & KDA_PROLOGUE_GATE_BF16, dk, dv, scr, (TIn*)dq,
-            (TIn*)dk_out, dla);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        {
+            LaunchScope ls("bwd_gate", stream);
+            const bool grouped = Hk != H;
+            bwd_gate_kernel<TIn><<<dim3(max_chunks, H, dk / kBwdCT), kSimtThreads, smG, stream>>>(
+                qq, kk, la, beta, hdr, off, cu, Tseq, N, H, Hk, pro & KDA_PROLOGUE_GATE_BF16, dk, dv, scr, (TIn*)dq,
+                (TIn*)dk_out, dla, grouped ? dq_acc : nullptr, grouped ? dk_acc : nullptr);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
+        if (Hk != H) {
+            LaunchScope ls("bwd_group_sum", stream);
+            const long long n_out = Ttot * Hk * dk;
+            const long long blocks = (n_out + 255) / 256;
+            if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+            bwd_group_sum_kernel<TIn><<<(unsigned)blocks, 256, 0, stream>>>(dq_acc, (TIn*)dq, n_out, H / Hk, dk);
+            bwd_group_sum_kernel<TIn><<<(unsigned)blocks, 256, 0, stream>>>(dk_acc, (TIn*)dk_out, n_out, H / Hk, dk);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
     }
     return cudaSuccess;
 }

@@ -86,10 +86,12 @@ kda_status make_plan(int B, int T, int H, int dk, int dv, bool varlen, int num_s
 // forward slot, the chunk's start state, its end cotangent and the state-side scratch.
 struct BwdPlan {
     Plan f;
-    size_t slot_bytes, state_bytes, scr_bytes, total_bytes;
+    size_t slot_bytes, state_bytes, scr_bytes, acc_bytes, total_bytes;
 };
 
-kda_status make_bwd_plan(int B, int T, int H, int dk, int dv, bool varlen, int num_seqs, kda_dtype dt, BwdPlan& p)
+// Hk < H (grouped q/k heads) adds two fp32 per-value-head buffers for dq and dk, summed per group
+kda_status make_bwd_plan(int B, int T, int H, int Hk, int dk, int dv, bool varlen, int num_seqs, kda_dtype dt,
+                         BwdPlan& p)
 {
     const kda_status st = make_plan(B, T, H, dk, dv, varlen, num_seqs, dt, p.f);
     if (st != KDA_OK) return st;
@@ -98,7 +100,9 @@ kda_status make_bwd_plan(int B, int T, int H, int dk, int dv, bool varlen, int n
     p.slot_bytes = sizeof(float) * simt_slot_floats(dk, dv);
     p.state_bytes = sizeof(float) * (size_t)dk * dv;
     p.scr_bytes = sizeof(float) * bwd_scr_floats(dk, dv);
-    p.total_bytes = sizeof(WsHeader) + p.f.off_bytes + units * (p.slot_bytes + 2 * p.state_bytes + p.scr_bytes);
+    p.acc_bytes = (Hk != H) ? round_up(sizeof(float) * (size_t)p.f.Ttot * H * dk, kAlign) : 0;
+    p.total_bytes = sizeof(WsHeader) + p.f.off_bytes + units * (p.slot_bytes + 2 * p.state_bytes + p.scr_bytes) +
+                    2 * p.acc_bytes;
     return KDA_OK;
 }
 
@@ -239,11 +243,15 @@ kda_status kda_decode_step(const void* q, const void* k, const void* v, const fl
 }
 
 kda_status kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int varlen, int num_seqs,
-                                        kda_dtype dt, size_t* bytes)
+                                        kda_dtype dt, const kda_options* opt, size_t* bytes)
 {
     if (!bytes) return KDA_ERR_INVALID_ARG;
+    int Hk = H;
+    unsigned pro = 0;
+    const kda_status so = parse_options(opt, H, Hk, pro);
+    if (so != KDA_OK) return so;
     BwdPlan p;
-    const kda_status st = make_bwd_plan(B, T, H, dk, dv, varlen != 0, num_seqs, dt, p);
+    const kda_status st = make_bwd_plan(B, T, H, Hk, dk, dv, varlen != 0, num_seqs, dt, p);
     if (st != KDA_OK) return st;
     *bytes = p.total_bytes;
     return KDA_OK;
@@ -260,9 +268,9 @@ kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, const void
     unsigned pro = 0;
     const kda_status so = parse_options(opt, H, Hk, pro);
     if (so != KDA_OK) return so;
-    if (Hk != H || (pro & ~KDA_PROLOGUE_GATE_BF16)) return KDA_ERR_UNSUPPORTED;
+    if (pro & ~KDA_PROLOGUE_GATE_BF16) return KDA_ERR_UNSUPPORTED;
     BwdPlan p;
-    const kda_status st = make_bwd_plan(B, T, H, dk, dv, cu_seqlens != nullptr, num_seqs, dt, p);
+    const kda_status st = make_bwd_plan(B, T, H, Hk, dk, dv, cu_seqlens != nullptr, num_seqs, dt, p);
     if (st != KDA_OK) return st;
     if (p.f.Ttot > 0 && (!q || !k || !v || !log_alpha || !beta || !dout || !dq || !dk_out || !dv_out ||
                          !dlog_alpha || !dbeta))
@@ -281,6 +289,7 @@ kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, const void
     char* states = slots + units * p.slot_bytes;
     char* cot = states + units * p.state_bytes;
     char* scr = cot + units * p.state_bytes;
+    char* acc = scr + units * p.scr_bytes;  // grouped heads only
     {
         LaunchScope ls("chunk_table", stream);
         chunk_table_kernel<<<1, kTableThreads, 0, stream>>>(cu_seqlens, p.f.N, p.f.Tseq, p.f.Ttot, hdr, off,
@@ -290,13 +299,14 @@ kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, const void
     // the per-unit regions are indexed by (chunk, head) with the dense strides of the kernels
     const cudaError_t e = (dt == KDA_BF16)
         ? launch_simt_backward<__nv_bfloat16>(q, k, v, log_alpha, beta, S0, dout, dS_final, dq, dk_out, dv_out,
-                                              dlog_alpha, dbeta, dS0, hdr, off, cu_seqlens, p.f.Tseq, p.f.N, H, pro,
-                                              dk, dv, p.f.max_chunks, (float*)slots, (float*)states, (float*)cot,
-                                              (float*)scr, stream)
+                                              dlog_alpha, dbeta, dS0, hdr, off, cu_seqlens, p.f.Tseq, p.f.N, H, Hk,
+                                              pro, dk, dv, p.f.max_chunks, p.f.Ttot, (float*)slots, (float*)states,
+                                              (float*)cot, (float*)scr, (float*)acc, (float*)(acc + p.acc_bytes),
+                                              stream)
         : launch_simt_backward<float>(q, k, v, log_alpha, beta, S0, dout, dS_final, dq, dk_out, dv_out, dlog_alpha,
-                                      dbeta, dS0, hdr, off, cu_seqlens, p.f.Tseq, p.f.N, H, pro, dk, dv,
-                                      p.f.max_chunks, (float*)slots, (float*)states, (float*)cot, (float*)scr,
-                                      stream);
+                                      dbeta, dS0, hdr, off, cu_seqlens, p.f.Tseq, p.f.N, H, Hk, pro, dk, dv,
+                                      p.f.max_chunks, p.f.Ttot, (float*)slots, (float*)states, (float*)cot,
+                                      (float*)scr, (float*)acc, (float*)(acc + p.acc_bytes), stream);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

@@ -47,7 +47,8 @@ ABI = {
     "kda_decode_step_ex": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, ctypes.POINTER(KdaOptions), _P]),
     "kda_gated_rmsnorm": (_I, [_P, _P, _P, _P, ctypes.c_longlong, _I, _I, ctypes.c_float, _I, _I, _P]),
     "kda_chunk_fwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
-    "kda_chunk_bwd_workspace_size": (_I, [_I, _I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_SZ)]),
+    "kda_chunk_bwd_workspace_size": (_I, [_I, _I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(KdaOptions),
+                                         ctypes.POINTER(_SZ)]),
     "kda_chunk_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
                            ctypes.POINTER(KdaOptions), _P, _SZ, _P]),
     "kda_chunk_fwd_host_workspace_size": (_I, [_I, _I, _I, _I, _I, _I, ctypes.POINTER(KdaOptions), _I,
@@ -287,12 +288,14 @@ def chunk_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha:
 
 
 def bwd_workspace_size(B: int, T: int, H: int, dk: int, dv: int, varlen: bool = False, num_seqs: int = 0,
-                       dtype: torch.dtype = torch.bfloat16) -> int:
+                       dtype: torch.dtype = torch.bfloat16, qk_heads: Optional[int] = None) -> int:
     lib = load_library()
     n = ctypes.c_size_t(0)
     dt = KDA_BF16 if dtype == torch.bfloat16 else KDA_F32
+    opt = KdaOptions(num_qk_heads=qk_heads or 0, prologue=0)
     _check("kda_chunk_bwd_workspace_size",
-           lib.kda_chunk_bwd_workspace_size(B, T, H, dk, dv, int(bool(varlen)), num_seqs, dt, ctypes.byref(n)))
+           lib.kda_chunk_bwd_workspace_size(B, T, H, dk, dv, int(bool(varlen)), num_seqs, dt, ctypes.byref(opt),
+                                            ctypes.byref(n)))
     return n.value
 
 
@@ -303,22 +306,22 @@ def chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torc
     """Backward pass of ``chunk_fwd`` (``kda_chunk_bwd``): the derivatives of
     ``L = sum(dout * out) + sum(dS_final * S_final)`` with respect to every input.
 
-    Inputs as ``chunk_fwd`` (one q/k head per value head; log_alpha fp32 or bf16) plus ``dout``
+    Inputs as ``chunk_fwd`` (q, k with H or Hk heads; log_alpha fp32 or bf16) plus ``dout``
     (layout and dtype of ``out``) and ``dS_final`` ([N, H, dk, dv] fp32 or None).  Returns a dict
     ``dq, dk, dv`` (dtype of q), ``dlog_alpha`` (fp32), ``dbeta`` (fp32) and ``dS0`` (fp32, or None
     when ``want_dS0`` is False).  ``grads`` may hold preallocated output tensors under those keys."""
     lib = load_library()
     _req(q, "q")
     dev, dtq = q.device, q.dtype
-    B, T, H, dk = q.shape
-    dv = v.shape[-1]
+    B, T, Hk, dk = q.shape
+    H, dv = v.shape[2], v.shape[-1]
     for t, name in ((k, "k"), (v, "v"), (dout, "dout")):
         _req(t, name, dtq, dev)
     _req(log_alpha, "log_alpha", None, dev)
     pro = _gate_bits(log_alpha, 0)
     _req(beta, "beta", torch.float32, dev)
     if k.shape != q.shape or tuple(log_alpha.shape) != (B, T, H, dk) or tuple(v.shape) != (B, T, H, dv) or \
-            tuple(beta.shape) != (B, T, H) or dout.shape != v.shape:
+            tuple(beta.shape) != (B, T, H) or dout.shape != v.shape or H % Hk != 0:
         raise ValueError("inconsistent shapes")
     N = B
     if cu_seqlens is not None:
@@ -346,12 +349,12 @@ def chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torc
     if not want_dS0:
         g["dS0"] = None
     sh = _stream_handle(stream, dev)
-    ws_bytes = bwd_workspace_size(B, T, H, dk, dv, cu_seqlens is not None, N, dtq)
+    ws_bytes = bwd_workspace_size(B, T, H, dk, dv, cu_seqlens is not None, N, dtq, qk_heads=Hk)
     if workspace is None:
         workspace = _get_workspace(ws_bytes, dev, sh)
     else:
         _req(workspace, "workspace", torch.uint8, dev)
-    opt = KdaOptions(num_qk_heads=0, prologue=pro)
+    opt = KdaOptions(num_qk_heads=Hk, prologue=pro)
     rc = lib.kda_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0), _ptr(cu_seqlens), N,
                            _ptr(dout), _ptr(dS_final), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]),
                            _ptr(g["dlog_alpha"]), _ptr(g["dbeta"]), _ptr(g["dS0"]), B, T, H, dk, dv, _dt(q),

@@ -231,17 +231,19 @@ kda_status kda_chunk_fwd_host(const void* q, const void* k, const void* v, const
  *   dS_final   [N, H, dk, dv] fp32, or NULL: dL/dS_final = 0.
  *   dq, dk     [B, T, H, dk] in dt;  dv [B, T, H, dv] in dt;  dlog_alpha [B, T, H, dk] fp32;
  *   dbeta      [B, T, H] fp32;  dS0 [N, H, dk, dv] fp32 or NULL (not wanted).  All written whole.
- *   opt        NULL, or num_qk_heads 0 / H and prologue 0 or KDA_PROLOGUE_GATE_BF16 (log_alpha in
- *              bf16); anything else returns KDA_ERR_UNSUPPORTED.
- *   workspace  >= kda_chunk_bwd_workspace_size(...) bytes, 256-byte aligned, owned by the caller
- *              (about 4 * 64 * max(dk, dv) * 4 bytes per (64-token chunk, head) plus the state and
- *              its cotangent for each chunk).
+ *   opt        NULL, or grouped q/k heads (num_qk_heads = Hk: q, k, dq, dk are [.., Hk, dk]; dq and dk
+ *              sum the contributions of the H / Hk value heads that read each q/k head) and prologue 0
+ *              or KDA_PROLOGUE_GATE_BF16 (log_alpha in bf16).  Other prologue bits return
+ *              KDA_ERR_UNSUPPORTED.
+ *   workspace  >= kda_chunk_bwd_workspace_size(...) bytes (same opt), 256-byte aligned, owned by
+ *              the caller: per (64-token chunk, head) the fp32 chunk intermediates, the chunk's state
+ *              and its cotangent; with grouped heads also two fp32 [T, H, dk] buffers.
  * Pointers 16-byte aligned (cu_seqlens 4), device memory, no overlap between outputs and inputs.
  * Errors: as kda_chunk_fwd.  Asynchronous on `stream`; a malformed cu_seqlens sets the device
  * error word (read by kda_check) and computes nothing.
  */
 kda_status kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int varlen, int num_seqs,
-                                        kda_dtype dt, size_t* bytes);
+                                        kda_dtype dt, const kda_options* opt, size_t* bytes);
 kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, const void* log_alpha, const float* beta,
                          const float* S0, const int32_t* cu_seqlens, int num_seqs, const void* dout,
                          const float* dS_final, void* dq, void* dk, void* dv, float* dlog_alpha, float* dbeta,

@@ -165,3 +165,22 @@ def test_backward_prefill_32k_sampled():
         got = gr[key][:, heads] if key == "dS0" else gr[key][:, :, heads]
         e = max_rel(np64(got), ref[key])
         assert e <= BWD_TOL["bf16"][key], f"{key}: {e:.3e}"
+
+
+@pytest.mark.parametrize("dtype,d,H,Hk,T", [("bf16", 128, 4, 2, 200), ("f32", 64, 6, 3, 150), ("bf16", 128, 4, 1, 97)])
+def test_backward_grouped_heads(dtype, d, H, Hk, T):
+    """Grouped q/k heads (num_qk_heads = Hk): dq and dk come back with Hk heads, each the sum over the
+    value heads that read it (the oracle repeats q/k per value head and sums)."""
+    w = synth.Workload("bwdg", "prefill", 2, T, H, d, d, dtype, 61, s0_std=0.5)
+    inp = synth.prefill_inputs(w)
+    inp["q"] = inp["q"][:, :, :Hk].contiguous()
+    inp["k"] = inp["k"][:, :, :Hk].contiguous()
+    run_and_compare(inp, dtype)
+
+
+def test_backward_grouped_varlen():
+    w = synth.Workload("bwdgv", "prefill", 1, 0, 6, 128, 128, "bf16", 62, s0_std=0.5)
+    inp = synth.prefill_inputs(w, lengths=[70, 1, 130, 64])
+    inp["q"] = inp["q"][:, :, :2].contiguous()
+    inp["k"] = inp["k"][:, :, :2].contiguous()
+    run_and_compare(inp, "bf16")

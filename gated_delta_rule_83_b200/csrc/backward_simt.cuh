@@ -766,20 +766,99 @@ bwd_gate_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const void
     }
 }
 
-// grouped q/k heads: dq[t][hk][c] = sum over the G value heads hk*G .. hk*G+G-1 of the per-value-head
-// gradients (value head h reads q/k head h / G)
+// ------------------------------------------------------------------------------------------------
+// Input prologue, forwards and backwards.  Before the backward proper, the transforms of the
+// forward's prologue are applied once into the workspace (q/k normalised and rounded to the input
+// precision as the forward does, log alpha = log sigmoid(a), beta = sigmoid(b)), so every kernel
+// below sees the inputs the forward used.  Afterwards the gradients are carried back to the raw
+// inputs: dx = dx_hat / n - x (x . dx_hat) / n^3 for the norm (n = sqrt(sum x^2 + eps); the
+// rounding to the input precision is passed straight through), da = dlog_alpha sigmoid(-a),
+// db = dbeta sigmoid(b) (1 - sigmoid(b)).
+// ------------------------------------------------------------------------------------------------
+constexpr int kRowWarps = 8;  // one warp per (token, head) row, 8 rows per CTA
+
 template <typename TIn>
+__global__ void __launch_bounds__(32 * kRowWarps)
+bwd_qk_norm_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, TIn* __restrict__ qn, TIn* __restrict__ kn,
+                   long long rows, int dk)
+{
+    const long long row = (long long)blockIdx.x * kRowWarps + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31, per = dk / 32;
+    if (row >= rows) return;
+    const TIn* src = blockIdx.y ? k : q;
+    TIn* dst = blockIdx.y ? kn : qn;
+    float x[4], ss = 0.f;
+    for (int m = 0; m < per; ++m) {
+        x[m] = to_f32(src[(size_t)row * dk + lane + 32 * m]);
+        ss = fmaf(x[m], x[m], ss);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float inv = rsqrtf(ss + kQkNormEps);
+    for (int m = 0; m < per; ++m) dst[(size_t)row * dk + lane + 32 * m] = from_f32<TIn>(x[m] * inv);
+}
+
+// log alpha = log sigmoid(a) (gate logits, fp32 or bf16) and beta = sigmoid(b), into fp32 buffers
 __global__ void __launch_bounds__(256)
-bwd_group_sum_kernel(const float* __restrict__ acc, TIn* __restrict__ out, long long n_out, int G, int dk)
+bwd_gate_act_kernel(const void* __restrict__ la, bool la16, bool logits, float* __restrict__ la_out, long long n_la,
+                    const float* __restrict__ beta, float* __restrict__ beta_out, long long n_beta)
 {
     const long long e = (long long)blockIdx.x * 256 + threadIdx.x;
-    if (e >= n_out) return;
-    const long long row = e / dk;  // (t, hk)
-    const int c = (int)(e - row * dk);
-    const float* src = acc + (size_t)row * G * dk + c;  // rows t*H + hk*G + g are consecutive
-    float s = 0.f;
-    for (int g = 0; g < G; ++g) s += src[(size_t)g * dk];
-    out[e] = from_f32<TIn>(s);
+    if (la_out && e < n_la) {
+        const float x = la16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(la)[e])
+                             : reinterpret_cast<const float*>(la)[e];
+        la_out[e] = logits ? log_sigmoid_f(x) : x;
+    }
+    if (beta_out && e < n_beta) beta_out[e] = sigmoid_f(beta[e]);
+}
+
+// dq, dk of the raw q/k heads: sum over the G value heads of each q/k head (value head h reads q/k
+// head h / G; rows t*H + hk*G + g are consecutive in acc), then, with the norm, its chain rule
+template <typename TIn>
+__global__ void __launch_bounds__(32 * kRowWarps)
+bwd_qk_grad_kernel(const float* __restrict__ acc, const TIn* __restrict__ x_raw, TIn* __restrict__ out, long long rows,
+                   int G, int dk, bool l2norm)
+{
+    const long long row = (long long)blockIdx.x * kRowWarps + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31, per = dk / 32;
+    if (row >= rows) return;
+    float g[4], x[4], ss = 0.f, dot = 0.f;
+    for (int m = 0; m < per; ++m) {
+        const int c = lane + 32 * m;
+        float s = 0.f;
+        for (int j = 0; j < G; ++j) s += acc[((size_t)row * G + j) * dk + c];
+        g[m] = s;
+        x[m] = l2norm ? to_f32(x_raw[(size_t)row * dk + c]) : 0.f;
+        ss = fmaf(x[m], x[m], ss);
+        dot = fmaf(x[m], g[m], dot);
+    }
+    if (l2norm) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            dot += __shfl_xor_sync(0xffffffffu, dot, o);
+        }
+        const float inv = rsqrtf(ss + kQkNormEps), inv3 = inv * inv * inv;
+        for (int m = 0; m < per; ++m) g[m] = g[m] * inv - x[m] * dot * inv3;
+    }
+    for (int m = 0; m < per; ++m) out[(size_t)row * dk + lane + 32 * m] = from_f32<TIn>(g[m]);
+}
+
+// in place: dlog_alpha *= sigmoid(-a) for gate logits a; dbeta *= sigmoid(b) (1 - sigmoid(b))
+__global__ void __launch_bounds__(256)
+bwd_gate_act_grad_kernel(const void* __restrict__ la, bool la16, float* __restrict__ dla, long long n_la,
+                         const float* __restrict__ beta, float* __restrict__ dbeta, long long n_beta)
+{
+    const long long e = (long long)blockIdx.x * 256 + threadIdx.x;
+    if (dla && e < n_la) {
+        const float a = la16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(la)[e])
+                             : reinterpret_cast<const float*>(la)[e];
+        dla[e] *= sigmoid_f(-a);
+    }
+    if (dbeta && e < n_beta) {
+        const float sb = sigmoid_f(beta[e]);
+        dbeta[e] *= sb * (1.f - sb);
+    }
 }
 
 inline size_t bwd_fwd_chain_smem(int dk, int dv)
@@ -835,10 +914,42 @@ template <typename TIn>
 cudaError_t launch_simt_backward(const void* q, const void* k, const void* v, const void* la, const float* beta,
                                  const float* S0, const void* dout, const float* dS_final, void* dq, void* dk_out,
                                  void* dv_out, float* dla, float* dbeta, float* dS0, const WsHeader* hdr,
-                                 const int* off, const int32_t* cu, int Tseq, int N, int H, int Hk, unsigned pro,
+                                 const int* off, const int32_t* cu, int Tseq, int N, int H, int Hk, unsigned pro_raw,
                                  int dk, int dv, int max_chunks, long long Ttot, float* slots, float* S_chunks,
-                                 float* dSn_chunks, float* scr, float* dq_acc, float* dk_acc, cudaStream_t stream)
+                                 float* dSn_chunks, float* scr, float* dq_acc, float* dk_acc, void* qn, void* kn,
+                                 float* la_act, float* beta_act, cudaStream_t stream)
 {
+    // the raw inputs, and the transformed ones every kernel below reads (the input prologue)
+    const void *q_raw = q, *k_raw = k, *la_raw = la;
+    const float* beta_raw = beta;
+    const bool grouped = Hk != H, l2norm = (pro_raw & KDA_PROLOGUE_L2NORM_QK) != 0;
+    unsigned pro = pro_raw & KDA_PROLOGUE_GATE_BF16;
+    cudaError_t e0 = cudaSuccess;
+    if (l2norm && Ttot > 0) {
+        LaunchScope ls("bwd_qk_norm", stream);
+        const long long rows = Ttot * Hk, blocks = (rows + kRowWarps - 1) / kRowWarps;
+        if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+        bwd_qk_norm_kernel<TIn><<<dim3((unsigned)blocks, 2), 32 * kRowWarps, 0, stream>>>(
+            (const TIn*)q, (const TIn*)k, (TIn*)qn, (TIn*)kn, rows, dk);
+        if ((e0 = cudaGetLastError()) != cudaSuccess) return e0;
+        q = qn;
+        k = kn;
+    }
+    if ((pro_raw & (KDA_PROLOGUE_GATE_LOGITS | KDA_PROLOGUE_BETA_LOGITS)) && Ttot > 0) {
+        LaunchScope ls("bwd_gate_act", stream);
+        const bool gl = (pro_raw & KDA_PROLOGUE_GATE_LOGITS) != 0, bl = (pro_raw & KDA_PROLOGUE_BETA_LOGITS) != 0;
+        const long long n_la = Ttot * H * dk, blocks = (n_la + 255) / 256;
+        if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+        bwd_gate_act_kernel<<<(unsigned)blocks, 256, 0, stream>>>(la, (pro_raw & KDA_PROLOGUE_GATE_BF16) != 0, true,
+                                                                   gl ? la_act : nullptr, n_la, beta,
+                                                                   bl ? beta_act : nullptr, Ttot * H);
+        if ((e0 = cudaGetLastError()) != cudaSuccess) return e0;
+        if (gl) {
+            la = la_act;
+            pro = 0;  // the activated gates are fp32
+        }
+        if (bl) beta = beta_act;
+    }
     const size_t smA = simt_intra_smem(dk, dv), smS = bwd_state_side_smem(dk, dv), smU = bwd_ut_smem(),
                  smG = bwd_gate_smem();
     cudaError_t e = cudaFuncSetAttribute(simt_intra_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smA);
@@ -877,19 +988,30 @@ cudaError_t launch_simt_backward(const void* q, const void* k, const void* v, co
         }
         {
             LaunchScope ls("bwd_gate", stream);
-            const bool grouped = Hk != H;
             bwd_gate_kernel<TIn><<<dim3(max_chunks, H, dk / kBwdCT), kSimtThreads, smG, stream>>>(
                 qq, kk, la, beta, hdr, off, cu, Tseq, N, H, Hk, pro & KDA_PROLOGUE_GATE_BF16, dk, dv, scr, (TIn*)dq,
-                (TIn*)dk_out, dla, grouped ? dq_acc : nullptr, grouped ? dk_acc : nullptr);
+                (TIn*)dk_out, dla, (grouped || l2norm) ? dq_acc : nullptr, (grouped || l2norm) ? dk_acc : nullptr);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
         }
-        if (Hk != H) {
-            LaunchScope ls("bwd_group_sum", stream);
-            const long long n_out = Ttot * Hk * dk;
-            const long long blocks = (n_out + 255) / 256;
+        if (grouped || l2norm) {  // per-value-head dq, dk -> the raw q/k heads
+            LaunchScope ls("bwd_qk_grad", stream);
+            const long long rows = Ttot * Hk, blocks = (rows + kRowWarps - 1) / kRowWarps;
             if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
-            bwd_group_sum_kernel<TIn><<<(unsigned)blocks, 256, 0, stream>>>(dq_acc, (TIn*)dq, n_out, H / Hk, dk);
-            bwd_group_sum_kernel<TIn><<<(unsigned)blocks, 256, 0, stream>>>(dk_acc, (TIn*)dk_out, n_out, H / Hk, dk);
+            bwd_qk_grad_kernel<TIn><<<(unsigned)blocks, 32 * kRowWarps, 0, stream>>>(
+                dq_acc, (const TIn*)q_raw, (TIn*)dq, rows, H / Hk, dk, l2norm);
+            bwd_qk_grad_kernel<TIn><<<(unsigned)blocks, 32 * kRowWarps, 0, stream>>>(
+                dk_acc, (const TIn*)k_raw, (TIn*)dk_out, rows, H / Hk, dk, l2norm);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
+        if (pro_raw & (KDA_PROLOGUE_GATE_LOGITS | KDA_PROLOGUE_BETA_LOGITS)) {
+            LaunchScope ls("bwd_gate_act_grad", stream);
+            const long long n_la = Ttot * H * dk, n_b = Ttot * H;
+            const long long blocks = (n_la + 255) / 256;
+            if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+            const bool gl = (pro_raw & KDA_PROLOGUE_GATE_LOGITS) != 0, bl = (pro_raw & KDA_PROLOGUE_BETA_LOGITS) != 0;
+            bwd_gate_act_grad_kernel<<<(unsigned)blocks, 256, 0, stream>>>(
+                la_raw, (pro_raw & KDA_PROLOGUE_GATE_BF16) != 0, gl ? dla : nullptr, n_la, beta_raw,
+                bl ? dbeta : nullptr, n_b);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
         }
     }

@@ -86,12 +86,13 @@ kda_status make_plan(int B, int T, int H, int dk, int dv, bool varlen, int num_s
 // forward slot, the chunk's start state, its end cotangent and the state-side scratch.
 struct BwdPlan {
     Plan f;
-    size_t slot_bytes, state_bytes, scr_bytes, acc_bytes, total_bytes;
+    size_t slot_bytes, state_bytes, scr_bytes, acc_bytes, qk_bytes, la_bytes, beta_bytes, total_bytes;
 };
 
-// Hk < H (grouped q/k heads) adds two fp32 per-value-head buffers for dq and dk, summed per group
-kda_status make_bwd_plan(int B, int T, int H, int Hk, int dk, int dv, bool varlen, int num_seqs, kda_dtype dt,
-                         BwdPlan& p)
+// Hk < H (grouped q/k heads) or the q/k norm adds two fp32 per-value-head buffers for dq and dk;
+// the prologue bits add buffers for the transformed inputs (normalised q, k; activated gates, beta)
+kda_status make_bwd_plan(int B, int T, int H, int Hk, unsigned pro, int dk, int dv, bool varlen, int num_seqs,
+                         kda_dtype dt, BwdPlan& p)
 {
     const kda_status st = make_plan(B, T, H, dk, dv, varlen, num_seqs, dt, p.f);
     if (st != KDA_OK) return st;
@@ -100,9 +101,15 @@ kda_status make_bwd_plan(int B, int T, int H, int Hk, int dk, int dv, bool varle
     p.slot_bytes = sizeof(float) * simt_slot_floats(dk, dv);
     p.state_bytes = sizeof(float) * (size_t)dk * dv;
     p.scr_bytes = sizeof(float) * bwd_scr_floats(dk, dv);
-    p.acc_bytes = (Hk != H) ? round_up(sizeof(float) * (size_t)p.f.Ttot * H * dk, kAlign) : 0;
-    p.total_bytes = sizeof(WsHeader) + p.f.off_bytes + units * (p.slot_bytes + 2 * p.state_bytes + p.scr_bytes) +
-                    2 * p.acc_bytes;
+    const size_t Tt = (size_t)p.f.Ttot, esz = dt == KDA_BF16 ? 2 : 4;
+    const bool l2 = (pro & KDA_PROLOGUE_L2NORM_QK) != 0;
+    p.acc_bytes = (Hk != H || l2) ? round_up(sizeof(float) * Tt * H * dk, kAlign) : 0;
+    p.qk_bytes = l2 ? round_up(esz * Tt * Hk * dk, kAlign) : 0;
+    p.la_bytes = (pro & KDA_PROLOGUE_GATE_LOGITS) ? round_up(sizeof(float) * Tt * H * dk, kAlign) : 0;
+    p.beta_bytes = (pro & KDA_PROLOGUE_BETA_LOGITS) ? round_up(sizeof(float) * Tt * H, kAlign) : 0;
+    p.total_bytes = round_up(sizeof(WsHeader) + p.f.off_bytes +
+                             units * (p.slot_bytes + 2 * p.state_bytes + p.scr_bytes), kAlign) +
+                    2 * p.acc_bytes + 2 * p.qk_bytes + p.la_bytes + p.beta_bytes;
     return KDA_OK;
 }
 
@@ -251,7 +258,7 @@ kda_status kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int
     const kda_status so = parse_options(opt, H, Hk, pro);
     if (so != KDA_OK) return so;
     BwdPlan p;
-    const kda_status st = make_bwd_plan(B, T, H, Hk, dk, dv, varlen != 0, num_seqs, dt, p);
+    const kda_status st = make_bwd_plan(B, T, H, Hk, pro, dk, dv, varlen != 0, num_seqs, dt, p);
     if (st != KDA_OK) return st;
     *bytes = p.total_bytes;
     return KDA_OK;
@@ -268,9 +275,8 @@ kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, const void
     unsigned pro = 0;
     const kda_status so = parse_options(opt, H, Hk, pro);
     if (so != KDA_OK) return so;
-    if (pro & ~KDA_PROLOGUE_GATE_BF16) return KDA_ERR_UNSUPPORTED;
     BwdPlan p;
-    const kda_status st = make_bwd_plan(B, T, H, Hk, dk, dv, cu_seqlens != nullptr, num_seqs, dt, p);
+    const kda_status st = make_bwd_plan(B, T, H, Hk, pro, dk, dv, cu_seqlens != nullptr, num_seqs, dt, p);
     if (st != KDA_OK) return st;
     if (p.f.Ttot > 0 && (!q || !k || !v || !log_alpha || !beta || !dout || !dq || !dk_out || !dv_out ||
                          !dlog_alpha || !dbeta))
@@ -289,7 +295,12 @@ kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, const void
     char* states = slots + units * p.slot_bytes;
     char* cot = states + units * p.state_bytes;
     char* scr = cot + units * p.state_bytes;
-    char* acc = scr + units * p.scr_bytes;  // grouped heads only
+    char* acc = ws + round_up(sizeof(WsHeader) + p.f.off_bytes +
+                              units * (p.slot_bytes + 2 * p.state_bytes + p.scr_bytes), kAlign);
+    char* qn = acc + 2 * p.acc_bytes;  // prologue buffers (empty when their bit is off)
+    char* kn = qn + p.qk_bytes;
+    char* la_act = kn + p.qk_bytes;
+    char* beta_act = la_act + p.la_bytes;
     {
         LaunchScope ls("chunk_table", stream);
         chunk_table_kernel<<<1, kTableThreads, 0, stream>>>(cu_seqlens, p.f.N, p.f.Tseq, p.f.Ttot, hdr, off,
@@ -302,11 +313,12 @@ kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, const void
                                               dlog_alpha, dbeta, dS0, hdr, off, cu_seqlens, p.f.Tseq, p.f.N, H, Hk,
                                               pro, dk, dv, p.f.max_chunks, p.f.Ttot, (float*)slots, (float*)states,
                                               (float*)cot, (float*)scr, (float*)acc, (float*)(acc + p.acc_bytes),
-                                              stream)
+                                              qn, kn, (float*)la_act, (float*)beta_act, stream)
         : launch_simt_backward<float>(q, k, v, log_alpha, beta, S0, dout, dS_final, dq, dk_out, dv_out, dlog_alpha,
                                       dbeta, dS0, hdr, off, cu_seqlens, p.f.Tseq, p.f.N, H, Hk, pro, dk, dv,
                                       p.f.max_chunks, p.f.Ttot, (float*)slots, (float*)states, (float*)cot,
-                                      (float*)scr, (float*)acc, (float*)(acc + p.acc_bytes), stream);
+                                      (float*)scr, (float*)acc, (float*)(acc + p.acc_bytes), qn, kn,
+                                      (float*)la_act, (float*)beta_act, stream);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

@@ -288,11 +288,11 @@ def chunk_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha:
 
 
 def bwd_workspace_size(B: int, T: int, H: int, dk: int, dv: int, varlen: bool = False, num_seqs: int = 0,
-                       dtype: torch.dtype = torch.bfloat16, qk_heads: Optional[int] = None) -> int:
+                       dtype: torch.dtype = torch.bfloat16, qk_heads: Optional[int] = None, prologue: int = 0) -> int:
     lib = load_library()
     n = ctypes.c_size_t(0)
     dt = KDA_BF16 if dtype == torch.bfloat16 else KDA_F32
-    opt = KdaOptions(num_qk_heads=qk_heads or 0, prologue=0)
+    opt = KdaOptions(num_qk_heads=qk_heads or 0, prologue=prologue)
     _check("kda_chunk_bwd_workspace_size",
            lib.kda_chunk_bwd_workspace_size(B, T, H, dk, dv, int(bool(varlen)), num_seqs, dt, ctypes.byref(opt),
                                             ctypes.byref(n)))
@@ -302,14 +302,17 @@ def bwd_workspace_size(B: int, T: int, H: int, dk: int, dv: int, varlen: bool = 
 def chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor, beta: torch.Tensor,
               dout: torch.Tensor, S0: Optional[torch.Tensor] = None, dS_final: Optional[torch.Tensor] = None,
               cu_seqlens: Optional[torch.Tensor] = None, want_dS0: bool = True, grads: Optional[dict] = None,
-              workspace: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None) -> dict:
+              workspace: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None,
+              prologue: int = 0) -> dict:
     """Backward pass of ``chunk_fwd`` (``kda_chunk_bwd``): the derivatives of
     ``L = sum(dout * out) + sum(dS_final * S_final)`` with respect to every input.
 
     Inputs as ``chunk_fwd`` (q, k with H or Hk heads; log_alpha fp32 or bf16) plus ``dout``
     (layout and dtype of ``out``) and ``dS_final`` ([N, H, dk, dv] fp32 or None).  Returns a dict
     ``dq, dk, dv`` (dtype of q), ``dlog_alpha`` (fp32), ``dbeta`` (fp32) and ``dS0`` (fp32, or None
-    when ``want_dS0`` is False).  ``grads`` may hold preallocated output tensors under those keys."""
+    when ``want_dS0`` is False).  ``grads`` may hold preallocated output tensors under those keys.
+    ``prologue``: the PROLOGUE_* bits the forward call used; the gradients are then those of the raw
+    inputs."""
     lib = load_library()
     _req(q, "q")
     dev, dtq = q.device, q.dtype
@@ -318,7 +321,7 @@ def chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torc
     for t, name in ((k, "k"), (v, "v"), (dout, "dout")):
         _req(t, name, dtq, dev)
     _req(log_alpha, "log_alpha", None, dev)
-    pro = _gate_bits(log_alpha, 0)
+    pro = _gate_bits(log_alpha, prologue)
     _req(beta, "beta", torch.float32, dev)
     if k.shape != q.shape or tuple(log_alpha.shape) != (B, T, H, dk) or tuple(v.shape) != (B, T, H, dv) or \
             tuple(beta.shape) != (B, T, H) or dout.shape != v.shape or H % Hk != 0:
@@ -349,7 +352,7 @@ def chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torc
     if not want_dS0:
         g["dS0"] = None
     sh = _stream_handle(stream, dev)
-    ws_bytes = bwd_workspace_size(B, T, H, dk, dv, cu_seqlens is not None, N, dtq, qk_heads=Hk)
+    ws_bytes = bwd_workspace_size(B, T, H, dk, dv, cu_seqlens is not None, N, dtq, qk_heads=Hk, prologue=pro)
     if workspace is None:
         workspace = _get_workspace(ws_bytes, dev, sh)
     else:

@@ -231,10 +231,12 @@ kda_status kda_chunk_fwd_host(const void* q, const void* k, const void* v, const
  *   dS_final   [N, H, dk, dv] fp32, or NULL: dL/dS_final = 0.
  *   dq, dk     [B, T, H, dk] in dt;  dv [B, T, H, dv] in dt;  dlog_alpha [B, T, H, dk] fp32;
  *   dbeta      [B, T, H] fp32;  dS0 [N, H, dk, dv] fp32 or NULL (not wanted).  All written whole.
- *   opt        NULL, or grouped q/k heads (num_qk_heads = Hk: q, k, dq, dk are [.., Hk, dk]; dq and dk
- *              sum the contributions of the H / Hk value heads that read each q/k head) and prologue 0
- *              or KDA_PROLOGUE_GATE_BF16 (log_alpha in bf16).  Other prologue bits return
- *              KDA_ERR_UNSUPPORTED.
+ *   opt        NULL, or the options of the forward call: grouped q/k heads (num_qk_heads = Hk: q, k,
+ *              dq, dk are [.., Hk, dk]; dq and dk sum the contributions of the H / Hk value heads that
+ *              read each q/k head) and any KDA_PROLOGUE_* bits.  With prologue bits the inputs are the
+ *              raw ones the forward took and the gradients are those of the raw inputs: through the
+ *              q/k norm (its rounding to the input precision passed straight through), the
+ *              log-sigmoid of the gate logits and the sigmoid of the beta logits.
  *   workspace  >= kda_chunk_bwd_workspace_size(...) bytes (same opt), 256-byte aligned, owned by
  *              the caller: per (64-token chunk, head) the fp32 chunk intermediates, the chunk's state
  *              and its cotangent; with grouped heads also two fp32 [T, H, dk] buffers.

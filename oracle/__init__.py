@@ -24,7 +24,8 @@ step differentiated as written, walking the tokens backwards.
 ``gated_rmsnorm`` is the output gate (grouped RMS norm times the gate z).
 
 ``prologue`` is the input transform of the kernels' optional prologue (q/k L2 normalisation,
-log-sigmoid gate logits, sigmoid beta logits), applied in front of the other functions.
+log-sigmoid gate logits, sigmoid beta logits), applied in front of the other functions;
+``prologue_bwd`` carries gradients back through it (the chain rule of each transform).
 
 ``seq``, ``chunked`` and ``decode_step`` also take q and k with fewer heads than v (grouped heads:
 value head h reads q/k head h // (H // Hk)), as in the head-count comments of the review's GDN
@@ -277,6 +278,30 @@ def prologue(q, k, log_alpha, beta, l2norm_qk=False, gate_logits=False, beta_log
     if beta_logits:
         b = sp.expit(b)
     return q, k, la, b
+
+
+def prologue_bwd(q, k, log_alpha, beta, grads, l2norm_qk=False, gate_logits=False, beta_logits=False):
+    """The chain rule through ``prologue``: given the raw inputs and the gradients with respect to
+    the transformed ones (a dict from ``bwd`` on ``prologue``'s outputs), return the gradients with
+    respect to the raw inputs (a new dict; dv and dS0 pass through).  fp64 numpy:
+
+    * x_hat = x / n, n = sqrt(sum x^2 + eps):  dx = dx_hat / n - x (x . dx_hat) / n^3
+    * log_alpha = log sigmoid(a):              da = dlog_alpha * sigmoid(-a)
+    * beta = sigmoid(b):                       db = dbeta * sigmoid(b) (1 - sigmoid(b))"""
+    import scipy.special as sp
+    q, k, la, b = (np.asarray(x, dtype=np.float64) for x in (q, k, log_alpha, beta))
+    g = dict(grads)
+    if l2norm_qk:
+        for name, x in (("dq", q), ("dk", k)):
+            n = np.sqrt(np.sum(x * x, axis=-1, keepdims=True) + QK_NORM_EPS)
+            dxh = np.asarray(g[name], dtype=np.float64)
+            g[name] = dxh / n - x * np.sum(x * dxh, axis=-1, keepdims=True) / n ** 3
+    if gate_logits:
+        g["dlog_alpha"] = np.asarray(g["dlog_alpha"], dtype=np.float64) * sp.expit(-la)
+    if beta_logits:
+        s = sp.expit(b)
+        g["dbeta"] = np.asarray(g["dbeta"], dtype=np.float64) * s * (1.0 - s)
+    return g
 
 
 def gated_rmsnorm(o, z, weight=None, group=None, eps=1e-6, gate="none"):

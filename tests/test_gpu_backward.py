@@ -184,3 +184,46 @@ def test_backward_grouped_varlen():
     inp["q"] = inp["q"][:, :, :2].contiguous()
     inp["k"] = inp["k"][:, :, :2].contiguous()
     run_and_compare(inp, "bf16")
+
+
+@pytest.mark.parametrize("dtype,d,flags,Hk", [("bf16", 128, 7, 4), ("f32", 64, 7, 4), ("bf16", 128, 1, 2),
+                                               ("bf16", 128, 2, 4), ("f32", 128, 4, 4)])
+def test_backward_through_prologue(dtype, d, flags, Hk):
+    """The prologue bits of the forward (q/k L2 norm, gate logits, beta logits): gradients of the raw
+    inputs.  Reference: oracle.prologue (the kernels' rounding of the normalised q/k to the input
+    precision applied too), oracle.bwd on the transformed inputs, then oracle.prologue_bwd."""
+    m = kda()
+    g = torch.Generator().manual_seed(71)
+    B, T, H = 2, 150, 4
+    dt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    q = (torch.randn(B, T, Hk, d, generator=g) * 3.0).to(dt)
+    k = (torch.randn(B, T, Hk, d, generator=g) * 0.2).to(dt)
+    v = torch.randn(B, T, H, d, generator=g).to(dt)
+    a = torch.randn(B, T, H, d, generator=g) + 3.0
+    b = torch.randn(B, T, H, generator=g)
+    if not flags & 1:
+        q = torch.nn.functional.normalize(q.float(), dim=-1).to(dt)
+        k = torch.nn.functional.normalize(k.float(), dim=-1).to(dt)
+    if not flags & 2:
+        a = torch.nn.functional.logsigmoid(a)
+    if not flags & 4:
+        b = torch.sigmoid(b)
+    S0 = torch.randn(B, H, d, d, generator=g) * 0.3
+    do = torch.randn(B, T, H, d, generator=g).to(dt)
+    dsf = torch.randn(B, H, d, d, generator=g) * 0.5
+    gr = m.chunk_bwd(q.to(DEV), k.to(DEV), v.to(DEV), a.to(DEV), b.to(DEV), do.to(DEV), S0=S0.to(DEV),
+                     dS_final=dsf.to(DEV), prologue=flags)
+    m.check()
+    raw = [synth.to_oracle(x) for x in (q, k, a, b)]
+    fl = dict(l2norm_qk=bool(flags & 1), gate_logits=bool(flags & 2), beta_logits=bool(flags & 4))
+    qh, kh, la, bb = oracle.prologue(*raw, **fl)
+    if flags & 1:  # the kernels round the normalised q, k to the input precision
+        qh = torch.from_numpy(qh).to(dt).double().numpy()
+        kh = torch.from_numpy(kh).to(dt).double().numpy()
+    ref = oracle.bwd(qh, kh, synth.to_oracle(v), la, bb, do.double().numpy(), S0=S0.double().numpy(),
+                     dS_final=dsf.double().numpy())
+    ref = oracle.prologue_bwd(*raw, ref, **fl)
+    errs = {key: max_rel(np64(gr[key]), ref[key]) for key in KEYS}
+    tol = {key: max(t, 2e-3) for key, t in BWD_TOL[dtype].items()}  # fp32 prologue arithmetic on both ends
+    bad = {key: e for key, e in errs.items() if not e <= tol[key]}
+    assert not bad, f"gradient errors above tolerance: {bad} (all: {errs})"

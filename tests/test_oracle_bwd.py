@@ -159,3 +159,41 @@ def test_bwd_checkpoint_boundaries(T, o=oracle):
     fd = loss(plus, do, dsf, o) - loss(minus, do, dsf, o)
     an = float(np.sum(g["dlog_alpha"] * (2 * EPS * d)))
     assert abs(fd - an) <= 1e-5 * abs(an)
+
+
+def test_prologue_bwd_matches_finite_differences(o=oracle):
+    """The chain rule through the input prologue (L2-normalised q/k, log-sigmoid gate logits, sigmoid
+    beta logits), pinned by finite differences of the composition prologue -> recurrence.  The
+    transformed inputs are kept in fp64 on both sides of the difference (the oracle recurrence takes
+    float32, so the perturbation goes through the exact fp64 prologue and a float32 rounding that is
+    the same for the base point and the analytic side).  Catches: a missing 1/n or projection term in
+    the norm, sigma(a) in place of sigma(-a), a missing (1 - sigma) factor."""
+    rng = np.random.default_rng(21)
+    T, H, dk, dv = 9, 2, 4, 3
+    q = rng.standard_normal((T, H, dk)) * 2.0
+    k = rng.standard_normal((T, H, dk)) * 0.7
+    v = rng.standard_normal((T, H, dv))
+    a = rng.normal(2.0, 1.0, (T, H, dk))
+    b = rng.standard_normal((T, H))
+    do = rng.standard_normal((T, H, dv))
+    flags = dict(l2norm_qk=True, gate_logits=True, beta_logits=True)
+
+    def f(q_, k_, a_, b_):
+        qq, kk, la, bb = o.prologue(q_, k_, a_, b_, **flags)
+        out, _ = o.seq(qq, kk, v, la, bb)
+        return float(np.sum(out * do))
+
+    qq, kk, la, bb = o.prologue(q, k, a, b, **flags)
+    g = o.bwd(qq, kk, v, la, bb, do)
+    g = o.prologue_bwd(q, k, a, b, g, **flags)
+    eps = 1e-4
+    for name, key, x in (("q", "dq", q), ("k", "dk", k), ("a", "dlog_alpha", a), ("b", "dbeta", b)):
+        d = rng.standard_normal(x.shape)
+        args = dict(q_=q, k_=k, a_=a, b_=b)
+        plus, minus = dict(args), dict(args)
+        plus[name + "_"] = x + eps * d
+        minus[name + "_"] = x - eps * d
+        fd = (f(**plus) - f(**minus)) / (2 * eps)
+        an = float(np.sum(g[key] * d))
+        # float32 rounding of the transformed inputs inside the oracle recurrence bounds the agreement
+        assert abs(fd - an) <= 2e-3 * abs(an) + 1e-6, f"{name}: fd {fd!r} vs analytic {an!r}"

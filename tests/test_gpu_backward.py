@@ -227,3 +227,20 @@ def test_backward_through_prologue(dtype, d, flags, Hk):
     tol = {key: max(t, 2e-3) for key, t in BWD_TOL[dtype].items()}  # fp32 prologue arithmetic on both ends
     bad = {key: e for key, e in errs.items() if not e <= tol[key]}
     assert not bad, f"gradient errors above tolerance: {bad} (all: {errs})"
+
+
+def test_backward_empty_and_zero_length_sequences():
+    """Packed sequences of length 0 among others, and a call with no tokens at all: the empty
+    sequences get dS0 = dS_final and the others match the oracle."""
+    m = kda()
+    w = synth.Workload("bwde", "prefill", 1, 0, 2, 64, 64, "f32", 81, s0_std=0.5)
+    inp = synth.prefill_inputs(w, lengths=[0, 5, 0, 64, 3])
+    run_and_compare(inp, "f32")
+    # no tokens: every gradient is empty and dS0 equals dS_final
+    z = lambda *s: torch.zeros(*s, device=DEV)  # noqa: E731
+    cu = torch.tensor([0, 0, 0], dtype=torch.int32, device=DEV)
+    dsf = torch.randn(2, 2, 64, 64, device=DEV)
+    g = m.chunk_bwd(z(1, 0, 2, 64), z(1, 0, 2, 64), z(1, 0, 2, 64), z(1, 0, 2, 64), z(1, 0, 2), z(1, 0, 2, 64),
+                    S0=z(2, 2, 64, 64), dS_final=dsf, cu_seqlens=cu)
+    m.check()
+    assert torch.equal(g["dS0"], dsf)

@@ -12,9 +12,10 @@
 //   1. forward recompute: the CUDA-core phase A, then its phase B storing every chunk's start
 //      state S_c and its corrected values U.
 //   2. reverse chain over chunks (one CTA per (sequence, head, 32 state columns), chunks last to
-//      first), carrying D = dL/dS_next:
-//          dU = P^T dO + Kd D
-//          D <- Diag(gam) D + Qg^T dO - W^T dU          (= dL/dS at the chunk start)
+//      first), carrying D = dL/dS_next, with E = P^T dO and F = Qg^T dO computed chunk-parallel
+//      beforehand (they do not depend on D):
+//          dU = E + Kd D
+//          D <- Diag(gam) D + F - W^T dU                 (= dL/dS at the chunk start)
 //      storing every chunk's end cotangent D_c and dU; D after the first chunk is dL/dS0.
 //   3. chunk-parallel, state side (one CTA per (chunk, head)): with S_c, D_c, U and dU,
 //          dQg = dO S_c^T,  dW = -dU S_c^T,  dKd = U D_c^T,  dP = lower_incl(dO U^T),
@@ -169,79 +170,121 @@ bwd_fwd_chain_kernel(const float* __restrict__ S0, const WsHeader* __restrict__ 
 }
 
 // ------------------------------------------------------------------------------------------------
-// Step 2: reverse chain of the state cotangent (chunks last to first).  {P, Kd} and {Qg, W, gam}
-// of the next chunk are copied while the current chunk's other half computes; dO of the next chunk
-// is loaded into registers one half-step ahead.
+// Step 2a: the dO terms of the reverse chain, chunk-parallel (one CTA per (chunk, head)):
+//     E = P^T dO  (64 x dv, into the unit's dU scratch),   F = Qg^T dO  (dk x dv)
+// Neither depends on the carried cotangent, so the chain itself only does the D-dependent half.
 // ------------------------------------------------------------------------------------------------
-template <typename TIn, int DK>
+template <typename TIn, int DK, int DV>
+__global__ void __launch_bounds__(kSimtThreads, 2)
+bwd_do_terms_kernel(const TIn* __restrict__ dout, const WsHeader* __restrict__ hdr, const int* __restrict__ off,
+                    const int32_t* __restrict__ cu, int Tseq, int N, int H, const float* __restrict__ slots,
+                    float* __restrict__ scr, float* __restrict__ F_chunks)
+{
+    extern __shared__ __align__(16) float smem[];
+    const int j = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+    if (hdr->bad || j >= hdr->total_chunks) return;
+    int n, L;
+    long long t0;
+    locate_chunk(j, off, cu, Tseq, N, n, t0, L);
+    constexpr int L64 = kChunk + 1, LK = DK + 1, LV = DV + 1;
+    float* sP = smem;                 // [64][65]
+    float* sQ = sP + kChunk * L64;    // [64][DK+1]  Qg
+    float* sO = sQ + kChunk * LK;     // [64][DV+1]  dO (rows past the end zero)
+    const size_t u = (size_t)j * H + h;
+    const float* slot = slots + u * simt_slot_floats(DK, DV);
+    const float* gQ = slot + (size_t)kChunk * DK;
+    const float* gP = slot + 3 * (size_t)kChunk * DK;
+    for (int e = tid; e < kChunk * kChunk; e += kSimtThreads) sP[(e / kChunk) * L64 + (e % kChunk)] = gP[e];
+    for (int e = tid; e < kChunk * DK; e += kSimtThreads) sQ[(e / DK) * LK + (e % DK)] = gQ[e];
+    for (int e = tid; e < kChunk * DV; e += kSimtThreads) {
+        const int r = e / DV, jj = e % DV;
+        sO[r * LV + jj] = (r < L) ? to_f32(dout[((size_t)(t0 + r) * H + h) * DV + jj]) : 0.f;
+    }
+    __syncthreads();
+    const int tr = tid >> 4, tc = tid & 15;
+    {   // E = P^T dO
+        float acc[4][DV / 16] = {};
+        mm_acc<4, DV / 16>(acc, sP, 1, L64, sO, LV, 1, kChunk, tr, tc);
+        float* gE = scr + u * bwd_scr_floats(DK, DV) + (size_t)kChunk * DV;
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < DV / 16; ++b) gE[(size_t)(tr + 16 * a) * DV + tc + 16 * b] = acc[a][b];
+    }
+    float* gF = F_chunks + u * DK * DV;
+#pragma unroll 1
+    for (int c0 = 0; c0 < DK; c0 += kChunk) {  // F = Qg^T dO, 64 rows at a time
+        float acc[4][DV / 16] = {};
+        mm_acc<4, DV / 16>(acc, sQ + c0, 1, LK, sO, LV, 1, kChunk, tr, tc);
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < DV / 16; ++b) gF[(size_t)(c0 + tr + 16 * a) * DV + tc + 16 * b] = acc[a][b];
+    }
+}
+
+// ------------------------------------------------------------------------------------------------
+// Step 2b: reverse chain of the state cotangent (chunks last to first):
+//     dU = E + Kd D,   D <- Diag(gam) D + F - W^T dU
+// {Kd, E} and {W, F, gam} of the next chunk are copied while the current chunk's other half runs.
+// ------------------------------------------------------------------------------------------------
+template <int DK>
 __global__ void __launch_bounds__(kSimtThreads)
-bwd_dstate_kernel(const TIn* __restrict__ dout, const float* __restrict__ dS_final, float* __restrict__ dS0,
-                  const WsHeader* __restrict__ hdr, const int* __restrict__ off, const int32_t* __restrict__ cu,
-                  int Tseq, int N, int H, int dv, const float* __restrict__ slots, float* __restrict__ dSn_chunks,
-                  float* __restrict__ scr)
+bwd_dstate_kernel(const float* __restrict__ dS_final, float* __restrict__ dS0, const WsHeader* __restrict__ hdr,
+                  const int* __restrict__ off, int N, int H, int dv, const float* __restrict__ slots,
+                  float* __restrict__ dSn_chunks, float* __restrict__ scr, const float* __restrict__ F_chunks)
 {
     extern __shared__ __align__(16) float smem[];
     const int n = blockIdx.x, h = blockIdx.y, v0 = blockIdx.z * kSimtNV, tid = threadIdx.x;
     if (hdr->bad) return;
     constexpr int NV = kSimtNV, TMD = DK / 16;
-    constexpr int OPT = kChunk * NV / kSimtThreads;  // dO elements per thread
     float* sD = smem;                 // [DK][NV]   D = dL/dS
     float* sW = sD + DK * NV;         // [64][DK]
-    float* sQ = sW + kChunk * DK;     // [64][DK]
-    float* sKd = sQ + kChunk * DK;    // [64][DK]
-    float* sP = sKd + kChunk * DK;    // [64][64]
-    float* sO = sP + kChunk * kChunk; // [64][NV]   dO
-    float* sU = sO + kChunk * NV;     // [64][NV]   dU
-    float* sG = sU + kChunk * NV;     // [DK]
+    float* sKd = sW + kChunk * DK;    // [64][DK]
+    float* sE = sKd + kChunk * DK;    // [64][NV]   E
+    float* sU = sE + kChunk * NV;     // [64][NV]   dU
+    float* sF = sU + kChunk * NV;     // [DK][NV]
+    float* sG = sF + DK * NV;         // [DK]
     const int tr = tid >> 4, tc = tid & 15;
     const size_t slot_f = simt_slot_floats(DK, dv), scr_f = bwd_scr_floats(DK, dv);
     const size_t sidx = ((size_t)n * H + h) * DK * dv;
     for (int e = tid; e < DK * NV; e += kSimtThreads)
         sD[e] = dS_final ? dS_final[sidx + (size_t)(e / NV) * dv + v0 + (e % NV)] : 0.f;
-    long long s0, s1;
-    seq_bounds(n, cu, Tseq, s0, s1);
     const int j0 = off[n], j1 = off[n + 1];
-    auto issue_pk = [&](int j) {
-        const float* slot = slots + ((size_t)j * H + h) * slot_f;
-        bwd_cp_block(sKd, slot + 2 * (size_t)kChunk * DK, kChunk * DK);
-        bwd_cp_block(sP, slot + 3 * (size_t)kChunk * DK, kChunk * kChunk);
+    auto issue_k = [&](int j) {  // Kd and the E columns of chunk j
+        const size_t u = (size_t)j * H + h;
+        bwd_cp_block(sKd, slots + u * slot_f + 2 * (size_t)kChunk * DK, kChunk * DK);
+        const float* gE = scr + u * scr_f + (size_t)kChunk * dv + v0;
+        for (int e = 4 * tid; e < kChunk * NV; e += 4 * kSimtThreads)
+            bwd_cp16(sE + e, gE + (size_t)(e / NV) * dv + (e % NV), 16);
         bwd_cp_commit();
     };
-    auto issue_qw = [&](int j) {
-        const float* slot = slots + ((size_t)j * H + h) * slot_f;
+    auto issue_w = [&](int j) {  // W, the F columns and gam of chunk j
+        const size_t u = (size_t)j * H + h;
+        const float* slot = slots + u * slot_f;
         bwd_cp_block(sW, slot, kChunk * DK);
-        bwd_cp_block(sQ, slot + (size_t)kChunk * DK, kChunk * DK);
+        const float* gF = F_chunks + u * DK * dv + v0;
+        for (int e = 4 * tid; e < DK * NV; e += 4 * kSimtThreads)
+            bwd_cp16(sF + e, gF + (size_t)(e / NV) * dv + (e % NV), 16);
         bwd_cp_block(sG, slot + (size_t)kChunk * (3 * DK + kChunk + dv), DK);
         bwd_cp_commit();
     };
-    float od[OPT];  // dO of the chunk about to be processed, rows past its end zero
-    auto load_do = [&](int j) {
-        long long t0;
-        int L;
-        bwd_chunk_span(j, n, off, s0, s1, t0, L);
-#pragma unroll
-        for (int m = 0; m < OPT; ++m) {
-            const int e = tid + m * kSimtThreads, r = e / NV, jj = e % NV;
-            od[m] = (r < L) ? to_f32(dout[((size_t)(t0 + r) * H + h) * dv + v0 + jj]) : 0.f;
-        }
-    };
     if (j0 < j1) {
-        issue_pk(j1 - 1);
-        issue_qw(j1 - 1);
-        load_do(j1 - 1);
+        issue_k(j1 - 1);
+        issue_w(j1 - 1);
     }
     for (int j = j1 - 1; j >= j0; --j) {
         const size_t u = (size_t)j * H + h;
-        bwd_cp_wait<1>();  // P, Kd of chunk j
-        __syncthreads();   // ... visible to all, and the previous step is done with D and dO
-#pragma unroll
-        for (int m = 0; m < OPT; ++m) sO[tid + m * kSimtThreads] = od[m];
+        bwd_cp_wait<1>();  // Kd, E of chunk j
+        __syncthreads();   // ... visible to all, and the previous step is done with D
         float* dst = dSn_chunks + u * DK * dv + v0;
         for (int e = tid; e < DK * NV; e += kSimtThreads) dst[(size_t)(e / NV) * dv + (e % NV)] = sD[e];
-        __syncthreads();
-        {  // dU = P^T dO + Kd D
-            float x[4][2] = {};
-            mm_acc<4, 2>(x, sP, 1, kChunk, sO, NV, 1, kChunk, tr, tc);
+        {  // dU = E + Kd D
+            float x[4][2];
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int b = 0; b < 2; ++b) x[a][b] = sE[(tr + 16 * a) * NV + tc + 16 * b];
             mm_acc<4, 2>(x, sKd, DK, 1, sD, NV, 1, DK, tr, tc);
             float* gdU = scr + u * scr_f + (size_t)kChunk * dv + v0;
 #pragma unroll
@@ -253,27 +296,28 @@ bwd_dstate_kernel(const TIn* __restrict__ dout, const float* __restrict__ dS_fin
                     gdU[(size_t)i * dv + jj] = x[a][b];
                 }
         }
-        __syncthreads();
-        if (j > j0) issue_pk(j - 1);
+        __syncthreads();  // dU complete; Kd and E are free for the next chunk
+        if (j > j0) issue_k(j - 1);
         else bwd_cp_commit();
-        bwd_cp_wait<1>();  // Qg, W, gam of chunk j
+        bwd_cp_wait<1>();  // W, F, gam of chunk j
         __syncthreads();
-        {  // D <- Diag(gam) D + Qg^T dO - W^T dU
+        {  // D <- Diag(gam) D + F - W^T dU
             float acc[TMD][2], neg[TMD][2] = {};
 #pragma unroll
             for (int a = 0; a < TMD; ++a)
 #pragma unroll
-                for (int b = 0; b < 2; ++b) acc[a][b] = sG[tr + 16 * a] * sD[(tr + 16 * a) * NV + tc + 16 * b];
-            mm_acc<TMD, 2>(acc, sQ, 1, DK, sO, NV, 1, kChunk, tr, tc);
+                for (int b = 0; b < 2; ++b) {
+                    const int c = tr + 16 * a, jj = tc + 16 * b;
+                    acc[a][b] = fmaf(sG[c], sD[c * NV + jj], sF[c * NV + jj]);
+                }
             mm_acc<TMD, 2>(neg, sW, 1, DK, sU, NV, 1, kChunk, tr, tc);
-            if (j > j0) load_do(j - 1);
-            __syncthreads();  // every thread has read the old D, Qg, W
+            __syncthreads();  // every thread has read the old D, W, F
 #pragma unroll
             for (int a = 0; a < TMD; ++a)
 #pragma unroll
                 for (int b = 0; b < 2; ++b) sD[(tr + 16 * a) * NV + tc + 16 * b] = acc[a][b] - neg[a][b];
         }
-        if (j > j0) issue_qw(j - 1);
+        if (j > j0) issue_w(j - 1);
         else bwd_cp_commit();
     }
     bwd_cp_wait<0>();
@@ -869,7 +913,11 @@ inline size_t bwd_fwd_chain_smem(int dk, int dv)
 inline size_t bwd_dstate_smem(int dk, int dv)
 {
     (void)dv;
-    return sizeof(float) * ((size_t)dk * kSimtNV + 3 * kChunk * dk + kChunk * kChunk + 2 * kChunk * kSimtNV + dk);
+    return sizeof(float) * ((size_t)2 * dk * kSimtNV + 2 * kChunk * dk + 2 * kChunk * kSimtNV + dk);
+}
+inline size_t bwd_do_terms_smem(int dk, int dv)
+{
+    return sizeof(float) * ((size_t)kChunk * (kChunk + 1) + kChunk * (dk + 1) + kChunk * (dv + 1));
 }
 inline size_t bwd_state_side_smem(int dk, int dv)
 {
@@ -885,26 +933,36 @@ inline size_t bwd_gate_smem()
     return sizeof(float) * ((size_t)3 * kChunk * kBwdL64 + 7 * kChunk * kBwdLT + kChunk + kBwdCT);
 }
 
-template <typename TIn, int DK>
+template <typename TIn, int DK, int DV>
 cudaError_t launch_bwd_chains(const float* S0, const void* dout, const float* dS_final, float* dS0,
-                              const WsHeader* hdr, const int* off, const int32_t* cu, int Tseq, int N, int H, int dv,
-                              const float* slots, float* S_chunks, float* dSn_chunks, float* scr, cudaStream_t stream)
+                              const WsHeader* hdr, const int* off, const int32_t* cu, int Tseq, int N, int H,
+                              int max_chunks, const float* slots, float* S_chunks, float* dSn_chunks, float* scr,
+                              float* F_chunks, cudaStream_t stream)
 {
-    const size_t smF = bwd_fwd_chain_smem(DK, dv), smD = bwd_dstate_smem(DK, dv);
+    const size_t smF = bwd_fwd_chain_smem(DK, DV), smD = bwd_dstate_smem(DK, DV), smT = bwd_do_terms_smem(DK, DV);
     cudaError_t e = cudaFuncSetAttribute(bwd_fwd_chain_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smF);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(bwd_dstate_kernel<TIn, DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smD);
+        e = cudaFuncSetAttribute(bwd_dstate_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smD);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(bwd_do_terms_kernel<TIn, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smT);
     if (e != cudaSuccess) return e;
-    const dim3 grid(N, H, dv / kSimtNV);
+    const dim3 grid(N, H, DV / kSimtNV);
     {
         LaunchScope ls("bwd_fwd_states", stream);
-        bwd_fwd_chain_kernel<DK><<<grid, kSimtThreads, smF, stream>>>(S0, hdr, off, cu, Tseq, N, H, dv, slots,
+        bwd_fwd_chain_kernel<DK><<<grid, kSimtThreads, smF, stream>>>(S0, hdr, off, cu, Tseq, N, H, DV, slots,
                                                                       S_chunks, scr);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
+    if (max_chunks > 0) {
+        LaunchScope ls("bwd_do_terms", stream);
+        bwd_do_terms_kernel<TIn, DK, DV><<<dim3(max_chunks, H), kSimtThreads, smT, stream>>>(
+            (const TIn*)dout, hdr, off, cu, Tseq, N, H, slots, scr, F_chunks);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     LaunchScope ls("bwd_dstate", stream);
-    bwd_dstate_kernel<TIn, DK><<<grid, kSimtThreads, smD, stream>>>((const TIn*)dout, dS_final, dS0, hdr, off, cu,
-                                                                   Tseq, N, H, dv, slots, dSn_chunks, scr);
+    bwd_dstate_kernel<DK><<<grid, kSimtThreads, smD, stream>>>(dS_final, dS0, hdr, off, N, H, DV, slots, dSn_chunks,
+                                                               scr, F_chunks);
     return cudaGetLastError();
 }
 
@@ -916,8 +974,8 @@ cudaError_t launch_simt_backward(const void* q, const void* k, const void* v, co
                                  void* dv_out, float* dla, float* dbeta, float* dS0, const WsHeader* hdr,
                                  const int* off, const int32_t* cu, int Tseq, int N, int H, int Hk, unsigned pro_raw,
                                  int dk, int dv, int max_chunks, long long Ttot, float* slots, float* S_chunks,
-                                 float* dSn_chunks, float* scr, float* dq_acc, float* dk_acc, void* qn, void* kn,
-                                 float* la_act, float* beta_act, cudaStream_t stream)
+                                 float* dSn_chunks, float* scr, float* F_chunks, float* dq_acc, float* dk_acc,
+                                 void* qn, void* kn, float* la_act, float* beta_act, cudaStream_t stream)
 {
     // the raw inputs, and the transformed ones every kernel below reads (the input prologue)
     const void *q_raw = q, *k_raw = k, *la_raw = la;
@@ -967,10 +1025,12 @@ cudaError_t launch_simt_backward(const void* q, const void* k, const void* v, co
             qq, kk, vv, la, beta, hdr, off, cu, Tseq, N, H, Hk, pro & KDA_PROLOGUE_GATE_BF16, dk, dv, slots);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    e = (dk == 128) ? launch_bwd_chains<TIn, 128>(S0, dout, dS_final, dS0, hdr, off, cu, Tseq, N, H, dv, slots,
-                                                  S_chunks, dSn_chunks, scr, stream)
-                    : launch_bwd_chains<TIn, 64>(S0, dout, dS_final, dS0, hdr, off, cu, Tseq, N, H, dv, slots,
-                                                 S_chunks, dSn_chunks, scr, stream);
+#define KDA_BWD_CHAINS(DKV, DVV)                                                                              \
+    launch_bwd_chains<TIn, DKV, DVV>(S0, dout, dS_final, dS0, hdr, off, cu, Tseq, N, H, max_chunks, slots, S_chunks, \
+                                     dSn_chunks, scr, F_chunks, stream)
+    e = (dk == 128) ? (dv == 128 ? KDA_BWD_CHAINS(128, 128) : KDA_BWD_CHAINS(128, 64))
+                    : (dv == 128 ? KDA_BWD_CHAINS(64, 128) : KDA_BWD_CHAINS(64, 64));
+#undef KDA_BWD_CHAINS
     if (e != cudaSuccess) return e;
     if (max_chunks > 0) {
         {

@@ -108,7 +108,7 @@ kda_status make_bwd_plan(int B, int T, int H, int Hk, unsigned pro, int dk, int 
     p.la_bytes = (pro & KDA_PROLOGUE_GATE_LOGITS) ? round_up(sizeof(float) * Tt * H * dk, kAlign) : 0;
     p.beta_bytes = (pro & KDA_PROLOGUE_BETA_LOGITS) ? round_up(sizeof(float) * Tt * H, kAlign) : 0;
     p.total_bytes = round_up(sizeof(WsHeader) + p.f.off_bytes +
-                             units * (p.slot_bytes + 2 * p.state_bytes + p.scr_bytes), kAlign) +
+                             units * (p.slot_bytes + 3 * p.state_bytes + p.scr_bytes), kAlign) +
                     2 * p.acc_bytes + 2 * p.qk_bytes + p.la_bytes + p.beta_bytes;
     return KDA_OK;
 }
@@ -295,8 +295,9 @@ kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, const void
     char* states = slots + units * p.slot_bytes;
     char* cot = states + units * p.state_bytes;
     char* scr = cot + units * p.state_bytes;
+    char* fdo = scr + units * p.scr_bytes;  // F = Qg^T dO per chunk
     char* acc = ws + round_up(sizeof(WsHeader) + p.f.off_bytes +
-                              units * (p.slot_bytes + 2 * p.state_bytes + p.scr_bytes), kAlign);
+                              units * (p.slot_bytes + 3 * p.state_bytes + p.scr_bytes), kAlign);
     char* qn = acc + 2 * p.acc_bytes;  // prologue buffers (empty when their bit is off)
     char* kn = qn + p.qk_bytes;
     char* la_act = kn + p.qk_bytes;
@@ -312,13 +313,14 @@ kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, const void
         ? launch_simt_backward<__nv_bfloat16>(q, k, v, log_alpha, beta, S0, dout, dS_final, dq, dk_out, dv_out,
                                               dlog_alpha, dbeta, dS0, hdr, off, cu_seqlens, p.f.Tseq, p.f.N, H, Hk,
                                               pro, dk, dv, p.f.max_chunks, p.f.Ttot, (float*)slots, (float*)states,
-                                              (float*)cot, (float*)scr, (float*)acc, (float*)(acc + p.acc_bytes),
-                                              qn, kn, (float*)la_act, (float*)beta_act, stream)
+                                              (float*)cot, (float*)scr, (float*)fdo, (float*)acc,
+                                              (float*)(acc + p.acc_bytes), qn, kn, (float*)la_act,
+                                              (float*)beta_act, stream)
         : launch_simt_backward<float>(q, k, v, log_alpha, beta, S0, dout, dS_final, dq, dk_out, dv_out, dlog_alpha,
                                       dbeta, dS0, hdr, off, cu_seqlens, p.f.Tseq, p.f.N, H, Hk, pro, dk, dv,
                                       p.f.max_chunks, p.f.Ttot, (float*)slots, (float*)states, (float*)cot,
-                                      (float*)scr, (float*)acc, (float*)(acc + p.acc_bytes), qn, kn,
-                                      (float*)la_act, (float*)beta_act, stream);
+                                      (float*)scr, (float*)fdo, (float*)acc, (float*)(acc + p.acc_bytes), qn,
+                                      kn, (float*)la_act, (float*)beta_act, stream);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

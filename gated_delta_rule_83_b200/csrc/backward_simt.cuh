@@ -537,9 +537,9 @@ bwd_ut_kernel(const TIn* __restrict__ k, const TIn* __restrict__ v, const void* 
         for (int e = tid; e < kChunk * kBwdCT; e += kSimtThreads) {
             const int r = e / kBwdCT, cc = e % kBwdCT;
             const float g = tg[r * LT + cc], x = g - tref[cc], kv = tk[r * LT + cc];
-            tA[r * LT + cc] = wide ? 0.f : kv * expf(x);   // Kf
-            tB[r * LT + cc] = wide ? 0.f : kv * expf(-x);  // Kb
-            tC[r * LT + cc] = kv * expf(g);                // Kt
+            tA[r * LT + cc] = wide ? 0.f : kv * fast_exp(x);   // Kf
+            tB[r * LT + cc] = wide ? 0.f : kv * fast_exp(-x);  // Kb
+            tC[r * LT + cc] = kv * fast_exp(g);                // Kt
         }
         __syncthreads();
         if (!wide) {
@@ -553,7 +553,7 @@ bwd_ut_kernel(const TIn* __restrict__ k, const TIn* __restrict__ v, const void* 
                     if (i >= r) continue;
                     float x = 0.f;
                     for (int cc = 0; cc < kBwdCT; ++cc)
-                        x = fmaf(tk[r * LT + cc] * tk[i * LT + cc], expf(tg[r * LT + cc] - tg[i * LT + cc]), x);
+                        x = fmaf(tk[r * LT + cc] * tk[i * LT + cc], fast_exp(tg[r * LT + cc] - tg[i * LT + cc]), x);
                     accA[a][b] += x;
                 }
         }
@@ -720,7 +720,7 @@ bwd_gate_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const void
         for (int e = tid; e < kChunk * kBwdCT; e += kSimtThreads) {
             const int r = e / kBwdCT, cc = e % kBwdCT;
             const float x = tg[r * LT + cc] - tref[cc];
-            const float ex = expf(x), emx = expf(-x);
+            const float ex = fast_exp(x), emx = fast_exp(-x);
             tA[r * LT + cc] = tk[r * LT + cc] * ex;   // Kf
             tB[r * LT + cc] = tk[r * LT + cc] * emx;  // Kb
             tC[r * LT + cc] = tq[r * LT + cc] * ex;   // Qf
@@ -742,13 +742,13 @@ bwd_gate_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const void
                 const int r = tr + 16 * a, cc = tc + 16 * b;
                 const float gr = tg[r * LT + cc];
                 for (int i = 0; i <= r; ++i) {
-                    const float ke = tk[i * LT + cc] * expf(gr - tg[i * LT + cc]);
+                    const float ke = tk[i * LT + cc] * fast_exp(gr - tg[i * LT + cc]);
                     rowP[a][b] = fmaf(sdP[r * L64 + i], ke, rowP[a][b]);
                     rowA[a][b] = fmaf(sM[r * L64 + i], ke, rowA[a][b]);
                 }
                 for (int i = r; i < kChunk; ++i)
                     col[a][b] = fmaf(fmaf(sdP[i * L64 + r], tq[i * LT + cc], sM[i * L64 + r] * tk[i * LT + cc]),
-                                     expf(tg[i * LT + cc] - gr), col[a][b]);
+                                     fast_exp(tg[i * LT + cc] - gr), col[a][b]);
             }
     }
     mm_acc<4, 2>(dkt, sN, 1, L64, tD, LT, 1, kChunk, tr, tc);
@@ -761,13 +761,13 @@ bwd_gate_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const void
             const float g = tg[r * LT + cc], gl = tg[(kChunk - 1) * LT + cc];
             if (!wide) {
                 const float x = g - tref[cc];
-                const float ex = expf(x);
+                const float ex = fast_exp(x);
                 rowP[a][b] *= ex;
                 rowA[a][b] *= ex;
-                col[a][b] *= expf(-x);
+                col[a][b] *= fast_exp(-x);
             }
             const float kt = dkt[a][b] * sb[r];
-            const float eg = expf(g), egl = expf(gl - g);
+            const float eg = fast_exp(g), egl = fast_exp(gl - g);
             const float qv = tq[r * LT + cc], kv = tk[r * LT + cc];
             const size_t gi = (size_t)r * dk + c0 + cc;
             const float dQg = gdQg[gi], dKd = gdKd[gi];
@@ -801,7 +801,7 @@ bwd_gate_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const void
         const int cc = tid;
         float s = 0.f;
         for (int r = 0; r < kChunk; ++r) s += tA[r * LT + cc];
-        s += gdGam[c0 + cc] * expf(tg[(kChunk - 1) * LT + cc]);
+        s += gdGam[c0 + cc] * fast_exp(tg[(kChunk - 1) * LT + cc]);
         float acc = s;
         for (int r = kChunk - 1; r >= 0; --r) {
             acc += tB[r * LT + cc];

@@ -27,6 +27,16 @@
 namespace kda {
 
 constexpr int kSimtThreads = 256;
+
+// e^x from the hardware's base-2 exponential (ex2.approx, relative error ~2^-22 over the normal
+// range; results below 2^-126 flush to zero, which every use here can take: the factors are decays
+// or the factorised halves of one, and the products they enter are sums of such terms)
+__device__ __forceinline__ float fast_exp(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x * 1.4426950408889634f));
+    return y;
+}
 constexpr int kSimtNV = 32;  // state columns per phase-B CTA
 
 // fp32 workspace slot of one (chunk, head): W | Qg | Kd [64 x dk] | P [64 x 64] | Uv [64 x dv] | gam [dk]
@@ -175,11 +185,11 @@ simt_intra_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TI
     for (int e = tid; e < kChunk * dk; e += kSimtThreads) {
         const int r = e / dk, c = e % dk, x = r * LK + c;
         const float gl = sg[(kChunk - 1) * LK + c];
-        const float eg = expf(sg[x]);
+        const float eg = fast_exp(sg[x]);
         gQ[e] = sq[x] * eg;
-        gKd[e] = sk[x] * expf(gl - sg[x]);
+        gKd[e] = sk[x] * fast_exp(gl - sg[x]);
         sKt[x] = sk[x] * eg;
-        if (r == 0) gGam[c] = expf(gl);
+        if (r == 0) gGam[c] = fast_exp(gl);
     }
     __syncthreads();
 
@@ -190,9 +200,9 @@ simt_intra_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TI
             const int r = e / dk, c = e % dk, x0 = r * LK + c;
             const float x = sg[x0] - sref[c];
             const float kv = sk[x0];
-            sk[x0] = kv * expf(x);
-            sq[x0] = sq[x0] * expf(x);
-            sg[x0] = kv * expf(-x);
+            sk[x0] = kv * fast_exp(x);
+            sq[x0] = sq[x0] * fast_exp(x);
+            sg[x0] = kv * fast_exp(-x);
         }
         __syncthreads();
         // A = Kf Kb^T and P = Qf Kb^T, register-tiled (4 x 4 per thread, shared Kb reads)
@@ -229,7 +239,7 @@ simt_intra_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TI
             float a = 0.f, p = 0.f;
             if (i <= r) {
                 for (int c = 0; c < dk; ++c) {
-                    const float kk = sk[i * LK + c] * expf(sg[r * LK + c] - sg[i * LK + c]);
+                    const float kk = sk[i * LK + c] * fast_exp(sg[r * LK + c] - sg[i * LK + c]);
                     a = fmaf(sk[r * LK + c], kk, a);
                     p = fmaf(sq[r * LK + c], kk, p);
                 }

@@ -49,6 +49,24 @@ __host__ __device__ inline size_t simt_slot_floats(int dk, int dv)
 // below stay finite in fp32: each factor is e^{+-x} with |x| <= kFactorSpread / 2 <= 80.
 constexpr float kFactorSpread = 160.f;
 
+// 8 consecutive values widened to fp32 (the address is 16-byte aligned)
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float* f)
+{
+    const uint4 r = *reinterpret_cast<const uint4*>(p);
+    const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&r);
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const float2 t = __bfloat1622float2(b[m]);
+        f[2 * m] = t.x;
+        f[2 * m + 1] = t.y;
+    }
+}
+__device__ __forceinline__ void load8(const float* p, float* f)
+{
+    const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+
 // acc[i][j] += sum_k A(tr + 16 i, k) B(k, tc + 16 j), with A(r, k) = A[r * ars + k * aks] and
 // B(k, c) = B[k * bks + c * bcs] in shared memory (thread tid: tr = tid / 16, tc = tid % 16).  Each
 // thread owns a TM x TN block of interleaved rows and columns, so the B reads of a warp fall on
@@ -115,22 +133,33 @@ simt_intra_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TI
     const int tr = tid >> 4, tc = tid & 15;
 
     if (tid == 0) s_wide = 0;
-    for (int e = tid; e < kChunk * dk; e += kSimtThreads) {
-        const int r = e / dk, c = e % dk;
-        float kv = 0.f, qv = 0.f, lv = 0.f;
+    // 8 consecutive channels per thread and step (16- or 32-byte loads); rows past the end read as 0
+    for (int e = tid; e < kChunk * dk / 8; e += kSimtThreads) {
+        const int r = e / (dk / 8), c = 8 * (e % (dk / 8));
+        float kv[8] = {}, qv[8] = {}, lv[8] = {};
         if (r < L) {
             const size_t gi = ((size_t)(t0 + r) * H + h) * dk + c;
             const size_t qi = ((size_t)(t0 + r) * Hk + h / (H / Hk)) * dk + c;  // q/k head of value head h
-            kv = to_f32(k[qi]); qv = to_f32(q[qi]);
-            lv = (pro & KDA_PROLOGUE_GATE_BF16) ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(log_alpha)[gi])
-                                                : reinterpret_cast<const float*>(log_alpha)[gi];
-            if (pro & KDA_PROLOGUE_GATE_LOGITS) lv = log_sigmoid_f(lv);  // rows past the end stay 0 (identity)
+            load8(k + qi, kv);
+            load8(q + qi, qv);
+            if (pro & KDA_PROLOGUE_GATE_BF16) load8(reinterpret_cast<const __nv_bfloat16*>(log_alpha) + gi, lv);
+            else load8(reinterpret_cast<const float*>(log_alpha) + gi, lv);
+            if (pro & KDA_PROLOGUE_GATE_LOGITS)  // rows past the end stay 0 (identity)
+                for (int m = 0; m < 8; ++m) lv[m] = log_sigmoid_f(lv[m]);
         }
-        sk[r * LK + c] = kv; sq[r * LK + c] = qv; sg[r * LK + c] = lv;
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            sk[r * LK + c + m] = kv[m];
+            sq[r * LK + c + m] = qv[m];
+            sg[r * LK + c + m] = lv[m];
+        }
     }
-    for (int e = tid; e < kChunk * dv; e += kSimtThreads) {
-        const int r = e / dv, c = e % dv;
-        sv[r * LV + c] = (r < L) ? to_f32(v[((size_t)(t0 + r) * H + h) * dv + c]) : 0.f;
+    for (int e = tid; e < kChunk * dv / 8; e += kSimtThreads) {
+        const int r = e / (dv / 8), c = 8 * (e % (dv / 8));
+        float vv[8] = {};
+        if (r < L) load8(v + ((size_t)(t0 + r) * H + h) * dv + c, vv);
+#pragma unroll
+        for (int m = 0; m < 8; ++m) sv[r * LV + c + m] = vv[m];
     }
     for (int r = tid; r < kChunk; r += kSimtThreads) {
         float b = 0.f;

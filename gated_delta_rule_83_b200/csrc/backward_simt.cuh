@@ -194,11 +194,24 @@ bwd_do_terms_kernel(const TIn* __restrict__ dout, const WsHeader* __restrict__ h
     const float* slot = slots + u * simt_slot_floats(DK, DV);
     const float* gQ = slot + (size_t)kChunk * DK;
     const float* gP = slot + 3 * (size_t)kChunk * DK;
-    for (int e = tid; e < kChunk * kChunk; e += kSimtThreads) sP[(e / kChunk) * L64 + (e % kChunk)] = gP[e];
-    for (int e = tid; e < kChunk * DK; e += kSimtThreads) sQ[(e / DK) * LK + (e % DK)] = gQ[e];
-    for (int e = tid; e < kChunk * DV; e += kSimtThreads) {
-        const int r = e / DV, jj = e % DV;
-        sO[r * LV + jj] = (r < L) ? to_f32(dout[((size_t)(t0 + r) * H + h) * DV + jj]) : 0.f;
+    for (int e = tid; e < kChunk * kChunk / 8; e += kSimtThreads) {
+        float f[8];
+        load8(gP + 8 * e, f);
+#pragma unroll
+        for (int m = 0; m < 8; ++m) sP[((8 * e) / kChunk) * L64 + (8 * e) % kChunk + m] = f[m];
+    }
+    for (int e = tid; e < kChunk * DK / 8; e += kSimtThreads) {
+        float f[8];
+        load8(gQ + 8 * e, f);
+#pragma unroll
+        for (int m = 0; m < 8; ++m) sQ[((8 * e) / DK) * LK + (8 * e) % DK + m] = f[m];
+    }
+    for (int e = tid; e < kChunk * DV / 8; e += kSimtThreads) {
+        const int r = e / (DV / 8), jj = 8 * (e % (DV / 8));
+        float f[8] = {};
+        if (r < L) load8(dout + ((size_t)(t0 + r) * H + h) * DV + jj, f);
+#pragma unroll
+        for (int m = 0; m < 8; ++m) sO[r * LV + jj + m] = f[m];
     }
     __syncthreads();
     const int tr = tid >> 4, tc = tid & 15;
@@ -362,11 +375,18 @@ bwd_state_side_kernel(const TIn* __restrict__ dout, const WsHeader* __restrict__
     float* oP = oKd + (size_t)kChunk * dk;
     float* oGam = oP + (size_t)kChunk * kChunk;
 
-    for (int e = tid; e < kChunk * dv; e += kSimtThreads) {
-        const int r = e / dv, jj = e % dv;
-        sO[r * LDV + jj] = (r < L) ? to_f32(dout[((size_t)(t0 + r) * H + h) * dv + jj]) : 0.f;
-        sU[r * LDV + jj] = oU[e];
-        sdU[r * LDV + jj] = odU[e];
+    for (int e = tid; e < kChunk * dv / 8; e += kSimtThreads) {
+        const int r = e / (dv / 8), jj = 8 * (e % (dv / 8));
+        float fo[8] = {}, fu[8], fd[8];
+        if (r < L) load8(dout + ((size_t)(t0 + r) * H + h) * dv + jj, fo);
+        load8(oU + (size_t)r * dv + jj, fu);
+        load8(odU + (size_t)r * dv + jj, fd);
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            sO[r * LDV + jj + m] = fo[m];
+            sU[r * LDV + jj + m] = fu[m];
+            sdU[r * LDV + jj + m] = fd[m];
+        }
     }
     __syncthreads();
     const int tr = tid >> 4, tc = tid & 15;
@@ -384,10 +404,16 @@ bwd_state_side_kernel(const TIn* __restrict__ dout, const WsHeader* __restrict__
     // dQg = dO S_c^T, dW = -dU S_c^T, dKd = U D_c^T, dgam = rowsum(D_c * S_c), 64 channels at a time
     for (int c0 = 0; c0 < dk; c0 += kChunk) {
         __syncthreads();
-        for (int e = tid; e < kChunk * dv; e += kSimtThreads) {
-            const int cc = e / dv, jj = e % dv;
-            sS[cc * LDV + jj] = Sc[(size_t)(c0 + cc) * dv + jj];
-            sD[cc * LDV + jj] = Dc[(size_t)(c0 + cc) * dv + jj];
+        for (int e = tid; e < kChunk * dv / 8; e += kSimtThreads) {
+            const int cc = e / (dv / 8), jj = 8 * (e % (dv / 8));
+            float fs[8], fd[8];
+            load8(Sc + (size_t)(c0 + cc) * dv + jj, fs);
+            load8(Dc + (size_t)(c0 + cc) * dv + jj, fd);
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                sS[cc * LDV + jj + m] = fs[m];
+                sD[cc * LDV + jj + m] = fd[m];
+            }
         }
         __syncthreads();
         float aq[4][4] = {}, aw[4][4] = {}, ak[4][4] = {};
@@ -438,15 +464,16 @@ __device__ __forceinline__ void bwd_gate_tile(const void* __restrict__ log_alpha
                                               int H, int h, int dk, int c0, float* tg, float* tref, int* s_wide)
 {
     const int tid = threadIdx.x;
-    for (int e = tid; e < kChunk * kBwdCT; e += kSimtThreads) {
-        const int r = e / kBwdCT, cc = e % kBwdCT;
-        float x = 0.f;
+    for (int e = tid; e < kChunk * kBwdCT / 8; e += kSimtThreads) {
+        const int r = e / (kBwdCT / 8), cc = 8 * (e % (kBwdCT / 8));
+        float x[8] = {};
         if (r < L) {
             const size_t ia = ((size_t)(t0 + r) * H + h) * dk + c0 + cc;
-            x = la16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(log_alpha)[ia])
-                     : reinterpret_cast<const float*>(log_alpha)[ia];
+            if (la16) load8(reinterpret_cast<const __nv_bfloat16*>(log_alpha) + ia, x);
+            else load8(reinterpret_cast<const float*>(log_alpha) + ia, x);
         }
-        tg[r * kBwdLT + cc] = x;
+#pragma unroll
+        for (int m = 0; m < 8; ++m) tg[r * kBwdLT + cc + m] = x[m];
     }
     __syncthreads();
     if (tid < kBwdCT) {
@@ -466,17 +493,23 @@ template <typename TIn>
 __device__ __forceinline__ void bwd_load_tile(const TIn* __restrict__ x, long long t0, int L, int H, int h, int d,
                                               int c0, float* t)
 {
-    for (int e = threadIdx.x; e < kChunk * kBwdCT; e += kSimtThreads) {
-        const int r = e / kBwdCT, cc = e % kBwdCT;
-        t[r * kBwdLT + cc] = (r < L) ? to_f32(x[((size_t)(t0 + r) * H + h) * d + c0 + cc]) : 0.f;
+    for (int e = threadIdx.x; e < kChunk * kBwdCT / 8; e += kSimtThreads) {
+        const int r = e / (kBwdCT / 8), cc = 8 * (e % (kBwdCT / 8));
+        float f[8] = {};
+        if (r < L) load8(x + ((size_t)(t0 + r) * H + h) * d + c0 + cc, f);
+#pragma unroll
+        for (int m = 0; m < 8; ++m) t[r * kBwdLT + cc + m] = f[m];
     }
 }
 
 __device__ __forceinline__ void bwd_load_scr_tile(const float* __restrict__ x, int ld, int c0, float* t)
 {
-    for (int e = threadIdx.x; e < kChunk * kBwdCT; e += kSimtThreads) {
-        const int r = e / kBwdCT, cc = e % kBwdCT;
-        t[r * kBwdLT + cc] = x[(size_t)r * ld + c0 + cc];
+    for (int e = threadIdx.x; e < kChunk * kBwdCT / 8; e += kSimtThreads) {
+        const int r = e / (kBwdCT / 8), cc = 8 * (e % (kBwdCT / 8));
+        float f[8];
+        load8(x + (size_t)r * ld + c0 + cc, f);
+#pragma unroll
+        for (int m = 0; m < 8; ++m) t[r * kBwdLT + cc + m] = f[m];
     }
 }
 

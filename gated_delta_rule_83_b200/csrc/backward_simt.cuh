@@ -735,12 +735,29 @@ bwd_gate_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const void
     const int tr = tid >> 4, tc = tid & 15;
 
     if (tid == 0) s_wide = 0;
+    // this thread's dQg and dKd (rows tr + 16 a, channels c0 + tc + 16 b), in flight from the start
+    float pq[4][2], pk[4][2];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+            const size_t gi = (size_t)(tr + 16 * a) * dk + c0 + tc + 16 * b;
+            pq[a][b] = gdQg[gi];
+            pk[a][b] = gdKd[gi];
+        }
     for (int r = tid; r < kChunk; r += kSimtThreads) sb[r] = (r < L) ? beta[(size_t)(t0 + r) * H + h] : 0.f;
-    for (int e = tid; e < kChunk * kChunk; e += kSimtThreads) {
-        const int x = (e / kChunk) * L64 + (e % kChunk);
-        sN[x] = gN[e];
-        sM[x] = gdAt[e];
-        sdP[x] = gdP[e];
+    for (int e = tid; e < kChunk * kChunk / 8; e += kSimtThreads) {
+        float fn[8], fa[8], fp[8];
+        load8(gN + 8 * e, fn);
+        load8(gdAt + 8 * e, fa);
+        load8(gdP + 8 * e, fp);
+        const int x = ((8 * e) / kChunk) * L64 + (8 * e) % kChunk;
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            sN[x + m] = fn[m];
+            sM[x + m] = fa[m];
+            sdP[x + m] = fp[m];
+        }
     }
     bwd_load_tile(k, t0, L, Hk, h / (H / Hk), dk, c0, tk);  // the q/k head of value head h
     bwd_load_tile(q, t0, L, Hk, h / (H / Hk), dk, c0, tq);
@@ -802,8 +819,7 @@ bwd_gate_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const void
             const float kt = dkt[a][b] * sb[r];
             const float eg = fast_exp(g), egl = fast_exp(gl - g);
             const float qv = tq[r * LT + cc], kv = tk[r * LT + cc];
-            const size_t gi = (size_t)r * dk + c0 + cc;
-            const float dQg = gdQg[gi], dKd = gdKd[gi];
+            const float dQg = pq[a][b], dKd = pk[a][b];
             const float vq = rowP[a][b] + dQg * eg;
             const float vk = rowA[a][b] + col[a][b] + kt * eg + dKd * egl;
             accg[a][b] = qv * rowP[a][b] + kv * rowA[a][b] - kv * col[a][b] + (dQg * qv + kt * kv) * eg -

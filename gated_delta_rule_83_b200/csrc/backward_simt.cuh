@@ -610,15 +610,14 @@ bwd_ut_kernel(const TIn* __restrict__ k, const TIn* __restrict__ v, const void* 
     __syncthreads();
 
     // ---- step 4b: the UT transform backwards
-    if (tid < kChunk) {  // N = (I + Diag(beta) At)^{-1}, column tid, rows in order
-        const int jj = tid;
-        for (int r = 0; r < kChunk; ++r) {
-            float t = (r == jj) ? 1.f : 0.f;
-            for (int i = jj; i < r; ++i) t = fmaf(-sb[r] * sAt[r * L64 + i], sN[i * L64 + jj], t);
-            sN[r * L64 + jj] = (jj <= r) ? t : 0.f;
-        }
+    // N = (I + Diag(beta) At)^{-1}: Diag(beta) At copied into N, then inverted in place (the tiles
+    // tC..tD are idle here and serve as scratch)
+    for (int e = tid; e < kChunk * kChunk; e += kSimtThreads) {
+        const int r = e / kChunk, i = e % kChunk;
+        sN[r * L64 + i] = sb[r] * sAt[r * L64 + i];
     }
     __syncthreads();
+    simt_unit_lower_inverse(sN, tC);
     if (tid < kChunk) {  // dbeta_i = sum_r dT[r][i] N[r][i]   (T = N Diag(beta))
         float x = 0.f;
         for (int r = tid; r < kChunk; ++r) x = fmaf(sM[r * L64 + tid], sN[r * L64 + tid], x);

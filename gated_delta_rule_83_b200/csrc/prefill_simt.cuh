@@ -102,6 +102,83 @@ __device__ __forceinline__ void simt_apply_t(const float* sT, const float* X, fl
         for (int b = 0; b < D / 16; ++b) out[(size_t)(tr + 16 * a) * D + tc + 16 * b] = acc[a][b];
 }
 
+// X = (I + A)^{-1} for a strictly lower-triangular 64 x 64 A (row stride 65), in place of A, by
+// block doubling on all 256 threads: the four 16 x 16 diagonal blocks by forward substitution, then
+// X_10 = -X_11 A_10 X_00 for the 16-row pairs and again for the two 32-row halves.  Above the
+// diagonal the result holds zeros (A does), on it ones.  Y: scratch of 32 x 33 floats.
+__device__ __forceinline__ void simt_unit_lower_inverse(float* __restrict__ A, float* __restrict__ Y)
+{
+    constexpr int LS = kChunk + 1;
+    const int tid = threadIdx.x;
+    {   // diagonal blocks: thread (block b, column jj), rows in order
+        const int b = 16 * (tid >> 4), jj = tid & 15;
+        float x[16];
+        if (tid < 64) {
+            float sacc[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) sacc[r] = 0.f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                x[i] = (i == jj) ? 1.f : ((i < jj) ? 0.f : -sacc[i]);
+#pragma unroll
+                for (int r = i + 1; r < 16; ++r) sacc[r] = fmaf(A[(b + r) * LS + b + i], x[i], sacc[r]);
+            }
+        }
+        __syncthreads();
+        if (tid < 64)
+#pragma unroll
+            for (int r = 0; r < 16; ++r) A[(b + r) * LS + b + jj] = x[r];
+        __syncthreads();
+    }
+    {   // blocks (1,0) and (3,2) of 16: thread (pair p, row rr, columns cc, cc + 1)
+        const int p = tid >> 7, rr = (tid >> 3) & 15, cc = (tid & 7) * 2;
+        const int bi = 16 * (2 * p + 1), bj = 16 * (2 * p);
+        float y0 = 0.f, y1 = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const float a = A[(bi + rr) * LS + bj + k];
+            y0 = fmaf(a, A[(bj + k) * LS + bj + cc], y0);
+            y1 = fmaf(a, A[(bj + k) * LS + bj + cc + 1], y1);
+        }
+        Y[(p * 16 + rr) * 33 + cc] = y0;
+        Y[(p * 16 + rr) * 33 + cc + 1] = y1;
+        __syncthreads();
+        float x0 = 0.f, x1 = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const float xi = A[(bi + rr) * LS + bi + k];
+            x0 = fmaf(xi, Y[(p * 16 + k) * 33 + cc], x0);
+            x1 = fmaf(xi, Y[(p * 16 + k) * 33 + cc + 1], x1);
+        }
+        A[(bi + rr) * LS + bj + cc] = -x0;
+        A[(bi + rr) * LS + bj + cc + 1] = -x1;
+        __syncthreads();
+    }
+    {   // rows 32..63 x columns 0..31: thread (row rr, columns cc .. cc + 3)
+        const int rr = tid >> 3, cc = (tid & 7) * 4;
+        float y[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+        for (int k = 0; k < 32; ++k) {
+            const float a = A[(32 + rr) * LS + k];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) y[m] = fmaf(a, A[k * LS + cc + m], y[m]);
+        }
+#pragma unroll
+        for (int m = 0; m < 4; ++m) Y[rr * 33 + cc + m] = y[m];
+        __syncthreads();
+        float x[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+        for (int k = 0; k < 32; ++k) {
+            const float xi = A[(32 + rr) * LS + 32 + k];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) x[m] = fmaf(xi, Y[k * 33 + cc + m], x[m]);
+        }
+#pragma unroll
+        for (int m = 0; m < 4; ++m) A[(32 + rr) * LS + cc + m] = -x[m];
+        __syncthreads();
+    }
+}
+
 template <typename TIn>
 __global__ void __launch_bounds__(kSimtThreads)
 simt_intra_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
@@ -279,16 +356,13 @@ simt_intra_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TI
     }
     __syncthreads();
 
-    // T = (I + A)^{-1} diag(beta): thread jj owns column jj; rows in order.
-    if (tid < kChunk) {
-        const int jj = tid;
-        for (int r = 0; r < kChunk; ++r) {
-            float t = (r == jj) ? sb[r] : 0.f;
-            for (int i = jj; i < r; ++i) t = fmaf(-sA[r * L64 + i], sT[i * L64 + jj], t);
-            sT[r * L64 + jj] = (jj <= r) ? t : 0.f;
-        }
+    // T = (I + A)^{-1} diag(beta): the inverse in place of A (Kf, Qf and Kb are dead: sg is scratch)
+    simt_unit_lower_inverse(sA, sg);
+    for (int e = tid; e < kChunk * kChunk; e += kSimtThreads) {
+        const int r = e / kChunk, i = e % kChunk;
+        sT[r * L64 + i] = (i <= r) ? sA[r * L64 + i] * sb[i] : 0.f;
+        gP[e] = sP[r * L64 + i];
     }
-    for (int e = tid; e < kChunk * kChunk; e += kSimtThreads) gP[e] = sP[(e / kChunk) * L64 + (e % kChunk)];
     __syncthreads();
 
     // W = T Kt, Uv = T V (T is lower triangular with zeros above the diagonal)

@@ -174,3 +174,28 @@ def test_host_pipeline_rejects_before_launch(lib):
     assert lib.kda_chunk_fwd_host(*args, 128, None, 1 << 40, None) == 5        # no workspace
     assert lib.kda_chunk_fwd_host(*args, 128, fake, 16, None) == 5             # workspace too small
 
+
+
+def test_backward_rejects_before_launch(lib):
+    """kda_chunk_bwd validates options, shapes, pointers and the workspace before any CUDA call."""
+    from gated_delta_rule_83_b200.kda import KdaOptions
+    fake = 0x100000
+    n = ctypes.c_size_t(0)
+    assert lib.kda_chunk_bwd_workspace_size(1, 256, 4, 128, 128, 0, 0, 0, None, ctypes.byref(n)) == 0
+    plain = n.value
+    grouped = KdaOptions(num_qk_heads=2)
+    assert lib.kda_chunk_bwd_workspace_size(1, 256, 4, 128, 128, 0, 0, 0, ctypes.byref(grouped), ctypes.byref(n)) == 0
+    assert n.value > plain                                     # per-value-head dq/dk buffers
+    assert lib.kda_chunk_bwd_workspace_size(1, 256, 4, 96, 128, 0, 0, 0, None, ctypes.byref(n)) == 2  # dk
+    bad = KdaOptions(num_qk_heads=3)                           # 4 % 3 != 0
+    base = (fake, fake, fake, fake, fake, None, None, 0, fake, None, fake, fake, fake, fake, fake, None,
+            1, 256, 4, 128, 128, 0)
+    assert lib.kda_chunk_bwd(*base, ctypes.byref(bad), fake, 1 << 40, None) == 1
+    assert lib.kda_chunk_bwd(*base, None, None, 1 << 40, None) == 5          # no workspace
+    assert lib.kda_chunk_bwd(*base, None, fake, 16, None) == 5                # workspace too small
+    mis = list(base)
+    mis[8] = fake + 4                                                         # misaligned dout
+    assert lib.kda_chunk_bwd(*mis, None, fake, 1 << 40, None) == 1
+    nul = list(base)
+    nul[10] = None                                                            # no dq
+    assert lib.kda_chunk_bwd(*nul, None, fake, 1 << 40, None) == 1

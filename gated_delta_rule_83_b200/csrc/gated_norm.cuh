@@ -60,51 +60,41 @@ __device__ __forceinline__ float sigmoid_fast(float x)
     return 1.f / (1.f + e);
 }
 
-// LG = log2(lanes per group) = log2(group / 8); d = channels per row (64 or 128).  Each thread
-// handles kNormPer chunks kNormThreads apart, all loads issued before any arithmetic.
-constexpr int kNormPer = 2;
-
+// LG = log2(lanes per group) = log2(group / 8); d = channels per row (64 or 128).  One 8-channel
+// chunk per thread at 32 registers, so eight CTAs (2,048 threads) per SM keep loads in flight.
 template <typename T, int LG>
-__global__ void __launch_bounds__(kNormThreads)
+__global__ void __launch_bounds__(kNormThreads, 8)
 gated_rmsnorm_kernel(const T* __restrict__ o, const T* __restrict__ z, const float* __restrict__ weight, T* y,
                      long long chunks, int d, float inv_group, float eps, int sigmoid_gate)
 {
-    const long long base = (long long)blockIdx.x * (kNormThreads * kNormPer) + threadIdx.x;
-    float x[kNormPer][8], g[kNormPer][8];
+    const long long t = (long long)blockIdx.x * kNormThreads + threadIdx.x;
+    const bool live = t < chunks;                  // every lane joins the shuffles below
+    const long long e0 = (live ? t : 0) * 8;       // first element of this thread's 8 channels
+    float x[8], g[8];
+    Vec8<T>::load(o + e0, x);
+    Vec8<T>::load(z + e0, g);
+    float ss = 0.f;
 #pragma unroll
-    for (int i = 0; i < kNormPer; ++i) {  // every lane joins the shuffles below: dead chunks read chunk 0
-        const long long t = base + (long long)i * kNormThreads;
-        const long long e0 = (t < chunks ? t : 0) * 8;
-        Vec8<T>::load(o + e0, x[i]);
-        Vec8<T>::load(z + e0, g[i]);
+    for (int m = 0; m < 8; ++m) ss = fmaf(x[m], x[m], ss);
+#pragma unroll
+    for (int s = 0; s < LG; ++s) ss += __shfl_xor_sync(0xffffffffu, ss, 1 << s);
+    const float r = rsqrtf(ss * inv_group + eps);
+    const int c0 = 8 * (int)(t & (d / 8 - 1));     // first channel within the row (d / 8 is 8 or 16)
+    float w[8];
+    if (weight) {
+        const float4 a = __ldg(reinterpret_cast<const float4*>(weight + c0));
+        const float4 b = __ldg(reinterpret_cast<const float4*>(weight + c0) + 1);
+        w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w; w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+    } else {
+#pragma unroll
+        for (int m = 0; m < 8; ++m) w[m] = 1.f;
     }
-    const int cmask = d / 8 - 1;  // chunks per row - 1 (d is 64 or 128)
 #pragma unroll
-    for (int i = 0; i < kNormPer; ++i) {
-        const long long t = base + (long long)i * kNormThreads;
-        float ss = 0.f;
-#pragma unroll
-        for (int m = 0; m < 8; ++m) ss = fmaf(x[i][m], x[i][m], ss);
-#pragma unroll
-        for (int s = 0; s < LG; ++s) ss += __shfl_xor_sync(0xffffffffu, ss, 1 << s);
-        const float r = rsqrtf(ss * inv_group + eps);
-        const int c0 = 8 * (int)(t & cmask);  // first channel of this chunk within its row
-        float w[8];
-        if (weight) {
-            const float4 a = __ldg(reinterpret_cast<const float4*>(weight + c0));
-            const float4 b = __ldg(reinterpret_cast<const float4*>(weight + c0) + 1);
-            w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w; w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
-        } else {
-#pragma unroll
-            for (int m = 0; m < 8; ++m) w[m] = 1.f;
-        }
-#pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            const float gate = sigmoid_gate ? sigmoid_fast(g[i][m]) : g[i][m];
-            x[i][m] = x[i][m] * r * w[m] * gate;
-        }
-        if (t < chunks) Vec8<T>::store(y + t * 8, x[i]);
+    for (int m = 0; m < 8; ++m) {
+        const float gate = sigmoid_gate ? sigmoid_fast(g[m]) : g[m];
+        x[m] = x[m] * r * w[m] * gate;
     }
+    if (live) Vec8<T>::store(y + e0, x);
 }
 
 template <typename T>
@@ -113,7 +103,7 @@ cudaError_t launch_gated_rmsnorm(const void* o, const void* z, const float* weig
 {
     const long long chunks = rows * (d / 8);
     if (chunks == 0) return cudaSuccess;
-    const long long blocks = (chunks + kNormThreads * kNormPer - 1) / (kNormThreads * kNormPer);
+    const long long blocks = (chunks + kNormThreads - 1) / kNormThreads;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
     const T *oo = (const T*)o, *zz = (const T*)z;
     T* yy = (T*)y;

@@ -372,78 +372,133 @@ simt_intra_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TI
     else simt_apply_t<64>(sT, sv, gUv, tr, tc);
 }
 
-template <typename TOut>
+// 16-byte asynchronous global -> shared copies in commit groups (phase B's operand prefetch)
+__device__ __forceinline__ void simt_cp16(float* dst, const float* src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+                 "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void simt_cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void simt_cp_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void simt_cp_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// rows x cols floats from a dense global array into a shared array of row stride ld (cols and ld
+// multiples of 4)
+__device__ __forceinline__ void simt_cp_rows(float* dst, int ld, const float* src, int src_ld, int rows, int cols)
+{
+    const int per = cols / 4;
+    for (int e = threadIdx.x; e < rows * per; e += kSimtThreads) {
+        const int r = e / per, c = 4 * (e % per);
+        simt_cp16(dst + r * ld + c, src + (size_t)r * src_ld + c);
+    }
+}
+
+// Phase B: one CTA per (sequence, head, 32 state columns), chunks in order.  Chunk c's W and its Uv
+// columns arrive in one cp.async group, Qg, P, Kd and gam in another, each while the previous
+// chunk's other half computes.  Products are register-tiled (rows tr + 16 a, columns tc + 16 b).
+template <typename TOut, int DK>
 __global__ void __launch_bounds__(kSimtThreads)
 simt_inter_kernel(const float* S0, float* S_final, TOut* __restrict__ out, const WsHeader* __restrict__ hdr,
-                  const int* __restrict__ off, const int32_t* __restrict__ cu, int Tseq, int N, int H, int dk, int dv,
+                  const int* __restrict__ off, const int32_t* __restrict__ cu, int Tseq, int N, int H, int dv,
                   const float* __restrict__ slots)
 {
     extern __shared__ __align__(16) float smem[];
     const int n = blockIdx.x, h = blockIdx.y, v0 = blockIdx.z * kSimtNV, tid = threadIdx.x;
     if (hdr->bad) return;
-    constexpr int NV = kSimtNV;
-    float* sS = smem;                       // [dk][NV]
-    float* sW = sS + dk * NV;               // [64][dk]
-    float* sQ = sW + kChunk * dk;           // [64][dk]
-    float* sKd = sQ + kChunk * dk;          // [64][dk]
-    float* sP = sKd + kChunk * dk;          // [64][64]
-    float* sUv = sP + kChunk * kChunk;      // [64][NV]
-    float* sU = sUv + kChunk * NV;          // [64][NV]
-    float* sG = sU + kChunk * NV;           // [dk]
-
-    const size_t sidx = ((size_t)n * H + h) * dk * dv;
-    for (int e = tid; e < dk * NV; e += kSimtThreads) {
-        const int c = e / NV, jj = e % NV;
-        sS[e] = S0 ? S0[sidx + (size_t)c * dv + v0 + jj] : 0.f;
-    }
+    constexpr int NV = kSimtNV, TMD = DK / 16;
+    constexpr int LK = DK + 4, LP = kChunk + 4;  // padded rows: the two rows a warp reads sit on distinct banks
+    float* sS = smem;                 // [DK][NV]
+    float* sW = sS + DK * NV;         // [64][DK+4]
+    float* sQ = sW + kChunk * LK;     // [64][DK+4]
+    float* sKd = sQ + kChunk * LK;    // [64][DK+4]
+    float* sP = sKd + kChunk * LK;    // [64][68]
+    float* sUv = sP + kChunk * LP;    // [64][NV]
+    float* sU = sUv + kChunk * NV;    // [64][NV]
+    float* sG = sU + kChunk * NV;     // [DK]
+    const int tr = tid >> 4, tc = tid & 15;
+    const size_t slot_f = simt_slot_floats(DK, dv);
+    const size_t sidx = ((size_t)n * H + h) * DK * dv;
+    for (int e = tid; e < DK * NV; e += kSimtThreads)
+        sS[e] = S0 ? S0[sidx + (size_t)(e / NV) * dv + v0 + (e % NV)] : 0.f;
     long long s0, s1;
     seq_bounds(n, cu, Tseq, s0, s1);
-    const size_t slot_f = simt_slot_floats(dk, dv);
-    for (int j = off[n]; j < off[n + 1]; ++j) {
-        const long long t0 = s0 + (long long)(j - off[n]) * kChunk;
-        const int L = (s1 - t0) < kChunk ? (int)(s1 - t0) : kChunk;
+    const int j0 = off[n], j1 = off[n + 1];
+    auto issue_w = [&](int j) {  // W and the Uv columns of chunk j
         const float* slot = slots + ((size_t)j * H + h) * slot_f;
-        const float* gW = slot;
-        const float* gQ = gW + (size_t)kChunk * dk;
-        const float* gKd = gQ + (size_t)kChunk * dk;
-        const float* gP = gKd + (size_t)kChunk * dk;
-        const float* gUv = gP + (size_t)kChunk * kChunk;
-        const float* gGam = gUv + (size_t)kChunk * dv;
-        __syncthreads();  // previous chunk finished with the staged operands
-        for (int e = tid; e < kChunk * dk; e += kSimtThreads) { sW[e] = gW[e]; sQ[e] = gQ[e]; sKd[e] = gKd[e]; }
-        for (int e = tid; e < kChunk * kChunk; e += kSimtThreads) sP[e] = gP[e];
-        for (int e = tid; e < kChunk * NV; e += kSimtThreads) sUv[e] = gUv[(e / NV) * dv + v0 + (e % NV)];
-        for (int e = tid; e < dk; e += kSimtThreads) sG[e] = gGam[e];
-        __syncthreads();
-        for (int e = tid; e < kChunk * NV; e += kSimtThreads) {
-            const int r = e / NV, jj = e % NV;
-            float x = 0.f;
-            for (int c = 0; c < dk; ++c) x = fmaf(sW[r * dk + c], sS[c * NV + jj], x);
-            sU[e] = sUv[e] - x;
-        }
-        __syncthreads();
-        for (int e = tid; e < kChunk * NV; e += kSimtThreads) {
-            const int r = e / NV, jj = e % NV;
-            if (r >= L) continue;
-            float o = 0.f;
-            for (int c = 0; c < dk; ++c) o = fmaf(sQ[r * dk + c], sS[c * NV + jj], o);
-            for (int i = 0; i <= r; ++i) o = fmaf(sP[r * kChunk + i], sU[i * NV + jj], o);
-            out[((size_t)(t0 + r) * H + h) * dv + v0 + jj] = from_f32<TOut>(o);
-        }
-        __syncthreads();
-        for (int e = tid; e < dk * NV; e += kSimtThreads) {
-            const int c = e / NV, jj = e % NV;
-            float s = sG[c] * sS[e];
-            for (int i = 0; i < kChunk; ++i) s = fmaf(sKd[i * dk + c], sU[i * NV + jj], s);
-            sS[e] = s;
-        }
+        simt_cp_rows(sW, LK, slot, DK, kChunk, DK);
+        simt_cp_rows(sUv, NV, slot + (size_t)kChunk * (3 * DK + kChunk) + v0, dv, kChunk, NV);
+        simt_cp_commit();
+    };
+    auto issue_q = [&](int j) {  // Qg, Kd, P and gam of chunk j
+        const float* slot = slots + ((size_t)j * H + h) * slot_f;
+        simt_cp_rows(sQ, LK, slot + (size_t)kChunk * DK, DK, kChunk, DK);
+        simt_cp_rows(sKd, LK, slot + 2 * (size_t)kChunk * DK, DK, kChunk, DK);
+        simt_cp_rows(sP, LP, slot + 3 * (size_t)kChunk * DK, kChunk, kChunk, kChunk);
+        simt_cp_rows(sG, DK, slot + (size_t)kChunk * (3 * DK + kChunk + dv), DK, 1, DK);
+        simt_cp_commit();
+    };
+    if (j0 < j1) {
+        issue_w(j0);
+        issue_q(j0);
     }
+    for (int j = j0; j < j1; ++j) {
+        const long long t0 = s0 + (long long)(j - j0) * kChunk;
+        const int L = (s1 - t0) < kChunk ? (int)(s1 - t0) : kChunk;
+        simt_cp_wait1();  // W and Uv of chunk j (Qg, Kd, P may still be in flight)
+        __syncthreads();
+        {   // U = Uv - W S
+            float x[4][2] = {};
+            mm_acc<4, 2>(x, sW, LK, 1, sS, NV, 1, DK, tr, tc);
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int b = 0; b < 2; ++b) {
+                    const int r = tr + 16 * a, jj = tc + 16 * b;
+                    sU[r * NV + jj] = sUv[r * NV + jj] - x[a][b];
+                }
+        }
+        __syncthreads();
+        if (j + 1 < j1) issue_w(j + 1);
+        else simt_cp_commit();  // one group per step keeps the wait counts aligned
+        simt_cp_wait1();        // Qg, Kd, P, gam of chunk j
+        __syncthreads();
+        {   // out = Qg S + P U (rows past the end are not written)
+            float o[4][2] = {};
+            mm_acc<4, 2>(o, sQ, LK, 1, sS, NV, 1, DK, tr, tc);
+            mm_acc<4, 2>(o, sP, LP, 1, sU, NV, 1, kChunk, tr, tc);
+            if (out)
+#pragma unroll
+                for (int a = 0; a < 4; ++a) {
+                    const int r = tr + 16 * a;
+                    if (r < L)
+#pragma unroll
+                        for (int b = 0; b < 2; ++b)
+                            out[((size_t)(t0 + r) * H + h) * dv + v0 + tc + 16 * b] = from_f32<TOut>(o[a][b]);
+                }
+        }
+        {   // S <- Diag(gam) S + Kd^T U
+            float acc[TMD][2];
+#pragma unroll
+            for (int a = 0; a < TMD; ++a)
+#pragma unroll
+                for (int b = 0; b < 2; ++b) acc[a][b] = sG[tr + 16 * a] * sS[(tr + 16 * a) * NV + tc + 16 * b];
+            mm_acc<TMD, 2>(acc, sKd, 1, LK, sU, NV, 1, kChunk, tr, tc);
+            __syncthreads();  // every thread has read the old S (and Qg, P, Kd)
+#pragma unroll
+            for (int a = 0; a < TMD; ++a)
+#pragma unroll
+                for (int b = 0; b < 2; ++b) sS[(tr + 16 * a) * NV + tc + 16 * b] = acc[a][b];
+        }
+        __syncthreads();
+        if (j + 1 < j1) issue_q(j + 1);
+        else simt_cp_commit();
+    }
+    simt_cp_wait0();
     __syncthreads();
     if (S_final)
-        for (int e = tid; e < dk * NV; e += kSimtThreads) {
-            const int c = e / NV, jj = e % NV;
-            S_final[sidx + (size_t)c * dv + v0 + jj] = sS[e];
-        }
+        for (int e = tid; e < DK * NV; e += kSimtThreads)
+            S_final[sidx + (size_t)(e / NV) * dv + v0 + (e % NV)] = sS[e];
 }
 
 inline size_t simt_intra_smem(int dk, int dv)
@@ -453,7 +508,8 @@ inline size_t simt_intra_smem(int dk, int dv)
 inline size_t simt_inter_smem(int dk, int dv)
 {
     (void)dv;
-    return sizeof(float) * ((size_t)dk * kSimtNV + 3 * kChunk * dk + kChunk * kChunk + 2 * kChunk * kSimtNV + dk);
+    return sizeof(float) * ((size_t)dk * kSimtNV + 3 * kChunk * (dk + 4) + kChunk * (kChunk + 4) +
+                            2 * kChunk * kSimtNV + dk);
 }
 
 template <typename TIn>
@@ -465,7 +521,8 @@ cudaError_t launch_simt_prefill(const void* q, const void* k, const void* v, con
     const size_t smA = simt_intra_smem(dk, dv), smB = simt_inter_smem(dk, dv);
     cudaError_t e = cudaFuncSetAttribute(simt_intra_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smA);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(simt_inter_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smB);
+    e = cudaFuncSetAttribute(dk == 128 ? simt_inter_kernel<TIn, 128> : simt_inter_kernel<TIn, 64>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smB);
     if (e != cudaSuccess) return e;
     if (max_chunks > 0) {
         LaunchScope ls("simt_intra", stream);
@@ -475,8 +532,9 @@ cudaError_t launch_simt_prefill(const void* q, const void* k, const void* v, con
         if (e != cudaSuccess) return e;
     }
     LaunchScope ls("simt_inter", stream);
-    simt_inter_kernel<TIn><<<dim3(N, H, dv / kSimtNV), kSimtThreads, smB, stream>>>(
-        S0, S_final, (TIn*)out, hdr, off, cu, Tseq, N, H, dk, dv, slots);
+    auto* inter = dk == 128 ? simt_inter_kernel<TIn, 128> : simt_inter_kernel<TIn, 64>;
+    inter<<<dim3(N, H, dv / kSimtNV), kSimtThreads, smB, stream>>>(S0, S_final, (TIn*)out, hdr, off, cu, Tseq, N, H,
+                                                                   dv, slots);
     return cudaGetLastError();
 }
 

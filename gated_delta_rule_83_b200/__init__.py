@@ -11,7 +11,7 @@ Public API (a thin binding of the C ABI in include/kda.h):
 from .kda import (PROLOGUE_BETA_LOGITS, PROLOGUE_GATE_BF16, PROLOGUE_GATE_LOGITS, PROLOGUE_L2NORM_QK,  # noqa: F401
                   KdaError,
                   bwd_workspace_size, check, chunk_bwd, chunk_fwd, chunk_fwd_host, decode_step, gated_rmsnorm, load_library,
-                  profile_begin, profile_end, version, workspace_size)
+                  profile_begin, profile_end, release_workspaces, version, workspace_size)
 
 __all__ = ["chunk_fwd", "chunk_fwd_host", "chunk_bwd", "decode_step", "gated_rmsnorm", "check", "workspace_size",
-           "bwd_workspace_size", "load_library", "version", "KdaError"]
+           "bwd_workspace_size", "release_workspaces", "load_library", "version", "KdaError"]

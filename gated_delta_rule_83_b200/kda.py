@@ -135,7 +135,13 @@ def _stream_handle(stream: Optional[torch.cuda.Stream], device) -> int:
     return s.cuda_stream
 
 
-_workspaces = {}
+_workspaces = {}  # (device, stream handle) -> the largest workspace a call on that stream has needed
+
+
+def release_workspaces() -> None:
+    """Drop the cached per-stream workspaces (the backward's can be several GB).  Calls made after
+    this allocate again on first use; pass ``workspace=`` to manage the memory yourself."""
+    _workspaces.clear()
 
 
 def workspace_size(B: int, T: int, H: int, dk: int, dv: int, varlen: bool = False, num_seqs: int = 0,

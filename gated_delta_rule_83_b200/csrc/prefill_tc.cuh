@@ -158,25 +158,36 @@ __device__ __forceinline__ void ut_inverse_64_inplace(float* __restrict__ sA, fl
         *reinterpret_cast<float2*>(sA + (bi + rr) * kAS + bj + cc) = make_float2(-x0, -x1);
         __syncthreads();
     }
-    {   // level 2: rows 32..63, columns 0..31; thread -> (row rr, columns cc..cc+3)
-        const int rr = tid >> 3, cc = (tid & 7) * 4;
-        float y[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
-            const float a = sA[(32 + rr) * kAS + k];
-            const float4 xv = *reinterpret_cast<const float4*>(sA + k * kAS + cc);
-            y[0] = fmaf(a, xv.x, y[0]); y[1] = fmaf(a, xv.y, y[1]); y[2] = fmaf(a, xv.z, y[2]); y[3] = fmaf(a, xv.w, y[3]);
+    {   // level 2: rows 32..63, columns 0..31, on warps 0-3: thread -> (rows r0, r0 + 1, columns
+        // cc..cc+3).  Each right-hand float4 serves two rows, which halves the shared-memory
+        // wavefronts of the 128-bit loads; X22 is lower triangular, so warp w stops at row 8 w + 7.
+        const int r0 = 2 * (tid >> 3), cc = (tid & 7) * 4;
+        if (tid < 128) {
+            float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+            for (int k = 0; k < 32; ++k) {
+                const float a0 = sA[(32 + r0) * kAS + k], a1 = sA[(33 + r0) * kAS + k];
+                const float4 xv = *reinterpret_cast<const float4*>(sA + k * kAS + cc);
+                y0[0] = fmaf(a0, xv.x, y0[0]); y0[1] = fmaf(a0, xv.y, y0[1]); y0[2] = fmaf(a0, xv.z, y0[2]); y0[3] = fmaf(a0, xv.w, y0[3]);
+                y1[0] = fmaf(a1, xv.x, y1[0]); y1[1] = fmaf(a1, xv.y, y1[1]); y1[2] = fmaf(a1, xv.z, y1[2]); y1[3] = fmaf(a1, xv.w, y1[3]);
+            }
+            *reinterpret_cast<float4*>(sY + r0 * 36 + cc) = make_float4(y0[0], y0[1], y0[2], y0[3]);
+            *reinterpret_cast<float4*>(sY + (r0 + 1) * 36 + cc) = make_float4(y1[0], y1[1], y1[2], y1[3]);
         }
-        *reinterpret_cast<float4*>(sY + rr * 36 + cc) = make_float4(y[0], y[1], y[2], y[3]);
         __syncthreads();
-        float x[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
-            const float xi = sA[(32 + rr) * kAS + 32 + k];
-            const float4 yv = *reinterpret_cast<const float4*>(sY + k * 36 + cc);
-            x[0] = fmaf(xi, yv.x, x[0]); x[1] = fmaf(xi, yv.y, x[1]); x[2] = fmaf(xi, yv.z, x[2]); x[3] = fmaf(xi, yv.w, x[3]);
+        if (tid < 128) {
+            const int kend = 8 * (tid >> 5) + 8;  // rows of this warp: 8 w .. 8 w + 7 (X22[r][k] = 0 for k > r)
+            float x0[4] = {0.f, 0.f, 0.f, 0.f}, x1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+            for (int k = 0; k < kend; ++k) {
+                const float a0 = sA[(32 + r0) * kAS + 32 + k], a1 = sA[(33 + r0) * kAS + 32 + k];
+                const float4 yv = *reinterpret_cast<const float4*>(sY + k * 36 + cc);
+                x0[0] = fmaf(a0, yv.x, x0[0]); x0[1] = fmaf(a0, yv.y, x0[1]); x0[2] = fmaf(a0, yv.z, x0[2]); x0[3] = fmaf(a0, yv.w, x0[3]);
+                x1[0] = fmaf(a1, yv.x, x1[0]); x1[1] = fmaf(a1, yv.y, x1[1]); x1[2] = fmaf(a1, yv.z, x1[2]); x1[3] = fmaf(a1, yv.w, x1[3]);
+            }
+            *reinterpret_cast<float4*>(sA + (32 + r0) * kAS + cc) = make_float4(-x0[0], -x0[1], -x0[2], -x0[3]);
+            *reinterpret_cast<float4*>(sA + (33 + r0) * kAS + cc) = make_float4(-x1[0], -x1[1], -x1[2], -x1[3]);
         }
-        *reinterpret_cast<float4*>(sA + (32 + rr) * kAS + cc) = make_float4(-x[0], -x[1], -x[2], -x[3]);
         __syncthreads();
     }
 }

@@ -134,28 +134,35 @@ __device__ __forceinline__ void ut_inverse_64_inplace(float* __restrict__ sA, fl
         }
         __syncthreads();
     }
-    {   // level 1: blocks (1,0) and (3,2); thread -> (pair p, row rr, columns cc, cc+1)
-        const int p = tid >> 7, rr = (tid >> 3) & 15, cc = (tid & 7) * 2;
+    {   // level 1: blocks (1,0) and (3,2) on warps 0-1: thread -> (pair p, rows ra and ra + 8,
+        // columns cc..cc+3); rows ra = 0..7 of a warp sit on distinct banks (row stride 68)
+        const int p = tid >> 5, ra = (tid >> 2) & 7, cc = (tid & 3) * 4;
         const int bi = 16 * (2 * p + 1), bj = 16 * (2 * p);
-        float y0 = 0.f, y1 = 0.f;
+        if (tid < 64) {
+            float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            const float a = sA[(bi + rr) * kAS + bj + k];
-            const float2 xv = *reinterpret_cast<const float2*>(sA + (bj + k) * kAS + bj + cc);
-            y0 = fmaf(a, xv.x, y0);
-            y1 = fmaf(a, xv.y, y1);
+            for (int k = 0; k < 16; ++k) {
+                const float a0 = sA[(bi + ra) * kAS + bj + k], a1 = sA[(bi + ra + 8) * kAS + bj + k];
+                const float4 xv = *reinterpret_cast<const float4*>(sA + (bj + k) * kAS + bj + cc);
+                y0[0] = fmaf(a0, xv.x, y0[0]); y0[1] = fmaf(a0, xv.y, y0[1]); y0[2] = fmaf(a0, xv.z, y0[2]); y0[3] = fmaf(a0, xv.w, y0[3]);
+                y1[0] = fmaf(a1, xv.x, y1[0]); y1[1] = fmaf(a1, xv.y, y1[1]); y1[2] = fmaf(a1, xv.z, y1[2]); y1[3] = fmaf(a1, xv.w, y1[3]);
+            }
+            *reinterpret_cast<float4*>(sY + (p * 16 + ra) * 36 + cc) = make_float4(y0[0], y0[1], y0[2], y0[3]);
+            *reinterpret_cast<float4*>(sY + (p * 16 + ra + 8) * 36 + cc) = make_float4(y1[0], y1[1], y1[2], y1[3]);
         }
-        *reinterpret_cast<float2*>(sY + (p * 16 + rr) * 34 + cc) = make_float2(y0, y1);
         __syncthreads();  // A_10 read: X_10 takes its place
-        float x0 = 0.f, x1 = 0.f;
+        if (tid < 64) {
+            float x0[4] = {0.f, 0.f, 0.f, 0.f}, x1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            const float xi = sA[(bi + rr) * kAS + bi + k];
-            const float2 yv = *reinterpret_cast<const float2*>(sY + (p * 16 + k) * 34 + cc);
-            x0 = fmaf(xi, yv.x, x0);
-            x1 = fmaf(xi, yv.y, x1);
+            for (int k = 0; k < 16; ++k) {
+                const float a0 = sA[(bi + ra) * kAS + bi + k], a1 = sA[(bi + ra + 8) * kAS + bi + k];
+                const float4 yv = *reinterpret_cast<const float4*>(sY + (p * 16 + k) * 36 + cc);
+                x0[0] = fmaf(a0, yv.x, x0[0]); x0[1] = fmaf(a0, yv.y, x0[1]); x0[2] = fmaf(a0, yv.z, x0[2]); x0[3] = fmaf(a0, yv.w, x0[3]);
+                x1[0] = fmaf(a1, yv.x, x1[0]); x1[1] = fmaf(a1, yv.y, x1[1]); x1[2] = fmaf(a1, yv.z, x1[2]); x1[3] = fmaf(a1, yv.w, x1[3]);
+            }
+            *reinterpret_cast<float4*>(sA + (bi + ra) * kAS + bj + cc) = make_float4(-x0[0], -x0[1], -x0[2], -x0[3]);
+            *reinterpret_cast<float4*>(sA + (bi + ra + 8) * kAS + bj + cc) = make_float4(-x1[0], -x1[1], -x1[2], -x1[3]);
         }
-        *reinterpret_cast<float2*>(sA + (bi + rr) * kAS + bj + cc) = make_float2(-x0, -x1);
         __syncthreads();
     }
     {   // level 2: rows 32..63, columns 0..31, on warps 0-3: thread -> (rows r0, r0 + 1, columns

@@ -116,15 +116,20 @@ __device__ __forceinline__ void ut_inverse_64_inplace(float* __restrict__ sA, fl
     {   // diagonal 16 x 16 blocks: thread -> (block, column jj); written back once every block is read
         const int b = 16 * (tid >> 4), jj = tid & 15;
         float x[16];
-        if (tid < 64) {  // right-looking: once x_i is known, fold it into the partial sums of rows > i
-            float s[16];
+        if (tid < 64) {  // left-looking: x_r = -sum_{i<r} A[r][i] x_i, row r read as 128-bit words;
+                         // each sum takes x_{r-1} last, so the rows' chains overlap
 #pragma unroll
-            for (int r = 0; r < 16; ++r) s[r] = 0.f;
+            for (int r = 0; r < 16; ++r) {
+                float s = 0.f;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                x[i] = (i == jj) ? 1.f : ((i < jj) ? 0.f : -s[i]);
+                for (int i4 = 0; i4 < r; i4 += 4) {
+                    const float4 a4 = *reinterpret_cast<const float4*>(sA + (b + r) * kAS + b + i4);
+                    const float av[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
-                for (int r = i + 1; r < 16; ++r) s[r] = fmaf(sA[(b + r) * kAS + b + i], x[i], s[r]);
+                    for (int j = 0; j < 4; ++j)
+                        if (i4 + j < r) s = fmaf(av[j], x[i4 + j], s);
+                }
+                x[r] = (r == jj) ? 1.f : ((r < jj) ? 0.f : -s);
             }
         }
         __syncthreads();

@@ -210,13 +210,13 @@ __device__ __forceinline__ void ut_inverse_64_inplace(float* __restrict__ sA, fl
 // Persistent: CTA b starts with (chunk, head) unit b (unit u = chunk * H + head) and claims each
 // further unit from a work counter one unit ahead, so that its inputs can be prefetched.
 // Each input buffer is refilled with the next unit's data as soon as the current unit is done with
-// it: v once MMA2 has read it, log_alpha once MMA3 has read P (the last tenant of its region), k and
-// q once the last images have left for the workspace.
+// it: log_alpha once MMA3 has read P (the last tenant of its region); k, q and v once the last images
+// (Q' in the q rows, O0 in the v tile) have left for the workspace.
 constexpr int kAThreads = 256;
 constexpr uint32_t kA_KQ = 0;        // 32 KB: [k; q] -> [Kf; Qf] stacked (128 rows, atom columns at 0 / 16384)
                                      //   -> W in the k rows, Q' in the q rows
-constexpr uint32_t kA_V = 32768;     // 16 KB: v
-constexpr uint32_t kA_B = 49152;     // 16 KB: Kb -> T -> Uv -> O0
+constexpr uint32_t kA_V = 32768;     // 16 KB: v -> O0
+constexpr uint32_t kA_B = 49152;     // 16 KB: Kb -> T -> Uv
 constexpr uint32_t kA_G = 65536;     // 32 KB: log_alpha (fp32, or bf16 in the upper 16 KB) -> g fp32 [64][128]
                                      //   -> A / X fp32 [64][68] + scratch + P tile
 constexpr uint32_t kA_Ysc = kA_G + 17408;   // solve scratch 32 x 36 fp32
@@ -668,7 +668,6 @@ tc_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         fence_before_sync();
         ok = __syncthreads_and(ok);
         if (tid == 0) {
-            if (has_next) issue_v(s_next_hl[0], s_next[1]);  // the v tile is free: MMA2 has read it
             if (ok) {
                 // W and Uv images out (bulk), then [P W | P Uv] = P [W | Uv]
                 bulk_s2g(slot + kSlotW, sb + kA_KQ, 8192);
@@ -684,7 +683,6 @@ tc_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 mma_commit(mbar);
             }
-            bulk_wait_read();  // the Uv tile is overwritten by O0 below
         }
         ok = mbar_wait_ab(mbar, mphase, s_abort) && ok;
         mphase ^= 1;
@@ -712,7 +710,7 @@ tc_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         *p = pack8(qf);
                     }
                 }
-            } else {  // O0 = P Uv -> the Uv tile's place
+            } else {  // O0 = P Uv -> the v tile's place (MMA2 has read v; the Uv image may still be leaving)
 #pragma unroll
                 for (int b2 = 0; b2 < 64; b2 += 32) {
                     float a2[32];
@@ -721,24 +719,27 @@ tc_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     tmem_wait_ld();
 #pragma unroll
                     for (int m = 0; m < 4; ++m)
-                        *reinterpret_cast<uint4*>(sm + kA_B + sw128_chunk_off(rowq, (hc + b2) / 8 + m, 64)) = pack8(a2 + 8 * m);
+                        *reinterpret_cast<uint4*>(sm + kA_V + sw128_chunk_off(rowq, (hc + b2) / 8 + m, 64)) = pack8(a2 + 8 * m);
                 }
             }
         }
         fence_proxy_async();
         fence_before_sync();
         __syncthreads();
-        if (tid == 0) {  // Q' and O0 images out; then the next chunk's k and q take the stacked tile
+        if (tid == 0) {  // Q' and O0 images out; then the next chunk's k, q and v take their tiles
             if (ok) {
                 bulk_s2g(slot + kSlotQ, sb + kA_KQ + 8192, 8192);
                 bulk_s2g(slot + kSlotQ + 8192, sb + kA_KQ + kKQ_LBO + 8192, 8192);
-                bulk_s2g(slot + kSlotO0, sb + kA_B, 16384);
+                bulk_s2g(slot + kSlotO0, sb + kA_V, 16384);
                 bulk_commit();
             }
-            bulk_wait_read();
-            if (has_next) issue_kq(s_next_hl[0], s_next[1]);
+            bulk_wait_read();  // every image of this unit has been read out of shared memory
+            if (has_next) {
+                issue_kq(s_next_hl[0], s_next[1]);
+                issue_v(s_next_hl[0], s_next[1]);
+            }
         }
-        ok = __syncthreads_and(ok);  // the Kb tile of the next chunk may overwrite O0 from here on
+        ok = __syncthreads_and(ok);  // the Kb tile of the next chunk may overwrite the Uv image from here on
         if (!ok) break;
         u = s_next[0];
         t0 = s_next[1];

@@ -722,24 +722,27 @@ tc_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         *reinterpret_cast<uint4*>(sm + kA_V + sw128_chunk_off(rowq, (hc + b2) / 8 + m, 64)) = pack8(a2 + 8 * m);
                 }
             }
-        }
-        fence_proxy_async();
-        fence_before_sync();
-        __syncthreads();
-        if (tid == 0) {  // Q' and O0 images out; then the next chunk's k, q and v take their tiles
-            if (ok) {
-                bulk_s2g(slot + kSlotQ, sb + kA_KQ + 8192, 8192);
-                bulk_s2g(slot + kSlotQ + 8192, sb + kA_KQ + kKQ_LBO + 8192, 8192);
-                bulk_s2g(slot + kSlotO0, sb + kA_V, 16384);
+            // the warp's 16 rows of its image (Q' or O0) leave at once: one 2 KB run per atom column.
+            // The issuing lane waits until they have been read (bulk groups are per thread); thread 0's
+            // wait also covers the W and Uv images.
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) {
+                const uint32_t src = warp < 4 ? sb + kA_KQ + 8192 + 2048 * wq : sb + kA_V + 2048 * wq;
+                const uint32_t lbo = warp < 4 ? kKQ_LBO : 8192u;
+                uint8_t* dst = slot + (warp < 4 ? kSlotQ : kSlotO0) + 2048 * wq;
+                bulk_s2g(dst, src, 2048);
+                bulk_s2g(dst + 8192, src + lbo, 2048);
                 bulk_commit();
             }
-            bulk_wait_read();  // every image of this unit has been read out of shared memory
-            if (has_next) {
-                issue_kq(s_next_hl[0], s_next[1]);
-                issue_v(s_next_hl[0], s_next[1]);
-            }
         }
-        ok = __syncthreads_and(ok);  // the Kb tile of the next chunk may overwrite the Uv image from here on
+        if (lane == 0) bulk_wait_read();  // every image of this unit has been read out of shared memory
+        fence_before_sync();
+        ok = __syncthreads_and(ok);  // the next chunk's tiles (k, q, v; Kb over the Uv image) may land from here on
+        if (tid == 0 && has_next) {
+            issue_kq(s_next_hl[0], s_next[1]);
+            issue_v(s_next_hl[0], s_next[1]);
+        }
         if (!ok) break;
         u = s_next[0];
         t0 = s_next[1];
@@ -753,8 +756,8 @@ tc_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             (void)mbar_wait(mbar_kq, pn);
             (void)mbar_wait(mbar_v, pn);
         }
-        bulk_wait_all();
     }
+    if (lane == 0) bulk_wait_all();  // every lane that issued image stores
     cp_async_wait_all();
     fence_before_sync();
     __syncthreads();

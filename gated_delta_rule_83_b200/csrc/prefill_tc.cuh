@@ -796,6 +796,19 @@ __device__ __forceinline__ void tc_issue_stage(uint32_t stage_addr, uint32_t ful
     bulk_g2s(stage_addr + kStGam, slot + kSlotGam, 512, full_bar);
 }
 
+// the same regions of a chunk's slot, into L2 only, a few chunks before tc_issue_stage needs them
+__device__ __forceinline__ void tc_prefetch_stage(const uint8_t* slot, int vt)
+{
+    using namespace tc;
+    bulk_prefetch_l2(slot + kSlotW, 16384);
+    bulk_prefetch_l2(slot + kSlotQ, 16384);
+    bulk_prefetch_l2(slot + kSlotKd, 16384);
+    bulk_prefetch_l2(slot + kSlotUv + (vt >> 1) * 8192, 8192);
+    bulk_prefetch_l2(slot + kSlotO0 + (vt >> 1) * 8192, 8192);
+    bulk_prefetch_l2(slot + kSlotGam, 512);
+}
+constexpr int kBPrefetch = 2;  // L2 prefetch distance beyond the shared-memory stages (chunks)
+
 __global__ void __launch_bounds__(kBThreads, 1)
 tc_inter_kernel(const float* S0, float* S_final, __nv_bfloat16* __restrict__ out, const WsHeader* __restrict__ hdr,
                 const int* __restrict__ off, const int32_t* __restrict__ cu, int Tseq, int N, int H,
@@ -854,9 +867,12 @@ tc_inter_kernel(const float* S0, float* S_final, __nv_bfloat16* __restrict__ out
     }
     fence_proxy_async();
     __syncthreads();  // barriers initialised, TMEM address visible, S tile written
-    if (warp == 5 && lane == 0)
+    if (warp == 5 && lane == 0) {
         for (int s = 0; s < kBStages && s < nch; ++s)
             tc_issue_stage(sb + s * kStageBytes, bar_full + 8 * s, slots + ((size_t)(jb + s) * H + h) * kSlotBytes, vt);
+        for (int s = kBStages; s < kBStages + kBPrefetch && s < nch; ++s)
+            tc_prefetch_stage(slots + ((size_t)(jb + s) * H + h) * kSlotBytes, vt);
+    }
     const uint32_t tmem = *s_tmem;
     const uint32_t tw = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
     const uint32_t id_d1 = idesc_bf16(128, kTcNV, false, true);  // [W; Q'] S   (S MN-major)
@@ -909,11 +925,20 @@ tc_inter_kernel(const float* S0, float* S_final, __nv_bfloat16* __restrict__ out
         } else if (warp == 5) {
             if (refill && lane == 0) {  // stage s fully consumed (128 compute-thread arrivals) -> refill
                 ok = ok && mbar_wait_ab(bar_empty + 8 * s, (uint32_t)(it / kBStages) & 1u, s_abort);
-                if (ok)
+                if (ok) {
                     tc_issue_stage(st, bar_full + 8 * s, slots + ((size_t)(jb + it + kBStages) * H + h) * kSlotBytes, vt);
+                    if (it + kBStages + kBPrefetch < nch)
+                        tc_prefetch_stage(slots + ((size_t)(jb + it + kBStages + kBPrefetch) * H + h) * kSlotBytes, vt);
+                }
             }
         } else {
             ok = ok && mbar_wait_ab(bar_full + 8 * s, (uint32_t)(it / kBStages) & 1u, s_abort);
+            // this thread's Uv (warps 0-1) or O0 (warps 2-3) row and e^{g_last} are read before MMA1 is waited for
+            uint4 raw[4];
+#pragma unroll
+            for (int m = 0; m < 4; ++m)
+                raw[m] = *reinterpret_cast<const uint4*>(stp + (warp < 2 ? kStUv : kStO0) + sw128_chunk_off(c & 63, cq + m, 64));
+            const float gam = *reinterpret_cast<const float*>(stp + kStGam + 4 * c);
             ok = ok && mbar_wait_ab(bar_d1, par, s_abort);
             fence_after_sync();
             float x[32];
@@ -921,9 +946,6 @@ tc_inter_kernel(const float* S0, float* S_final, __nv_bfloat16* __restrict__ out
             tmem_ld16(tw + kTmD1 + 16, x + 16);
             tmem_wait_ld();
             if (warp < 2) {  // U = Uv - X, row r = c
-                uint4 raw[4];
-#pragma unroll
-                for (int m = 0; m < 4; ++m) raw[m] = *reinterpret_cast<const uint4*>(stp + kStUv + sw128_chunk_off(c, cq + m, 64));
                 uint4 pk[4];
 #pragma unroll
                 for (int m = 0; m < 4; ++m) {
@@ -939,9 +961,6 @@ tc_inter_kernel(const float* S0, float* S_final, __nv_bfloat16* __restrict__ out
                 named_arrive(1, 96);
             } else {  // out = O' + O0, row r = c - 64
                 const int r = c - 64;
-                uint4 raw[4];
-#pragma unroll
-                for (int m = 0; m < 4; ++m) raw[m] = *reinterpret_cast<const uint4*>(stp + kStO0 + sw128_chunk_off(r & 63, cq + m, 64));
                 if (r < L && ok) {
                     uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)(t0 + r) * H + h) * 128 + v0);
 #pragma unroll
@@ -954,7 +973,6 @@ tc_inter_kernel(const float* S0, float* S_final, __nv_bfloat16* __restrict__ out
                     }
                 }
             }
-            const float gam = *reinterpret_cast<const float*>(stp + kStGam + 4 * c);
             ok = ok && mbar_wait_ab(bar_y, par, s_abort);
             fence_after_sync();
             if (refill) mbar_arrive(bar_empty + 8 * s);  // last read of stage s done (MMAs on it complete)

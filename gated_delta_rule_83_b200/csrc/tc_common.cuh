@@ -183,6 +183,13 @@ __device__ __forceinline__ bool mbar_wait_ab(uint32_t addr, uint32_t parity, vol
 }
 
 // ---- bulk copy global -> shared (completion counted on an mbarrier) ---------------------------
+// bulk prefetch of a global range into L2 (no shared memory, no completion to wait for); address and
+// size multiples of 16 bytes
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ void bulk_g2s(uint32_t dst_smem, const void* src, uint32_t bytes, uint32_t mbar)
 {
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(

@@ -807,7 +807,7 @@ __device__ __forceinline__ void tc_prefetch_stage(const uint8_t* slot, int vt)
     bulk_prefetch_l2(slot + kSlotO0 + (vt >> 1) * 8192, 8192);
     bulk_prefetch_l2(slot + kSlotGam, 512);
 }
-constexpr int kBPrefetch = 2;  // L2 prefetch distance beyond the shared-memory stages (chunks)
+constexpr int kBPrefetch = 4;  // L2 prefetch distance beyond the shared-memory stages (chunks)
 
 __global__ void __launch_bounds__(kBThreads, 1)
 tc_inter_kernel(const float* S0, float* S_final, __nv_bfloat16* __restrict__ out, const WsHeader* __restrict__ hdr,

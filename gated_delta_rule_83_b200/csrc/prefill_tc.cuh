@@ -479,22 +479,42 @@ tc_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
 
         if (!wide) {
+            // a lane's 8 channels span 32 bytes of fp32 rows: lanes 4-7 of each quarter-warp read their
+            // upper 16 bytes first, so that one 128-bit load instruction covers all eight 16-byte bank
+            // groups of a 128-byte line (no two-way conflict)
+            const int h0 = 4 * ((ch >> 2) & 1);
+            float ref8[8], d8[8];
+            {
+                const float4 a0 = *reinterpret_cast<const float4*>(s_ref + 8 * ch + h0);
+                const float4 a1 = *reinterpret_cast<const float4*>(s_ref + 8 * ch + (h0 ^ 4));
+                const float4 b0 = *reinterpret_cast<const float4*>(s_D + 8 * ch + h0);
+                const float4 b1 = *reinterpret_cast<const float4*>(s_D + 8 * ch + (h0 ^ 4));
+                const float x0[4] = {a0.x, a0.y, a0.z, a0.w}, x1[4] = {a1.x, a1.y, a1.z, a1.w};
+                const float y0[4] = {b0.x, b0.y, b0.z, b0.w}, y1[4] = {b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    ref8[m] = h0 ? x1[m] : x0[m];
+                    ref8[m + 4] = h0 ? x0[m] : x1[m];
+                    d8[m] = h0 ? y1[m] : y0[m];
+                    d8[m + 4] = h0 ? y0[m] : y1[m];
+                }
+            }
 #pragma unroll
             for (int jj = 0; jj < 4; ++jj) {
                 const int r = rb + 16 * jj;
-                const float4 ra = *reinterpret_cast<const float4*>(s_ref + 8 * ch);
-                const float4 rbv = *reinterpret_cast<const float4*>(s_ref + 8 * ch + 4);
-                const float4 da = *reinterpret_cast<const float4*>(s_D + 8 * ch);
-                const float4 db = *reinterpret_cast<const float4*>(s_D + 8 * ch + 4);
-                const float ref8[8] = {ra.x, ra.y, ra.z, ra.w, rbv.x, rbv.y, rbv.z, rbv.w};
-                const float d8[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
                 const uint32_t ok_ = sw128_chunk_off(r, ch, 128), oq = sw128_chunk_off(64 + r, ch, 128);
                 float kv[8], qv[8];
                 unpack8(*reinterpret_cast<const uint4*>(sm + kA_KQ + ok_), kv);
                 unpack8(*reinterpret_cast<const uint4*>(sm + kA_KQ + oq), qv);
-                const float4 ga = *reinterpret_cast<const float4*>(sG + r * kGS + 8 * ch);
-                const float4 gb = *reinterpret_cast<const float4*>(sG + r * kGS + 8 * ch + 4);
-                const float g8[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+                const float4 ga = *reinterpret_cast<const float4*>(sG + r * kGS + 8 * ch + h0);
+                const float4 gb = *reinterpret_cast<const float4*>(sG + r * kGS + 8 * ch + (h0 ^ 4));
+                const float gx[4] = {ga.x, ga.y, ga.z, ga.w}, gy[4] = {gb.x, gb.y, gb.z, gb.w};
+                float g8[8];
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    g8[m] = h0 ? gy[m] : gx[m];
+                    g8[m + 4] = h0 ? gx[m] : gy[m];
+                }
                 float kf[8], qf[8], kb[8], kd[8];
 #pragma unroll
                 for (int m = 0; m < 8; ++m) {

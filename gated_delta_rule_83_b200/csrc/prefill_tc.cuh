@@ -624,14 +624,26 @@ tc_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // UT transform (X in place of A), then T = X diag(beta) as a bf16 K-major tile over Kb
         if (ok) ut_inverse_64_inplace(sA, sY);
         uint4 tch[2];
+        {   // 128-bit loads of the 8 values; lanes 4-7 of a quarter-warp take their upper half first so
+            // that no two lanes of a load share a bank group
+            const int c8 = tid & 7, hs = 4 * ((tid >> 2) & 1);
+            const float4 b0 = *reinterpret_cast<const float4*>(s_beta + 8 * c8 + hs);
+            const float4 b1 = *reinterpret_cast<const float4*>(s_beta + 8 * c8 + (hs ^ 4));
 #pragma unroll
-        for (int u2 = 0; u2 < 2; ++u2) {
-            const int e = tid + kAThreads * u2;
-            const int r = e >> 3, c8 = e & 7;
-            float t8[8];
+            for (int u2 = 0; u2 < 2; ++u2) {
+                const int r = (tid + kAThreads * u2) >> 3;
+                const float4 x0 = *reinterpret_cast<const float4*>(sA + r * kAS + 8 * c8 + hs);
+                const float4 x1 = *reinterpret_cast<const float4*>(sA + r * kAS + 8 * c8 + (hs ^ 4));
+                const float p0[4] = {x0.x * b0.x, x0.y * b0.y, x0.z * b0.z, x0.w * b0.w};
+                const float p1[4] = {x1.x * b1.x, x1.y * b1.y, x1.z * b1.z, x1.w * b1.w};
+                float t8[8];
 #pragma unroll
-            for (int m = 0; m < 8; ++m) t8[m] = sA[r * kAS + 8 * c8 + m] * s_beta[8 * c8 + m];
-            tch[u2] = pack8(t8);
+                for (int m = 0; m < 4; ++m) {
+                    t8[m] = hs ? p1[m] : p0[m];
+                    t8[m + 4] = hs ? p0[m] : p1[m];
+                }
+                tch[u2] = pack8(t8);
+            }
         }
         __syncthreads();
 #pragma unroll

@@ -3,6 +3,9 @@
 // included below; this file only checks arguments and launches.
 #include <cstdio>
 #include <cstring>
+#include <memory>
+#include <mutex>
+#include <vector>
 
 #include "kda.h"
 #include "backward_simt.cuh"
@@ -416,31 +419,22 @@ kda_status kda_check(kda_stream_t stream_)
 // their own pool up front, plugin hooks that forbid cudaMalloc, fixed memory budgets), the
 // workspace comes from a static device array compiled into this file instead of from the caller.
 // The array exists once per GPU that loads the library and lives until the process exits.  In
-// host code its name is only a host-side stand-in, so its device address is looked up (once per
-// device, with that device current) with cudaGetSymbolAddress and passed to the kernels like any
-// other workspace pointer.  All calls on a device share the array; calls that overlap on the GPU
-// race.  Every scratch byte a kernel reads is written earlier in the same call, so nothing needs
-// clearing between calls.
+// host code its name is only a host-side stand-in, so its device address is looked up with
+// cudaGetSymbolAddress on every call, on the device current at the call, and passed to the
+// kernels like any other workspace pointer (a host-side lookup: no allocation, no stream work;
+// looking it up each time also follows the module if the device's context is ever recreated).
+// All calls on a device share the array; calls that overlap on the GPU race.  Every scratch byte
+// a kernel reads is written earlier in the same call, so nothing needs clearing between calls.
 // ------------------------------------------------------------------------------------------------
 static __device__ __align__(256) unsigned char g_noalloc_scratch[KDA_NOALLOC_SCRATCH_BYTES];
 
 namespace {
 
-constexpr int kNoallocMaxDevices = 64;
-std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kNoallocMaxDevices] = {};
-
 kda_status noalloc_scratch_address(void** ptr)
 {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoallocMaxDevices) return KDA_ERR_CUDA;
-    std::lock_guard<std::mutex> g(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return KDA_ERR_CUDA;
-        g_noalloc_ptr[dev] = p;
-    }
-    *ptr = g_noalloc_ptr[dev];
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return KDA_ERR_CUDA;
+    *ptr = p;
     return KDA_OK;
 }
 
@@ -501,6 +495,79 @@ kda_status make_host_plan(int B, int T, int H, int Hk, int dk, int dv, kda_dtype
 
 }  // namespace
 
+namespace {
+
+// Copy streams and events of kda_chunk_fwd_host, created on the first call for a (device, caller
+// stream) pair and reused by every later call on that pair (kda_host_release() destroys them).
+struct HostRes {
+    int dev = -1;
+    cudaStream_t caller = nullptr;
+    cudaStream_t cin = nullptr, cout = nullptr;
+    cudaEvent_t ev_in[2] = {}, ev_comp[2] = {}, ev_out[2] = {}, ev_start = nullptr;
+    std::mutex mu;
+};
+
+std::mutex g_host_mu;
+std::vector<std::unique_ptr<HostRes>> g_host_res;
+
+void destroy_host_res(HostRes& r)
+{
+    for (int i = 0; i < 2; ++i) {
+        if (r.ev_in[i]) cudaEventDestroy(r.ev_in[i]);
+        if (r.ev_comp[i]) cudaEventDestroy(r.ev_comp[i]);
+        if (r.ev_out[i]) cudaEventDestroy(r.ev_out[i]);
+    }
+    if (r.ev_start) cudaEventDestroy(r.ev_start);
+    if (r.cin) cudaStreamDestroy(r.cin);
+    if (r.cout) cudaStreamDestroy(r.cout);
+}
+
+HostRes* host_resources(cudaStream_t caller)
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+    std::lock_guard<std::mutex> g(g_host_mu);
+    for (auto& r : g_host_res)
+        if (r->dev == dev && r->caller == caller) return r.get();
+    auto r = std::make_unique<HostRes>();
+    r->dev = dev;
+    r->caller = caller;
+    bool ok = cudaStreamCreateWithFlags(&r->cin, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&r->cout, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&r->ev_start, cudaEventDisableTiming) == cudaSuccess;
+    for (int i = 0; i < 2 && ok; ++i)
+        ok = cudaEventCreateWithFlags(&r->ev_in[i], cudaEventDisableTiming) == cudaSuccess &&
+             cudaEventCreateWithFlags(&r->ev_comp[i], cudaEventDisableTiming) == cudaSuccess &&
+             cudaEventCreateWithFlags(&r->ev_out[i], cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) {
+        destroy_host_res(*r);
+        return nullptr;
+    }
+    g_host_res.push_back(std::move(r));
+    return g_host_res.back().get();
+}
+
+}  // namespace
+
+extern "C" kda_status kda_host_release(void)
+{
+    std::lock_guard<std::mutex> g(g_host_mu);
+    int cur = -1;
+    const bool have_cur = cudaGetDevice(&cur) == cudaSuccess;
+    kda_status st = KDA_OK;
+    for (auto& r : g_host_res) {
+        std::lock_guard<std::mutex> call_guard(r->mu);
+        if (cudaSetDevice(r->dev) != cudaSuccess) st = KDA_ERR_CUDA;
+        // work queued on these streams completes first; then they are released
+        if (cudaStreamSynchronize(r->cin) != cudaSuccess || cudaStreamSynchronize(r->cout) != cudaSuccess)
+            st = KDA_ERR_CUDA;
+        destroy_host_res(*r);
+    }
+    g_host_res.clear();
+    if (have_cur) cudaSetDevice(cur);
+    return st;
+}
+
 extern "C" kda_status kda_chunk_fwd_host_workspace_size(int B, int T, int H, int dk, int dv, kda_dtype dt,
                                                         const kda_options* opt, int segment_tokens, size_t* bytes)
 {
@@ -545,20 +612,18 @@ extern "C" kda_status kda_chunk_fwd_host(const void* q, const void* k, const voi
     const char* src[5] = {(const char*)q, (const char*)k, (const char*)v, (const char*)log_alpha,
                           (const char*)beta};
 
-    cudaStream_t cin = nullptr, cout = nullptr;
-    cudaEvent_t ev_in[2] = {nullptr, nullptr}, ev_comp[2] = {nullptr, nullptr}, ev_out[2] = {nullptr, nullptr};
-    cudaEvent_t ev_start = nullptr;
+    HostRes* hr = host_resources(stream);
+    if (!hr) return KDA_ERR_CUDA;
+    std::lock_guard<std::mutex> call_guard(hr->mu);  // one call at a time on these copy streams
+    cudaStream_t cin = hr->cin, cout = hr->cout;
+    cudaEvent_t* ev_in = hr->ev_in;
+    cudaEvent_t* ev_comp = hr->ev_comp;
+    cudaEvent_t* ev_out = hr->ev_out;
     kda_status rs = KDA_ERR_CUDA;
-    bool ok = cudaStreamCreateWithFlags(&cin, cudaStreamNonBlocking) == cudaSuccess &&
-              cudaStreamCreateWithFlags(&cout, cudaStreamNonBlocking) == cudaSuccess &&
-              cudaEventCreateWithFlags(&ev_start, cudaEventDisableTiming) == cudaSuccess;
-    for (int i = 0; i < 2 && ok; ++i)
-        ok = cudaEventCreateWithFlags(&ev_in[i], cudaEventDisableTiming) == cudaSuccess &&
-             cudaEventCreateWithFlags(&ev_comp[i], cudaEventDisableTiming) == cudaSuccess &&
-             cudaEventCreateWithFlags(&ev_out[i], cudaEventDisableTiming) == cudaSuccess;
     // the copy streams start after everything already queued on the caller's stream
-    ok = ok && cudaEventRecord(ev_start, stream) == cudaSuccess && cudaStreamWaitEvent(cin, ev_start, 0) == cudaSuccess &&
-         cudaStreamWaitEvent(cout, ev_start, 0) == cudaSuccess;
+    bool ok = cudaEventRecord(hr->ev_start, stream) == cudaSuccess &&
+              cudaStreamWaitEvent(cin, hr->ev_start, 0) == cudaSuccess &&
+              cudaStreamWaitEvent(cout, hr->ev_start, 0) == cudaSuccess;
     const size_t sbytes = sizeof(float) * (size_t)B * H * dk * dv;
     if (ok) ok = (S0 ? cudaMemcpyAsync(state, S0, sbytes, cudaMemcpyHostToDevice, stream)
                      : cudaMemsetAsync(state, 0, sbytes, stream)) == cudaSuccess;
@@ -604,13 +669,5 @@ extern "C" kda_status kda_chunk_fwd_host(const void* q, const void* k, const voi
     for (int b = 0; b < 2 && ok; ++b)
         if (p.nseg > b) ok = cudaStreamWaitEvent(stream, ev_out[b], 0) == cudaSuccess;
     if (ok) rs = KDA_OK;
-    for (int i = 0; i < 2; ++i) {
-        if (ev_in[i]) cudaEventDestroy(ev_in[i]);
-        if (ev_comp[i]) cudaEventDestroy(ev_comp[i]);
-        if (ev_out[i]) cudaEventDestroy(ev_out[i]);
-    }
-    if (ev_start) cudaEventDestroy(ev_start);
-    if (cin) cudaStreamDestroy(cin);
-    if (cout) cudaStreamDestroy(cout);
     return rs;
 }

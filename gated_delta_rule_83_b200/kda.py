@@ -55,6 +55,7 @@ ABI = {
                                               ctypes.POINTER(_SZ)]),
     "kda_chunk_fwd_host": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.POINTER(KdaOptions),
                                 _I, _P, _SZ, _P]),
+    "kda_host_release": (_I, []),
     "kda_check": (_I, [_P]),
     "kda_selftest_timeout": (_I, [_P]),
     "kda_profile_begin": (_I, []),
@@ -142,6 +143,12 @@ def release_workspaces() -> None:
     """Drop the cached per-stream workspaces (the backward's can be several GB).  Calls made after
     this allocate again on first use; pass ``workspace=`` to manage the memory yourself."""
     _workspaces.clear()
+
+
+def release_host_resources() -> None:
+    """Destroy the copy streams and events that ``chunk_fwd_host`` keeps per (device, stream)
+    (``kda_host_release``); later calls create them again."""
+    _check("kda_host_release", load_library().kda_host_release())
 
 
 def workspace_size(B: int, T: int, H: int, dk: int, dv: int, varlen: bool = False, num_seqs: int = 0,
@@ -375,23 +382,67 @@ def chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torc
 NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024  # KDA_NOALLOC_SCRATCH_BYTES in include/kda.h
 
 
+def _check_noalloc_args(q, k, v, log_alpha, beta, S0, out, S_final, cu_seqlens):
+    """Argument checks of ``chunk_fwd_noalloc``, types and shapes first, placement last, so that a
+    malformed call raises before any pointer reaches the library.  Returns (B, T, H, dk, dv, N)."""
+    named = (("q", q), ("k", k), ("v", v), ("log_alpha", log_alpha), ("beta", beta), ("out", out))
+    for name, t in named + (("S0", S0), ("S_final", S_final), ("cu_seqlens", cu_seqlens)):
+        if t is not None and not isinstance(t, torch.Tensor):
+            raise TypeError(f"{name} must be a torch.Tensor")
+    for name, t in named:
+        if t is None:
+            raise TypeError(f"{name} is required")
+    if q.dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError(f"q must be bfloat16 or float32, got {q.dtype}")
+    for name, t in (("k", k), ("v", v), ("out", out)):
+        if t.dtype != q.dtype:
+            raise TypeError(f"{name} must be {q.dtype}, got {t.dtype}")
+    # the entry point takes float* gates: a bf16 log_alpha would be read past its end
+    for name, t in (("log_alpha", log_alpha), ("beta", beta), ("S0", S0), ("S_final", S_final)):
+        if t is not None and t.dtype != torch.float32:
+            raise TypeError(f"{name} must be torch.float32, got {t.dtype}")
+    if q.dim() != 4 or v.dim() != 4:
+        raise ValueError("q must be [B, T, H, dk] and v [B, T, H, dv]")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if tuple(k.shape) != (B, T, H, dk) or tuple(v.shape) != (B, T, H, dv) or \
+            tuple(log_alpha.shape) != (B, T, H, dk) or tuple(beta.shape) != (B, T, H):
+        raise ValueError("inconsistent shapes (the allocation-free entry point has no grouped q/k heads)")
+    if tuple(out.shape) != (B, T, H, dv):
+        raise ValueError(f"out must be [{B}, {T}, {H}, {dv}]")
+    N = B
+    if cu_seqlens is not None:
+        if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2:
+            raise TypeError("cu_seqlens must be a 1-D torch.int32 tensor of N + 1 offsets")
+        if B != 1:
+            raise ValueError("packed varlen input needs B == 1")
+        N = cu_seqlens.numel() - 1
+    for name, t in (("S0", S0), ("S_final", S_final)):
+        if t is not None and tuple(t.shape) != (N, H, dk, dv):
+            raise ValueError(f"{name} must be [{N}, {H}, {dk}, {dv}]")
+    dev = q.device
+    for name, t in named + (("S0", S0), ("S_final", S_final), ("cu_seqlens", cu_seqlens)):
+        if t is not None:
+            _req(t, name, None, dev)
+    return B, T, H, dk, dv, N
+
+
 def chunk_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor,
-                      beta: torch.Tensor, S0: torch.Tensor, out: torch.Tensor, S_final: Optional[torch.Tensor],
-                      cu_seqlens: Optional[torch.Tensor] = None,
+                      beta: torch.Tensor, S0: Optional[torch.Tensor], out: torch.Tensor,
+                      S_final: Optional[torch.Tensor], cu_seqlens: Optional[torch.Tensor] = None,
                       stream: Optional[torch.cuda.Stream] = None) -> None:
     """``kda_chunk_fwd_noalloc``: the chunked prefill for callers that cannot allocate device memory
     (the library's built-in scratch replaces the workspace).  Every buffer, ``out`` and ``S_final``
-    included, is the caller's; nothing is allocated here either.  Problems whose workspace would
-    exceed ``NOALLOC_SCRATCH_BYTES`` raise ``KdaError`` (KDA_ERR_WORKSPACE)."""
+    included, is the caller's; nothing is allocated here either.  Shapes as ``chunk_fwd`` with
+    Hk = H; log_alpha, beta, S0 and S_final fp32 (S0 None = zero state, S_final None = not
+    written).  Problems whose workspace would exceed ``NOALLOC_SCRATCH_BYTES`` raise ``KdaError``
+    (KDA_ERR_WORKSPACE)."""
+    B, T, H, dk, dv, N = _check_noalloc_args(q, k, v, log_alpha, beta, S0, out, S_final, cu_seqlens)
     lib = load_library()
-    B, T, H, dk = q.shape
-    dv = v.shape[-1]
-    N = B if cu_seqlens is None else cu_seqlens.numel() - 1
-    for t, name in ((q, "q"), (k, "k"), (v, "v"), (log_alpha, "log_alpha"), (beta, "beta"), (out, "out")):
-        _req(t, name)
-    rc = lib.kda_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0),
-                                   _ptr(cu_seqlens), N, _ptr(out), _ptr(S_final), B, T, H, dk, dv, _dt(q),
-                                   _stream_handle(stream, q.device))
+    with torch.cuda.device(q.device):  # the scratch address is looked up on the current device
+        rc = lib.kda_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0),
+                                       _ptr(cu_seqlens), N, _ptr(out), _ptr(S_final), B, T, H, dk, dv, _dt(q),
+                                       _stream_handle(stream, q.device))
     _check("kda_chunk_fwd_noalloc", rc)
 
 

@@ -200,8 +200,10 @@ kda_status kda_decode_step_ex(const void* q, const void* k, const void* v, const
  *   workspace    DEVICE memory, >= kda_chunk_fwd_host_workspace_size(...) bytes, 256-byte aligned:
  *                two input and two output segment buffers, the state and the chunk workspace.
  * Asynchronous on `stream`: the host buffers must stay untouched, and out / S_final are complete,
- * only once `stream` has been synchronised (the call's copy streams are joined into it).  Creates
- * and destroys two streams and a few events per call.  Errors: as kda_chunk_fwd_ex, and
+ * only once `stream` has been synchronised (the call's copy streams are joined into it).  The two
+ * copy streams and their events are created by the first call for a (current device, `stream`)
+ * pair and reused by every later call on that pair (calls on one pair from several host threads
+ * are serialised on the host); kda_host_release() destroys them.  Errors: as kda_chunk_fwd_ex, and
  * KDA_ERR_INVALID_ARG for a segment length that is not a positive multiple of 64, T <= 0 or a NULL
  * input; after KDA_ERR_CUDA the outputs are undefined.
  */
@@ -211,6 +213,13 @@ kda_status kda_chunk_fwd_host(const void* q, const void* k, const void* v, const
                               const float* beta, const float* S0, void* out, float* S_final, int B, int T,
                               int H, int dk, int dv, kda_dtype dt, const kda_options* opt, int segment_tokens,
                               void* workspace, size_t workspace_bytes, kda_stream_t stream);
+
+/*
+ * kda_host_release -- waits for the copy streams that kda_chunk_fwd_host keeps per (device, caller
+ * stream) pair and destroys them and their events, on every device that has some.  Later calls
+ * create them again.  Returns KDA_OK, or KDA_ERR_CUDA if a synchronisation or destroy failed.
+ */
+kda_status kda_host_release(void);
 
 /*
  * kda_chunk_bwd -- the backward pass of kda_chunk_fwd (training): the derivatives of a scalar loss

@@ -199,3 +199,63 @@ def test_backward_rejects_before_launch(lib):
     nul = list(base)
     nul[10] = None                                                            # no dq
     assert lib.kda_chunk_bwd(*nul, None, fake, 1 << 40, None) == 1
+
+
+def _noalloc_inputs(B=1, T=100, H=2, d=128, dtype=None):
+    import torch
+    dt = dtype or torch.bfloat16
+    z = lambda *s, t=dt: torch.zeros(*s, dtype=t)
+    return dict(q=z(B, T, H, d), k=z(B, T, H, d), v=z(B, T, H, d), log_alpha=z(B, T, H, d, t=torch.float32),
+                beta=z(B, T, H, t=torch.float32), S0=z(B, H, d, d, t=torch.float32), out=z(B, T, H, d),
+                S_final=z(B, H, d, d, t=torch.float32))
+
+
+@pytest.mark.parametrize("field,bad,exc", [
+    ("log_alpha", "bf16", TypeError),      # the entry point reads float gates: bf16 would overrun
+    ("beta", "bf16", TypeError),
+    ("S0", "bf16", TypeError),
+    ("S_final", "f64", TypeError),
+    ("k", "f32", TypeError),               # q/k/v/out share one dtype
+    ("out", "f32", TypeError),
+    ("k", "shape", ValueError),
+    ("v", "shape", ValueError),
+    ("log_alpha", "shape", ValueError),
+    ("beta", "shape", ValueError),
+    ("S0", "shape", ValueError),
+    ("out", "shape", ValueError),
+    ("S_final", "shape", ValueError),
+    ("out", None, TypeError),              # out is required
+    ("q", "cpu", ValueError),              # well-formed but not on a GPU
+])
+def test_noalloc_binding_rejects_bad_arguments(field, bad, exc):
+    """chunk_fwd_noalloc checks dtypes and shapes before placement and before touching the
+    library, so every malformed call raises here without a GPU (and without a launch on one)."""
+    import torch
+    import gated_delta_rule_83_b200 as m
+    a = _noalloc_inputs()
+    t = a[field]
+    if bad == "bf16":
+        a[field] = t.to(torch.bfloat16)
+    elif bad == "f32":
+        a[field] = t.float()
+    elif bad == "f64":
+        a[field] = t.double()
+    elif bad == "shape":
+        a[field] = t[..., :-1] if t.dim() > 1 else t[:-1]
+    elif bad is None:
+        a[field] = None
+    with pytest.raises(exc):
+        m.chunk_fwd_noalloc(a["q"], a["k"], a["v"], a["log_alpha"], a["beta"], a["S0"], a["out"], a["S_final"])
+
+
+def test_noalloc_scratch_limit_boundary(lib):
+    """The built-in scratch (KDA_NOALLOC_SCRATCH_BYTES) holds 25 chunks of 32 heads at bf16, d = 128:
+    1,600 tokens fit, 1,664 are rejected on the host with KDA_ERR_WORKSPACE."""
+    from gated_delta_rule_83_b200 import kda
+    limit = kda.NOALLOC_SCRATCH_BYTES
+    assert _ws(lib, 1, 1600, 32, 128, 128, 0, 0, 0)[1] <= limit
+    assert _ws(lib, 1, 1664, 32, 128, 128, 0, 0, 0)[1] > limit
+    fake = ctypes.c_void_p(0x100000)  # never dereferenced: the size check comes first
+    rc = lib.kda_chunk_fwd_noalloc(fake, fake, fake, fake, fake, None, None, 0, fake, None, 1, 1664, 32, 128, 128, 0,
+                                   None)
+    assert rc == 5

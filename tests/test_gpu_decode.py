@@ -50,9 +50,13 @@ def test_decode_256x512_sampled():
         og = np.stack([np64(out[n, h]) for n, h in pairs])[:, None]
         worst = max(worst, out_err(og, o_ref))
     m.check()
-    assert worst <= TOL["bf16"][0]
     sg = np.stack([np64(S[n, h]) for n, h in pairs])[:, None]
-    assert state_err(sg, S_ref) <= TOL["bf16"][1]
+    es = state_err(sg, S_ref)
+    print(f"\nPARITY decode_256x512 pairs {pairs}: worst max-abs out error / max|o| over 512 steps = {worst:.3e} "
+          f"(tol {TOL['bf16'][0]:g}); relative Frobenius state error after 512 steps = {es:.3e} "
+          f"(tol {TOL['bf16'][1]:g})")
+    assert worst <= TOL["bf16"][0]
+    assert es <= TOL["bf16"][1]
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])

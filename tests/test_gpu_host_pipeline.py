@@ -76,3 +76,25 @@ def test_host_pipeline_without_state_buffers():
     assert sf is None
     o_dev, _ = device_call(inp)
     assert torch.equal(out, o_dev)
+
+
+def test_host_pipeline_reuses_and_releases_its_streams():
+    """Calls on one stream reuse the cached copy streams and events; on a second stream they get
+    their own; after release_host_resources() a call creates them again.  Every result stays
+    bit-identical to the device call."""
+    m = kda()
+    w = synth.Workload("host_r", "prefill", 1, 320, 2, 128, 128, "bf16", 54, s0_std=0.2)
+    inp = synth.prefill_inputs(w)
+    h = pinned(inp)
+    o_dev, s_dev = device_call(inp)
+    side = torch.cuda.Stream()
+    for stream in (None, None, side, None):
+        out, sf = m.chunk_fwd_host(h["q"], h["k"], h["v"], h["log_alpha"], h["beta"], S0=h["S0"],
+                                   segment_tokens=64, stream=stream)
+        m.check()
+        assert torch.equal(out, o_dev) and torch.equal(sf, s_dev)
+    m.release_host_resources()
+    out, sf = m.chunk_fwd_host(h["q"], h["k"], h["v"], h["log_alpha"], h["beta"], S0=h["S0"], segment_tokens=128)
+    m.check()
+    assert torch.equal(out, o_dev) and torch.equal(sf, s_dev)
+    m.release_host_resources()

@@ -4,7 +4,7 @@ memory budget).  It runs on the library's built-in static scratch instead of a c
 
 This file is collected last on purpose (pytest orders files by name), so a run that stops at the
 first failure has already run every other test.  It must pass in a fresh process and after the
-other tests: the scratch lookup happens on the first call on the device.
+other tests: the scratch address is looked up on the device current at each call.
 """
 import ctypes
 
@@ -12,7 +12,7 @@ import pytest
 import torch
 
 from gated_delta_rule_83_b200 import synth
-from tests.kda_testutil import TOL, np64, out_err, state_err
+from tests.kda_testutil import TOL, np64, oracle_prefill, out_err, state_err
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -34,9 +34,13 @@ def _noalloc(lib, d, out, sf, cu=None):
                                      ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
 
 
-@pytest.mark.parametrize("dtype,dk,dv,T,lengths", [("bf16", 128, 128, 300, None), ("f32", 64, 64, 130, None),
-                                                   ("bf16", 128, 128, None, [1, 64, 65, 130])])
+CASES = [("bf16", 128, 128, 300, None), ("f32", 64, 64, 130, None), ("bf16", 128, 128, None, [1, 64, 65, 130])]
+
+
+@pytest.mark.parametrize("dtype,dk,dv,T,lengths", CASES)
 def test_noalloc_matches_workspace_entry_point(dtype, dk, dv, T, lengths):
+    """Same kernels on the same inputs: the C entry point's results equal the workspace entry
+    point's bit for bit, on two calls in a row (the second reuses the scratch the first left)."""
     import gated_delta_rule_83_b200 as kda
     lib = _lib()
     w = synth.Workload("noalloc", "prefill", 2, 0, 2, dk, dv, dtype, 99, s0_std=0.2)
@@ -45,14 +49,42 @@ def test_noalloc_matches_workspace_entry_point(dtype, dk, dv, T, lengths):
     ref_out, ref_S = kda.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], S0=inp["S0"],
                                    cu_seqlens=cu)
     kda.check()
-    tol_o, tol_s = TOL[dtype]
-    for call in range(2):  # two calls in a row share (and reuse) the built-in scratch
+    for call in range(2):
         out = torch.full_like(ref_out, float("nan"))
         sf = torch.full_like(ref_S, float("nan"))
         assert _noalloc(lib, inp, out, sf, cu) == 0
         kda.check()
-        assert out_err(np64(out), np64(ref_out)) <= tol_o, f"call {call}: output differs"
-        assert state_err(np64(sf), np64(ref_S)) <= tol_s, f"call {call}: final state differs"
+        assert torch.equal(out, ref_out), f"call {call}: output differs from kda_chunk_fwd"
+        assert torch.equal(sf, ref_S), f"call {call}: final state differs from kda_chunk_fwd"
+
+
+@pytest.mark.parametrize("dtype,dk,dv,T,lengths", CASES[::2])
+def test_noalloc_against_oracle(dtype, dk, dv, T, lengths):
+    """The binding (kda.chunk_fwd_noalloc) against the fp64 oracle at the operator's tolerances."""
+    import gated_delta_rule_83_b200 as kda
+    w = synth.Workload("noalloc", "prefill", 2, 0, 2, dk, dv, dtype, 98, s0_std=0.2)
+    inp = synth.prefill_inputs(w, T=T, lengths=lengths)
+    d = {k: (v.to(DEV) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    out = torch.empty(d["v"].shape, dtype=d["q"].dtype, device=DEV)
+    sf = torch.empty_like(d["S0"])
+    for _ in range(2):
+        kda.chunk_fwd_noalloc(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"], out, sf,
+                              cu_seqlens=d["cu_seqlens"])
+        kda.check()
+        o_ref, s_ref = oracle_prefill(inp)
+        tol_o, tol_s = TOL[dtype]
+        assert out_err(np64(out), o_ref) <= tol_o
+        assert state_err(np64(sf), s_ref) <= tol_s
+
+
+def test_noalloc_binding_rejects_bf16_gates_on_gpu():
+    import gated_delta_rule_83_b200 as kda
+    w = synth.Workload("noalloc", "prefill", 1, 128, 2, 128, 128, "bf16", 97, s0_std=0.2)
+    d = synth.prefill_inputs(w, device=DEV)
+    out = torch.empty(d["v"].shape, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(TypeError):
+        kda.chunk_fwd_noalloc(d["q"], d["k"], d["v"], d["log_alpha"].to(torch.bfloat16), d["beta"], d["S0"], out,
+                              None)
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():

@@ -150,16 +150,30 @@ kda_status kda_decode_step(const void* q, const void* k, const void* v, const fl
  *                                             bit-identical to the fp32 call on the same values; the
  *                                             largest input of the prefill is halved.  Any dt.
  *                 Other bits: KDA_ERR_INVALID_ARG.
+ *   schedule      How the tensor-core prefill (bf16 q/k/v, dk = dv = 128) is launched; every
+ *                 schedule computes the same chunk form, the results agree up to fp32 rounding:
+ *                   KDA_SCHEDULE_AUTO      (0) the library's choice (at present the two-pass one);
+ *                   KDA_SCHEDULE_TWO_PASS  (1) the intra-chunk kernel over all (chunk, head) units,
+ *                                              then the sequential kernel over the chains;
+ *                   KDA_SCHEDULE_FUSED     (2) one persistent launch: producer CTAs build the units
+ *                                              and publish a ready flag per unit, one chain CTA per
+ *                                              (sequence, head) consumes them from L2 as they
+ *                                              appear.  Taken for up to 64 chains, else two-pass.
+ *                 Ignored by the fp32 / d = 64 path and by decode.  Other values: KDA_ERR_INVALID_ARG.
  *   reserved      Must be zero (KDA_ERR_INVALID_ARG otherwise).
  */
 #define KDA_PROLOGUE_L2NORM_QK 1u
 #define KDA_PROLOGUE_GATE_LOGITS 2u
 #define KDA_PROLOGUE_BETA_LOGITS 4u
 #define KDA_PROLOGUE_GATE_BF16 8u
+#define KDA_SCHEDULE_AUTO 0
+#define KDA_SCHEDULE_TWO_PASS 1
+#define KDA_SCHEDULE_FUSED 2
 typedef struct {
     int num_qk_heads;
     unsigned prologue;
-    int reserved[6];
+    int schedule;
+    int reserved[5];
 } kda_options;
 
 /*

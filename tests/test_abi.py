@@ -22,6 +22,16 @@ def declared_functions():
     return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\**\s+\**(kda_\w+)\s*\(", src, flags=re.M)))
 
 
+def test_options_struct_matches_header():
+    """kda_options in the binding has the header's field order and size (8 ints)."""
+    from gated_delta_rule_83_b200.kda import KdaOptions
+    src = open(os.path.join(ROOT, "include", "kda.h")).read()
+    body = re.search(r"typedef struct \{(.*?)\} kda_options;", src, flags=re.S).group(1)
+    names = re.findall(r"(\w+)(?:\[\d+\])?;", body)
+    assert names == [f[0] for f in KdaOptions._fields_]
+    assert ctypes.sizeof(KdaOptions) == 32
+
+
 def test_header_declares_entry_points():
     names = declared_functions()
     for required in ("kda_chunk_fwd", "kda_decode_step", "kda_chunk_fwd_workspace_size", "kda_check",
@@ -110,6 +120,11 @@ def test_options_are_validated_before_launch(lib):
     assert lib.kda_chunk_fwd_ex(*args, ctypes.byref(res), fake, 1 << 30, None) == 1
     unknown = KdaOptions(prologue=16)               # not a KDA_PROLOGUE_* bit
     assert lib.kda_chunk_fwd_ex(*args, ctypes.byref(unknown), fake, 1 << 30, None) == 1
+    for bad_schedule in (-1, 3):                    # not a KDA_SCHEDULE_* value
+        sch = KdaOptions(schedule=bad_schedule)
+        assert lib.kda_chunk_fwd_ex(*args, ctypes.byref(sch), fake, 1 << 30, None) == 1
+    fused = KdaOptions(schedule=2)                  # valid: fails only on the missing workspace
+    assert lib.kda_chunk_fwd_ex(*args, ctypes.byref(fused), None, 1 << 30, None) == 5
     ok_group = KdaOptions(num_qk_heads=3, prologue=15)
     # a valid group with a missing workspace fails only on the workspace, like kda_chunk_fwd
     assert lib.kda_chunk_fwd_ex(*args, ctypes.byref(ok_group), None, 1 << 30, None) == 5

@@ -10,7 +10,7 @@ Public API (a thin binding of the C ABI in include/kda.h):
     check()                                               # raise on a device-side error
 """
 from .kda import (PROLOGUE_BETA_LOGITS, PROLOGUE_GATE_BF16, PROLOGUE_GATE_LOGITS, PROLOGUE_L2NORM_QK,  # noqa: F401
-                  SCHEDULE_AUTO, SCHEDULE_FUSED, SCHEDULE_TWO_PASS, KdaError,
+                  KdaError,
                   bwd_workspace_size, check, chunk_bwd, chunk_fwd, chunk_fwd_host, chunk_fwd_noalloc, decode_step, gated_rmsnorm,
                   load_library, profile_begin, profile_end, release_host_resources, release_workspaces, version,
                   workspace_size)

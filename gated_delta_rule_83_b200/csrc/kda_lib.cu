@@ -54,7 +54,7 @@ struct Plan {
     long long Ttot;   // total tokens
     int max_chunks;   // upper bound on the number of chunks
     bool tc;
-    size_t off_bytes, flag_bytes, slot_bytes, total_bytes;
+    size_t off_bytes, slot_bytes, total_bytes;
 };
 
 kda_status make_plan(int B, int T, int H, int dk, int dv, bool varlen, int num_seqs, kda_dtype dt, Plan& p)
@@ -81,9 +81,7 @@ kda_status make_plan(int B, int T, int H, int dk, int dv, bool varlen, int num_s
     p.tc = use_tc_path(dt, dk, dv);
     p.off_bytes = round_up(sizeof(int) * (2 * (size_t)p.N + 1), kAlign);  // off[N+1] + order[N]
     p.slot_bytes = p.tc ? tc_slot_bytes() : round_up(sizeof(float) * simt_slot_floats(dk, dv), kAlign);
-    // tensor-core path: one ready flag per (chunk, head) for the fused launch
-    p.flag_bytes = p.tc ? round_up(sizeof(uint32_t) * (size_t)p.max_chunks * (size_t)H, kAlign) : 0;
-    p.total_bytes = sizeof(WsHeader) + p.off_bytes + p.flag_bytes + (size_t)p.max_chunks * (size_t)H * p.slot_bytes;
+    p.total_bytes = sizeof(WsHeader) + p.off_bytes + (size_t)p.max_chunks * (size_t)H * p.slot_bytes;
     return KDA_OK;
 }
 
@@ -118,18 +116,15 @@ kda_status make_bwd_plan(int B, int T, int H, int Hk, unsigned pro, int dk, int 
     return KDA_OK;
 }
 
-// Options of the extended entry points: Hk = q/k heads (0 -> H), prologue bits, prefill schedule;
-// reserved fields must be zero.
-kda_status parse_options(const kda_options* opt, int H, int& Hk, unsigned& pro, int* schedule = nullptr)
+// Options of the extended entry points: Hk = q/k heads (0 -> H), prologue bits; reserved fields
+// must be zero.
+kda_status parse_options(const kda_options* opt, int H, int& Hk, unsigned& pro)
 {
     Hk = H;
     pro = 0;
-    if (schedule) *schedule = KDA_SCHEDULE_AUTO;
     if (!opt) return KDA_OK;
     for (int r : opt->reserved)
         if (r != 0) return KDA_ERR_INVALID_ARG;
-    if (opt->schedule < KDA_SCHEDULE_AUTO || opt->schedule > KDA_SCHEDULE_FUSED) return KDA_ERR_INVALID_ARG;
-    if (schedule) *schedule = opt->schedule;
     if (opt->num_qk_heads != 0) {
         if (opt->num_qk_heads < 0 || H % opt->num_qk_heads != 0) return KDA_ERR_INVALID_ARG;
         Hk = opt->num_qk_heads;
@@ -178,9 +173,9 @@ kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v, const v
                             void* workspace, size_t workspace_bytes, kda_stream_t stream_)
 {
     cudaStream_t stream = (cudaStream_t)stream_;
-    int Hk = H, schedule = KDA_SCHEDULE_AUTO;
+    int Hk = H;
     unsigned pro = 0;
-    const kda_status so = parse_options(opt, H, Hk, pro, &schedule);
+    const kda_status so = parse_options(opt, H, Hk, pro);
     if (so != KDA_OK) return so;
     Plan p;
     const kda_status st = make_plan(B, T, H, dk, dv, cu_seqlens != nullptr, num_seqs, dt, p);
@@ -195,8 +190,7 @@ kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v, const v
     char* ws = (char*)workspace;
     WsHeader* hdr = (WsHeader*)ws;
     int* off = (int*)(ws + sizeof(WsHeader));
-    uint32_t* flags = p.flag_bytes ? (uint32_t*)(ws + sizeof(WsHeader) + p.off_bytes) : nullptr;
-    char* slots = ws + sizeof(WsHeader) + p.off_bytes + p.flag_bytes;
+    char* slots = ws + sizeof(WsHeader) + p.off_bytes;
 
     {
         LaunchScope ls("chunk_table", stream);
@@ -207,9 +201,8 @@ kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v, const v
 
     cudaError_t e;
     if (p.tc) {
-        // the automatic choice is the two-pass schedule: the fused one does not yet beat it
         e = launch_tc_prefill(q, k, v, log_alpha, beta, S0, S_final, out, hdr, off, cu_seqlens, p.Tseq, p.N, H, Hk, pro,
-                              p.max_chunks, p.Ttot, slots, schedule == KDA_SCHEDULE_FUSED ? flags : nullptr, stream);
+                              p.max_chunks, p.Ttot, slots, stream);
     } else if (dt == KDA_BF16) {
         e = launch_simt_prefill<__nv_bfloat16>(q, k, v, log_alpha, beta, S0, S_final, out, hdr, off, cu_seqlens,
                                                p.Tseq, p.N, H, Hk, pro, dk, dv, p.max_chunks, (float*)slots, stream);

@@ -42,9 +42,8 @@ constexpr bool kTcPathReady = true;
 
 // ---- workspace slot of one (chunk, head), bytes ------------------------------------------------
 // Every image is a 64-row SW128 tile, bf16 [64 x 128] (two 8 KB atom columns), exactly as phase A
-// holds it in shared memory, so phase A writes each with bulk copies.  Slots are head-major: the slot
-// of (global chunk j, head h) is h * J + j (J = the workspace's chunk capacity), so that each chain
-// reads one contiguous run of slots.
+// holds it in shared memory, so phase A writes each with bulk copies.  The slot of unit u = chunk * H
+// + head is slot u: the slots of one chunk row (all heads) are adjacent.
 constexpr uint32_t kSlotW = 0;          // W
 constexpr uint32_t kSlotQ = 16384;      // Q'
 constexpr uint32_t kSlotKd = 32768;     // Kd  (MN-major A operand of Kd^T U)
@@ -226,6 +225,7 @@ constexpr uint32_t kA_P = kA_G + 22528;     // P bf16 [64][64] tile (1024-aligne
 constexpr uint32_t kA_Misc = kA_G + 32768;  // small arrays, TMEM address, flags, mbarriers (4 KB)
 constexpr uint32_t kA_Smem = kA_Misc + 4096 + 1024;  // + 1024 for aligning the dynamic base
 constexpr int kGS = 128;             // row stride of the g tile (floats)
+constexpr int kACopyThread = 160;    // warp 5, lane 0: issues the next log_alpha load
 constexpr uint32_t kKQ_LBO = 16384;  // distance between the atom columns of the stacked [k; q] tile
 
 __device__ __forceinline__ void bulk_s2g(void* dst, uint32_t src_smem, uint32_t bytes)
@@ -254,64 +254,19 @@ __device__ __forceinline__ void tc_unit(long long u, int H, const int* __restric
     }
 }
 
-// Production order of the units.  The two-kernel path takes units in slot order (u = chunk * H + head).
-// The fused kernel takes regular batches chunk-major across sequences, i = (c * N + n) * H + head, so
-// that every sequence's chain is fed from the start; packed (varlen) input keeps the slot order.
-template <bool FUSED>
-__device__ __forceinline__ void tc_prod_unit(long long i, int H, const int* __restrict__ off,
-                                             const int32_t* __restrict__ cu, int Tseq, int N, long long& u, int& h,
-                                             int& n, long long& t0, int& L)
-{
-    if (FUSED && cu == nullptr) {
-        const long long NH = (long long)N * H;
-        const long long c = i / NH;
-        const long long r = i - c * NH;
-        n = (int)(r / H);
-        h = (int)(r - (long long)n * H);
-        const long long cpb = (Tseq + kChunk - 1) / kChunk;
-        u = ((long long)n * cpb + c) * H + h;
-        t0 = (long long)n * Tseq + c * kChunk;
-        L = (int)min((long long)kChunk, (long long)Tseq - c * kChunk);
-    } else {
-        u = i;
-        tc_unit(i, H, off, cu, Tseq, N, h, n, t0, L);
-    }
-}
-
-// Ready flags of the fused kernel: a producer publishes unit u once its images are complete in
-// global memory; the chain that consumes it acquires the flag before its bulk copies.
-__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v)
-{
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p)
-{
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-// orders this thread's generic-proxy global accesses with its async-proxy (bulk copy) ones
-__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
-
 // PRO: some q/k or beta/gate-activation prologue bit is set (the plain instance carries none of that code)
 // LA16: log_alpha arrives as bf16 (16 KB per unit, landed in the upper half of the gate region and
 // widened to the fp32 g tile by the gate scan)
-// FUSED: the producer role of the fused kernel (production order of tc_prod_unit<true>; every unit,
-// the first included, is claimed from the work counter, so a unit is only ever held by a running CTA;
-// each unit's ready flag is published once its images are complete)
-// first / stride (two-kernel path): this CTA's first production index and the number of CTAs
-template <bool PRO, bool LA16, bool FUSED>
-__device__ __forceinline__ void
-tc_intra_body(uint8_t* sm, long long first, long long stride, const CUtensorMap* tm_q_, const CUtensorMap* tm_k_,
-              const CUtensorMap* tm_v_, const CUtensorMap* tm_la_, const float* __restrict__ beta,
-              WsHeader* __restrict__ hdr, const int* __restrict__ off, const int32_t* __restrict__ cu, int Tseq,
-              int N, int H, int G, unsigned pro, int J, uint8_t* __restrict__ slots, uint32_t* __restrict__ flags)
+template <bool PRO, bool LA16>
+__global__ void __launch_bounds__(kAThreads, 2)
+tc_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_la,
+                const float* __restrict__ beta, WsHeader* __restrict__ hdr, const int* __restrict__ off,
+                const int32_t* __restrict__ cu, int Tseq, int N, int H, int G, unsigned pro,
+                uint8_t* __restrict__ slots)
 {
     using namespace tc;
-    const CUtensorMap& tm_q = *tm_q_;
-    const CUtensorMap& tm_k = *tm_k_;
-    const CUtensorMap& tm_v = *tm_v_;
-    const CUtensorMap& tm_la = *tm_la_;
+    extern __shared__ uint8_t smem_raw[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     long long nunits;
     if (cu == nullptr) {
@@ -320,14 +275,9 @@ tc_intra_body(uint8_t* sm, long long first, long long stride, const CUtensorMap*
         if (hdr->bad) return;
         nunits = (long long)hdr->total_chunks * H;
     }
-    if (FUSED) {  // the first unit, claimed like every later one
-        if (tid == 0) *reinterpret_cast<volatile long long*>(sm + kA_Misc + 3376) = atomicAdd(&hdr->next_unit, 1);
-        __syncthreads();
-        first = *reinterpret_cast<volatile long long*>(sm + kA_Misc + 3376);
-        __syncthreads();
-    }
-    if (first >= nunits) return;
+    if ((long long)blockIdx.x >= nunits) return;
 
+    uint8_t* sm = align1024(smem_raw);
     const uint32_t sb = smem_u32(sm);
     float* s_beta = reinterpret_cast<float*>(sm + kA_Misc);          // [64]
     float* s_ref = reinterpret_cast<float*>(sm + kA_Misc + 256);     // [128] (log2 units)
@@ -342,11 +292,9 @@ tc_intra_body(uint8_t* sm, long long first, long long stride, const CUtensorMap*
     const uint32_t mbar = smem_u32(sm + kA_Misc + 3344);     // MMA completions
     const uint32_t mbar_la = smem_u32(sm + kA_Misc + 3352);  // log_alpha landed
     const uint32_t mbar_kq = mbar_la + 8, mbar_v = mbar_la + 16;
-    // the unit after this one, claimed and decoded by thread 0: {production index, t0}, {head,
-    // length} and its slot index
+    // the unit after this one, claimed and decoded by thread 0: {u, t0} and {head, length}
     long long* s_next = reinterpret_cast<long long*>(sm + kA_Misc + 3376);
     int* s_next_hl = reinterpret_cast<int*>(sm + kA_Misc + 3392);
-    long long* s_next_u = reinterpret_cast<long long*>(sm + kA_Misc + 3400);
     float* sG = reinterpret_cast<float*>(sm + kA_G);
     float* sA = reinterpret_cast<float*>(sm + kA_G);                 // after the gating pass
     float* sY = reinterpret_cast<float*>(sm + kA_Ysc);
@@ -374,9 +322,13 @@ tc_intra_body(uint8_t* sm, long long first, long long stride, const CUtensorMap*
     };
 
     int h, n, L;
-    long long t0, u;
-    tc_prod_unit<FUSED>(first, H, off, cu, Tseq, N, u, h, n, t0, L);
+    long long t0;
+    tc_unit(blockIdx.x, H, off, cu, Tseq, N, h, n, t0, L);
     if (tid == 0) {
+        prefetch_tensormap(&tm_q);
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+        prefetch_tensormap(&tm_la);
         *s_abort = 0;
         mbar_init(mbar, 1);
         mbar_init(mbar_la, 1);
@@ -406,13 +358,11 @@ tc_intra_body(uint8_t* sm, long long first, long long stride, const CUtensorMap*
     bool ok = true, has_next = false;
     int it = 0;
 
-    long long u_prev = -1;  // FUSED: the unit whose ready flag is still to be published
-    for (long long i = first; i < nunits; ++it) {
-        int claim = 0;  // thread 0: the next unit (stride + claim), from the work counter
+    for (long long u = blockIdx.x; u < nunits; ++it) {
+        int claim = 0;  // thread 0: the next unit (gridDim.x + claim), from the work counter
         if (tid == 0) claim = atomicAdd(&hdr->next_unit, 1);
         const uint32_t par = (uint32_t)it & 1u;
-        const long long su = (long long)h * J + (u - h) / H;  // slot of unit u = chunk * H + head
-        uint8_t* slot = slots + (size_t)su * kSlotBytes;
+        uint8_t* slot = slots + (size_t)u * kSlotBytes;
 
         if (tid == 0) *s_wide = 0;
         ok = mbar_wait_ab(mbar_la, par, s_abort) && ok;
@@ -447,18 +397,7 @@ tc_intra_body(uint8_t* sm, long long first, long long stride, const CUtensorMap*
             }
         }
         if (hf == 0) s_carry[c] = gl[31];
-        if (FUSED && u_prev >= 0) {
-            // the previous unit's image stores (bulk groups of lane 0 of each warp, issued before this
-            // unit started any) and its Kd / e^{g_last} stores complete before its flag is published
-            if (lane == 0) bulk_wait_all();
-            fence_proxy_async_global();
-            __threadfence();
-        }
         __syncthreads();
-        if (FUSED && u_prev >= 0) {
-            if (tid == 0) st_release_gpu(flags + u_prev, 1u);
-            u_prev = -1;
-        }
         float lo, hi;
         if (hf == 1) {
             const float cr = s_carry[c];
@@ -498,14 +437,12 @@ tc_intra_body(uint8_t* sm, long long first, long long stride, const CUtensorMap*
         if (tid == 0) {  // decode the claimed next unit for the prefetches below
             int hh = 0, nn = 0, LL = 0;
             long long tt = 0;
-            long long uu = 0;
-            const long long un = FUSED ? (long long)claim : stride + claim;
-            if (un < nunits) tc_prod_unit<FUSED>(un, H, off, cu, Tseq, N, uu, hh, nn, tt, LL);
+            const long long un = (long long)gridDim.x + claim;
+            if (un < nunits) tc_unit(un, H, off, cu, Tseq, N, hh, nn, tt, LL);
             s_next[0] = un;
             s_next[1] = tt;
             s_next_hl[0] = hh;
             s_next_hl[1] = LL;
-            *s_next_u = uu;
         }
         ok = mbar_wait_ab(mbar_kq, par, s_abort) && ok;  // k and q in place
         cp_async_wait_all();                             // beta in place
@@ -747,7 +684,10 @@ tc_intra_body(uint8_t* sm, long long first, long long stride, const CUtensorMap*
                     tmem_ld16_pair<64>(trow + b2 + 16, a2 + 16);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int m = 0; m < 32; ++m) a2[m] *= s_E[hc + b2 + m];
+                    for (int m = 0; m < 32; m += 4) {
+                        const float4 e4 = *reinterpret_cast<const float4*>(s_E + hc + b2 + m);
+                        a2[m] *= e4.x; a2[m + 1] *= e4.y; a2[m + 2] *= e4.z; a2[m + 3] *= e4.w;
+                    }
 #pragma unroll
                     for (int m = 0; m < 4; ++m)
                         *reinterpret_cast<uint4*>(sm + kA_KQ + sw128_chunk_off(rowq, (hc + b2) / 8 + m, 128)) = pack8(a2 + 8 * m);
@@ -789,8 +729,10 @@ tc_intra_body(uint8_t* sm, long long first, long long stride, const CUtensorMap*
         mphase ^= 1;
         fence_after_sync();
         ok = __syncthreads_and(ok);
-        if (has_next) {  // the log_alpha region is free (P consumed) and beta has been read
-            if (tid == 0) issue_la(s_next_hl[0], s_next[1]);
+        if (has_next) {  // the log_alpha region is free (P consumed) and beta has been read.  Copies are
+                         // issued by lanes of different warps, so that no single thread on the
+                         // critical path waits for all of them.
+            if (tid == kACopyThread) issue_la(s_next_hl[0], s_next[1]);
             if (tid < 64) issue_beta(s_next_hl[0], s_next[1], s_next_hl[1]);
         }
         if (ok) {
@@ -806,8 +748,11 @@ tc_intra_body(uint8_t* sm, long long first, long long stride, const CUtensorMap*
                         uint4* p = reinterpret_cast<uint4*>(sm + kA_KQ + sw128_chunk_off(64 + rowq, (hc + b2) / 8 + m, 128));
                         float qf[8];
                         unpack8(*p, qf);
+                        const float4 e0 = *reinterpret_cast<const float4*>(s_E + hc + b2 + 8 * m);
+                        const float4 e1 = *reinterpret_cast<const float4*>(s_E + hc + b2 + 8 * m + 4);
+                        const float ev[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) qf[e] = qf[e] * s_E[hc + b2 + 8 * m + e] - a2[8 * m + e];
+                        for (int e = 0; e < 8; ++e) qf[e] = qf[e] * ev[e] - a2[8 * m + e];
                         *p = pack8(qf);
                     }
                 }
@@ -840,51 +785,27 @@ tc_intra_body(uint8_t* sm, long long first, long long stride, const CUtensorMap*
         if (lane == 0) bulk_wait_read();  // every image of this unit has been read out of shared memory
         fence_before_sync();
         ok = __syncthreads_and(ok);  // the next chunk's tiles (k, q, v; Kb over the Uv image) may land from here on
-        if (tid == 0 && has_next) {
-            issue_kq(s_next_hl[0], s_next[1]);
-            issue_v(s_next_hl[0], s_next[1]);
+        if (has_next) {
+            if (tid == 0) issue_kq(s_next_hl[0], s_next[1]);
+            if (tid == 32) issue_v(s_next_hl[0], s_next[1]);
         }
         if (!ok) break;
-        if (FUSED) u_prev = su;
-        i = s_next[0];
-        u = *s_next_u;
+        u = s_next[0];
         t0 = s_next[1];
         h = s_next_hl[0];
         L = s_next_hl[1];
     }
-    if (FUSED && u_prev >= 0) {  // the last unit of this CTA
-        if (lane == 0) bulk_wait_all();
-        fence_proxy_async_global();
-        __threadfence();
-        __syncthreads();
-        if (tid == 0) st_release_gpu(flags + u_prev, 1u);
-    }
-    if (tid == 0) {
-        if (!ok && has_next) {  // loads for the next chunk may still be landing: bounded waits
-            const uint32_t pn = ((uint32_t)it + 1u) & 1u;
-            (void)mbar_wait(mbar_la, pn);
-            (void)mbar_wait(mbar_kq, pn);
-            (void)mbar_wait(mbar_v, pn);
-        }
+    if (tid == 0 && !ok && has_next) {  // loads for the next chunk may still be landing: bounded waits
+        const uint32_t pn = ((uint32_t)it + 1u) & 1u;
+        (void)mbar_wait(mbar_la, pn);
+        (void)mbar_wait(mbar_kq, pn);
+        (void)mbar_wait(mbar_v, pn);
     }
     if (lane == 0) bulk_wait_all();  // every lane that issued image stores
     cp_async_wait_all();
     fence_before_sync();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, 256);
-}
-
-template <bool PRO, bool LA16>
-__global__ void __launch_bounds__(kAThreads, 2)
-tc_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_la,
-                const float* __restrict__ beta, WsHeader* __restrict__ hdr, const int* __restrict__ off,
-                const int32_t* __restrict__ cu, int Tseq, int N, int H, int G, unsigned pro, int J,
-                uint8_t* __restrict__ slots)
-{
-    extern __shared__ uint8_t smem_raw[];
-    tc_intra_body<PRO, LA16, false>(align1024(smem_raw), blockIdx.x, gridDim.x, &tm_q, &tm_k, &tm_v, &tm_la, beta,
-                                    hdr, off, cu, Tseq, N, H, G, pro, J, slots, nullptr);
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -934,7 +855,7 @@ constexpr int kBPrefetch = 4;  // L2 prefetch distance beyond the shared-memory 
 
 __global__ void __launch_bounds__(kBThreads, 1)
 tc_inter_kernel(const float* S0, float* S_final, __nv_bfloat16* __restrict__ out, const WsHeader* __restrict__ hdr,
-                const int* __restrict__ off, const int32_t* __restrict__ cu, int Tseq, int N, int H, int J,
+                const int* __restrict__ off, const int32_t* __restrict__ cu, int Tseq, int N, int H,
                 const uint8_t* __restrict__ slots)
 {
     using namespace tc;
@@ -956,6 +877,7 @@ tc_inter_kernel(const float* S0, float* S_final, __nv_bfloat16* __restrict__ out
     volatile int* s_abort = reinterpret_cast<volatile int*>(sm + kB_Misc + 132);
 
     const int jb = off[n], je = off[n + 1], nch = je - jb;
+    const uint8_t* hslots = slots + (size_t)h * kSlotBytes;  // this head's slots, H slots apart
     long long s0, s1;
     seq_bounds(n, cu, Tseq, s0, s1);
 
@@ -992,9 +914,9 @@ tc_inter_kernel(const float* S0, float* S_final, __nv_bfloat16* __restrict__ out
     __syncthreads();  // barriers initialised, TMEM address visible, S tile written
     if (warp == 5 && lane == 0) {
         for (int s = 0; s < kBStages && s < nch; ++s)
-            tc_issue_stage(sb + s * kStageBytes, bar_full + 8 * s, slots + ((size_t)h * J + jb + s) * kSlotBytes, vt);
+            tc_issue_stage(sb + s * kStageBytes, bar_full + 8 * s, hslots + (size_t)(jb + s) * H * kSlotBytes, vt);
         for (int s = kBStages; s < kBStages + kBPrefetch && s < nch; ++s)
-            tc_prefetch_stage(slots + ((size_t)h * J + jb + s) * kSlotBytes, vt);
+            tc_prefetch_stage(hslots + (size_t)(jb + s) * H * kSlotBytes, vt);
     }
     const uint32_t tmem = *s_tmem;
     const uint32_t tw = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
@@ -1049,9 +971,9 @@ tc_inter_kernel(const float* S0, float* S_final, __nv_bfloat16* __restrict__ out
             if (refill && lane == 0) {  // stage s fully consumed (128 compute-thread arrivals) -> refill
                 ok = ok && mbar_wait_ab(bar_empty + 8 * s, (uint32_t)(it / kBStages) & 1u, s_abort);
                 if (ok) {
-                    tc_issue_stage(st, bar_full + 8 * s, slots + ((size_t)h * J + jb + it + kBStages) * kSlotBytes, vt);
+                    tc_issue_stage(st, bar_full + 8 * s, hslots + (size_t)(jb + it + kBStages) * H * kSlotBytes, vt);
                     if (it + kBStages + kBPrefetch < nch)
-                        tc_prefetch_stage(slots + ((size_t)h * J + jb + it + kBStages + kBPrefetch) * kSlotBytes, vt);
+                        tc_prefetch_stage(hslots + (size_t)(jb + it + kBStages + kBPrefetch) * H * kSlotBytes, vt);
                 }
             }
         } else {
@@ -1126,399 +1048,6 @@ tc_inter_kernel(const float* S0, float* S_final, __nv_bfloat16* __restrict__ out
     if (warp == 0) tmem_dealloc(tmem, 64);
 }
 
-// ------------------------------------------------------------------------------------------------
-// Fused prefill: the intra-chunk units and the sequential chains in one persistent launch.  CTAs
-// [0, C) each run the whole chain of one (sequence, head) over all 128 state columns; the other CTAs
-// run tc_intra_body<FUSED> and publish a ready flag per unit.  Per chunk a chain runs
-//     [X; O'] = [W; Q'] S_c                 tcgen05 M=128 N=128 K=128   (S_c: bf16 copy of the state)
-//     U = Uv - X (bf16 tile);  out = O' + O0
-//     S_{c+1} = Diag(e^{g_last}) S_c + Kd^T U   tcgen05 M=128 N=128 K=64, accumulated onto the fp32
-//                                               state in TMEM, which holds Diag(e^{g_last}) S_c by then
-// Roles inside a chain CTA (8 warps; warp w owns TMEM lanes 32 (w % 4).. and state columns 64 (w / 4)..):
-//   thread 0      issues both MMAs and the bulk copies of the next chunks' [W; Q'] halves and Kd tiles;
-//   warps 0,1,4,5 write U (token rows 0-63): MMA2 waits for these four warps only;
-//   warps 2,3,6,7 write the outputs (token rows 64-127 of [X; O']);
-//   thread 192    polls the producers' ready flags a few chunks ahead, once per chunk while MMA1 runs,
-//                 and publishes the progress in shared memory, from where the other threads take it;
-//   all threads   the state epilogue; the Uv / O0 rows and e^{g_last} of the next chunk are loaded a
-//                 chunk ahead.
-// Producers never wait on chains and claim every unit from a work counter, so a chain only ever waits
-// on a unit that a running producer holds.  Every wait is bounded and raises KDA_ERR_TIMEOUT when it
-// gives up.
-// ------------------------------------------------------------------------------------------------
-constexpr uint32_t kC_S = 0;          // S tile: bf16 [128 rows][128] SW128 (MN-major B), 32 KB; the U tile
-                                      //   (bf16 [64][128], 16 KB) overlays its first half between MMA1 and MMA2
-constexpr uint32_t kC_WQ = 32768;     // ring of 3 blocks of 16 KB: one atom column (64 of the 128 K) of the
-                                      //   stacked [W; Q'] A operand each; chunk c uses blocks 2c, 2c+1 (mod 3)
-constexpr uint32_t kC_Kd = 81920;     // 2 Kd tiles (MN-major A), 16 KB each; chunk c uses tile c & 1
-constexpr uint32_t kC_Misc = 114688;  // mbarriers, TMEM address, abort flag, published progress
-constexpr uint32_t kC_Smem = 114816;  // the dynamic shared memory base is 1024-aligned (checked)
-constexpr uint32_t kF_Smem = kC_Smem > kA_Smem ? kC_Smem : kA_Smem;
-constexpr int kFusedMaxChains = 64;   // more (sequence, head) chains than this: the two-kernel path
-constexpr int kChainLookahead = 4;    // chunks beyond the next one whose flags are polled ahead
-constexpr int kChainPoller = 192;     // warp 6, lane 0: an output warp, idle while MMA1 runs
-constexpr long long kFlagWaitCycles = 4000000000LL;  // ~2 s: far beyond any legitimate wait on a producer
-
-__device__ __forceinline__ uint32_t ld_relaxed_gpu(const uint32_t* p)
-{
-    uint32_t v;
-    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
-__device__ __forceinline__ void st_release_cta(uint32_t saddr, int v)
-{
-    asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(saddr), "r"(v) : "memory");
-}
-__device__ __forceinline__ int ld_acquire_cta(uint32_t saddr)
-{
-    int v;
-    asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(saddr) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ void tc_chain_body(uint8_t* sm, int ci, const float* S0, float* S_final,
-                                              __nv_bfloat16* __restrict__ out, const WsHeader* __restrict__ hdr,
-                                              const int* __restrict__ off, const int32_t* __restrict__ cu, int Tseq,
-                                              int N, int H, int J, const uint8_t* __restrict__ slots,
-                                              const uint32_t* __restrict__ flags)
-{
-    using namespace tc;
-    if (hdr->bad) return;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int q4 = warp & 3, hcol = warp >> 2;   // TMEM lane quarter, 64-column half of the state
-    const int row = 32 * q4 + lane;              // state row (key channel); token row of [X; O'] for q4 < 2 / >= 2
-    const int r64 = row & 63;
-    const int rank = ci / H, h = ci - rank * H;  // longest sequences first
-    const int n = off[N + 1 + rank];
-    const int jb = off[n], nch = off[n + 1] - jb;
-    long long s0, s1;
-    seq_bounds(n, cu, Tseq, s0, s1);
-    const uint32_t sb = smem_u32(sm);
-    const uint32_t full_wq = smem_u32(sm + kC_Misc);  // 3 barriers: a [W; Q'] block landed
-    const uint32_t full_kd = full_wq + 24;            // 2 barriers: a Kd tile landed
-    const uint32_t bar_half = full_wq + 40;           // MMA1 has read its first block
-    const uint32_t bar_d1 = full_wq + 48;             // [X; O'] ready (MMA1 complete)
-    const uint32_t bar_y = full_wq + 56;              // MMA2 complete
-    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + kC_Misc + 64);
-    volatile int* s_abort = reinterpret_cast<volatile int*>(sm + kC_Misc + 68);
-    const uint32_t s_pf = smem_u32(sm + kC_Misc + 72);  // chunks 0 .. *s_pf are published (acquired by the poller)
-
-    auto slot_of = [&](int c) { return slots + ((size_t)h * J + jb + c) * kSlotBytes; };
-    auto flag_of = [&](int c) { return flags + (size_t)h * J + jb + c; };
-    bool ok = true;
-
-    // ---- poller (thread kChainPoller) ----
-    int pf_local = -1;
-    auto poll_nb = [&](int limit) {  // acquire the published chunks among pf_local + 1 .. limit, no waiting:
-        limit = min(limit, nch - 1);  // four relaxed flag loads in flight, one acquire fence for those set
-        if (pf_local >= limit) return;
-        uint32_t v[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) v[k] = pf_local + 1 + k <= limit ? ld_relaxed_gpu(flag_of(pf_local + 1 + k)) : 0u;
-        int got = 0;
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-            if (got == k && v[k]) got = k + 1;
-        if (got) {
-            fence_acq_rel_gpu();
-            pf_local += got;
-            st_release_cta(s_pf, pf_local);
-        }
-    };
-    // every thread: chunk c must be published.  The poller waits on the producer's flag (bounded);
-    // the others wait for the poller.
-    auto need = [&](int c) {
-        if (!ok) return;
-        const long long start = clock64();
-        if (tid == kChainPoller) {
-            while (pf_local < c) {
-                poll_nb(c);
-                if (pf_local >= c) break;
-                if (*s_abort || clock64() - start > kFlagWaitCycles) {
-                    if (!*s_abort) set_error(KDA_ERR_TIMEOUT);
-                    *s_abort = 1;
-                    ok = false;
-                    return;
-                }
-                __nanosleep(32);
-            }
-        } else {
-            while (ld_acquire_cta(s_pf) < c) {
-                if (*s_abort || clock64() - start > kFlagWaitCycles) {
-                    *s_abort = 1;
-                    ok = false;
-                    return;
-                }
-            }
-        }
-    };
-
-    // ---- thread 0's copy bookkeeping ----
-    // pf_seen: progress covered by thread 0's last proxy fence; wq_m: next [W; Q'] half (m = 2 c + j) to
-    // copy; kd_n: next Kd tile; *_done: chunks whose MMA barrier thread 0 has seen complete; n_*: barrier
-    // phases started (for the waits of a failing CTA)
-    int pf_seen = -1, wq_m = 0, kd_n = 0, half_done = 0, d1_done = 0, y_done = 0;
-    int n_wq[3] = {0, 0, 0}, n_kd[2] = {0, 0}, n_half = 0, n_d1 = 0, n_y = 0;
-    auto pump = [&]() {  // copy every [W; Q'] half and Kd tile whose chunk is published and whose buffer is free
-        const int pf = ld_acquire_cta(s_pf);
-        if (pf > pf_seen) {  // the acquire (by the poller) precedes the async-proxy reads of the copies
-            fence_proxy_async_global();
-            pf_seen = pf;
-        }
-        while (wq_m < 2 * nch && (wq_m >> 1) <= pf_seen) {
-            const int m = wq_m;
-            if (m >= 3) {  // the block's previous user, half m - 3, must have been read by its MMA1
-                const int cc = (m - 3) >> 1;
-                if (((m - 3) & 1) ? cc >= d1_done : cc >= half_done) break;
-            }
-            const int b = m % 3, j = m & 1;
-            const uint8_t* slot = slot_of(m >> 1);
-            const uint32_t dst = sb + kC_WQ + (uint32_t)b * 16384u, bar = full_wq + 8u * (uint32_t)b;
-            mbar_arrive_expect_tx(bar, 16384);
-            bulk_g2s(dst, slot + kSlotW + j * 8192, 8192, bar);         // W rows of this atom column
-            bulk_g2s(dst + 8192, slot + kSlotQ + j * 8192, 8192, bar);  // Q' rows
-            ++n_wq[b];
-            ++wq_m;
-        }
-        while (kd_n < nch && kd_n <= pf_seen && kd_n - 2 < y_done) {  // tile kd_n & 1: read by MMA2 of kd_n - 2
-            const uint32_t bar = full_kd + 8u * (uint32_t)(kd_n & 1);
-            mbar_arrive_expect_tx(bar, 16384);
-            bulk_g2s(sb + kC_Kd + (uint32_t)(kd_n & 1) * 16384u, slot_of(kd_n) + kSlotKd, 16384, bar);
-            ++n_kd[kd_n & 1];
-            ++kd_n;
-        }
-    };
-
-    if (tid == 0) {
-        for (int b = 0; b < 3; ++b) mbar_init(full_wq + 8 * b, 1);
-        for (int b = 0; b < 2; ++b) mbar_init(full_kd + 8 * b, 1);
-        mbar_init(bar_half, 1);
-        mbar_init(bar_d1, 1);
-        mbar_init(bar_y, 1);
-        mbar_fence_init();
-        *s_abort = 0;
-        st_release_cta(s_pf, -1);
-    }
-    if (warp == 0) {
-        tmem_alloc(smem_u32(s_tmem), 256);
-        tmem_relinquish();
-    }
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
-    const uint32_t tmem = *s_tmem;
-    const uint32_t tl = tmem + ((uint32_t)(32 * q4) << 16);  // this warp's lane quarter
-    const int c0 = 64 * hcol;                                 // this thread's 64 state / output columns
-    const size_t srow = (((size_t)n * H + h) * 128 + row) * 128 + c0;
-
-    // the next chunk's Uv (token rows 0-63) or O0 (64-127) row and e^{g_last}, a chunk ahead
-    uint4 raw[8];
-    float gam = 1.f;
-    auto load_rows = [&](int c) {
-        const uint8_t* slot = slot_of(c);
-        gam = __ldcg(reinterpret_cast<const float*>(slot + kSlotGam) + row);
-#pragma unroll
-        for (int m = 0; m < 8; ++m)
-            raw[m] = __ldcg(reinterpret_cast<const uint4*>(slot + (q4 < 2 ? kSlotUv : kSlotO0) +
-                                                          sw128_chunk_off(r64, 8 * hcol + m, 64)));
-    };
-    if (nch > 0) {
-        need(0);
-        if (tid == kChainPoller) poll_nb(kChainLookahead);
-        __syncthreads();
-        if (ok) load_rows(0);
-    }
-    // S0 -> its bf16 copy in the S tile, and Diag(e^{g_last}) S0 in TMEM columns [0, 128)
-    {
-        float sn[64];
-#pragma unroll
-        for (int m = 0; m < 64; m += 4) {
-            const float4 x = S0 ? *reinterpret_cast<const float4*>(S0 + srow + m) : make_float4(0.f, 0.f, 0.f, 0.f);
-            sn[m] = x.x; sn[m + 1] = x.y; sn[m + 2] = x.z; sn[m + 3] = x.w;
-        }
-#pragma unroll
-        for (int m = 0; m < 8; ++m)
-            *reinterpret_cast<uint4*>(sm + kC_S + sw128_chunk_off(row, 8 * hcol + m, 128)) = pack8(sn + 8 * m);
-        if (nch == 0) {
-            if (S_final) {
-#pragma unroll
-                for (int m = 0; m < 64; m += 4)
-                    *reinterpret_cast<float4*>(S_final + srow + m) = make_float4(sn[m], sn[m + 1], sn[m + 2], sn[m + 3]);
-            }
-        } else {
-#pragma unroll
-            for (int m = 0; m < 64; ++m) sn[m] *= gam;
-#pragma unroll
-            for (int m = 0; m < 64; m += 16) tmem_st16(tl + c0 + m, sn + m);
-        }
-    }
-    tmem_wait_st();
-    if (tid == 0 && nch > 0 && ok) pump();
-    fence_proxy_async();
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
-
-    const uint32_t id1 = idesc_bf16(128, 128, false, true);  // [W; Q'] S   (S MN-major)
-    const uint32_t id2 = idesc_bf16(128, 128, true, true);   // Kd^T U      (Kd, U MN-major)
-    const uint64_t dS = desc_sw128(sb + kC_S, 128 * 128, 1024u), dU = desc_sw128(sb + kC_S, 64 * 128, 1024u);
-    for (int c = 0; c < nch; ++c) {
-        const uint32_t par = (uint32_t)c & 1u;
-        const int mA = 2 * c, mB = 2 * c + 1;  // the chunk's two [W; Q'] halves
-        const long long t0 = s0 + (long long)c * 64;
-        const int L = (s1 - t0) < 64 ? (int)(s1 - t0) : 64;
-        const bool more = c + 1 < nch;
-        if (tid == 0) {
-            if (ok) pump();
-            ok = ok && mbar_wait_ab(full_wq + 8u * (mA % 3), (uint32_t)(mA / 3) & 1u, s_abort);
-            ok = ok && mbar_wait_ab(full_wq + 8u * (mB % 3), (uint32_t)(mB / 3) & 1u, s_abort);
-            fence_after_sync();
-            if (ok) {
-#pragma unroll
-                for (int kk = 0; kk < 128; kk += 16) {
-                    const int m = kk < 64 ? mA : mB;
-                    const uint64_t dA = desc_sw128(sb + kC_WQ + (uint32_t)(m % 3) * 16384u + ((kk & 63) << 1), 16u, 1024u);
-                    mma_bf16(tmem + 128, dA, dS + (uint64_t)((kk * 128) >> 4), id1, kk > 0);
-                    if (kk == 48) {
-                        mma_commit(bar_half);
-                        ++n_half;
-                    }
-                }
-                mma_commit(bar_d1);
-                ++n_d1;
-                pump();  // the next chunk's first half and Kd tile, if published
-                ok = mbar_wait_ab(bar_half, par, s_abort);
-                half_done = c + 1;
-                if (ok) pump();  // the next chunk's second half
-            }
-        }
-        __syncwarp();
-        ok = ok && mbar_wait_ab(bar_d1, par, s_abort);
-        if (tid == 0) d1_done = c + 1;
-        fence_after_sync();
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            float x[32];
-            tmem_ld16(tl + 128 + c0 + 32 * half, x);
-            tmem_ld16(tl + 128 + c0 + 32 * half + 16, x + 16);
-            tmem_wait_ld();
-            if (q4 < 2) {  // U = Uv - X -> the U tile (the S tile's first half: MMA1 has read S)
-#pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    float uu[8];
-                    unpack8(raw[4 * half + m], uu);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) uu[e] -= x[8 * m + e];
-                    *reinterpret_cast<uint4*>(sm + kC_S + sw128_chunk_off(r64, 8 * hcol + 4 * half + m, 64)) = pack8(uu);
-                }
-            } else if (r64 < L && ok) {  // out = O' + O0
-                uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)(t0 + r64) * H + h) * 128 + c0 + 32 * half);
-#pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    float o[8];
-                    unpack8(raw[4 * half + m], o);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) o[e] += x[8 * m + e];
-                    dst[m] = pack8(o);
-                }
-            }
-        }
-        if (q4 < 2) {  // U written: MMA2 may run (the four U warps arrive, the issuing warp waits)
-            fence_proxy_async();
-            fence_before_sync();
-            if (warp == 0) named_sync(1, 128); else named_arrive(1, 128);
-        }
-        if (tid == 0) {
-            fence_after_sync();
-            ok = ok && mbar_wait_ab(full_kd + 8u * par, (uint32_t)(c >> 1) & 1u, s_abort);
-            if (ok) {
-                const uint64_t dK = desc_sw128(sb + kC_Kd + par * 16384u, 64 * 128, 1024u);
-#pragma unroll
-                for (int kk = 0; kk < 64; kk += 16)
-                    mma_bf16(tmem + 0, dK + (uint64_t)((kk * 128) >> 4), dU + (uint64_t)((kk * 128) >> 4), id2, 1u);
-                mma_commit(bar_y);
-                ++n_y;
-            }
-        }
-        __syncwarp();
-        // the next chunk's rows and e^{g_last} (the state already carries this chunk's decay)
-        if (more) {
-            need(c + 1);
-            if (ok) load_rows(c + 1);
-        }
-        ok = ok && mbar_wait_ab(bar_y, par, s_abort);
-        fence_after_sync();
-        if (tid == 0) {
-            y_done = c + 1;
-            if (ok) pump();  // the Kd tile of chunk c + 2 (MMA2 of chunk c has read its buffer)
-        }
-        __syncwarp();
-        // S_{c+1} from TMEM -> its bf16 copy for the next chunk's MMA1, and Diag(e^{g_last}) S_{c+1} back
-        // into TMEM, onto which MMA2 of chunk c + 1 accumulates
-        float sn[64];
-#pragma unroll
-        for (int m = 0; m < 64; m += 16) tmem_ld16(tl + c0 + m, sn + m);
-        tmem_wait_ld();
-#pragma unroll
-        for (int m = 0; m < 8; ++m)
-            *reinterpret_cast<uint4*>(sm + kC_S + sw128_chunk_off(row, 8 * hcol + m, 128)) = pack8(sn + 8 * m);
-        if (more) {
-#pragma unroll
-            for (int m = 0; m < 64; ++m) sn[m] *= gam;
-#pragma unroll
-            for (int m = 0; m < 64; m += 16) tmem_st16(tl + c0 + m, sn + m);
-            tmem_wait_st();
-        } else if (S_final && ok) {
-#pragma unroll
-            for (int m = 0; m < 64; m += 4)
-                *reinterpret_cast<float4*>(S_final + srow + m) = make_float4(sn[m], sn[m + 1], sn[m + 2], sn[m + 3]);
-        }
-        fence_proxy_async();
-        fence_before_sync();
-        // S tile written, the scaled state stored and [X; O'] read: the next MMA1 may start (only the
-        // issuing warp waits)
-        if (warp == 0) named_sync(2, kAThreads); else named_arrive(2, kAThreads);
-        if (tid == kChainPoller && ok) poll_nb(c + 1 + kChainLookahead);  // while the next MMA1 runs
-        fence_after_sync();
-    }
-    ok = __syncthreads_and(ok && !*s_abort);
-    if (tid == 0 && !ok) {  // copies and MMAs that may still be in flight: bounded waits for the last of each
-        for (int b = 0; b < 3; ++b)
-            if (n_wq[b]) (void)mbar_wait(full_wq + 8 * b, (uint32_t)(n_wq[b] - 1) & 1u);
-        for (int b = 0; b < 2; ++b)
-            if (n_kd[b]) (void)mbar_wait(full_kd + 8 * b, (uint32_t)(n_kd[b] - 1) & 1u);
-        if (n_half) (void)mbar_wait(bar_half, (uint32_t)(n_half - 1) & 1u);
-        if (n_d1) (void)mbar_wait(bar_d1, (uint32_t)(n_d1 - 1) & 1u);
-        if (n_y) (void)mbar_wait(bar_y, (uint32_t)(n_y - 1) & 1u);
-    }
-    fence_before_sync();
-    __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, 256);
-}
-
-template <bool PRO, bool LA16>
-__global__ void __launch_bounds__(kAThreads, 2)
-tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_la,
-                const float* __restrict__ beta, WsHeader* __restrict__ hdr, const int* __restrict__ off,
-                const int32_t* __restrict__ cu, int Tseq, int N, int H, int G, unsigned pro, int J,
-                uint8_t* __restrict__ slots, uint32_t* __restrict__ flags, int nchain, const float* S0,
-                float* S_final, __nv_bfloat16* __restrict__ out)
-{
-    extern __shared__ __align__(1024) uint8_t fused_smem[];
-    if (tc::smem_u32(fused_smem) & 1023u) {  // the chain role's layout assumes a 1024-aligned base
-        if (threadIdx.x == 0) set_error(KDA_ERR_UNSUPPORTED);
-        return;
-    }
-    if ((int)blockIdx.x < nchain)
-        tc_chain_body(fused_smem, blockIdx.x, S0, S_final, out, hdr, off, cu, Tseq, N, H, J, slots, flags);
-    else
-        tc_intra_body<PRO, LA16, true>(fused_smem, (long long)blockIdx.x - nchain, (long long)gridDim.x - nchain,
-                                       &tm_q, &tm_k, &tm_v, &tm_la, beta, hdr, off, cu, Tseq, N, H, G, pro, J,
-                                       slots, flags);
-}
-
 // cuTensorMapEncodeTiled, fetched from the driver through the runtime (no link against libcuda)
 typedef CUresult (*TensorMapEncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                       const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -1557,42 +1086,11 @@ inline bool make_token_map(CUtensorMap* m, const void* base, bool bf16, int H, l
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Fused or two-kernel: the fused launch takes up to kFusedMaxChains chains, so that most CTAs produce.
-// Returns true when the fused kernel was launched (err holds the launch status).
-template <bool PRO, bool LA16>
-inline bool try_launch_fused(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                             const CUtensorMap& tla, const float* beta, const WsHeader* hdr, const int* off,
-                             const int32_t* cu, int Tseq, int N, int H, int Hk, unsigned pro, int J, char* slots,
-                             uint32_t* flags, long long units, const float* S0, float* S_final, void* out, int sms,
-                             cudaStream_t stream, cudaError_t& err)
-{
-    err = cudaSuccess;
-    const long long chains = (long long)N * H;
-    if (flags == nullptr || chains > kFusedMaxChains || chains <= 0) return false;
-    auto* kern = tc_fused_kernel<PRO, LA16>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kF_Smem) != cudaSuccess) {
-        (void)cudaGetLastError();
-        return false;
-    }
-    // Two CTAs fit an SM (128 registers x 256 threads and 113 KB of shared memory each).  The launch
-    // needs no residency guarantee: chains wait only on units that a running producer has claimed,
-    // and every SM but the chains' keeps at least one producer, so some producer always runs.
-    const int grid = 2 * sms;
-    if (grid - chains < chains || chains >= sms) return false;
-    err = cudaMemsetAsync(flags, 0, sizeof(uint32_t) * (size_t)units, stream);
-    if (err != cudaSuccess) return true;
-    LaunchScope ls("tc_fused", stream);
-    kern<<<grid, kAThreads, kF_Smem, stream>>>(tq, tk, tv, tla, beta, const_cast<WsHeader*>(hdr), off, cu, Tseq, N, H,
-                                               H / Hk, pro, J, (uint8_t*)slots, flags, (int)chains, S0, S_final,
-                                               (__nv_bfloat16*)out);
-    err = cudaGetLastError();
-    return true;
-}
-
 inline cudaError_t launch_tc_prefill(const void* q, const void* k, const void* v, const void* la, const float* beta,
                                      const float* S0, float* S_final, void* out, const WsHeader* hdr, const int* off,
                                      const int32_t* cu, int Tseq, int N, int H, int Hk, unsigned pro, int max_chunks,
-                                     long long Ttot, char* slots, uint32_t* flags, cudaStream_t stream)
+                                     long long Ttot,
+                                     char* slots, cudaStream_t stream)
 {
     // instance: (any q/k, beta or gate-activation bit, bf16 gates)
     const bool la16 = (pro & KDA_PROLOGUE_GATE_BF16) != 0, pr = (pro & ~KDA_PROLOGUE_GATE_BF16) != 0;
@@ -1611,25 +1109,10 @@ inline cudaError_t launch_tc_prefill(const void* q, const void* k, const void* v
         int dev = 0, sms = 148;
         if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         const long long units = (long long)max_chunks * H;
-        {
-            bool launched;
-            if (pr)
-                launched = la16 ? try_launch_fused<true, true>(tq, tk, tv, tla, beta, hdr, off, cu, Tseq, N, H, Hk, pro,
-                                                               max_chunks, slots, flags, units, S0, S_final, out, sms, stream, e)
-                                : try_launch_fused<true, false>(tq, tk, tv, tla, beta, hdr, off, cu, Tseq, N, H, Hk,
-                                                                pro, max_chunks, slots, flags, units, S0, S_final, out, sms, stream, e);
-            else
-                launched = la16 ? try_launch_fused<false, true>(tq, tk, tv, tla, beta, hdr, off, cu, Tseq, N, H, Hk,
-                                                                pro, max_chunks, slots, flags, units, S0, S_final, out, sms, stream, e)
-                                : try_launch_fused<false, false>(tq, tk, tv, tla, beta, hdr, off, cu, Tseq, N, H, Hk,
-                                                                 pro, max_chunks, slots, flags, units, S0, S_final, out, sms, stream,
-                                                                 e);
-            if (launched) return e;
-        }
         const unsigned grid = (unsigned)(units < 2LL * sms ? units : 2LL * sms);
         LaunchScope ls("tc_intra", stream);
         kern<<<grid, kAThreads, kA_Smem, stream>>>(tq, tk, tv, tla, beta, const_cast<WsHeader*>(hdr), off, cu, Tseq,
-                                                  N, H, H / Hk, pro, max_chunks, (uint8_t*)slots);
+                                                  N, H, H / Hk, pro, (uint8_t*)slots);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
@@ -1637,7 +1120,7 @@ inline cudaError_t launch_tc_prefill(const void* q, const void* k, const void* v
     const long long nb = (long long)N * H * (128 / kTcNV);
     if (nb > 0x7fffffffLL) return cudaErrorInvalidValue;
     tc_inter_kernel<<<(unsigned)nb, kBThreads, kB_Smem, stream>>>(
-        S0, S_final, (__nv_bfloat16*)out, hdr, off, cu, Tseq, N, H, max_chunks, (const uint8_t*)slots);
+        S0, S_final, (__nv_bfloat16*)out, hdr, off, cu, Tseq, N, H, (const uint8_t*)slots);
     return cudaGetLastError();
 }
 

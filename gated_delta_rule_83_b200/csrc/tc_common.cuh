@@ -223,6 +223,12 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst_smem, const void* tmap,
         : "memory");
 }
 
+// brings a tensor map (kernel parameter space) into the descriptor cache ahead of its first use
+__device__ __forceinline__ void prefetch_tensormap(const void* tmap)
+{
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
+}
+
 // ---- small helpers ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b)
 {

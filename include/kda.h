@@ -150,30 +150,16 @@ kda_status kda_decode_step(const void* q, const void* k, const void* v, const fl
  *                                             bit-identical to the fp32 call on the same values; the
  *                                             largest input of the prefill is halved.  Any dt.
  *                 Other bits: KDA_ERR_INVALID_ARG.
- *   schedule      How the tensor-core prefill (bf16 q/k/v, dk = dv = 128) is launched; every
- *                 schedule computes the same chunk form, the results agree up to fp32 rounding:
- *                   KDA_SCHEDULE_AUTO      (0) the library's choice (at present the two-pass one);
- *                   KDA_SCHEDULE_TWO_PASS  (1) the intra-chunk kernel over all (chunk, head) units,
- *                                              then the sequential kernel over the chains;
- *                   KDA_SCHEDULE_FUSED     (2) one persistent launch: producer CTAs build the units
- *                                              and publish a ready flag per unit, one chain CTA per
- *                                              (sequence, head) consumes them from L2 as they
- *                                              appear.  Taken for up to 64 chains, else two-pass.
- *                 Ignored by the fp32 / d = 64 path and by decode.  Other values: KDA_ERR_INVALID_ARG.
  *   reserved      Must be zero (KDA_ERR_INVALID_ARG otherwise).
  */
 #define KDA_PROLOGUE_L2NORM_QK 1u
 #define KDA_PROLOGUE_GATE_LOGITS 2u
 #define KDA_PROLOGUE_BETA_LOGITS 4u
 #define KDA_PROLOGUE_GATE_BF16 8u
-#define KDA_SCHEDULE_AUTO 0
-#define KDA_SCHEDULE_TWO_PASS 1
-#define KDA_SCHEDULE_FUSED 2
 typedef struct {
     int num_qk_heads;
     unsigned prologue;
-    int schedule;
-    int reserved[5];
+    int reserved[6];
 } kda_options;
 
 /*
@@ -330,11 +316,14 @@ kda_status kda_selftest_timeout(kda_stream_t stream);
  * KDA_NOALLOC_SCRATCH_BYTES bytes of static device memory on every GPU that loads the library,
  * held until the process exits.  It calls no cudaMalloc, cudaFree or allocating library routine.
  *   - Limit: a problem whose kda_chunk_fwd_workspace_size() exceeds KDA_NOALLOC_SCRATCH_BYTES is
- *     rejected with KDA_ERR_WORKSPACE before anything is launched.  With bf16, dk = dv = 128 and
- *     H = 32 that is a few thousand tokens per call; longer inputs can be fed in pieces, passing
- *     S_final of one call as S0 of the next.
- *   - The first call on a device looks up the array's device address on that device (make that
- *     device current first); make this first call before any stream capture.
+ *     rejected with KDA_ERR_WORKSPACE before anything is launched.  For bf16 with dk = dv = 128 the
+ *     workspace is 512 B (more past 31 sequences) plus 82,432 B per (chunk, head), with
+ *     ceil(T / 64) chunks per sequence for regular batches and T / 64 + num_seqs for packed input:
+ *     at H = 32, 25 chunks, i.e. 1,600 tokens of one sequence.  Longer inputs can be fed in
+ *     pieces, passing S_final of one call as S0 of the next.
+ *   - Every call looks up the array's device address on the device current at the call (make
+ *     the device of the tensors current); make the first call on a device before any stream
+ *     capture, since it may load the library's device code on that device.
  *   - All calls on a device share the one array: calls that overlap on the GPU (e.g. on two
  *     streams at once) race and corrupt each other's results.  Serialise them.  The kernels
  *     rewrite every scratch byte they read within the same call, so nothing has to start zeroed

@@ -120,11 +120,6 @@ def test_options_are_validated_before_launch(lib):
     assert lib.kda_chunk_fwd_ex(*args, ctypes.byref(res), fake, 1 << 30, None) == 1
     unknown = KdaOptions(prologue=16)               # not a KDA_PROLOGUE_* bit
     assert lib.kda_chunk_fwd_ex(*args, ctypes.byref(unknown), fake, 1 << 30, None) == 1
-    for bad_schedule in (-1, 3):                    # not a KDA_SCHEDULE_* value
-        sch = KdaOptions(schedule=bad_schedule)
-        assert lib.kda_chunk_fwd_ex(*args, ctypes.byref(sch), fake, 1 << 30, None) == 1
-    fused = KdaOptions(schedule=2)                  # valid: fails only on the missing workspace
-    assert lib.kda_chunk_fwd_ex(*args, ctypes.byref(fused), None, 1 << 30, None) == 5
     ok_group = KdaOptions(num_qk_heads=3, prologue=15)
     # a valid group with a missing workspace fails only on the workspace, like kda_chunk_fwd
     assert lib.kda_chunk_fwd_ex(*args, ctypes.byref(ok_group), None, 1 << 30, None) == 5

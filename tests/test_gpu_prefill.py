@@ -26,11 +26,10 @@ def small_workload(dtype="bf16", dk=128, dv=128, s0_std=0.5, seed=123):
     return synth.Workload("test", "prefill", 2, 0, 2, dk, dv, dtype, seed, s0_std=s0_std)
 
 
-def run_and_compare(inp, dtype, pairs=None, check_all=True, tol=None, schedule=0):
+def run_and_compare(inp, dtype, pairs=None, check_all=True, tol=None):
     m = kda()
     d = {k: (v.to(DEV) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
-    out, sf = m.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], S0=d["S0"], cu_seqlens=d["cu_seqlens"],
-                          schedule=schedule)
+    out, sf = m.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], S0=d["S0"], cu_seqlens=d["cu_seqlens"])
     m.check()
     o_ref, s_ref = oracle_prefill(inp, pairs=pairs)
     o_gpu, s_gpu = np64(out), np64(sf)
@@ -74,44 +73,19 @@ def test_dtypes_and_dims(dtype, dk, dv, T):
     run_and_compare(synth.prefill_inputs(w, T=T), dtype)
 
 
-@pytest.mark.parametrize("H,T,lengths", [(72, 130, None), (4, None, [3, 64, 65, 1, 200, 0, 129, 64, 70, 17, 5, 90,
-                                                                      128, 33, 64, 100, 2])])
-def test_two_kernel_path(H, T, lengths):
-    """More (sequence, head) chains than the fused launch takes (72 and 68 > 64): the intra-chunk
-    and the sequential kernels run as two launches over the same workspace."""
-    w = synth.Workload("test", "prefill", 1, 0, H, 128, 128, "bf16", 321, s0_std=0.5)
-    run_and_compare(synth.prefill_inputs(w, T=T, lengths=lengths), "bf16")
-
-
-@pytest.mark.parametrize("B,H,T", [(1, 64, 200), (3, 21, 257), (2, 1, 1000), (4, 16, 64), (1, 2, 1), (1, 4, 65)])
-def test_fused_schedule_shapes(B, H, T):
-    """The fused schedule at its chain limit (64), with several sequences of a regular batch (chunk-major
-    production across sequences), a single long chain, one chunk per sequence and ragged tails."""
+@pytest.mark.parametrize("B,H,T", [(1, 72, 130), (3, 21, 257), (2, 1, 1000), (4, 16, 64), (1, 2, 1), (1, 4, 65)])
+def test_tc_launch_shapes(B, H, T):
+    """Tensor-core prefill over many heads, several sequences of a regular batch, one long chain,
+    one chunk per sequence and ragged tails."""
     w = synth.Workload("test", "prefill", B, 0, H, 128, 128, "bf16", 322, s0_std=0.5)
-    run_and_compare(synth.prefill_inputs(w, T=T), "bf16", schedule=2)
+    run_and_compare(synth.prefill_inputs(w, T=T), "bf16")
 
 
-def test_fused_schedule_varlen_and_gates():
-    """Fused schedule with packed sequences (empty ones included) and extreme gates."""
-    w = small_workload("bf16")
-    inp = synth.prefill_inputs(w, lengths=[1, 63, 64, 0, 65, 200, 17, 128])
-    run_and_compare(inp, "bf16", schedule=2)
-    inp = synth.prefill_inputs(w, T=200)
-    inp["log_alpha"][..., ::7] = -30.0
-    run_and_compare(inp, "bf16", schedule=2)
-
-
-def test_schedules_agree():
-    """Two-pass and fused schedules on the same input: equal up to fp32 rounding."""
-    m = kda()
-    w = synth.Workload("test", "prefill", 2, 0, 8, 128, 128, "bf16", 323, s0_std=0.5)
-    d = synth.prefill_inputs(w, device=DEV, T=700)
-    res = []
-    for sch in (1, 2):
-        res.append(m.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], S0=d["S0"], schedule=sch))
-    m.check()
-    assert out_err(np64(res[1][0]), np64(res[0][0])) <= 1e-2
-    assert state_err(np64(res[1][1]), np64(res[0][1])) <= 1e-3
+def test_tc_many_sequences():
+    """17 packed sequences of 4 heads, empty and one-token sequences among them."""
+    w = synth.Workload("test", "prefill", 1, 0, 4, 128, 128, "bf16", 321, s0_std=0.5)
+    lengths = [3, 64, 65, 1, 200, 0, 129, 64, 70, 17, 5, 90, 128, 33, 64, 100, 2]
+    run_and_compare(synth.prefill_inputs(w, lengths=lengths), "bf16")
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
@@ -223,13 +197,6 @@ def test_prefill_32k_sampled():
     w = synth.WORKLOADS["prefill_32k"]
     inp = synth.prefill_inputs(w, device=DEV)
     report("prefill_32k heads 0/17/31", *run_and_compare(inp, "bf16", pairs=[(0, 0), (0, 17), (0, 31)]))
-
-
-def test_prefill_32k_fused_schedule_sampled():
-    w = synth.WORKLOADS["prefill_32k"]
-    inp = synth.prefill_inputs(w, device=DEV)
-    report("prefill_32k fused schedule, heads 0/17/31",
-           *run_and_compare(inp, "bf16", pairs=[(0, 0), (0, 17), (0, 31)], schedule=2))
 
 
 def test_varlen_64k_sampled():

@@ -103,15 +103,20 @@ __device__ __forceinline__ void named_arrive(int id, int threads)
 }
 
 // ------------------------------------------------------------------------------------------------
-// UT transform, in place: a strictly lower 64 x 64 A (fp32, row stride 68, zero on and above the
-// diagonal) is overwritten by X = (I + A)^{-1}, by recursive doubling: the four 16 x 16 diagonal
-// blocks by forward substitution; then, inside each 32 x 32 half, X_10 = -X_11 A_10 X_00; then the
-// 32 x 32 off-diagonal block X_10 = -X_11 A_10 X_00 of the whole.  256 threads.  Y: scratch of
-// 32 x 36 floats (16-byte aligned rows).
+// UT transform: from a strictly lower 64 x 64 A (fp32, row stride 68, zero on and above the diagonal)
+// to T = (I + A)^{-1} diag(beta), written as a bf16 K-major SW128 64 x 64 tile (the A operand of
+// [W' | Uv] = T [Kf | v]).  X = (I + A)^{-1} by recursive doubling: the four 16 x 16 diagonal blocks
+// by forward substitution; then, inside each 32 x 32 half, X_10 = -X_11 A_10 X_00; then the 32 x 32
+// off-diagonal block X_10 = -X_11 A_10 X_00 of the whole.  X overwrites A in place where a later
+// level reads it.  Each level also writes its blocks of T as soon as they are final, and threads idle
+// in the first level zero the blocks above the diagonal, so no separate pass packs T.  256 threads;
+// the levels use 64, 64 and 128 of them (with two CTAs per SM the idle warps' issue slots go to the
+// other CTA).  sY: scratch of 32 x 36 floats (16-byte aligned rows).
 // ------------------------------------------------------------------------------------------------
 constexpr int kAS = 68;  // row stride of A / X
 
-__device__ __forceinline__ void ut_inverse_64_inplace(float* __restrict__ sA, float* __restrict__ sY)
+__device__ __forceinline__ void ut_transform_T(float* __restrict__ sA, float* __restrict__ sY,
+                                               const float* __restrict__ s_beta, uint8_t* __restrict__ tT)
 {
     const int tid = threadIdx.x;
     {   // diagonal 16 x 16 blocks: thread -> (block, column jj); written back once every block is read
@@ -132,11 +137,22 @@ __device__ __forceinline__ void ut_inverse_64_inplace(float* __restrict__ sA, fl
                 }
                 x[r] = (r == jj) ? 1.f : ((r < jj) ? 0.f : -s);
             }
+        } else if (tid < 64 + 192) {  // the blocks of T above the diagonal: 192 chunks of 16 bytes
+            const int z = tid - 64;
+            int row, ch;
+            if (z < 96) { row = z / 6; ch = 2 + z % 6; }
+            else if (z < 160) { row = 16 + (z - 96) / 4; ch = 4 + (z - 96) % 4; }
+            else { row = 32 + (z - 160) / 2; ch = 6 + (z - 160) % 2; }
+            *reinterpret_cast<uint4*>(tT + tc::sw128_chunk_off(row, ch, 64)) = make_uint4(0, 0, 0, 0);
         }
         __syncthreads();
         if (tid < 64) {
+            const float bj = s_beta[b + jj];
 #pragma unroll
-            for (int r = 0; r < 16; ++r) sA[(b + r) * kAS + b + jj] = x[r];
+            for (int r = 0; r < 16; ++r) {
+                sA[(b + r) * kAS + b + jj] = x[r];
+                *reinterpret_cast<__nv_bfloat16*>(tT + tc::sw128_off(b + r, b + jj, 64)) = __float2bfloat16_rn(x[r] * bj);
+            }
         }
         __syncthreads();
     }
@@ -168,12 +184,18 @@ __device__ __forceinline__ void ut_inverse_64_inplace(float* __restrict__ sA, fl
             }
             *reinterpret_cast<float4*>(sA + (bi + ra) * kAS + bj + cc) = make_float4(-x0[0], -x0[1], -x0[2], -x0[3]);
             *reinterpret_cast<float4*>(sA + (bi + ra + 8) * kAS + bj + cc) = make_float4(-x1[0], -x1[1], -x1[2], -x1[3]);
+            const float4 be = *reinterpret_cast<const float4*>(s_beta + bj + cc);
+            *reinterpret_cast<uint2*>(tT + tc::sw128_off(bi + ra, bj + cc, 64)) =
+                make_uint2(tc::pack_bf16(-x0[0] * be.x, -x0[1] * be.y), tc::pack_bf16(-x0[2] * be.z, -x0[3] * be.w));
+            *reinterpret_cast<uint2*>(tT + tc::sw128_off(bi + ra + 8, bj + cc, 64)) =
+                make_uint2(tc::pack_bf16(-x1[0] * be.x, -x1[1] * be.y), tc::pack_bf16(-x1[2] * be.z, -x1[3] * be.w));
         }
         __syncthreads();
     }
     {   // level 2: rows 32..63, columns 0..31, on warps 0-3: thread -> (rows r0, r0 + 1, columns
         // cc..cc+3).  Each right-hand float4 serves two rows, which halves the shared-memory
         // wavefronts of the 128-bit loads; X22 is lower triangular, so warp w stops at row 8 w + 7.
+        // The block is final here: only its T values are written.
         const int r0 = 2 * (tid >> 3), cc = (tid & 7) * 4;
         if (tid < 128) {
             float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
@@ -198,11 +220,15 @@ __device__ __forceinline__ void ut_inverse_64_inplace(float* __restrict__ sA, fl
                 x0[0] = fmaf(a0, yv.x, x0[0]); x0[1] = fmaf(a0, yv.y, x0[1]); x0[2] = fmaf(a0, yv.z, x0[2]); x0[3] = fmaf(a0, yv.w, x0[3]);
                 x1[0] = fmaf(a1, yv.x, x1[0]); x1[1] = fmaf(a1, yv.y, x1[1]); x1[2] = fmaf(a1, yv.z, x1[2]); x1[3] = fmaf(a1, yv.w, x1[3]);
             }
-            *reinterpret_cast<float4*>(sA + (32 + r0) * kAS + cc) = make_float4(-x0[0], -x0[1], -x0[2], -x0[3]);
-            *reinterpret_cast<float4*>(sA + (33 + r0) * kAS + cc) = make_float4(-x1[0], -x1[1], -x1[2], -x1[3]);
+            const float4 be = *reinterpret_cast<const float4*>(s_beta + cc);
+            *reinterpret_cast<uint2*>(tT + tc::sw128_off(32 + r0, cc, 64)) =
+                make_uint2(tc::pack_bf16(-x0[0] * be.x, -x0[1] * be.y), tc::pack_bf16(-x0[2] * be.z, -x0[3] * be.w));
+            *reinterpret_cast<uint2*>(tT + tc::sw128_off(33 + r0, cc, 64)) =
+                make_uint2(tc::pack_bf16(-x1[0] * be.x, -x1[1] * be.y), tc::pack_bf16(-x1[2] * be.z, -x1[3] * be.w));
         }
-        __syncthreads();
     }
+    tc::fence_proxy_async();  // T is read by the tensor core
+    __syncthreads();
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -627,38 +653,8 @@ tc_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         fence_before_sync();
         ok = __syncthreads_and(ok);  // A and the P tile complete; the tensor core is done with Kb
 
-        // UT transform (X in place of A), then T = X diag(beta) as a bf16 K-major tile over Kb
-        if (ok) ut_inverse_64_inplace(sA, sY);
-        uint4 tch[2];
-        {   // 128-bit loads of the 8 values; lanes 4-7 of a quarter-warp take their upper half first so
-            // that no two lanes of a load share a bank group
-            const int c8 = tid & 7, hs = 4 * ((tid >> 2) & 1);
-            const float4 b0 = *reinterpret_cast<const float4*>(s_beta + 8 * c8 + hs);
-            const float4 b1 = *reinterpret_cast<const float4*>(s_beta + 8 * c8 + (hs ^ 4));
-#pragma unroll
-            for (int u2 = 0; u2 < 2; ++u2) {
-                const int r = (tid + kAThreads * u2) >> 3;
-                const float4 x0 = *reinterpret_cast<const float4*>(sA + r * kAS + 8 * c8 + hs);
-                const float4 x1 = *reinterpret_cast<const float4*>(sA + r * kAS + 8 * c8 + (hs ^ 4));
-                const float p0[4] = {x0.x * b0.x, x0.y * b0.y, x0.z * b0.z, x0.w * b0.w};
-                const float p1[4] = {x1.x * b1.x, x1.y * b1.y, x1.z * b1.z, x1.w * b1.w};
-                float t8[8];
-#pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    t8[m] = hs ? p1[m] : p0[m];
-                    t8[m + 4] = hs ? p0[m] : p1[m];
-                }
-                tch[u2] = pack8(t8);
-            }
-        }
-        __syncthreads();
-#pragma unroll
-        for (int u2 = 0; u2 < 2; ++u2) {
-            const int e = tid + kAThreads * u2;
-            *reinterpret_cast<uint4*>(sm + kA_B + sw128_chunk_off(e >> 3, e & 7, 64)) = tch[u2];
-        }
-        fence_proxy_async();
-        __syncthreads();
+        // UT transform: T = (I + A)^{-1} diag(beta) as a bf16 K-major tile over Kb (MMA1 has read Kb)
+        if (ok) ut_transform_T(sA, sY, s_beta, sm + kA_B);
         if (tid == 0) ok = mbar_wait_ab(mbar_v, par, s_abort) && ok;  // v in place
         if (ok && tid == 0) {  // W' = T Kf (B: k rows of the stacked tile), Uv = T v
             fence_after_sync();

@@ -381,6 +381,10 @@ def run_ours(args):
         # bf16 gates (KDA_PROLOGUE_GATE_BF16): the largest input halved, 1284 instead of 1540 B per token-head
         extra["prefill_32k_gate_bf16"] = bench_prefill_workload(torch, kda, synth, dev, stream, world, rank,
                                                                 "prefill_32k", steps=5, warmup=2, gate_bf16=True)
+        torch.cuda.empty_cache()
+        # the output gate in the prefill's epilogue (kda_chunk_fwd_gated): 128-channel group, sigmoid(z)
+        extra["prefill_32k_output_gate"] = bench_prefill_workload(torch, kda, synth, dev, stream, world, rank,
+                                                                  "prefill_32k", steps=5, warmup=2, output_gate=True)
 
     gnorm = None
     if not args.no_extra and args.only is None:
@@ -420,12 +424,14 @@ def run_ours(args):
 
 
 def bench_prefill_workload(torch, kda, synth, dev, stream, world, rank, name, steps, warmup, qk_heads=None,
-                           prologue=0, gate_bf16=False):
+                           prologue=0, gate_bf16=False, output_gate=False):
     """Device-timed throughput of another prefill workload (same method as the headline).  With
     ``qk_heads``, q and k keep only that many heads, shared by groups of value heads.  With
     ``prologue`` the call passes that kda_options.prologue value (the workload's inputs stand in
     for raw projections: the in-kernel transforms cost the same whatever the values).  With
-    ``gate_bf16`` log_alpha is passed as bf16 (half its bytes)."""
+    ``gate_bf16`` log_alpha is passed as bf16 (half its bytes).  With ``output_gate`` the call applies
+    the output gate (seeded bf16 z of out's shape, fp32 weight, one 128-channel group, sigmoid) and
+    writes the gated output instead of o."""
     w = synth.WORKLOADS[name]
     inp = synth.prefill_inputs(w, device=dev, seed=replica_seed(w.seed, rank))
     q, k, v, la, beta, S0, cu = (inp[x] for x in ("q", "k", "v", "log_alpha", "beta", "S0", "cu_seqlens"))
@@ -436,12 +442,17 @@ def bench_prefill_workload(torch, kda, synth, dev, stream, world, rank, name, st
         la = la.to(torch.bfloat16)
         inp["log_alpha"] = la
     out = torch.empty_like(v)
+    gate = {}
+    if output_gate:
+        g = torch.Generator(device=dev).manual_seed(replica_seed(w.seed + 1000, rank))
+        gate = dict(z=torch.randn(v.shape, generator=g, device=dev).to(torch.bfloat16),
+                    gate_weight=torch.rand(w.dv, generator=g, device=dev) + 0.5, gate_act="sigmoid")
     N = q.shape[0] if cu is None else cu.numel() - 1
     S_fin = torch.empty((N, w.H, w.dk, w.dv), dtype=torch.float32, device=dev)
     tokens = q.shape[0] * q.shape[1]
 
     def step():
-        kda.chunk_fwd(q, k, v, la, beta, S0=S0, cu_seqlens=cu, out=out, S_final=S_fin, prologue=prologue)
+        kda.chunk_fwd(q, k, v, la, beta, S0=S0, cu_seqlens=cu, out=out, S_final=S_fin, prologue=prologue, **gate)
 
     for _ in range(warmup):
         step()
@@ -464,10 +475,12 @@ def bench_prefill_workload(torch, kda, synth, dev, stream, world, rank, name, st
         desc += f"; input prologue {prologue} (q/k L2 norm, log-sigmoid gate logits, sigmoid beta logits in-kernel)"
     if gate_bf16:
         desc += "; log_alpha in bf16"
+    if output_gate:
+        desc += "; output gate in the epilogue (bf16 z read, gated output written instead of o; group 128, sigmoid)"
     res = {"desc": desc, "tokens": tokens, "steps": steps, "ms_per_step": ms / steps,
            "value": job_throughput(world, tokens, steps, ms), "unit": "tokens/s",
            "kernels": {k_: {"launches": n, "ms": t} for k_, (n, t) in prof.items()}}
-    del inp, q, k, v, la, beta, S0, out, S_fin
+    del inp, q, k, v, la, beta, S0, out, S_fin, gate
     return res
 
 

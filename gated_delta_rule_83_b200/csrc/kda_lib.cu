@@ -167,10 +167,11 @@ kda_status kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int
     return KDA_OK;
 }
 
-kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v, const void* log_alpha, const float* beta,
-                            const float* S0, const int32_t* cu_seqlens, int num_seqs, void* out, float* S_final,
-                            int B, int T, int H, int dk, int dv, kda_dtype dt, const kda_options* opt,
-                            void* workspace, size_t workspace_bytes, kda_stream_t stream_)
+kda_status kda_chunk_fwd_gated(const void* q, const void* k, const void* v, const void* log_alpha, const float* beta,
+                               const float* S0, const int32_t* cu_seqlens, int num_seqs, void* out, float* S_final,
+                               int B, int T, int H, int dk, int dv, kda_dtype dt, const kda_options* opt,
+                               const kda_output_gate* gate, void* workspace, size_t workspace_bytes,
+                               kda_stream_t stream_)
 {
     cudaStream_t stream = (cudaStream_t)stream_;
     int Hk = H;
@@ -180,6 +181,17 @@ kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v, const v
     Plan p;
     const kda_status st = make_plan(B, T, H, dk, dv, cu_seqlens != nullptr, num_seqs, dt, p);
     if (st != KDA_OK) return st;
+    int group = 0;
+    if (gate) {
+        for (int r : gate->reserved)
+            if (r != 0) return KDA_ERR_INVALID_ARG;
+        group = gate->group == 0 ? dv : gate->group;
+        if (group < 8 || group > dv || (group & (group - 1)) != 0) return KDA_ERR_INVALID_ARG;
+        if (!(gate->eps > 0.f) || (gate->act != KDA_GATE_IDENTITY && gate->act != KDA_GATE_SIGMOID))
+            return KDA_ERR_INVALID_ARG;
+        if (p.Ttot > 0 && (!gate->z || !aligned16(gate->z))) return KDA_ERR_INVALID_ARG;
+        if (gate->weight && !aligned16(gate->weight)) return KDA_ERR_INVALID_ARG;
+    }
     if (p.Ttot > 0 && (!q || !k || !v || !log_alpha || !beta || !out)) return KDA_ERR_INVALID_ARG;
     const void* ptrs[] = {q, k, v, log_alpha, beta, S0, out, S_final};
     for (const void* x : ptrs)
@@ -201,16 +213,39 @@ kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v, const v
 
     cudaError_t e;
     if (p.tc) {
+        // the tensor-core path applies the gate in phase B's epilogue, from the fp32 output
+        OutGate og{};
+        if (gate)
+            og = OutGate{(const __nv_bfloat16*)gate->z, gate->weight, 1.f / (float)group, gate->eps, group,
+                         gate->act == KDA_GATE_SIGMOID ? 1 : 0};
         e = launch_tc_prefill(q, k, v, log_alpha, beta, S0, S_final, out, hdr, off, cu_seqlens, p.Tseq, p.N, H, Hk, pro,
-                              p.max_chunks, p.Ttot, slots, stream);
-    } else if (dt == KDA_BF16) {
-        e = launch_simt_prefill<__nv_bfloat16>(q, k, v, log_alpha, beta, S0, S_final, out, hdr, off, cu_seqlens,
-                                               p.Tseq, p.N, H, Hk, pro, dk, dv, p.max_chunks, (float*)slots, stream);
+                              p.max_chunks, p.Ttot, slots, gate ? &og : nullptr, stream);
     } else {
-        e = launch_simt_prefill<float>(q, k, v, log_alpha, beta, S0, S_final, out, hdr, off, cu_seqlens, p.Tseq,
-                                       p.N, H, Hk, pro, dk, dv, p.max_chunks, (float*)slots, stream);
+        e = dt == KDA_BF16
+            ? launch_simt_prefill<__nv_bfloat16>(q, k, v, log_alpha, beta, S0, S_final, out, hdr, off, cu_seqlens,
+                                                 p.Tseq, p.N, H, Hk, pro, dk, dv, p.max_chunks, (float*)slots, stream)
+            : launch_simt_prefill<float>(q, k, v, log_alpha, beta, S0, S_final, out, hdr, off, cu_seqlens, p.Tseq,
+                                         p.N, H, Hk, pro, dk, dv, p.max_chunks, (float*)slots, stream);
+        // the CUDA-core path writes o, then the gate runs over it in place
+        if (e == cudaSuccess && gate && p.Ttot > 0) {
+            const long long rows = p.Ttot * H;
+            const int sg = gate->act == KDA_GATE_SIGMOID ? 1 : 0;
+            e = dt == KDA_BF16
+                ? launch_gated_rmsnorm<__nv_bfloat16>(out, gate->z, gate->weight, out, rows, dv, group, gate->eps, sg,
+                                                      stream)
+                : launch_gated_rmsnorm<float>(out, gate->z, gate->weight, out, rows, dv, group, gate->eps, sg, stream);
+        }
     }
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v, const void* log_alpha, const float* beta,
+                            const float* S0, const int32_t* cu_seqlens, int num_seqs, void* out, float* S_final,
+                            int B, int T, int H, int dk, int dv, kda_dtype dt, const kda_options* opt,
+                            void* workspace, size_t workspace_bytes, kda_stream_t stream)
+{
+    return kda_chunk_fwd_gated(q, k, v, log_alpha, beta, S0, cu_seqlens, num_seqs, out, S_final, B, T, H, dk, dv, dt,
+                               opt, nullptr, workspace, workspace_bytes, stream);
 }
 
 kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const float* log_alpha, const float* beta,

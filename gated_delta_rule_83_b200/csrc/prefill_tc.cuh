@@ -821,6 +821,26 @@ constexpr uint32_t kB_Misc = kB_U + 8192;          // mbarriers + TMEM address
 constexpr uint32_t kB_Smem = kB_Misc + 256 + 1024;
 constexpr uint32_t kTmD1 = 0, kTmY = 32;           // TMEM columns: [X; O'] and Y
 
+// The output gate in phase B's epilogue, y = o / sqrt(mean_group(o^2) + eps) * w * act(z) (the grouped,
+// gated RMS norm of the attention review's GDN/KDA pseudo-code and Ring-linear notes), computed from the
+// fp32 o = O' + O0 before it is rounded: o is never written.  A group of 8, 16 or 32 channels lies inside
+// one CTA's 32-column slice (kGateLocal); a group of 64 or 128 spans 2 or 4 slices, whose CTAs run as one
+// 4-CTA cluster and trade per-row partial sums of squares through distributed shared memory (kGateCluster).
+struct OutGate {
+    const __nv_bfloat16* z;  // [tokens][H][128], the layout of out
+    const float* w;          // [128] fp32, or nullptr (= ones)
+    float inv_g, eps;        // 1 / group, eps
+    int group;               // channels per norm group: 8, 16, 32, 64 or 128
+    int sigmoid;             // act = sigmoid (1) or identity (0)
+};
+constexpr int kGateNone = 0, kGateLocal = 1, kGateCluster = 2;
+// gated variants: the slice of w at kB_Misc + 256 (128 B); partial sums xs[2 parities][4 slices][64 rows]
+// fp32 at kB_Misc + 512 (2 KB); two exchange mbarriers at kB_Misc + 64; the next chunk's z rows (64 x 64 B,
+// 16-byte chunk m of row r at chunk m ^ ((r >> 1) & 3)) at kB_Z
+constexpr uint32_t kB_W = kB_Misc + 256, kB_X = kB_Misc + 512, kB_Z = kB_X + 2048;
+constexpr uint32_t kB_SmemGate = kB_Z + 4096 + 1024;
+static_assert(kB_SmemGate <= 232448, "phase B shared memory");
+
 __device__ __forceinline__ void tc_issue_stage(uint32_t stage_addr, uint32_t full_bar, const uint8_t* slot, int vt)
 {
     using namespace tc;
@@ -849,10 +869,24 @@ __device__ __forceinline__ void tc_prefetch_stage(const uint8_t* slot, int vt)
 }
 constexpr int kBPrefetch = 4;  // L2 prefetch distance beyond the shared-memory stages (chunks)
 
-__global__ void __launch_bounds__(kBThreads, 1)
+// row r of chunk j of the sequence [s0, s1): this CTA's 32 columns of z, copied asynchronously into the
+// row's 64 bytes at kB_Z (cp.async: no register waits on the load; rows past the end are zero-filled)
+__device__ __forceinline__ void copy_z_row(uint32_t zbuf, const __nv_bfloat16* z, long long s0, long long s1, int j,
+                                           int r, int H, int h, int v0)
+{
+    const long long t0 = s0 + (long long)j * 64;
+    const bool in = t0 + r < s1;
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(z + ((size_t)(t0 + (in ? r : 0)) * H + h) * 128 + v0);
+#pragma unroll
+    for (int m = 0; m < 4; ++m)
+        cp_async16(zbuf + (uint32_t)(r * 64 + ((m ^ ((r >> 1) & 3)) << 4)), src + 16 * m, in ? 16u : 0u);
+}
+
+template <int GATE>
+__global__ void __launch_bounds__(GATE == kGateNone ? kBThreads : kBThreads + 64, 1)
 tc_inter_kernel(const float* S0, float* S_final, __nv_bfloat16* __restrict__ out, const WsHeader* __restrict__ hdr,
                 const int* __restrict__ off, const int32_t* __restrict__ cu, int Tseq, int N, int H,
-                const uint8_t* __restrict__ slots)
+                const uint8_t* __restrict__ slots, OutGate gate)
 {
     using namespace tc;
     extern __shared__ uint8_t smem_raw[];
@@ -871,6 +905,8 @@ tc_inter_kernel(const float* S0, float* S_final, __nv_bfloat16* __restrict__ out
     const uint32_t bar_empty = bar_y + 8;               // kBStages barriers: stage consumed (128 arrivals)
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + kB_Misc + 128);
     volatile int* s_abort = reinterpret_cast<volatile int*>(sm + kB_Misc + 132);
+    const uint32_t bar_x = smem_u32(sm + kB_Misc + 64);  // kGateCluster: 2 exchange barriers (by chunk parity)
+    volatile int* s_xabort = reinterpret_cast<volatile int*>(sm + kB_Misc + 136);  // the exchange gave up
 
     const int jb = off[n], je = off[n + 1], nch = je - jb;
     const uint8_t* hslots = slots + (size_t)h * kSlotBytes;  // this head's slots, H slots apart
@@ -881,10 +917,17 @@ tc_inter_kernel(const float* S0, float* S_final, __nv_bfloat16* __restrict__ out
         for (int s = 0; s < kBStages; ++s) mbar_init(bar_full + 8 * s, 1);
         mbar_init(bar_d1, 1);
         mbar_init(bar_y, 1);
-        for (int s = 0; s < kBStages; ++s) mbar_init(bar_empty + 8 * s, kBCompute);
+        for (int s = 0; s < kBStages; ++s) mbar_init(bar_empty + 8 * s, GATE == kGateNone ? kBCompute : kBCompute + 64);
+        if (GATE == kGateCluster) {  // one local arrival (with the expected bytes) per phase
+            mbar_init(bar_x, 1);
+            mbar_init(bar_x + 8, 1);
+        }
         mbar_fence_init();
         *s_abort = 0;
+        if (GATE == kGateCluster) *s_xabort = 0;
     }
+    if (GATE != kGateNone && tid < kTcNV)
+        reinterpret_cast<float*>(sm + kB_W)[tid] = gate.w ? gate.w[v0 + tid] : 1.f;
     if (warp == 0) {
         tmem_alloc(smem_u32(s_tmem), 64);
         tmem_relinquish();
@@ -907,7 +950,10 @@ tc_inter_kernel(const float* S0, float* S_final, __nv_bfloat16* __restrict__ out
         for (int m = 0; m < 4; ++m) *reinterpret_cast<uint4*>(sm + kB_S + sw128_chunk_off(c, m, 128)) = pack8(S + 8 * m);
     }
     fence_proxy_async();
-    __syncthreads();  // barriers initialised, TMEM address visible, S tile written
+    if (GATE == kGateCluster)
+        cluster_sync();  // also every peer's exchange barriers initialised before the first remote arrival
+    else
+        __syncthreads();  // barriers initialised, TMEM address visible, S tile written
     if (warp == 5 && lane == 0) {
         for (int s = 0; s < kBStages && s < nch; ++s)
             tc_issue_stage(sb + s * kStageBytes, bar_full + 8 * s, hslots + (size_t)(jb + s) * H * kSlotBytes, vt);
@@ -921,15 +967,31 @@ tc_inter_kernel(const float* S0, float* S_final, __nv_bfloat16* __restrict__ out
     // descriptor bases; per K step only the 14-bit start address field advances (never carries)
     const uint64_t dS = desc_sw128(sb + kB_S, 128 * 128, 1024u), dU = desc_sw128(sb + kB_U, 64 * 128, 1024u);
     bool ok = true;
+    if (GATE != kGateNone && warp >= 6 && nch > 0)  // gated epilogue warps: the first chunk's z rows
+        copy_z_row(sb + kB_Z, gate.z, s0, s1, 0, tid - kBThreads, H, h, v0);
+    // kGateCluster: the partial-sum array and exchange barriers of the other CTAs of this CTA's group, as
+    // shared::cluster addresses (the same offsets in every CTA)
+    uint32_t peer_x[3] = {0, 0, 0}, peer_bar[3] = {0, 0, 0};
+    const int npeer = gate.group == 128 ? 3 : 1;  // a 128-channel group spans all four slices, 64 a pair
+    if (GATE == kGateCluster && warp >= 6) {
+#pragma unroll
+        for (int q = 0; q < 3; ++q) {
+            const uint32_t pv = gate.group == 128 ? (uint32_t)((vt + 1 + q) & 3) : (uint32_t)(vt ^ 1);
+            peer_x[q] = cluster_map(smem_u32(sm + kB_X), pv);
+            peer_bar[q] = cluster_map(bar_x, pv);
+        }
+    }
 
     // Roles per chunk (no CTA-wide barrier inside the loop):
     //   warp 4 (MMA)     : [X; O'] = [W; Q'] S once the S tile is ready (barrier 2), Y = Kd^T U once
     //                      the U tile is ready (barrier 1)
     //   warps 0-1        : U = Uv - X -> U tile, arrive on barrier 1
-    //   warps 2-3        : out = O' + O0
+    //   warps 2-3        : out = O' + O0 (ungated)
     //   warps 0-3        : S <- e^{g_last} S + Y -> S tile; arrive on the stage's "empty" mbarrier
     //                      (stage read) and on barrier 2 (S ready)
     //   warp 5 (copies)  : refills the stage of chunk it with chunk it+3 once it is empty
+    //   warps 6-7 (gated): read O' and O0, arrive on barrier 2 and the stage's "empty" mbarrier, then
+    //                      form o = O' + O0 and the gated output while the next chunk runs
     // A bounded wait that gives up raises the CTA's abort flag; every later wait then fails at once,
     // so the loop still runs its barriers to the end without hanging and exits quickly.
     for (int it = 0; it < nch; ++it) {
@@ -941,7 +1003,7 @@ tc_inter_kernel(const float* S0, float* S_final, __nv_bfloat16* __restrict__ out
         const uint32_t par = (uint32_t)it & 1u;
         const bool refill = it + kBStages < nch;
         if (warp == 4) {
-            if (it > 0) named_sync(2, 160);  // S tile of this chunk written
+            if (it > 0) named_sync(2, GATE == kGateNone ? 160 : 224);  // S tile written (and, gated, O' read)
             if (lane == 0) {
                 ok = ok && mbar_wait_ab(bar_full + 8 * s, (uint32_t)(it / kBStages) & 1u, s_abort);
                 fence_after_sync();
@@ -964,7 +1026,7 @@ tc_inter_kernel(const float* S0, float* S_final, __nv_bfloat16* __restrict__ out
                 mma_commit(bar_y);
             }
         } else if (warp == 5) {
-            if (refill && lane == 0) {  // stage s fully consumed (128 compute-thread arrivals) -> refill
+            if (refill && lane == 0) {  // stage s fully consumed (every reader arrived) -> refill
                 ok = ok && mbar_wait_ab(bar_empty + 8 * s, (uint32_t)(it / kBStages) & 1u, s_abort);
                 if (ok) {
                     tc_issue_stage(st, bar_full + 8 * s, hslots + (size_t)(jb + it + kBStages) * H * kSlotBytes, vt);
@@ -972,45 +1034,140 @@ tc_inter_kernel(const float* S0, float* S_final, __nv_bfloat16* __restrict__ out
                         tc_prefetch_stage(hslots + (size_t)(jb + it + kBStages + kBPrefetch) * H * kSlotBytes, vt);
                 }
             }
-        } else {
+        } else if (GATE != kGateNone && warp >= 6) {
+            // epilogue warps (gated): row r of O' is TMEM lane 64 + r, which warps 6 and 7 address
+            const int r = tid - kBThreads;
             ok = ok && mbar_wait_ab(bar_full + 8 * s, (uint32_t)(it / kBStages) & 1u, s_abort);
-            // this thread's Uv (warps 0-1) or O0 (warps 2-3) row and e^{g_last} are read before MMA1 is waited for
             uint4 raw[4];
 #pragma unroll
             for (int m = 0; m < 4; ++m)
-                raw[m] = *reinterpret_cast<const uint4*>(stp + (warp < 2 ? kStUv : kStO0) + sw128_chunk_off(c & 63, cq + m, 64));
-            const float gam = *reinterpret_cast<const float*>(stp + kStGam + 4 * c);
+                raw[m] = *reinterpret_cast<const uint4*>(stp + kStO0 + sw128_chunk_off(r, cq + m, 64));
             ok = ok && mbar_wait_ab(bar_d1, par, s_abort);
             fence_after_sync();
             float x[32];
             tmem_ld16(tw + kTmD1, x);
             tmem_ld16(tw + kTmD1 + 16, x + 16);
             tmem_wait_ld();
-            if (warp < 2) {  // U = Uv - X, row r = c
-                uint4 pk[4];
+            fence_before_sync();
+            if (it + 1 < nch) named_arrive(2, 224);      // O' read: the next MMA1 may overwrite it
+            if (refill) mbar_arrive(bar_empty + 8 * s);  // O0 read
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {  // o = O' + O0, kept in fp32
+                float u[8];
+                unpack8(raw[m], u);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) x[8 * m + e] += u[e];
+            }
+            float p[4];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                p[m] = 0.f;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) p[m] = fmaf(x[8 * m + e], x[8 * m + e], p[m]);
+            }
+            float rs[4];
+            bool xok = true;
+            const int g0 = gate.group == 128 ? 0 : (vt & 2), g1 = gate.group == 128 ? 4 : (vt & 2) + 2;
+            const uint32_t bx = bar_x + 8u * (uint32_t)(it & 1);
+            // this slice's share of the row's sum of squares -> its own slot and the other CTAs of the group.
+            // The exchange runs whatever `ok` says, so that every CTA's phases stay matched; it stops only
+            // after one of its own waits has timed out (s_xabort).
+            if (GATE == kGateCluster && !*s_xabort) {
+                const float part = (p[0] + p[1]) + (p[2] + p[3]);
+                const uint32_t xo = 4u * (uint32_t)((it & 1) * 256 + vt * 64 + r), bo = 8u * (uint32_t)(it & 1);
+                *reinterpret_cast<float*>(sm + kB_X + xo) = part;
+                if (r == 0) mbar_arrive_expect_tx(bx, (uint32_t)(g1 - g0 - 1) * 64u * 4u);
+#pragma unroll
+                for (int q = 0; q < 3; ++q)
+                    if (q < npeer) st_async_cluster_f32(peer_x[q] + xo, part, peer_bar[q] + bo);
+            }
+            // g = act(z) w while the partial sums travel; the next chunk's z row goes into the same shared
+            // bytes as soon as this one is in registers (unpacked), a whole chunk ahead of its use
+            cp_async_wait_all();
+            float gz[32];
+#pragma unroll
+            for (int m = 0; m < 4; ++m)
+                unpack8(*reinterpret_cast<const uint4*>(sm + kB_Z + r * 64 + ((m ^ ((r >> 1) & 3)) << 4)), gz + 8 * m);
+            if (it + 1 < nch) copy_z_row(sb + kB_Z, gate.z, s0, s1, it + 1, r, H, h, v0);
+            {
+                const float4* sw = reinterpret_cast<const float4*>(sm + kB_W);
 #pragma unroll
                 for (int m = 0; m < 4; ++m) {
-                    float u[8];
-                    unpack8(raw[m], u);
+                    const float4 wa = sw[2 * m], wb = sw[2 * m + 1];
+                    const float w8[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) u[e] -= x[8 * m + e];
-                    pk[m] = pack8(u);
+                    for (int e = 0; e < 8; ++e)
+                        gz[8 * m + e] = w8[e] * (gate.sigmoid ? sigmoid_tanh(gz[8 * m + e]) : gz[8 * m + e]);
                 }
+            }
+            if (GATE == kGateCluster) {
+                const float* xs = reinterpret_cast<const float*>(sm + kB_X) + (it & 1) * 256 + r;
+                xok = !*s_xabort && mbar_wait(bx, (uint32_t)(it >> 1) & 1u);
+                if (!xok) *s_xabort = 1;
+                const float ss = gate.group == 128 ? (xs[0] + xs[64]) + (xs[128] + xs[192]) : xs[g0 * 64] + xs[g0 * 64 + 64];
+                rs[0] = rs[1] = rs[2] = rs[3] = rsqrtf(ss * gate.inv_g + gate.eps);
+            } else {
+                if (gate.group >= 16) {
+                    p[0] = p[1] = p[0] + p[1];
+                    p[2] = p[3] = p[2] + p[3];
+                }
+                if (gate.group >= 32) p[0] = p[1] = p[2] = p[3] = p[0] + p[2];
 #pragma unroll
-                for (int m = 0; m < 4; ++m) *reinterpret_cast<uint4*>(sm + kB_U + sw128_chunk_off(c, m, 64)) = pk[m];
-                fence_proxy_async();
-                named_arrive(1, 96);
-            } else {  // out = O' + O0, row r = c - 64
-                const int r = c - 64;
-                if (r < L && ok) {
-                    uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)(t0 + r) * H + h) * 128 + v0);
+                for (int m = 0; m < 4; ++m) rs[m] = rsqrtf(p[m] * gate.inv_g + gate.eps);
+            }
+            if (r < L && ok && xok) {
+                uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)(t0 + r) * H + h) * 128 + v0);
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    float yv[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) yv[e] = x[8 * m + e] * rs[m] * gz[8 * m + e];
+                    dst[m] = pack8(yv);
+                }
+            }
+        } else {
+            ok = ok && mbar_wait_ab(bar_full + 8 * s, (uint32_t)(it / kBStages) & 1u, s_abort);
+            // this thread's Uv (warps 0-1) or O0 (warps 2-3) row and e^{g_last} are read before MMA1 is waited for
+            uint4 raw[4];
+            if (GATE == kGateNone || warp < 2) {
+#pragma unroll
+                for (int m = 0; m < 4; ++m)
+                    raw[m] = *reinterpret_cast<const uint4*>(stp + (warp < 2 ? kStUv : kStO0) + sw128_chunk_off(c & 63, cq + m, 64));
+            }
+            const float gam = *reinterpret_cast<const float*>(stp + kStGam + 4 * c);
+            if (GATE == kGateNone || warp < 2) {  // gated: warps 2-3 only carry the state
+                ok = ok && mbar_wait_ab(bar_d1, par, s_abort);
+                fence_after_sync();
+                float x[32];
+                tmem_ld16(tw + kTmD1, x);
+                tmem_ld16(tw + kTmD1 + 16, x + 16);
+                tmem_wait_ld();
+                if (warp < 2) {  // U = Uv - X, row r = c
+                    uint4 pk[4];
 #pragma unroll
                     for (int m = 0; m < 4; ++m) {
                         float u[8];
                         unpack8(raw[m], u);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) u[e] += x[8 * m + e];
-                        dst[m] = pack8(u);
+                        for (int e = 0; e < 8; ++e) u[e] -= x[8 * m + e];
+                        pk[m] = pack8(u);
+                    }
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) *reinterpret_cast<uint4*>(sm + kB_U + sw128_chunk_off(c, m, 64)) = pk[m];
+                    fence_proxy_async();
+                    named_arrive(1, 96);
+                } else {  // out = O' + O0, row r = c - 64
+                    const int r = c - 64;
+                    if (r < L && ok) {
+                        uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)(t0 + r) * H + h) * 128 + v0);
+#pragma unroll
+                        for (int m = 0; m < 4; ++m) {
+                            float u[8];
+                            unpack8(raw[m], u);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) u[e] += x[8 * m + e];
+                            dst[m] = pack8(u);
+                        }
                     }
                 }
             }
@@ -1030,7 +1187,7 @@ tc_inter_kernel(const float* S0, float* S_final, __nv_bfloat16* __restrict__ out
             for (int m = 0; m < 4; ++m) *reinterpret_cast<uint4*>(sm + kB_S + sw128_chunk_off(c, m, 128)) = pk[m];
             fence_proxy_async();
             fence_before_sync();
-            if (it + 1 < nch) named_arrive(2, 160);  // S tile ready for the next chunk
+            if (it + 1 < nch) named_arrive(2, GATE == kGateNone ? 160 : 224);  // S tile ready for the next chunk
         }
     }
     ok = __syncthreads_and(ok && !*s_abort);
@@ -1042,6 +1199,7 @@ tc_inter_kernel(const float* S0, float* S_final, __nv_bfloat16* __restrict__ out
     fence_before_sync();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, 64);
+    if (GATE == kGateCluster) cluster_sync();  // no CTA leaves while a peer may still write its shared memory
 }
 
 // cuTensorMapEncodeTiled, fetched from the driver through the runtime (no link against libcuda)
@@ -1086,7 +1244,7 @@ inline cudaError_t launch_tc_prefill(const void* q, const void* k, const void* v
                                      const float* S0, float* S_final, void* out, const WsHeader* hdr, const int* off,
                                      const int32_t* cu, int Tseq, int N, int H, int Hk, unsigned pro, int max_chunks,
                                      long long Ttot,
-                                     char* slots, cudaStream_t stream)
+                                     char* slots, const OutGate* gate, cudaStream_t stream)
 {
     // instance: (any q/k, beta or gate-activation bit, bf16 gates)
     const bool la16 = (pro & KDA_PROLOGUE_GATE_BF16) != 0, pr = (pro & ~KDA_PROLOGUE_GATE_BF16) != 0;
@@ -1094,7 +1252,11 @@ inline cudaError_t launch_tc_prefill(const void* q, const void* k, const void* v
                     : (la16 ? tc_intra_kernel<false, true> : tc_intra_kernel<false, false>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kA_Smem);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(tc_inter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kB_Smem);
+    const int gmode = !gate ? kGateNone : gate->group <= kTcNV ? kGateLocal : kGateCluster;
+    auto* kernB = gmode == kGateNone ? tc_inter_kernel<kGateNone>
+                : gmode == kGateLocal ? tc_inter_kernel<kGateLocal> : tc_inter_kernel<kGateCluster>;
+    const uint32_t smemB = gmode == kGateNone ? kB_Smem : kB_SmemGate;
+    e = cudaFuncSetAttribute(kernB, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smemB);
     if (e != cudaSuccess) return e;
     if (max_chunks > 0 && Ttot > 0) {
         alignas(64) CUtensorMap tq, tk, tv, tla;
@@ -1115,9 +1277,22 @@ inline cudaError_t launch_tc_prefill(const void* q, const void* k, const void* v
     LaunchScope ls("tc_inter", stream);
     const long long nb = (long long)N * H * (128 / kTcNV);
     if (nb > 0x7fffffffLL) return cudaErrorInvalidValue;
-    tc_inter_kernel<<<(unsigned)nb, kBThreads, kB_Smem, stream>>>(
-        S0, S_final, (__nv_bfloat16*)out, hdr, off, cu, Tseq, N, H, (const uint8_t*)slots);
-    return cudaGetLastError();
+    const OutGate g = gate ? *gate : OutGate{nullptr, nullptr, 0.f, 0.f, 0, 0};
+    // the four slice CTAs of one (sequence, head) are consecutive in the grid: a cluster of 4 along x
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)nb);
+    cfg.blockDim = dim3(gmode == kGateNone ? kBThreads : kBThreads + 64);
+    cfg.dynamicSmemBytes = smemB;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 128 / kTcNV;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = gmode == kGateCluster ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernB, S0, S_final, (__nv_bfloat16*)out, hdr, off, cu, Tseq, N, H,
+                              (const uint8_t*)slots, g);
 }
 
 }  // namespace kda

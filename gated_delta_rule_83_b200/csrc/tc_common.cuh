@@ -196,6 +196,36 @@ __device__ __forceinline__ bool mbar_wait_ab(uint32_t addr, uint32_t parity, vol
     return false;
 }
 
+// ---- thread-block cluster: distributed shared memory between the CTAs of one cluster ----------
+__device__ __forceinline__ uint32_t cluster_ctarank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// the shared::cluster address of `local_addr` (a shared::cta address) in the CTA of rank `rank`
+__device__ __forceinline__ uint32_t cluster_map(uint32_t local_addr, uint32_t rank)
+{
+    uint32_t a;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(local_addr), "r"(rank));
+    return a;
+}
+// Asynchronous 4-byte store into the shared memory of another CTA of the cluster (both addresses are
+// shared::cluster addresses in that CTA).  Its completion counts 4 bytes of transactions on that CTA's
+// mbarrier, which the receiver waits on like on a bulk copy; the sender neither waits nor fences, so
+// the store does not wait for this thread's outstanding global loads and stores.
+__device__ __forceinline__ void st_async_cluster_f32(uint32_t cluster_addr, float v, uint32_t cluster_bar)
+{
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(cluster_addr),
+                 "r"(__float_as_uint(v)), "r"(cluster_bar)
+                 : "memory");
+}
+// every thread of every CTA of the cluster (release / acquire at cluster scope)
+__device__ __forceinline__ void cluster_sync()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 // ---- bulk copy global -> shared (completion counted on an mbarrier) ---------------------------
 // bulk prefetch of a global range into L2 (no shared memory, no completion to wait for); address and
 // size multiples of 16 bytes
@@ -245,6 +275,14 @@ __device__ __forceinline__ float ex2_approx(float x)
     return y;
 }
 constexpr float kLog2e = 1.4426950408889634f;
+// sigmoid(x) = 0.5 + 0.5 tanh(x / 2), the tanh from the hardware's approximation (tanh.approx.f32, one
+// instruction; relative error about 2^-11, below a bf16 rounding of the result)
+__device__ __forceinline__ float sigmoid_tanh(float x)
+{
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
+    return fmaf(0.5f, t, 0.5f);
+}
 // log2(x) with the hardware's approximate base-2 logarithm (x > 0, normal range)
 __device__ __forceinline__ float lg2_approx(float x)
 {

@@ -29,6 +29,14 @@ class KdaOptions(ctypes.Structure):
     _fields_ = [("num_qk_heads", ctypes.c_int), ("prologue", ctypes.c_uint), ("reserved", ctypes.c_int * 6)]
 
 
+class KdaOutputGate(ctypes.Structure):
+    """``kda_output_gate`` of include/kda.h (the output gate of ``kda_chunk_fwd_gated``)."""
+    _fields_ = [("z", ctypes.c_void_p), ("weight", ctypes.c_void_p), ("group", ctypes.c_int),
+                ("eps", ctypes.c_float), ("act", ctypes.c_int), ("reserved", ctypes.c_int * 3)]
+
+
+GATE_ACT = {"none": 0, "sigmoid": 1}  # kda_gate_act
+
 # kda_options.prologue bits (KDA_PROLOGUE_* in include/kda.h)
 PROLOGUE_L2NORM_QK = 1     # q and k normalised per (token, q/k head) over d_k inside the kernels
 PROLOGUE_GATE_LOGITS = 2   # log_alpha holds raw gate logits a: log_alpha = log sigmoid(a)
@@ -46,6 +54,8 @@ ABI = {
                               ctypes.POINTER(KdaOptions), _P, _SZ, _P]),
     "kda_decode_step_ex": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, ctypes.POINTER(KdaOptions), _P]),
     "kda_gated_rmsnorm": (_I, [_P, _P, _P, _P, ctypes.c_longlong, _I, _I, ctypes.c_float, _I, _I, _P]),
+    "kda_chunk_fwd_gated": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _I,
+                                 ctypes.POINTER(KdaOptions), ctypes.POINTER(KdaOutputGate), _P, _SZ, _P]),
     "kda_chunk_fwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
     "kda_chunk_bwd_workspace_size": (_I, [_I, _I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(KdaOptions),
                                          ctypes.POINTER(_SZ)]),
@@ -174,7 +184,9 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torc
               S0: Optional[torch.Tensor] = None, cu_seqlens: Optional[torch.Tensor] = None,
               out: Optional[torch.Tensor] = None, S_final: Optional[torch.Tensor] = None,
               output_final_state: bool = True, workspace: Optional[torch.Tensor] = None,
-              stream: Optional[torch.cuda.Stream] = None, prologue: int = 0) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+              stream: Optional[torch.cuda.Stream] = None, prologue: int = 0,
+              z: Optional[torch.Tensor] = None, gate_weight: Optional[torch.Tensor] = None, gate_group: int = 0,
+              gate_eps: float = 1e-6, gate_act: str = "none") -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Chunked KDA prefill (``kda_chunk_fwd``).
 
     q, k: [B, T, Hk, dk]; log_alpha: [B, T, H, dk]; v: [B, T, H, dv]; beta: [B, T, H]; q/k/v bf16 or
@@ -182,7 +194,12 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torc
     a divisor of H (grouped heads, ``kda_chunk_fwd_ex``: value head h reads q/k head h // (H // Hk)).
     S0 / S_final: [N, H, dk, dv] fp32 (N = B, or len(cu_seqlens) - 1 for packed varlen input with B = 1).
     ``prologue``: PROLOGUE_* bits (raw q/k and gate logits transformed inside the kernels).
-    Returns (out [B, T, H, dv] in q's dtype, S_final or None).  S_final may be S0 (in place)."""
+    Returns (out [B, T, H, dv] in q's dtype, S_final or None).  S_final may be S0 (in place).
+
+    With ``z`` ([B, T, H, dv], q's dtype) the output gate is applied inside the prefill
+    (``kda_chunk_fwd_gated``): out = o / sqrt(mean_group(o^2) + gate_eps) * gate_weight * act(z),
+    gate_weight [dv] fp32 or None, gate_group 0 (= dv) or a power of two >= 8, gate_act "none" or
+    "sigmoid"; o itself is not returned."""
     lib = load_library()
     _req(q, "q")
     dev = q.device
@@ -223,7 +240,26 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torc
         workspace = _get_workspace(ws_bytes, dev, sh)
     else:
         _req(workspace, "workspace", torch.uint8, dev)
-    if Hk == H and not prologue:
+    if z is not None:
+        _req(z, "z", dtq, dev)
+        if tuple(z.shape) != (B, T, H, dv):
+            raise ValueError(f"z must be [{B}, {T}, {H}, {dv}]")
+        if z.data_ptr() == out.data_ptr() and z.numel():
+            raise ValueError("z must not alias out")
+        if gate_weight is not None:
+            _req(gate_weight, "gate_weight", torch.float32, dev)
+            if tuple(gate_weight.shape) != (dv,):
+                raise ValueError(f"gate_weight must be [{dv}]")
+        if gate_act not in GATE_ACT:
+            raise ValueError(f"gate_act must be one of {sorted(GATE_ACT)}")
+        g = KdaOutputGate(z=_ptr(z), weight=_ptr(gate_weight), group=gate_group, eps=gate_eps,
+                          act=GATE_ACT[gate_act])
+        opt = KdaOptions(num_qk_heads=Hk, prologue=prologue)
+        rc = lib.kda_chunk_fwd_gated(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0),
+                                     _ptr(cu_seqlens), N, _ptr(out), _ptr(S_final), B, T, H, dk, dv, _dt(q),
+                                     ctypes.byref(opt), ctypes.byref(g), _ptr(workspace), workspace.numel(), sh)
+        _check("kda_chunk_fwd_gated", rc)
+    elif Hk == H and not prologue:
         rc = lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0), _ptr(cu_seqlens),
                                N, _ptr(out), _ptr(S_final), B, T, H, dk, dv, _dt(q), _ptr(workspace),
                                workspace.numel(), sh)

@@ -290,6 +290,45 @@ kda_status kda_gated_rmsnorm(const void* o, const void* z, const float* weight, 
                              int group, float eps, kda_gate_act act, kda_dtype dt, kda_stream_t stream);
 
 /*
+ * kda_chunk_fwd_gated -- the prefill with the output gate applied: `out` receives
+ *
+ *     y = o / sqrt(mean_g(o^2) + eps) * weight * act(z)
+ *
+ * (the operation of kda_gated_rmsnorm) where o is the output kda_chunk_fwd_ex would write; o itself
+ * is not written anywhere.  On the tensor-core path (bf16, dk = dv = 128) the gate runs in the
+ * epilogue that forms o, from its fp32 value before any rounding, so y costs one read of z instead of
+ * a write and a read of o; groups of 64 or 128 channels are reduced across the four CTAs that own a
+ * head's output columns.  On every other path the prefill writes o to `out` and kda_gated_rmsnorm
+ * runs over it in place on the same stream.  The fused epilogue evaluates sigmoid(z) as
+ * 0.5 + 0.5 tanh(z / 2) with the hardware's tanh approximation (absolute error about 2^-11, below the
+ * bf16 rounding of y).
+ *
+ *   gate->z        [B, T, H, dv] element type dt (the layout of out), 16-byte aligned; may be NULL
+ *                  only when there are no tokens.  Must not alias out.
+ *   gate->weight   [dv] fp32, or NULL (= ones); 16-byte aligned.
+ *   gate->group    channels per norm group: 0 (= dv) or a power of two in [8, dv].
+ *   gate->eps      > 0.
+ *   gate->act      KDA_GATE_IDENTITY or KDA_GATE_SIGMOID.
+ *   gate->reserved must be zero.
+ * gate = NULL is exactly kda_chunk_fwd_ex.  All other arguments, the workspace, the errors and the
+ * asynchrony are those of kda_chunk_fwd_ex; a bad gate field returns KDA_ERR_INVALID_ARG before
+ * anything is launched.
+ */
+typedef struct {
+    const void* z;
+    const float* weight;
+    int group;
+    float eps;
+    kda_gate_act act;
+    int reserved[3];
+} kda_output_gate;
+kda_status kda_chunk_fwd_gated(const void* q, const void* k, const void* v, const void* log_alpha, const float* beta,
+                               const float* S0, const int32_t* cu_seqlens, int num_seqs, void* out, float* S_final,
+                               int B, int T, int H, int dk, int dv, kda_dtype dt, const kda_options* opt,
+                               const kda_output_gate* gate, void* workspace, size_t workspace_bytes,
+                               kda_stream_t stream);
+
+/*
  * kda_check -- synchronise `stream`, then read and clear the device error word of the current
  * device.  Returns KDA_OK, KDA_ERR_CUDA (a sticky CUDA error), KDA_ERR_BAD_SEQLENS or
  * KDA_ERR_TIMEOUT.

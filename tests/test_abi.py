@@ -32,6 +32,16 @@ def test_options_struct_matches_header():
     assert ctypes.sizeof(KdaOptions) == 32
 
 
+def test_output_gate_struct_matches_header():
+    """kda_output_gate in the binding has the header's field order and size (2 pointers, 6 ints)."""
+    from gated_delta_rule_83_b200.kda import KdaOutputGate
+    src = open(os.path.join(ROOT, "include", "kda.h")).read()
+    body = re.search(r"typedef struct \{([^}]*)\} kda_output_gate;", src).group(1)
+    names = re.findall(r"\**(\w+)(?:\[\d+\])?;", body)
+    assert names == [f[0] for f in KdaOutputGate._fields_]
+    assert ctypes.sizeof(KdaOutputGate) == 40
+
+
 def test_header_declares_entry_points():
     names = declared_functions()
     for required in ("kda_chunk_fwd", "kda_decode_step", "kda_chunk_fwd_workspace_size", "kda_check",
@@ -141,6 +151,35 @@ def test_gated_rmsnorm_rejects_before_launch(lib):
     assert lib.kda_gated_rmsnorm(fake, fake, None, fake, 10, 128, 0, c(1e-6), 5, 0, None) == 1     # act
     assert lib.kda_gated_rmsnorm(fake + 8, fake, None, fake, 10, 128, 0, c(1e-6), 0, 0, None) == 1  # aligned
     assert lib.kda_gated_rmsnorm(None, None, None, None, 0, 128, 0, c(1e-6), 0, 0, None) == 0      # rows = 0
+
+
+def test_gated_prefill_rejects_before_launch(lib):
+    """kda_chunk_fwd_gated checks every gate field before anything else is launched; a NULL gate is
+    kda_chunk_fwd_ex (here: the same workspace error)."""
+    from gated_delta_rule_83_b200.kda import KdaOutputGate
+    fake = 0x100000  # never dereferenced
+    args = (fake, fake, fake, fake, fake, None, None, 0, fake, None, 1, 64, 2, 128, 128, 0, None)
+
+    def rc(**kw):
+        g = KdaOutputGate(z=kw.pop("z", fake), weight=kw.pop("weight", None), group=kw.pop("group", 0),
+                          eps=kw.pop("eps", 1e-6), act=kw.pop("act", 1))
+        for i, r in enumerate(kw.pop("reserved", ())):
+            g.reserved[i] = r
+        return lib.kda_chunk_fwd_gated(*args, ctypes.byref(g), None, 1 << 30, None)
+
+    assert rc(group=24) == 1          # not a power of two
+    assert rc(group=256) == 1         # more than dv
+    assert rc(group=4) == 1           # fewer than 8
+    assert rc(eps=0.0) == 1
+    assert rc(eps=-1.0) == 1
+    assert rc(act=2) == 1
+    assert rc(z=None) == 1            # tokens but no gate input
+    assert rc(z=fake + 8) == 1        # misaligned
+    assert rc(weight=fake + 4) == 1   # misaligned
+    assert rc(reserved=(0, 1)) == 1
+    assert rc(group=8) == 5           # a valid gate fails only on the missing workspace
+    assert rc(group=128, act=0) == 5
+    assert lib.kda_chunk_fwd_gated(*args, None, None, 1 << 30, None) == 5
 
 
 def test_missing_library_fails_loudly(tmp_path):

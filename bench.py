@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--no-extra", action="store_true", help="skip the varlen and 1M-token workloads")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override the prefill sequence length (profiling of a smaller case only)")
+    ap.add_argument("--output-gate", action="store_true",
+                    help="with --only prefill: apply the output gate in the prefill (profiling of that variant)")
     return ap.parse_args()
 
 
@@ -269,8 +271,16 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
     in_bytes = sum(x.numel() * x.element_size() for x in (q, k, v, la, beta) if x is not None)
 
+    gate = {}
+    if args.output_gate:
+        if args.only != "prefill":
+            raise SystemExit("--output-gate profiles the gated prefill: use it with --only prefill")
+        gg = torch.Generator(device=dev).manual_seed(replica_seed(w.seed + 1000, rank))
+        gate = dict(z=torch.randn(v.shape, generator=gg, device=dev).to(v.dtype),
+                    gate_weight=torch.rand(dv, generator=gg, device=dev) + 0.5, gate_act="sigmoid")
+
     def step():
-        kda.chunk_fwd(q, k, v, la, beta, S0=S0, cu_seqlens=cu, out=out, S_final=S_fin)
+        kda.chunk_fwd(q, k, v, la, beta, S0=S0, cu_seqlens=cu, out=out, S_final=S_fin, **gate)
 
     for _ in range(args.warmup):
         step()

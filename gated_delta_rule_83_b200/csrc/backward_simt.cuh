@@ -1016,6 +1016,12 @@ cudaError_t launch_bwd_chains(const float* S0, const void* dout, const float* dS
 
 // Steps 1-4.  Workspace regions (all per (chunk, head) of the forward's chunk table): the
 // CUDA-core forward slots, chunk start states, chunk end cotangents and the per-chunk scratch.
+// the tensor-core state side (backward_tc.cuh): bf16 inputs with dk = dv = 128
+cudaError_t launch_bwd_state_side_tc(const void* dout, const WsHeader* hdr, const int* off, const int32_t* cu,
+                                     int Tseq, int N, int H, int max_chunks, const float* S_chunks,
+                                     const float* dSn_chunks, float* scr, cudaStream_t stream);
+bool bwd_state_side_tc_ok(bool bf16, int dk, int dv);
+
 template <typename TIn>
 cudaError_t launch_simt_backward(const void* q, const void* k, const void* v, const void* la, const float* beta,
                                  const float* S0, const void* dout, const float* dS_final, void* dq, void* dk_out,
@@ -1081,7 +1087,11 @@ cudaError_t launch_simt_backward(const void* q, const void* k, const void* v, co
 #undef KDA_BWD_CHAINS
     if (e != cudaSuccess) return e;
     if (max_chunks > 0) {
-        {
+        if (bwd_state_side_tc_ok(sizeof(TIn) == 2, dk, dv)) {
+            e = launch_bwd_state_side_tc(dout, hdr, off, cu, Tseq, N, H, max_chunks, S_chunks, dSn_chunks, scr,
+                                         stream);
+            if (e != cudaSuccess) return e;
+        } else {
             LaunchScope ls("bwd_state_side", stream);
             bwd_state_side_kernel<TIn><<<dim3(max_chunks, H), kSimtThreads, smS, stream>>>(
                 (const TIn*)dout, hdr, off, cu, Tseq, N, H, dk, dv, S_chunks, dSn_chunks, scr);

@@ -9,6 +9,7 @@
 
 #include "kda.h"
 #include "backward_simt.cuh"
+#include "backward_tc.cuh"
 #include "common.cuh"
 #include "chunks.cuh"
 #include "decode.cuh"

@@ -981,6 +981,15 @@ inline size_t bwd_gate_smem()
     return sizeof(float) * ((size_t)3 * kChunk * kBwdL64 + 7 * kChunk * kBwdLT + kChunk + kBwdCT);
 }
 
+// the tensor-core kernels of the backward (backward_tc.cuh): bf16 inputs with dk = dv = 128
+bool bwd_state_side_tc_ok(bool bf16, int dk, int dv);
+cudaError_t launch_bwd_state_side_tc(const void* dout, const WsHeader* hdr, const int* off, const int32_t* cu,
+                                     int Tseq, int N, int H, int max_chunks, const float* S_chunks,
+                                     const float* dSn_chunks, float* scr, cudaStream_t stream);
+cudaError_t launch_bwd_do_terms_tc(const void* dout, const WsHeader* hdr, const int* off, const int32_t* cu,
+                                   int Tseq, int N, int H, int max_chunks, const float* slots, float* scr,
+                                   float* F_chunks, cudaStream_t stream);
+
 template <typename TIn, int DK, int DV>
 cudaError_t launch_bwd_chains(const float* S0, const void* dout, const float* dS_final, float* dS0,
                               const WsHeader* hdr, const int* off, const int32_t* cu, int Tseq, int N, int H,
@@ -1002,7 +1011,10 @@ cudaError_t launch_bwd_chains(const float* S0, const void* dout, const float* dS
                                                                       S_chunks, scr);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    if (max_chunks > 0) {
+    if (max_chunks > 0 && bwd_state_side_tc_ok(sizeof(TIn) == 2, DK, DV)) {
+        e = launch_bwd_do_terms_tc(dout, hdr, off, cu, Tseq, N, H, max_chunks, slots, scr, F_chunks, stream);
+        if (e != cudaSuccess) return e;
+    } else if (max_chunks > 0) {
         LaunchScope ls("bwd_do_terms", stream);
         bwd_do_terms_kernel<TIn, DK, DV><<<dim3(max_chunks, H), kSimtThreads, smT, stream>>>(
             (const TIn*)dout, hdr, off, cu, Tseq, N, H, slots, scr, F_chunks);
@@ -1016,11 +1028,6 @@ cudaError_t launch_bwd_chains(const float* S0, const void* dout, const float* dS
 
 // Steps 1-4.  Workspace regions (all per (chunk, head) of the forward's chunk table): the
 // CUDA-core forward slots, chunk start states, chunk end cotangents and the per-chunk scratch.
-// the tensor-core state side (backward_tc.cuh): bf16 inputs with dk = dv = 128
-cudaError_t launch_bwd_state_side_tc(const void* dout, const WsHeader* hdr, const int* off, const int32_t* cu,
-                                     int Tseq, int N, int H, int max_chunks, const float* S_chunks,
-                                     const float* dSn_chunks, float* scr, cudaStream_t stream);
-bool bwd_state_side_tc_ok(bool bf16, int dk, int dv);
 
 template <typename TIn>
 cudaError_t launch_simt_backward(const void* q, const void* k, const void* v, const void* la, const float* beta,

@@ -283,6 +283,138 @@ bwd_state_side_tc_kernel(const __nv_bfloat16* __restrict__ dout, const WsHeader*
     if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
+// ------------------------------------------------------------------------------------------------
+// The dO terms of the reverse chain, chunk-parallel (one CTA per (chunk, head)):
+//     E = P^T dO  (64 x dv, into the unit's dU scratch),   F = Qg^T dO  (dk x dv)
+// formed as one transposed product dO^T [P | Qg] (M = 128 value channels, N = 64 + 128, K = 64
+// tokens; both operands MN-major, i.e. the row-major token tiles as they are), so that the value
+// channel lands on the TMEM lane and the stores of E and F coalesce.  dO is exact in bf16; P and Qg
+// (fp32, from the forward's slot) are split into bf16 hi and lo parts: dO [P | Qg]_hi + dO [P | Qg]_lo.
+// ------------------------------------------------------------------------------------------------
+constexpr uint32_t kTO = 0;             // dO: 64 token rows x 128 (two atom columns), 16 KB
+constexpr uint32_t kTB_hi = 16384;      // [P | Qg] hi: 64 token rows x 192 (three atom columns), 24 KB
+constexpr uint32_t kTB_lo = 40960;      // ... lo
+constexpr uint32_t kTMisc = 65536;      // mbarrier | TMEM base address
+// 100 KB requested (64 KB used) so that at most two CTAs share an SM: two 256-column TMEM allocations
+constexpr uint32_t kDoTermsSmem = 102400;
+
+__global__ void __launch_bounds__(128)
+bwd_do_terms_tc_kernel(const __nv_bfloat16* __restrict__ dout, const WsHeader* __restrict__ hdr,
+                       const int* __restrict__ off, const int32_t* __restrict__ cu, int Tseq, int N, int H,
+                       const float* __restrict__ slots, float* __restrict__ scr, float* __restrict__ F_chunks)
+{
+    using namespace tc;
+    constexpr int D = 128;
+    extern __shared__ uint8_t smem_raw[];
+    const int j = blockIdx.x, h = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (hdr->bad || j >= hdr->total_chunks) return;
+    int n, L;
+    long long t0;
+    locate_chunk(j, off, cu, Tseq, N, n, t0, L);
+    uint8_t* sm = align1024(smem_raw);
+    const uint32_t sb = smem_u32(sm);
+    const uint32_t mbar = sb + kTMisc;
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + kTMisc + 8);
+    const size_t u = (size_t)j * H + h;
+    const float* slot = slots + u * simt_slot_floats(D, D);
+    const float* gQ = slot + (size_t)kChunk * D;
+    const float* gP = slot + 3 * (size_t)kChunk * D;
+    float* gE = scr + u * bwd_scr_floats(D, D) + (size_t)kChunk * D;
+    float* gF = F_chunks + u * D * D;
+
+    if (tid == 0) {
+        mbar_init(mbar, 1);
+        mbar_fence_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(s_tmem), 256);
+        tmem_relinquish();
+    }
+    // token rows -> SW128 tiles with 64-element atom columns (chunk ch of row r: 8 consecutive columns)
+    const uint4 z4 = make_uint4(0, 0, 0, 0);
+    {
+        const int ch = tid & 15, rq = tid >> 4;  // dO and Qg: rows rq + 8 m, chunk ch of 16
+        uint4 dov[8];
+        float fq[8][8];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            const int r = rq + 8 * m;
+            dov[m] = r < L ? *reinterpret_cast<const uint4*>(dout + ((size_t)(t0 + r) * H + h) * D + 8 * ch) : z4;
+            load8(gQ + (size_t)r * D + 8 * ch, fq[m]);
+        }
+        const int cp = tid & 7, rp = tid >> 3;   // P: rows rp + 16 m, chunk cp of 8
+        float fp[4][8];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) load8(gP + (size_t)(rp + 16 * m) * kChunk + 8 * cp, fp[m]);
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            const int r = rq + 8 * m;
+            uint4 hi, lo;
+            *reinterpret_cast<uint4*>(sm + kTO + sw128_chunk_off(r, ch, 64)) = dov[m];
+            split8(fq[m], hi, lo);
+            *reinterpret_cast<uint4*>(sm + kTB_hi + sw128_chunk_off(r, 8 + ch, 64)) = hi;
+            *reinterpret_cast<uint4*>(sm + kTB_lo + sw128_chunk_off(r, 8 + ch, 64)) = lo;
+        }
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            uint4 hi, lo;
+            split8(fp[m], hi, lo);
+            *reinterpret_cast<uint4*>(sm + kTB_hi + sw128_chunk_off(rp + 16 * m, cp, 64)) = hi;
+            *reinterpret_cast<uint4*>(sm + kTB_lo + sw128_chunk_off(rp + 16 * m, cp, 64)) = lo;
+        }
+    }
+    fence_proxy_async();
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = *s_tmem;
+    if (tid == 0) {
+        const uint32_t id = idesc_bf16(128, 192, true, true);
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+            for (int k0 = 0; k0 < kChunk; k0 += 16)
+                mma_bf16(tmem, desc_mnmajor(sb + kTO, kChunk, k0), desc_mnmajor(sb + (t ? kTB_lo : kTB_hi), kChunk, k0),
+                         id, (t > 0 || k0 > 0) ? 1u : 0u);
+        mma_commit(mbar);
+    }
+    const bool ok = mbar_wait(mbar, 0);
+    fence_after_sync();
+    if (ok) {  // lane = value channel jv; columns 0-63: E[i][jv], 64-191: F[c][jv]
+        const int jv = 32 * warp + lane;
+        const uint32_t tl = tmem + ((uint32_t)(32 * warp) << 16);
+#pragma unroll
+        for (int cb = 0; cb < 192; cb += 32) {
+            float v[32];
+            tmem_ld16(tl + cb, v);
+            tmem_ld16(tl + cb + 16, v + 16);
+            tmem_wait_ld();
+#pragma unroll
+            for (int m = 0; m < 32; ++m) {
+                const int col = cb + m;
+                if (col < kChunk) gE[(size_t)col * D + jv] = v[m];
+                else gF[(size_t)(col - kChunk) * D + jv] = v[m];
+            }
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 256);
+}
+
+inline cudaError_t launch_bwd_do_terms_tc(const void* dout, const WsHeader* hdr, const int* off, const int32_t* cu,
+                                          int Tseq, int N, int H, int max_chunks, const float* slots, float* scr,
+                                          float* F_chunks, cudaStream_t stream)
+{
+    cudaError_t e = cudaFuncSetAttribute(bwd_do_terms_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kDoTermsSmem);
+    if (e != cudaSuccess) return e;
+    LaunchScope ls("bwd_do_terms_tc", stream);
+    bwd_do_terms_tc_kernel<<<dim3(max_chunks, H), 128, kDoTermsSmem, stream>>>(
+        (const __nv_bfloat16*)dout, hdr, off, cu, Tseq, N, H, slots, scr, F_chunks);
+    return cudaGetLastError();
+}
+
 inline bool bwd_state_side_tc_ok(bool bf16, int dk, int dv) { return kTcPathReady && bf16 && dk == 128 && dv == 128; }
 
 inline cudaError_t launch_bwd_state_side_tc(const void* dout, const WsHeader* hdr, const int* off, const int32_t* cu,

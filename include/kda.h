@@ -232,7 +232,10 @@ kda_status kda_host_release(void);
  * "Kimi Linear" explainer (section "Kimi Delta Attention的技术内核"), taken through the chunk form
  * its section "硬件效率的深度优化" lists: the forward is recomputed chunk-parallel keeping only each
  * chunk's start state, the state cotangent runs backwards over the chunks, and the input
- * derivatives are again chunk-parallel.  Arithmetic is fp32 on CUDA cores.
+ * derivatives are again chunk-parallel.  Arithmetic is fp32 on CUDA cores; for bf16 inputs with
+ * dk = dv = 128 the state-side products and the output-cotangent terms run on the tensor cores with
+ * each fp32 operand split into two bf16 parts (hi*hi + hi*lo + lo*hi, about 16 significant bits),
+ * which keeps the same fp32-level accuracy.
  *
  *   q, k, v, log_alpha, beta, S0, cu_seqlens, num_seqs, B, T, H, dk, dv, dt:  exactly as given to
  *                kda_chunk_fwd (same layout, same meaning).

@@ -989,6 +989,10 @@ cudaError_t launch_bwd_state_side_tc(const void* dout, const WsHeader* hdr, cons
 cudaError_t launch_bwd_do_terms_tc(const void* dout, const WsHeader* hdr, const int* off, const int32_t* cu,
                                    int Tseq, int N, int H, int max_chunks, const float* slots, float* scr,
                                    float* F_chunks, cudaStream_t stream);
+cudaError_t launch_bwd_gate_tc(const void* q, const void* k, const void* la, bool la16, const float* beta,
+                               const WsHeader* hdr, const int* off, const int32_t* cu, int Tseq, int N, int H,
+                               int Hk, int max_chunks, const float* scr, void* dq, void* dk_out, float* dla,
+                               float* dq_acc, float* dk_acc, cudaStream_t stream);
 
 template <typename TIn, int DK, int DV>
 cudaError_t launch_bwd_chains(const float* S0, const void* dout, const float* dS_final, float* dS0,
@@ -1111,7 +1115,12 @@ cudaError_t launch_simt_backward(const void* q, const void* k, const void* v, co
                 (TIn*)dv_out, dbeta);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
         }
-        {
+        if (bwd_state_side_tc_ok(sizeof(TIn) == 2, dk, dv)) {
+            e = launch_bwd_gate_tc(qq, kk, la, (pro & KDA_PROLOGUE_GATE_BF16) != 0, beta, hdr, off, cu, Tseq, N, H,
+                                   Hk, max_chunks, scr, dq, dk_out, dla, (grouped || l2norm) ? dq_acc : nullptr,
+                                   (grouped || l2norm) ? dk_acc : nullptr, stream);
+            if (e != cudaSuccess) return e;
+        } else {
             LaunchScope ls("bwd_gate", stream);
             bwd_gate_kernel<TIn><<<dim3(max_chunks, H, dk / kBwdCT), kSimtThreads, smG, stream>>>(
                 qq, kk, la, beta, hdr, off, cu, Tseq, N, H, Hk, pro & KDA_PROLOGUE_GATE_BF16, dk, dv, scr, (TIn*)dq,

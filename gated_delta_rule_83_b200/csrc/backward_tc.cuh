@@ -415,6 +415,369 @@ inline cudaError_t launch_bwd_do_terms_tc(const void* dout, const WsHeader* hdr,
     return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------------------------------------
+// The input side's second half (per (chunk, head, 64-channel half)): dq, dk and dlog_alpha
+// through the gated products P = Qf Kb^T, At = Kf Kb^T and the gating (bwd_gate_kernel computes the
+// same on CUDA cores).  The five products, each M = 64 token rows, N = 64 channels, K = 64 tokens,
+//     rowP = dP Kb,  rowA = dAt Kb,  col = dP^T Qf + dAt^T Kf,  dkt = N^T dW,
+// are tcgen05 MMAs with split-bf16 operands (hi*hi + hi*lo + lo*hi).  dP, dAt and N are stored once as
+// row-major tiles: K-major for the first two products and read MN-major (the same bytes) for the
+// transposed ones.  A 32-channel tile whose in-chunk gate spread exceeds kFactorSpread takes the
+// exact per-element factors on the CUDA cores instead, as the CUDA-core kernel does.
+// ------------------------------------------------------------------------------------------------
+constexpr uint32_t kG_Phi = 0, kG_Plo = 8192, kG_Ahi = 16384, kG_Alo = 24576, kG_Nhi = 32768, kG_Nlo = 40960;
+constexpr uint32_t kG_Kbhi = 49152, kG_Kblo = 57344, kG_Qfhi = 65536, kG_Qflo = 73728, kG_Kfhi = 81920,
+                   kG_Kflo = 90112, kG_Whi = 98304, kG_Wlo = 106496;
+constexpr uint32_t kG_G = 114688;                   // fp32 [64][64]: the cumulative gate g (natural log)
+constexpr uint32_t kG_K = 131072, kG_Q = 139264;    // bf16 [64][64] k and q, row-major
+constexpr uint32_t kG_Misc = 147456;                // beta [64] | ref [64] | quarter totals, lo, hi [4][64] x3 | flags
+constexpr uint32_t kG_Smem = kG_Misc + 4096 + 1024;
+constexpr int kG_LS = 68;                           // row stride (floats) of the dg staging over the B tiles
+static_assert(kG_Smem <= 232448, "gate shared memory");
+
+// One CTA per item (unit, half) = blockIdx.x (a persistent variant that prefetched its next item into
+// L2 measured slower: 4.25 against 3.77 ms per 32K step).
+template <bool LA16>
+__global__ void __launch_bounds__(256, 1)
+bwd_gate_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                   const void* __restrict__ log_alpha, const float* __restrict__ beta, const WsHeader* __restrict__ hdr,
+                   const int* __restrict__ off, const int32_t* __restrict__ cu, int Tseq, int N, int H, int Hk,
+                   const float* __restrict__ scr, __nv_bfloat16* __restrict__ dq, __nv_bfloat16* __restrict__ dk_out,
+                   float* __restrict__ dla, float* __restrict__ dq_acc, float* __restrict__ dk_acc)
+{
+    using namespace tc;
+    constexpr int D = 128;
+    extern __shared__ uint8_t smem_raw[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (hdr->bad) return;
+    const long long items = (long long)hdr->total_chunks * H * 2;
+    if ((long long)blockIdx.x >= items) return;
+    uint8_t* sm = align1024(smem_raw);
+    const uint32_t sb = smem_u32(sm);
+    float* sG = reinterpret_cast<float*>(sm + kG_G);
+    const __nv_bfloat16* sK = reinterpret_cast<const __nv_bfloat16*>(sm + kG_K);
+    const __nv_bfloat16* sQ = reinterpret_cast<const __nv_bfloat16*>(sm + kG_Q);
+    float* sbeta = reinterpret_cast<float*>(sm + kG_Misc);
+    float* sref = sbeta + 64;
+    float* stot = sref + 64;    // [4][64] quarter totals (gate scan), then [4][64] dg partial sums
+    float* slo = stot + 256;    // [4][64]
+    float* shi = slo + 256;     // [4][64]
+    int* swide = reinterpret_cast<int*>(shi + 256);  // [2] one flag per 32-channel tile
+    const uint32_t mbar = smem_u32(swide + 4);
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(swide + 6);
+    float* sAccG = reinterpret_cast<float*>(sm + kG_Kbhi);  // dg staging over the B tiles (after the MMAs)
+    float* sAccL = sAccG + 64 * kG_LS;
+    const size_t scr_unit = bwd_scr_floats(D, D);
+
+    if (tid == 0) {
+        mbar_init(mbar, 1);
+        mbar_fence_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(s_tmem), 256);
+        tmem_relinquish();
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = *s_tmem;
+    // epilogue mapping: row r = 16 qd + lane % 16, channels cb .. cb + 15 (one 32-channel tile hh)
+    const int qd = warp & 3, hh = warp >> 2;
+    const int r = 16 * qd + (lane & 15), cb = 32 * hh + 16 * (lane >> 4);
+    uint32_t ph = 0;
+
+    for (long long it = blockIdx.x; it < items; it += gridDim.x, ph ^= 1u) {
+        const long long uu = it >> 1;
+        const int j = (int)(uu / H), h = (int)(uu - (long long)j * H), c0 = 64 * (int)(it & 1);
+        int n, L;
+        long long t0;
+        locate_chunk(j, off, cu, Tseq, N, n, t0, L);
+        const float* o = scr + (size_t)uu * scr_unit;
+        const float* gN = o;
+        const float* gdAt = o + (size_t)kChunk * D;
+        const float* gdQg = o + 2 * (size_t)kChunk * D;
+        const float* gdW = gdQg + (size_t)kChunk * D;
+        const float* gdKd = gdW + (size_t)kChunk * D;
+        const float* gdP = gdKd + (size_t)kChunk * D;
+        const float* gdGam = gdP + (size_t)kChunk * kChunk;
+        const int hq = h / (H / Hk);  // the q/k head of value head h
+        if (tid == 0) swide[0] = swide[1] = 0;
+        if (tid < 64) sbeta[tid] = tid < L ? beta[(size_t)(t0 + tid) * H + h] : 0.f;
+        // this thread's dQg and dKd, in flight from the start
+        float dqg[16], dkd[16];
+#pragma unroll
+        for (int x = 0; x < 16; x += 4) {
+            const float4 a = *reinterpret_cast<const float4*>(gdQg + (size_t)r * D + c0 + cb + x);
+            const float4 b = *reinterpret_cast<const float4*>(gdKd + (size_t)r * D + c0 + cb + x);
+            dqg[x] = a.x; dqg[x + 1] = a.y; dqg[x + 2] = a.z; dqg[x + 3] = a.w;
+            dkd[x] = b.x; dkd[x + 1] = b.y; dkd[x + 2] = b.z; dkd[x + 3] = b.w;
+        }
+        // loads: task e = tid + 256 m -> row e / 8, 8-element chunk e % 8 of the 64 columns
+        {
+            float fP[2][8], fA[2][8], fN[2][8], fW[2][8], fg[2][8];
+            uint4 kr[2], qr[2];
+#pragma unroll
+            for (int m = 0; m < 2; ++m) {
+                const int e = tid + 256 * m, rr = e >> 3, ch = e & 7;
+                load8(gdP + (size_t)rr * kChunk + 8 * ch, fP[m]);
+                load8(gdAt + (size_t)rr * kChunk + 8 * ch, fA[m]);
+                load8(gN + (size_t)rr * kChunk + 8 * ch, fN[m]);
+                load8(gdW + (size_t)rr * D + c0 + 8 * ch, fW[m]);
+                const bool in = rr < L;
+                const size_t ia = ((size_t)(t0 + (in ? rr : 0)) * H + h) * D + c0 + 8 * ch;
+                if (LA16) load8(reinterpret_cast<const __nv_bfloat16*>(log_alpha) + ia, fg[m]);
+                else load8(reinterpret_cast<const float*>(log_alpha) + ia, fg[m]);
+                if (!in)
+#pragma unroll
+                    for (int x = 0; x < 8; ++x) fg[m][x] = 0.f;  // rows past the chunk's end add nothing
+                const size_t iq = ((size_t)(t0 + (in ? rr : 0)) * Hk + hq) * D + c0 + 8 * ch;
+                kr[m] = in ? *reinterpret_cast<const uint4*>(k + iq) : make_uint4(0, 0, 0, 0);
+                qr[m] = in ? *reinterpret_cast<const uint4*>(q + iq) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int m = 0; m < 2; ++m) {
+                const int e = tid + 256 * m, rr = e >> 3, ch = e & 7;
+                const uint32_t so = sw128_chunk_off(rr, ch, 64);
+                uint4 hi, lo;
+                split8(fP[m], hi, lo);
+                *reinterpret_cast<uint4*>(sm + kG_Phi + so) = hi;
+                *reinterpret_cast<uint4*>(sm + kG_Plo + so) = lo;
+                split8(fA[m], hi, lo);
+                *reinterpret_cast<uint4*>(sm + kG_Ahi + so) = hi;
+                *reinterpret_cast<uint4*>(sm + kG_Alo + so) = lo;
+                split8(fN[m], hi, lo);
+                *reinterpret_cast<uint4*>(sm + kG_Nhi + so) = hi;
+                *reinterpret_cast<uint4*>(sm + kG_Nlo + so) = lo;
+                split8(fW[m], hi, lo);
+                *reinterpret_cast<uint4*>(sm + kG_Whi + so) = hi;
+                *reinterpret_cast<uint4*>(sm + kG_Wlo + so) = lo;
+                *reinterpret_cast<float4*>(sG + rr * 64 + 8 * ch) = make_float4(fg[m][0], fg[m][1], fg[m][2], fg[m][3]);
+                *reinterpret_cast<float4*>(sG + rr * 64 + 8 * ch + 4) = make_float4(fg[m][4], fg[m][5], fg[m][6], fg[m][7]);
+                *reinterpret_cast<uint4*>(sm + kG_K + (rr * 64 + 8 * ch) * 2) = kr[m];
+                *reinterpret_cast<uint4*>(sm + kG_Q + (rr * 64 + 8 * ch) * 2) = qr[m];
+            }
+        }
+        __syncthreads();
+        // cumulative gate per channel: thread (channel c, quarter qt) scans rows 16 qt .. 16 qt + 15, then
+        // adds the totals of the quarters before it; the reference is the centre of [min, max] over the
+        // chunk (the chunk start g = 0 included), as in the CUDA-core kernel
+        {
+            const int c = tid & 63, qt = tid >> 6;
+            float gv[16], acc = 0.f;
+#pragma unroll
+            for (int x = 0; x < 16; ++x) {
+                acc += sG[(16 * qt + x) * 64 + c];
+                gv[x] = acc;
+            }
+            stot[qt * 64 + c] = acc;
+            __syncthreads();
+            float carry = 0.f;
+            for (int p2 = 0; p2 < qt; ++p2) carry += stot[p2 * 64 + c];
+            float lo = qt == 0 ? 0.f : carry, hi = lo;
+#pragma unroll
+            for (int x = 0; x < 16; ++x) {
+                gv[x] += carry;
+                lo = fminf(lo, gv[x]);
+                hi = fmaxf(hi, gv[x]);
+                sG[(16 * qt + x) * 64 + c] = gv[x];
+            }
+            slo[qt * 64 + c] = lo;
+            shi[qt * 64 + c] = hi;
+            __syncthreads();
+            if (tid < 64) {
+                lo = fminf(fminf(slo[c], slo[64 + c]), fminf(slo[128 + c], slo[192 + c]));
+                hi = fmaxf(fmaxf(shi[c], shi[64 + c]), fmaxf(shi[128 + c], shi[192 + c]));
+                sref[c] = 0.5f * (lo + hi);
+                if (!(hi - lo <= kFactorSpread)) atomicOr(&swide[c >> 5], 1);
+            }
+            __syncthreads();
+        }
+        // Kf = k e^{g - ref}, Kb = k e^{ref - g}, Qf = q e^{g - ref} (zero in a wide tile: unused there)
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+            const int e = tid + 256 * m, a = e >> 3, ch = e & 7;
+            const bool wide = swide[ch >> 2] != 0;
+            float kf[8], kb[8], qf[8];
+#pragma unroll
+            for (int x = 0; x < 8; ++x) {
+                const int c = 8 * ch + x;
+                const float xx = sG[a * 64 + c] - sref[c];
+                const float ex = wide ? 0.f : fast_exp(xx), emx = wide ? 0.f : fast_exp(-xx);
+                const float kv = __bfloat162float(sK[a * 64 + c]), qv = __bfloat162float(sQ[a * 64 + c]);
+                kf[x] = kv * ex;
+                kb[x] = kv * emx;
+                qf[x] = qv * ex;
+            }
+            const uint32_t so = sw128_chunk_off(a, ch, 64);
+            uint4 hi, lo;
+            split8(kb, hi, lo);
+            *reinterpret_cast<uint4*>(sm + kG_Kbhi + so) = hi;
+            *reinterpret_cast<uint4*>(sm + kG_Kblo + so) = lo;
+            split8(qf, hi, lo);
+            *reinterpret_cast<uint4*>(sm + kG_Qfhi + so) = hi;
+            *reinterpret_cast<uint4*>(sm + kG_Qflo + so) = lo;
+            split8(kf, hi, lo);
+            *reinterpret_cast<uint4*>(sm + kG_Kfhi + so) = hi;
+            *reinterpret_cast<uint4*>(sm + kG_Kflo + so) = lo;
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+        fence_after_sync();
+        if (tid == 0) {
+            const uint32_t idK = idesc_bf16(64, 64, false, true), idT = idesc_bf16(64, 64, true, true);
+            // three split terms of one product: (A_hi, B_hi), (A_hi, B_lo), (A_lo, B_hi)
+            auto prod = [&](uint32_t d, uint32_t ahi, uint32_t alo, bool amn, uint32_t bhi, uint32_t blo, uint32_t id,
+                            bool first) {
+                const uint32_t as[3] = {ahi, ahi, alo}, bs[3] = {bhi, blo, bhi};
+#pragma unroll
+                for (int t = 0; t < 3; ++t)
+#pragma unroll
+                    for (int k0 = 0; k0 < kChunk; k0 += 16)
+                        mma_bf16(tmem + d, amn ? desc_mnmajor(sb + as[t], 64, k0) : desc_kmajor(sb + as[t], 64, k0),
+                                 desc_mnmajor(sb + bs[t], 64, k0), id, (first && t == 0 && k0 == 0) ? 0u : 1u);
+            };
+            prod(0, kG_Phi, kG_Plo, false, kG_Kbhi, kG_Kblo, idK, true);     // rowP = dP Kb
+            prod(64, kG_Ahi, kG_Alo, false, kG_Kbhi, kG_Kblo, idK, true);    // rowA = dAt Kb
+            prod(128, kG_Phi, kG_Plo, true, kG_Qfhi, kG_Qflo, idT, true);    // col = dP^T Qf
+            prod(128, kG_Ahi, kG_Alo, true, kG_Kfhi, kG_Kflo, idT, false);   //     + dAt^T Kf
+            prod(192, kG_Nhi, kG_Nlo, true, kG_Whi, kG_Wlo, idT, true);      // dkt = N^T dW
+            mma_commit(mbar);
+        }
+        const bool ok = mbar_wait(mbar, ph);
+        fence_after_sync();
+        const bool wide = swide[hh] != 0;
+        float rowP[16], rowA[16], col[16], dkt[16];
+        {
+            const uint32_t tl = tmem + ((uint32_t)(32 * qd) << 16) + 32 * hh;
+            tmem_ld16_pair<16>(tl, rowP);
+            tmem_ld16_pair<16>(tl + 64, rowA);
+            tmem_ld16_pair<16>(tl + 128, col);
+            tmem_ld16_pair<16>(tl + 192, dkt);
+            tmem_wait_ld();
+        }
+        if (wide) {  // exact per-element factors e^{g_r - g_i} (never above 1), dP and dAt as hi + lo
+#pragma unroll
+            for (int x = 0; x < 16; ++x) {
+                const int c = cb + x;
+                const float gr = sG[r * 64 + c];
+                float p = 0.f, a = 0.f, cl = 0.f;
+                for (int i = 0; i <= r; ++i) {
+                    const float ke = __bfloat162float(sK[i * 64 + c]) * fast_exp(gr - sG[i * 64 + c]);
+                    const uint32_t oi = sw128_off(r, i, 64);
+                    const float dpv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + kG_Phi + oi)) +
+                                      __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + kG_Plo + oi));
+                    const float dav = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + kG_Ahi + oi)) +
+                                      __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + kG_Alo + oi));
+                    p = fmaf(dpv, ke, p);
+                    a = fmaf(dav, ke, a);
+                }
+                for (int i = r; i < kChunk; ++i) {
+                    const uint32_t oi = sw128_off(i, r, 64);
+                    const float dpv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + kG_Phi + oi)) +
+                                      __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + kG_Plo + oi));
+                    const float dav = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + kG_Ahi + oi)) +
+                                      __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + kG_Alo + oi));
+                    cl = fmaf(fmaf(dpv, __bfloat162float(sQ[i * 64 + c]), dav * __bfloat162float(sK[i * 64 + c])),
+                              fast_exp(sG[i * 64 + c] - gr), cl);
+                }
+                rowP[x] = p;
+                rowA[x] = a;
+                col[x] = cl;
+            }
+        }
+        // the element-wise gradients (as in the CUDA-core kernel); dg staged over the B tiles (the MMAs
+        // that read them are complete) for the reverse cumulative sum
+        {
+            float vq[16], vk[16];
+#pragma unroll
+            for (int x = 0; x < 16; ++x) {
+                const int c = cb + x;
+                const float g = sG[r * 64 + c], gl = sG[63 * 64 + c];
+                float rp = rowP[x], ra = rowA[x], cl = col[x];
+                if (!wide) {
+                    const float xx = g - sref[c];
+                    const float ex = fast_exp(xx);
+                    rp *= ex;
+                    ra *= ex;
+                    cl *= fast_exp(-xx);
+                }
+                const float kt = dkt[x] * sbeta[r];
+                const float eg = fast_exp(g), egl = fast_exp(gl - g);
+                const float qv = __bfloat162float(sQ[r * 64 + c]), kv = __bfloat162float(sK[r * 64 + c]);
+                vq[x] = rp + dqg[x] * eg;
+                vk[x] = ra + cl + kt * eg + dkd[x] * egl;
+                sAccG[r * kG_LS + c] = qv * rp + kv * ra - kv * cl + (dqg[x] * qv + kt * kv) * eg - dkd[x] * kv * egl;
+                sAccL[r * kG_LS + c] = dkd[x] * kv * egl;  // chunk-end term of g_last, summed below
+            }
+            if (r < L && ok) {
+                const size_t oi = ((size_t)(t0 + r) * H + h) * D + c0 + cb;
+                if (dq_acc) {  // grouped heads or the q/k norm: per value head, summed afterwards
+#pragma unroll
+                    for (int x = 0; x < 16; x += 4) {
+                        *reinterpret_cast<float4*>(dq_acc + oi + x) = make_float4(vq[x], vq[x + 1], vq[x + 2], vq[x + 3]);
+                        *reinterpret_cast<float4*>(dk_acc + oi + x) = make_float4(vk[x], vk[x + 1], vk[x + 2], vk[x + 3]);
+                    }
+                } else {
+#pragma unroll
+                    for (int x = 0; x < 16; x += 8) {
+                        *reinterpret_cast<uint4*>(dq + oi + x) = pack8(vq + x);
+                        *reinterpret_cast<uint4*>(dk_out + oi + x) = pack8(vk + x);
+                    }
+                }
+            }
+        }
+        fence_before_sync();
+        __syncthreads();
+        // dlog_alpha = reverse cumulative sum of dg (plus the g_last terms), channel c = tid % 64 over the
+        // row quarter qt = tid / 64: quarter sums first, then each quarter's suffix
+        {
+            const int c = tid & 63, qt = tid >> 6;
+            float sl = 0.f, sg = 0.f;
+#pragma unroll
+            for (int x = 0; x < 16; ++x) {
+                sl += sAccL[(16 * qt + x) * kG_LS + c];
+                sg += sAccG[(16 * qt + x) * kG_LS + c];
+            }
+            slo[qt * 64 + c] = sl;  // the scan's scratch is free again
+            shi[qt * 64 + c] = sg;
+            __syncthreads();
+            float acc = gdGam[c0 + c] * fast_exp(sG[63 * 64 + c]);
+            for (int p2 = 0; p2 < 4; ++p2) acc += slo[p2 * 64 + c];
+            for (int p2 = qt + 1; p2 < 4; ++p2) acc += shi[p2 * 64 + c];
+            if (ok)
+                for (int x = 15; x >= 0; --x) {
+                    const int rr = 16 * qt + x;
+                    acc += sAccG[rr * kG_LS + c];
+                    if (rr < L) dla[((size_t)(t0 + rr) * H + h) * D + c0 + c] = acc;
+                }
+        }
+        fence_before_sync();
+        __syncthreads();  // the tiles, the staging and TMEM free for the next item
+        fence_after_sync();
+    }
+    if (warp == 0) tmem_dealloc(tmem, 256);
+}
+
+inline cudaError_t launch_bwd_gate_tc(const void* q, const void* k, const void* la, bool la16, const float* beta,
+                                      const WsHeader* hdr, const int* off, const int32_t* cu, int Tseq, int N, int H,
+                                      int Hk, int max_chunks, const float* scr, void* dq, void* dk_out, float* dla,
+                                      float* dq_acc, float* dk_acc, cudaStream_t stream)
+{
+    auto* kern = la16 ? bwd_gate_tc_kernel<true> : bwd_gate_tc_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kG_Smem);
+    if (e != cudaSuccess) return e;
+    const long long items = (long long)max_chunks * H * 2;
+    if (items == 0) return cudaSuccess;
+    if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
+    const unsigned grid = (unsigned)items;
+    LaunchScope ls("bwd_gate_tc", stream);
+    kern<<<grid, 256, kG_Smem, stream>>>(
+        (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, la, beta, hdr, off, cu, Tseq, N, H, Hk, scr,
+        (__nv_bfloat16*)dq, (__nv_bfloat16*)dk_out, dla, dq_acc, dk_acc);
+    return cudaGetLastError();
+}
+
 inline bool bwd_state_side_tc_ok(bool bf16, int dk, int dv) { return kTcPathReady && bf16 && dk == 128 && dv == 128; }
 
 inline cudaError_t launch_bwd_state_side_tc(const void* dout, const WsHeader* hdr, const int* off, const int32_t* cu,

@@ -101,6 +101,22 @@ def test_backward_strong_decay_exact_factors():
     run_and_compare(inp, "f32")
 
 
+@pytest.mark.parametrize("channels", ["all", "first_tile"])
+def test_backward_strong_decay_exact_factors_bf16(channels):
+    """The same on the bf16 d = 128 path, whose input-side kernel runs on the tensor cores: a
+    32-channel tile with a wide gate spread takes the exact per-element factors; with only the first
+    tile's channels decaying fast, the other tiles keep the factorised form in the same unit."""
+    w = synth.Workload("bwdw16", "prefill", 1, 140, 2, 128, 128, "bf16", 38, s0_std=0.5)
+    inp = synth.prefill_inputs(w)
+    g = torch.Generator().manual_seed(39)
+    strong = -8.0 * torch.rand(inp["log_alpha"].shape, generator=g)
+    if channels == "all":
+        inp["log_alpha"] = strong
+    else:
+        inp["log_alpha"][..., :32] = strong[..., :32]
+    run_and_compare(inp, "bf16")
+
+
 def test_backward_bf16_gates():
     """log_alpha passed as bf16 (KDA_PROLOGUE_GATE_BF16): same result as the fp32 call on the
     widened values."""

@@ -513,10 +513,19 @@ __device__ __forceinline__ void bwd_load_scr_tile(const float* __restrict__ x, i
     }
 }
 
+// Step 4a on the tensor cores (backward_tc.cuh; bf16 inputs, dk = dv = 128): At (strictly lower,
+// factorised tiles only) and dT (lower, inclusive) into sAt and sM, with the exact products of the
+// wide tiles added into accA at the thread's (tr, tc) elements; scratch = the kernel's shared memory
+// below sb
+__device__ void bwd_ut_step4a_tc(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+                                 const void* __restrict__ log_alpha, bool la16, long long t0, int L, int H, int Hk,
+                                 int h, const float* __restrict__ gdW, const float* __restrict__ gdU, float* smem,
+                                 float* sAt, float* sM, float (&accA)[4][4]);
+
 // Step 4, first half (one CTA per (chunk, head)): At and dT over all channel and value tiles, the
 // UT transform backwards (N, dbeta, dM -> dAt) and dV.  N and dAt go to the unit's scratch (over U
 // and dU, both dead by then) for the second half.
-template <typename TIn>
+template <typename TIn, bool TC>
 __global__ void __launch_bounds__(kSimtThreads, 2)
 bwd_ut_kernel(const TIn* __restrict__ k, const TIn* __restrict__ v, const void* __restrict__ log_alpha,
               const float* __restrict__ beta, const WsHeader* __restrict__ hdr, const int* __restrict__ off,
@@ -558,56 +567,61 @@ bwd_ut_kernel(const TIn* __restrict__ k, const TIn* __restrict__ v, const void* 
 
     // ---- step 4a: At and dT = dW Kt^T + dU V^T, accumulated in registers over tiles
     float accA[4][4] = {}, accT[4][4] = {};
-    for (int c0 = 0; c0 < dk; c0 += kBwdCT) {
-        __syncthreads();
-        if (tid == 0) s_wide = 0;
-        __syncthreads();
-        bwd_load_tile(k, t0, L, Hk, h / (H / Hk), dk, c0, tk);  // the q/k head of value head h
-        bwd_gate_tile(log_alpha, la16, t0, L, H, h, dk, c0, tg, tref, &s_wide);
-        bwd_load_scr_tile(gdW, dk, c0, tD);
-        __syncthreads();
-        const bool wide = s_wide != 0;
-        for (int e = tid; e < kChunk * kBwdCT; e += kSimtThreads) {
-            const int r = e / kBwdCT, cc = e % kBwdCT;
-            const float g = tg[r * LT + cc], x = g - tref[cc], kv = tk[r * LT + cc];
-            tA[r * LT + cc] = wide ? 0.f : kv * fast_exp(x);   // Kf
-            tB[r * LT + cc] = wide ? 0.f : kv * fast_exp(-x);  // Kb
-            tC[r * LT + cc] = kv * fast_exp(g);                // Kt
-        }
-        __syncthreads();
-        if (!wide) {
-            mm_acc<4, 4>(accA, tA, LT, 1, tB, 1, LT, kBwdCT, tr, tc);
-        } else {
+    if constexpr (TC) {
+        bwd_ut_step4a_tc(reinterpret_cast<const __nv_bfloat16*>(k), reinterpret_cast<const __nv_bfloat16*>(v),
+                         log_alpha, la16, t0, L, H, Hk, h, gdW, gdU, smem, sAt, sM, accA);
+    } else {
+        for (int c0 = 0; c0 < dk; c0 += kBwdCT) {
+            __syncthreads();
+            if (tid == 0) s_wide = 0;
+            __syncthreads();
+            bwd_load_tile(k, t0, L, Hk, h / (H / Hk), dk, c0, tk);  // the q/k head of value head h
+            bwd_gate_tile(log_alpha, la16, t0, L, H, h, dk, c0, tg, tref, &s_wide);
+            bwd_load_scr_tile(gdW, dk, c0, tD);
+            __syncthreads();
+            const bool wide = s_wide != 0;
+            for (int e = tid; e < kChunk * kBwdCT; e += kSimtThreads) {
+                const int r = e / kBwdCT, cc = e % kBwdCT;
+                const float g = tg[r * LT + cc], x = g - tref[cc], kv = tk[r * LT + cc];
+                tA[r * LT + cc] = wide ? 0.f : kv * fast_exp(x);   // Kf
+                tB[r * LT + cc] = wide ? 0.f : kv * fast_exp(-x);  // Kb
+                tC[r * LT + cc] = kv * fast_exp(g);                // Kt
+            }
+            __syncthreads();
+            if (!wide) {
+                mm_acc<4, 4>(accA, tA, LT, 1, tB, 1, LT, kBwdCT, tr, tc);
+            } else {
 #pragma unroll
-            for (int a = 0; a < 4; ++a)
+                for (int a = 0; a < 4; ++a)
 #pragma unroll
-                for (int b = 0; b < 4; ++b) {
-                    const int r = tr + 16 * a, i = tc + 16 * b;
-                    if (i >= r) continue;
-                    float x = 0.f;
-                    for (int cc = 0; cc < kBwdCT; ++cc)
-                        x = fmaf(tk[r * LT + cc] * tk[i * LT + cc], fast_exp(tg[r * LT + cc] - tg[i * LT + cc]), x);
-                    accA[a][b] += x;
-                }
+                    for (int b = 0; b < 4; ++b) {
+                        const int r = tr + 16 * a, i = tc + 16 * b;
+                        if (i >= r) continue;
+                        float x = 0.f;
+                        for (int cc = 0; cc < kBwdCT; ++cc)
+                            x = fmaf(tk[r * LT + cc] * tk[i * LT + cc], fast_exp(tg[r * LT + cc] - tg[i * LT + cc]), x);
+                        accA[a][b] += x;
+                    }
+            }
+            mm_acc<4, 4>(accT, tD, LT, 1, tC, 1, LT, kBwdCT, tr, tc);
         }
-        mm_acc<4, 4>(accT, tD, LT, 1, tC, 1, LT, kBwdCT, tr, tc);
+        for (int c0 = 0; c0 < dv; c0 += kBwdCT) {
+            __syncthreads();
+            bwd_load_tile(v, t0, L, H, h, dv, c0, tk);
+            bwd_load_scr_tile(gdU, dv, c0, tD);
+            __syncthreads();
+            mm_acc<4, 4>(accT, tD, LT, 1, tk, 1, LT, kBwdCT, tr, tc);
+        }
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const int r = tr + 16 * a, i = tc + 16 * b;
+                sAt[r * L64 + i] = (i < r) ? accA[a][b] : 0.f;
+                sM[r * L64 + i] = (i <= r) ? accT[a][b] : 0.f;
+            }
+        __syncthreads();
     }
-    for (int c0 = 0; c0 < dv; c0 += kBwdCT) {
-        __syncthreads();
-        bwd_load_tile(v, t0, L, H, h, dv, c0, tk);
-        bwd_load_scr_tile(gdU, dv, c0, tD);
-        __syncthreads();
-        mm_acc<4, 4>(accT, tD, LT, 1, tk, 1, LT, kBwdCT, tr, tc);
-    }
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-            const int r = tr + 16 * a, i = tc + 16 * b;
-            sAt[r * L64 + i] = (i < r) ? accA[a][b] : 0.f;
-            sM[r * L64 + i] = (i <= r) ? accT[a][b] : 0.f;
-        }
-    __syncthreads();
 
     // ---- step 4b: the UT transform backwards
     // N = (I + Diag(beta) At)^{-1}: Diag(beta) At copied into N, then inverted in place (the tiles
@@ -1079,7 +1093,10 @@ cudaError_t launch_simt_backward(const void* q, const void* k, const void* v, co
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(bwd_state_side_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smS);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(bwd_ut_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smU);
+        e = cudaFuncSetAttribute(bwd_ut_kernel<TIn, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smU);
+    if (e == cudaSuccess && sizeof(TIn) == 2)
+        e = cudaFuncSetAttribute(bwd_ut_kernel<TIn, sizeof(TIn) == 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smU);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(bwd_gate_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smG);
     if (e != cudaSuccess) return e;
@@ -1109,8 +1126,10 @@ cudaError_t launch_simt_backward(const void* q, const void* k, const void* v, co
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
         }
         {
-            LaunchScope ls("bwd_ut", stream);
-            bwd_ut_kernel<TIn><<<dim3(max_chunks, H), kSimtThreads, smU, stream>>>(
+            const bool tc = bwd_state_side_tc_ok(sizeof(TIn) == 2, dk, dv);
+            LaunchScope ls(tc ? "bwd_ut_tc" : "bwd_ut", stream);
+            auto* kut = tc ? bwd_ut_kernel<TIn, sizeof(TIn) == 2> : bwd_ut_kernel<TIn, false>;
+            kut<<<dim3(max_chunks, H), kSimtThreads, smU, stream>>>(
                 kk, vv, la, beta, hdr, off, cu, Tseq, N, H, Hk, pro & KDA_PROLOGUE_GATE_BF16, dk, dv, scr,
                 (TIn*)dv_out, dbeta);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;

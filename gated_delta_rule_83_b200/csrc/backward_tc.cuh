@@ -778,6 +778,263 @@ inline cudaError_t launch_bwd_gate_tc(const void* q, const void* k, const void* 
     return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------------------------------------
+// Step 4a of the input side's first half on the tensor cores (called by bwd_ut_kernel<bf16, true>):
+//     At = strict_lower(Kf Kb^T),   dT = lower_incl(dW Kt^T + dU V^T)
+// over two 64-channel blocks of the key dimension and two of the value dimension, accumulated in
+// TMEM by split-bf16 MMAs (M = N = K = 64 per block).  The scratch is the kernel's own shared memory
+// below its beta array, which the UT step reuses afterwards for its fp32 matrices.  A 32-channel
+// tile with a wide gate spread contributes to At through exact per-element factors on the CUDA cores
+// (accA, at the thread's (tr + 16 a, tc + 16 b) elements), as in the CUDA-core loop.
+// ------------------------------------------------------------------------------------------------
+constexpr uint32_t kU_Kfhi = 0, kU_Kflo = 8192, kU_Kbhi = 16384, kU_Kblo = 24576;  // K-major [token][64 ch]
+constexpr uint32_t kU_Ahi = 32768, kU_Alo = 40960;  // dW or dU block [token r][64]
+constexpr uint32_t kU_Bhi = 49152, kU_Blo = 57344;  // Kt or V block [token i][64]
+constexpr uint32_t kU_G = 65536;                    // fp32 [64][64] cumulative gate of the block
+constexpr uint32_t kU_K = 81920;                    // bf16 [64][64] k of the block
+constexpr uint32_t kU_S = 90112;                    // scan scratch: totals, lo, hi [4][64] x 3 | ref [64] | wide [2]
+constexpr uint32_t kU_End = kU_S + 3072 + 256 + 16;
+static_assert(kU_End + 1024 <= sizeof(float) * (3 * kChunk * kBwdL64 + 6 * kChunk * kBwdLT),
+              "step 4a scratch must fit below bwd_ut_kernel's beta array");
+
+__device__ void bwd_ut_step4a_tc(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+                                 const void* __restrict__ log_alpha, bool la16, long long t0, int L, int H, int Hk,
+                                 int h, const float* __restrict__ gdW, const float* __restrict__ gdU, float* smem,
+                                 float* sAt, float* sM, float (&accA)[4][4])
+{
+    using namespace tc;
+    constexpr int D = 128, L64 = kBwdL64;
+    __shared__ uint64_t s_mbar;
+    __shared__ uint32_t s_tm;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, tr = tid >> 4, tcc = tid & 15;
+    uint8_t* ab = align1024(reinterpret_cast<uint8_t*>(smem));
+    const uint32_t sbs = smem_u32(ab);
+    const uint32_t mbar = smem_u32(&s_mbar);
+    float* sG = reinterpret_cast<float*>(ab + kU_G);
+    __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(ab + kU_K);
+    float* stot = reinterpret_cast<float*>(ab + kU_S);
+    float* slo = stot + 256;
+    float* shi = slo + 256;
+    float* sref = shi + 256;
+    int* swide = reinterpret_cast<int*>(sref + 64);
+    const int hq = h / (H / Hk);  // the q/k head of value head h
+    const uint4 z4 = make_uint4(0, 0, 0, 0);
+
+    __syncthreads();  // the caller is done with this memory
+    if (tid == 0) {
+        mbar_init(mbar, 1);
+        mbar_fence_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(&s_tm), 128);
+        tmem_relinquish();
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = s_tm;  // At in columns 0..63, dT in 64..127 (M = 64 accumulators)
+    const uint32_t idK = idesc_bf16(64, 64, false, false);
+    uint32_t ph = 0;
+    bool ok = true;
+
+    // key-channel blocks: At += Kf Kb^T, dT += dW Kt^T
+    for (int blk = 0; blk < 2; ++blk, ph ^= 1u) {
+        const int c0 = 64 * blk;
+        if (tid == 0) swide[0] = swide[1] = 0;
+        {
+            float fw[2][8], fg[2][8];
+            uint4 kr[2];
+#pragma unroll
+            for (int m = 0; m < 2; ++m) {
+                const int e = tid + 256 * m, rr = e >> 3, ch = e & 7;
+                load8(gdW + (size_t)rr * D + c0 + 8 * ch, fw[m]);
+                const bool in = rr < L;
+                const size_t ia = ((size_t)(t0 + (in ? rr : 0)) * H + h) * D + c0 + 8 * ch;
+                if (la16) load8(reinterpret_cast<const __nv_bfloat16*>(log_alpha) + ia, fg[m]);
+                else load8(reinterpret_cast<const float*>(log_alpha) + ia, fg[m]);
+                if (!in)
+#pragma unroll
+                    for (int x = 0; x < 8; ++x) fg[m][x] = 0.f;  // rows past the chunk's end add nothing
+                kr[m] = in ? *reinterpret_cast<const uint4*>(k + ((size_t)(t0 + rr) * Hk + hq) * D + c0 + 8 * ch) : z4;
+            }
+#pragma unroll
+            for (int m = 0; m < 2; ++m) {
+                const int e = tid + 256 * m, rr = e >> 3, ch = e & 7;
+                uint4 hi, lo;
+                split8(fw[m], hi, lo);
+                *reinterpret_cast<uint4*>(ab + kU_Ahi + sw128_chunk_off(rr, ch, 64)) = hi;
+                *reinterpret_cast<uint4*>(ab + kU_Alo + sw128_chunk_off(rr, ch, 64)) = lo;
+                *reinterpret_cast<float4*>(sG + rr * 64 + 8 * ch) = make_float4(fg[m][0], fg[m][1], fg[m][2], fg[m][3]);
+                *reinterpret_cast<float4*>(sG + rr * 64 + 8 * ch + 4) = make_float4(fg[m][4], fg[m][5], fg[m][6], fg[m][7]);
+                *reinterpret_cast<uint4*>(sK + rr * 64 + 8 * ch) = kr[m];
+            }
+        }
+        __syncthreads();
+        {  // cumulative gate: thread (channel c, quarter qt), as in the gate kernel
+            const int c = tid & 63, qt = tid >> 6;
+            float gv[16], acc = 0.f;
+#pragma unroll
+            for (int x = 0; x < 16; ++x) {
+                acc += sG[(16 * qt + x) * 64 + c];
+                gv[x] = acc;
+            }
+            stot[qt * 64 + c] = acc;
+            __syncthreads();
+            float carry = 0.f;
+            for (int p2 = 0; p2 < qt; ++p2) carry += stot[p2 * 64 + c];
+            float lo = qt == 0 ? 0.f : carry, hi = lo;
+#pragma unroll
+            for (int x = 0; x < 16; ++x) {
+                gv[x] += carry;
+                lo = fminf(lo, gv[x]);
+                hi = fmaxf(hi, gv[x]);
+                sG[(16 * qt + x) * 64 + c] = gv[x];
+            }
+            slo[qt * 64 + c] = lo;
+            shi[qt * 64 + c] = hi;
+            __syncthreads();
+            if (tid < 64) {
+                lo = fminf(fminf(slo[c], slo[64 + c]), fminf(slo[128 + c], slo[192 + c]));
+                hi = fmaxf(fmaxf(shi[c], shi[64 + c]), fmaxf(shi[128 + c], shi[192 + c]));
+                sref[c] = 0.5f * (lo + hi);
+                if (!(hi - lo <= kFactorSpread)) atomicOr(&swide[c >> 5], 1);
+            }
+            __syncthreads();
+        }
+        // Kf = k e^{g - ref}, Kb = k e^{ref - g} (zero in a wide tile), Kt = k e^{g}
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+            const int e = tid + 256 * m, a = e >> 3, ch = e & 7;
+            const bool wide = swide[ch >> 2] != 0;
+            float kf[8], kb[8], kt[8];
+#pragma unroll
+            for (int x = 0; x < 8; ++x) {
+                const int c = 8 * ch + x;
+                const float g = sG[a * 64 + c], xx = g - sref[c], kv = __bfloat162float(sK[a * 64 + c]);
+                kf[x] = wide ? 0.f : kv * fast_exp(xx);
+                kb[x] = wide ? 0.f : kv * fast_exp(-xx);
+                kt[x] = kv * fast_exp(g);
+            }
+            const uint32_t so = sw128_chunk_off(a, ch, 64);
+            uint4 hi, lo;
+            split8(kf, hi, lo);
+            *reinterpret_cast<uint4*>(ab + kU_Kfhi + so) = hi;
+            *reinterpret_cast<uint4*>(ab + kU_Kflo + so) = lo;
+            split8(kb, hi, lo);
+            *reinterpret_cast<uint4*>(ab + kU_Kbhi + so) = hi;
+            *reinterpret_cast<uint4*>(ab + kU_Kblo + so) = lo;
+            split8(kt, hi, lo);
+            *reinterpret_cast<uint4*>(ab + kU_Bhi + so) = hi;
+            *reinterpret_cast<uint4*>(ab + kU_Blo + so) = lo;
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+        fence_after_sync();
+        if (tid == 0) {
+            const uint32_t fa[3] = {kU_Kfhi, kU_Kfhi, kU_Kflo}, fb[3] = {kU_Kbhi, kU_Kblo, kU_Kbhi};
+            const uint32_t wa[3] = {kU_Ahi, kU_Ahi, kU_Alo}, wb[3] = {kU_Bhi, kU_Blo, kU_Bhi};
+#pragma unroll
+            for (int t = 0; t < 3; ++t)
+#pragma unroll
+                for (int k0 = 0; k0 < 64; k0 += 16) {
+                    const uint32_t acc = (blk > 0 || t > 0 || k0 > 0) ? 1u : 0u;
+                    mma_bf16(tmem, desc_kmajor(sbs + fa[t], 64, k0), desc_kmajor(sbs + fb[t], 64, k0), idK, acc);
+                    mma_bf16(tmem + 64, desc_kmajor(sbs + wa[t], 64, k0), desc_kmajor(sbs + wb[t], 64, k0), idK, acc);
+                }
+            mma_commit(mbar);
+        }
+        // a wide tile's At terms, exactly: sum over its channels of k_r k_i e^{g_r - g_i} (i < r)
+#pragma unroll 1
+        for (int w = 0; w < 2; ++w) {
+            if (!swide[w]) continue;
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    const int r = tr + 16 * a, i = tcc + 16 * b;
+                    if (i >= r) continue;
+                    float x = 0.f;
+                    for (int cc = 32 * w; cc < 32 * w + 32; ++cc)
+                        x = fmaf(__bfloat162float(sK[r * 64 + cc]) * __bfloat162float(sK[i * 64 + cc]),
+                                 fast_exp(sG[r * 64 + cc] - sG[i * 64 + cc]), x);
+                    accA[a][b] += x;
+                }
+        }
+        ok = mbar_wait(mbar, ph) && ok;
+        fence_after_sync();
+        __syncthreads();  // the tiles are free for the next block
+    }
+    // value blocks: dT += dU V^T (V is exact in bf16: dU_hi V + dU_lo V)
+    for (int blk = 0; blk < 2; ++blk, ph ^= 1u) {
+        const int c0 = 64 * blk;
+        {
+            float fu[2][8];
+            uint4 vr[2];
+#pragma unroll
+            for (int m = 0; m < 2; ++m) {
+                const int e = tid + 256 * m, rr = e >> 3, ch = e & 7;
+                load8(gdU + (size_t)rr * D + c0 + 8 * ch, fu[m]);
+                vr[m] = rr < L ? *reinterpret_cast<const uint4*>(v + ((size_t)(t0 + rr) * H + h) * D + c0 + 8 * ch) : z4;
+            }
+#pragma unroll
+            for (int m = 0; m < 2; ++m) {
+                const int e = tid + 256 * m, rr = e >> 3, ch = e & 7;
+                const uint32_t so = sw128_chunk_off(rr, ch, 64);
+                uint4 hi, lo;
+                split8(fu[m], hi, lo);
+                *reinterpret_cast<uint4*>(ab + kU_Ahi + so) = hi;
+                *reinterpret_cast<uint4*>(ab + kU_Alo + so) = lo;
+                *reinterpret_cast<uint4*>(ab + kU_Bhi + so) = vr[m];
+            }
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+        fence_after_sync();
+        if (tid == 0) {
+#pragma unroll
+            for (int t = 0; t < 2; ++t)
+#pragma unroll
+                for (int k0 = 0; k0 < 64; k0 += 16)
+                    mma_bf16(tmem + 64, desc_kmajor(sbs + (t ? kU_Alo : kU_Ahi), 64, k0), desc_kmajor(sbs + kU_Bhi, 64, k0),
+                             idK, 1u);
+            mma_commit(mbar);
+        }
+        ok = mbar_wait(mbar, ph) && ok;
+        fence_after_sync();
+        __syncthreads();
+    }
+    // At (strictly lower) and dT (lower, inclusive) from TMEM (M = 64: row 16 q + lane % 16, columns
+    // 32 half + 16 (lane / 16) .. +15), over the dead tiles
+    {
+        const int q = warp & 3, half = warp >> 2;
+        const int r = 16 * q + (lane & 15), cb = 32 * half + 16 * (lane >> 4);
+        const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16) + 32 * half;
+        float va[16], vt[16];
+        tmem_ld16_pair<16>(tl, va);
+        tmem_ld16_pair<16>(tl + 64, vt);
+        tmem_wait_ld();
+#pragma unroll
+        for (int x = 0; x < 16; ++x) {
+            const int i = cb + x;
+            sAt[r * L64 + i] = (i < r && ok) ? va[x] : 0.f;
+            sM[r * L64 + i] = (i <= r && ok) ? vt[x] : 0.f;
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            const int r = tr + 16 * a, i = tcc + 16 * b;
+            if (i < r) sAt[r * L64 + i] += accA[a][b];  // the wide tiles' exact terms (zero elsewhere)
+        }
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 128);
+}
+
 inline bool bwd_state_side_tc_ok(bool bf16, int dk, int dv) { return kTcPathReady && bf16 && dk == 128 && dv == 128; }
 
 inline cudaError_t launch_bwd_state_side_tc(const void* dout, const WsHeader* hdr, const int* off, const int32_t* cu,

@@ -1003,6 +1003,10 @@ cudaError_t launch_bwd_state_side_tc(const void* dout, const WsHeader* hdr, cons
 cudaError_t launch_bwd_do_terms_tc(const void* dout, const WsHeader* hdr, const int* off, const int32_t* cu,
                                    int Tseq, int N, int H, int max_chunks, const float* slots, float* scr,
                                    float* F_chunks, cudaStream_t stream);
+cudaError_t launch_bwd_chains_tc(const float* S0, const float* dS_final, float* dS0, const WsHeader* hdr,
+                                 const int* off, int N, int H, int max_chunks, const float* slots, float* S_chunks,
+                                 float* dSn_chunks, float* scr, const float* F_chunks, bool reverse,
+                                 cudaStream_t stream);
 cudaError_t launch_bwd_gate_tc(const void* q, const void* k, const void* la, bool la16, const float* beta,
                                const WsHeader* hdr, const int* off, const int32_t* cu, int Tseq, int N, int H,
                                int Hk, int max_chunks, const float* scr, void* dq, void* dk_out, float* dla,
@@ -1023,7 +1027,12 @@ cudaError_t launch_bwd_chains(const float* S0, const void* dout, const float* dS
                                  (int)smT);
     if (e != cudaSuccess) return e;
     const dim3 grid(N, H, DV / kSimtNV);
-    {
+    const bool tc = bwd_state_side_tc_ok(sizeof(TIn) == 2, DK, DV);
+    if (tc) {
+        e = launch_bwd_chains_tc(S0, dS_final, dS0, hdr, off, N, H, max_chunks, slots, S_chunks, dSn_chunks, scr,
+                                 F_chunks, false, stream);
+        if (e != cudaSuccess) return e;
+    } else {
         LaunchScope ls("bwd_fwd_states", stream);
         bwd_fwd_chain_kernel<DK><<<grid, kSimtThreads, smF, stream>>>(S0, hdr, off, cu, Tseq, N, H, DV, slots,
                                                                       S_chunks, scr);
@@ -1038,6 +1047,9 @@ cudaError_t launch_bwd_chains(const float* S0, const void* dout, const float* dS
             (const TIn*)dout, hdr, off, cu, Tseq, N, H, slots, scr, F_chunks);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
+    if (tc)
+        return launch_bwd_chains_tc(S0, dS_final, dS0, hdr, off, N, H, max_chunks, slots, S_chunks, dSn_chunks, scr,
+                                    F_chunks, true, stream);
     LaunchScope ls("bwd_dstate", stream);
     bwd_dstate_kernel<DK><<<grid, kSimtThreads, smD, stream>>>(dS_final, dS0, hdr, off, N, H, DV, slots, dSn_chunks,
                                                                scr, F_chunks);

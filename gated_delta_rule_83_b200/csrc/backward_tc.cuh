@@ -1035,7 +1035,291 @@ __device__ void bwd_ut_step4a_tc(const __nv_bfloat16* __restrict__ k, const __nv
     if (warp == 0) tmem_dealloc(tmem, 128);
 }
 
+// ------------------------------------------------------------------------------------------------
+// The two chains of the backward on the tensor cores.  Per (sequence, head, 32-column slice), chunks
+// in order (forward) or in reverse (reverse chain), with the carried matrix Z (the state S, or its
+// cotangent D) fp32 in registers (thread c owns row c):
+//   forward:  X = W S,   U = Uv - X,  S <- Diag(gam) S + Kd^T U          (stores S_c and U)
+//   reverse:  Z = Kd D,  dU = E + Z,  D <- Diag(gam) D + F - W^T dU      (stores D_c and dU)
+// the recurrences of bwd_fwd_chain_kernel and bwd_dstate_kernel.  Both products are split-bf16
+// tcgen05 MMAs (24 + 12 per chunk): W and Kd as bf16 hi/lo images written once per unit by
+// bwd_wk_images_kernel, Z and U split by the compute threads every chunk.  Warp roles as in the
+// forward's phase B: four compute warps, one MMA warp, one copy warp streaming the images through two
+// shared-memory stages.
+// ------------------------------------------------------------------------------------------------
+// the unit's image region inside its scratch (over dQg and dW, which the state side writes later):
+// W hi | W lo | Kd hi | Kd lo, each a 64-row x 128 SW128 tile (two 8 KB atom columns)
+__host__ __device__ inline size_t bwd_wk_image_offset_floats() { return 2 * (size_t)kChunk * 128; }
+constexpr uint32_t kImgW = 0, kImgWlo = 16384, kImgKd = 32768, kImgKdlo = 49152, kImgBytes = 65536;
+
+__global__ void __launch_bounds__(256)
+bwd_wk_images_kernel(const WsHeader* __restrict__ hdr, int H, const float* __restrict__ slots, float* __restrict__ scr)
+{
+    using namespace tc;
+    constexpr int D = 128;
+    const int j = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+    if (hdr->bad || j >= hdr->total_chunks) return;
+    const size_t u = (size_t)j * H + h;
+    const float* slot = slots + u * simt_slot_floats(D, D);
+    uint8_t* img = reinterpret_cast<uint8_t*>(scr + u * bwd_scr_floats(D, D) + bwd_wk_image_offset_floats());
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {  // task e: matrix e / 1024 (W, Kd), row (e % 1024) / 16, chunk e % 16
+        const int e = tid + 256 * m, mat = e >> 10, r = (e >> 4) & 63, ch = e & 15;
+        float f[8];
+        load8(slot + (size_t)mat * 2 * kChunk * D + (size_t)r * D + 8 * ch, f);
+        uint4 hi, lo;
+        split8(f, hi, lo);
+        const uint32_t o = (mat ? kImgKd : kImgW) + sw128_chunk_off(r, ch, 64);
+        *reinterpret_cast<uint4*>(img + o) = hi;
+        *reinterpret_cast<uint4*>(img + o + 16384) = lo;
+    }
+}
+
+constexpr int kChThreads = 192;                       // compute warps 0-3, MMA warp 4, copy warp 5
+constexpr uint32_t kChStage = 65536;                  // one unit's four images
+constexpr uint32_t kChZ = 2 * kChStage;               // Z hi, lo: 128 rows (K = key channel) x 32 (SW128, 16 KB each)
+constexpr uint32_t kChU = kChZ + 32768;               // U hi, lo: 64 rows (K = token) x 32 (8 KB each)
+constexpr uint32_t kChMisc = kChU + 16384;            // mbarriers | TMEM address | abort flag
+constexpr uint32_t kChSmem = kChMisc + 256 + 1024;
+static_assert(kChSmem <= 232448, "chain shared memory");
+
+template <bool REV>
+__global__ void __launch_bounds__(kChThreads, 1)
+bwd_chain_tc_kernel(const float* __restrict__ Z_init, float* __restrict__ Z_final, const WsHeader* __restrict__ hdr,
+                    const int* __restrict__ off, int N, int H, const float* __restrict__ slots, float* __restrict__ scr,
+                    float* __restrict__ Z_chunks, const float* __restrict__ F_chunks)
+{
+    using namespace tc;
+    constexpr int D = 128, NV = 32;
+    extern __shared__ uint8_t smem_raw[];
+    const int n = blockIdx.x, h = blockIdx.y, v0 = blockIdx.z * NV, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (hdr->bad) return;
+    uint8_t* sm = align1024(smem_raw);
+    const uint32_t sb = smem_u32(sm);
+    const uint32_t bar_full = sb + kChMisc;   // [2]
+    const uint32_t bar_empty = bar_full + 16;  // [2]: the stage's MMAs are complete
+    const uint32_t bar_p1 = bar_full + 32, bar_p2 = bar_full + 40;
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + kChMisc + 64);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(sm + kChMisc + 68);
+    const size_t slot_f = simt_slot_floats(D, D), scr_f = bwd_scr_floats(D, D);
+    const size_t zidx = ((size_t)n * H + h) * D * D;
+    const int j0 = off[n], j1 = off[n + 1], nch = j1 - j0;
+    auto chunk = [&](int it) { return REV ? j1 - 1 - it : j0 + it; };
+    auto img_of = [&](int j) {
+        return reinterpret_cast<const uint8_t*>(scr + ((size_t)j * H + h) * scr_f + bwd_wk_image_offset_floats());
+    };
+
+    if (tid == 0) {
+        mbar_init(bar_full, 1);
+        mbar_init(bar_full + 8, 1);
+        mbar_init(bar_empty, 1);
+        mbar_init(bar_empty + 8, 1);
+        mbar_init(bar_p1, 1);
+        mbar_init(bar_p2, 1);
+        mbar_fence_init();
+        *s_abort = 0;
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(s_tmem), 64);
+        tmem_relinquish();
+    }
+    // the carried matrix: thread c < 128 owns row c of this slice
+    const int c = tid;
+    float Z[NV];
+    if (warp < 4) {
+#pragma unroll
+        for (int m = 0; m < NV; m += 4) {
+            const float4 x = Z_init ? *reinterpret_cast<const float4*>(Z_init + zidx + (size_t)c * D + v0 + m)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+            Z[m] = x.x; Z[m + 1] = x.y; Z[m + 2] = x.z; Z[m + 3] = x.w;
+        }
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            uint4 hi, lo;
+            split8(Z + 8 * m, hi, lo);
+            *reinterpret_cast<uint4*>(sm + kChZ + sw128_chunk_off(c, m, 128)) = hi;
+            *reinterpret_cast<uint4*>(sm + kChZ + 16384 + sw128_chunk_off(c, m, 128)) = lo;
+        }
+    }
+    fence_proxy_async();
+    fence_before_sync();
+    __syncthreads();  // barriers initialised, TMEM address visible, Z tiles written
+    fence_after_sync();
+    if (warp == 5 && lane == 0) {
+        for (int s = 0; s < 2 && s < nch; ++s) {
+            const uint8_t* img = img_of(chunk(s));
+            mbar_arrive_expect_tx(bar_full + 8 * s, kImgBytes);
+            for (int q4 = 0; q4 < 4; ++q4) bulk_g2s(sb + s * kChStage + 16384 * q4, img + 16384 * q4, 16384, bar_full + 8 * s);
+        }
+        for (int s = 2; s < 4 && s < nch; ++s) bulk_prefetch_l2(img_of(chunk(s)), kImgBytes);
+    }
+    const uint32_t tmem = *s_tmem;  // P1 result in columns 0..31 (M = 64), P2 in 32..63 (M = 128)
+    bool ok = true;
+
+    for (int it = 0; it < nch; ++it) {
+        const int j = chunk(it), s = it & 1;
+        const uint32_t par = (uint32_t)it & 1u, spar = (uint32_t)(it >> 1) & 1u;
+        const size_t u = (size_t)j * H + h;
+        const uint32_t st = sb + s * kChStage;
+        // A of the first product (K-major) and of the second (its MN-major view): W and Kd, swapped for REV
+        const uint32_t a1 = REV ? kImgKd : kImgW, a2 = REV ? kImgW : kImgKd;
+        if (warp == 4) {
+            if (it > 0) named_sync(2, 160);  // Z tiles of this chunk written
+            if (lane == 0) {
+                ok = ok && mbar_wait_ab(bar_full + 8 * s, spar, s_abort);
+                fence_after_sync();
+                if (ok) {
+                    const uint32_t id1 = idesc_bf16(64, NV, false, true);
+                    const uint32_t as[3] = {a1, a1, a1 + 16384}, bs[3] = {kChZ, kChZ + 16384, kChZ};
+#pragma unroll
+                    for (int t = 0; t < 3; ++t)
+#pragma unroll
+                        for (int k0 = 0; k0 < D; k0 += 16)
+                            mma_bf16(tmem, desc_kmajor(st + as[t], 64, k0), desc_mnmajor(sb + bs[t], 128, k0), id1,
+                                     (t > 0 || k0 > 0) ? 1u : 0u);
+                    mma_commit(bar_p1);
+                }
+            }
+            named_sync(1, 160);  // U tiles written
+            if (lane == 0 && ok) {
+                fence_after_sync();
+                const uint32_t id2 = idesc_bf16(128, NV, true, true);
+                const uint32_t as[3] = {a2, a2, a2 + 16384}, bs[3] = {kChU, kChU + 8192, kChU};
+#pragma unroll
+                for (int t = 0; t < 3; ++t)
+#pragma unroll
+                    for (int k0 = 0; k0 < kChunk; k0 += 16)
+                        mma_bf16(tmem + 32, desc_mnmajor(st + as[t], 64, k0), desc_mnmajor(sb + bs[t], 64, k0), id2,
+                                 (t > 0 || k0 > 0) ? 1u : 0u);
+                mma_commit(bar_p2);
+                mma_commit(bar_empty + 8 * s);  // the stage's images are read
+            }
+        } else if (warp == 5) {
+            if (lane == 0 && it + 2 < nch) {
+                ok = ok && mbar_wait_ab(bar_empty + 8 * s, spar, s_abort);
+                if (ok) {
+                    const uint8_t* img = img_of(chunk(it + 2));
+                    mbar_arrive_expect_tx(bar_full + 8 * s, kImgBytes);
+                    for (int q4 = 0; q4 < 4; ++q4) bulk_g2s(st + 16384 * q4, img + 16384 * q4, 16384, bar_full + 8 * s);
+                    if (it + 4 < nch) bulk_prefetch_l2(img_of(chunk(it + 4)), kImgBytes);
+                }
+            }
+        } else {
+            // Z_c out (the chunk's start state, or the cotangent at its end) before the update
+            float* zc = Z_chunks + u * D * D + (size_t)c * D + v0;
+#pragma unroll
+            for (int m = 0; m < NV; m += 4) *reinterpret_cast<float4*>(zc + m) = make_float4(Z[m], Z[m + 1], Z[m + 2], Z[m + 3]);
+            // this thread's first-epilogue element row and columns, and its inputs, before the waits
+            const int q = warp, rr = 16 * q + (lane & 15), cb = 16 * (lane >> 4);
+            const float* slot = slots + u * slot_f;
+            float* o = scr + u * scr_f;
+            const float* uin = REV ? o + (size_t)kChunk * D : slot + (size_t)kChunk * (3 * D + kChunk);  // E : Uv
+            float* uout = REV ? o + (size_t)kChunk * D : o;                                               // dU : U
+            float ua[16];
+#pragma unroll
+            for (int m = 0; m < 16; m += 4) {
+                const float4 x = *reinterpret_cast<const float4*>(uin + (size_t)rr * D + v0 + cb + m);
+                ua[m] = x.x; ua[m + 1] = x.y; ua[m + 2] = x.z; ua[m + 3] = x.w;
+            }
+            const float gam = slot[(size_t)kChunk * (3 * D + kChunk + D) + c];
+            float fr[NV];
+            if (REV) {
+                const float* gF = F_chunks + u * D * D + (size_t)c * D + v0;
+#pragma unroll
+                for (int m = 0; m < NV; m += 4) {
+                    const float4 x = *reinterpret_cast<const float4*>(gF + m);
+                    fr[m] = x.x; fr[m + 1] = x.y; fr[m + 2] = x.z; fr[m + 3] = x.w;
+                }
+            }
+            ok = ok && mbar_wait_ab(bar_p1, par, s_abort);
+            fence_after_sync();
+            {  // U = Uv - X, or dU = E + Z (M = 64: row rr, columns cb .. cb + 15)
+                float x[16];
+                tmem_ld16_pair<16>(tmem + ((uint32_t)(32 * q) << 16), x);
+                tmem_wait_ld();
+#pragma unroll
+                for (int m = 0; m < 16; ++m) ua[m] = REV ? ua[m] + x[m] : ua[m] - x[m];
+                if (ok)
+#pragma unroll
+                    for (int m = 0; m < 16; m += 4)
+                        *reinterpret_cast<float4*>(uout + (size_t)rr * D + v0 + cb + m) =
+                            make_float4(ua[m], ua[m + 1], ua[m + 2], ua[m + 3]);
+#pragma unroll
+                for (int m = 0; m < 2; ++m) {
+                    uint4 hi, lo;
+                    split8(ua + 8 * m, hi, lo);
+                    *reinterpret_cast<uint4*>(sm + kChU + sw128_chunk_off(rr, cb / 8 + m, 64)) = hi;
+                    *reinterpret_cast<uint4*>(sm + kChU + 8192 + sw128_chunk_off(rr, cb / 8 + m, 64)) = lo;
+                }
+                fence_proxy_async();
+                fence_before_sync();
+                named_arrive(1, 160);
+            }
+            ok = ok && mbar_wait_ab(bar_p2, par, s_abort);
+            fence_after_sync();
+            {  // S <- Diag(gam) S + Kd^T U, or D <- Diag(gam) D + F - W^T dU (row c)
+                float y[NV];
+                const uint32_t tw = tmem + ((uint32_t)(32 * q) << 16) + 32;
+                tmem_ld16(tw, y);
+                tmem_ld16(tw + 16, y + 16);
+                tmem_wait_ld();
+#pragma unroll
+                for (int m = 0; m < NV; ++m) Z[m] = REV ? fmaf(gam, Z[m], fr[m] - y[m]) : fmaf(gam, Z[m], y[m]);
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    uint4 hi, lo;
+                    split8(Z + 8 * m, hi, lo);
+                    *reinterpret_cast<uint4*>(sm + kChZ + sw128_chunk_off(c, m, 128)) = hi;
+                    *reinterpret_cast<uint4*>(sm + kChZ + 16384 + sw128_chunk_off(c, m, 128)) = lo;
+                }
+                fence_proxy_async();
+                fence_before_sync();
+                if (it + 1 < nch) named_arrive(2, 160);
+            }
+        }
+    }
+    ok = __syncthreads_and(ok && !*s_abort);
+    if (REV && Z_final && warp < 4 && ok) {  // dS0
+#pragma unroll
+        for (int m = 0; m < NV; m += 4)
+            *reinterpret_cast<float4*>(Z_final + zidx + (size_t)c * D + v0 + m) = make_float4(Z[m], Z[m + 1], Z[m + 2], Z[m + 3]);
+    }
+    if (tid == 0 && !ok) {  // copies still in flight after a wait gave up: bounded waits for them
+        for (int s = 0; s < 2; ++s) (void)mbar_wait(bar_full + 8 * s, 0);
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 64);
+}
+
 inline bool bwd_state_side_tc_ok(bool bf16, int dk, int dv) { return kTcPathReady && bf16 && dk == 128 && dv == 128; }
+
+inline cudaError_t launch_bwd_chains_tc(const float* S0, const float* dS_final, float* dS0, const WsHeader* hdr,
+                                       const int* off, int N, int H, int max_chunks, const float* slots,
+                                       float* S_chunks, float* dSn_chunks, float* scr, const float* F_chunks,
+                                       bool reverse, cudaStream_t stream)
+{
+    cudaError_t e;
+    if (!reverse) {
+        if (max_chunks > 0) {
+            LaunchScope ls("bwd_wk_images", stream);
+            bwd_wk_images_kernel<<<dim3(max_chunks, H), 256, 0, stream>>>(hdr, H, slots, scr);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
+        e = cudaFuncSetAttribute(bwd_chain_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kChSmem);
+        if (e != cudaSuccess) return e;
+        LaunchScope ls("bwd_fwd_states_tc", stream);
+        bwd_chain_tc_kernel<false><<<dim3(N, H, 4), kChThreads, kChSmem, stream>>>(S0, nullptr, hdr, off, N, H, slots,
+                                                                                   scr, S_chunks, nullptr);
+        return cudaGetLastError();
+    }
+    e = cudaFuncSetAttribute(bwd_chain_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kChSmem);
+    if (e != cudaSuccess) return e;
+    LaunchScope ls("bwd_dstate_tc", stream);
+    bwd_chain_tc_kernel<true><<<dim3(N, H, 4), kChThreads, kChSmem, stream>>>(dS_final, dS0, hdr, off, N, H, slots, scr,
+                                                                              dSn_chunks, F_chunks);
+    return cudaGetLastError();
+}
 
 inline cudaError_t launch_bwd_state_side_tc(const void* dout, const WsHeader* hdr, const int* off, const int32_t* cu,
                                             int Tseq, int N, int H, int max_chunks, const float* S_chunks,

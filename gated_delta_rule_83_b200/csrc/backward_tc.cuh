@@ -1155,6 +1155,30 @@ bwd_chain_tc_kernel(const float* __restrict__ Z_init, float* __restrict__ Z_fina
     }
     const uint32_t tmem = *s_tmem;  // P1 result in columns 0..31 (M = 64), P2 in 32..63 (M = 128)
     bool ok = true;
+    // compute threads: a chunk's inputs (Uv or E at the first epilogue's row rr and columns cb .. cb + 15,
+    // gam of row c, and for REV the row c of F), loaded one chunk ahead
+    const int rr = 16 * (warp & 3) + (lane & 15), cb = 16 * (lane >> 4);
+    float ua[16], gam = 0.f, fr[NV];
+    auto load_inputs = [&](int it, float* ua_, float& gam_, float* fr_) {
+        const size_t uu = (size_t)chunk(it) * H + h;
+        const float* slot = slots + uu * slot_f;
+        const float* uin = REV ? scr + uu * scr_f + (size_t)kChunk * D : slot + (size_t)kChunk * (3 * D + kChunk);
+#pragma unroll
+        for (int m = 0; m < 16; m += 4) {
+            const float4 x = *reinterpret_cast<const float4*>(uin + (size_t)rr * D + v0 + cb + m);
+            ua_[m] = x.x; ua_[m + 1] = x.y; ua_[m + 2] = x.z; ua_[m + 3] = x.w;
+        }
+        gam_ = slot[(size_t)kChunk * (3 * D + kChunk + D) + c];
+        if (REV) {
+            const float* gF = F_chunks + uu * D * D + (size_t)c * D + v0;
+#pragma unroll
+            for (int m = 0; m < NV; m += 4) {
+                const float4 x = *reinterpret_cast<const float4*>(gF + m);
+                fr_[m] = x.x; fr_[m + 1] = x.y; fr_[m + 2] = x.z; fr_[m + 3] = x.w;
+            }
+        }
+    };
+    if (warp < 4 && nch > 0) load_inputs(0, ua, gam, fr);
 
     for (int it = 0; it < nch; ++it) {
         const int j = chunk(it), s = it & 1;
@@ -1209,28 +1233,11 @@ bwd_chain_tc_kernel(const float* __restrict__ Z_init, float* __restrict__ Z_fina
             float* zc = Z_chunks + u * D * D + (size_t)c * D + v0;
 #pragma unroll
             for (int m = 0; m < NV; m += 4) *reinterpret_cast<float4*>(zc + m) = make_float4(Z[m], Z[m + 1], Z[m + 2], Z[m + 3]);
-            // this thread's first-epilogue element row and columns, and its inputs, before the waits
-            const int q = warp, rr = 16 * q + (lane & 15), cb = 16 * (lane >> 4);
-            const float* slot = slots + u * slot_f;
+            const int q = warp;
             float* o = scr + u * scr_f;
-            const float* uin = REV ? o + (size_t)kChunk * D : slot + (size_t)kChunk * (3 * D + kChunk);  // E : Uv
-            float* uout = REV ? o + (size_t)kChunk * D : o;                                               // dU : U
-            float ua[16];
-#pragma unroll
-            for (int m = 0; m < 16; m += 4) {
-                const float4 x = *reinterpret_cast<const float4*>(uin + (size_t)rr * D + v0 + cb + m);
-                ua[m] = x.x; ua[m + 1] = x.y; ua[m + 2] = x.z; ua[m + 3] = x.w;
-            }
-            const float gam = slot[(size_t)kChunk * (3 * D + kChunk + D) + c];
-            float fr[NV];
-            if (REV) {
-                const float* gF = F_chunks + u * D * D + (size_t)c * D + v0;
-#pragma unroll
-                for (int m = 0; m < NV; m += 4) {
-                    const float4 x = *reinterpret_cast<const float4*>(gF + m);
-                    fr[m] = x.x; fr[m + 1] = x.y; fr[m + 2] = x.z; fr[m + 3] = x.w;
-                }
-            }
+            float* uout = REV ? o + (size_t)kChunk * D : o;  // dU (over E) : U
+            float ua_n[16], gam_n = 0.f, fr_n[NV];          // the next chunk's inputs, in flight meanwhile
+            if (it + 1 < nch) load_inputs(it + 1, ua_n, gam_n, fr_n);
             ok = ok && mbar_wait_ab(bar_p1, par, s_abort);
             fence_after_sync();
             {  // U = Uv - X, or dU = E + Z (M = 64: row rr, columns cb .. cb + 15)
@@ -1275,6 +1282,14 @@ bwd_chain_tc_kernel(const float* __restrict__ Z_init, float* __restrict__ Z_fina
                 fence_proxy_async();
                 fence_before_sync();
                 if (it + 1 < nch) named_arrive(2, 160);
+            }
+            if (it + 1 < nch) {
+#pragma unroll
+                for (int m = 0; m < 16; ++m) ua[m] = ua_n[m];
+                gam = gam_n;
+                if (REV)
+#pragma unroll
+                    for (int m = 0; m < NV; ++m) fr[m] = fr_n[m];
             }
         }
     }

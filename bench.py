@@ -565,8 +565,8 @@ def bench_backward(torch, kda, synth, dev, stream, world, rank, hbm, peak_kind, 
     tokens = q.shape[0] * q.shape[1]
     nbytes = BWD_BYTES_PER_TOKEN_HEAD * tokens * w.H
     ach = nbytes / (ms / steps * 1e-3) / 1e9
-    res = {"desc": f"{w.desc}; backward (kda_chunk_bwd), bf16 dO; state side, dO terms and the input side's "
-                   "products on tcgen05 (split-bf16 operands), the forward recompute and both chains fp32 on CUDA cores",
+    res = {"desc": f"{w.desc}; backward (kda_chunk_bwd), bf16 dO; every chunk product and both chains on "
+                   "tcgen05 with split-bf16 operands (fp32 accuracy); inverses, scans and element-wise work on CUDA cores",
            "tokens": tokens, "steps": steps, "ms_per_step": ms / steps,
            "value": job_throughput(world, tokens, steps, ms), "unit": "tokens/s",
            "kernels": {k_: {"launches": n, "ms": t} for k_, (n, t) in prof.items()},

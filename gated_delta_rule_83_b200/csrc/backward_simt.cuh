@@ -1101,7 +1101,10 @@ cudaError_t launch_simt_backward(const void* q, const void* k, const void* v, co
     }
     const size_t smA = simt_intra_smem(dk, dv), smS = bwd_state_side_smem(dk, dv), smU = bwd_ut_smem(),
                  smG = bwd_gate_smem();
-    cudaError_t e = cudaFuncSetAttribute(simt_intra_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smA);
+    const bool tcr = bwd_state_side_tc_ok(sizeof(TIn) == 2, dk, dv);  // the recompute's products on tcgen05
+    auto* kintra = tcr ? simt_intra_kernel<TIn, sizeof(TIn) == 2> : simt_intra_kernel<TIn, false>;
+    const size_t smAk = smA + (tcr ? 1024 : 0);
+    cudaError_t e = cudaFuncSetAttribute(kintra, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smAk);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(bwd_state_side_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smS);
     if (e == cudaSuccess)
@@ -1114,8 +1117,8 @@ cudaError_t launch_simt_backward(const void* q, const void* k, const void* v, co
     if (e != cudaSuccess) return e;
     const TIn *qq = (const TIn*)q, *kk = (const TIn*)k, *vv = (const TIn*)v;
     if (max_chunks > 0) {
-        LaunchScope ls("bwd_fwd_intra", stream);
-        simt_intra_kernel<TIn><<<dim3(max_chunks, H), kSimtThreads, smA, stream>>>(
+        LaunchScope ls(tcr ? "bwd_fwd_intra_tc" : "bwd_fwd_intra", stream);
+        kintra<<<dim3(max_chunks, H), kSimtThreads, smAk, stream>>>(
             qq, kk, vv, la, beta, hdr, off, cu, Tseq, N, H, Hk, pro & KDA_PROLOGUE_GATE_BF16, dk, dv, slots);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }

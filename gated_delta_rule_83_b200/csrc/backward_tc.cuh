@@ -1307,6 +1307,174 @@ bwd_chain_tc_kernel(const float* __restrict__ Z_init, float* __restrict__ Z_fina
     if (warp == 0) tmem_dealloc(tmem, 64);
 }
 
+// ------------------------------------------------------------------------------------------------
+// The backward's forward recompute (simt_intra_kernel<bf16, true>, dk = dv = 128): its two product
+// stages as split-bf16 tcgen05 MMAs, with the operand tiles over regions of the kernel's own shared
+// memory that are dead at that point (its fp32 layout, which starts 1024-aligned in this variant:
+// k, q, g, v, Kt at 33,024-byte strides, then A, P, T at 16,640): Qf over k (32 KB from offset 0),
+// Kf over v (from 99,328 to 132,096, the start of Kt), Kb over A and P (from 165,888; its last
+// 256 bytes reach into T, unused until the inverse), and in the second stage T, [Kt | V] and Kt's
+// lo part over k and q (64 KB from offset 0):
+//   A = strict_lower(diag(beta) Kf Kb^T), P = lower_incl(Qf Kb^T)     (factorised chunks only)
+//   [W | Uv] = T [Kt | V]                                             (one N = 256 product)
+// ------------------------------------------------------------------------------------------------
+// the MMA-completion barrier and 256 TMEM columns, at the kernel's start (read after its barriers)
+__device__ void simt_intra_tc_setup(uint32_t* s_tm, uint64_t* s_mb)
+{
+    using namespace tc;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(s_mb), 1);
+        mbar_fence_init();
+    }
+    if ((threadIdx.x >> 5) == 0) {
+        tmem_alloc(smem_u32(s_tm), 256);
+        tmem_relinquish();
+    }
+}
+
+__device__ void simt_intra_ap_tc(const float* sk, const float* sq, const float* sg, float* sv, const float* sb,
+                                 float* sA, float* sP, uint32_t* s_tm, uint64_t* s_mb)
+{
+    using namespace tc;
+    constexpr int LK = 129, L64 = kChunk + 1;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    uint8_t* tq = align1024(reinterpret_cast<uint8_t*>(const_cast<float*>(sk)));  // Qf hi | lo (over k)
+    uint8_t* tf = align1024(reinterpret_cast<uint8_t*>(sv));                       // Kf hi | lo (over v)
+    uint8_t* tb = align1024(reinterpret_cast<uint8_t*>(sA));                       // Kb hi | lo (over A, P)
+    const uint32_t mbar = smem_u32(s_mb);
+    // 64 rows x 16 chunks of 8 channels; rows are padded fp32 (stride 129), read as scalars
+    auto split_rows = [&](const float* src, uint8_t* dst) {
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const int e = tid + 256 * m, r = e >> 4, ch = e & 15;
+            float f[8];
+#pragma unroll
+            for (int x = 0; x < 8; ++x) f[x] = src[r * LK + 8 * ch + x];
+            uint4 hi, lo;
+            split8(f, hi, lo);
+            *reinterpret_cast<uint4*>(dst + sw128_chunk_off(r, ch, 64)) = hi;
+            *reinterpret_cast<uint4*>(dst + 16384 + sw128_chunk_off(r, ch, 64)) = lo;
+        }
+    };
+    split_rows(sk, tf);  // Kf (in sk) -> over v
+    split_rows(sg, tb);  // Kb (in sg) -> over A, P
+    __syncthreads();     // every read of sk is done
+    split_rows(sq, tq);  // Qf -> over k
+    fence_proxy_async();
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = *s_tm;
+    if (tid == 0) {
+        const uint32_t id = idesc_bf16(64, 64, false, false);
+        const uint32_t ta = smem_u32(tf), tqq = smem_u32(tq), tbb = smem_u32(tb);
+#pragma unroll
+        for (int t = 0; t < 3; ++t) {
+            const uint32_t ao = t == 2 ? 16384u : 0u, bo = t == 1 ? 16384u : 0u;
+#pragma unroll
+            for (int k0 = 0; k0 < 128; k0 += 16) {
+                const uint32_t acc = (t > 0 || k0 > 0) ? 1u : 0u;
+                mma_bf16(tmem, desc_kmajor(ta + ao, 64, k0), desc_kmajor(tbb + bo, 64, k0), id, acc);       // Kf Kb^T
+                mma_bf16(tmem + 64, desc_kmajor(tqq + ao, 64, k0), desc_kmajor(tbb + bo, 64, k0), id, acc);  // Qf Kb^T
+            }
+        }
+        mma_commit(mbar);
+    }
+    const bool ok = mbar_wait(mbar, 0);
+    fence_after_sync();
+    // M = 64 accumulators: row 16 q + lane % 16, columns 32 half + 16 (lane / 16) .. +15
+    const int q = warp & 3, half = warp >> 2, r = 16 * q + (lane & 15), cb = 32 * half + 16 * (lane >> 4);
+    float va[16], vp[16];
+    const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16) + 32 * half;
+    tmem_ld16_pair<16>(tl, va);
+    tmem_ld16_pair<16>(tl + 64, vp);
+    tmem_wait_ld();
+    __syncthreads();  // the Kb tiles under sA / sP are no longer read by anyone
+#pragma unroll
+    for (int x = 0; x < 16; ++x) {
+        const int i = cb + x;
+        sA[r * L64 + i] = (i < r && ok) ? sb[r] * va[x] : 0.f;
+        sP[r * L64 + i] = (i <= r && ok) ? vp[x] : 0.f;
+    }
+}
+
+__device__ void simt_intra_wuv_tc(const float* sT, const float* sKt, const __nv_bfloat16* __restrict__ v, long long t0,
+                                  int L, int H, int h, float* tiles, float* __restrict__ gW, float* __restrict__ gUv,
+                                  uint32_t* s_tm, uint64_t* s_mb, uint32_t phase)
+{
+    using namespace tc;
+    constexpr int LK = 129, L64 = kChunk + 1, D = 128;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    uint8_t* tt = align1024(reinterpret_cast<uint8_t*>(tiles));  // T hi | lo (8 KB each)
+    uint8_t* bh = tt + 16384;                                    // [Kt | V] hi: four atom columns (32 KB)
+    uint8_t* bl = bh + 32768;                                    // Kt lo: two atom columns (16 KB)
+    const uint32_t mbar = smem_u32(s_mb);
+    // T [r][i] (K-major, 64 x 64): 512 tasks of 8
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+        const int e = tid + 256 * m, r = e >> 3, ch = e & 7;
+        float f[8];
+#pragma unroll
+        for (int x = 0; x < 8; ++x) f[x] = sT[r * L64 + 8 * ch + x];
+        uint4 hi, lo;
+        split8(f, hi, lo);
+        *reinterpret_cast<uint4*>(tt + sw128_chunk_off(r, ch, 64)) = hi;
+        *reinterpret_cast<uint4*>(tt + 8192 + sw128_chunk_off(r, ch, 64)) = lo;
+    }
+    // Kt [i][c] and V [i][j] (MN-major: rows i = K): 1,024 tasks of 8 each
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const int e = tid + 256 * m, i = e >> 4, ch = e & 15;
+        float f[8];
+#pragma unroll
+        for (int x = 0; x < 8; ++x) f[x] = sKt[i * LK + 8 * ch + x];
+        uint4 hi, lo;
+        split8(f, hi, lo);
+        *reinterpret_cast<uint4*>(bh + sw128_chunk_off(i, ch, 64)) = hi;
+        *reinterpret_cast<uint4*>(bl + sw128_chunk_off(i, ch, 64)) = lo;
+        *reinterpret_cast<uint4*>(bh + sw128_chunk_off(i, 16 + ch, 64)) =
+            i < L ? *reinterpret_cast<const uint4*>(v + ((size_t)(t0 + i) * H + h) * D + 8 * ch) : make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async();
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = *s_tm;
+    if (tid == 0) {
+        const uint32_t id256 = idesc_bf16(64, 256, false, true), id128 = idesc_bf16(64, 128, false, true);
+        const uint32_t ta = smem_u32(tt), bhh = smem_u32(bh), bll = smem_u32(bl);
+#pragma unroll
+        for (int k0 = 0; k0 < kChunk; k0 += 16)
+            mma_bf16(tmem, desc_kmajor(ta, 64, k0), desc_mnmajor(bhh, 64, k0), id256, k0 > 0 ? 1u : 0u);  // T_hi B_hi
+#pragma unroll
+        for (int k0 = 0; k0 < kChunk; k0 += 16)
+            mma_bf16(tmem, desc_kmajor(ta, 64, k0), desc_mnmajor(bll, 64, k0), id128, 1u);  // T_hi Kt_lo
+#pragma unroll
+        for (int k0 = 0; k0 < kChunk; k0 += 16)
+            mma_bf16(tmem, desc_kmajor(ta + 8192, 64, k0), desc_mnmajor(bhh, 64, k0), id256, 1u);  // T_lo B_hi
+        mma_commit(mbar);
+    }
+    const bool ok = mbar_wait(mbar, phase);
+    fence_after_sync();
+    // M = 64: row 16 q + lane % 16; warps 0-3 columns 0..127 (W), warps 4-7 columns 128..255 (Uv)
+    const int q = warp & 3, half = warp >> 2, r = 16 * q + (lane & 15);
+    float* dst = (half == 0 ? gW : gUv) + (size_t)r * D;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        float x[16];
+        tmem_ld16_pair<16>(tmem + ((uint32_t)(32 * q) << 16) + 128 * half + 32 * t, x);
+        tmem_wait_ld();
+        const int c0 = 32 * t + 16 * (lane >> 4);
+        if (ok)
+#pragma unroll
+            for (int m = 0; m < 16; m += 4)
+                *reinterpret_cast<float4*>(dst + c0 + m) = make_float4(x[m], x[m + 1], x[m + 2], x[m + 3]);
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 256);
+}
+
 inline bool bwd_state_side_tc_ok(bool bf16, int dk, int dv) { return kTcPathReady && bf16 && dk == 128 && dv == 128; }
 
 inline cudaError_t launch_bwd_chains_tc(const float* S0, const float* dS_final, float* dS0, const WsHeader* hdr,

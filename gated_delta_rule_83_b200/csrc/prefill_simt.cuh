@@ -179,7 +179,16 @@ __device__ __forceinline__ void simt_unit_lower_inverse(float* __restrict__ A, f
     }
 }
 
-template <typename TIn>
+// the product stages on the tensor cores, for the backward's recompute with bf16 inputs and
+// dk = dv = 128 (defined with the backward's tensor-core kernels)
+__device__ void simt_intra_tc_setup(uint32_t* s_tm, uint64_t* s_mb);
+__device__ void simt_intra_ap_tc(const float* sk, const float* sq, const float* sg, float* sv, const float* sb,
+                                 float* sA, float* sP, uint32_t* s_tm, uint64_t* s_mb);
+__device__ void simt_intra_wuv_tc(const float* sT, const float* sKt, const __nv_bfloat16* __restrict__ v, long long t0,
+                                  int L, int H, int h, float* tiles, float* __restrict__ gW, float* __restrict__ gUv,
+                                  uint32_t* s_tm, uint64_t* s_mb, uint32_t phase);
+
+template <typename TIn, bool TC = false>
 __global__ void __launch_bounds__(kSimtThreads)
 simt_intra_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
                   const void* __restrict__ log_alpha, const float* __restrict__ beta, const WsHeader* __restrict__ hdr,
@@ -196,7 +205,10 @@ simt_intra_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TI
     // row strides padded by one float, so column walks of a warp hit distinct banks
     const int LK = dk + 1, LV = dv + 1;
     constexpr int L64 = kChunk + 1;
-    float* sk = smem;                       // [64][dk+1]  k, later k e^{g - ref}
+    // (TC: the layout starts on a 1024-byte boundary, so that the operand tiles placed over its dead
+    // regions are aligned and stay inside them; the launch adds 1024 bytes)
+    float* sk = TC ? reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(smem) + 1023) & ~uintptr_t(1023))
+                   : smem;                  // [64][dk+1]  k, later k e^{g - ref}
     float* sq = sk + kChunk * LK;           // [64][dk+1]  q, later q e^{g - ref}
     float* sg = sq + kChunk * LK;           // [64][dk+1]  g, later k e^{ref - g}
     float* sv = sg + kChunk * LK;           // [64][dv+1]
@@ -207,9 +219,12 @@ simt_intra_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TI
     float* sb = sT + kChunk * L64;          // [64]
     float* sref = sb + kChunk;              // [dk]
     __shared__ int s_wide;
+    __shared__ uint32_t s_tm;  // TC: TMEM base address and the MMA-completion barrier
+    __shared__ uint64_t s_mb;
     const int tr = tid >> 4, tc = tid & 15;
 
     if (tid == 0) s_wide = 0;
+    if constexpr (TC) simt_intra_tc_setup(&s_tm, &s_mb);
     // 8 consecutive channels per thread and step (16- or 32-byte loads); rows past the end read as 0
     for (int e = tid; e < kChunk * dk / 8; e += kSimtThreads) {
         const int r = e / (dk / 8), c = 8 * (e % (dk / 8));
@@ -311,6 +326,9 @@ simt_intra_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TI
             sg[x0] = kv * fast_exp(-x);
         }
         __syncthreads();
+        if constexpr (TC) {
+            simt_intra_ap_tc(sk, sq, sg, sv, sb, sA, sP, &s_tm, &s_mb);
+        } else {
         // A = Kf Kb^T and P = Qf Kb^T, register-tiled (4 x 4 per thread, shared Kb reads)
         float a_[4][4] = {}, p_[4][4] = {};
 #pragma unroll 2
@@ -338,6 +356,7 @@ simt_intra_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TI
                 sA[r * L64 + i] = (i < r) ? sb[r] * a_[a][b] : 0.f;
                 sP[r * L64 + i] = (i <= r) ? p_[a][b] : 0.f;
             }
+        }
     } else {
         // some channel decays by more than e^-160 inside the chunk: exact per-element factors
         for (int e = tid; e < kChunk * kChunk; e += kSimtThreads) {
@@ -366,10 +385,15 @@ simt_intra_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TI
     __syncthreads();
 
     // W = T Kt, Uv = T V (T is lower triangular with zeros above the diagonal)
-    if (dk == 128) simt_apply_t<128>(sT, sKt, gW, tr, tc);
-    else simt_apply_t<64>(sT, sKt, gW, tr, tc);
-    if (dv == 128) simt_apply_t<128>(sT, sv, gUv, tr, tc);
-    else simt_apply_t<64>(sT, sv, gUv, tr, tc);
+    if constexpr (TC) {  // the barrier's phase 0 was stage 1's (factorised chunks only)
+        simt_intra_wuv_tc(sT, sKt, reinterpret_cast<const __nv_bfloat16*>(v), t0, L, H, h, sk, gW, gUv, &s_tm, &s_mb,
+                          wide ? 0u : 1u);
+    } else {
+        if (dk == 128) simt_apply_t<128>(sT, sKt, gW, tr, tc);
+        else simt_apply_t<64>(sT, sKt, gW, tr, tc);
+        if (dv == 128) simt_apply_t<128>(sT, sv, gUv, tr, tc);
+        else simt_apply_t<64>(sT, sv, gUv, tr, tc);
+    }
 }
 
 // 16-byte asynchronous global -> shared copies in commit groups (phase B's operand prefetch)

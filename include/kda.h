@@ -233,10 +233,9 @@ kda_status kda_host_release(void);
  * its section "硬件效率的深度优化" lists: the forward is recomputed chunk-parallel keeping only each
  * chunk's start state, the state cotangent runs backwards over the chunks, and the input
  * derivatives are again chunk-parallel.  Arithmetic is fp32 on CUDA cores; for bf16 inputs with
- * dk = dv = 128 the state-side products, the output-cotangent terms and the gated products of the
- * input side run on the tensor cores with
- * each fp32 operand split into two bf16 parts (hi*hi + hi*lo + lo*hi, about 16 significant bits),
- * which keeps the same fp32-level accuracy.
+ * dk = dv = 128 every chunk product and both chains run on the tensor cores with each fp32 operand
+ * split into two bf16 parts (hi*hi + hi*lo + lo*hi, about 16 significant bits), which keeps the
+ * same fp32-level accuracy.
  *
  *   q, k, v, log_alpha, beta, S0, cu_seqlens, num_seqs, B, T, H, dk, dv, dt:  exactly as given to
  *                kda_chunk_fwd (same layout, same meaning).

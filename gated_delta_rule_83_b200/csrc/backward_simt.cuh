@@ -517,6 +517,9 @@ __device__ __forceinline__ void bwd_load_scr_tile(const float* __restrict__ x, i
 // factorised tiles only) and dT (lower, inclusive) into sAt and sM, with the exact products of the
 // wide tiles added into accA at the thread's (tr, tc) elements; scratch = the kernel's shared memory
 // below sb
+__device__ void bwd_ut_y_dm_tc(const float* sN, float* sM, float* tiles);
+__device__ void bwd_ut_dv_tc(const float* sN, const float* sb, const float* __restrict__ gdU, __nv_bfloat16* dv_out,
+                             long long t0, int L, int H, int h, float* tiles);
 __device__ void bwd_ut_step4a_tc(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
                                  const void* __restrict__ log_alpha, bool la16, long long t0, int L, int H, int Hk,
                                  int h, const float* __restrict__ gdW, const float* __restrict__ gdU, float* smem,
@@ -643,27 +646,31 @@ bwd_ut_kernel(const TIn* __restrict__ k, const TIn* __restrict__ v, const void* 
         sM[r * L64 + i] *= sb[i];
     }
     __syncthreads();
-    {  // Y = dN N^T
-        float acc[4][4] = {};
-        mm_acc<4, 4>(acc, sM, L64, 1, sN, 1, L64, kChunk, tr, tc);
+    if constexpr (TC) {
+        bwd_ut_y_dm_tc(sN, sM, tk);
+    } else {
+        {  // Y = dN N^T
+            float acc[4][4] = {};
+            mm_acc<4, 4>(acc, sM, L64, 1, sN, 1, L64, kChunk, tr, tc);
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
+            for (int a = 0; a < 4; ++a)
 #pragma unroll
-            for (int b = 0; b < 4; ++b) sY[(tr + 16 * a) * L64 + tc + 16 * b] = acc[a][b];
+                for (int b = 0; b < 4; ++b) sY[(tr + 16 * a) * L64 + tc + 16 * b] = acc[a][b];
+        }
+        __syncthreads();
+        {  // dM = -N^T Y, strictly lower (dN is no longer needed: overwritten in place)
+            float acc[4][4] = {};
+            mm_acc<4, 4>(acc, sN, 1, L64, sY, L64, 1, kChunk, tr, tc);
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    const int r = tr + 16 * a, i = tc + 16 * b;
+                    sM[r * L64 + i] = (i < r) ? -acc[a][b] : 0.f;
+                }
+        }
+        __syncthreads();
     }
-    __syncthreads();
-    {  // dM = -N^T Y, strictly lower (dN is no longer needed: overwritten in place)
-        float acc[4][4] = {};
-        mm_acc<4, 4>(acc, sN, 1, L64, sY, L64, 1, kChunk, tr, tc);
-#pragma unroll
-        for (int a = 0; a < 4; ++a)
-#pragma unroll
-            for (int b = 0; b < 4; ++b) {
-                const int r = tr + 16 * a, i = tc + 16 * b;
-                sM[r * L64 + i] = (i < r) ? -acc[a][b] : 0.f;
-            }
-    }
-    __syncthreads();
     if (tid < kChunk) {  // dbeta_r += sum_i dM[r][i] At[r][i];  dAt = Diag(beta) dM
         const int r = tid;
         float x = 0.f;
@@ -677,19 +684,23 @@ bwd_ut_kernel(const TIn* __restrict__ k, const TIn* __restrict__ v, const void* 
     for (int r = tid; r < L; r += kSimtThreads) dbeta[(size_t)(t0 + r) * H + h] = sdb[r];
 
     // ---- step 4d: dV = T^T dU = Diag(beta) N^T dU
-    for (int c0 = 0; c0 < dv; c0 += kBwdCT) {
-        __syncthreads();
-        bwd_load_scr_tile(gdU, dv, c0, tD);
-        __syncthreads();
-        float acc[4][2] = {};
-        mm_acc<4, 2>(acc, sN, 1, L64, tD, LT, 1, kChunk, tr, tc);
+    if constexpr (TC) {
+        bwd_ut_dv_tc(sN, sb, gdU, reinterpret_cast<__nv_bfloat16*>(dv_out), t0, L, H, h, tk);
+    } else {
+        for (int c0 = 0; c0 < dv; c0 += kBwdCT) {
+            __syncthreads();
+            bwd_load_scr_tile(gdU, dv, c0, tD);
+            __syncthreads();
+            float acc[4][2] = {};
+            mm_acc<4, 2>(acc, sN, 1, L64, tD, LT, 1, kChunk, tr, tc);
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
+            for (int a = 0; a < 4; ++a)
 #pragma unroll
-            for (int b = 0; b < 2; ++b) {
-                const int i = tr + 16 * a, cc = tc + 16 * b;
-                if (i < L) dv_out[((size_t)(t0 + i) * H + h) * dv + c0 + cc] = from_f32<TIn>(sb[i] * acc[a][b]);
-            }
+                for (int b = 0; b < 2; ++b) {
+                    const int i = tr + 16 * a, cc = tc + 16 * b;
+                    if (i < L) dv_out[((size_t)(t0 + i) * H + h) * dv + c0 + cc] = from_f32<TIn>(sb[i] * acc[a][b]);
+                }
+        }
     }
     // N and dAt out for the gate half (U and dU are no longer read)
     __syncthreads();

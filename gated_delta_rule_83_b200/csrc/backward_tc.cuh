@@ -825,10 +825,7 @@ __device__ void bwd_ut_step4a_tc(const __nv_bfloat16* __restrict__ k, const __nv
         mbar_init(mbar, 1);
         mbar_fence_init();
     }
-    if (warp == 0) {
-        tmem_alloc(smem_u32(&s_tm), 128);
-        tmem_relinquish();
-    }
+    if (warp == 0) tmem_alloc(smem_u32(&s_tm), 128);  // no relinquish: the UT stages allocate again
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
@@ -1305,6 +1302,181 @@ bwd_chain_tc_kernel(const float* __restrict__ Z_init, float* __restrict__ Z_fina
     fence_before_sync();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, 64);
+}
+
+// ------------------------------------------------------------------------------------------------
+// bwd_ut's UT step and dV on the tensor cores (bwd_ut_kernel<bf16, true>), split-bf16 as above, with
+// the operand tiles over the kernel's per-tile scratch (free after the inverse; 48 KB at most):
+//   Y = dN N^T  ->  dM = strict_lower(-N^T Y)  (into sM)          dV = Diag(beta) N^T dU
+// N and dN stay fp32 in sN / sM for the beta sums; N's tile serves K-major for Y and MN-major (its
+// transpose) for dM and dV.
+// ------------------------------------------------------------------------------------------------
+// 64 x 64 fp32 rows (stride 65) -> bf16 hi / lo SW128 tiles (one atom column)
+__device__ __forceinline__ void split_64x64(const float* src, uint8_t* hi, uint8_t* lo)
+{
+    constexpr int L64 = kChunk + 1;
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+        const int e = threadIdx.x + 256 * m, r = e >> 3, ch = e & 7;
+        float f[8];
+#pragma unroll
+        for (int x = 0; x < 8; ++x) f[x] = src[r * L64 + 8 * ch + x];
+        uint4 h4, l4;
+        split8(f, h4, l4);
+        *reinterpret_cast<uint4*>(hi + tc::sw128_chunk_off(r, ch, 64)) = h4;
+        *reinterpret_cast<uint4*>(lo + tc::sw128_chunk_off(r, ch, 64)) = l4;
+    }
+}
+
+__device__ void bwd_ut_y_dm_tc(const float* sN, float* sM, float* tiles)
+{
+    using namespace tc;
+    constexpr int L64 = kChunk + 1;
+    __shared__ uint64_t s_mb;
+    __shared__ uint32_t s_tm;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    uint8_t* ab = align1024(reinterpret_cast<uint8_t*>(tiles));  // dN | N | Y, hi and lo (8 KB each)
+    const uint32_t tb = smem_u32(ab), mbar = smem_u32(&s_mb);
+    __syncthreads();  // dN in sM, N in sM's neighbour, and the inverse's scratch is free
+    if (tid == 0) {
+        mbar_init(mbar, 1);
+        mbar_fence_init();
+    }
+    if (warp == 0) tmem_alloc(smem_u32(&s_tm), 128);  // no relinquish: the dV stage allocates again
+    split_64x64(sM, ab, ab + 8192);           // dN
+    split_64x64(sN, ab + 16384, ab + 24576);  // N
+    fence_proxy_async();
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = s_tm;
+    const int q = warp & 3, half = warp >> 2, r = 16 * q + (lane & 15), cb = 32 * half + 16 * (lane >> 4);
+    const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16) + 32 * half;
+    if (tid == 0) {  // Y[r][i'] = sum_i dN[r][i] N[i'][i]
+        const uint32_t id = idesc_bf16(64, 64, false, false);
+        const uint32_t as[3] = {0u, 0u, 8192u}, bs[3] = {16384u, 24576u, 16384u};
+#pragma unroll
+        for (int t = 0; t < 3; ++t)
+#pragma unroll
+            for (int k0 = 0; k0 < kChunk; k0 += 16)
+                mma_bf16(tmem, desc_kmajor(tb + as[t], 64, k0), desc_kmajor(tb + bs[t], 64, k0), id,
+                         (t > 0 || k0 > 0) ? 1u : 0u);
+        mma_commit(mbar);
+    }
+    bool ok = mbar_wait(mbar, 0);
+    fence_after_sync();
+    {  // Y -> hi / lo tiles (row r, columns cb .. cb + 15): the B operand of dM, read MN-major
+        float y[16];
+        tmem_ld16_pair<16>(tl, y);
+        tmem_wait_ld();
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+            uint4 h4, l4;
+            split8(y + 8 * m, h4, l4);
+            *reinterpret_cast<uint4*>(ab + 32768 + sw128_chunk_off(r, cb / 8 + m, 64)) = h4;
+            *reinterpret_cast<uint4*>(ab + 40960 + sw128_chunk_off(r, cb / 8 + m, 64)) = l4;
+        }
+    }
+    fence_proxy_async();
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    if (tid == 0) {  // (N^T Y)[r][i] = sum_a N[a][r] Y[a][i]
+        const uint32_t id = idesc_bf16(64, 64, true, true);
+        const uint32_t as[3] = {16384u, 16384u, 24576u}, bs[3] = {32768u, 40960u, 32768u};
+#pragma unroll
+        for (int t = 0; t < 3; ++t)
+#pragma unroll
+            for (int k0 = 0; k0 < kChunk; k0 += 16)
+                mma_bf16(tmem + 64, desc_mnmajor(tb + as[t], 64, k0), desc_mnmajor(tb + bs[t], 64, k0), id,
+                         (t > 0 || k0 > 0) ? 1u : 0u);
+        mma_commit(mbar);
+    }
+    ok = mbar_wait(mbar, 1) && ok;
+    fence_after_sync();
+    {
+        float d[16];
+        tmem_ld16_pair<16>(tl + 64, d);
+        tmem_wait_ld();
+#pragma unroll
+        for (int x = 0; x < 16; ++x) {
+            const int i = cb + x;
+            sM[r * L64 + i] = (i < r && ok) ? -d[x] : 0.f;
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 128);
+}
+
+__device__ void bwd_ut_dv_tc(const float* sN, const float* sb, const float* __restrict__ gdU, __nv_bfloat16* dv_out,
+                             long long t0, int L, int H, int h, float* tiles)
+{
+    using namespace tc;
+    constexpr int D = 128;
+    __shared__ uint64_t s_mb;
+    __shared__ uint32_t s_tm;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    uint8_t* ab = align1024(reinterpret_cast<uint8_t*>(tiles));  // N hi | lo (8 KB each), dU hi | lo (16 KB each)
+    const uint32_t tb = smem_u32(ab), mbar = smem_u32(&s_mb);
+    __syncthreads();
+    if (tid == 0) {
+        mbar_init(mbar, 1);
+        mbar_fence_init();
+    }
+    if (warp == 0) {  // the CTA's last allocation: the permit can go
+        tmem_alloc(smem_u32(&s_tm), 128);
+        tmem_relinquish();
+    }
+    split_64x64(sN, ab, ab + 8192);
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {  // dU [a][j] (MN-major B: rows a = K)
+        const int e = tid + 256 * m, a = e >> 4, ch = e & 15;
+        float f[8];
+        load8(gdU + (size_t)a * D + 8 * ch, f);
+        uint4 h4, l4;
+        split8(f, h4, l4);
+        *reinterpret_cast<uint4*>(ab + 16384 + sw128_chunk_off(a, ch, 64)) = h4;
+        *reinterpret_cast<uint4*>(ab + 32768 + sw128_chunk_off(a, ch, 64)) = l4;
+    }
+    fence_proxy_async();
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = s_tm;
+    if (tid == 0) {  // (N^T dU)[i][j] = sum_a N[a][i] dU[a][j]
+        const uint32_t id = idesc_bf16(64, 128, true, true);
+        const uint32_t as[3] = {0u, 0u, 8192u}, bs[3] = {16384u, 32768u, 16384u};
+#pragma unroll
+        for (int t = 0; t < 3; ++t)
+#pragma unroll
+            for (int k0 = 0; k0 < kChunk; k0 += 16)
+                mma_bf16(tmem, desc_mnmajor(tb + as[t], 64, k0), desc_mnmajor(tb + bs[t], 64, k0), id,
+                         (t > 0 || k0 > 0) ? 1u : 0u);
+        mma_commit(mbar);
+    }
+    const bool ok = mbar_wait(mbar, 0);
+    fence_after_sync();
+    // M = 64: row i = 16 q + lane % 16; warps 0-3 columns 0..63, warps 4-7 64..127
+    const int q = warp & 3, half = warp >> 2, i = 16 * q + (lane & 15);
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        float x[16];
+        tmem_ld16_pair<16>(tmem + ((uint32_t)(32 * q) << 16) + 64 * half + 32 * t, x);
+        tmem_wait_ld();
+        if (i < L && ok) {
+            const int c0 = 64 * half + 32 * t + 16 * (lane >> 4);
+            const float bi = sb[i];
+#pragma unroll
+            for (int m = 0; m < 16; ++m) x[m] *= bi;
+            uint4* dst = reinterpret_cast<uint4*>(dv_out + ((size_t)(t0 + i) * H + h) * D + c0);
+            dst[0] = pack8(x);
+            dst[1] = pack8(x + 8);
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 128);
 }
 
 // ------------------------------------------------------------------------------------------------
